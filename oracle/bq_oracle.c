@@ -1,0 +1,377 @@
+/*
+ * bq_oracle.c -- plain CPU oracle for block-scaled (MX) activation quantization
+ * and the block-scaled GEMM that consumes it.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product library links, calls or
+ * includes this file; only the tests, the package's smoke check and the
+ * benchmark's CPU-baseline leg use it.  It shares no code, header, table or
+ * constant generator with the CUDA path.
+ *
+ * Written to be read against the pages, not to be fast:
+ *   - every operand is decoded exactly and products are summed in fp64;
+ *   - the activation quantizer follows the step order of the
+ *     "formats.py" page (dsv41-sampled-drafting, code/offload/dspark/native):
+ *     module docstring "act_qdq reproduces kernel.act_quant ..." and the
+ *     functions act_scale / act_quant / act_qdq / _log2_ceil_pow2;
+ *   - the number formats follow the same page's module docstring
+ *     ("Formats" paragraph) and its constants FP4_TABLE, FP8_MAX, BLOCK,
+ *     E8M0_NAN, E4M3_NAN.
+ *
+ * Floating point: compile with -ffp-contract=off and without fast-math so that
+ * every float expression below is one IEEE binary32 operation, as the page's
+ * fp32 tensor arithmetic is.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_NAN_SCALE (-1) /* E8M0 byte 255 */
+#define ORACLE_ERR_NAN_CODE (-2)  /* E4M3 byte 0x7F or 0xFF */
+#define ORACLE_ERR_SHAPE (-3)     /* K not a multiple of 32, bad kind */
+#define ORACLE_ERR_NONFINITE (-4) /* NaN/Inf activation (outside the contract) */
+
+#define BLOCK 32 /* one scale per 32 consecutive elements ("BLOCK = 32") */
+
+/* ------------------------------------------------------------------ */
+/* Number formats ("Formats" paragraph of the formats.py page).        */
+/* ------------------------------------------------------------------ */
+
+/* E8M0: one byte b means 2^(b-127); b = 255 is NaN and is refused. */
+int oracle_decode_e8m0(uint8_t b, double *out) {
+  if (b == 255) return ORACLE_ERR_NAN_SCALE;
+  *out = ldexp(1.0, (int)b - 127);
+  return ORACLE_OK;
+}
+
+/* E2M1 (FP4) code -> value, from the format's fields: bit 3 sign, bits 2..1
+ * exponent (bias 1), bit 0 mantissa; exponent field 0 is the subnormal
+ * 0.m x 2^0.  Code 8 is -0.0.  (The page lists the result as FP4_TABLE; the
+ * tests compare this against that printed table.) */
+double oracle_decode_fp4(uint8_t code) {
+  int sign = (code >> 3) & 1;
+  int e = (code >> 1) & 3;
+  int m = code & 1;
+  double mag = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+  return sign ? -mag : mag;
+}
+
+/* E4M3 (e4m3fn): bias 7, no infinities, 0x7F/0xFF are NaN (refused).
+ * Normal: (-1)^s 2^(E-7) (1 + m/8); subnormal (E = 0): (-1)^s 2^-6 (m/8). */
+int oracle_decode_e4m3(uint8_t b, double *out) {
+  if ((b & 0x7F) == 0x7F) return ORACLE_ERR_NAN_CODE;
+  int s = b >> 7;
+  int E = (b >> 3) & 0xF;
+  int m = b & 7;
+  double mag = (E == 0) ? ldexp(m / 8.0, -6) : ldexp(1.0 + m / 8.0, E - 7);
+  *out = s ? -mag : mag;
+  return ORACLE_OK;
+}
+
+/* The 127 non-negative finite E4M3 magnitudes, indexed by code 0x00..0x7E;
+ * they increase strictly with the code. */
+static double e4m3_mag[127];
+static int e4m3_mag_ready = 0;
+static void e4m3_table_init(void) {
+  if (e4m3_mag_ready) return;
+  for (int c = 0; c < 127; ++c) oracle_decode_e4m3((uint8_t)c, &e4m3_mag[c]);
+  e4m3_mag_ready = 1;
+}
+
+/* Round a binary32 value to E4M3 with round-to-nearest, ties to even,
+ * saturating at +-448 (the page clamps to [-448, 448] before converting, so
+ * saturation is never what decides a result there).  The sign is kept:
+ * negative values that round to zero give 0x80 (-0).
+ * Method: find the two neighbouring representable magnitudes in the sorted
+ * table and pick the nearer; on a tie pick the even code (the code's low bit
+ * is the mantissa's low bit). */
+uint8_t oracle_encode_e4m3(float v) {
+  e4m3_table_init();
+  uint8_t sign = signbit(v) ? 0x80 : 0x00;
+  double a = fabs((double)v);
+  uint8_t code;
+  if (a >= e4m3_mag[126]) {
+    code = 126; /* 448 */
+  } else {
+    int lo = 0, hi = 126; /* invariant: mag[lo] <= a < mag[hi] */
+    while (hi - lo > 1) {
+      int mid = (lo + hi) / 2;
+      if (e4m3_mag[mid] <= a) lo = mid; else hi = mid;
+    }
+    double dlo = a - e4m3_mag[lo], dhi = e4m3_mag[hi] - a;
+    if (dlo < dhi) code = (uint8_t)lo;
+    else if (dhi < dlo) code = (uint8_t)hi;
+    else code = (uint8_t)((lo % 2 == 0) ? lo : hi);
+  }
+  return (uint8_t)(sign | code);
+}
+
+/* Element-wise oracle_encode_e4m3 over n values. */
+void oracle_encode_e4m3_n(const float *v, int64_t n, uint8_t *out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = oracle_encode_e4m3(v[i]);
+}
+
+static float bf16_to_f32(uint16_t h) {
+  uint32_t u = (uint32_t)h << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+/* binary32 -> bfloat16, round to nearest even (finite inputs; an overflow
+ * gives +-Inf as IEEE rounding does). */
+uint16_t oracle_f32_to_bf16(float f) {
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  if (isnan(f)) return (uint16_t)((u >> 16) | 0x40);
+  uint32_t lsb = (u >> 16) & 1;
+  u += 0x7FFF + lsb;
+  return (uint16_t)(u >> 16);
+}
+
+/* ------------------------------------------------------------------ */
+/* Activation quantization (formats.py page: act_scale, act_quant,      */
+/* act_qdq, _log2_ceil_pow2; docstring "act_qdq reproduces ...").       */
+/* ------------------------------------------------------------------ */
+
+/* The per-group steps, for one group of 32 binary32 values:
+ *   amax = max(max_i |x_i|, 1e-4)                       (fp32)
+ *   t    = fp32(amax * fp32(1/448))
+ *   e    = ceil(log2 t), read from t's exponent bits: the unbiased exponent,
+ *          plus one when any mantissa bit is set (t is a positive normal)
+ *   s    = 2^e;   scale byte = e + 127
+ *   q_i  = E4M3_RNE(clamp(x_i / s, -448, 448))
+ * Returns the scale byte, or -1 if the group holds a NaN or Inf. */
+static int act_quant_group(const float *x, uint8_t *q) {
+  float amax = 0.0f;
+  for (int i = 0; i < BLOCK; ++i) {
+    if (!isfinite(x[i])) return -1;
+    float ax = fabsf(x[i]);
+    if (ax > amax) amax = ax;
+  }
+  const float floor_ = 1e-4f;
+  if (amax < floor_) amax = floor_;
+  const float inv448 = (float)(1.0 / 448.0);
+  float t = amax * inv448;
+  uint32_t bits;
+  memcpy(&bits, &t, 4);
+  int e = (int)((bits >> 23) & 0xFF) - 127 + ((bits & 0x7FFFFF) != 0 ? 1 : 0);
+  float s = ldexpf(1.0f, e);
+  for (int i = 0; i < BLOCK; ++i) {
+    float y = x[i] / s;
+    if (y > 448.0f) y = 448.0f;
+    if (y < -448.0f) y = -448.0f;
+    q[i] = oracle_encode_e4m3(y);
+  }
+  return e + 127;
+}
+
+/* x: bf16 bit patterns, M rows of K elements, row stride ldx elements.
+ * q: [M, K] E4M3 codes (row stride K).  sf: [M, K/32] E8M0 bytes, row-major.
+ * Returns ORACLE_OK, ORACLE_ERR_SHAPE (K % 32 != 0) or ORACLE_ERR_NONFINITE. */
+int oracle_act_quant(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                     uint8_t *q, uint8_t *sf) {
+  if (K <= 0 || K % BLOCK) return ORACLE_ERR_SHAPE;
+  const int64_t G = K / BLOCK;
+  float buf[BLOCK];
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t g = 0; g < G; ++g) {
+      for (int i = 0; i < BLOCK; ++i) buf[i] = bf16_to_f32(x[m * ldx + g * BLOCK + i]);
+      int b = act_quant_group(buf, q + m * K + g * BLOCK);
+      if (b < 0) return ORACLE_ERR_NONFINITE;
+      sf[m * G + g] = (uint8_t)b;
+    }
+  }
+  return ORACLE_OK;
+}
+
+/* Same steps on binary32 input (used to pin the encoder and the scale rule on
+ * values that are not bf16). */
+int oracle_act_quant_f32(const float *x, int64_t M, int64_t K, uint8_t *q, uint8_t *sf) {
+  if (K <= 0 || K % BLOCK) return ORACLE_ERR_SHAPE;
+  const int64_t G = K / BLOCK;
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t g = 0; g < G; ++g) {
+      int b = act_quant_group(x + m * K + g * BLOCK, q + m * K + g * BLOCK);
+      if (b < 0) return ORACLE_ERR_NONFINITE;
+      sf[m * G + g] = (uint8_t)b;
+    }
+  return ORACLE_OK;
+}
+
+/* The dequantized activation: value = fp32(q) * s in binary32, then stored
+ * as bf16 (round to nearest even).  y: [M, K] bf16 bit patterns. */
+int oracle_act_qdq(const uint8_t *q, const uint8_t *sf, int64_t M, int64_t K, uint16_t *y) {
+  if (K <= 0 || K % BLOCK) return ORACLE_ERR_SHAPE;
+  const int64_t G = K / BLOCK;
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t k = 0; k < K; ++k) {
+      double qv, sv;
+      if (oracle_decode_e4m3(q[m * K + k], &qv)) return ORACLE_ERR_NAN_CODE;
+      if (oracle_decode_e8m0(sf[m * G + k / BLOCK], &sv)) return ORACLE_ERR_NAN_SCALE;
+      float v = (float)qv * (float)sv;
+      y[m * K + k] = oracle_f32_to_bf16(v);
+    }
+  return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Exact operand decode + fp64 GEMM with the fused epilogue.            */
+/* ------------------------------------------------------------------ */
+
+/* Weight kinds. */
+#define ORACLE_B_FP4 0     /* E2M1 packed [N, K/2], low nibble = even k; scales [N, K/32] */
+#define ORACLE_B_FP8BLK 1  /* E4M3 [N, K]; scales [ceil(N/32), ceil(K/32)], one per 32x32 block */
+#define ORACLE_B_FP8ROW 2  /* E4M3 [N, K]; scales [N, K/32] (MXFP8 along K) */
+
+#define ORACLE_ACT_NONE 0
+#define ORACLE_ACT_GELU 1
+
+typedef struct {
+  const uint8_t *aq, *asf;
+  const uint8_t *b, *bsf;
+  int bkind;
+  int64_t M, N, K;
+  const uint16_t *bias, *residual;
+  int64_t ld_res;
+  double alpha;
+  int act;
+  /* full output */
+  double *ref, *sumabs;
+  /* sampled output (when ms != NULL) */
+  const int64_t *ms, *ns;
+  int64_t count;
+  int64_t begin, end;
+  int status;
+} gemm_job;
+
+/* Decoded A value a[m][k] = e4m3(code) * 2^(b - 127) (exact in double). */
+static int dec_a(const gemm_job *J, int64_t m, int64_t k, double *v) {
+  double c, s;
+  if (oracle_decode_e4m3(J->aq[m * J->K + k], &c)) return ORACLE_ERR_NAN_CODE;
+  if (oracle_decode_e8m0(J->asf[m * (J->K / BLOCK) + k / BLOCK], &s)) return ORACLE_ERR_NAN_SCALE;
+  *v = c * s;
+  return ORACLE_OK;
+}
+
+/* Decoded B value b[n][k] for the three weight formats (formats.py page:
+ * decode_fp4, decode_fp8_block, fp4_codes). */
+static int dec_b(const gemm_job *J, int64_t n, int64_t k, double *v) {
+  const int64_t K = J->K;
+  double c, s;
+  uint8_t sb;
+  if (J->bkind == ORACLE_B_FP4) {
+    uint8_t byte = J->b[n * (K / 2) + k / 2];
+    uint8_t code = (k % 2 == 0) ? (byte & 0x0F) : (byte >> 4);
+    c = oracle_decode_fp4(code);
+    sb = J->bsf[n * (K / BLOCK) + k / BLOCK];
+  } else {
+    if (oracle_decode_e4m3(J->b[n * K + k], &c)) return ORACLE_ERR_NAN_CODE;
+    if (J->bkind == ORACLE_B_FP8BLK) {
+      int64_t kb = (K + BLOCK - 1) / BLOCK;
+      sb = J->bsf[(n / BLOCK) * kb + k / BLOCK];
+    } else {
+      sb = J->bsf[n * (K / BLOCK) + k / BLOCK];
+    }
+  }
+  if (oracle_decode_e8m0(sb, &s)) return ORACLE_ERR_NAN_SCALE;
+  *v = c * s;
+  return ORACLE_OK;
+}
+
+static double bf16d(const uint16_t *p, int64_t i) { return (double)bf16_to_f32(p[i]); }
+
+/* One output element: acc = sum_k a[m][k] b[n][k] in fp64, sumabs =
+ * sum_k |a b|; then ref = act(alpha * acc + bias[n]) + residual[m][n] with
+ * act = erf-GELU 0.5 t (1 + erf(t / sqrt 2)) or identity. */
+static int one_element(const gemm_job *J, const double *arow, int64_t m, int64_t n,
+                       double *ref, double *sabs) {
+  double acc = 0.0, sa = 0.0;
+  for (int64_t k = 0; k < J->K; ++k) {
+    double bv;
+    int st = dec_b(J, n, k, &bv);
+    if (st) return st;
+    double p = arow[k] * bv;
+    acc += p;
+    sa += fabs(p);
+  }
+  double t = J->alpha * acc;
+  if (J->bias) t += bf16d(J->bias, n);
+  if (J->act == ORACLE_ACT_GELU) t = 0.5 * t * (1.0 + erf(t / sqrt(2.0)));
+  if (J->residual) t += bf16d(J->residual, m * J->ld_res + n);
+  *ref = t;
+  *sabs = sa;
+  return ORACLE_OK;
+}
+
+static void *gemm_worker(void *arg) {
+  gemm_job *J = (gemm_job *)arg;
+  double *arow = (double *)malloc(sizeof(double) * (size_t)J->K);
+  if (!arow) { J->status = ORACLE_ERR_SHAPE; return NULL; }
+  J->status = ORACLE_OK;
+  if (J->ms == NULL) {
+    for (int64_t m = J->begin; m < J->end && !J->status; ++m) {
+      for (int64_t k = 0; k < J->K && !J->status; ++k) J->status = dec_a(J, m, k, &arow[k]);
+      for (int64_t n = 0; n < J->N && !J->status; ++n)
+        J->status = one_element(J, arow, m, n, &J->ref[m * J->N + n], &J->sumabs[m * J->N + n]);
+    }
+  } else {
+    for (int64_t i = J->begin; i < J->end && !J->status; ++i) {
+      int64_t m = J->ms[i], n = J->ns[i];
+      for (int64_t k = 0; k < J->K && !J->status; ++k) J->status = dec_a(J, m, k, &arow[k]);
+      if (!J->status) J->status = one_element(J, arow, m, n, &J->ref[i], &J->sumabs[i]);
+    }
+  }
+  free(arow);
+  return NULL;
+}
+
+static int run_jobs(gemm_job *proto, int64_t total, int nthreads) {
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > 256) nthreads = 256;
+  if ((int64_t)nthreads > total) nthreads = (int)(total > 0 ? total : 1);
+  gemm_job jobs[256];
+  pthread_t th[256];
+  int64_t per = (total + nthreads - 1) / nthreads;
+  for (int t = 0; t < nthreads; ++t) {
+    jobs[t] = *proto;
+    jobs[t].begin = t * per < total ? t * per : total;
+    jobs[t].end = (t + 1) * per < total ? (t + 1) * per : total;
+    pthread_create(&th[t], NULL, gemm_worker, &jobs[t]);
+  }
+  int status = ORACLE_OK;
+  for (int t = 0; t < nthreads; ++t) {
+    pthread_join(th[t], NULL);
+    if (jobs[t].status && !status) status = jobs[t].status;
+  }
+  return status;
+}
+
+/* Full GEMM: ref[m][n], sumabs[m][n] for all M x N outputs.
+ * A: aq [M, K] E4M3 codes, asf [M, K/32] E8M0 (row-major).
+ * B: see ORACLE_B_*.  bias: [N] bf16 or NULL.  residual: [M, ld_res] bf16 or
+ * NULL.  Rows are spread over nthreads POSIX threads. */
+int oracle_gemm(const uint8_t *aq, const uint8_t *asf, const uint8_t *b, const uint8_t *bsf,
+                int bkind, int64_t M, int64_t N, int64_t K, const uint16_t *bias,
+                const uint16_t *residual, int64_t ld_res, double alpha, int act,
+                double *ref, double *sumabs, int nthreads) {
+  if (K <= 0 || K % BLOCK || bkind < 0 || bkind > 2) return ORACLE_ERR_SHAPE;
+  gemm_job J = {aq, asf, b, bsf, bkind, M, N, K, bias, residual, ld_res, alpha, act,
+                ref, sumabs, NULL, NULL, 0, 0, 0, 0};
+  return run_jobs(&J, M, nthreads);
+}
+
+/* Sampled GEMM: the same per-element definition at count (m, n) pairs. */
+int oracle_gemm_sampled(const uint8_t *aq, const uint8_t *asf, const uint8_t *b,
+                        const uint8_t *bsf, int bkind, int64_t M, int64_t N, int64_t K,
+                        const uint16_t *bias, const uint16_t *residual, int64_t ld_res,
+                        double alpha, int act, const int64_t *ms, const int64_t *ns,
+                        int64_t count, double *ref, double *sumabs, int nthreads) {
+  if (K <= 0 || K % BLOCK || bkind < 0 || bkind > 2) return ORACLE_ERR_SHAPE;
+  (void)M;
+  gemm_job J = {aq, asf, b, bsf, bkind, M, N, K, bias, residual, ld_res, alpha, act,
+                ref, sumabs, ms, ns, count, 0, 0, 0};
+  return run_jobs(&J, count, nthreads);
+}
