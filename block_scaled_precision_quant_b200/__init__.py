@@ -1,0 +1,295 @@
+"""Python binding of libbq, the C-ABI library declared in include/bq.h.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libbq.so``.  Tensors must live on a CUDA device of compute
+capability 10.0 (B200); torch is used for device memory, streams and the
+optional allocation of outputs.  If ``libbq.so`` has not been built, the first
+call raises -- there is no CPU fallback.
+
+Build the library with ``python -m block_scaled_precision_quant_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbq.so")
+
+# status codes (include/bq.h)
+BQ_OK = 0
+BQ_ERR_NULL = 1
+BQ_ERR_SHAPE = 2
+BQ_ERR_ALIGN = 3
+BQ_ERR_NAN_SCALE = 4
+BQ_ERR_NAN_CODE = 5
+BQ_ERR_ARCH = 6
+BQ_ERR_WORKSPACE = 7
+BQ_ERR_CUDA = 8
+BQ_ERR_TIMEOUT = 9
+BQ_ERR_NONFINITE = 10
+BQ_ERR_INVALID = 11
+
+BQ_SF_ROW32 = 0
+BQ_SF_BLK32x32 = 1
+BQ_ACT_NONE = 0
+BQ_ACT_GELU = 1
+W_MXFP4, W_FP8BLK32, W_MXFP8 = 0, 1, 2
+
+EXPORTS = (
+    "bq_status_string", "bq_version", "bq_sf_bytes", "bq_act_quant", "bq_pack_weight_scales",
+    "bq_unpack_scales", "bq_gemm_mxfp8_mxfp4", "bq_gemm_mxfp8_fp8blk32", "bq_gemm_mxfp8_mxfp8",
+    "bq_gemm_workspace_bytes", "bq_gemm_mxfp8_mxfp4_epilogue", "bq_gemm_mxfp8_fp8blk32_epilogue",
+    "bq_gemm_mxfp8_mxfp8_epilogue", "bq_device_status", "bq_device_report",
+)
+
+
+class BqError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        msg = lib().bq_status_string(status).decode() if _lib is not None else str(status)
+        super().__init__(f"{what}: {msg}" if what else msg)
+
+
+class Epilogue(ctypes.Structure):
+    _fields_ = [("bias", ctypes.c_void_p), ("residual", ctypes.c_void_p),
+                ("ld_residual", ctypes.c_int64), ("alpha", ctypes.c_float), ("act", ctypes.c_int)]
+
+
+class Batch(ctypes.Structure):
+    _fields_ = [("count", ctypes.c_int64), ("stride_a", ctypes.c_int64),
+                ("stride_a_sf", ctypes.c_int64), ("stride_b", ctypes.c_int64),
+                ("stride_b_sf", ctypes.c_int64), ("stride_y", ctypes.c_int64),
+                ("stride_res", ctypes.c_int64)]
+
+
+class GemmConfig(ctypes.Structure):
+    _fields_ = [("block_n", ctypes.c_int), ("split_k", ctypes.c_int), ("swap_ab", ctypes.c_int),
+                ("reserved", ctypes.c_int)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def lib():
+    """The loaded libbq.so (ctypes.CDLL); raises if it was not built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m block_scaled_precision_quant_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        L.bq_status_string.argtypes = [i32]
+        L.bq_status_string.restype = ctypes.c_char_p
+        L.bq_version.restype = i32
+        L.bq_sf_bytes.argtypes = [i64, i64]
+        L.bq_sf_bytes.restype = sz
+        L.bq_act_quant.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp]
+        L.bq_act_quant.restype = i32
+        L.bq_pack_weight_scales.argtypes = [vp, i32, i64, i64, vp, vp, vp]
+        L.bq_pack_weight_scales.restype = i32
+        L.bq_unpack_scales.argtypes = [vp, i64, i64, vp, vp]
+        L.bq_unpack_scales.restype = i32
+        for name in ("bq_gemm_mxfp8_mxfp4", "bq_gemm_mxfp8_fp8blk32", "bq_gemm_mxfp8_mxfp8"):
+            f = getattr(L, name)
+            f.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp]
+            f.restype = i32
+        for name in ("bq_gemm_mxfp8_mxfp4_epilogue", "bq_gemm_mxfp8_fp8blk32_epilogue",
+                     "bq_gemm_mxfp8_mxfp8_epilogue"):
+            f = getattr(L, name)
+            f.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, ctypes.POINTER(Epilogue),
+                          ctypes.POINTER(Batch), vp, sz, ctypes.POINTER(GemmConfig), vp]
+            f.restype = i32
+        L.bq_gemm_workspace_bytes.argtypes = [i32, i64, i64, i64, i64, ctypes.POINTER(GemmConfig)]
+        L.bq_gemm_workspace_bytes.restype = sz
+        L.bq_device_status.argtypes = [vp]
+        L.bq_device_status.restype = i32
+        L.bq_device_report.argtypes = [ctypes.c_char_p, sz]
+        L.bq_device_report.restype = i32
+        _lib = L
+        return L
+
+
+# ------------------------------------------------------------------ helpers --
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream():
+    return ctypes.c_void_p(_torch().cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(status: int, what: str):
+    if status != BQ_OK:
+        raise BqError(status, what)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libbq works on CUDA tensors only")
+
+
+def sf_bytes(rows: int, K: int) -> int:
+    """Bytes of an MMA-layout scale buffer for rows x K (K % 32 == 0)."""
+    return int(lib().bq_sf_bytes(int(rows), int(K)))
+
+
+def version() -> int:
+    return int(lib().bq_version())
+
+
+def status_string(status: int) -> str:
+    return lib().bq_status_string(int(status)).decode()
+
+
+def device_report() -> str:
+    buf = ctypes.create_string_buffer(512)
+    lib().bq_device_report(buf, 512)
+    return buf.value.decode()
+
+
+def device_status():
+    """Synchronizes the current stream; raises BqError(BQ_ERR_TIMEOUT) if a
+    kernel gave up on a barrier wait since the last check."""
+    _check(lib().bq_device_status(_stream()), "device status")
+
+
+# ----------------------------------------------------------- act_quant -----
+
+def act_quant(x, q=None, sf_mma=None, sf_rowmajor=None, status=None):
+    """Per-32 MX quantization of a bf16 [M, K] CUDA tensor (row stride may
+    exceed K).  Returns (q uint8 [M, K] E4M3 codes, sf_mma uint8 MMA-layout
+    scales).  sf_rowmajor ([M, K/32] uint8) and status (int32 [1]) are
+    optional outputs filled when given."""
+    torch = _torch()
+    _need_cuda(x)
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a bf16 [M, K] tensor with unit column stride")
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    if sf_mma is None:
+        sf_mma = torch.empty((max(sf_bytes(M, K), 1),), dtype=torch.uint8, device=x.device)
+    _check(lib().bq_act_quant(_ptr(x), M, K, x.stride(0), _ptr(q), _ptr(sf_mma),
+                              _ptr(sf_rowmajor), _ptr(status), _stream()), "bq_act_quant")
+    return q, sf_mma
+
+
+def pack_weight_scales(scales, kind: int, N: int, K: int, out=None, e4m3_codes=None):
+    """E8M0 weight scales (ROW32 [N, K/32] or BLK32x32 [ceil(N/32), K/32]) to
+    the MMA layout.  Synchronizes the stream; raises on NaN scales or codes."""
+    torch = _torch()
+    _need_cuda(scales, e4m3_codes)
+    if out is None:
+        out = torch.empty((max(sf_bytes(N, K), 1),), dtype=torch.uint8, device=scales.device)
+    _check(lib().bq_pack_weight_scales(_ptr(scales), int(kind), N, K, _ptr(out),
+                                       _ptr(e4m3_codes), _stream()), "bq_pack_weight_scales")
+    return out
+
+
+def unpack_scales(sf_mma, rows: int, K: int, out=None):
+    """MMA-layout scales back to row-major [rows, K/32] uint8."""
+    torch = _torch()
+    _need_cuda(sf_mma)
+    if out is None:
+        out = torch.empty((rows, K // 32), dtype=torch.uint8, device=sf_mma.device)
+    _check(lib().bq_unpack_scales(_ptr(sf_mma), rows, K, _ptr(out), _stream()),
+           "bq_unpack_scales")
+    return out
+
+
+# ---------------------------------------------------------------- GEMM -----
+
+_ws = {}
+_ENTRY = {W_MXFP4: "bq_gemm_mxfp8_mxfp4", W_FP8BLK32: "bq_gemm_mxfp8_fp8blk32",
+          W_MXFP8: "bq_gemm_mxfp8_mxfp8"}
+
+
+def _config(block_n=0, split_k=0, swap_ab=-1):
+    return GemmConfig(int(block_n), int(split_k), int(swap_ab), 0)
+
+
+def workspace_bytes(weight_kind, M, N, K, batch=1, config=None) -> int:
+    cfg = config if config is not None else None
+    return int(lib().bq_gemm_workspace_bytes(int(weight_kind), M, N, K, batch,
+                                             ctypes.byref(cfg) if cfg is not None else None))
+
+
+def _workspace(device, nbytes):
+    """A zero-initialized per-device workspace, grown on demand.  The kernels
+    leave its ticket counters at zero after every call."""
+    torch = _torch()
+    key = device.index if device.index is not None else torch.cuda.current_device()
+    buf = _ws.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.zeros((max(nbytes, 256),), dtype=torch.uint8, device=device)
+        _ws[key] = buf
+    return buf
+
+
+def gemm(weight_kind, a_q, a_sf, b, b_sf, M, N, K, y=None, bias=None, residual=None,
+         alpha=1.0, act=BQ_ACT_NONE, batch=None, config=None, workspace=None):
+    """y = bf16(act(alpha * A B^T + bias) + residual) for weight_kind W_MXFP4,
+    W_FP8BLK32 or W_MXFP8.  batch: None or a dict with 'count' and byte
+    strides ('stride_a', 'stride_a_sf', 'stride_b', 'stride_b_sf', 'stride_y',
+    'stride_res'; 0 broadcasts).  config: GemmConfig or None (auto)."""
+    torch = _torch()
+    _need_cuda(a_q, a_sf, b, b_sf, bias, residual)
+    count = 1 if batch is None else int(batch["count"])
+    if y is None:
+        shape = (M, N) if batch is None else (count, M, N)
+        y = torch.empty(shape, dtype=torch.bfloat16, device=a_q.device)
+    plain = (bias is None and residual is None and alpha == 1.0 and act == BQ_ACT_NONE
+             and batch is None and config is None and workspace is None)
+    if plain:
+        f = getattr(lib(), _ENTRY[weight_kind])
+        _check(f(_ptr(a_q), _ptr(a_sf), _ptr(b), _ptr(b_sf), M, N, K, _ptr(y), _stream()),
+               _ENTRY[weight_kind])
+        return y
+    epi = Epilogue(bias.data_ptr() if bias is not None else None,
+                   residual.data_ptr() if residual is not None else None,
+                   residual.stride(-2) if residual is not None else 0, float(alpha), int(act))
+    bt = None
+    if batch is not None:
+        bt = Batch(count, *(int(batch.get(k, 0)) for k in (
+            "stride_a", "stride_a_sf", "stride_b", "stride_b_sf", "stride_y", "stride_res")))
+    need = workspace_bytes(weight_kind, M, N, K, count, config)
+    ws = workspace
+    if need and ws is None:
+        ws = _workspace(a_q.device, need)
+    f = getattr(lib(), _ENTRY[weight_kind] + "_epilogue")
+    _check(f(_ptr(a_q), _ptr(a_sf), _ptr(b), _ptr(b_sf), M, N, K, _ptr(y), ctypes.byref(epi),
+             ctypes.byref(bt) if bt is not None else None, _ptr(ws),
+             ws.numel() if ws is not None else 0,
+             ctypes.byref(config) if config is not None else None, _stream()),
+           _ENTRY[weight_kind] + "_epilogue")
+    return y
+
+
+def gemm_mxfp8_mxfp4(a_q, a_sf, b_fp4, b_sf, M, N, K, **kw):
+    return gemm(W_MXFP4, a_q, a_sf, b_fp4, b_sf, M, N, K, **kw)
+
+
+def gemm_mxfp8_fp8blk32(a_q, a_sf, b_e4m3, b_sf, M, N, K, **kw):
+    return gemm(W_FP8BLK32, a_q, a_sf, b_e4m3, b_sf, M, N, K, **kw)
+
+
+def gemm_mxfp8_mxfp8(a_q, a_sf, b_e4m3, b_sf, M, N, K, **kw):
+    return gemm(W_MXFP8, a_q, a_sf, b_e4m3, b_sf, M, N, K, **kw)
+
+
+config = _config

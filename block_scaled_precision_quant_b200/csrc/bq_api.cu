@@ -1,0 +1,518 @@
+// bq_api.cu -- host side of libbq: argument checks, tensor maps, schedule
+// choice and kernel launches behind the C ABI declared in include/bq.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "act_quant.cuh"
+#include "bq.h"
+#include "gemm_bs.cuh"
+
+namespace {
+
+// ------------------------------------------------------------ device state --
+
+// Error word the GEMM kernels write when a barrier wait gives up, and the
+// flag word of the prepack scans.  One copy per device (module globals).
+__device__ int g_dev_error;
+__device__ int g_pack_flags;
+
+constexpr int kMaxDevices = 64;
+
+struct DevInfo {
+  bool ready = false;
+  bool arch_ok = false;
+  int num_sms = 0;
+  int* err_ptr = nullptr;
+  int* flags_ptr = nullptr;
+};
+
+std::mutex g_mu;
+DevInfo g_dev[kMaxDevices];
+
+// Returns BQ_OK and fills `info` for the current device, BQ_ERR_ARCH if it is
+// not compute capability 10.0.
+int current_device(DevInfo** info) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevInfo& d = g_dev[dev];
+  if (!d.ready) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return BQ_ERR_CUDA;
+    d.arch_ok = (major == 10 && minor == 0);
+    if (d.arch_ok) {
+      if (cudaGetSymbolAddress(reinterpret_cast<void**>(&d.err_ptr), g_dev_error) != cudaSuccess ||
+          cudaGetSymbolAddress(reinterpret_cast<void**>(&d.flags_ptr), g_pack_flags) !=
+              cudaSuccess)
+        return BQ_ERR_CUDA;
+    }
+    d.ready = true;
+  }
+  *info = &d;
+  return d.arch_ok ? BQ_OK : BQ_ERR_ARCH;
+}
+
+inline bool aligned(const void* p, uintptr_t a) {
+  return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+
+inline int launch_status() {
+  return cudaGetLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
+// ------------------------------------------------------------- tensor maps --
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int get_encoder() {
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode ? BQ_OK : BQ_ERR_CUDA;
+}
+
+// K-major operand: `rows` rows of K codes (row stride `row_bytes`), optional
+// batch dimension (count, stride in bytes), box of 128 codes x box_rows rows,
+// 128B swizzle, zero fill outside the tensor.  fp4 selects the 4-bit type that
+// TMA expands to one byte-slot per code in shared memory (8 data bytes then 8
+// padding bytes per 16 codes), the operand layout kind::mxf8f6f4 reads.
+int make_operand_map(CUtensorMap* m, const void* base, bool fp4, int64_t K, int64_t rows,
+                     int64_t row_bytes, int64_t batch, int64_t batch_bytes, int box_rows) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_bytes),
+                           static_cast<cuuint64_t>(batch_bytes)};
+  cuuint32_t box[3] = {128u, static_cast<cuuint32_t>(box_rows), 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  const cuuint32_t rank = batch > 1 ? 3 : 2;
+  CUresult r = g_encode(m,
+                        fp4 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                        rank, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? BQ_OK : BQ_ERR_ALIGN;
+}
+
+// ---------------------------------------------------------------- schedule --
+
+enum WeightKind { kMxfp4 = 0, kFp8Blk32 = 1, kMxfp8 = 2 };
+
+struct Plan {
+  bool swap = false;
+  int bn = 256;
+  int splits = 1;
+  int kt_total = 0;
+  int kt_per_split = 0;
+  int tiles_p = 0, tiles_q = 0;
+  int64_t units = 0;
+  size_t ws_partial = 0, ws_ticket = 0;
+};
+
+int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
+
+int make_plan(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_config* cfg,
+              int num_sms, Plan* p) {
+  const int req_bn = cfg ? cfg->block_n : 0;
+  const int req_split = cfg ? cfg->split_k : 0;
+  const int req_swap = cfg ? cfg->swap_ab : -1;
+  if (req_bn != 0 && req_bn != 32 && req_bn != 64 && req_bn != 128 && req_bn != 256)
+    return BQ_ERR_INVALID;
+  if (req_split < 0 || req_split > 16 || req_swap < -1 || req_swap > 1) return BQ_ERR_INVALID;
+  p->kt_total = ceil_div(K, 128);
+  p->swap = req_swap == 1 || (req_swap == -1 && M <= 64);
+  if (p->swap) {
+    if (M > 64) return BQ_ERR_INVALID;
+    p->bn = req_bn ? req_bn : (M <= 32 ? 32 : 64);
+    if (p->bn != 32 && p->bn != 64) return BQ_ERR_INVALID;
+    p->tiles_p = ceil_div(N, 128);
+    p->tiles_q = ceil_div(M, p->bn);
+  } else {
+    p->bn = req_bn ? req_bn : (N > 128 ? 256 : 128);
+    if (p->bn != 128 && p->bn != 256) return BQ_ERR_INVALID;
+    p->tiles_p = ceil_div(M, 128);
+    p->tiles_q = ceil_div(N, p->bn);
+  }
+  const int64_t tiles = batch * p->tiles_p * p->tiles_q;
+  int splits = req_split;
+  if (splits == 0) {
+    splits = 1;
+    if (p->swap && tiles < num_sms) {
+      splits = static_cast<int>(num_sms / tiles);
+      if (splits > 16) splits = 16;
+      // keep at least two k-blocks per slice
+      if (splits > p->kt_total / 2) splits = p->kt_total / 2 > 0 ? p->kt_total / 2 : 1;
+    }
+  }
+  if (splits > p->kt_total) splits = p->kt_total;
+  p->kt_per_split = ceil_div(p->kt_total, splits);
+  p->splits = ceil_div(p->kt_total, p->kt_per_split);  // every slice non-empty
+  p->units = tiles * p->splits;
+  if (p->units > 0x7FFFFFFF) return BQ_ERR_SHAPE;
+  if (p->splits > 1) {
+    p->ws_partial = static_cast<size_t>(p->units) * 128 * p->bn * sizeof(float);
+    p->ws_ticket = static_cast<size_t>(tiles) * sizeof(int);
+  }
+  return BQ_OK;
+}
+
+size_t plan_ws_bytes(const Plan& p) {
+  if (p.splits <= 1) return 0;
+  return ((p.ws_partial + 255) & ~static_cast<size_t>(255)) + p.ws_ticket;
+}
+
+// --------------------------------------------------------------- launches --
+
+template <int BN, int STAGES, int ACC, bool SWAP, bool P_FP4, bool Q_FP4>
+int launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const bq::GemmArgs& args,
+                int64_t units, int num_sms, cudaStream_t stream) {
+  using L = bq::GemmSmem<BN, STAGES, ACC>;
+  auto kern = bq::gemm_bs_kernel<BN, STAGES, ACC, SWAP, P_FP4, Q_FP4>;
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) !=
+        cudaSuccess)
+      return BQ_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  int per_sm = 1;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, bq::kNumThreads, L::kBytes);
+  if (per_sm < 1) per_sm = 1;
+  // Co-resident CTAs share the SM's 512 TMEM columns.
+  const int tmem_fit = 512 / L::kTmemCols;
+  if (per_sm > tmem_fit) per_sm = tmem_fit;
+  int64_t grid = static_cast<int64_t>(num_sms) * per_sm;
+  if (grid > units) grid = units;
+  kern<<<static_cast<unsigned>(grid), bq::kNumThreads, L::kBytes, stream>>>(tp, tq, args);
+  return launch_status();
+}
+
+// Dispatch on (swap, bn, fp4 weights) to the compiled instances.
+int run_gemm(const Plan& pl, bool w_fp4, const CUtensorMap& tp, const CUtensorMap& tq,
+             const bq::GemmArgs& args, int num_sms, cudaStream_t st) {
+  if (!pl.swap) {
+    if (pl.bn == 256)
+      return w_fp4 ? launch_gemm<256, 4, 1, false, false, true>(tp, tq, args, pl.units, num_sms, st)
+                   : launch_gemm<256, 4, 1, false, false, false>(tp, tq, args, pl.units, num_sms, st);
+    return w_fp4 ? launch_gemm<128, 6, 2, false, false, true>(tp, tq, args, pl.units, num_sms, st)
+                 : launch_gemm<128, 6, 2, false, false, false>(tp, tq, args, pl.units, num_sms, st);
+  }
+  if (pl.bn == 32)
+    return w_fp4 ? launch_gemm<32, 4, 1, true, true, false>(tp, tq, args, pl.units, num_sms, st)
+                 : launch_gemm<32, 4, 1, true, false, false>(tp, tq, args, pl.units, num_sms, st);
+  return w_fp4 ? launch_gemm<64, 4, 1, true, true, false>(tp, tq, args, pl.units, num_sms, st)
+               : launch_gemm<64, 4, 1, true, false, false>(tp, tq, args, pl.units, num_sms, st);
+}
+
+int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, const void* b_sf,
+               int64_t M, int64_t N, int64_t K, void* y, const bq_epilogue* epi,
+               const bq_batch* batch, void* ws, size_t ws_bytes, const bq_gemm_config* cfg,
+               bq_stream_t stream) {
+  DevInfo* dev = nullptr;
+  int st = current_device(&dev);
+  if (st != BQ_OK) return st;
+  if (M < 0 || N < 0 || K <= 0 || K % 32 != 0) return BQ_ERR_SHAPE;
+  const int64_t count = batch ? batch->count : 1;
+  if (count < 0) return BQ_ERR_SHAPE;
+  if (M == 0 || N == 0 || count == 0) return BQ_OK;
+  if (!a_q || !a_sf || !b || !b_sf || !y) return BQ_ERR_NULL;
+  const bool w_fp4 = wk == kMxfp4;
+  if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF || count > 65535) return BQ_ERR_SHAPE;
+  if (N % 8 != 0) return BQ_ERR_SHAPE;
+  if (w_fp4 && K % 128 != 0) return BQ_ERR_SHAPE;
+  if (!aligned(a_q, 16) || !aligned(a_sf, 16) || !aligned(b_sf, 16) || !aligned(y, 16) ||
+      !aligned(b, w_fp4 ? 32 : 16))
+    return BQ_ERR_ALIGN;
+  const void* bias = epi ? epi->bias : nullptr;
+  const void* res = epi ? epi->residual : nullptr;
+  const int64_t ldres = epi ? epi->ld_residual : 0;
+  if (epi && epi->act != BQ_ACT_NONE && epi->act != BQ_ACT_GELU) return BQ_ERR_INVALID;
+  if (bias && !aligned(bias, 16)) return BQ_ERR_ALIGN;
+  if (res && (!aligned(res, 16) || ldres % 8 != 0 || ldres < N)) return BQ_ERR_ALIGN;
+  int64_t sa = 0, ssa = 0, sb = 0, ssb = 0, sy = 0, sr = 0;
+  if (batch && count > 1) {
+    sa = batch->stride_a;
+    ssa = batch->stride_a_sf;
+    sb = batch->stride_b;
+    ssb = batch->stride_b_sf;
+    sy = batch->stride_y;
+    sr = batch->stride_res;
+    if (sa < 0 || ssa < 0 || sb < 0 || ssb < 0 || sy < 0 || sr < 0) return BQ_ERR_SHAPE;
+    if (sa % 16 || ssa % 16 || ssb % 16 || sy % 16 || sr % 16 || sb % (w_fp4 ? 32 : 16))
+      return BQ_ERR_ALIGN;
+    if (sy == 0) return BQ_ERR_SHAPE;  // problems would overwrite each other
+  }
+  Plan pl;
+  st = make_plan(M, N, K, count, cfg, dev->num_sms, &pl);
+  if (st != BQ_OK) return st;
+  const size_t need = plan_ws_bytes(pl);
+  if (need > 0 && (!ws || ws_bytes < need || !aligned(ws, 16))) return BQ_ERR_WORKSPACE;
+  if (get_encoder() != BQ_OK) return BQ_ERR_CUDA;
+
+  // Tensor maps: activations A [M, K] (row stride K), weights B [N, K] or [N, K/2].
+  CUtensorMap map_a, map_b;
+  const int a_box = pl.swap ? pl.bn : 128;
+  const int b_box = pl.swap ? 128 : pl.bn;
+  const bool a_batched = count > 1 && sa != 0;
+  const bool b_batched = count > 1 && sb != 0;
+  st = make_operand_map(&map_a, a_q, false, K, M, K, a_batched ? count : 1, sa, a_box);
+  if (st != BQ_OK) return st;
+  st = make_operand_map(&map_b, b, w_fp4, K, N, w_fp4 ? K / 2 : K, b_batched ? count : 1, sb,
+                        b_box);
+  if (st != BQ_OK) return st;
+
+  bq::GemmArgs g;
+  memset(&g, 0, sizeof(g));
+  g.M = static_cast<int>(M);
+  g.N = static_cast<int>(N);
+  g.K = static_cast<int>(K);
+  g.batch = static_cast<int>(count);
+  g.kt_total = pl.kt_total;
+  g.splits = pl.splits;
+  g.kt_per_split = pl.kt_per_split;
+  g.tiles_p = pl.tiles_p;
+  g.tiles_q = pl.tiles_q;
+  g.raster_group = 8;
+  g.sf_katoms = ceil_div(K, 128);
+  g.sf_q_rowatoms = ceil_div(pl.swap ? M : N, 128);
+  const uint8_t* sfa = static_cast<const uint8_t*>(a_sf);
+  const uint8_t* sfb = static_cast<const uint8_t*>(b_sf);
+  g.sf_p = pl.swap ? sfb : sfa;
+  g.sf_q = pl.swap ? sfa : sfb;
+  g.sf_p_bstride = pl.swap ? ssb : ssa;
+  g.sf_q_bstride = pl.swap ? ssa : ssb;
+  g.p_batched = pl.swap ? b_batched : a_batched;
+  g.q_batched = pl.swap ? a_batched : b_batched;
+  g.y = static_cast<__nv_bfloat16*>(y);
+  g.ldy = N;
+  g.y_bstride = sy / 2;
+  g.bias = static_cast<const __nv_bfloat16*>(bias);
+  g.res = static_cast<const __nv_bfloat16*>(res);
+  g.ldres = ldres;
+  g.res_bstride = sr / 2;
+  g.alpha = epi ? epi->alpha : 1.0f;
+  g.act = epi ? epi->act : BQ_ACT_NONE;
+  if (pl.splits > 1) {
+    g.ws_partial = static_cast<float*>(ws);
+    g.ws_ticket = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) +
+                                         ((pl.ws_partial + 255) & ~static_cast<size_t>(255)));
+  }
+  g.err = dev->err_ptr;
+  const CUtensorMap& tp = pl.swap ? map_b : map_a;
+  const CUtensorMap& tq = pl.swap ? map_a : map_b;
+  return run_gemm(pl, w_fp4, tp, tq, g, dev->num_sms, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+// ================================================================== C ABI ==
+
+extern "C" {
+
+const char* bq_status_string(int status) {
+  switch (status) {
+    case BQ_OK: return "BQ_OK";
+    case BQ_ERR_NULL: return "BQ_ERR_NULL: a required pointer is NULL";
+    case BQ_ERR_SHAPE: return "BQ_ERR_SHAPE: size out of range or not a required multiple";
+    case BQ_ERR_ALIGN: return "BQ_ERR_ALIGN: address or stride breaks the alignment rule";
+    case BQ_ERR_NAN_SCALE: return "BQ_ERR_NAN_SCALE: E8M0 scale byte 255 (NaN)";
+    case BQ_ERR_NAN_CODE: return "BQ_ERR_NAN_CODE: E4M3 weight code 0x7F/0xFF (NaN)";
+    case BQ_ERR_ARCH: return "BQ_ERR_ARCH: device is not compute capability 10.0";
+    case BQ_ERR_WORKSPACE: return "BQ_ERR_WORKSPACE: workspace missing or too small";
+    case BQ_ERR_CUDA: return "BQ_ERR_CUDA: CUDA call or launch failed";
+    case BQ_ERR_TIMEOUT: return "BQ_ERR_TIMEOUT: a kernel gave up waiting on a barrier";
+    case BQ_ERR_NONFINITE: return "BQ_ERR_NONFINITE: NaN or Inf activation";
+    case BQ_ERR_INVALID: return "BQ_ERR_INVALID: enum or option out of range";
+    default: return "BQ_ERR_UNKNOWN";
+  }
+}
+
+int bq_version(void) { return 100; }
+
+size_t bq_sf_bytes(int64_t rows, int64_t K) {
+  if (rows < 0 || K <= 0 || K % 32 != 0) return 0;
+  return static_cast<size_t>((rows + 127) / 128) * static_cast<size_t>((K + 127) / 128) * 512;
+}
+
+int bq_act_quant(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, void* q_e4m3,
+                 void* sf_mma, void* sf_rowmajor, int* d_status, bq_stream_t stream) {
+  DevInfo* dev = nullptr;
+  int st = current_device(&dev);
+  if (st != BQ_OK) return st;
+  if (M < 0 || K <= 0 || K % 32 != 0 || ldx < K) return BQ_ERR_SHAPE;
+  if (M == 0) return BQ_OK;
+  if (!x_bf16 || !q_e4m3 || !sf_mma) return BQ_ERR_NULL;
+  if (!aligned(x_bf16, 16) || ldx % 8 != 0 || !aligned(q_e4m3, 16) || !aligned(sf_mma, 4))
+    return BQ_ERR_ALIGN;
+  const int64_t rows_pad = (M + 127) / 128 * 128;
+  const int64_t chunks = (K / 32 + 15) / 16;
+  if (rows_pad / 8 > 0x7FFFFFFF || chunks > 65535) return BQ_ERR_SHAPE;
+  dim3 grid(static_cast<unsigned>(rows_pad / 8), static_cast<unsigned>(chunks));
+  bq::act_quant_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x_bf16), M, K, ldx, rows_pad,
+      static_cast<uint8_t*>(q_e4m3), static_cast<uint8_t*>(sf_mma),
+      static_cast<uint8_t*>(sf_rowmajor), d_status);
+  return launch_status();
+}
+
+int bq_pack_weight_scales(const void* scales_u8, int kind, int64_t N, int64_t K, void* sf_mma,
+                          const void* e4m3_codes, bq_stream_t stream) {
+  DevInfo* dev = nullptr;
+  int st = current_device(&dev);
+  if (st != BQ_OK) return st;
+  if (kind != BQ_SF_ROW32 && kind != BQ_SF_BLK32x32) return BQ_ERR_INVALID;
+  if (N < 0 || K <= 0 || K % 32 != 0) return BQ_ERR_SHAPE;
+  if (N == 0) return BQ_OK;
+  if (!scales_u8 || !sf_mma) return BQ_ERR_NULL;
+  if (!aligned(sf_mma, 4) || (e4m3_codes && !aligned(e4m3_codes, 16))) return BQ_ERR_ALIGN;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(dev->flags_ptr, 0, sizeof(int), s) != cudaSuccess) return BQ_ERR_CUDA;
+  const int64_t G = K / 32;
+  const int64_t rows_pad = (N + 127) / 128 * 128;
+  const int64_t words = rows_pad * ((G + 3) / 4);
+  const int64_t blocks = (words + 255) / 256 < 4096 ? (words + 255) / 256 : 4096;
+  bq::pack_scales_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+      static_cast<const uint8_t*>(scales_u8), kind, N, G, rows_pad, static_cast<uint8_t*>(sf_mma),
+      dev->flags_ptr);
+  if (launch_status() != BQ_OK) return BQ_ERR_CUDA;
+  if (e4m3_codes) {
+    const int64_t n = N * K;
+    int64_t nb = (n / 16 + 255) / 256;
+    if (nb < 1) nb = 1;
+    if (nb > 4096) nb = 4096;
+    bq::scan_e4m3_nan_kernel<<<static_cast<unsigned>(nb), 256, 0, s>>>(
+        static_cast<const uint8_t*>(e4m3_codes), n, dev->flags_ptr);
+    if (launch_status() != BQ_OK) return BQ_ERR_CUDA;
+  }
+  int flags = 0;
+  if (cudaMemcpyAsync(&flags, dev->flags_ptr, sizeof(int), cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return BQ_ERR_CUDA;
+  if (flags & 1) return BQ_ERR_NAN_SCALE;
+  if (flags & 2) return BQ_ERR_NAN_CODE;
+  return BQ_OK;
+}
+
+int bq_unpack_scales(const void* sf_mma, int64_t rows, int64_t K, void* rowmajor,
+                     bq_stream_t stream) {
+  DevInfo* dev = nullptr;
+  int st = current_device(&dev);
+  if (st != BQ_OK) return st;
+  if (rows < 0 || K <= 0 || K % 32 != 0) return BQ_ERR_SHAPE;
+  if (rows == 0) return BQ_OK;
+  if (!sf_mma || !rowmajor) return BQ_ERR_NULL;
+  const int64_t total = rows * (K / 32);
+  const int64_t blocks = (total + 255) / 256 < 4096 ? (total + 255) / 256 : 4096;
+  bq::unpack_scales_kernel<<<static_cast<unsigned>(blocks), 256, 0,
+                             reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(sf_mma), rows, K / 32, static_cast<uint8_t*>(rowmajor));
+  return launch_status();
+}
+
+// The plain entries take no workspace, so their schedule never splits K.
+static const bq_gemm_config kNoSplit = {0, 1, -1, 0};
+
+int bq_gemm_mxfp8_mxfp4(const void* a_q, const void* a_sf, const void* b_fp4, const void* b_sf,
+                        int64_t M, int64_t N, int64_t K, void* y_bf16, bq_stream_t stream) {
+  return gemm_entry(kMxfp4, a_q, a_sf, b_fp4, b_sf, M, N, K, y_bf16, nullptr, nullptr, nullptr, 0,
+                    &kNoSplit, stream);
+}
+
+int bq_gemm_mxfp8_fp8blk32(const void* a_q, const void* a_sf, const void* b_e4m3,
+                           const void* b_sf, int64_t M, int64_t N, int64_t K, void* y_bf16,
+                           bq_stream_t stream) {
+  return gemm_entry(kFp8Blk32, a_q, a_sf, b_e4m3, b_sf, M, N, K, y_bf16, nullptr, nullptr,
+                    nullptr, 0, &kNoSplit, stream);
+}
+
+int bq_gemm_mxfp8_mxfp8(const void* a_q, const void* a_sf, const void* b_e4m3, const void* b_sf,
+                        int64_t M, int64_t N, int64_t K, void* y_bf16, bq_stream_t stream) {
+  return gemm_entry(kMxfp8, a_q, a_sf, b_e4m3, b_sf, M, N, K, y_bf16, nullptr, nullptr, nullptr,
+                    0, &kNoSplit, stream);
+}
+
+size_t bq_gemm_workspace_bytes(int weight_kind, int64_t M, int64_t N, int64_t K, int64_t batch,
+                               const bq_gemm_config* cfg) {
+  if (weight_kind < 0 || weight_kind > 2 || M <= 0 || N <= 0 || K <= 0 || batch <= 0) return 0;
+  DevInfo* dev = nullptr;
+  if (current_device(&dev) != BQ_OK) return 0;
+  Plan pl;
+  if (make_plan(M, N, K, batch, cfg, dev->num_sms, &pl) != BQ_OK) return 0;
+  return plan_ws_bytes(pl);
+}
+
+int bq_gemm_mxfp8_mxfp4_epilogue(const void* a_q, const void* a_sf, const void* b_fp4,
+                                 const void* b_sf, int64_t M, int64_t N, int64_t K, void* y_bf16,
+                                 const bq_epilogue* epi, const bq_batch* batch, void* workspace,
+                                 size_t workspace_bytes, const bq_gemm_config* cfg,
+                                 bq_stream_t stream) {
+  return gemm_entry(kMxfp4, a_q, a_sf, b_fp4, b_sf, M, N, K, y_bf16, epi, batch, workspace,
+                    workspace_bytes, cfg, stream);
+}
+
+int bq_gemm_mxfp8_fp8blk32_epilogue(const void* a_q, const void* a_sf, const void* b_e4m3,
+                                    const void* b_sf, int64_t M, int64_t N, int64_t K,
+                                    void* y_bf16, const bq_epilogue* epi, const bq_batch* batch,
+                                    void* workspace, size_t workspace_bytes,
+                                    const bq_gemm_config* cfg, bq_stream_t stream) {
+  return gemm_entry(kFp8Blk32, a_q, a_sf, b_e4m3, b_sf, M, N, K, y_bf16, epi, batch, workspace,
+                    workspace_bytes, cfg, stream);
+}
+
+int bq_gemm_mxfp8_mxfp8_epilogue(const void* a_q, const void* a_sf, const void* b_e4m3,
+                                 const void* b_sf, int64_t M, int64_t N, int64_t K, void* y_bf16,
+                                 const bq_epilogue* epi, const bq_batch* batch, void* workspace,
+                                 size_t workspace_bytes, const bq_gemm_config* cfg,
+                                 bq_stream_t stream) {
+  return gemm_entry(kMxfp8, a_q, a_sf, b_e4m3, b_sf, M, N, K, y_bf16, epi, batch, workspace,
+                    workspace_bytes, cfg, stream);
+}
+
+int bq_device_status(bq_stream_t stream) {
+  DevInfo* dev = nullptr;
+  int st = current_device(&dev);
+  if (st != BQ_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int err = 0;
+  if (cudaMemcpyAsync(&err, dev->err_ptr, sizeof(int), cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess ||
+      cudaMemsetAsync(dev->err_ptr, 0, sizeof(int), s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return BQ_ERR_CUDA;
+  return err ? BQ_ERR_TIMEOUT : BQ_OK;
+}
+
+int bq_device_report(char* buf, size_t n) {
+  if (!buf || n == 0) return BQ_ERR_NULL;
+  int dev = 0;
+  cudaDeviceProp p;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaGetDeviceProperties(&p, dev) != cudaSuccess) {
+    snprintf(buf, n, "no CUDA device");
+    return BQ_ERR_CUDA;
+  }
+  int clk = 0, mclk = 0;
+  cudaDeviceGetAttribute(&clk, cudaDevAttrClockRate, dev);
+  cudaDeviceGetAttribute(&mclk, cudaDevAttrMemoryClockRate, dev);
+  snprintf(buf, n, "%s cc %d.%d, %d SMs, L2 %d KiB, smem/block optin %zu KiB, sm clock %d MHz, mem clock %d MHz",
+           p.name, p.major, p.minor, p.multiProcessorCount, p.l2CacheSize / 1024,
+           p.sharedMemPerBlockOptin / 1024, clk / 1000, mclk / 1000);
+  return (p.major == 10 && p.minor == 0) ? BQ_OK : BQ_ERR_ARCH;
+}
+
+}  // extern "C"

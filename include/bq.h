@@ -1,0 +1,231 @@
+/*
+ * bq.h -- C ABI of libbq: MX (per-32, E8M0-scaled) activation quantization and
+ * block-scaled GEMMs for NVIDIA B200 (sm_100a).
+ *
+ * What the calls compute is defined on the "formats.py" page
+ * (dsv41-sampled-drafting, code/offload/dspark/native/formats.py): the
+ * activation quantizer (act_scale / act_quant, module docstring "act_qdq
+ * reproduces ...") and the exact decoders of the weight formats (module
+ * docstring "Formats", decode_fp4, decode_fp8_block).  The fused bias /
+ * residual / GELU epilogue follows the FlashRT "fp4-gemm" page ("Available
+ * Functions": nvfp4_gemm_bias_bf16, ..._bias_residual_bf16, ..._bias_gelu_bf16)
+ * and the AstrAI commit log (bias added in fp32 before the single bf16
+ * rounding; batch strides with stride 0 broadcasting a size-1 batch).
+ *
+ * Conventions for every call:
+ *   - All data pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or synchronizes on the data path.
+ *   - Every call is asynchronous on the caller's stream (NULL = the legacy
+ *     default stream); the return value only reports argument checks and
+ *     launch errors.  Exceptions, which synchronize the stream, are named.
+ *   - Sizes are 64-bit.  M or N equal to 0 returns BQ_OK without a launch.
+ *   - Argument faults are detected on the host before any launch; nothing is
+ *     launched when a call returns an error.
+ *   - The current device must be compute capability 10.0 (B200), else
+ *     BQ_ERR_ARCH.
+ *
+ * Layouts:
+ *   - bf16 activations x [M, K] row-major with row stride ldx elements.
+ *   - E4M3 codes (activations, FP8 weights) [rows, K] row-major, 1 byte each.
+ *   - MXFP4 weights [N, K/2] bytes; byte j of a row holds input 2j in the
+ *     low nibble and 2j+1 in the high nibble.
+ *   - bf16 output y [M, N] row-major, y = A * B^T.
+ *   - Scale factors in "MMA layout" (the layout the GEMM consumes): for a
+ *     matrix of R rows and K inputs the G = K/32 scale bytes of each row are
+ *     stored in 512-byte atoms of 128 rows x 4 scale columns.  The atom of
+ *     (row r, column c) is (r / 128) * ceil(G / 4) + c / 4 and the byte inside
+ *     it is (r % 32) * 16 + ((r / 32) % 4) * 4 + (c % 4).  Rows are padded to a
+ *     multiple of 128 and columns to a multiple of 4; the producers write the
+ *     padding bytes as 127 (2^0).  Size: bq_sf_bytes(R, K).
+ */
+#ifndef BQ_H
+#define BQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *bq_stream_t;
+
+/* ---- status codes ---------------------------------------------------- */
+enum {
+  BQ_OK = 0,
+  BQ_ERR_NULL = 1,        /* a required pointer is NULL */
+  BQ_ERR_SHAPE = 2,       /* size out of range or not a multiple the call needs */
+  BQ_ERR_ALIGN = 3,       /* base address or row stride breaks the 16-byte (FP4: 32-byte) rule */
+  BQ_ERR_NAN_SCALE = 4,   /* an E8M0 scale byte is 255 (NaN) -- prepack only */
+  BQ_ERR_NAN_CODE = 5,    /* an E4M3 weight code is 0x7F or 0xFF (NaN) -- prepack only */
+  BQ_ERR_ARCH = 6,        /* current device is not compute capability 10.0 */
+  BQ_ERR_WORKSPACE = 7,   /* workspace NULL or smaller than bq_gemm_workspace_bytes() */
+  BQ_ERR_CUDA = 8,        /* a CUDA runtime call or kernel launch failed */
+  BQ_ERR_TIMEOUT = 9,     /* a kernel gave up waiting on one of its own barriers */
+  BQ_ERR_NONFINITE = 10,  /* act_quant saw a NaN or Inf input */
+  BQ_ERR_INVALID = 11     /* an enum argument is out of range */
+};
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *bq_status_string(int status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int bq_version(void);
+
+/* Bytes of an MMA-layout scale buffer for `rows` rows and `K` inputs
+ * (K % 32 == 0): ceil(rows / 128) * ceil(K / 128) * 512.  0 for bad sizes. */
+size_t bq_sf_bytes(int64_t rows, int64_t K);
+
+/* ---- activation quantization ------------------------------------------ */
+
+/* bq_act_quant -- per-32 MX quantization of bf16 activations
+ * ("formats.py" page: act_scale, act_quant; docstring "act_qdq reproduces").
+ *
+ * For every 32 consecutive elements of a row: amax = max(max|x|, 1e-4) in
+ * fp32; t = fp32(amax * fp32(1/448)); e = ceil(log2 t) from t's exponent bits;
+ * scale byte = e + 127 (E8M0); q = E4M3 round-to-nearest-even of
+ * clamp(x / 2^e, -448, 448).  Bit-exact with that definition for finite input.
+ *
+ *   x_bf16      [M, K] bf16, row stride ldx elements (ldx >= K, ldx % 8 == 0,
+ *               base 16-byte aligned)
+ *   M, K        M >= 0; K > 0 and K % 32 == 0
+ *   q_e4m3      out [M, K] E4M3 codes, row stride K, 16-byte aligned
+ *   sf_mma      out bq_sf_bytes(M, K) bytes, MMA layout, padding written as 127
+ *   sf_rowmajor optional out [M, K/32] scale bytes row-major (NULL to skip)
+ *   d_status    optional device int; the kernel ORs in 1 when it meets a NaN
+ *               or Inf input (whose outputs are then unspecified).  The caller
+ *               zeroes it.  NULL to skip the check.
+ * Errors: BQ_ERR_NULL, BQ_ERR_SHAPE, BQ_ERR_ALIGN, BQ_ERR_ARCH, BQ_ERR_CUDA. */
+int bq_act_quant(const void *x_bf16, int64_t M, int64_t K, int64_t ldx, void *q_e4m3,
+                 void *sf_mma, void *sf_rowmajor, int *d_status, bq_stream_t stream);
+
+/* ---- weight scale prepack (off the hot path) --------------------------- */
+
+enum {
+  BQ_SF_ROW32 = 0,    /* scales [N, K/32]: one per 32 inputs of a row (MXFP4, MXFP8) */
+  BQ_SF_BLK32x32 = 1  /* scales [ceil(N/32), ceil(K/32)]: one per 32x32 block (FP8 weights) */
+};
+
+/* bq_pack_weight_scales -- E8M0 weight scales to MMA layout
+ * ("formats.py" page, docstring "Formats": FP4 scales [out, in/32], FP8 scales
+ * [ceil(out/32), ceil(in/32)]; decode_fp8_block repeats a block's scale over
+ * its 32 rows and 32 inputs).  A 32x32 block scale is written to each of its
+ * 32 rows.  Scans the scales for 255 (NaN) and, when e4m3_codes ([N, K]) is
+ * given, the codes for 0x7F/0xFF.  SYNCHRONIZES `stream` to report those.
+ *   sf_mma: out, bq_sf_bytes(N, K) bytes.  K % 32 == 0.
+ * Errors: BQ_ERR_NAN_SCALE, BQ_ERR_NAN_CODE (sf_mma content then unspecified),
+ *         BQ_ERR_NULL, BQ_ERR_SHAPE, BQ_ERR_INVALID, BQ_ERR_ARCH, BQ_ERR_CUDA. */
+int bq_pack_weight_scales(const void *scales_u8, int kind, int64_t N, int64_t K, void *sf_mma,
+                          const void *e4m3_codes, bq_stream_t stream);
+
+/* bq_unpack_scales -- MMA layout back to row-major [rows, K/32] bytes (for
+ * tests and inspection). */
+int bq_unpack_scales(const void *sf_mma, int64_t rows, int64_t K, void *rowmajor,
+                     bq_stream_t stream);
+
+/* ---- block-scaled GEMM -------------------------------------------------- */
+
+/* Operands of every GEMM call:
+ *   a_q   [M, K] E4M3 activation codes (from bq_act_quant), 16-byte aligned
+ *   a_sf  MMA-layout scales of A (from bq_act_quant), bq_sf_bytes(M, K)
+ *   b     weights, 16-byte aligned (MXFP4: 32-byte aligned):
+ *           mxfp4:    [N, K/2] packed E2M1, requires K % 128 == 0
+ *           fp8blk32: [N, K] E4M3 (32x32 block scales, packed by
+ *                     bq_pack_weight_scales(BQ_SF_BLK32x32))
+ *           mxfp8:    [N, K] E4M3 (per-32 row scales, from bq_act_quant or
+ *                     bq_pack_weight_scales(BQ_SF_ROW32))
+ *   b_sf  MMA-layout scales of B, bq_sf_bytes(N, K)
+ *   y     [M, N] bf16 out, N % 8 == 0, 16-byte aligned
+ * y[m, n] = bf16_RNE(sum_k a[m,k] b[n,k]) with a, b the decoded operands
+ * (code * 2^(scale-127)) and fp32 accumulation.
+ * Errors: BQ_ERR_NULL, BQ_ERR_SHAPE, BQ_ERR_ALIGN, BQ_ERR_ARCH, BQ_ERR_CUDA.
+ * No data is scanned on this path: NaN scales or codes give NaN outputs. */
+int bq_gemm_mxfp8_mxfp4(const void *a_q, const void *a_sf, const void *b_fp4, const void *b_sf,
+                        int64_t M, int64_t N, int64_t K, void *y_bf16, bq_stream_t stream);
+int bq_gemm_mxfp8_fp8blk32(const void *a_q, const void *a_sf, const void *b_e4m3,
+                           const void *b_sf, int64_t M, int64_t N, int64_t K, void *y_bf16,
+                           bq_stream_t stream);
+int bq_gemm_mxfp8_mxfp8(const void *a_q, const void *a_sf, const void *b_e4m3, const void *b_sf,
+                        int64_t M, int64_t N, int64_t K, void *y_bf16, bq_stream_t stream);
+
+enum { BQ_ACT_NONE = 0, BQ_ACT_GELU = 1 };
+
+/* Fused epilogue, applied in fp32 with one bf16 rounding at the end:
+ *   y = bf16_RNE( act(alpha * acc + bias[n]) + residual[m, n] )
+ * act: BQ_ACT_NONE or BQ_ACT_GELU (erf form 0.5 t (1 + erf(t / sqrt 2))).
+ * bias: [N] bf16 or NULL.  residual: [M, ld_residual] bf16 or NULL
+ * (ld_residual % 8 == 0, 16-byte aligned). */
+typedef struct {
+  const void *bias;
+  const void *residual;
+  int64_t ld_residual;
+  float alpha;
+  int act;
+} bq_epilogue;
+
+/* Batched GEMM: `count` independent problems.  Strides are in BYTES between
+ * consecutive problems; a stride of 0 broadcasts that operand (e.g. one weight
+ * shared by all problems).  stride_a_sf / stride_b_sf step the MMA-layout
+ * scale buffers and must be multiples of 16.  Bias is shared by all problems. */
+typedef struct {
+  int64_t count;
+  int64_t stride_a, stride_a_sf;
+  int64_t stride_b, stride_b_sf;
+  int64_t stride_y, stride_res;
+} bq_batch;
+
+/* Optional schedule override (tests and sweeps); NULL = built-in dispatch.
+ * block_n: 0 (auto); 128 or 256 weight rows per CTA tile, or with swap_ab 32 or
+ *          64 activation rows per CTA tile.
+ * split_k: 0 (auto) or 1..16 slices of K (needs a workspace when > 1).
+ * swap_ab: -1 (auto), 0, or 1 (weights on the 128-row MMA side, for M <= 64). */
+typedef struct {
+  int block_n;
+  int split_k;
+  int swap_ab;
+  int reserved;
+} bq_gemm_config;
+
+/* Workspace bytes the *_epilogue calls need for a problem (0 when the chosen
+ * schedule needs none).  weight_kind: 0 mxfp4, 1 fp8blk32, 2 mxfp8. */
+size_t bq_gemm_workspace_bytes(int weight_kind, int64_t M, int64_t N, int64_t K, int64_t batch,
+                               const bq_gemm_config *cfg);
+
+/* GEMM + fused epilogue (+ optional batch).  epi NULL = plain (alpha 1, no
+ * bias, residual or activation).  batch NULL = one problem.  workspace: device
+ * memory of at least bq_gemm_workspace_bytes(...) bytes (may be NULL when that
+ * is 0); the call leaves it ready for the next call, and calls that share one
+ * workspace must not overlap on the GPU. */
+int bq_gemm_mxfp8_mxfp4_epilogue(const void *a_q, const void *a_sf, const void *b_fp4,
+                                 const void *b_sf, int64_t M, int64_t N, int64_t K, void *y_bf16,
+                                 const bq_epilogue *epi, const bq_batch *batch, void *workspace,
+                                 size_t workspace_bytes, const bq_gemm_config *cfg,
+                                 bq_stream_t stream);
+int bq_gemm_mxfp8_fp8blk32_epilogue(const void *a_q, const void *a_sf, const void *b_e4m3,
+                                    const void *b_sf, int64_t M, int64_t N, int64_t K,
+                                    void *y_bf16, const bq_epilogue *epi, const bq_batch *batch,
+                                    void *workspace, size_t workspace_bytes,
+                                    const bq_gemm_config *cfg, bq_stream_t stream);
+int bq_gemm_mxfp8_mxfp8_epilogue(const void *a_q, const void *a_sf, const void *b_e4m3,
+                                 const void *b_sf, int64_t M, int64_t N, int64_t K, void *y_bf16,
+                                 const bq_epilogue *epi, const bq_batch *batch, void *workspace,
+                                 size_t workspace_bytes, const bq_gemm_config *cfg,
+                                 bq_stream_t stream);
+
+/* ---- diagnostics -------------------------------------------------------- */
+
+/* Reads and clears the library's device error word on the current device.
+ * SYNCHRONIZES `stream`.  Returns BQ_OK, or BQ_ERR_TIMEOUT when a kernel gave
+ * up on a barrier wait since the last call (its outputs are then invalid). */
+int bq_device_status(bq_stream_t stream);
+
+/* Writes a one-line report of the current device (name, compute capability,
+ * SM count, L2 size, clocks) into buf (always NUL-terminated). */
+int bq_device_report(char *buf, size_t n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BQ_H */

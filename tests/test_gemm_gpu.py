@@ -1,0 +1,289 @@
+"""Parity of the CUDA block-scaled GEMMs with the fp64 oracle.
+
+Every output element must satisfy |y - ref| <= ulp_bf16(|ref|) + 2^-20 * S with
+S = |alpha| sum_k |a_k b_k| (+ |bias| + |residual|, GELU branch scaled by 1.13),
+where ref is the oracle's exact-decode fp64 result.  Small and mid sizes are
+compared in full (several tiles plus ragged tails in M, N and K); the
+workloads' full sizes are compared on sampled outputs, in the launch
+configuration the benchmark uses.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import block_scaled_precision_quant_b200 as bq
+from block_scaled_precision_quant_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+OKIND = {bq.W_MXFP4: oracle.B_FP4, bq.W_FP8BLK32: oracle.B_FP8BLK, bq.W_MXFP8: oracle.B_FP8ROW}
+
+
+def to_dev_bf16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def to_dev_u8(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def bf16_to_f64(bits):
+    return (np.asarray(bits).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+class Case:
+    """Inputs of one GEMM problem (host copies for the oracle, device copies
+    for the CUDA path)."""
+
+    def __init__(self, wk, M, N, K, seed=0, act_gp=None, bias=False, residual=False,
+                 alpha=1.0, act=bq.BQ_ACT_NONE):
+        self.wk, self.M, self.N, self.K = wk, M, N, K
+        self.alpha, self.act = alpha, act
+        self.x = synth.activations(M, K, seed=seed, group_pow2=act_gp)
+        if wk == bq.W_MXFP4:
+            self.b, self.bsf = synth.mxfp4_weight(N, K, seed=seed + 100)
+        elif wk == bq.W_FP8BLK32:
+            self.b, self.bsf = synth.fp8_weight_blk32(N, K, seed=seed + 100)
+        else:
+            w = synth.activations(N, K, seed=seed + 100)
+            self.b, self.bsf = oracle.act_quant(w)
+        self.bias = synth.bias(N, seed=seed + 200) if bias else None
+        self.res = synth.residual(M, N, seed=seed + 300) if residual else None
+
+    def gpu(self, config=None, batch=None):
+        xd = to_dev_bf16(self.x)
+        aq, asf = bq.act_quant(xd)
+        bd = to_dev_u8(self.b)
+        kind = bq.BQ_SF_BLK32x32 if self.wk == bq.W_FP8BLK32 else bq.BQ_SF_ROW32
+        bsf = bq.pack_weight_scales(to_dev_u8(self.bsf), kind, self.N, self.K,
+                                    e4m3_codes=bd if self.wk != bq.W_MXFP4 else None)
+        y = bq.gemm(self.wk, aq, asf, bd, bsf, self.M, self.N, self.K,
+                    bias=to_dev_bf16(self.bias) if self.bias is not None else None,
+                    residual=to_dev_bf16(self.res) if self.res is not None else None,
+                    alpha=self.alpha, act=self.act, config=config)
+        bq.device_status()
+        self.aq_gpu = aq.cpu().numpy()
+        return bf16_to_f64(y.cpu().view(torch.int16).numpy().view(np.uint16))
+
+    def oracle_full(self):
+        aq, asf = oracle.act_quant(self.x)
+        return oracle.gemm(aq, asf, self.b, self.bsf, OKIND[self.wk], self.M, self.N, self.K,
+                           bias=self.bias, residual=self.res, alpha=self.alpha, act=self.act)
+
+    def oracle_sampled(self, ms, ns):
+        aq, asf = oracle.act_quant(self.x)
+        return oracle.gemm_sampled(aq, asf, self.b, self.bsf, OKIND[self.wk], self.M, self.N,
+                                   self.K, ms, ns, bias=self.bias, residual=self.res,
+                                   alpha=self.alpha, act=self.act)
+
+    def tol(self, ref, sabs, ms=None, ns=None):
+        babs = None
+        rabs = None
+        if self.bias is not None:
+            babs = np.abs(bf16_to_f64(self.bias))
+            babs = babs[None, :] if ms is None else babs[ns]
+        if self.res is not None:
+            rabs = np.abs(bf16_to_f64(self.res))
+            rabs = rabs if ms is None else rabs[ms, ns]
+        return oracle.gemm_tolerance(ref, sabs, self.alpha, babs, rabs, self.act)
+
+
+def assert_close(y, ref, tol, what=""):
+    err = np.abs(y - ref)
+    bad = np.argwhere(~(err <= tol))
+    assert bad.size == 0, (f"{what}: {bad.shape[0]} of {err.size} outside tolerance; first "
+                           f"{[(tuple(i), float(y[tuple(i)]), float(ref[tuple(i)])) for i in bad[:4]]}")
+
+
+def run_full(case, config=None):
+    y = case.gpu(config)
+    ref, sabs = case.oracle_full()
+    aq_oracle, _ = oracle.act_quant(case.x)
+    assert np.array_equal(case.aq_gpu, aq_oracle)
+    assert_close(y, ref, case.tol(ref, sabs), f"{case.wk} {case.M}x{case.N}x{case.K}")
+    return y, ref, sabs
+
+
+def run_sampled(case, n=4000, seed=0, config=None):
+    y = case.gpu(config)
+    rng = np.random.default_rng(seed)
+    ms = rng.integers(0, case.M, n)
+    ns = rng.integers(0, case.N, n)
+    # always include the corners and the last tile's tail
+    ms = np.concatenate([ms, [0, case.M - 1, 0, case.M - 1]])
+    ns = np.concatenate([ns, [0, 0, case.N - 1, case.N - 1]])
+    ref, sabs = case.oracle_sampled(ms, ns)
+    assert_close(y[ms, ns], ref, case.tol(ref, sabs, ms, ns), f"{case.wk} sampled")
+
+
+# ------------------------------------------------------------ small / mid --
+
+@pytest.mark.parametrize("wk", [bq.W_MXFP4, bq.W_FP8BLK32, bq.W_MXFP8])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 128), (200, 264, 384), (257, 520, 256),
+                                   (130, 128, 512)])
+def test_multi_tile_ragged(wk, M, N, K):
+    run_full(Case(wk, M, N, K, seed=M + N))
+
+
+@pytest.mark.parametrize("wk", [bq.W_FP8BLK32, bq.W_MXFP8])
+@pytest.mark.parametrize("K", [32, 96, 352, 640])
+def test_k_tails(wk, K):
+    run_full(Case(wk, 150, 136, K, seed=K))
+
+
+def test_pr1_reference_config():
+    """act_quant then MXFP8 x MXFP4, M=64 N=512 K=1024, A scaled by 2^U{-4..4}
+    per group, no bias (compared in full)."""
+    run_full(Case(bq.W_MXFP4, 64, 512, 1024, seed=0, act_gp=(-4, 4)))
+
+
+@pytest.mark.parametrize("block_n", [128, 256])
+@pytest.mark.parametrize("wk", [bq.W_MXFP4, bq.W_FP8BLK32])
+def test_block_n_choices(block_n, wk):
+    run_full(Case(wk, 300, 520, 512, seed=3), config=bq.config(block_n=block_n, split_k=1,
+                                                                swap_ab=0))
+
+
+# ------------------------------------------------------------- epilogues --
+
+@pytest.mark.parametrize("wk", [bq.W_MXFP4, bq.W_FP8BLK32])
+@pytest.mark.parametrize("bias,res,act,alpha", [(True, False, bq.BQ_ACT_NONE, 1.0),
+                                                (False, True, bq.BQ_ACT_NONE, 1.0),
+                                                (True, True, bq.BQ_ACT_NONE, 0.5),
+                                                (True, False, bq.BQ_ACT_GELU, 1.0),
+                                                (False, False, bq.BQ_ACT_GELU, 2.0)])
+def test_epilogues(wk, bias, res, act, alpha):
+    run_full(Case(wk, 190, 264, 256, seed=7, bias=bias, residual=res, act=act, alpha=alpha))
+
+
+# ------------------------------------------------- decode: swap + split-K --
+
+@pytest.mark.parametrize("M", [1, 17, 41, 64])
+@pytest.mark.parametrize("split", [0, 1, 3])
+def test_decode_swap_split(M, split):
+    c = Case(bq.W_MXFP4, M, 640, 1536, seed=M, bias=True)
+    run_full(c, config=bq.config(split_k=split, swap_ab=1))
+
+
+@pytest.mark.parametrize("wk", [bq.W_FP8BLK32, bq.W_MXFP8])
+def test_decode_fp8_weights(wk):
+    run_full(Case(wk, 41, 384, 1024, seed=2, residual=True), config=bq.config(swap_ab=1))
+
+
+def test_decode_without_swap():
+    run_full(Case(bq.W_MXFP4, 41, 640, 1536, seed=9, bias=True),
+             config=bq.config(swap_ab=0, split_k=1))
+
+
+def test_split_k_non_swap():
+    run_full(Case(bq.W_FP8BLK32, 256, 384, 2048, seed=4, residual=True),
+             config=bq.config(swap_ab=0, split_k=4, block_n=128))
+
+
+def test_split_k_repeatable():
+    """Fixed slice order: repeated launches give identical bits."""
+    c = Case(bq.W_MXFP4, 41, 1536, 6144, seed=1, bias=True)
+    y0 = c.gpu()
+    for _ in range(3):
+        assert np.array_equal(c.gpu(), y0)
+
+
+@pytest.mark.parametrize("N,K", [(4608, 1536), (6144, 1536), (1536, 6144)])
+def test_decode_workload_full(N, K):
+    """Decode-shaped linear (M=41, fused bias), compared in full."""
+    run_full(Case(bq.W_MXFP4, 41, N, K, seed=1, bias=True))
+
+
+# ----------------------------------------------------------------- batch --
+
+def test_batched_broadcast_weight_bias_gelu():
+    """Independent problems over one broadcast weight (stride 0), bias+GELU."""
+    count, M, N, K = 3, 200, 264, 256
+    xs = [synth.activations(M, K, seed=40 + i) for i in range(count)]
+    b, bsf = synth.mxfp4_weight(N, K, seed=50)
+    bias = synth.bias(N, seed=51)
+    aqs, sfs = zip(*[bq.act_quant(to_dev_bf16(x)) for x in xs])
+    aq = torch.stack(aqs)
+    asf = torch.stack(sfs)
+    bsf_d = bq.pack_weight_scales(to_dev_u8(bsf), bq.BQ_SF_ROW32, N, K)
+    y = bq.gemm(bq.W_MXFP4, aq, asf, to_dev_u8(b), bsf_d, M, N, K, bias=to_dev_bf16(bias),
+                act=bq.BQ_ACT_GELU,
+                batch=dict(count=count, stride_a=M * K, stride_a_sf=asf.shape[1], stride_b=0,
+                           stride_b_sf=0, stride_y=M * N * 2))
+    bq.device_status()
+    yv = bf16_to_f64(y.cpu().view(torch.int16).numpy().view(np.uint16))
+    for i in range(count):
+        q, s = oracle.act_quant(xs[i])
+        ref, sabs = oracle.gemm(q, s, b, bsf, oracle.B_FP4, M, N, K, bias=bias,
+                                act=oracle.ACT_GELU)
+        tol = oracle.gemm_tolerance(ref, sabs, 1.0, np.abs(bf16_to_f64(bias))[None, :], None,
+                                    oracle.ACT_GELU)
+        assert_close(yv[i], ref, tol, f"batch {i}")
+
+
+# ------------------------------------------------------- full-size sampled --
+
+def test_fp8blk32_residual_full_size():
+    """FP8 E4M3 weights with 32x32 block scales, 1024 x 4096 x 4096, residual."""
+    run_sampled(Case(bq.W_FP8BLK32, 1024, 4096, 4096, seed=2, residual=True), n=3000)
+
+
+def test_square_mxfp8_full_size():
+    """Square MXFP8 x MXFP8 GEMM, 8192^3, alpha 1."""
+    run_sampled(Case(bq.W_MXFP8, 8192, 8192, 8192, seed=3), n=600)
+
+
+def test_down_projection_full_size():
+    """Down-projection 4096 x 1536 x 6144, MXFP4 weights."""
+    run_sampled(Case(bq.W_MXFP4, 4096, 1536, 6144, seed=4), n=3000)
+
+
+# ---------------------------------------------------------------- errors --
+
+def test_argument_errors():
+    c = Case(bq.W_MXFP4, 16, 128, 128)
+    aq, asf = bq.act_quant(to_dev_bf16(c.x))
+    bd = to_dev_u8(c.b)
+    bsf = bq.pack_weight_scales(to_dev_u8(c.bsf), bq.BQ_SF_ROW32, 128, 128)
+    with pytest.raises(bq.BqError) as e:  # N not a multiple of 8
+        bq.gemm(bq.W_MXFP4, aq, asf, bd, bsf, 16, 124, 128)
+    assert e.value.status == bq.BQ_ERR_SHAPE
+    with pytest.raises(bq.BqError) as e:  # FP4 weights need K % 128 == 0
+        bq.gemm(bq.W_MXFP4, aq, asf, bd, bsf, 16, 128, 96)
+    assert e.value.status == bq.BQ_ERR_SHAPE
+    with pytest.raises(bq.BqError) as e:  # split-K without a workspace
+        f = bq.lib().bq_gemm_mxfp8_mxfp4_epilogue
+        cfg = bq.config(split_k=2, swap_ab=1)
+        import ctypes
+        st = f(aq.data_ptr(), asf.data_ptr(), bd.data_ptr(), bsf.data_ptr(), 16, 128, 256,
+               torch.empty((16, 128), dtype=torch.bfloat16, device="cuda").data_ptr(), None, None,
+               None, 0, ctypes.byref(cfg), None)
+        bq._check(st, "split without workspace")
+    assert e.value.status in (bq.BQ_ERR_WORKSPACE, bq.BQ_ERR_SHAPE)
+    with pytest.raises(bq.BqError) as e:  # invalid enum
+        bq.gemm(bq.W_MXFP4, aq, asf, bd, bsf, 16, 128, 128, act=7)
+    assert e.value.status == bq.BQ_ERR_INVALID
+
+
+def test_pack_refuses_nan_scale_and_code():
+    s = np.full((64, 4), 127, np.uint8)
+    s[5, 2] = 255
+    with pytest.raises(bq.BqError) as e:
+        bq.pack_weight_scales(to_dev_u8(s), bq.BQ_SF_ROW32, 64, 128)
+    assert e.value.status == bq.BQ_ERR_NAN_SCALE
+    codes = np.zeros((64, 128), np.uint8)
+    codes[7, 99] = 0xFF
+    with pytest.raises(bq.BqError) as e:
+        bq.pack_weight_scales(to_dev_u8(np.full((2, 4), 127, np.uint8)), bq.BQ_SF_BLK32x32, 64,
+                              128, e4m3_codes=to_dev_u8(codes))
+    assert e.value.status == bq.BQ_ERR_NAN_CODE
+
+
+def test_pack_layout_blk32():
+    """BLK32x32 scales repeat over the 32 rows of their block; padding is 127."""
+    N, K = 100, 160
+    s = synth.uniform_bytes(((N + 31) // 32, K // 32), seed=1, lo=100, hi=140)
+    out = bq.pack_weight_scales(to_dev_u8(s), bq.BQ_SF_BLK32x32, N, K)
+    rows = bq.unpack_scales(out, N, K).cpu().numpy()
+    assert np.array_equal(rows, np.repeat(s, 32, axis=0)[:N])
