@@ -41,7 +41,8 @@ EXPORTS = (
     "bq_status_string", "bq_version", "bq_sf_bytes", "bq_act_quant", "bq_pack_weight_scales",
     "bq_unpack_scales", "bq_gemm_mxfp8_mxfp4", "bq_gemm_mxfp8_fp8blk32", "bq_gemm_mxfp8_mxfp8",
     "bq_gemm_workspace_bytes", "bq_gemm_mxfp8_mxfp4_epilogue", "bq_gemm_mxfp8_fp8blk32_epilogue",
-    "bq_gemm_mxfp8_mxfp8_epilogue", "bq_device_status", "bq_device_report",
+    "bq_gemm_mxfp8_mxfp8_epilogue", "bq_device_status", "bq_device_status_detail",
+    "bq_device_report",
 )
 
 
@@ -111,6 +112,8 @@ def lib():
         L.bq_gemm_workspace_bytes.restype = sz
         L.bq_device_status.argtypes = [vp]
         L.bq_device_status.restype = i32
+        L.bq_device_status_detail.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+        L.bq_device_status_detail.restype = i32
         L.bq_device_report.argtypes = [ctypes.c_char_p, sz]
         L.bq_device_report.restype = i32
         _lib = L
@@ -164,8 +167,11 @@ def device_report() -> str:
 
 def device_status():
     """Synchronizes the current stream; raises BqError(BQ_ERR_TIMEOUT) if a
-    kernel gave up on a barrier wait since the last check."""
-    _check(lib().bq_device_status(_stream()), "device status")
+    kernel gave up on a barrier wait since the last check (the message carries
+    the raw error word naming the wait site)."""
+    detail = ctypes.c_int(0)
+    st = lib().bq_device_status_detail(_stream(), ctypes.byref(detail))
+    _check(st, f"device status (detail 0x{detail.value:x})")
 
 
 # ----------------------------------------------------------- act_quant -----

@@ -51,46 +51,51 @@ __global__ void __launch_bounds__(256) act_quant_kernel(
   const int64_t g = static_cast<int64_t>(blockIdx.y) * 16 + (lane >> 1);  // this lane's group
   const int half = lane & 1;
 
+  // Every lane runs the shuffles below (full-warp masks); lanes without data
+  // (past the row's last group, or padding rows) carry zeros through them.
+  const bool active = row < M && g < G;
+  const int64_t col = g * 32 + half * 16;
+  uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+  if (active) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + row * ldx + col);
+    const uint4 v0 = __ldg(src);
+    const uint4 v1 = __ldg(src + 1);
+    w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+    w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+  }
+  // amax over |x| as an integer max of the magnitude bits (order-preserving
+  // for non-negative floats); non-finite detection from the exponent bits.
+  uint32_t mx = 0, bad = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t lo = w[i] & 0x7FFFu, hi = (w[i] >> 16) & 0x7FFFu;
+    mx = max(mx, max(lo, hi));
+    bad |= ((lo & 0x7F80u) == 0x7F80u) | ((hi & 0x7F80u) == 0x7F80u);
+  }
+  mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
   uint32_t sbyte = 127;
-  if (row < M) {
-    if (g < G) {
-      const int64_t col = g * 32 + half * 16;
-      const uint4 *src = reinterpret_cast<const uint4 *>(x + row * ldx + col);
-      const uint4 v0 = __ldg(src);
-      const uint4 v1 = __ldg(src + 1);
-      const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-      // amax over |x| as an integer max of the magnitude bits (order-preserving
-      // for non-negative floats); non-finite detection from the exponent bits.
-      uint32_t mx = 0, bad = 0;
+  if (active) {
+    if (bad && status) atomicOr(status, 1);
+    const float amax = fmaxf(__uint_as_float(mx << 16), 1e-4f);
+    const float t = __fmul_rn(amax, __uint_as_float(0x3B124925u));  // fp32(1/448)
+    const uint32_t tb = __float_as_uint(t);
+    const int e = static_cast<int>((tb >> 23) & 0xFFu) - 127 + ((tb & 0x7FFFFFu) != 0u ? 1 : 0);
+    sbyte = static_cast<uint32_t>(e + 127);
+    const float inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e
+    float f[16];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint32_t lo = w[i] & 0x7FFFu, hi = (w[i] >> 16) & 0x7FFFu;
-        mx = max(mx, max(lo, hi));
-        bad |= ((lo & 0x7F80u) == 0x7F80u) | ((hi & 0x7F80u) == 0x7F80u);
-      }
-      mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
-      if (bad && status) atomicOr(status, 1);
-      const float amax = fmaxf(__uint_as_float(mx << 16), 1e-4f);
-      const float t = __fmul_rn(amax, __uint_as_float(0x3B124925u));  // fp32(1/448)
-      const uint32_t tb = __float_as_uint(t);
-      const int e = static_cast<int>((tb >> 23) & 0xFFu) - 127 + ((tb & 0x7FFFFFu) != 0u ? 1 : 0);
-      sbyte = static_cast<uint32_t>(e + 127);
-      const float inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e
-      float f[16];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        f[2 * i] = fminf(fmaxf(__fmul_rn(__uint_as_float(w[i] << 16), inv), -448.0f), 448.0f);
-        f[2 * i + 1] =
-            fminf(fmaxf(__fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), inv), -448.0f), 448.0f);
-      }
-      uint4 out;
-      out.x = e4m3x4(f[0], f[1], f[2], f[3]);
-      out.y = e4m3x4(f[4], f[5], f[6], f[7]);
-      out.z = e4m3x4(f[8], f[9], f[10], f[11]);
-      out.w = e4m3x4(f[12], f[13], f[14], f[15]);
-      *reinterpret_cast<uint4 *>(q + row * K + col) = out;
-      if (sf_row && half == 0) sf_row[row * G + g] = static_cast<uint8_t>(sbyte);
+    for (int i = 0; i < 8; ++i) {
+      f[2 * i] = fminf(fmaxf(__fmul_rn(__uint_as_float(w[i] << 16), inv), -448.0f), 448.0f);
+      f[2 * i + 1] =
+          fminf(fmaxf(__fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), inv), -448.0f), 448.0f);
     }
+    uint4 out;
+    out.x = e4m3x4(f[0], f[1], f[2], f[3]);
+    out.y = e4m3x4(f[4], f[5], f[6], f[7]);
+    out.z = e4m3x4(f[8], f[9], f[10], f[11]);
+    out.w = e4m3x4(f[12], f[13], f[14], f[15]);
+    *reinterpret_cast<uint4 *>(q + row * K + col) = out;
+    if (sf_row && half == 0) sf_row[row * G + g] = static_cast<uint8_t>(sbyte);
   }
   // Gather the bytes of groups 4j..4j+3 of this chunk (lanes 8j, 8j+2, 8j+4,
   // 8j+6) and store them as one word; groups past G (column padding) and rows

@@ -124,6 +124,9 @@ struct Plan {
 
 int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
+constexpr int64_t kMaxSplitTiles = 16384;                       // output tiles of a split-K call
+constexpr size_t kTicketRegion = kMaxSplitTiles * sizeof(int);  // 64 KiB
+
 int make_plan(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_config* cfg,
               int num_sms, Plan* p) {
   const int req_bn = cfg ? cfg->block_n : 0;
@@ -163,15 +166,19 @@ int make_plan(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_conf
   p->units = tiles * p->splits;
   if (p->units > 0x7FFFFFFF) return BQ_ERR_SHAPE;
   if (p->splits > 1) {
+    if (tiles > kMaxSplitTiles) return BQ_ERR_SHAPE;
     p->ws_partial = static_cast<size_t>(p->units) * 128 * p->bn * sizeof(float);
     p->ws_ticket = static_cast<size_t>(tiles) * sizeof(int);
   }
   return BQ_OK;
 }
 
+// Split-K workspace: a fixed region of per-tile tickets at the start (the
+// same bytes for every problem, so a call never finds another call's partial
+// sums where it expects zeroed tickets), then the fp32 partial tiles.
 size_t plan_ws_bytes(const Plan& p) {
   if (p.splits <= 1) return 0;
-  return ((p.ws_partial + 255) & ~static_cast<size_t>(255)) + p.ws_ticket;
+  return kTicketRegion + p.ws_partial;
 }
 
 // --------------------------------------------------------------- launches --
@@ -308,9 +315,8 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
   g.alpha = epi ? epi->alpha : 1.0f;
   g.act = epi ? epi->act : BQ_ACT_NONE;
   if (pl.splits > 1) {
-    g.ws_partial = static_cast<float*>(ws);
-    g.ws_ticket = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) +
-                                         ((pl.ws_partial + 255) & ~static_cast<size_t>(255)));
+    g.ws_ticket = static_cast<int*>(ws);
+    g.ws_partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kTicketRegion);
   }
   g.err = dev->err_ptr;
   const CUtensorMap& tp = pl.swap ? map_b : map_a;
@@ -484,7 +490,7 @@ int bq_gemm_mxfp8_mxfp8_epilogue(const void* a_q, const void* a_sf, const void* 
                     workspace_bytes, cfg, stream);
 }
 
-int bq_device_status(bq_stream_t stream) {
+int bq_device_status_detail(bq_stream_t stream, int* detail) {
   DevInfo* dev = nullptr;
   int st = current_device(&dev);
   if (st != BQ_OK) return st;
@@ -495,8 +501,11 @@ int bq_device_status(bq_stream_t stream) {
       cudaMemsetAsync(dev->err_ptr, 0, sizeof(int), s) != cudaSuccess ||
       cudaStreamSynchronize(s) != cudaSuccess)
     return BQ_ERR_CUDA;
+  if (detail) *detail = err;
   return err ? BQ_ERR_TIMEOUT : BQ_OK;
 }
+
+int bq_device_status(bq_stream_t stream) { return bq_device_status_detail(stream, nullptr); }
 
 int bq_device_report(char* buf, size_t n) {
   if (!buf || n == 0) return BQ_ERR_NULL;

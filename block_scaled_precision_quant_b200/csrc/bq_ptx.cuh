@@ -8,6 +8,8 @@
 #include <cuda.h>
 #include <stdint.h>
 
+// Device error word: 0 = fine; otherwise BQ_DEV_ERR_TIMEOUT | (site << 8) of
+// the first wait that gave up.
 #define BQ_DEV_ERR_TIMEOUT 1
 
 #ifndef BQ_WAIT_NS
@@ -15,6 +17,15 @@
 #endif
 
 namespace bq {
+
+// Wait sites reported in the device error word.
+enum WaitSite : int {
+  kWaitProdEmpty = 1,      // producer waiting for a free stage
+  kWaitMmaTmemEmpty = 2,   // MMA issuer waiting for a drained accumulator
+  kWaitMmaFull = 3,        // MMA issuer waiting for a loaded stage
+  kWaitEpiFull = 4,        // epilogue waiting for a finished accumulator
+  kWaitDrain = 5,          // MMA issuer draining before teardown
+};
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -62,7 +73,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // up after BQ_WAIT_NS (or as soon as *abort is set by another role), records
 // the timeout in *err and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err,
-                                          volatile int *abort) {
+                                          volatile int *abort, int site) {
   const uint32_t b = smem_u32(bar);
   if (mbar_try_wait(b, parity)) return true;
   const uint64_t t0 = globaltimer();
@@ -73,19 +84,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *e
     if (*abort) return false;
     if (globaltimer() - t0 > BQ_WAIT_NS) {
       *abort = 1;
-      if (err) atomicExch(err, BQ_DEV_ERR_TIMEOUT);
+      if (err) atomicCAS(err, 0, BQ_DEV_ERR_TIMEOUT | (site << 8));
       return false;
     }
   }
 }
 
 // Bounded wait that ignores the abort flag (used to drain before teardown).
-__device__ __forceinline__ bool mbar_wait_timed(uint64_t *bar, uint32_t parity, int *err) {
+__device__ __forceinline__ bool mbar_wait_timed(uint64_t *bar, uint32_t parity, int *err,
+                                                int site) {
   const uint32_t b = smem_u32(bar);
   const uint64_t t0 = globaltimer();
   while (!mbar_try_wait(b, parity)) {
     if (globaltimer() - t0 > BQ_WAIT_NS) {
-      if (err) atomicExch(err, BQ_DEV_ERR_TIMEOUT);
+      if (err) atomicCAS(err, 0, BQ_DEV_ERR_TIMEOUT | (site << 8));
       return false;
     }
   }

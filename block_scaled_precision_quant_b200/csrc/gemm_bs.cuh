@@ -83,7 +83,6 @@ struct GemmSmem {
   static constexpr int kSfCols = 4 + kSfqCols;  // TMEM columns of scales per stage
   static constexpr int kBytesP = kBlockP * kBlockK;
   static constexpr int kBytesQ = BN * kBlockK;
-  static constexpr int kStageBytes = kBytesP + kBytesQ + kSfAtom + kSfqAtoms * kSfAtom;
   static constexpr int kOffQ = STAGES * kBytesP;
   static constexpr int kOffSfp = kOffQ + STAGES * kBytesQ;
   static constexpr int kOffSfq = kOffSfp + STAGES * kSfAtom;
@@ -255,6 +254,12 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   const int total_units = a.batch * a.tiles_p * a.tiles_q * a.splits;
+  // Transaction bytes of one stage.  A 4-bit operand lands in shared memory
+  // with one byte-slot per code, but the transaction count is the packed size
+  // (half the footprint).
+  constexpr uint32_t kTxBytes = (P_FP4 ? L::kBytesP / 2 : L::kBytesP) +
+                                (Q_FP4 ? L::kBytesQ / 2 : L::kBytesQ) + kSfAtom +
+                                L::kSfqAtoms * kSfAtom;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
@@ -273,11 +278,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const uint8_t *sfq = a.sf_q + b * a.sf_q_bstride +
                              static_cast<int64_t>(q_row0 / 128) * a.sf_katoms * kSfAtom;
         for (int kt = kt0; kt < kt1; ++kt) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, a.err, abort_flag)) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, a.err, abort_flag, kWaitProdEmpty)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
+          mbar_arrive_expect_tx(&full[stage], kTxBytes);
           const int kx = kt * kBlockK;
           if (a.p_batched)
             tma_load_3d(s_p + stage * L::kBytesP, &tm_p, &full[stage], kx, tp * kBlockP, b);
@@ -322,11 +327,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const int kt0 = split * a.kt_per_split;
         const int kt1 = min(a.kt_total, kt0 + a.kt_per_split);
         const uint32_t sfq_row_off = static_cast<uint32_t>((tq * BN) % 128) / 32;
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, a.err, abort_flag)) break;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, a.err, abort_flag, kWaitMmaTmemEmpty)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kt = kt0; kt < kt1; ++kt) {
-          if (!mbar_wait(&full[stage], phase, a.err, abort_flag)) {
+          if (!mbar_wait(&full[stage], phase, a.err, abort_flag, kWaitMmaFull)) {
             ok = false;
             break;
           }
@@ -363,7 +368,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       // Wait until every MMA this thread issued has completed before the
       // TMEM is released (bounded; after an abort also give them time).
       tc_commit(drain);
-      if (!mbar_wait_timed(drain, 0, a.err)) sleep_ns(200000);
+      if (!mbar_wait_timed(drain, 0, a.err, kWaitDrain)) sleep_ns(200000);
     }
   } else {
     // ------------------------------------------------------------ epilogue --
@@ -375,7 +380,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     for (int unit = blockIdx.x; unit < total_units; unit += gridDim.x) {
       int b, tp, tq, split, tile;
       decode_unit(a, unit, b, tp, tq, split, tile);
-      if (!mbar_wait(&tfull[acc], acc_phase, a.err, abort_flag)) break;
+      __syncwarp();
+      if (!mbar_wait(&tfull[acc], acc_phase, a.err, abort_flag, kWaitEpiFull)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + acc * BN + (static_cast<uint32_t>(quad * 32) << 16);
       const int prow = tp * kBlockP + row;
@@ -383,6 +389,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t v[32];
+          __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the stores
           tmem_ld_32x32b_x32(t_row + c * 32, v);
           tmem_ld_wait();
           float f[32];
@@ -400,6 +407,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t v[32];
+          __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the stores
           tmem_ld_32x32b_x32(t_row + c * 32, v);
           tmem_ld_wait();
 #pragma unroll
@@ -412,12 +420,14 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[acc]);
         __threadfence();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        __syncwarp();
+        asm volatile("barrier.sync 1, 128;" ::: "memory");
         if (epi_tid == 0) {
           const int prev = atomicAdd(&a.ws_ticket[tile], 1);
           *last_flag = (prev == a.splits - 1);
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        __syncwarp();
+        asm volatile("barrier.sync 1, 128;" ::: "memory");
         if (*last_flag) {
           __threadfence();
           const float *base =
@@ -442,7 +452,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           }
           if (epi_tid == 0) a.ws_ticket[tile] = 0;  // ready for the next call
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        __syncwarp();
+        asm volatile("barrier.sync 1, 128;" ::: "memory");
       }
       if (++acc == ACC) {
         acc = 0;

@@ -195,8 +195,11 @@ size_t bq_gemm_workspace_bytes(int weight_kind, int64_t M, int64_t N, int64_t K,
 /* GEMM + fused epilogue (+ optional batch).  epi NULL = plain (alpha 1, no
  * bias, residual or activation).  batch NULL = one problem.  workspace: device
  * memory of at least bq_gemm_workspace_bytes(...) bytes (may be NULL when that
- * is 0); the call leaves it ready for the next call, and calls that share one
- * workspace must not overlap on the GPU. */
+ * is 0), 16-byte aligned.  Its first 64 KiB hold per-tile counters that must be
+ * zero before the first use (e.g. a zero-filled allocation); every call that
+ * completes leaves them zero again, so one workspace serves any sequence of
+ * problems.  Calls that share one workspace must not overlap on the GPU.  A
+ * split-K schedule is limited to 16384 output tiles (else BQ_ERR_SHAPE). */
 int bq_gemm_mxfp8_mxfp4_epilogue(const void *a_q, const void *a_sf, const void *b_fp4,
                                  const void *b_sf, int64_t M, int64_t N, int64_t K, void *y_bf16,
                                  const bq_epilogue *epi, const bq_batch *batch, void *workspace,
@@ -219,6 +222,12 @@ int bq_gemm_mxfp8_mxfp8_epilogue(const void *a_q, const void *a_sf, const void *
  * SYNCHRONIZES `stream`.  Returns BQ_OK, or BQ_ERR_TIMEOUT when a kernel gave
  * up on a barrier wait since the last call (its outputs are then invalid). */
 int bq_device_status(bq_stream_t stream);
+
+/* bq_device_status, also returning the raw error word in *detail (may be
+ * NULL): 0, or 1 | (site << 8) where site names the first wait that gave up
+ * (1 producer/free stage, 2 MMA/free accumulator, 3 MMA/loaded stage,
+ * 4 epilogue/finished accumulator, 5 teardown drain).  SYNCHRONIZES. */
+int bq_device_status_detail(bq_stream_t stream, int *detail);
 
 /* Writes a one-line report of the current device (name, compute capability,
  * SM count, L2 size, clocks) into buf (always NUL-terminated). */

@@ -1,0 +1,61 @@
+"""Host-side logic of bench.py: algorithmic byte/flop counts, the multi-rank
+timing reduction (2 gloo ranks on CPU) and the reference arm's rank handling."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+
+def test_decode_algorithmic_bytes():
+    # weights 4.25 bits/weight + activations + bias + bf16 output (MB)
+    got = [bench.gemm_bytes(sp) / 1e6 for sp in bench.WORKLOADS["decode"]["layers"]]
+    assert [round(g, 2) for g in got] == [4.21, 5.59, 5.4]
+    assert bench.gemm_flops(bench.WORKLOADS["decode"]["layers"][0]) == 2.0 * 41 * 4608 * 1536
+
+
+def test_act_quant_bytes_per_element():
+    assert bench.act_quant_bytes(("x", "mxfp4", 1, 0, 32, 1, {})) == 32 * 3.03125
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    bench.init_dist(world, "gloo")
+    bench.barrier(world)
+    m = bench.reduce_max(10.0 + rank, world)
+    bench.barrier(world)
+    import torch.distributed as dist
+    dist.destroy_process_group()
+    q.put((rank, m))
+
+
+def test_reduce_max_over_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = dict(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert out == {0: 11.0, 1: 11.0}
+
+
+def test_reference_arm_other_ranks_do_nothing(capsys, monkeypatch):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"]) == 0
+    assert capsys.readouterr().out == ""

@@ -52,6 +52,9 @@ class Case:
         self.res = synth.residual(M, N, seed=seed + 300) if residual else None
 
     def gpu(self, config=None, batch=None):
+        return self.gpu_with(config=config)
+
+    def gpu_with(self, config=None, workspace=None):
         xd = to_dev_bf16(self.x)
         aq, asf = bq.act_quant(xd)
         bd = to_dev_u8(self.b)
@@ -61,7 +64,7 @@ class Case:
         y = bq.gemm(self.wk, aq, asf, bd, bsf, self.M, self.N, self.K,
                     bias=to_dev_bf16(self.bias) if self.bias is not None else None,
                     residual=to_dev_bf16(self.res) if self.res is not None else None,
-                    alpha=self.alpha, act=self.act, config=config)
+                    alpha=self.alpha, act=self.act, config=config, workspace=workspace)
         bq.device_status()
         self.aq_gpu = aq.cpu().numpy()
         return bf16_to_f64(y.cpu().view(torch.int16).numpy().view(np.uint16))
@@ -287,3 +290,18 @@ def test_pack_layout_blk32():
     out = bq.pack_weight_scales(to_dev_u8(s), bq.BQ_SF_BLK32x32, N, K)
     rows = bq.unpack_scales(out, N, K).cpu().numpy()
     assert np.array_equal(rows, np.repeat(s, 32, axis=0)[:N])
+
+
+def test_workspace_shared_across_problems():
+    """One workspace serves a sequence of split-K problems of different
+    shapes; the ticket region is zero again after every call."""
+    shapes = [(41, 640, 1536, 5), (17, 1536, 6144, 12), (64, 384, 1024, 3), (5, 4608, 1536, 4)]
+    need = max(bq.workspace_bytes(bq.W_MXFP4, M, N, K, 1, bq.config(split_k=s, swap_ab=1))
+               for M, N, K, s in shapes)
+    ws = torch.zeros((need,), dtype=torch.uint8, device="cuda")
+    for i, (M, N, K, s) in enumerate(shapes * 2):
+        c = Case(bq.W_MXFP4, M, N, K, seed=60 + i, bias=True)
+        y = c.gpu_with(config=bq.config(split_k=s, swap_ab=1), workspace=ws)
+        ref, sabs = c.oracle_full()
+        assert_close(y, ref, c.tol(ref, sabs), f"shared workspace {M}x{N}x{K}/{s}")
+        assert int(ws[:65536].count_nonzero().item()) == 0
