@@ -472,6 +472,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-run", type=int, default=0, metavar="R",
+                    help="no timing: build one input set and run every layer's step R "
+                         "times eagerly (for ncu captures of single launches)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
@@ -497,6 +500,17 @@ def main(argv=None):
 def run_ours(args, spec, world, rank, local, device):
     import torch
     import block_scaled_precision_quant_b200 as bq
+
+    if args.profile_run:
+        layers = [Layer(sp, 1, 11 * (i + 1), device) for i, sp in enumerate(spec["layers"])]
+        for _ in range(args.profile_run):
+            for L in layers:
+                L.launches(0)
+        torch.cuda.synchronize()
+        bq.device_status()
+        if rank == 0:
+            print(json.dumps({"profile_run": args.profile_run, "workload": spec["desc"]}))
+        return 0
 
     layers_spec = spec["layers"]
     l2 = torch.cuda.get_device_properties(device).L2_cache_size

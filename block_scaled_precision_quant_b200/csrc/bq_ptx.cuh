@@ -71,15 +71,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Wait until the phase with the given parity of `bar` has completed.  Gives
 // up after BQ_WAIT_NS (or as soon as *abort is set by another role), records
-// the timeout in *err and returns false.
+// the wait site in *err and returns false.  The timer is only read after
+// many failed polls, so ordinary waits never touch it.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err,
                                           volatile int *abort, int site) {
   const uint32_t b = smem_u32(bar);
-  if (mbar_try_wait(b, parity)) return true;
+#pragma unroll 1
+  for (int i = 0; i < 4096; ++i)
+    if (mbar_try_wait(b, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
 #pragma unroll 1
-    for (int i = 0; i < 32; ++i)
+    for (int i = 0; i < 256; ++i)
       if (mbar_try_wait(b, parity)) return true;
     if (*abort) return false;
     if (globaltimer() - t0 > BQ_WAIT_NS) {
@@ -94,6 +97,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *e
 __device__ __forceinline__ bool mbar_wait_timed(uint64_t *bar, uint32_t parity, int *err,
                                                 int site) {
   const uint32_t b = smem_u32(bar);
+#pragma unroll 1
+  for (int i = 0; i < 4096; ++i)
+    if (mbar_try_wait(b, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (!mbar_try_wait(b, parity)) {
     if (globaltimer() - t0 > BQ_WAIT_NS) {
