@@ -42,7 +42,7 @@ EXPORTS = (
     "bq_unpack_scales", "bq_gemm_mxfp8_mxfp4", "bq_gemm_mxfp8_fp8blk32", "bq_gemm_mxfp8_mxfp8",
     "bq_gemm_workspace_bytes", "bq_gemm_mxfp8_mxfp4_epilogue", "bq_gemm_mxfp8_fp8blk32_epilogue",
     "bq_gemm_mxfp8_mxfp8_epilogue", "bq_device_status", "bq_device_status_detail",
-    "bq_device_report",
+    "bq_device_report", "bq_gemm_mxfp8_mxfp4_epilogue_noalloc", "bq_noalloc_scratch_bytes",
 )
 
 
@@ -108,6 +108,11 @@ def lib():
             f.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, ctypes.POINTER(Epilogue),
                           ctypes.POINTER(Batch), vp, sz, ctypes.POINTER(GemmConfig), vp]
             f.restype = i32
+        L.bq_gemm_mxfp8_mxfp4_epilogue_noalloc.argtypes = [
+            vp, vp, vp, vp, i64, i64, i64, vp, ctypes.POINTER(Epilogue), ctypes.POINTER(Batch),
+            ctypes.POINTER(GemmConfig), vp]
+        L.bq_gemm_mxfp8_mxfp4_epilogue_noalloc.restype = i32
+        L.bq_noalloc_scratch_bytes.restype = sz
         L.bq_gemm_workspace_bytes.argtypes = [i32, i64, i64, i64, i64, ctypes.POINTER(GemmConfig)]
         L.bq_gemm_workspace_bytes.restype = sz
         L.bq_device_status.argtypes = [vp]

@@ -472,6 +472,37 @@ int bq_gemm_mxfp8_mxfp4_epilogue(const void* a_q, const void* a_sf, const void* 
                     workspace_bytes, cfg, stream);
 }
 
+// ------------------------------------------------ allocation-free variant --
+//
+// For callers that cannot allocate device memory themselves -- an inference
+// plugin that is handed only its input and output buffers, or a latency-bound
+// serving loop whose memory is fixed when it starts -- this entry point runs
+// the MXFP4-weight GEMM (with its K-split schedule) against a scratch area the
+// library owns: a fixed-size array in the module's global memory, created
+// when the library is loaded on a device and kept until the process exits.
+
+constexpr size_t kNoAllocScratchBytes = 8u << 20;  // 8 MiB per device
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on each device, looked up once per device
+// (with that device current).  In host code the array's name is only a
+// host-side stand-in, never a device address.
+static void* g_noalloc_ptr[kMaxDevices] = {};
+
+static int noalloc_scratch(void** ptr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return BQ_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *ptr = g_noalloc_ptr[dev];
+  return BQ_OK;
+}
+
 int bq_gemm_mxfp8_fp8blk32_epilogue(const void* a_q, const void* a_sf, const void* b_e4m3,
                                     const void* b_sf, int64_t M, int64_t N, int64_t K,
                                     void* y_bf16, const bq_epilogue* epi, const bq_batch* batch,
@@ -489,6 +520,38 @@ int bq_gemm_mxfp8_mxfp8_epilogue(const void* a_q, const void* a_sf, const void* 
   return gemm_entry(kMxfp8, a_q, a_sf, b_e4m3, b_sf, M, N, K, y_bf16, epi, batch, workspace,
                     workspace_bytes, cfg, stream);
 }
+
+int bq_gemm_mxfp8_mxfp4_epilogue_noalloc(const void* a_q, const void* a_sf, const void* b_fp4,
+                                         const void* b_sf, int64_t M, int64_t N, int64_t K,
+                                         void* y_bf16, const bq_epilogue* epi,
+                                         const bq_batch* batch, const bq_gemm_config* cfg,
+                                         bq_stream_t stream) {
+  DevInfo* dev = nullptr;
+  int st = current_device(&dev);
+  if (st != BQ_OK) return st;
+  const int64_t count = batch ? batch->count : 1;
+  if (M < 0 || N < 0 || K <= 0 || K % 32 != 0 || count < 0) return BQ_ERR_SHAPE;
+  if (M == 0 || N == 0 || count == 0) return BQ_OK;
+  Plan pl;
+  st = make_plan(M, N, K, count, cfg, dev->num_sms, &pl);
+  if (st != BQ_OK) return st;
+  const size_t need = plan_ws_bytes(pl);
+  if (need > kNoAllocScratchBytes) return BQ_ERR_WORKSPACE;  // problem too large for the scratch
+  void* scratch = nullptr;
+  if (need > 0) {
+    st = noalloc_scratch(&scratch);
+    if (st != BQ_OK) return st;
+    // The scratch keeps whatever the previous call left: zero this call's
+    // ticket counters before the kernel reads them.
+    if (cudaMemsetAsync(scratch, 0, pl.ws_ticket, reinterpret_cast<cudaStream_t>(stream)) !=
+        cudaSuccess)
+      return BQ_ERR_CUDA;
+  }
+  return gemm_entry(kMxfp4, a_q, a_sf, b_fp4, b_sf, M, N, K, y_bf16, epi, batch, scratch,
+                    need > 0 ? kNoAllocScratchBytes : 0, cfg, stream);
+}
+
+size_t bq_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
 
 int bq_device_status_detail(bq_stream_t stream, int* detail) {
   DevInfo* dev = nullptr;

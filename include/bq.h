@@ -216,6 +216,36 @@ int bq_gemm_mxfp8_mxfp8_epilogue(const void *a_q, const void *a_sf, const void *
                                  size_t workspace_bytes, const bq_gemm_config *cfg,
                                  bq_stream_t stream);
 
+/* ---- allocation-free GEMM -------------------------------------------------
+ *
+ * No counterpart on the pages: this is a library convenience.
+ *
+ * bq_gemm_mxfp8_mxfp4_epilogue_noalloc -- the same computation, arguments and
+ * errors as bq_gemm_mxfp8_mxfp4_epilogue, for callers that cannot allocate
+ * device memory (for example a plugin inside another runtime that is given only
+ * its input and output buffers, or a serving loop whose memory is fixed at
+ * start-up).  Instead of a caller-provided workspace, the K-split schedule uses
+ * scratch memory the library owns: one array of bq_noalloc_scratch_bytes()
+ * bytes (8 MiB) in global memory on every device that loads the library, held
+ * until the process exits.  The call allocates nothing (no cudaMalloc or
+ * allocating library routine).
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any stream
+ *     capture.
+ *   - Every call clears the counters it needs on its stream before the kernel;
+ *     all calls share the one array, so calls that overlap on the GPU (other
+ *     streams, other host threads) race -- serialize them.
+ *   - A problem whose schedule needs more scratch than the array holds returns
+ *     BQ_ERR_WORKSPACE without launching (use the workspace variant instead). */
+int bq_gemm_mxfp8_mxfp4_epilogue_noalloc(const void *a_q, const void *a_sf, const void *b_fp4,
+                                         const void *b_sf, int64_t M, int64_t N, int64_t K,
+                                         void *y_bf16, const bq_epilogue *epi,
+                                         const bq_batch *batch, const bq_gemm_config *cfg,
+                                         bq_stream_t stream);
+
+/* Size in bytes of the library-owned scratch array used by the _noalloc call. */
+size_t bq_noalloc_scratch_bytes(void);
+
 /* ---- diagnostics -------------------------------------------------------- */
 
 /* Reads and clears the library's device error word on the current device.

@@ -1,0 +1,85 @@
+"""The allocation-free GEMM entry point (bq_gemm_mxfp8_mxfp4_epilogue_noalloc).
+
+Some callers cannot allocate device memory (a plugin given only its inputs and
+outputs, a serving loop with a fixed memory budget); this entry point runs the
+K-split MXFP4 GEMM on a scratch array the library owns.  The test calls it
+through the C ABI twice in a row (the second call finds the first call's
+leftovers in the shared scratch) and compares each result with the existing
+workspace entry point, within the tolerance the parity tests use.  The file is
+named to be collected last; it passes on its own in a fresh process too.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import block_scaled_precision_quant_b200 as bq
+from block_scaled_precision_quant_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev_bf16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def _f64(y):
+    return (y.cpu().view(torch.int16).numpy().view(np.uint16).astype(np.uint32) << 16) \
+        .view(np.float32).astype(np.float64)
+
+
+def test_noalloc_matches_workspace_entry_twice():
+    L = bq.lib()
+    M, N, K = 41, 4608, 1536
+    cfg = bq.config(split_k=4, swap_ab=1)
+    need = bq.workspace_bytes(bq.W_MXFP4, M, N, K, 1, cfg)
+    assert 0 < need <= L.bq_noalloc_scratch_bytes()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for call in range(2):
+        x = synth.activations(M, K, seed=70 + call)
+        w, ws = synth.mxfp4_weight(N, K, seed=80 + call)
+        bias = synth.bias(N, seed=90 + call)
+        aq, asf = bq.act_quant(_dev_bf16(x))
+        wd = torch.from_numpy(w).cuda()
+        wsf = bq.pack_weight_scales(torch.from_numpy(ws).cuda(), bq.BQ_SF_ROW32, N, K)
+        bd = _dev_bf16(bias)
+        epi = bq.Epilogue(bd.data_ptr(), None, 0, 1.0, bq.BQ_ACT_NONE)
+
+        y_new = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        st = L.bq_gemm_mxfp8_mxfp4_epilogue_noalloc(
+            aq.data_ptr(), asf.data_ptr(), wd.data_ptr(), wsf.data_ptr(), M, N, K,
+            y_new.data_ptr(), ctypes.byref(epi), None, ctypes.byref(cfg), stream)
+        assert st == bq.BQ_OK, bq.status_string(st)
+
+        work = torch.zeros((need,), dtype=torch.uint8, device="cuda")
+        y_old = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        st = L.bq_gemm_mxfp8_mxfp4_epilogue(
+            aq.data_ptr(), asf.data_ptr(), wd.data_ptr(), wsf.data_ptr(), M, N, K,
+            y_old.data_ptr(), ctypes.byref(epi), None, work.data_ptr(), need,
+            ctypes.byref(cfg), stream)
+        assert st == bq.BQ_OK, bq.status_string(st)
+        bq.device_status()
+
+        q, s = oracle.act_quant(x)
+        _, sabs = oracle.gemm(q, s, w, ws, oracle.B_FP4, M, N, K, bias=bias)
+        old = _f64(y_old)
+        babs = np.abs((bias.astype(np.uint32) << 16).view(np.float32).astype(np.float64))
+        tol = oracle.gemm_tolerance(old, sabs, 1.0, babs[None, :])
+        new = _f64(y_new)
+        assert np.all(np.isfinite(new))
+        assert np.all(np.abs(new - old) <= tol), f"call {call}"
+
+
+def test_noalloc_rejects_problems_beyond_the_scratch():
+    L = bq.lib()
+    M, N, K = 64, 16384, 4096
+    cfg = bq.config(split_k=16, swap_ab=1)
+    assert bq.workspace_bytes(bq.W_MXFP4, M, N, K, 1, cfg) > L.bq_noalloc_scratch_bytes()
+    dummy = torch.zeros((1 << 20,), dtype=torch.uint8, device="cuda")
+    st = L.bq_gemm_mxfp8_mxfp4_epilogue_noalloc(
+        dummy.data_ptr(), dummy.data_ptr(), dummy.data_ptr(), dummy.data_ptr(), M, N, K,
+        dummy.data_ptr(), None, None, ctypes.byref(cfg),
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == bq.BQ_ERR_WORKSPACE
