@@ -35,6 +35,7 @@ BQ_SF_ROW32 = 0
 BQ_SF_BLK32x32 = 1
 BQ_ACT_NONE = 0
 BQ_ACT_GELU = 1
+BQ_SPLIT_AUTO, BQ_SPLIT_WORKSPACE, BQ_SPLIT_CLUSTER = 0, 1, 2
 W_MXFP4, W_FP8BLK32, W_MXFP8 = 0, 1, 2
 
 EXPORTS = (
@@ -67,7 +68,7 @@ class Batch(ctypes.Structure):
 
 class GemmConfig(ctypes.Structure):
     _fields_ = [("block_n", ctypes.c_int), ("split_k", ctypes.c_int), ("swap_ab", ctypes.c_int),
-                ("reserved", ctypes.c_int)]
+                ("split_mode", ctypes.c_int), ("k_chunks", ctypes.c_int)]
 
 
 _lib = None
@@ -230,8 +231,8 @@ _ENTRY = {W_MXFP4: "bq_gemm_mxfp8_mxfp4", W_FP8BLK32: "bq_gemm_mxfp8_fp8blk32",
           W_MXFP8: "bq_gemm_mxfp8_mxfp8"}
 
 
-def _config(block_n=0, split_k=0, swap_ab=-1):
-    return GemmConfig(int(block_n), int(split_k), int(swap_ab), 0)
+def _config(block_n=0, split_k=0, swap_ab=-1, split_mode=0, k_chunks=0):
+    return GemmConfig(int(block_n), int(split_k), int(swap_ab), int(split_mode), int(k_chunks))
 
 
 def workspace_bytes(weight_kind, M, N, K, batch=1, config=None) -> int:

@@ -21,6 +21,8 @@
 #include <cuda_fp8.h>
 #include <stdint.h>
 
+#include "bq_ptx.cuh"
+
 namespace bq {
 
 // Byte offset of scale (row r, column c) in an MMA-layout buffer with
@@ -56,6 +58,10 @@ __global__ void __launch_bounds__(256) act_quant_kernel(
   const bool active = row < M && g < G;
   const int64_t col = g * 32 + half * 16;
   uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+  // Programmatic dependent launch: x may come from the kernel before this one;
+  // the kernel after this one (the GEMM) may begin its prologue now.
+  griddep_wait();
+  griddep_launch_dependents();
   if (active) {
     const uint4 *src = reinterpret_cast<const uint4 *>(x + row * ldx + col);
     const uint4 v0 = __ldg(src);

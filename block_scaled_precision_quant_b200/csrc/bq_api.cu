@@ -90,15 +90,41 @@ int get_encoder() {
 // 128B swizzle, zero fill outside the tensor.  fp4 selects the 4-bit type that
 // TMA expands to one byte-slot per code in shared memory (8 data bytes then 8
 // padding bytes per 16 codes), the operand layout kind::mxf8f6f4 reads.
+// With kc > 1 (K % 128 == 0) K is viewed as (128 codes, K/128 chunks) so one
+// box of {128, box_rows, kc} brings kc consecutive 128-K chunks, each landing
+// as its own 128B-swizzled [box_rows][128 B] tile.
 int make_operand_map(CUtensorMap* m, const void* base, bool fp4, int64_t K, int64_t rows,
-                     int64_t row_bytes, int64_t batch, int64_t batch_bytes, int box_rows) {
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows),
-                        static_cast<cuuint64_t>(batch)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_bytes),
-                           static_cast<cuuint64_t>(batch_bytes)};
-  cuuint32_t box[3] = {128u, static_cast<cuuint32_t>(box_rows), 1u};
-  cuuint32_t estr[3] = {1u, 1u, 1u};
-  const cuuint32_t rank = batch > 1 ? 3 : 2;
+                     int64_t row_bytes, int64_t batch, int64_t batch_bytes, int box_rows,
+                     int kc) {
+  cuuint64_t dims[4];
+  cuuint64_t strides[3];
+  cuuint32_t box[4];
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  cuuint32_t rank;
+  if (kc <= 1) {
+    dims[0] = static_cast<cuuint64_t>(K);
+    dims[1] = static_cast<cuuint64_t>(rows);
+    dims[2] = static_cast<cuuint64_t>(batch);
+    strides[0] = static_cast<cuuint64_t>(row_bytes);
+    strides[1] = static_cast<cuuint64_t>(batch_bytes);
+    box[0] = 128u;
+    box[1] = static_cast<cuuint32_t>(box_rows);
+    box[2] = 1u;
+    rank = batch > 1 ? 3 : 2;
+  } else {
+    dims[0] = 128;
+    dims[1] = static_cast<cuuint64_t>(rows);
+    dims[2] = static_cast<cuuint64_t>(K / 128);
+    dims[3] = static_cast<cuuint64_t>(batch);
+    strides[0] = static_cast<cuuint64_t>(row_bytes);
+    strides[1] = fp4 ? 64u : 128u;  // bytes per 128-code chunk
+    strides[2] = static_cast<cuuint64_t>(batch_bytes);
+    box[0] = 128u;
+    box[1] = static_cast<cuuint32_t>(box_rows);
+    box[2] = static_cast<cuuint32_t>(kc);
+    box[3] = 1u;
+    rank = batch > 1 ? 4 : 3;
+  }
   CUresult r = g_encode(m,
                         fp4 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8,
                         rank, const_cast<void*>(base), dims, strides, box, estr,
@@ -113,6 +139,8 @@ enum WeightKind { kMxfp4 = 0, kFp8Blk32 = 1, kMxfp8 = 2 };
 
 struct Plan {
   bool swap = false;
+  int kc = 1;            // 128-K chunks per pipeline stage
+  bool cluster = false;  // K slices reduced through DSMEM inside a thread-block cluster
   int bn = 256;
   int splits = 1;
   int kt_total = 0;
@@ -126,15 +154,20 @@ int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
 constexpr int64_t kMaxSplitTiles = 16384;                       // output tiles of a split-K call
 constexpr size_t kTicketRegion = kMaxSplitTiles * sizeof(int);  // 64 KiB
+constexpr int kMaxClusterSplit = 8;                             // portable cluster size
 
 int make_plan(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_config* cfg,
               int num_sms, Plan* p) {
   const int req_bn = cfg ? cfg->block_n : 0;
   const int req_split = cfg ? cfg->split_k : 0;
   const int req_swap = cfg ? cfg->swap_ab : -1;
+  const int req_mode = cfg ? cfg->split_mode : BQ_SPLIT_AUTO;
   if (req_bn != 0 && req_bn != 32 && req_bn != 64 && req_bn != 128 && req_bn != 256)
     return BQ_ERR_INVALID;
   if (req_split < 0 || req_split > 16 || req_swap < -1 || req_swap > 1) return BQ_ERR_INVALID;
+  if (req_mode < BQ_SPLIT_AUTO || req_mode > BQ_SPLIT_CLUSTER) return BQ_ERR_INVALID;
+  const int req_kc = cfg ? cfg->k_chunks : 0;
+  if (req_kc < 0 || req_kc > 4 || req_kc == 3) return BQ_ERR_INVALID;
   p->kt_total = ceil_div(K, 128);
   p->swap = req_swap == 1 || (req_swap == -1 && M <= 64);
   if (p->swap) {
@@ -144,28 +177,62 @@ int make_plan(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_conf
     p->tiles_p = ceil_div(N, 128);
     p->tiles_q = ceil_div(M, p->bn);
   } else {
-    p->bn = req_bn ? req_bn : (N > 128 ? 256 : 128);
-    if (p->bn != 128 && p->bn != 256) return BQ_ERR_INVALID;
     p->tiles_p = ceil_div(M, 128);
+    if (req_bn) {
+      p->bn = req_bn;
+    } else {
+      // Wave model from the schedule sweeps: a 128x256 tile does the work of
+      // two 128x128 tiles in ~0.82x their time; pick the width whose waves of
+      // persistent CTAs finish first.
+      const int64_t t256 = batch * p->tiles_p * ceil_div(N, 256);
+      const int64_t t128 = batch * p->tiles_p * ceil_div(N, 128);
+      const double c256 = static_cast<double>((t256 + num_sms - 1) / num_sms) * 256.0;
+      const double c128 = static_cast<double>((t128 + num_sms - 1) / num_sms) * 128.0 / 0.82;
+      p->bn = (N > 128 && c256 <= c128) ? 256 : 128;
+    }
+    if (p->bn != 128 && p->bn != 256) return BQ_ERR_INVALID;
     p->tiles_q = ceil_div(N, p->bn);
   }
   const int64_t tiles = batch * p->tiles_p * p->tiles_q;
   int splits = req_split;
   if (splits == 0) {
     splits = 1;
-    if (p->swap && tiles < num_sms) {
-      splits = static_cast<int>(num_sms / tiles);
-      if (splits > 16) splits = 16;
-      // keep at least two k-blocks per slice
-      if (splits > p->kt_total / 2) splits = p->kt_total / 2 > 0 ? p->kt_total / 2 : 1;
+    // Decode tiles: a cluster split pays one DSMEM exchange (~2-3 us of sync
+    // and skew), so it only wins when each tile has a long K loop (>= 24 K
+    // blocks, e.g. the 6144-deep down-projection): then spread it over a
+    // power-of-two cluster while the grid stays within one CTA per SM.
+    if (p->swap && req_mode != BQ_SPLIT_WORKSPACE && p->kt_total >= 24) {
+      while (splits * 2 <= kMaxClusterSplit && tiles * splits * 2 <= num_sms &&
+             p->kt_total / (splits * 2) >= 4)
+        splits *= 2;
     }
   }
   if (splits > p->kt_total) splits = p->kt_total;
+  const bool pow2 = (splits & (splits - 1)) == 0;
+  p->cluster = p->swap && splits > 1 && pow2 && splits <= kMaxClusterSplit &&
+               req_mode != BQ_SPLIT_WORKSPACE;
+  if (req_mode == BQ_SPLIT_CLUSTER && splits > 1 && !p->cluster) return BQ_ERR_INVALID;
+  // K blocks are dealt out evenly: slice s covers [s*KT/S, (s+1)*KT/S), never empty.
+  p->splits = splits;
   p->kt_per_split = ceil_div(p->kt_total, splits);
-  p->splits = ceil_div(p->kt_total, p->kt_per_split);  // every slice non-empty
   p->units = tiles * p->splits;
   if (p->units > 0x7FFFFFFF) return BQ_ERR_SHAPE;
-  if (p->splits > 1) {
+  // Chunks per stage: several 128-K chunks behind one barrier need whole
+  // chunks (K % 128 == 0); the swap-AB tiles take 4, the wide tiles 2.
+  const int kc_max = p->swap ? 4 : 2;
+  if (req_kc > 1 && (K % 128 != 0 || req_kc > kc_max)) return BQ_ERR_INVALID;
+  if (req_kc > 1 && p->splits > 1 && !p->cluster) return BQ_ERR_INVALID;
+  // Sweeps: 4 chunks for unsplit swap tiles, 1 for cluster slices (two CTAs
+  // per SM), 2 for 128-wide tiles, 1 for 256-wide tiles.
+  int kc_auto = 1;
+  if (K % 128 == 0) {
+    if (p->swap)
+      kc_auto = p->splits == 1 ? 4 : 1;
+    else
+      kc_auto = (p->bn == 128 && p->splits == 1) ? 2 : 1;
+  }
+  p->kc = req_kc ? req_kc : kc_auto;
+  if (p->splits > 1 && !p->cluster) {
     if (tiles > kMaxSplitTiles) return BQ_ERR_SHAPE;
     p->ws_partial = static_cast<size_t>(p->units) * 128 * p->bn * sizeof(float);
     p->ws_ticket = static_cast<size_t>(tiles) * sizeof(int);
@@ -177,53 +244,111 @@ int make_plan(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_conf
 // same bytes for every problem, so a call never finds another call's partial
 // sums where it expects zeroed tickets), then the fp32 partial tiles.
 size_t plan_ws_bytes(const Plan& p) {
-  if (p.splits <= 1) return 0;
+  if (p.splits <= 1 || p.cluster) return 0;
   return kTicketRegion + p.ws_partial;
 }
 
 // --------------------------------------------------------------- launches --
 
-template <int BN, int STAGES, int ACC, bool SWAP, bool P_FP4, bool Q_FP4>
+template <int BN, int STAGES, int ACC, bool SWAP, bool P_FP4, bool Q_FP4, int MODE, int KC>
 int launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const bq::GemmArgs& args,
                 int64_t units, int num_sms, cudaStream_t stream) {
-  using L = bq::GemmSmem<BN, STAGES, ACC>;
-  auto kern = bq::gemm_bs_kernel<BN, STAGES, ACC, SWAP, P_FP4, Q_FP4>;
+  constexpr bool CSPLIT = MODE == bq::kSplitCluster;
+  using L = bq::GemmSmem<BN, STAGES, ACC, CSPLIT, KC>;
+  auto kern = bq::gemm_bs_kernel<BN, STAGES, ACC, SWAP, P_FP4, Q_FP4, MODE, KC>;
   static bool attr_set[kMaxDevices] = {};
+  static int per_sm_cache[kMaxDevices] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (!attr_set[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) !=
-        cudaSuccess)
+            cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
       return BQ_ERR_CUDA;
+    int per_sm = 1;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, bq::kNumThreads, L::kBytes);
+    if (per_sm < 1) per_sm = 1;
+    // Co-resident CTAs share the SM's 512 TMEM columns.
+    const int tmem_fit = 512 / L::kTmemCols;
+    if (per_sm > tmem_fit) per_sm = tmem_fit;
+    per_sm_cache[dev] = per_sm;
     attr_set[dev] = true;
   }
-  int per_sm = 1;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, bq::kNumThreads, L::kBytes);
-  if (per_sm < 1) per_sm = 1;
-  // Co-resident CTAs share the SM's 512 TMEM columns.
-  const int tmem_fit = 512 / L::kTmemCols;
-  if (per_sm > tmem_fit) per_sm = tmem_fit;
-  int64_t grid = static_cast<int64_t>(num_sms) * per_sm;
-  if (grid > units) grid = units;
-  kern<<<static_cast<unsigned>(grid), bq::kNumThreads, L::kBytes, stream>>>(tp, tq, args);
+  const int per_sm = per_sm_cache[dev];
+  const int S = CSPLIT ? args.splits : 1;
+  int64_t grid = static_cast<int64_t>(num_sms) * per_sm / S * S;
+  if (grid < S) grid = S;
+  if (grid > units) grid = units;  // units is a multiple of S
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(static_cast<unsigned>(grid));
+  lc.blockDim = dim3(bq::kNumThreads);
+  lc.dynamicSmemBytes = L::kBytes;
+  lc.stream = stream;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  // May start while the preceding kernel (the activation quantizer) finishes:
+  // prologue and weight loads overlap it; griddepcontrol.wait guards the rest.
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  if (CSPLIT) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = static_cast<unsigned>(S);
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  lc.attrs = attr;
+  lc.numAttrs = na;
+  if (cudaLaunchKernelEx(&lc, kern, tp, tq, args) != cudaSuccess) {
+    cudaGetLastError();
+    return BQ_ERR_CUDA;
+  }
   return launch_status();
 }
 
-// Dispatch on (swap, bn, fp4 weights) to the compiled instances.
+template <int BN, int STAGES, int ACC, bool SWAP, int MODE, int KC>
+int launch_kind(bool w_fp4, const CUtensorMap& tp, const CUtensorMap& tq,
+                const bq::GemmArgs& args, int64_t u, int num_sms, cudaStream_t st) {
+  // FP4 weights sit on the P side with SWAP, on the Q side otherwise.
+  if (w_fp4)
+    return launch_gemm<BN, STAGES, ACC, SWAP, SWAP, !SWAP, MODE, KC>(tp, tq, args, u, num_sms, st);
+  return launch_gemm<BN, STAGES, ACC, SWAP, false, false, MODE, KC>(tp, tq, args, u, num_sms, st);
+}
+
+// Dispatch on (swap, bn, chunks per stage, split mode, fp4 weights) to the
+// compiled instances.  Stage counts fill ~200 KB of shared memory.
 int run_gemm(const Plan& pl, bool w_fp4, const CUtensorMap& tp, const CUtensorMap& tq,
-             const bq::GemmArgs& args, int num_sms, cudaStream_t st) {
+             const bq::GemmArgs& a, int ns, cudaStream_t st) {
+  const int64_t u = pl.units;
+  constexpr int kNone = bq::kSplitNone, kWs = bq::kSplitWorkspace, kCl = bq::kSplitCluster;
+  const bool b32 = pl.bn == 32;
   if (!pl.swap) {
-    if (pl.bn == 256)
-      return w_fp4 ? launch_gemm<256, 4, 1, false, false, true>(tp, tq, args, pl.units, num_sms, st)
-                   : launch_gemm<256, 4, 1, false, false, false>(tp, tq, args, pl.units, num_sms, st);
-    return w_fp4 ? launch_gemm<128, 6, 2, false, false, true>(tp, tq, args, pl.units, num_sms, st)
-                 : launch_gemm<128, 6, 2, false, false, false>(tp, tq, args, pl.units, num_sms, st);
+    if (pl.bn == 256) {
+      if (pl.splits > 1) return launch_kind<256, 4, 1, false, kWs, 1>(w_fp4, tp, tq, a, u, ns, st);
+      return pl.kc == 2 ? launch_kind<256, 2, 1, false, kNone, 2>(w_fp4, tp, tq, a, u, ns, st)
+                        : launch_kind<256, 4, 1, false, kNone, 1>(w_fp4, tp, tq, a, u, ns, st);
+    }
+    if (pl.splits > 1) return launch_kind<128, 6, 2, false, kWs, 1>(w_fp4, tp, tq, a, u, ns, st);
+    return pl.kc == 2 ? launch_kind<128, 3, 2, false, kNone, 2>(w_fp4, tp, tq, a, u, ns, st)
+                      : launch_kind<128, 6, 2, false, kNone, 1>(w_fp4, tp, tq, a, u, ns, st);
   }
-  if (pl.bn == 32)
-    return w_fp4 ? launch_gemm<32, 4, 1, true, true, false>(tp, tq, args, pl.units, num_sms, st)
-                 : launch_gemm<32, 4, 1, true, false, false>(tp, tq, args, pl.units, num_sms, st);
-  return w_fp4 ? launch_gemm<64, 4, 1, true, true, false>(tp, tq, args, pl.units, num_sms, st)
-               : launch_gemm<64, 4, 1, true, false, false>(tp, tq, args, pl.units, num_sms, st);
+  if (pl.cluster) {
+    if (pl.kc == 4)
+      return b32 ? launch_kind<32, 1, 1, true, kCl, 4>(w_fp4, tp, tq, a, u, ns, st)
+                 : launch_kind<64, 1, 1, true, kCl, 4>(w_fp4, tp, tq, a, u, ns, st);
+    return b32 ? launch_kind<32, 3, 1, true, kCl, 1>(w_fp4, tp, tq, a, u, ns, st)
+               : launch_kind<64, 3, 1, true, kCl, 1>(w_fp4, tp, tq, a, u, ns, st);
+  }
+  if (pl.splits > 1)
+    return b32 ? launch_kind<32, 4, 1, true, kWs, 1>(w_fp4, tp, tq, a, u, ns, st)
+               : launch_kind<64, 4, 1, true, kWs, 1>(w_fp4, tp, tq, a, u, ns, st);
+  if (pl.kc == 4)
+    return b32 ? launch_kind<32, 2, 1, true, kNone, 4>(w_fp4, tp, tq, a, u, ns, st)
+               : launch_kind<64, 2, 1, true, kNone, 4>(w_fp4, tp, tq, a, u, ns, st);
+  return b32 ? launch_kind<32, 8, 1, true, kNone, 1>(w_fp4, tp, tq, a, u, ns, st)
+             : launch_kind<64, 8, 1, true, kNone, 1>(w_fp4, tp, tq, a, u, ns, st);
 }
 
 int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, const void* b_sf,
@@ -277,10 +402,10 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
   const int b_box = pl.swap ? 128 : pl.bn;
   const bool a_batched = count > 1 && sa != 0;
   const bool b_batched = count > 1 && sb != 0;
-  st = make_operand_map(&map_a, a_q, false, K, M, K, a_batched ? count : 1, sa, a_box);
+  st = make_operand_map(&map_a, a_q, false, K, M, K, a_batched ? count : 1, sa, a_box, pl.kc);
   if (st != BQ_OK) return st;
   st = make_operand_map(&map_b, b, w_fp4, K, N, w_fp4 ? K / 2 : K, b_batched ? count : 1, sb,
-                        b_box);
+                        b_box, pl.kc);
   if (st != BQ_OK) return st;
 
   bq::GemmArgs g;
@@ -297,6 +422,8 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
   g.raster_group = 8;
   g.sf_katoms = ceil_div(K, 128);
   g.sf_q_rowatoms = ceil_div(pl.swap ? M : N, 128);
+  g.split_lg = 0;
+  while ((1 << g.split_lg) < pl.splits) ++g.split_lg;
   const uint8_t* sfa = static_cast<const uint8_t*>(a_sf);
   const uint8_t* sfb = static_cast<const uint8_t*>(b_sf);
   g.sf_p = pl.swap ? sfb : sfa;
@@ -314,7 +441,7 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
   g.res_bstride = sr / 2;
   g.alpha = epi ? epi->alpha : 1.0f;
   g.act = epi ? epi->act : BQ_ACT_NONE;
-  if (pl.splits > 1) {
+  if (pl.splits > 1 && !pl.cluster) {
     g.ws_ticket = static_cast<int*>(ws);
     g.ws_partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kTicketRegion);
   }
@@ -368,11 +495,22 @@ int bq_act_quant(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, void* q_
   const int64_t rows_pad = (M + 127) / 128 * 128;
   const int64_t chunks = (K / 32 + 15) / 16;
   if (rows_pad / 8 > 0x7FFFFFFF || chunks > 65535) return BQ_ERR_SHAPE;
-  dim3 grid(static_cast<unsigned>(rows_pad / 8), static_cast<unsigned>(chunks));
-  bq::act_quant_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __nv_bfloat16*>(x_bf16), M, K, ldx, rows_pad,
-      static_cast<uint8_t*>(q_e4m3), static_cast<uint8_t*>(sf_mma),
-      static_cast<uint8_t*>(sf_rowmajor), d_status);
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(static_cast<unsigned>(rows_pad / 8), static_cast<unsigned>(chunks));
+  lc.blockDim = dim3(256);
+  lc.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  if (cudaLaunchKernelEx(&lc, bq::act_quant_kernel, static_cast<const __nv_bfloat16*>(x_bf16), M,
+                         K, ldx, rows_pad, static_cast<uint8_t*>(q_e4m3),
+                         static_cast<uint8_t*>(sf_mma), static_cast<uint8_t*>(sf_rowmajor),
+                         d_status) != cudaSuccess) {
+    cudaGetLastError();
+    return BQ_ERR_CUDA;
+  }
   return launch_status();
 }
 
@@ -432,7 +570,7 @@ int bq_unpack_scales(const void* sf_mma, int64_t rows, int64_t K, void* rowmajor
 }
 
 // The plain entries take no workspace, so their schedule never splits K.
-static const bq_gemm_config kNoSplit = {0, 1, -1, 0};
+static const bq_gemm_config kNoSplit = {0, 1, -1, BQ_SPLIT_AUTO, 0};
 
 int bq_gemm_mxfp8_mxfp4(const void* a_q, const void* a_sf, const void* b_fp4, const void* b_sf,
                         int64_t M, int64_t N, int64_t K, void* y_bf16, bq_stream_t stream) {

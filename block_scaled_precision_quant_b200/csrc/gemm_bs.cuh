@@ -57,6 +57,7 @@ struct GemmArgs {
   int raster_group;
   int sf_katoms;   // scale atoms along K = ceil(K / 128)
   int sf_q_rowatoms;  // 128-row scale bands of the Q-side operand = ceil(rows_q / 128)
+  int split_lg;       // log2(splits) for cluster split-K
   // scale buffers (MMA layout) of the P- and Q-side operands, batch strides in bytes
   const uint8_t *sf_p;
   const uint8_t *sf_q;
@@ -76,18 +77,36 @@ struct GemmArgs {
   int *err;
 };
 
-template <int BN, int STAGES, int ACC>
+// How the K slices of an output tile are combined (a compile-time property of
+// each kernel instance, so an instance carries only the code it runs).
+enum SplitMode : int { kSplitNone = 0, kSplitWorkspace = 1, kSplitCluster = 2 };
+
+// Shared-memory layout of one kernel instance.  A stage holds KC chunks of
+// 128 K (each chunk a 128B-swizzled K-major tile per operand) and the
+// chunks' scale-factor atoms; more bytes behind one stage barrier means fewer
+// barrier round trips per byte, which is what bounds a CTA's copy rate.
+template <int BN, int STAGES, int ACC, bool CSPLIT = false, int KC = 1>
 struct GemmSmem {
   static constexpr int kSfqAtoms = BN > 128 ? BN / 128 : 1;
   static constexpr int kSfqCols = 4 * kSfqAtoms;
-  static constexpr int kSfCols = 4 + kSfqCols;  // TMEM columns of scales per stage
-  static constexpr int kBytesP = kBlockP * kBlockK;
-  static constexpr int kBytesQ = BN * kBlockK;
+  static constexpr int kSfColsChunk = 4 + kSfqCols;  // TMEM scale columns per K chunk
+  static constexpr int kSfCols = KC * kSfColsChunk;  // TMEM scale columns per stage
+  static constexpr int kChunkP = kBlockP * kBlockK;  // bytes of one 128-K chunk, P side
+  static constexpr int kChunkQ = BN * kBlockK;       // Q side
+  static constexpr int kBytesP = KC * kChunkP;
+  static constexpr int kBytesQ = KC * kChunkQ;
+  static constexpr int kSfpBytes = KC * kSfAtom;              // per stage
+  static constexpr int kSfqBytes = KC * kSfqAtoms * kSfAtom;  // per stage
   static constexpr int kOffQ = STAGES * kBytesP;
   static constexpr int kOffSfp = kOffQ + STAGES * kBytesQ;
-  static constexpr int kOffSfq = kOffSfp + STAGES * kSfAtom;
-  static constexpr int kOffBar = kOffSfq + STAGES * kSfqAtoms * kSfAtom;
-  static constexpr int kNumBars = 2 * STAGES + 2 * ACC + 1;
+  static constexpr int kOffSfq = kOffSfp + STAGES * kSfpBytes;
+  // cluster split-K: receive buffer [S slices][128/S rows][BN + 4] fp32 (the
+  // +4 pad keeps float4 row accesses free of bank conflicts)
+  static constexpr int kRecvStride = BN + 4;
+  static constexpr int kOffPart = kOffSfq + STAGES * kSfqBytes;
+  static constexpr int kBytesPart = CSPLIT ? kBlockP * kRecvStride * 4 : 0;
+  static constexpr int kOffBar = kOffPart + kBytesPart;
+  static constexpr int kNumBars = 2 * STAGES + 2 * ACC + 1 + (CSPLIT ? 2 : 0);
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 64 + 1024;  // + alignment slack
   static constexpr int kTmemUsed = ACC * BN + STAGES * kSfCols;
@@ -112,23 +131,36 @@ __device__ __forceinline__ uint32_t make_idesc(uint32_t fmt_p, uint32_t fmt_q, i
   return d;
 }
 
-__device__ __forceinline__ void decode_unit(const GemmArgs &a, int unit, int &b, int &tp, int &tq,
-                                            int &split, int &tile) {
-  split = unit % a.splits;
-  tile = unit / a.splits;
+// Work unit -> (batch, P tile, Q tile, K slice) with grouped rasterization
+// over P tiles, and the unit's K-block range (slices dealt out evenly, never
+// empty while splits <= K blocks).  32-bit arithmetic throughout.
+struct UnitPos {
+  int b, tp, tq, split, tile, kt0, kt1;
+};
+
+__device__ __forceinline__ UnitPos unit_pos(const GemmArgs &a, int unit) {
+  UnitPos u;
+  u.split = unit % a.splits;
+  u.tile = unit / a.splits;
   const int per_batch = a.tiles_p * a.tiles_q;
-  b = tile / per_batch;
-  const int idx = tile - b * per_batch;
+  u.b = u.tile / per_batch;
+  const int idx = u.tile - u.b * per_batch;
   const int group = a.raster_group * a.tiles_q;
   const int g = idx / group;
   const int first_p = g * a.raster_group;
   const int gp = min(a.raster_group, a.tiles_p - first_p);
   const int r = idx - g * group;
-  tp = first_p + r % gp;
-  tq = r / gp;
+  u.tp = first_p + r % gp;
+  u.tq = r / gp;
+  u.kt0 = (u.split * a.kt_total) / a.splits;
+  u.kt1 = ((u.split + 1) * a.kt_total) / a.splits;
+  return u;
 }
 
-__device__ __forceinline__ float gelu_erf(float t) {
+// erf-form GELU.  Kept out of line: the epilogue is unrolled over many
+// values, and inlining erff at every one of them would bloat the straight-line
+// code every call fetches, GELU or not.
+__device__ __noinline__ float gelu_erf(float t) {
   return 0.5f * t * (1.0f + erff(t * 0.70710678118654752f));
 }
 
@@ -190,27 +222,183 @@ __device__ __forceinline__ void emit32(const GemmArgs &a, int b, int prow, int q
       *reinterpret_cast<uint4 *>(yrow + n) = make_uint4(o[0], o[1], o[2], o[3]);
     }
   } else {
+    // Thread = output column n, its 32 values = rows m = q0 .. q0+31: one
+    // bf16 per row; across the warp each row's store is 64 contiguous bytes.
     const int n = prow;
-    if (n >= a.N) return;
+    if (n >= a.N || q0 >= a.M) return;
     const float bias = a.bias ? __bfloat162float(a.bias[n]) : 0.0f;
+    const int cnt = min(32, a.M - q0);
+    __nv_bfloat16 *yp = a.y + b * a.y_bstride + static_cast<int64_t>(q0) * a.ldy + n;
+    const int ldy = static_cast<int>(a.ldy);
+    if (a.res == nullptr && a.act == 0) {
+      const float alpha = a.alpha;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int m = q0 + j;
-      if (m >= a.M) break;
-      const float res =
-          a.res ? __bfloat162float(a.res[b * a.res_bstride + static_cast<int64_t>(m) * a.ldres + n])
-                : 0.0f;
-      a.y[b * a.y_bstride + static_cast<int64_t>(m) * a.ldy + n] =
-          __float2bfloat16_rn(epi_value(a, f[j], bias, res));
+      for (int j = 0; j < 32; ++j)
+        if (j < cnt) yp[j * ldy] = __float2bfloat16_rn(alpha * f[j] + bias);
+    } else {
+      const __nv_bfloat16 *rp =
+          a.res ? a.res + b * a.res_bstride + static_cast<int64_t>(q0) * a.ldres + n : nullptr;
+      const int ldr = static_cast<int>(a.ldres);
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (j < cnt) {
+          const float res = rp ? __bfloat162float(rp[j * ldr]) : 0.0f;
+          yp[j * ldy] = __float2bfloat16_rn(epi_value(a, f[j], bias, res));
+        }
     }
   }
 }
 
-template <int BN, int STAGES, int ACC, bool SWAP, bool P_FP4, bool Q_FP4>
+__device__ __forceinline__ void epi_bar_sync() {
+  __syncwarp();
+  asm volatile("barrier.sync 1, 128;" ::: "memory");  // the 4 epilogue warps
+}
+
+// Swap-AB output of 4 consecutive weight rows n..n+3 at activation row m
+// (y[m][n..n+3], 8-byte store); n % 4 == 0 and N % 8 == 0, so the group is
+// either fully inside the output or fully outside.
+__device__ __forceinline__ void emit4_swap(const GemmArgs &a, int b, int n, int m, float4 f) {
+  if (m >= a.M || n >= a.N) return;
+  float bias[4] = {0.f, 0.f, 0.f, 0.f}, res[4] = {0.f, 0.f, 0.f, 0.f};
+  if (a.bias) {
+    const uint2 v = *reinterpret_cast<const uint2 *>(a.bias + n);
+    bias[0] = bf16_bits_to_f32(v.x & 0xFFFF);
+    bias[1] = bf16_bits_to_f32(v.x >> 16);
+    bias[2] = bf16_bits_to_f32(v.y & 0xFFFF);
+    bias[3] = bf16_bits_to_f32(v.y >> 16);
+  }
+  if (a.res) {
+    const uint2 v = *reinterpret_cast<const uint2 *>(
+        a.res + b * a.res_bstride + static_cast<int64_t>(m) * a.ldres + n);
+    res[0] = bf16_bits_to_f32(v.x & 0xFFFF);
+    res[1] = bf16_bits_to_f32(v.x >> 16);
+    res[2] = bf16_bits_to_f32(v.y & 0xFFFF);
+    res[3] = bf16_bits_to_f32(v.y >> 16);
+  }
+  const __nv_bfloat162 lo =
+      __floats2bfloat162_rn(epi_value(a, f.x, bias[0], res[0]), epi_value(a, f.y, bias[1], res[1]));
+  const __nv_bfloat162 hi =
+      __floats2bfloat162_rn(epi_value(a, f.z, bias[2], res[2]), epi_value(a, f.w, bias[3], res[3]));
+  uint2 o;
+  o.x = *reinterpret_cast<const uint32_t *>(&lo);
+  o.y = *reinterpret_cast<const uint32_t *>(&hi);
+  *reinterpret_cast<uint2 *>(a.y + b * a.y_bstride + static_cast<int64_t>(m) * a.ldy + n) = o;
+}
+
+// Cluster split-K reduction of one CTA's row slice, S = 2^LG slices.  The
+// slice is rows [split * 128/S, (split+1) * 128/S) of the tile; a thread owns
+// 4 consecutive rows (the same for every column it handles) and the columns
+// (epi_tid + 128 i) / quads.  All BN/4 DSMEM loads are issued before any sum;
+// each output is then summed in slice order 0..S-1.
+// Loads one operand side of one stage (KC chunks of 128 K starting at K
+// block kt, of which `nvalid` belong to the unit): the weights (P side with
+// SWAP, Q side otherwise) or the activations, each with its scale atoms.
+// KC == 1 uses 2-D (3-D batched) maps with the K offset in elements; KC > 1
+// uses maps that view K as (128, K/128 chunks), so one copy brings all chunks.
+template <int BN, int STAGES, int ACC, bool SWAP, bool CSPLIT, int KC>
+__device__ __forceinline__ void issue_half(const GemmArgs &a, const CUtensorMap *tm_p,
+                                           const CUtensorMap *tm_q, uint8_t *smem,
+                                           uint64_t *full, int st, int kt, int nvalid,
+                                           const UnitPos &u, bool weights) {
+  using L = GemmSmem<BN, STAGES, ACC, CSPLIT, KC>;
+  if (weights == SWAP) {  // P side
+    uint8_t *dst = smem + st * L::kBytesP;
+    const int row = u.tp * kBlockP;
+    if constexpr (KC == 1) {
+      if (a.p_batched)
+        tma_load_3d(dst, tm_p, &full[st], kt * kBlockK, row, u.b);
+      else
+        tma_load_2d(dst, tm_p, &full[st], kt * kBlockK, row);
+    } else {
+      if (a.p_batched)
+        tma_load_4d(dst, tm_p, &full[st], 0, row, kt, u.b);
+      else
+        tma_load_3d(dst, tm_p, &full[st], 0, row, kt);
+    }
+    const uint8_t *sfp = a.sf_p + u.b * a.sf_p_bstride +
+                         (static_cast<int64_t>(u.tp) * a.sf_katoms + kt) * kSfAtom;
+    bulk_load(smem + L::kOffSfp + st * L::kSfpBytes, sfp, nvalid * kSfAtom, &full[st]);
+  } else {  // Q side
+    const int q_row0 = u.tq * BN;
+    uint8_t *dst = smem + L::kOffQ + st * L::kBytesQ;
+    if constexpr (KC == 1) {
+      if (a.q_batched)
+        tma_load_3d(dst, tm_q, &full[st], kt * kBlockK, q_row0, u.b);
+      else
+        tma_load_2d(dst, tm_q, &full[st], kt * kBlockK, q_row0);
+    } else {
+      if (a.q_batched)
+        tma_load_4d(dst, tm_q, &full[st], 0, q_row0, kt, u.b);
+      else
+        tma_load_3d(dst, tm_q, &full[st], 0, q_row0, kt);
+    }
+#pragma unroll
+    for (int j = 0; j < L::kSfqAtoms; ++j) {
+      // A band past the operand's last row would be outside the scale buffer;
+      // those rows are zero-filled by TMA, so any finite scale band serves --
+      // reuse the last one.
+      const int band = min(q_row0 / 128 + j, a.sf_q_rowatoms - 1);
+      const uint8_t *sfq = a.sf_q + u.b * a.sf_q_bstride +
+                           (static_cast<int64_t>(band) * a.sf_katoms + kt) * kSfAtom;
+      bulk_load(smem + L::kOffSfq + st * L::kSfqBytes + j * KC * kSfAtom, sfq, nvalid * kSfAtom,
+                &full[st]);
+    }
+  }
+}
+
+// Cluster split-K, second half: this CTA owns rows [split * R, (split+1) * R)
+// (R = 128 / S) of the output tile and has received every slice's fp32
+// partial of those rows in its receive buffer.  A thread owns one row (the
+// same for every column group it handles), sums the S slices in slice order
+// and writes 4 columns (activation rows m) per group.
+template <int BN, int LG>
+__device__ __forceinline__ void cluster_reduce_local(const GemmArgs &a, const UnitPos &u,
+                                                     int epi_tid, const float *recv) {
+  constexpr int S = 1 << LG;
+  constexpr int R = kBlockP >> LG;
+  constexpr int kStride = BN + 4;
+  constexpr int kIters = R * (BN / 4) / 128;
+  static_assert(kIters >= 1 && R * (BN / 4) % 128 == 0, "slice shape");
+  const int rl = epi_tid % R;
+  const int n = u.tp * kBlockP + u.split * R + rl;
+  if (n >= a.N) return;
+  const float bias = a.bias ? __bfloat162float(a.bias[n]) : 0.0f;
+#pragma unroll
+  for (int i = 0; i < kIters; ++i) {
+    const int c4 = (epi_tid + 128 * i) / R;
+    float4 acc = *reinterpret_cast<const float4 *>(recv + rl * kStride + c4 * 4);
+#pragma unroll
+    for (int s = 1; s < S; ++s) {
+      const float4 v = *reinterpret_cast<const float4 *>(recv + (s * R + rl) * kStride + c4 * 4);
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    const float vals[4] = {acc.x, acc.y, acc.z, acc.w};
+    const int m0 = u.tq * BN + c4 * 4;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int m = m0 + j;
+      if (m < a.M) {
+        const float res =
+            a.res ? __bfloat162float(a.res[u.b * a.res_bstride + static_cast<int64_t>(m) * a.ldres + n])
+                  : 0.0f;
+        a.y[u.b * a.y_bstride + static_cast<int64_t>(m) * a.ldy + n] =
+            __float2bfloat16_rn(epi_value(a, vals[j], bias, res));
+      }
+    }
+  }
+}
+
+template <int BN, int STAGES, int ACC, bool SWAP, bool P_FP4, bool Q_FP4, int MODE, int KC>
 __global__ void __launch_bounds__(kNumThreads, 1)
     gemm_bs_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
                    const GemmArgs a) {
-  using L = GemmSmem<BN, STAGES, ACC>;
+  constexpr bool CSPLIT = MODE == kSplitCluster;
+  static_assert(!CSPLIT || SWAP, "cluster split-K is built for the swap-AB (decode) tiles");
+  static_assert(!CSPLIT || ACC == 1, "cluster split-K uses one accumulator");
+  using L = GemmSmem<BN, STAGES, ACC, CSPLIT, KC>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -223,86 +411,106 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   uint64_t *tfull = empty + STAGES;
   uint64_t *tempty = tfull + ACC;
   uint64_t *drain = tempty + ACC;
+  uint64_t *peer_ready = drain + 1;  // CSPLIT: every slice's rows for this CTA have arrived
+  uint64_t *peer_free = drain + 2;   // CSPLIT: every owner has consumed the previous tile
+  float *recv = reinterpret_cast<float *>(smem + L::kOffPart);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
   int *last_flag = reinterpret_cast<int *>(smem + L::kOffMisc + 8);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
+  const int total_units = a.batch * a.tiles_p * a.tiles_q * a.splits;
+  // Transaction bytes of a stage with `nv` chunks inside the unit.  The
+  // operand copies always move whole boxes (chunks past the tensor are zero
+  // filled); a 4-bit operand lands in shared memory with one byte-slot per
+  // code but counts its packed size (half the footprint).  Scale atoms are
+  // copied for the unit's chunks only.
+  auto tx_bytes = [](int nv) -> uint32_t {
+    return static_cast<uint32_t>((P_FP4 ? L::kBytesP / 2 : L::kBytesP) +
+                                 (Q_FP4 ? L::kBytesQ / 2 : L::kBytesQ) +
+                                 nv * (1 + L::kSfqAtoms) * kSfAtom);
+  };
 
+  // Thread 0 (the producer) sets up the barriers and at once issues the weight
+  // half of the first unit's first stages: the weights do not depend on the
+  // kernel before this one in the stream, and these copies then overlap the
+  // TMEM allocation, the cluster barrier and (under programmatic dependent
+  // launch) the tail of that kernel.
+  int pre_n = 0;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+    for (int st = 0; st < STAGES; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], 1);
     }
-    for (int s = 0; s < ACC; ++s) {
-      mbar_init(&tfull[s], 1);
-      mbar_init(&tempty[s], 4);  // one arrival per epilogue warp
+    for (int st = 0; st < ACC; ++st) {
+      mbar_init(&tfull[st], 1);
+      mbar_init(&tempty[st], 4);  // one arrival per epilogue warp
     }
     mbar_init(drain, 1);
+    if constexpr (CSPLIT) {
+      mbar_init(peer_ready, a.splits);
+      mbar_init(peer_free, a.splits);
+    }
     *abort_flag = 0;
     fence_mbar_init();
-  }
-  if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_p);
     tma_prefetch_desc(&tm_q);
+    if (static_cast<int>(blockIdx.x) < total_units) {
+      const UnitPos u = unit_pos(a, blockIdx.x);
+      pre_n = min(STAGES, (u.kt1 - u.kt0 + KC - 1) / KC);
+      for (int j = 0; j < pre_n; ++j) {
+        const int kt = u.kt0 + j * KC;
+        const int nv = min(KC, u.kt1 - kt);
+        mbar_arrive_expect_tx(&full[j], tx_bytes(nv));
+        issue_half<BN, STAGES, ACC, SWAP, CSPLIT, KC>(a, &tm_p, &tm_q, smem, full, j, kt, nv, u,
+                                                      true);
+      }
+    }
   }
   if (warp == 1) tmem_alloc(tmem_slot, L::kTmemCols);
   tc_fence_before();
   __syncthreads();
+  // Peers store into this CTA's receive buffer and arrive on its barriers:
+  // every CTA of the cluster must have initialised its barriers first.
+  if constexpr (CSPLIT) cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-
-  const int total_units = a.batch * a.tiles_p * a.tiles_q * a.splits;
-  // Transaction bytes of one stage.  A 4-bit operand lands in shared memory
-  // with one byte-slot per code, but the transaction count is the packed size
-  // (half the footprint).
-  constexpr uint32_t kTxBytes = (P_FP4 ? L::kBytesP / 2 : L::kBytesP) +
-                                (Q_FP4 ? L::kBytesQ / 2 : L::kBytesQ) + kSfAtom +
-                                L::kSfqAtoms * kSfAtom;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
     if (lane == 0) {
+      // Everything from here may read what the preceding kernel wrote.
+      griddep_wait();
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      bool first = true;
       for (int unit = blockIdx.x; unit < total_units && ok; unit += gridDim.x) {
-        int b, tp, tq, split, tile;
-        decode_unit(a, unit, b, tp, tq, split, tile);
-        const int kt0 = split * a.kt_per_split;
-        const int kt1 = min(a.kt_total, kt0 + a.kt_per_split);
-        const int q_row0 = tq * BN;
-        const uint8_t *sfp = a.sf_p + b * a.sf_p_bstride +
-                             static_cast<int64_t>(tp) * a.sf_katoms * kSfAtom;
-        const uint8_t *sfq = a.sf_q + b * a.sf_q_bstride +
-                             static_cast<int64_t>(q_row0 / 128) * a.sf_katoms * kSfAtom;
-        for (int kt = kt0; kt < kt1; ++kt) {
+        const UnitPos u = unit_pos(a, unit);
+        int kt = u.kt0;
+        if (first) {  // activation halves of the stages issued before the barrier
+          for (int j = 0; j < pre_n; ++j) {
+            const int kj = u.kt0 + j * KC;
+            issue_half<BN, STAGES, ACC, SWAP, CSPLIT, KC>(a, &tm_p, &tm_q, smem, full, j, kj,
+                                                          min(KC, u.kt1 - kj), u, false);
+          }
+          kt += pre_n * KC;
+          stage = pre_n % STAGES;
+          phase = pre_n == STAGES ? 1u : 0u;
+          first = false;
+        }
+        for (; kt < u.kt1; kt += KC) {
           if (!mbar_wait(&empty[stage], phase ^ 1, a.err, abort_flag, kWaitProdEmpty)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], kTxBytes);
-          const int kx = kt * kBlockK;
-          if (a.p_batched)
-            tma_load_3d(s_p + stage * L::kBytesP, &tm_p, &full[stage], kx, tp * kBlockP, b);
-          else
-            tma_load_2d(s_p + stage * L::kBytesP, &tm_p, &full[stage], kx, tp * kBlockP);
-          if (a.q_batched)
-            tma_load_3d(s_q + stage * L::kBytesQ, &tm_q, &full[stage], kx, q_row0, b);
-          else
-            tma_load_2d(s_q + stage * L::kBytesQ, &tm_q, &full[stage], kx, q_row0);
-          bulk_load(s_sfp + stage * kSfAtom, sfp + kt * kSfAtom, kSfAtom, &full[stage]);
-#pragma unroll
-          for (int j = 0; j < L::kSfqAtoms; ++j) {
-            // A band past the operand's last row would be outside the scale
-            // buffer; those rows are zero-filled by TMA, so any finite scale
-            // band serves -- reuse the last one.
-            const int band = min(q_row0 / 128 + j, a.sf_q_rowatoms - 1) - q_row0 / 128;
-            bulk_load(s_sfq + (stage * L::kSfqAtoms + j) * kSfAtom,
-                      sfq + (static_cast<int64_t>(band) * a.sf_katoms + kt) * kSfAtom, kSfAtom,
-                      &full[stage]);
-          }
+          const int nv = min(KC, u.kt1 - kt);
+          mbar_arrive_expect_tx(&full[stage], tx_bytes(nv));
+          issue_half<BN, STAGES, ACC, SWAP, CSPLIT, KC>(a, &tm_p, &tm_q, smem, full, stage, kt, nv,
+                                                        u, true);
+          issue_half<BN, STAGES, ACC, SWAP, CSPLIT, KC>(a, &tm_p, &tm_q, smem, full, stage, kt, nv,
+                                                        u, false);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
@@ -322,35 +530,40 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int unit = blockIdx.x; unit < total_units && ok; unit += gridDim.x) {
-        int b, tp, tq, split, tile;
-        decode_unit(a, unit, b, tp, tq, split, tile);
-        const int kt0 = split * a.kt_per_split;
-        const int kt1 = min(a.kt_total, kt0 + a.kt_per_split);
-        const uint32_t sfq_row_off = static_cast<uint32_t>((tq * BN) % 128) / 32;
+        const UnitPos u = unit_pos(a, unit);
+        const uint32_t sfq_row_off = static_cast<uint32_t>((u.tq * BN) % 128) / 32;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1, a.err, abort_flag, kWaitMmaTmemEmpty)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kt = kt0; kt < kt1; ++kt) {
+        for (int kt = u.kt0; kt < u.kt1; kt += KC) {
           if (!mbar_wait(&full[stage], phase, a.err, abort_flag, kWaitMmaFull)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sf_t = tmem_base + ACC * BN + stage * L::kSfCols;
-          tc_cp_sf(sf_t, desc_sf_32x128b(smem_u32(s_sfp + stage * kSfAtom)));
+          const int nv = min(KC, u.kt1 - kt);  // chunks of this stage inside the unit
+          const uint32_t sf_stage = tmem_base + ACC * BN + stage * L::kSfCols;
+          const uint32_t pa0 = smem_u32(s_p + stage * L::kBytesP);
+          const uint32_t qa0 = smem_u32(s_q + stage * L::kBytesQ);
+          const uint32_t sfp0 = smem_u32(s_sfp + stage * L::kSfpBytes);
+          const uint32_t sfq0 = smem_u32(s_sfq + stage * L::kSfqBytes);
+#pragma unroll 1
+          for (int c = 0; c < nv; ++c) {
+            const uint32_t sf_t = sf_stage + c * L::kSfColsChunk;
+            tc_cp_sf(sf_t, desc_sf_32x128b(sfp0 + c * kSfAtom));
 #pragma unroll
-          for (int j = 0; j < L::kSfqAtoms; ++j)
-            tc_cp_sf(sf_t + 4 + 4 * j,
-                     desc_sf_32x128b(smem_u32(s_sfq + (stage * L::kSfqAtoms + j) * kSfAtom)));
-          const uint32_t pa = smem_u32(s_p + stage * L::kBytesP);
-          const uint32_t qa = smem_u32(s_q + stage * L::kBytesQ);
+            for (int j = 0; j < L::kSfqAtoms; ++j)
+              tc_cp_sf(sf_t + 4 + 4 * j, desc_sf_32x128b(sfq0 + (j * KC + c) * kSfAtom));
+            const uint32_t pa = pa0 + c * L::kChunkP;
+            const uint32_t qa = qa0 + c * L::kChunkQ;
 #pragma unroll
-          for (int ks = 0; ks < kBlockK / kMmaK; ++ks) {
-            const uint32_t idesc = make_idesc(P_FP4 ? kFmtE2M1 : kFmtE4M3,
-                                              Q_FP4 ? kFmtE2M1 : kFmtE4M3, BN, ks);
-            tc_mma_mxf8f6f4(d_tmem, desc_kmajor_sw128(pa + ks * kMmaK),
-                            desc_kmajor_sw128(qa + ks * kMmaK), idesc, sf_t,
-                            sf_t + 4 + sfq_row_off, (kt > kt0 || ks > 0) ? 1u : 0u);
+            for (int ks = 0; ks < kBlockK / kMmaK; ++ks) {
+              const uint32_t idesc = make_idesc(P_FP4 ? kFmtE2M1 : kFmtE4M3,
+                                                Q_FP4 ? kFmtE2M1 : kFmtE4M3, BN, ks);
+              tc_mma_mxf8f6f4(d_tmem, desc_kmajor_sw128(pa + ks * kMmaK),
+                              desc_kmajor_sw128(qa + ks * kMmaK), idesc, sf_t,
+                              sf_t + 4 + sfq_row_off, (kt > u.kt0 || c > 0 || ks > 0) ? 1u : 0u);
+            }
           }
           tc_commit(&empty[stage]);
           if (++stage == STAGES) {
@@ -377,15 +590,72 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     const int epi_tid = threadIdx.x - 64;  // 0..127
     int acc = 0;
     uint32_t acc_phase = 0;
+    uint32_t ready_phase = 0, free_phase = 0;
+    bool free_pending = false;  // CSPLIT: owners may still be reading the previous tile
     for (int unit = blockIdx.x; unit < total_units; unit += gridDim.x) {
-      int b, tp, tq, split, tile;
-      decode_unit(a, unit, b, tp, tq, split, tile);
+      const UnitPos u = unit_pos(a, unit);
       __syncwarp();
       if (!mbar_wait(&tfull[acc], acc_phase, a.err, abort_flag, kWaitEpiFull)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + acc * BN + (static_cast<uint32_t>(quad * 32) << 16);
-      const int prow = tp * kBlockP + row;
-      if (a.splits == 1) {
+      const int prow = u.tp * kBlockP + row;
+      if constexpr (MODE == kSplitCluster) {
+        // Cluster split-K: the S CTAs of this cluster hold the S K-slices of
+        // one output tile.  Every CTA pushes each row of its fp32 partial
+        // straight from TMEM registers into the receive buffer of the CTA that
+        // owns that row (DSMEM stores), signals the owners, then finishes its
+        // own 128/S rows from local shared memory.
+        const int lg = a.split_lg;
+        const int S = 1 << lg;
+        if (free_pending) {  // the owners' receive buffers are free again
+          if (!mbar_wait_cluster(peer_free, free_phase, a.err, abort_flag, kWaitPeerDone)) break;
+          free_phase ^= 1;
+          free_pending = false;
+        }
+        const int R = kBlockP >> lg;
+        const uint32_t owner = static_cast<uint32_t>(row >> (7 - lg));
+        const uint32_t dst =
+            mapa_shared(smem_u32(recv), owner) +
+            static_cast<uint32_t>((u.split * R + (row & (R - 1))) * L::kRecvStride * 4);
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          __syncwarp();
+          tmem_ld_32x32b_x32(t_row + c * 32, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            st_dsmem_u4(dst + static_cast<uint32_t>((c * 32 + 4 * q) * 4), v[4 * q], v[4 * q + 1],
+                        v[4 * q + 2], v[4 * q + 3]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
+        epi_bar_sync();
+        if (epi_tid == 0) {
+          fence_acq_rel_cluster();
+          const uint32_t rb = smem_u32(peer_ready);
+          for (int r = 0; r < S; ++r) mbar_arrive_cluster(mapa_shared(rb, static_cast<uint32_t>(r)));
+        }
+        if (!mbar_wait_cluster(peer_ready, ready_phase, a.err, abort_flag, kWaitPeerReady)) break;
+        ready_phase ^= 1;
+        switch (lg) {
+          case 1: cluster_reduce_local<BN, 1>(a, u, epi_tid, recv); break;
+          case 2: cluster_reduce_local<BN, 2>(a, u, epi_tid, recv); break;
+          default: cluster_reduce_local<BN, 3>(a, u, epi_tid, recv); break;
+        }
+        if (unit + static_cast<int>(gridDim.x) < total_units) {
+          // another tile follows: release this CTA's receive buffer to the pushers
+          epi_bar_sync();
+          if (epi_tid == 0) {
+            fence_acq_rel_cluster();
+            const uint32_t fb = smem_u32(peer_free);
+            for (int r = 0; r < S; ++r)
+              mbar_arrive_cluster(mapa_shared(fb, static_cast<uint32_t>(r)));
+          }
+          free_pending = true;
+        }
+      } else if constexpr (MODE == kSplitNone) {
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t v[32];
@@ -395,19 +665,20 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           float f[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
-          emit32<SWAP>(a, b, prow, tq * BN + c * 32, f);
+          emit32<SWAP>(a, u.b, prow, u.tq * BN + c * 32, f);
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[acc]);
       } else {
+        static_assert(MODE == kSplitWorkspace, "split mode");
         // Split-K: publish this slice's partial tile, then the last slice to
         // arrive reduces all slices in slice order.
         float *mine = a.ws_partial + (static_cast<int64_t>(unit) * kBlockP + row) * BN;
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t v[32];
-          __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the stores
+          __syncwarp();
           tmem_ld_32x32b_x32(t_row + c * 32, v);
           tmem_ld_wait();
 #pragma unroll
@@ -420,40 +691,39 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[acc]);
         __threadfence();
-        __syncwarp();
-        asm volatile("barrier.sync 1, 128;" ::: "memory");
+        epi_bar_sync();
         if (epi_tid == 0) {
-          const int prev = atomicAdd(&a.ws_ticket[tile], 1);
+          const int prev = atomicAdd(&a.ws_ticket[u.tile], 1);
           *last_flag = (prev == a.splits - 1);
         }
-        __syncwarp();
-        asm volatile("barrier.sync 1, 128;" ::: "memory");
+        epi_bar_sync();
         if (*last_flag) {
           __threadfence();
           const float *base =
-              a.ws_partial + (static_cast<int64_t>(tile) * a.splits * kBlockP + row) * BN;
+              a.ws_partial + (static_cast<int64_t>(u.tile) * a.splits * kBlockP + row) * BN;
 #pragma unroll 1
           for (int c = 0; c < BN / 32; ++c) {
             float f[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) f[j] = 0.0f;
-            for (int s = 0; s < a.splits; ++s) {
-              const float *src = base + static_cast<int64_t>(s) * kBlockP * BN + c * 32;
+            for (int sl = 0; sl < a.splits; ++sl) {
+              const float *src = base + static_cast<int64_t>(sl) * kBlockP * BN + c * 32;
+              float4 w[8];
 #pragma unroll
-              for (int j = 0; j < 32; j += 4) {
-                const float4 v = __ldcg(reinterpret_cast<const float4 *>(src + j));
-                f[j] += v.x;
-                f[j + 1] += v.y;
-                f[j + 2] += v.z;
-                f[j + 3] += v.w;
+              for (int j = 0; j < 8; ++j) w[j] = __ldcg(reinterpret_cast<const float4 *>(src) + j);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                f[4 * j] += w[j].x;
+                f[4 * j + 1] += w[j].y;
+                f[4 * j + 2] += w[j].z;
+                f[4 * j + 3] += w[j].w;
               }
             }
-            emit32<SWAP>(a, b, prow, tq * BN + c * 32, f);
+            emit32<SWAP>(a, u.b, prow, u.tq * BN + c * 32, f);
           }
-          if (epi_tid == 0) a.ws_ticket[tile] = 0;  // ready for the next call
+          if (epi_tid == 0) a.ws_ticket[u.tile] = 0;  // ready for the next call
         }
-        __syncwarp();
-        asm volatile("barrier.sync 1, 128;" ::: "memory");
+        epi_bar_sync();
       }
       if (++acc == ACC) {
         acc = 0;

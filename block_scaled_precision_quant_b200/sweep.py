@@ -1,0 +1,117 @@
+"""Schedule sweep for the block-scaled GEMM.
+
+For one problem shape, times every candidate schedule (bq_gemm_config) with
+CUDA-graph replay over rotating weight copies (more bytes than L2 holds, so
+weights stream from HBM) and prints one JSON line per candidate:
+
+    python -m block_scaled_precision_quant_b200.sweep M N K [kind] [--batch B]
+
+kind: mxfp4 (default), fp8blk32, mxfp8.  The built-in dispatch of bq_api.cu is
+derived from these measurements.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import sys
+
+import numpy as np
+
+
+def candidates(M, N, K):
+    import block_scaled_precision_quant_b200 as bq
+    out = []
+    if M <= 64:
+        for split in (1, 2, 4, 8):
+            modes = [bq.BQ_SPLIT_CLUSTER] if split > 1 else [bq.BQ_SPLIT_AUTO]
+            if split > 1:
+                modes.append(bq.BQ_SPLIT_WORKSPACE)
+            for mode in modes:
+                for kc in (1, 4):
+                    if kc > 1 and (K % 128 or mode == bq.BQ_SPLIT_WORKSPACE):
+                        continue
+                    out.append(bq.config(split_k=split, swap_ab=1, split_mode=mode, k_chunks=kc))
+    for bn in (128, 256):
+        for kc in (1, 2):
+            if kc > 1 and K % 128:
+                continue
+            out.append(bq.config(block_n=bn, split_k=1, swap_ab=0, k_chunks=kc))
+    return out
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("M", type=int)
+    ap.add_argument("N", type=int)
+    ap.add_argument("K", type=int)
+    ap.add_argument("kind", nargs="?", default="mxfp4")
+    ap.add_argument("--reps", type=int, default=20)
+    args = ap.parse_args(argv)
+    import torch
+    import block_scaled_precision_quant_b200 as bq
+    from block_scaled_precision_quant_b200 import synth
+    M, N, K = args.M, args.N, args.K
+    wk = {"mxfp4": bq.W_MXFP4, "fp8blk32": bq.W_FP8BLK32, "mxfp8": bq.W_MXFP8}[args.kind]
+    dev = torch.device("cuda")
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        x = torch.from_numpy(synth.activations(M, K, seed=1).view(np.int16)) \
+            .view(torch.bfloat16).to(dev)
+        aq, asf = bq.act_quant(x)
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        wbytes = N * K // 2 if wk == bq.W_MXFP4 else N * K
+        copies = max(1, min(64, int(np.ceil(2.5 * l2 / max(wbytes, 1)))))
+        ws = []
+        for c in range(copies):
+            if wk == bq.W_MXFP4:
+                b, s = synth.mxfp4_weight(N, K, seed=10 + c)
+                kind = bq.BQ_SF_ROW32
+            elif wk == bq.W_FP8BLK32:
+                b, s = synth.fp8_weight_blk32(N, K, seed=10 + c)
+                kind = bq.BQ_SF_BLK32x32
+            else:
+                b = synth.uniform_bytes((N, K), seed=10 + c, lo=0, hi=0x7E)
+                s = synth.uniform_bytes((N, K // 32), seed=20 + c, lo=118, hi=126)
+                kind = bq.BQ_SF_ROW32
+            bd = torch.from_numpy(b).to(dev)
+            ws.append((bd, bq.pack_weight_scales(torch.from_numpy(s).to(dev), kind, N, K)))
+        bias = torch.zeros(N, dtype=torch.bfloat16, device=dev)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        for cfg in candidates(M, N, K):
+            need = bq.workspace_bytes(wk, M, N, K, 1, cfg)
+            work = torch.zeros((max(need, 16),), dtype=torch.uint8, device=dev) if need else None
+            desc = dict(block_n=cfg.block_n, split_k=cfg.split_k, swap_ab=cfg.swap_ab,
+                        split_mode=cfg.split_mode, k_chunks=cfg.k_chunks)
+            try:
+                def run(c):
+                    bq.gemm(wk, aq, asf, ws[c][0], ws[c][1], M, N, K, y=y, bias=bias,
+                            config=cfg, workspace=work)
+                for c in range(copies):
+                    run(c)
+                torch.cuda.synchronize()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    for c in range(copies):
+                        run(c)
+                for _ in range(3):
+                    g.replay()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for _ in range(args.reps):
+                    g.replay()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                bq.device_status()
+                us = e0.elapsed_time(e1) * 1e3 / (args.reps * copies)
+                gbytes = (wbytes + N * K / 32 + M * K * 33 / 32 + 2 * M * N) / (us * 1e-6) / 1e9
+                print(json.dumps(dict(shape=[M, N, K], kind=args.kind, cfg=desc,
+                                      us=round(us, 3), tflops=round(2 * M * N * K / us / 1e6, 1),
+                                      gbs=round(gbytes, 1))), flush=True)
+            except bq.BqError as e:
+                print(json.dumps(dict(shape=[M, N, K], cfg=desc, error=str(e))), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -140,7 +140,13 @@ int bq_unpack_scales(const void *sf_mma, int64_t rows, int64_t K, void *rowmajor
  * y[m, n] = bf16_RNE(sum_k a[m,k] b[n,k]) with a, b the decoded operands
  * (code * 2^(scale-127)) and fp32 accumulation.
  * Errors: BQ_ERR_NULL, BQ_ERR_SHAPE, BQ_ERR_ALIGN, BQ_ERR_ARCH, BQ_ERR_CUDA.
- * No data is scanned on this path: NaN scales or codes give NaN outputs. */
+ * No data is scanned on this path: NaN scales or codes give NaN outputs.
+ * Launch order: the GEMM kernels (and bq_act_quant) use programmatic dependent
+ * launch -- a GEMM may start while the kernel just before it in the stream is
+ * still running.  It waits for that kernel before reading the activations,
+ * scales, bias or residual and before writing y, but it may read the weight
+ * operand b and b_sf early: they must not be written by the kernel issued
+ * immediately before the GEMM on the same stream (anything older has finished). */
 int bq_gemm_mxfp8_mxfp4(const void *a_q, const void *a_sf, const void *b_fp4, const void *b_sf,
                         int64_t M, int64_t N, int64_t K, void *y_bf16, bq_stream_t stream);
 int bq_gemm_mxfp8_fp8blk32(const void *a_q, const void *a_sf, const void *b_e4m3,
@@ -176,15 +182,26 @@ typedef struct {
 } bq_batch;
 
 /* Optional schedule override (tests and sweeps); NULL = built-in dispatch.
- * block_n: 0 (auto); 128 or 256 weight rows per CTA tile, or with swap_ab 32 or
- *          64 activation rows per CTA tile.
- * split_k: 0 (auto) or 1..16 slices of K (needs a workspace when > 1).
- * swap_ab: -1 (auto), 0, or 1 (weights on the 128-row MMA side, for M <= 64). */
+ * block_n:    0 (auto); 128 or 256 weight rows per CTA tile, or with swap_ab 32
+ *             or 64 activation rows per CTA tile.
+ * split_k:    0 (auto) or 1..16 slices of K.
+ * swap_ab:    -1 (auto), 0, or 1 (weights on the 128-row MMA side, for M <= 64).
+ * split_mode: how K slices are combined, always in slice order:
+ *             BQ_SPLIT_AUTO      cluster when possible, else workspace;
+ *             BQ_SPLIT_WORKSPACE fp32 partials in the caller's workspace, the
+ *                                last slice to finish reduces (needs workspace);
+ *             BQ_SPLIT_CLUSTER   the slices of a tile form a thread-block cluster
+ *                                and reduce through distributed shared memory
+ *                                (swap_ab tiles, split_k a power of two <= 8;
+ *                                no workspace). */
+enum { BQ_SPLIT_AUTO = 0, BQ_SPLIT_WORKSPACE = 1, BQ_SPLIT_CLUSTER = 2 };
 typedef struct {
   int block_n;
   int split_k;
   int swap_ab;
-  int reserved;
+  int split_mode;
+  int k_chunks; /* 128-K chunks per pipeline stage: 0 (auto), 1, 2 or (swap_ab) 4;
+                   more than 1 needs K % 128 == 0 and no workspace split */
 } bq_gemm_config;
 
 /* Workspace bytes the *_epilogue calls need for a problem (0 when the chosen

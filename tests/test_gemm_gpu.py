@@ -141,11 +141,21 @@ def test_pr1_reference_config():
     run_full(Case(bq.W_MXFP4, 64, 512, 1024, seed=0, act_gp=(-4, 4)))
 
 
+@pytest.mark.parametrize("k_chunks", [1, 2])
 @pytest.mark.parametrize("block_n", [128, 256])
 @pytest.mark.parametrize("wk", [bq.W_MXFP4, bq.W_FP8BLK32])
-def test_block_n_choices(block_n, wk):
-    run_full(Case(wk, 300, 520, 512, seed=3), config=bq.config(block_n=block_n, split_k=1,
-                                                                swap_ab=0))
+def test_block_n_choices(block_n, wk, k_chunks):
+    run_full(Case(wk, 300, 520, 640, seed=3), config=bq.config(block_n=block_n, split_k=1,
+                                                                swap_ab=0, k_chunks=k_chunks))
+
+
+@pytest.mark.parametrize("k_chunks", [1, 4])
+@pytest.mark.parametrize("M", [7, 41])
+def test_swap_k_chunks(M, k_chunks):
+    """Swap-AB tiles with one or four 128-K chunks per stage (K = 10 chunks:
+    the last stage is partial)."""
+    run_full(Case(bq.W_MXFP4, M, 384, 1280, seed=M + k_chunks, bias=True),
+             config=bq.config(split_k=1, swap_ab=1, k_chunks=k_chunks))
 
 
 # ------------------------------------------------------------- epilogues --
@@ -169,6 +179,34 @@ def test_decode_swap_split(M, split):
     run_full(c, config=bq.config(split_k=split, swap_ab=1))
 
 
+@pytest.mark.parametrize("M", [1, 17, 41, 64])
+@pytest.mark.parametrize("split", [2, 4, 8])
+def test_decode_cluster_split(M, split):
+    """K slices of a tile in one thread-block cluster, reduced through DSMEM."""
+    c = Case(bq.W_MXFP4, M, 640, 1536, seed=M + split, bias=True, residual=(split == 4))
+    cfg = bq.config(split_k=split, swap_ab=1, split_mode=bq.BQ_SPLIT_CLUSTER)
+    assert bq.workspace_bytes(bq.W_MXFP4, M, 640, 1536, 1, cfg) == 0
+    run_full(c, config=cfg)
+
+
+@pytest.mark.parametrize("wk", [bq.W_FP8BLK32, bq.W_MXFP8])
+def test_decode_cluster_split_fp8_weights(wk):
+    cfg = bq.config(split_k=8, swap_ab=1, split_mode=bq.BQ_SPLIT_CLUSTER)
+    run_full(Case(wk, 41, 384, 2048, seed=5, residual=True, alpha=0.5), config=cfg)
+
+
+def test_cluster_split_persistent_tiles():
+    """More clusters of work than fit at once: clusters loop over several tiles
+    (the partial buffer is reused after every peer finished reading it)."""
+    cfg = bq.config(split_k=8, swap_ab=1, split_mode=bq.BQ_SPLIT_CLUSTER)
+    run_full(Case(bq.W_MXFP4, 33, 8192, 1024, seed=8, bias=True), config=cfg)
+
+
+def test_decode_auto_plan_uses_no_workspace():
+    for N, K in ((4608, 1536), (6144, 1536), (1536, 6144)):
+        assert bq.workspace_bytes(bq.W_MXFP4, 41, N, K, 1) == 0
+
+
 @pytest.mark.parametrize("wk", [bq.W_FP8BLK32, bq.W_MXFP8])
 def test_decode_fp8_weights(wk):
     run_full(Case(wk, 41, 384, 1024, seed=2, residual=True), config=bq.config(swap_ab=1))
@@ -182,6 +220,13 @@ def test_decode_without_swap():
 def test_split_k_non_swap():
     run_full(Case(bq.W_FP8BLK32, 256, 384, 2048, seed=4, residual=True),
              config=bq.config(swap_ab=0, split_k=4, block_n=128))
+
+
+@pytest.mark.parametrize("M", [17, 41])
+def test_decode_workspace_split_balanced(M):
+    """Workspace split-K with a slice count that does not divide the K blocks."""
+    run_full(Case(bq.W_MXFP4, M, 640, 1536, seed=M + 1, bias=True),
+             config=bq.config(split_k=5, swap_ab=1, split_mode=bq.BQ_SPLIT_WORKSPACE))
 
 
 def test_split_k_repeatable():
@@ -255,15 +300,23 @@ def test_argument_errors():
     with pytest.raises(bq.BqError) as e:  # FP4 weights need K % 128 == 0
         bq.gemm(bq.W_MXFP4, aq, asf, bd, bsf, 16, 128, 96)
     assert e.value.status == bq.BQ_ERR_SHAPE
-    with pytest.raises(bq.BqError) as e:  # split-K without a workspace
+    c2 = Case(bq.W_MXFP4, 16, 128, 512)  # operands sized for K = 512 (4 K blocks)
+    aq2, asf2 = bq.act_quant(to_dev_bf16(c2.x))
+    bd2 = to_dev_u8(c2.b)
+    bsf2 = bq.pack_weight_scales(to_dev_u8(c2.bsf), bq.BQ_SF_ROW32, 128, 512)
+    with pytest.raises(bq.BqError) as e:  # workspace split-K without a workspace
         f = bq.lib().bq_gemm_mxfp8_mxfp4_epilogue
-        cfg = bq.config(split_k=2, swap_ab=1)
+        cfg = bq.config(split_k=2, swap_ab=1, split_mode=bq.BQ_SPLIT_WORKSPACE)
         import ctypes
-        st = f(aq.data_ptr(), asf.data_ptr(), bd.data_ptr(), bsf.data_ptr(), 16, 128, 256,
+        st = f(aq2.data_ptr(), asf2.data_ptr(), bd2.data_ptr(), bsf2.data_ptr(), 16, 128, 512,
                torch.empty((16, 128), dtype=torch.bfloat16, device="cuda").data_ptr(), None, None,
                None, 0, ctypes.byref(cfg), None)
         bq._check(st, "split without workspace")
-    assert e.value.status in (bq.BQ_ERR_WORKSPACE, bq.BQ_ERR_SHAPE)
+    assert e.value.status == bq.BQ_ERR_WORKSPACE
+    with pytest.raises(bq.BqError) as e:  # cluster split needs a power-of-two slice count
+        bq.gemm(bq.W_MXFP4, aq2, asf2, bd2, bsf2, 16, 128, 512,
+                config=bq.config(split_k=3, swap_ab=1, split_mode=bq.BQ_SPLIT_CLUSTER))
+    assert e.value.status == bq.BQ_ERR_INVALID
     with pytest.raises(bq.BqError) as e:  # invalid enum
         bq.gemm(bq.W_MXFP4, aq, asf, bd, bsf, 16, 128, 128, act=7)
     assert e.value.status == bq.BQ_ERR_INVALID
@@ -296,12 +349,14 @@ def test_workspace_shared_across_problems():
     """One workspace serves a sequence of split-K problems of different
     shapes; the ticket region is zero again after every call."""
     shapes = [(41, 640, 1536, 5), (17, 1536, 6144, 12), (64, 384, 1024, 3), (5, 4608, 1536, 4)]
-    need = max(bq.workspace_bytes(bq.W_MXFP4, M, N, K, 1, bq.config(split_k=s, swap_ab=1))
+    mode = bq.BQ_SPLIT_WORKSPACE
+    need = max(bq.workspace_bytes(bq.W_MXFP4, M, N, K, 1,
+                                  bq.config(split_k=s, swap_ab=1, split_mode=mode))
                for M, N, K, s in shapes)
     ws = torch.zeros((need,), dtype=torch.uint8, device="cuda")
     for i, (M, N, K, s) in enumerate(shapes * 2):
         c = Case(bq.W_MXFP4, M, N, K, seed=60 + i, bias=True)
-        y = c.gpu_with(config=bq.config(split_k=s, swap_ab=1), workspace=ws)
+        y = c.gpu_with(config=bq.config(split_k=s, swap_ab=1, split_mode=mode), workspace=ws)
         ref, sabs = c.oracle_full()
         assert_close(y, ref, c.tol(ref, sabs), f"shared workspace {M}x{N}x{K}/{s}")
         assert int(ws[:65536].count_nonzero().item()) == 0

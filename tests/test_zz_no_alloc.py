@@ -33,7 +33,7 @@ def _f64(y):
 def test_noalloc_matches_workspace_entry_twice():
     L = bq.lib()
     M, N, K = 41, 4608, 1536
-    cfg = bq.config(split_k=4, swap_ab=1)
+    cfg = bq.config(split_k=4, swap_ab=1, split_mode=bq.BQ_SPLIT_WORKSPACE)
     need = bq.workspace_bytes(bq.W_MXFP4, M, N, K, 1, cfg)
     assert 0 < need <= L.bq_noalloc_scratch_bytes()
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
@@ -75,7 +75,7 @@ def test_noalloc_matches_workspace_entry_twice():
 def test_noalloc_rejects_problems_beyond_the_scratch():
     L = bq.lib()
     M, N, K = 64, 16384, 4096
-    cfg = bq.config(split_k=16, swap_ab=1)
+    cfg = bq.config(split_k=16, swap_ab=1, split_mode=bq.BQ_SPLIT_WORKSPACE)
     assert bq.workspace_bytes(bq.W_MXFP4, M, N, K, 1, cfg) > L.bq_noalloc_scratch_bytes()
     dummy = torch.zeros((1 << 20,), dtype=torch.uint8, device="cuda")
     st = L.bq_gemm_mxfp8_mxfp4_epilogue_noalloc(
