@@ -265,8 +265,9 @@ def gemm(weight_kind, a_q, a_sf, b, b_sf, M, N, K, y=None, bias=None, residual=N
     if y is None:
         shape = (M, N) if batch is None else (count, M, N)
         y = torch.empty(shape, dtype=torch.bfloat16, device=a_q.device)
+    need = workspace_bytes(weight_kind, M, N, K, count, config)
     plain = (bias is None and residual is None and alpha == 1.0 and act == BQ_ACT_NONE
-             and batch is None and config is None and workspace is None)
+             and batch is None and config is None and workspace is None and need == 0)
     if plain:
         f = getattr(lib(), _ENTRY[weight_kind])
         _check(f(_ptr(a_q), _ptr(a_sf), _ptr(b), _ptr(b_sf), M, N, K, _ptr(y), _stream()),
@@ -279,7 +280,6 @@ def gemm(weight_kind, a_q, a_sf, b, b_sf, M, N, K, y=None, bias=None, residual=N
     if batch is not None:
         bt = Batch(count, *(int(batch.get(k, 0)) for k in (
             "stride_a", "stride_a_sf", "stride_b", "stride_b_sf", "stride_y", "stride_res")))
-    need = workspace_bytes(weight_kind, M, N, K, count, config)
     ws = workspace
     if need and ws is None:
         ws = _workspace(a_q.device, need)

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -195,12 +196,14 @@ int make_plan(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_conf
   }
   const int64_t tiles = batch * p->tiles_p * p->tiles_q;
   int splits = req_split;
+  const bool use_ws = req_mode == BQ_SPLIT_WORKSPACE;
   if (splits == 0) {
     splits = 1;
-    // Decode tiles: a cluster split pays one DSMEM exchange (~2-3 us of sync
-    // and skew), so it only wins when each tile has a long K loop (>= 24 K
-    // blocks, e.g. the 6144-deep down-projection): then spread it over a
-    // power-of-two cluster while the grid stays within one CTA per SM.
+    // Decode tiles (sweeps): up to ~12 K blocks an unsplit tile with 4-chunk
+    // stages is fastest -- a split pays ~3 us of exchange (fence, ticket and
+    // a gather through L2, or a DSMEM exchange), more than it saves.  With a
+    // long K loop (>= 24 K blocks) a power-of-two cluster split wins: spread
+    // it while the grid stays within one CTA per SM.
     if (p->swap && req_mode != BQ_SPLIT_WORKSPACE && p->kt_total >= 24) {
       while (splits * 2 <= kMaxClusterSplit && tiles * splits * 2 <= num_sms &&
              p->kt_total / (splits * 2) >= 4)
@@ -209,8 +212,7 @@ int make_plan(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_conf
   }
   if (splits > p->kt_total) splits = p->kt_total;
   const bool pow2 = (splits & (splits - 1)) == 0;
-  p->cluster = p->swap && splits > 1 && pow2 && splits <= kMaxClusterSplit &&
-               req_mode != BQ_SPLIT_WORKSPACE;
+  p->cluster = p->swap && splits > 1 && pow2 && splits <= kMaxClusterSplit && !use_ws;
   if (req_mode == BQ_SPLIT_CLUSTER && splits > 1 && !p->cluster) return BQ_ERR_INVALID;
   // K blocks are dealt out evenly: slice s covers [s*KT/S, (s+1)*KT/S), never empty.
   p->splits = splits;
@@ -248,13 +250,22 @@ size_t plan_ws_bytes(const Plan& p) {
   return kTicketRegion + p.ws_partial;
 }
 
+// The plan a call runs; one that needs more workspace than given is refused.
+int plan_for_call(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_config* cfg,
+                  int num_sms, const void* ws, size_t ws_bytes, Plan* p) {
+  const int st = make_plan(M, N, K, batch, cfg, num_sms, p);
+  if (st != BQ_OK) return st;
+  const size_t need = plan_ws_bytes(*p);
+  return (need == 0 || (ws && ws_bytes >= need)) ? BQ_OK : BQ_ERR_WORKSPACE;
+}
+
 // --------------------------------------------------------------- launches --
 
 template <int BN, int STAGES, int ACC, bool SWAP, bool P_FP4, bool Q_FP4, int MODE, int KC>
 int launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const bq::GemmArgs& args,
                 int64_t units, int num_sms, cudaStream_t stream) {
   constexpr bool CSPLIT = MODE == bq::kSplitCluster;
-  using L = bq::GemmSmem<BN, STAGES, ACC, CSPLIT, KC>;
+  using L = bq::KernelSmem<BN, STAGES, ACC, SWAP, MODE, KC>;
   auto kern = bq::gemm_bs_kernel<BN, STAGES, ACC, SWAP, P_FP4, Q_FP4, MODE, KC>;
   static bool attr_set[kMaxDevices] = {};
   static int per_sm_cache[kMaxDevices] = {};
@@ -289,6 +300,8 @@ int launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const bq::GemmArgs
   int na = 0;
   // May start while the preceding kernel (the activation quantizer) finishes:
   // prologue and weight loads overlap it; griddepcontrol.wait guards the rest.
+  // The kernel in turn releases its own dependents once every CTA is past that
+  // wait, so the next programmatic launch overlaps this one's mainloop.
   attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[na].val.programmaticStreamSerializationAllowed = 1;
   ++na;
@@ -390,15 +403,21 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
     if (sy == 0) return BQ_ERR_SHAPE;  // problems would overwrite each other
   }
   Plan pl;
-  st = make_plan(M, N, K, count, cfg, dev->num_sms, &pl);
+  st = plan_for_call(M, N, K, count, cfg, dev->num_sms, ws, ws_bytes, &pl);
   if (st != BQ_OK) return st;
   const size_t need = plan_ws_bytes(pl);
-  if (need > 0 && (!ws || ws_bytes < need || !aligned(ws, 16))) return BQ_ERR_WORKSPACE;
+  if (need > 0 && !aligned(ws, 16)) return BQ_ERR_WORKSPACE;
   if (get_encoder() != BQ_OK) return BQ_ERR_CUDA;
 
   // Tensor maps: activations A [M, K] (row stride K), weights B [N, K] or [N, K/2].
   CUtensorMap map_a, map_b;
-  const int a_box = pl.swap ? pl.bn : 128;
+  // Swap-AB with every activation row in one tile: the box ends at the last
+  // row (rounded up to 8), which copies far faster than a box whose trailing
+  // rows all fall outside the tensor.
+  const int a_box =
+      pl.swap ? (pl.tiles_q == 1 ? static_cast<int>(std::min<int64_t>(pl.bn, (M + 7) / 8 * 8))
+                                 : pl.bn)
+              : 128;
   const int b_box = pl.swap ? 128 : pl.bn;
   const bool a_batched = count > 1 && sa != 0;
   const bool b_batched = count > 1 && sb != 0;
@@ -422,6 +441,7 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
   g.raster_group = 8;
   g.sf_katoms = ceil_div(K, 128);
   g.sf_q_rowatoms = ceil_div(pl.swap ? M : N, 128);
+  g.q_box_rows = pl.swap ? a_box : b_box;
   g.split_lg = 0;
   while ((1 << g.split_lg) < pl.splits) ++g.split_lg;
   const uint8_t* sfa = static_cast<const uint8_t*>(a_sf);
@@ -670,15 +690,15 @@ int bq_gemm_mxfp8_mxfp4_epilogue_noalloc(const void* a_q, const void* a_sf, cons
   const int64_t count = batch ? batch->count : 1;
   if (M < 0 || N < 0 || K <= 0 || K % 32 != 0 || count < 0) return BQ_ERR_SHAPE;
   if (M == 0 || N == 0 || count == 0) return BQ_OK;
-  Plan pl;
-  st = make_plan(M, N, K, count, cfg, dev->num_sms, &pl);
-  if (st != BQ_OK) return st;
-  const size_t need = plan_ws_bytes(pl);
-  if (need > kNoAllocScratchBytes) return BQ_ERR_WORKSPACE;  // problem too large for the scratch
   void* scratch = nullptr;
-  if (need > 0) {
-    st = noalloc_scratch(&scratch);
-    if (st != BQ_OK) return st;
+  st = noalloc_scratch(&scratch);
+  if (st != BQ_OK) return st;
+  // Same planning as the call below makes with this scratch as its workspace
+  // (a schedule that needs more than the scratch is refused).
+  Plan pl;
+  st = plan_for_call(M, N, K, count, cfg, dev->num_sms, scratch, kNoAllocScratchBytes, &pl);
+  if (st != BQ_OK) return st;
+  if (plan_ws_bytes(pl) > 0) {
     // The scratch keeps whatever the previous call left: zero this call's
     // ticket counters before the kernel reads them.
     if (cudaMemsetAsync(scratch, 0, pl.ws_ticket, reinterpret_cast<cudaStream_t>(stream)) !=
@@ -686,7 +706,7 @@ int bq_gemm_mxfp8_mxfp4_epilogue_noalloc(const void* a_q, const void* a_sf, cons
       return BQ_ERR_CUDA;
   }
   return gemm_entry(kMxfp4, a_q, a_sf, b_fp4, b_sf, M, N, K, y_bf16, epi, batch, scratch,
-                    need > 0 ? kNoAllocScratchBytes : 0, cfg, stream);
+                    kNoAllocScratchBytes, cfg, stream);
 }
 
 size_t bq_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }

@@ -27,6 +27,7 @@ enum WaitSite : int {
   kWaitDrain = 5,          // MMA issuer draining before teardown
   kWaitPeerReady = 6,      // epilogue waiting for the cluster's partial tiles
   kWaitPeerDone = 7,       // epilogue waiting for the owners to free their receive buffers
+  kWaitLanding = 8,        // last K slice waiting for the other slices' partial tiles
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -253,6 +254,18 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
           "r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+// 16-byte asynchronous copy global -> shared through L2 (bypassing L1, so it
+// sees other SMs' stores that a device-scope fence has ordered before).
+__device__ __forceinline__ void cp_async_16(void *smem_dst, const void *gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
+               : "memory");
+}
+
+// Waits for every cp_async_16 this thread issued.
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05 --

@@ -41,7 +41,17 @@ constexpr int kBlockP = 128;  // MMA M
 constexpr int kBlockK = 128;  // inputs per stage: 128 one-byte codes = one 128B-swizzle row
 constexpr int kMmaK = 32;     // inputs per tcgen05.mma (one scale per row per MMA)
 constexpr int kSfAtom = 512;  // bytes of one 128-row x 4-column scale atom
-constexpr int kNumThreads = 192;
+// Warp roles: 0 weight-operand copies (and barrier set-up), 1 TMEM
+// allocation and MMA issue, 2-5 epilogue (one TMEM lane quadrant each),
+// 6 activation-operand copies, 7 weight-scale copies, 8 activation-scale
+// copies.  A thread issues about one copy per ~700 SM cycles whatever its
+// size, while an SM serves several issuing threads at once: four copy
+// threads, each arriving on every stage barrier with its own bytes.
+constexpr int kNumThreads = 288;
+constexpr int kActWarp = 6;
+constexpr int kWsfWarp = 7;
+constexpr int kAsfWarp = 8;
+constexpr int kCopyThreads = 4;
 
 // tcgen05 operand formats (instruction descriptor fields a_format / b_format).
 constexpr uint32_t kFmtE4M3 = 0;
@@ -58,6 +68,12 @@ struct GemmArgs {
   int sf_katoms;   // scale atoms along K = ceil(K / 128)
   int sf_q_rowatoms;  // 128-row scale bands of the Q-side operand = ceil(rows_q / 128)
   int split_lg;       // log2(splits) for cluster split-K
+  // Rows of the Q-side copy box (<= BN): when one Q tile covers all of a
+  // short operand, the box stops at the operand's last row rounded up to 8;
+  // the tile rows past it are never loaded and only feed output columns that
+  // are not stored.  A KC-chunk box lands as KC consecutive blocks of
+  // q_box_rows x 128 bytes.
+  int q_box_rows;
   // scale buffers (MMA layout) of the P- and Q-side operands, batch strides in bytes
   const uint8_t *sf_p;
   const uint8_t *sf_q;
@@ -85,7 +101,8 @@ enum SplitMode : int { kSplitNone = 0, kSplitWorkspace = 1, kSplitCluster = 2 };
 // 128 K (each chunk a 128B-swizzled K-major tile per operand) and the
 // chunks' scale-factor atoms; more bytes behind one stage barrier means fewer
 // barrier round trips per byte, which is what bounds a CTA's copy rate.
-template <int BN, int STAGES, int ACC, bool CSPLIT = false, int KC = 1>
+template <int BN, int STAGES, int ACC, bool CSPLIT = false, int KC = 1, bool OUT_STAGE = false,
+          bool LANDING = false>
 struct GemmSmem {
   static constexpr int kSfqAtoms = BN > 128 ? BN / 128 : 1;
   static constexpr int kSfqCols = 4 * kSfqAtoms;
@@ -105,8 +122,20 @@ struct GemmSmem {
   static constexpr int kRecvStride = BN + 4;
   static constexpr int kOffPart = kOffSfq + STAGES * kSfqBytes;
   static constexpr int kBytesPart = CSPLIT ? kBlockP * kRecvStride * 4 : 0;
-  static constexpr int kOffBar = kOffPart + kBytesPart;
-  static constexpr int kNumBars = 2 * STAGES + 2 * ACC + 1 + (CSPLIT ? 2 : 0);
+  // swap-AB output staging: the bf16 tile [BN rows m][128 columns n]
+  static constexpr int kOffOut = kOffPart + kBytesPart;
+  static constexpr int kBytesOut = OUT_STAGE ? BN * kBlockP * 2 : 0;
+  // swap-AB workspace split: this slice's fp32 partial tile [BN m][128 n],
+  // then the landing area for the other slices' partial tiles ([slice][m][128
+  // n], as many slices per round as fit)
+  static constexpr int kOffAcc = kOffOut + kBytesOut;
+  static constexpr int kBytesAcc = LANDING ? BN * kBlockP * 4 : 0;
+  static constexpr int kOffLand = kOffAcc + kBytesAcc;
+  static constexpr int kBytesLand = LANDING ? 64 * 1024 : 0;
+  static constexpr int kOffBiasS = kOffLand + kBytesLand;  // the tile's 128 biases (fp32)
+  static constexpr int kBytesBiasS = LANDING ? kBlockP * 4 : 0;
+  static constexpr int kOffBar = kOffBiasS + kBytesBiasS;
+  static constexpr int kNumBars = 2 * STAGES + 2 * ACC + 1 + (CSPLIT ? 2 : 0) + (LANDING ? 1 : 0);
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 64 + 1024;  // + alignment slack
   static constexpr int kTmemUsed = ACC * BN + STAGES * kSfCols;
@@ -118,6 +147,13 @@ struct GemmSmem {
   static_assert(kTmemUsed <= 512, "TMEM budget");
   static_assert(kBytes <= 232448, "shared memory budget");
 };
+
+// The layout a kernel instance uses: unsplit swap-AB tiles stage their bf16
+// output in shared memory for row-contiguous stores; swap-AB workspace splits
+// gather the slices' partial tiles in shared memory.
+template <int BN, int STAGES, int ACC, bool SWAP, int MODE, int KC>
+using KernelSmem = GemmSmem<BN, STAGES, ACC, MODE == kSplitCluster, KC,
+                            SWAP && MODE == kSplitNone, SWAP && MODE == kSplitWorkspace>;
 
 __device__ __forceinline__ uint32_t make_idesc(uint32_t fmt_p, uint32_t fmt_q, int bn, int sf_id) {
   uint32_t d = 0;
@@ -176,10 +212,11 @@ __device__ __forceinline__ float epi_value(const GemmArgs &a, float acc, float b
 }
 
 // Writes 32 accumulator values of one TMEM lane: row `prow` of the P side,
-// columns q0 .. q0+31 of the Q side, batch b.
+// columns q0 .. q0+31 of the Q side, batch b.  Swap-AB: `bias_swap` is the
+// bias of output column prow, fetched by the caller.
 template <bool SWAP>
 __device__ __forceinline__ void emit32(const GemmArgs &a, int b, int prow, int q0,
-                                       const float (&f)[32]) {
+                                       const float (&f)[32], float bias_swap) {
   if constexpr (!SWAP) {
     const int m = prow;
     if (m >= a.M) return;
@@ -226,7 +263,7 @@ __device__ __forceinline__ void emit32(const GemmArgs &a, int b, int prow, int q
     // bf16 per row; across the warp each row's store is 64 contiguous bytes.
     const int n = prow;
     if (n >= a.N || q0 >= a.M) return;
-    const float bias = a.bias ? __bfloat162float(a.bias[n]) : 0.0f;
+    const float bias = bias_swap;
     const int cnt = min(32, a.M - q0);
     __nv_bfloat16 *yp = a.y + b * a.y_bstride + static_cast<int64_t>(q0) * a.ldy + n;
     const int ldy = static_cast<int>(a.ldy);
@@ -254,54 +291,92 @@ __device__ __forceinline__ void epi_bar_sync() {
   asm volatile("barrier.sync 1, 128;" ::: "memory");  // the 4 epilogue warps
 }
 
-// Swap-AB output of 4 consecutive weight rows n..n+3 at activation row m
-// (y[m][n..n+3], 8-byte store); n % 4 == 0 and N % 8 == 0, so the group is
-// either fully inside the output or fully outside.
-__device__ __forceinline__ void emit4_swap(const GemmArgs &a, int b, int n, int m, float4 f) {
-  if (m >= a.M || n >= a.N) return;
-  float bias[4] = {0.f, 0.f, 0.f, 0.f}, res[4] = {0.f, 0.f, 0.f, 0.f};
-  if (a.bias) {
-    const uint2 v = *reinterpret_cast<const uint2 *>(a.bias + n);
-    bias[0] = bf16_bits_to_f32(v.x & 0xFFFF);
-    bias[1] = bf16_bits_to_f32(v.x >> 16);
-    bias[2] = bf16_bits_to_f32(v.y & 0xFFFF);
-    bias[3] = bf16_bits_to_f32(v.y >> 16);
+// Swap-AB epilogue, first half: the 32 values of output column n = prow
+// (rows m = q0 .. q0+31, tile columns c0 .. c0+31) become final bf16 values
+// in the staging tile stage[c][n - n0].  Across a warp each row is written as
+// 64 contiguous bytes.  The epilogue runs once per tile, so its code is
+// fetched cold: the bias-only case gets a short straight-line body.
+__device__ __forceinline__ void stage32_swap(const GemmArgs &a, int b, int prow, int nl, int q0,
+                                             int c0, const float (&f)[32], float bias,
+                                             __nv_bfloat16 *stage) {
+  __nv_bfloat16 *dst = stage + c0 * kBlockP + nl;
+  if (a.res == nullptr && a.act == 0) {
+    const float alpha = a.alpha;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) dst[j * kBlockP] = __float2bfloat16_rn(alpha * f[j] + bias);
+    return;
   }
-  if (a.res) {
-    const uint2 v = *reinterpret_cast<const uint2 *>(
-        a.res + b * a.res_bstride + static_cast<int64_t>(m) * a.ldres + n);
-    res[0] = bf16_bits_to_f32(v.x & 0xFFFF);
-    res[1] = bf16_bits_to_f32(v.x >> 16);
-    res[2] = bf16_bits_to_f32(v.y & 0xFFFF);
-    res[3] = bf16_bits_to_f32(v.y >> 16);
+  const __nv_bfloat16 *rcol =
+      a.res ? a.res + b * a.res_bstride + static_cast<int64_t>(q0) * a.ldres + prow : nullptr;
+#pragma unroll 1
+  for (int j = 0; j < 32; j += 8) {
+    float r[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      r[i] = (rcol && q0 + j + i < a.M)
+                 ? __bfloat162float(rcol[static_cast<int64_t>(j + i) * a.ldres])
+                 : 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      // f is indexed by a loop counter here; select the 8 values with a
+      // switch-free form the compiler keeps in registers.
+      float v = 0.0f;
+#pragma unroll
+      for (int t = 0; t < 32; t += 8)
+        if (t == j) v = f[t + i];
+      dst[(j + i) * kBlockP] = __float2bfloat16_rn(epi_value(a, v, bias, r[i]));
+    }
   }
-  const __nv_bfloat162 lo =
-      __floats2bfloat162_rn(epi_value(a, f.x, bias[0], res[0]), epi_value(a, f.y, bias[1], res[1]));
-  const __nv_bfloat162 hi =
-      __floats2bfloat162_rn(epi_value(a, f.z, bias[2], res[2]), epi_value(a, f.w, bias[3], res[3]));
-  uint2 o;
-  o.x = *reinterpret_cast<const uint32_t *>(&lo);
-  o.y = *reinterpret_cast<const uint32_t *>(&hi);
-  *reinterpret_cast<uint2 *>(a.y + b * a.y_bstride + static_cast<int64_t>(m) * a.ldy + n) = o;
 }
 
-// Cluster split-K reduction of one CTA's row slice, S = 2^LG slices.  The
-// slice is rows [split * 128/S, (split+1) * 128/S) of the tile; a thread owns
-// 4 consecutive rows (the same for every column it handles) and the columns
-// (epi_tid + 128 i) / quads.  All BN/4 DSMEM loads are issued before any sum;
-// each output is then summed in slice order 0..S-1.
-// Loads one operand side of one stage (KC chunks of 128 K starting at K
-// block kt, of which `nvalid` belong to the unit): the weights (P side with
-// SWAP, Q side otherwise) or the activations, each with its scale atoms.
-// KC == 1 uses 2-D (3-D batched) maps with the K offset in elements; KC > 1
-// uses maps that view K as (128, K/128 chunks), so one copy brings all chunks.
-template <int BN, int STAGES, int ACC, bool SWAP, bool CSPLIT, int KC>
-__device__ __forceinline__ void issue_half(const GemmArgs &a, const CUtensorMap *tm_p,
+// Final value of output y[m][n] (swap-AB element), general epilogue.
+__device__ __forceinline__ float swap_value(const GemmArgs &a, int b, int m, int n, float acc,
+                                            float bias) {
+  const float r =
+      a.res ? __bfloat162float(a.res[b * a.res_bstride + static_cast<int64_t>(m) * a.ldres + n])
+            : 0.0f;
+  return epi_value(a, acc, bias, r);
+}
+
+// Swap-AB epilogue, second half: the staged tile goes out as 16-byte vectors,
+// each row m of the tile as 256 contiguous bytes of y (N % 8 == 0 keeps every
+// vector wholly inside or outside the output).
+template <int BN>
+__device__ __forceinline__ void copy_out_swap(const GemmArgs &a, const UnitPos &u, int epi_tid,
+                                              const __nv_bfloat16 *stage) {
+  const int n0 = u.tp * kBlockP;
+  const int m0 = u.tq * BN;
+  const int rows = min(BN, a.M - m0);
+  const int nvec = min(kBlockP / 8, (a.N - n0) / 8);
+  __nv_bfloat16 *ybase = a.y + u.b * a.y_bstride + static_cast<int64_t>(m0) * a.ldy + n0;
+#pragma unroll 2
+  for (int i = epi_tid; i < rows * (kBlockP / 8); i += 128) {
+    const int r = i / (kBlockP / 8);
+    const int v = i % (kBlockP / 8);
+    if (v < nvec)
+      *reinterpret_cast<uint4 *>(ybase + static_cast<int64_t>(r) * a.ldy + v * 8) =
+          *reinterpret_cast<const uint4 *>(stage + r * kBlockP + v * 8);
+  }
+}
+
+// Loads one part of one stage (KC chunks of 128 K starting at K block kt, of
+// which `nvalid` belong to the unit): the operand tile or the scale atoms of
+// the P side or the Q side.  KC == 1 uses 2-D (3-D batched) maps with the K
+// offset in elements; KC > 1 uses maps that view K as (128, K/128 chunks), so
+// one copy brings all chunks.  Scale atoms of one 128-row band are contiguous
+// along K, so one bulk copy per band brings a stage's atoms.
+template <int BN, class L, int KC>
+__device__ __forceinline__ void issue_part(const GemmArgs &a, const CUtensorMap *tm_p,
                                            const CUtensorMap *tm_q, uint8_t *smem,
                                            uint64_t *full, int st, int kt, int nvalid,
-                                           const UnitPos &u, bool weights) {
-  using L = GemmSmem<BN, STAGES, ACC, CSPLIT, KC>;
-  if (weights == SWAP) {  // P side
+                                           const UnitPos &u, bool p_side, bool scales) {
+  if (p_side) {
+    if (scales) {
+      const uint8_t *sfp = a.sf_p + u.b * a.sf_p_bstride +
+                           (static_cast<int64_t>(u.tp) * a.sf_katoms + kt) * kSfAtom;
+      bulk_load(smem + L::kOffSfp + st * L::kSfpBytes, sfp, nvalid * kSfAtom, &full[st]);
+      return;
+    }
     uint8_t *dst = smem + st * L::kBytesP;
     const int row = u.tp * kBlockP;
     if constexpr (KC == 1) {
@@ -315,11 +390,22 @@ __device__ __forceinline__ void issue_half(const GemmArgs &a, const CUtensorMap 
       else
         tma_load_3d(dst, tm_p, &full[st], 0, row, kt);
     }
-    const uint8_t *sfp = a.sf_p + u.b * a.sf_p_bstride +
-                         (static_cast<int64_t>(u.tp) * a.sf_katoms + kt) * kSfAtom;
-    bulk_load(smem + L::kOffSfp + st * L::kSfpBytes, sfp, nvalid * kSfAtom, &full[st]);
-  } else {  // Q side
+  } else {
     const int q_row0 = u.tq * BN;
+    if (scales) {
+#pragma unroll
+      for (int j = 0; j < L::kSfqAtoms; ++j) {
+        // A band past the operand's last row would be outside the scale
+        // buffer; those rows are never stored, so any finite scale band
+        // serves -- reuse the last one.
+        const int band = min(q_row0 / 128 + j, a.sf_q_rowatoms - 1);
+        const uint8_t *sfq = a.sf_q + u.b * a.sf_q_bstride +
+                             (static_cast<int64_t>(band) * a.sf_katoms + kt) * kSfAtom;
+        bulk_load(smem + L::kOffSfq + st * L::kSfqBytes + j * KC * kSfAtom, sfq,
+                  nvalid * kSfAtom, &full[st]);
+      }
+      return;
+    }
     uint8_t *dst = smem + L::kOffQ + st * L::kBytesQ;
     if constexpr (KC == 1) {
       if (a.q_batched)
@@ -332,17 +418,6 @@ __device__ __forceinline__ void issue_half(const GemmArgs &a, const CUtensorMap 
       else
         tma_load_3d(dst, tm_q, &full[st], 0, q_row0, kt);
     }
-#pragma unroll
-    for (int j = 0; j < L::kSfqAtoms; ++j) {
-      // A band past the operand's last row would be outside the scale buffer;
-      // those rows are zero-filled by TMA, so any finite scale band serves --
-      // reuse the last one.
-      const int band = min(q_row0 / 128 + j, a.sf_q_rowatoms - 1);
-      const uint8_t *sfq = a.sf_q + u.b * a.sf_q_bstride +
-                           (static_cast<int64_t>(band) * a.sf_katoms + kt) * kSfAtom;
-      bulk_load(smem + L::kOffSfq + st * L::kSfqBytes + j * KC * kSfAtom, sfq, nvalid * kSfAtom,
-                &full[st]);
-    }
   }
 }
 
@@ -350,10 +425,12 @@ __device__ __forceinline__ void issue_half(const GemmArgs &a, const CUtensorMap 
 // (R = 128 / S) of the output tile and has received every slice's fp32
 // partial of those rows in its receive buffer.  A thread owns one row (the
 // same for every column group it handles), sums the S slices in slice order
-// and writes 4 columns (activation rows m) per group.
+// and writes 4 columns (activation rows m) per group; `bias` is that row's
+// bias, fetched by the caller.
 template <int BN, int LG>
 __device__ __forceinline__ void cluster_reduce_local(const GemmArgs &a, const UnitPos &u,
-                                                     int epi_tid, const float *recv) {
+                                                     int epi_tid, const float *recv,
+                                                     float bias) {
   constexpr int S = 1 << LG;
   constexpr int R = kBlockP >> LG;
   constexpr int kStride = BN + 4;
@@ -362,7 +439,6 @@ __device__ __forceinline__ void cluster_reduce_local(const GemmArgs &a, const Un
   const int rl = epi_tid % R;
   const int n = u.tp * kBlockP + u.split * R + rl;
   if (n >= a.N) return;
-  const float bias = a.bias ? __bfloat162float(a.bias[n]) : 0.0f;
 #pragma unroll
   for (int i = 0; i < kIters; ++i) {
     const int c4 = (epi_tid + 128 * i) / R;
@@ -398,7 +474,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   constexpr bool CSPLIT = MODE == kSplitCluster;
   static_assert(!CSPLIT || SWAP, "cluster split-K is built for the swap-AB (decode) tiles");
   static_assert(!CSPLIT || ACC == 1, "cluster split-K uses one accumulator");
-  using L = GemmSmem<BN, STAGES, ACC, CSPLIT, KC>;
+  using L = KernelSmem<BN, STAGES, ACC, SWAP, MODE, KC>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -413,6 +489,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   uint64_t *drain = tempty + ACC;
   uint64_t *peer_ready = drain + 1;  // CSPLIT: every slice's rows for this CTA have arrived
   uint64_t *peer_free = drain + 2;   // CSPLIT: every owner has consumed the previous tile
+  uint64_t *land_bar = drain + 1;    // workspace split: a round of partial tiles has landed
   float *recv = reinterpret_cast<float *>(smem + L::kOffPart);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
@@ -421,26 +498,27 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   const int total_units = a.batch * a.tiles_p * a.tiles_q * a.splits;
-  // Transaction bytes of a stage with `nv` chunks inside the unit.  The
-  // operand copies always move whole boxes (chunks past the tensor are zero
-  // filled); a 4-bit operand lands in shared memory with one byte-slot per
-  // code but counts its packed size (half the footprint).  Scale atoms are
-  // copied for the unit's chunks only.
-  auto tx_bytes = [](int nv) -> uint32_t {
-    return static_cast<uint32_t>((P_FP4 ? L::kBytesP / 2 : L::kBytesP) +
-                                 (Q_FP4 ? L::kBytesQ / 2 : L::kBytesQ) +
-                                 nv * (1 + L::kSfqAtoms) * kSfAtom);
+  // Transaction bytes one producer expects for its half of a stage with `nv`
+  // chunks inside the unit.  The operand copies always move whole boxes
+  // (chunks past the tensor are zero filled); a 4-bit operand lands in shared
+  // memory with one byte-slot per code but counts its packed size (half the
+  // footprint).  Scale atoms are copied for the unit's chunks only.
+  const int q_box_bytes = KC * a.q_box_rows * kBlockK;
+  auto tx_part = [q_box_bytes](int nv, bool p_side, bool scales) -> uint32_t {
+    if (scales) return static_cast<uint32_t>(nv * (p_side ? 1 : L::kSfqAtoms) * kSfAtom);
+    return p_side ? static_cast<uint32_t>(P_FP4 ? L::kBytesP / 2 : L::kBytesP)
+                  : static_cast<uint32_t>(Q_FP4 ? q_box_bytes / 2 : q_box_bytes);
   };
 
-  // Thread 0 (the producer) sets up the barriers and at once issues the weight
-  // half of the first unit's first stages: the weights do not depend on the
-  // kernel before this one in the stream, and these copies then overlap the
-  // TMEM allocation, the cluster barrier and (under programmatic dependent
+  // Thread 0 (the weight-operand copier) sets up the barriers and at once issues
+  // the weight tiles of the first unit's first stages: the weights do not depend on
+  // the kernel before this one in the stream, and these copies then overlap
+  // the TMEM allocation, the cluster barrier and (under programmatic dependent
   // launch) the tail of that kernel.
   int pre_n = 0;
   if (threadIdx.x == 0) {
     for (int st = 0; st < STAGES; ++st) {
-      mbar_init(&full[st], 1);
+      mbar_init(&full[st], kCopyThreads);  // one arrival per copy thread
       mbar_init(&empty[st], 1);
     }
     for (int st = 0; st < ACC; ++st) {
@@ -452,6 +530,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       mbar_init(peer_ready, a.splits);
       mbar_init(peer_free, a.splits);
     }
+    if constexpr (L::kBytesLand > 0) mbar_init(land_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_p);
@@ -462,9 +541,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       for (int j = 0; j < pre_n; ++j) {
         const int kt = u.kt0 + j * KC;
         const int nv = min(KC, u.kt1 - kt);
-        mbar_arrive_expect_tx(&full[j], tx_bytes(nv));
-        issue_half<BN, STAGES, ACC, SWAP, CSPLIT, KC>(a, &tm_p, &tm_q, smem, full, j, kt, nv, u,
-                                                      true);
+        mbar_arrive_expect_tx(&full[j], tx_part(nv, SWAP, false));
+        issue_part<BN, L, KC>(a, &tm_p, &tm_q, smem, full, j, kt, nv, u, SWAP, false);
       }
     }
   }
@@ -477,11 +555,21 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer --
+  if (warp == 0 || warp >= kActWarp) {
+    // ----------------------------------------------------------- producers --
+    // All four walk the same stage ring; each arrives once per stage with the
+    // bytes of its own part.  The weight copies never wait for the preceding
+    // kernel; the activation copies do, and once every CTA's activation-operand
+    // thread is past that wait the next kernel in the stream may launch (it,
+    // in turn, waits for this grid before reading its outputs).
     if (lane == 0) {
-      // Everything from here may read what the preceding kernel wrote.
-      griddep_wait();
+      const bool weights = warp == 0 || warp == kWsfWarp;
+      const bool scales = warp == kWsfWarp || warp == kAsfWarp;
+      const bool p_side = weights == SWAP;
+      if (!weights) {
+        griddep_wait();
+        if (!scales) griddep_launch_dependents();
+      }
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -489,28 +577,20 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       for (int unit = blockIdx.x; unit < total_units && ok; unit += gridDim.x) {
         const UnitPos u = unit_pos(a, unit);
         int kt = u.kt0;
-        if (first) {  // activation halves of the stages issued before the barrier
-          for (int j = 0; j < pre_n; ++j) {
-            const int kj = u.kt0 + j * KC;
-            issue_half<BN, STAGES, ACC, SWAP, CSPLIT, KC>(a, &tm_p, &tm_q, smem, full, j, kj,
-                                                          min(KC, u.kt1 - kj), u, false);
-          }
+        if (first && warp == 0) {  // stages whose weight tile went out before the barrier
           kt += pre_n * KC;
           stage = pre_n % STAGES;
           phase = pre_n == STAGES ? 1u : 0u;
-          first = false;
         }
+        first = false;
         for (; kt < u.kt1; kt += KC) {
           if (!mbar_wait(&empty[stage], phase ^ 1, a.err, abort_flag, kWaitProdEmpty)) {
             ok = false;
             break;
           }
           const int nv = min(KC, u.kt1 - kt);
-          mbar_arrive_expect_tx(&full[stage], tx_bytes(nv));
-          issue_half<BN, STAGES, ACC, SWAP, CSPLIT, KC>(a, &tm_p, &tm_q, smem, full, stage, kt, nv,
-                                                        u, true);
-          issue_half<BN, STAGES, ACC, SWAP, CSPLIT, KC>(a, &tm_p, &tm_q, smem, full, stage, kt, nv,
-                                                        u, false);
+          mbar_arrive_expect_tx(&full[stage], tx_part(nv, p_side, scales));
+          issue_part<BN, L, KC>(a, &tm_p, &tm_q, smem, full, stage, kt, nv, u, p_side, scales);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
@@ -532,6 +612,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       for (int unit = blockIdx.x; unit < total_units && ok; unit += gridDim.x) {
         const UnitPos u = unit_pos(a, unit);
         const uint32_t sfq_row_off = static_cast<uint32_t>((u.tq * BN) % 128) / 32;
+        const uint32_t q_chunk = static_cast<uint32_t>(a.q_box_rows * kBlockK);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1, a.err, abort_flag, kWaitMmaTmemEmpty)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
@@ -555,7 +636,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             for (int j = 0; j < L::kSfqAtoms; ++j)
               tc_cp_sf(sf_t + 4 + 4 * j, desc_sf_32x128b(sfq0 + (j * KC + c) * kSfAtom));
             const uint32_t pa = pa0 + c * L::kChunkP;
-            const uint32_t qa = qa0 + c * L::kChunkQ;
+            const uint32_t qa = qa0 + c * q_chunk;
 #pragma unroll
             for (int ks = 0; ks < kBlockK / kMmaK; ++ks) {
               const uint32_t idesc = make_idesc(P_FP4 ? kFmtE2M1 : kFmtE4M3,
@@ -590,15 +671,28 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     const int epi_tid = threadIdx.x - 64;  // 0..127
     int acc = 0;
     uint32_t acc_phase = 0;
-    uint32_t ready_phase = 0, free_phase = 0;
+    uint32_t ready_phase = 0, free_phase = 0, land_phase = 0;
     bool free_pending = false;  // CSPLIT: owners may still be reading the previous tile
+    // The bias and residual may come from the preceding kernel.
+    griddep_wait();
     for (int unit = blockIdx.x; unit < total_units; unit += gridDim.x) {
       const UnitPos u = unit_pos(a, unit);
+      const int prow = u.tp * kBlockP + row;
+      // Swap-AB: the output column (bias index) of this thread's row is known
+      // before the accumulator is; fetch its bias while the mainloop runs.
+      float bias_n = 0.0f;
+      if constexpr (SWAP) {
+        const int n = CSPLIT ? u.tp * kBlockP + u.split * (kBlockP >> a.split_lg) +
+                                   (epi_tid & ((kBlockP >> a.split_lg) - 1))
+                             : prow;
+        if (a.bias && n < a.N) bias_n = __bfloat162float(a.bias[n]);
+        if constexpr (L::kBytesBiasS > 0)
+          reinterpret_cast<float *>(smem + L::kOffBiasS)[row] = bias_n;
+      }
       __syncwarp();
       if (!mbar_wait(&tfull[acc], acc_phase, a.err, abort_flag, kWaitEpiFull)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + acc * BN + (static_cast<uint32_t>(quad * 32) << 16);
-      const int prow = u.tp * kBlockP + row;
       if constexpr (MODE == kSplitCluster) {
         // Cluster split-K: the S CTAs of this cluster hold the S K-slices of
         // one output tile.  Every CTA pushes each row of its fp32 partial
@@ -640,9 +734,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         if (!mbar_wait_cluster(peer_ready, ready_phase, a.err, abort_flag, kWaitPeerReady)) break;
         ready_phase ^= 1;
         switch (lg) {
-          case 1: cluster_reduce_local<BN, 1>(a, u, epi_tid, recv); break;
-          case 2: cluster_reduce_local<BN, 2>(a, u, epi_tid, recv); break;
-          default: cluster_reduce_local<BN, 3>(a, u, epi_tid, recv); break;
+          case 1: cluster_reduce_local<BN, 1>(a, u, epi_tid, recv, bias_n); break;
+          case 2: cluster_reduce_local<BN, 2>(a, u, epi_tid, recv, bias_n); break;
+          default: cluster_reduce_local<BN, 3>(a, u, epi_tid, recv, bias_n); break;
         }
         if (unit + static_cast<int>(gridDim.x) < total_units) {
           // another tile follows: release this CTA's receive buffer to the pushers
@@ -655,6 +749,29 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           }
           free_pending = true;
         }
+      } else if constexpr (MODE == kSplitNone && SWAP) {
+        // Stage the tile as bf16, release the accumulator, then write the
+        // tile row by row.
+        __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(smem + L::kOffOut);
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          const int q0 = u.tq * BN + c * 32;
+          if (q0 >= a.M) break;  // warp-uniform: the remaining columns are all past M
+          uint32_t v[32];
+          __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the stores
+          tmem_ld_32x32b_x32(t_row + c * 32, v);
+          tmem_ld_wait();
+          float f[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
+          if (prow < a.N) stage32_swap(a, u.b, prow, row, q0, c * 32, f, bias_n, stage);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
+        epi_bar_sync();
+        copy_out_swap<BN>(a, u, epi_tid, stage);
+        if (unit + static_cast<int>(gridDim.x) < total_units) epi_bar_sync();  // staging free
       } else if constexpr (MODE == kSplitNone) {
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
@@ -665,11 +782,145 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           float f[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
-          emit32<SWAP>(a, u.b, prow, u.tq * BN + c * 32, f);
+          emit32<SWAP>(a, u.b, prow, u.tq * BN + c * 32, f, bias_n);
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[acc]);
+      } else if constexpr (MODE == kSplitWorkspace && SWAP) {
+        // Split-K, swap-AB: publish this slice's fp32 partial (valid rows m
+        // only, stored [m][n] so a warp writes 128 contiguous bytes per m) and
+        // take a ticket.  The last slice of the tile to arrive sums all slices
+        // in slice order -- its own straight from TMEM -- and writes the tile
+        // through the staging buffer.
+        const int mt = min(BN, a.M - u.tq * BN);  // valid tile rows m
+        const int64_t slice_floats = static_cast<int64_t>(BN) * kBlockP;
+        const float *tile_ws = a.ws_partial + static_cast<int64_t>(u.tile) * a.splits * slice_floats;
+        float *mine = a.ws_partial + static_cast<int64_t>(unit) * slice_floats + row;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          const int q0 = c * 32;
+          if (q0 >= mt) break;  // warp-uniform
+          uint32_t v[32];
+          __syncwarp();
+          tmem_ld_32x32b_x32(t_row + c * 32, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (q0 + j < mt) __stcg(mine + (q0 + j) * kBlockP, __uint_as_float(v[j]));
+        }
+        epi_bar_sync();  // every partial store of this CTA is issued
+        if (epi_tid == 0) {
+          __threadfence();  // ... and visible device-wide before the ticket
+          const int prev = atomicAdd(&a.ws_ticket[u.tile], 1);
+          const int last = prev == a.splits - 1;
+          if (last) {
+            a.ws_ticket[u.tile] = 0;  // ready for the next call
+            __threadfence();          // the other slices' partials are visible from here
+          }
+          *last_flag = last;
+        }
+        epi_bar_sync();
+        if (*last_flag) {
+          // The other slices' partial tiles arrive by bulk copies (one per
+          // slice, as many per round as the landing area holds) while this
+          // slice's own partial goes from TMEM into shared memory in the same
+          // [m][n] layout.  Then every thread sums float4 groups of the tile
+          // (up to BN/4 of them, all loads independent) in slice order and
+          // writes them, 4 outputs of one row m per store.
+          float *land = reinterpret_cast<float *>(smem + L::kOffLand);
+          float *own = reinterpret_cast<float *>(smem + L::kOffAcc);
+          const int tile_floats = mt * kBlockP;
+          const int groups = mt * (kBlockP / 4);  // float4 groups of the tile
+          const int cap = L::kBytesLand / (tile_floats * 4);  // >= 2 (mt <= 64)
+          float4 r[BN / 4];
+#pragma unroll
+          for (int i = 0; i < BN / 4; ++i) r[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+          bool ok = true, dumped = false;
+#pragma unroll 1
+          for (int s0 = 0; s0 < a.splits && ok;) {
+            // slices [s0, s1) of this round hold `n` landed (other) slices
+            int s1 = s0, n = 0;
+            while (s1 < a.splits && (n < cap || s1 == u.split)) {
+              if (s1 != u.split) ++n;
+              ++s1;
+            }
+            if (n > 0 && epi_tid == 0) {
+              mbar_arrive_expect_tx(land_bar, static_cast<uint32_t>(n * tile_floats * 4));
+              int slot = 0;
+              for (int sl = s0; sl < s1; ++sl)
+                if (sl != u.split)
+                  bulk_load(land + (slot++) * tile_floats, tile_ws + sl * slice_floats,
+                            static_cast<uint32_t>(tile_floats * 4), land_bar);
+            }
+            if (!dumped) {
+#pragma unroll 1
+              for (int c = 0; c < BN / 32; ++c) {
+                if (c * 32 >= mt) break;  // warp-uniform
+                uint32_t v[32];
+                __syncwarp();
+                tmem_ld_32x32b_x32(t_row + c * 32, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (c * 32 + j < mt) own[(c * 32 + j) * kBlockP + row] = __uint_as_float(v[j]);
+              }
+              dumped = true;
+            }
+            epi_bar_sync();  // the own tile (and the biases) are in shared memory
+            if (n > 0) {
+              ok = mbar_wait(land_bar, land_phase, a.err, abort_flag, kWaitLanding);
+              land_phase ^= 1;
+            }
+            int slot = 0;
+#pragma unroll 1
+            for (int sl = s0; sl < s1 && ok; ++sl) {
+              const float4 *src = reinterpret_cast<const float4 *>(
+                  sl == u.split ? own : land + (slot++) * tile_floats);
+#pragma unroll
+              for (int i = 0; i < BN / 4; ++i) {
+                const int g = epi_tid + 128 * i;
+                if (g < groups) {
+                  const float4 w = src[g];
+                  r[i].x += w.x;
+                  r[i].y += w.y;
+                  r[i].z += w.z;
+                  r[i].w += w.w;
+                }
+              }
+            }
+            epi_bar_sync();  // the landing area is free for the next round
+            s0 = s1;
+          }
+          const float *bias_s = reinterpret_cast<const float *>(smem + L::kOffBiasS);
+          const bool lean = a.res == nullptr && a.act == 0;
+#pragma unroll
+          for (int i = 0; i < BN / 4; ++i) {
+            const int g = epi_tid + 128 * i;
+            const int m = g / (kBlockP / 4);
+            const int nl = (g % (kBlockP / 4)) * 4;
+            const int n = u.tp * kBlockP + nl;
+            if (g < groups && n < a.N) {
+              const float vals[4] = {r[i].x, r[i].y, r[i].z, r[i].w};
+              float o[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                o[j] = lean ? a.alpha * vals[j] + bias_s[nl + j]
+                            : swap_value(a, u.b, u.tq * BN + m, n + j, vals[j], bias_s[nl + j]);
+              const __nv_bfloat162 lo = __floats2bfloat162_rn(o[0], o[1]);
+              const __nv_bfloat162 hi = __floats2bfloat162_rn(o[2], o[3]);
+              uint2 pk;
+              pk.x = *reinterpret_cast<const uint32_t *>(&lo);
+              pk.y = *reinterpret_cast<const uint32_t *>(&hi);
+              *reinterpret_cast<uint2 *>(a.y + u.b * a.y_bstride +
+                                         static_cast<int64_t>(u.tq * BN + m) * a.ldy + n) = pk;
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
+        epi_bar_sync();  // last_flag and the shared tiles are free again
       } else {
         static_assert(MODE == kSplitWorkspace, "split mode");
         // Split-K: publish this slice's partial tile, then the last slice to
@@ -719,7 +970,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 f[4 * j + 3] += w[j].w;
               }
             }
-            emit32<SWAP>(a, u.b, prow, u.tq * BN + c * 32, f);
+            emit32<SWAP>(a, u.b, prow, u.tq * BN + c * 32, f, bias_n);
           }
           if (epi_tid == 0) a.ws_ticket[u.tile] = 0;  // ready for the next call
         }

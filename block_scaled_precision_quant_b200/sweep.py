@@ -22,15 +22,19 @@ def candidates(M, N, K):
     import block_scaled_precision_quant_b200 as bq
     out = []
     if M <= 64:
-        for split in (1, 2, 4, 8):
-            modes = [bq.BQ_SPLIT_CLUSTER] if split > 1 else [bq.BQ_SPLIT_AUTO]
-            if split > 1:
-                modes.append(bq.BQ_SPLIT_WORKSPACE)
-            for mode in modes:
-                for kc in (1, 4):
-                    if kc > 1 and (K % 128 or mode == bq.BQ_SPLIT_WORKSPACE):
-                        continue
-                    out.append(bq.config(split_k=split, swap_ab=1, split_mode=mode, k_chunks=kc))
+        kt = (K + 127) // 128
+        for kc in (1, 4):
+            if kc == 1 or K % 128 == 0:
+                out.append(bq.config(split_k=1, swap_ab=1, k_chunks=kc))
+        for split in (2, 4, 8):
+            for kc in (1, 4):
+                if split <= kt and (kc == 1 or K % 128 == 0):
+                    out.append(bq.config(split_k=split, swap_ab=1, split_mode=bq.BQ_SPLIT_CLUSTER,
+                                         k_chunks=kc))
+        for split in (2, 3, 4, 6, 8, 12, 16):
+            if split <= kt:
+                out.append(bq.config(split_k=split, swap_ab=1, split_mode=bq.BQ_SPLIT_WORKSPACE,
+                                     k_chunks=1))
     for bn in (128, 256):
         for kc in (1, 2):
             if kc > 1 and K % 128:

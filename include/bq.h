@@ -146,7 +146,10 @@ int bq_unpack_scales(const void *sf_mma, int64_t rows, int64_t K, void *rowmajor
  * still running.  It waits for that kernel before reading the activations,
  * scales, bias or residual and before writing y, but it may read the weight
  * operand b and b_sf early: they must not be written by the kernel issued
- * immediately before the GEMM on the same stream (anything older has finished). */
+ * immediately before the GEMM on the same stream (anything older has finished).
+ * Once all its thread blocks are past that wait, a GEMM lets the next kernel
+ * of the stream launch if that kernel was launched programmatically (as this
+ * library's are); such a kernel waits for the GEMM before touching its output. */
 int bq_gemm_mxfp8_mxfp4(const void *a_q, const void *a_sf, const void *b_fp4, const void *b_sf,
                         int64_t M, int64_t N, int64_t K, void *y_bf16, bq_stream_t stream);
 int bq_gemm_mxfp8_fp8blk32(const void *a_q, const void *a_sf, const void *b_e4m3,

@@ -207,6 +207,23 @@ def test_decode_auto_plan_uses_no_workspace():
         assert bq.workspace_bytes(bq.W_MXFP4, 41, N, K, 1) == 0
 
 
+@pytest.mark.parametrize("M", [1, 17, 41, 64])
+@pytest.mark.parametrize("split", [2, 3, 4, 12])
+def test_decode_swap_workspace_split(M, split):
+    """Swap-AB split-K through the workspace: partial rows m < M only, the
+    last slice sums all slices in slice order (its own from TMEM)."""
+    c = Case(bq.W_MXFP4, M, 640, 1536, seed=M + 7 * split, bias=True,
+             residual=(split == 3), act=bq.BQ_ACT_GELU if split == 4 else bq.BQ_ACT_NONE)
+    run_full(c, config=bq.config(split_k=split, swap_ab=1, split_mode=bq.BQ_SPLIT_WORKSPACE))
+
+
+def test_workspace_split_persistent_tiles():
+    """More split units than CTAs: each CTA walks several tiles, reusing its
+    staging buffer and ticket flag."""
+    cfg = bq.config(split_k=4, swap_ab=1, split_mode=bq.BQ_SPLIT_WORKSPACE)
+    run_full(Case(bq.W_MXFP4, 33, 8192, 1024, seed=18, bias=True), config=cfg)
+
+
 @pytest.mark.parametrize("wk", [bq.W_FP8BLK32, bq.W_MXFP8])
 def test_decode_fp8_weights(wk):
     run_full(Case(wk, 41, 384, 1024, seed=2, residual=True), config=bq.config(swap_ab=1))
