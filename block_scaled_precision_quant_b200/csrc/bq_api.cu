@@ -182,13 +182,18 @@ int make_plan(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_conf
     if (req_bn) {
       p->bn = req_bn;
     } else {
-      // Wave model from the schedule sweeps: a 128x256 tile does the work of
-      // two 128x128 tiles in ~0.82x their time; pick the width whose waves of
-      // persistent CTAs finish first.
+      // Wave model fitted to the schedule sweeps (in units of one 128x256
+      // K-block step): a 128x128 tile takes 0.61 of that per K block, and a
+      // 128x256 tile, whose single TMEM accumulator leaves its epilogue
+      // unoverlapped, pays ~7 units of epilogue per tile; 128x128 tiles keep
+      // two accumulators and expose only the last epilogue.  Pick the width
+      // whose waves of persistent CTAs finish first.
       const int64_t t256 = batch * p->tiles_p * ceil_div(N, 256);
       const int64_t t128 = batch * p->tiles_p * ceil_div(N, 128);
-      const double c256 = static_cast<double>((t256 + num_sms - 1) / num_sms) * 256.0;
-      const double c128 = static_cast<double>((t128 + num_sms - 1) / num_sms) * 128.0 / 0.82;
+      const double kt = static_cast<double>(ceil_div(K, 128));
+      const double c256 = static_cast<double>((t256 + num_sms - 1) / num_sms) * (kt + 7.0);
+      const double c128 =
+          static_cast<double>((t128 + num_sms - 1) / num_sms) * kt * 0.61 + 3.5;
       p->bn = (N > 128 && c256 <= c128) ? 256 : 128;
     }
     if (p->bn != 128 && p->bn != 256) return BQ_ERR_INVALID;

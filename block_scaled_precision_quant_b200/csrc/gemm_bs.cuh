@@ -193,10 +193,11 @@ __device__ __forceinline__ UnitPos unit_pos(const GemmArgs &a, int unit) {
   return u;
 }
 
-// erf-form GELU.  Kept out of line: the epilogue is unrolled over many
-// values, and inlining erff at every one of them would bloat the straight-line
-// code every call fetches, GELU or not.
-__device__ __noinline__ float gelu_erf(float t) {
+// erf-form GELU, inline: an out-of-line call per element costs the unrolled
+// epilogue its registers at every call and dominated GELU layers.  Callers
+// branch on the activation once per group of values, so code without GELU
+// never runs through it.
+__device__ __forceinline__ float gelu_erf(float t) {
   return 0.5f * t * (1.0f + erff(t * 0.70710678118654752f));
 }
 
@@ -248,12 +249,18 @@ __device__ __forceinline__ void emit32(const GemmArgs &a, int b, int prow, int q
           res8[2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
         }
       }
+      float t[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) t[j] = a.alpha * f[8 * g + j] + bias8[j];
+      if (a.act == 1) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) t[j] = gelu_erf(t[j]);
+      }
       uint32_t o[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float lo = epi_value(a, f[8 * g + 2 * j], bias8[2 * j], res8[2 * j]);
-        const float hi = epi_value(a, f[8 * g + 2 * j + 1], bias8[2 * j + 1], res8[2 * j + 1]);
-        const __nv_bfloat162 p2 = __floats2bfloat162_rn(lo, hi);
+        const __nv_bfloat162 p2 = __floats2bfloat162_rn(t[2 * j] + res8[2 * j],
+                                                        t[2 * j + 1] + res8[2 * j + 1]);
         o[j] = *reinterpret_cast<const uint32_t *>(&p2);
       }
       *reinterpret_cast<uint4 *>(yrow + n) = make_uint4(o[0], o[1], o[2], o[3]);

@@ -4,10 +4,11 @@ For one problem shape, times every candidate schedule (bq_gemm_config) with
 CUDA-graph replay over rotating weight copies (more bytes than L2 holds, so
 weights stream from HBM) and prints one JSON line per candidate:
 
-    python -m block_scaled_precision_quant_b200.sweep M N K [kind] [--batch B]
+    python -m block_scaled_precision_quant_b200.sweep M N K [kind] [--batch B] [--gelu]
 
-kind: mxfp4 (default), fp8blk32, mxfp8.  The built-in dispatch of bq_api.cu is
-derived from these measurements.
+kind: mxfp4 (default), fp8blk32, mxfp8.  --batch B runs B independent problems
+over one broadcast weight (batch stride 0), --gelu adds bias + GELU.  The
+built-in dispatch of bq_api.cu is derived from these measurements.
 """
 from __future__ import annotations
 
@@ -50,18 +51,28 @@ def main(argv=None):
     ap.add_argument("K", type=int)
     ap.add_argument("kind", nargs="?", default="mxfp4")
     ap.add_argument("--reps", type=int, default=20)
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--gelu", action="store_true")
     args = ap.parse_args(argv)
     import torch
     import block_scaled_precision_quant_b200 as bq
     from block_scaled_precision_quant_b200 import synth
-    M, N, K = args.M, args.N, args.K
+    M, N, K, B = args.M, args.N, args.K, args.batch
     wk = {"mxfp4": bq.W_MXFP4, "fp8blk32": bq.W_FP8BLK32, "mxfp8": bq.W_MXFP8}[args.kind]
     dev = torch.device("cuda")
     stream = torch.cuda.Stream()
     with torch.cuda.stream(stream):
-        x = torch.from_numpy(synth.activations(M, K, seed=1).view(np.int16)) \
-            .view(torch.bfloat16).to(dev)
-        aq, asf = bq.act_quant(x)
+        aqs, asfs = [], []
+        for b in range(B):
+            x = torch.from_numpy(synth.activations(M, K, seed=1 + b).view(np.int16)) \
+                .view(torch.bfloat16).to(dev)
+            q, f = bq.act_quant(x)
+            aqs.append(q)
+            asfs.append(f)
+        aq = torch.stack(aqs).reshape(B * M, K)
+        asf = torch.stack(asfs)
+        batch = None if B == 1 else dict(count=B, stride_a=M * K, stride_a_sf=asf.shape[1],
+                                         stride_b=0, stride_b_sf=0, stride_y=M * N * 2)
         l2 = torch.cuda.get_device_properties(dev).L2_cache_size
         wbytes = N * K // 2 if wk == bq.W_MXFP4 else N * K
         copies = max(1, min(64, int(np.ceil(2.5 * l2 / max(wbytes, 1)))))
@@ -79,17 +90,18 @@ def main(argv=None):
                 kind = bq.BQ_SF_ROW32
             bd = torch.from_numpy(b).to(dev)
             ws.append((bd, bq.pack_weight_scales(torch.from_numpy(s).to(dev), kind, N, K)))
-        bias = torch.zeros(N, dtype=torch.bfloat16, device=dev)
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        bias = torch.from_numpy(synth.bias(N, seed=3).view(np.int16)).view(torch.bfloat16).to(dev)
+        y = torch.empty((B, M, N) if B > 1 else (M, N), dtype=torch.bfloat16, device=dev)
+        act = bq.BQ_ACT_GELU if args.gelu else bq.BQ_ACT_NONE
         for cfg in candidates(M, N, K):
-            need = bq.workspace_bytes(wk, M, N, K, 1, cfg)
+            need = bq.workspace_bytes(wk, M, N, K, B, cfg)
             work = torch.zeros((max(need, 16),), dtype=torch.uint8, device=dev) if need else None
             desc = dict(block_n=cfg.block_n, split_k=cfg.split_k, swap_ab=cfg.swap_ab,
                         split_mode=cfg.split_mode, k_chunks=cfg.k_chunks)
             try:
                 def run(c):
                     bq.gemm(wk, aq, asf, ws[c][0], ws[c][1], M, N, K, y=y, bias=bias,
-                            config=cfg, workspace=work)
+                            act=act, batch=batch, config=cfg, workspace=work)
                 for c in range(copies):
                     run(c)
                 torch.cuda.synchronize()
@@ -108,9 +120,10 @@ def main(argv=None):
                 torch.cuda.synchronize()
                 bq.device_status()
                 us = e0.elapsed_time(e1) * 1e3 / (args.reps * copies)
-                gbytes = (wbytes + N * K / 32 + M * K * 33 / 32 + 2 * M * N) / (us * 1e-6) / 1e9
-                print(json.dumps(dict(shape=[M, N, K], kind=args.kind, cfg=desc,
-                                      us=round(us, 3), tflops=round(2 * M * N * K / us / 1e6, 1),
+                gbytes = (wbytes + N * K / 32 + B * (M * K * 33 / 32 + 2 * M * N)) / (us * 1e-6) / 1e9
+                print(json.dumps(dict(shape=[M, N, K], batch=B, gelu=args.gelu, kind=args.kind,
+                                      cfg=desc, us=round(us, 3),
+                                      tflops=round(2 * B * M * N * K / us / 1e6, 1),
                                       gbs=round(gbytes, 1))), flush=True)
             except bq.BqError as e:
                 print(json.dumps(dict(shape=[M, N, K], cfg=desc, error=str(e))), flush=True)
