@@ -68,7 +68,8 @@ class Batch(ctypes.Structure):
 
 class GemmConfig(ctypes.Structure):
     _fields_ = [("block_n", ctypes.c_int), ("split_k", ctypes.c_int), ("swap_ab", ctypes.c_int),
-                ("split_mode", ctypes.c_int), ("k_chunks", ctypes.c_int)]
+                ("split_mode", ctypes.c_int), ("k_chunks", ctypes.c_int),
+                ("cta_pair", ctypes.c_int)]
 
 
 _lib = None
@@ -231,8 +232,9 @@ _ENTRY = {W_MXFP4: "bq_gemm_mxfp8_mxfp4", W_FP8BLK32: "bq_gemm_mxfp8_fp8blk32",
           W_MXFP8: "bq_gemm_mxfp8_mxfp8"}
 
 
-def _config(block_n=0, split_k=0, swap_ab=-1, split_mode=0, k_chunks=0):
-    return GemmConfig(int(block_n), int(split_k), int(swap_ab), int(split_mode), int(k_chunks))
+def _config(block_n=0, split_k=0, swap_ab=-1, split_mode=0, k_chunks=0, cta_pair=0):
+    return GemmConfig(int(block_n), int(split_k), int(swap_ab), int(split_mode), int(k_chunks),
+                      int(cta_pair))
 
 
 def workspace_bytes(weight_kind, M, N, K, batch=1, config=None) -> int:

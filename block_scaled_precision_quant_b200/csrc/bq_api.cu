@@ -12,6 +12,7 @@
 #include "act_quant.cuh"
 #include "bq.h"
 #include "gemm_bs.cuh"
+#include "gemm_pair.cuh"
 
 namespace {
 
@@ -134,12 +135,33 @@ int make_operand_map(CUtensorMap* m, const void* base, bool fp4, int64_t K, int6
   return r == CUDA_SUCCESS ? BQ_OK : BQ_ERR_ALIGN;
 }
 
+// A scale buffer (MMA layout: 128-row bands of K-block atoms, 512 bytes each)
+// viewed as (128 words, K blocks, bands[, batch]); a box is `kc` consecutive
+// atoms of `bands_box` bands.
+int make_scale_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int64_t batch,
+                   int64_t batch_bytes, int kc, int bands_box) {
+  const int64_t katoms = (K + 127) / 128;
+  const int64_t bands = (rows + 127) / 128;
+  cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(katoms), static_cast<cuuint64_t>(bands),
+                        static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[3] = {512, static_cast<cuuint64_t>(katoms * 512),
+                           static_cast<cuuint64_t>(batch_bytes)};
+  cuuint32_t box[4] = {128u, static_cast<cuuint32_t>(kc), static_cast<cuuint32_t>(bands_box), 1u};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, batch > 1 ? 4 : 3,
+                        const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? BQ_OK : BQ_ERR_ALIGN;
+}
+
 // ---------------------------------------------------------------- schedule --
 
 enum WeightKind { kMxfp4 = 0, kFp8Blk32 = 1, kMxfp8 = 2 };
 
 struct Plan {
   bool swap = false;
+  bool pair = false;     // 256x256 tiles on CTA pairs (cta_group::2 MMA)
   int kc = 1;            // 128-K chunks per pipeline stage
   bool cluster = false;  // K slices reduced through DSMEM inside a thread-block cluster
   int bn = 256;
@@ -169,6 +191,8 @@ int make_plan(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_conf
   if (req_mode < BQ_SPLIT_AUTO || req_mode > BQ_SPLIT_CLUSTER) return BQ_ERR_INVALID;
   const int req_kc = cfg ? cfg->k_chunks : 0;
   if (req_kc < 0 || req_kc > 4 || req_kc == 3) return BQ_ERR_INVALID;
+  const int req_pair = cfg ? cfg->cta_pair : 0;
+  if (req_pair < 0 || req_pair > 2) return BQ_ERR_INVALID;
   p->kt_total = ceil_div(K, 128);
   p->swap = req_swap == 1 || (req_swap == -1 && M <= 64);
   if (p->swap) {
@@ -219,6 +243,26 @@ int make_plan(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_conf
   const bool pow2 = (splits & (splits - 1)) == 0;
   p->cluster = p->swap && splits > 1 && pow2 && splits <= kMaxClusterSplit && !use_ws;
   if (req_mode == BQ_SPLIT_CLUSTER && splits > 1 && !p->cluster) return BQ_ERR_INVALID;
+  // 256x256 pair tiles (sweeps: +3-8 % over the best single-SM tile once a
+  // tile's K loop is >= 32 blocks and the pairs fill the SMs; shorter loops
+  // lose to 128x128 tiles, whose two accumulators hide the epilogue).
+  const bool auto_pair = req_pair == 0 && req_bn == 0 && req_split <= 1 && req_kc != 4 &&
+                         !p->swap && splits == 1 && p->kt_total >= 32 &&
+                         5 * batch * ceil_div(M, 256) * ceil_div(N, 256) >= 2 * num_sms;
+  if (req_pair == 2 || auto_pair) {  // 256x256 tiles on CTA pairs: wide tiles, no split
+    if (p->swap || splits != 1 || (req_bn != 0 && req_bn != 256)) return BQ_ERR_INVALID;
+    if (req_kc > 2 || (req_kc == 2 && K % 128 != 0)) return BQ_ERR_INVALID;
+    p->pair = true;
+    p->bn = 256;
+    p->tiles_p = ceil_div(M, 256);
+    p->tiles_q = ceil_div(N, 256);
+    p->splits = 1;
+    p->kt_per_split = p->kt_total;
+    p->units = batch * p->tiles_p * p->tiles_q;
+    if (p->units > 0x7FFFFFFF) return BQ_ERR_SHAPE;
+    p->kc = req_kc ? req_kc : (K % 128 == 0 ? 2 : 1);
+    return BQ_OK;
+  }
   // K blocks are dealt out evenly: slice s covers [s*KT/S, (s+1)*KT/S), never empty.
   p->splits = splits;
   p->kt_per_split = ceil_div(p->kt_total, splits);
@@ -335,6 +379,48 @@ int launch_kind(bool w_fp4, const CUtensorMap& tp, const CUtensorMap& tq,
   return launch_gemm<BN, STAGES, ACC, SWAP, false, false, MODE, KC>(tp, tq, args, u, num_sms, st);
 }
 
+template <int STAGES, int KC, bool Q_FP4>
+int launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
+                const CUtensorMap& tsb, const bq::GemmArgs& args, int64_t units, int num_sms,
+                cudaStream_t stream) {
+  using L = bq::PairSmem<STAGES, KC>;
+  auto kern = bq::gemm_pair_kernel<STAGES, KC, Q_FP4>;
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+      return BQ_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  // One CTA per SM (shared memory and TMEM), so at most num_sms / 2 pairs.
+  int64_t pairs = num_sms / 2;
+  if (pairs > units) pairs = units;
+  if (pairs < 1) pairs = 1;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+  lc.blockDim = dim3(bq::kNumThreads);
+  lc.dynamicSmemBytes = L::kBytes;
+  lc.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 2;
+  if (cudaLaunchKernelEx(&lc, kern, ta, tb, tsa, tsb, args) != cudaSuccess) {
+    cudaGetLastError();
+    return BQ_ERR_CUDA;
+  }
+  return launch_status();
+}
+
 // Dispatch on (swap, bn, chunks per stage, split mode, fp4 weights) to the
 // compiled instances.  Stage counts fill ~200 KB of shared memory.
 int run_gemm(const Plan& pl, bool w_fp4, const CUtensorMap& tp, const CUtensorMap& tq,
@@ -423,7 +509,7 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
       pl.swap ? (pl.tiles_q == 1 ? static_cast<int>(std::min<int64_t>(pl.bn, (M + 7) / 8 * 8))
                                  : pl.bn)
               : 128;
-  const int b_box = pl.swap ? 128 : pl.bn;
+  const int b_box = (pl.swap || pl.pair) ? 128 : pl.bn;  // a pair CTA loads 128 of 256 rows
   const bool a_batched = count > 1 && sa != 0;
   const bool b_batched = count > 1 && sb != 0;
   st = make_operand_map(&map_a, a_q, false, K, M, K, a_batched ? count : 1, sa, a_box, pl.kc);
@@ -471,6 +557,21 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
     g.ws_partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kTicketRegion);
   }
   g.err = dev->err_ptr;
+  if (pl.pair) {
+    CUtensorMap map_sfa, map_sfb;
+    st = make_scale_map(&map_sfa, a_sf, M, K, a_batched ? count : 1, ssa, pl.kc, 1);
+    if (st != BQ_OK) return st;
+    st = make_scale_map(&map_sfb, b_sf, N, K, b_batched ? count : 1, ssb, pl.kc, 2);
+    if (st != BQ_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t u = pl.units;
+    const int ns = dev->num_sms;
+    if (pl.kc == 2)
+      return w_fp4 ? launch_pair<3, 2, true>(map_a, map_b, map_sfa, map_sfb, g, u, ns, s)
+                   : launch_pair<3, 2, false>(map_a, map_b, map_sfa, map_sfb, g, u, ns, s);
+    return w_fp4 ? launch_pair<6, 1, true>(map_a, map_b, map_sfa, map_sfb, g, u, ns, s)
+                 : launch_pair<6, 1, false>(map_a, map_b, map_sfa, map_sfb, g, u, ns, s);
+  }
   const CUtensorMap& tp = pl.swap ? map_b : map_a;
   const CUtensorMap& tq = pl.swap ? map_a : map_b;
   return run_gemm(pl, w_fp4, tp, tq, g, dev->num_sms, reinterpret_cast<cudaStream_t>(stream));
@@ -595,7 +696,7 @@ int bq_unpack_scales(const void* sf_mma, int64_t rows, int64_t K, void* rowmajor
 }
 
 // The plain entries take no workspace, so their schedule never splits K.
-static const bq_gemm_config kNoSplit = {0, 1, -1, BQ_SPLIT_AUTO, 0};
+static const bq_gemm_config kNoSplit = {0, 1, -1, BQ_SPLIT_AUTO, 0, 0};
 
 int bq_gemm_mxfp8_mxfp4(const void* a_q, const void* a_sf, const void* b_fp4, const void* b_sf,
                         int64_t M, int64_t N, int64_t K, void* y_bf16, bq_stream_t stream) {

@@ -41,6 +41,10 @@ def candidates(M, N, K):
             if kc > 1 and K % 128:
                 continue
             out.append(bq.config(block_n=bn, split_k=1, swap_ab=0, k_chunks=kc))
+    if M > 64:
+        for kc in (1, 2):
+            if kc == 1 or K % 128 == 0:
+                out.append(bq.config(split_k=1, swap_ab=0, k_chunks=kc, cta_pair=2))
     return out
 
 
@@ -97,7 +101,7 @@ def main(argv=None):
             need = bq.workspace_bytes(wk, M, N, K, B, cfg)
             work = torch.zeros((max(need, 16),), dtype=torch.uint8, device=dev) if need else None
             desc = dict(block_n=cfg.block_n, split_k=cfg.split_k, swap_ab=cfg.swap_ab,
-                        split_mode=cfg.split_mode, k_chunks=cfg.k_chunks)
+                        split_mode=cfg.split_mode, k_chunks=cfg.k_chunks, cta_pair=cfg.cta_pair)
             try:
                 def run(c):
                     bq.gemm(wk, aq, asf, ws[c][0], ws[c][1], M, N, K, y=y, bias=bias,

@@ -205,6 +205,8 @@ typedef struct {
   int split_mode;
   int k_chunks; /* 128-K chunks per pipeline stage: 0 (auto), 1, 2 or (swap_ab) 4;
                    more than 1 needs K % 128 == 0 and no workspace split */
+  int cta_pair; /* 0 (auto), 1 single-SM tiles, 2 256x256 tiles on pairs of SMs (a
+                   2-CTA cluster sharing each MMA; wide tiles, no split, k_chunks <= 2) */
 } bq_gemm_config;
 
 /* Workspace bytes the *_epilogue calls need for a problem (0 when the chosen

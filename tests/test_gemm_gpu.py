@@ -234,6 +234,67 @@ def test_decode_without_swap():
              config=bq.config(swap_ab=0, split_k=1))
 
 
+# ------------------------------------------------------------ CTA pairs --
+
+PAIR = dict(split_k=1, swap_ab=0, cta_pair=2)
+
+
+@pytest.mark.parametrize("kc", [1, 2])
+def test_pair_tiles_ragged(kc):
+    """256x256 tiles on CTA pairs (one cta_group::2 MMA per K step): ragged
+    M, N and K, several tiles each way, both stage shapes."""
+    c = Case(bq.W_MXFP4, 300, 520, 640, seed=61 + kc, bias=True)
+    run_full(c, config=bq.config(k_chunks=kc, **PAIR))
+
+
+@pytest.mark.parametrize("wk", [bq.W_FP8BLK32, bq.W_MXFP8])
+def test_pair_tiles_fp8_weights_residual(wk):
+    c = Case(wk, 512, 768, 512, seed=63, residual=True, alpha=0.75)
+    run_full(c, config=bq.config(**PAIR))
+
+
+def test_pair_tiles_persistent_gelu():
+    """More pair tiles than pairs of SMs: each pair walks several tiles (the
+    accumulator handed back by both CTAs' epilogues each time)."""
+    c = Case(bq.W_MXFP4, 1280, 2048, 256, seed=64, bias=True, act=bq.BQ_ACT_GELU)
+    run_full(c, config=bq.config(**PAIR))
+
+
+def test_pair_tiles_batched_broadcast():
+    count, M, N, K = 3, 260, 264, 384
+    xs = [synth.activations(M, K, seed=70 + i) for i in range(count)]
+    b, bsf = synth.mxfp4_weight(N, K, seed=75)
+    bias = synth.bias(N, seed=76)
+    aqs, sfs = zip(*[bq.act_quant(to_dev_bf16(x)) for x in xs])
+    aq = torch.stack(aqs)
+    asf = torch.stack(sfs)
+    bsf_d = bq.pack_weight_scales(to_dev_u8(bsf), bq.BQ_SF_ROW32, N, K)
+    y = bq.gemm(bq.W_MXFP4, aq.reshape(count * M, K), asf, to_dev_u8(b), bsf_d, M, N, K,
+                bias=to_dev_bf16(bias), act=bq.BQ_ACT_GELU, config=bq.config(**PAIR),
+                batch=dict(count=count, stride_a=M * K, stride_a_sf=asf.shape[1], stride_b=0,
+                           stride_b_sf=0, stride_y=M * N * 2))
+    bq.device_status()
+    yb = bf16_to_f64(y.cpu().view(torch.int16).numpy().view(np.uint16))
+    for i, x in enumerate(xs):
+        q, s = oracle.act_quant(x)
+        ref, sabs = oracle.gemm(q, s, b, bsf, oracle.B_FP4, M, N, K, bias=bias,
+                                act=bq.BQ_ACT_GELU)
+        tol = oracle.gemm_tolerance(ref, sabs, 1.0, np.abs(bf16_to_f64(bias))[None, :], None,
+                                    bq.BQ_ACT_GELU)
+        assert_close(yb[i], ref, tol, f"pair batch {i}")
+
+
+def test_pair_tiles_refusals():
+    c = Case(bq.W_MXFP4, 300, 520, 640)
+    for cfg in (bq.config(split_k=2, swap_ab=0, cta_pair=2),
+                bq.config(swap_ab=1, cta_pair=2),
+                bq.config(block_n=128, split_k=1, swap_ab=0, cta_pair=2),
+                bq.config(split_k=1, swap_ab=0, cta_pair=3)):
+        with pytest.raises(bq.BqError) as e:
+            c.gpu(cfg)
+        assert e.value.status == bq.BQ_ERR_INVALID
+
+
 def test_split_k_non_swap():
     run_full(Case(bq.W_FP8BLK32, 256, 384, 2048, seed=4, residual=True),
              config=bq.config(swap_ab=0, split_k=4, block_n=128))
