@@ -155,6 +155,20 @@ int make_scale_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, in
   return r == CUDA_SUCCESS ? BQ_OK : BQ_ERR_ALIGN;
 }
 
+// The output y (bf16, row pitch N) as (N, M[, batch]); box 32 x 128 with the
+// 64-byte swizzle the epilogue's staging tile uses.
+int make_y_map(CUtensorMap* m, void* y, int64_t M, int64_t N, int64_t batch, int64_t batch_bytes) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M),
+                        static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(N * 2), static_cast<cuuint64_t>(batch_bytes)};
+  cuuint32_t box[3] = {32u, 128u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, batch > 1 ? 3 : 2, y, dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? BQ_OK : BQ_ERR_ALIGN;
+}
+
 // ---------------------------------------------------------------- schedule --
 
 enum WeightKind { kMxfp4 = 0, kFp8Blk32 = 1, kMxfp8 = 2 };
@@ -311,7 +325,8 @@ int plan_for_call(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_
 // --------------------------------------------------------------- launches --
 
 template <int BN, int STAGES, int ACC, bool SWAP, bool P_FP4, bool Q_FP4, int MODE, int KC>
-int launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const bq::GemmArgs& args,
+int launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap& ty,
+                const bq::GemmArgs& args,
                 int64_t units, int num_sms, cudaStream_t stream) {
   constexpr bool CSPLIT = MODE == bq::kSplitCluster;
   using L = bq::KernelSmem<BN, STAGES, ACC, SWAP, MODE, KC>;
@@ -363,7 +378,7 @@ int launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const bq::GemmArgs
   }
   lc.attrs = attr;
   lc.numAttrs = na;
-  if (cudaLaunchKernelEx(&lc, kern, tp, tq, args) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&lc, kern, tp, tq, ty, args) != cudaSuccess) {
     cudaGetLastError();
     return BQ_ERR_CUDA;
   }
@@ -371,18 +386,20 @@ int launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const bq::GemmArgs
 }
 
 template <int BN, int STAGES, int ACC, bool SWAP, int MODE, int KC>
-int launch_kind(bool w_fp4, const CUtensorMap& tp, const CUtensorMap& tq,
+int launch_kind(bool w_fp4, const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap& ty,
                 const bq::GemmArgs& args, int64_t u, int num_sms, cudaStream_t st) {
   // FP4 weights sit on the P side with SWAP, on the Q side otherwise.
   if (w_fp4)
-    return launch_gemm<BN, STAGES, ACC, SWAP, SWAP, !SWAP, MODE, KC>(tp, tq, args, u, num_sms, st);
-  return launch_gemm<BN, STAGES, ACC, SWAP, false, false, MODE, KC>(tp, tq, args, u, num_sms, st);
+    return launch_gemm<BN, STAGES, ACC, SWAP, SWAP, !SWAP, MODE, KC>(tp, tq, ty, args, u, num_sms,
+                                                                    st);
+  return launch_gemm<BN, STAGES, ACC, SWAP, false, false, MODE, KC>(tp, tq, ty, args, u, num_sms,
+                                                                    st);
 }
 
 template <int STAGES, int KC, bool Q_FP4>
 int launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
-                const CUtensorMap& tsb, const bq::GemmArgs& args, int64_t units, int num_sms,
-                cudaStream_t stream) {
+                const CUtensorMap& tsb, const CUtensorMap& ty, const bq::GemmArgs& args,
+                int64_t units, int num_sms, cudaStream_t stream) {
   using L = bq::PairSmem<STAGES, KC>;
   auto kern = bq::gemm_pair_kernel<STAGES, KC, Q_FP4>;
   static bool attr_set[kMaxDevices] = {};
@@ -414,7 +431,7 @@ int launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
   attr[1].val.clusterDim.z = 1;
   lc.attrs = attr;
   lc.numAttrs = 2;
-  if (cudaLaunchKernelEx(&lc, kern, ta, tb, tsa, tsb, args) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&lc, kern, ta, tb, tsa, tsb, ty, args) != cudaSuccess) {
     cudaGetLastError();
     return BQ_ERR_CUDA;
   }
@@ -424,35 +441,35 @@ int launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
 // Dispatch on (swap, bn, chunks per stage, split mode, fp4 weights) to the
 // compiled instances.  Stage counts fill ~200 KB of shared memory.
 int run_gemm(const Plan& pl, bool w_fp4, const CUtensorMap& tp, const CUtensorMap& tq,
-             const bq::GemmArgs& a, int ns, cudaStream_t st) {
+             const CUtensorMap& ty, const bq::GemmArgs& a, int ns, cudaStream_t st) {
   const int64_t u = pl.units;
   constexpr int kNone = bq::kSplitNone, kWs = bq::kSplitWorkspace, kCl = bq::kSplitCluster;
   const bool b32 = pl.bn == 32;
   if (!pl.swap) {
     if (pl.bn == 256) {
-      if (pl.splits > 1) return launch_kind<256, 4, 1, false, kWs, 1>(w_fp4, tp, tq, a, u, ns, st);
-      return pl.kc == 2 ? launch_kind<256, 2, 1, false, kNone, 2>(w_fp4, tp, tq, a, u, ns, st)
-                        : launch_kind<256, 4, 1, false, kNone, 1>(w_fp4, tp, tq, a, u, ns, st);
+      if (pl.splits > 1) return launch_kind<256, 4, 1, false, kWs, 1>(w_fp4, tp, tq, ty, a, u, ns, st);
+      return pl.kc == 2 ? launch_kind<256, 2, 1, false, kNone, 2>(w_fp4, tp, tq, ty, a, u, ns, st)
+                        : launch_kind<256, 4, 1, false, kNone, 1>(w_fp4, tp, tq, ty, a, u, ns, st);
     }
-    if (pl.splits > 1) return launch_kind<128, 6, 2, false, kWs, 1>(w_fp4, tp, tq, a, u, ns, st);
-    return pl.kc == 2 ? launch_kind<128, 3, 2, false, kNone, 2>(w_fp4, tp, tq, a, u, ns, st)
-                      : launch_kind<128, 6, 2, false, kNone, 1>(w_fp4, tp, tq, a, u, ns, st);
+    if (pl.splits > 1) return launch_kind<128, 6, 2, false, kWs, 1>(w_fp4, tp, tq, ty, a, u, ns, st);
+    return pl.kc == 2 ? launch_kind<128, 3, 2, false, kNone, 2>(w_fp4, tp, tq, ty, a, u, ns, st)
+                      : launch_kind<128, 6, 2, false, kNone, 1>(w_fp4, tp, tq, ty, a, u, ns, st);
   }
   if (pl.cluster) {
     if (pl.kc == 4)
-      return b32 ? launch_kind<32, 1, 1, true, kCl, 4>(w_fp4, tp, tq, a, u, ns, st)
-                 : launch_kind<64, 1, 1, true, kCl, 4>(w_fp4, tp, tq, a, u, ns, st);
-    return b32 ? launch_kind<32, 3, 1, true, kCl, 1>(w_fp4, tp, tq, a, u, ns, st)
-               : launch_kind<64, 3, 1, true, kCl, 1>(w_fp4, tp, tq, a, u, ns, st);
+      return b32 ? launch_kind<32, 1, 1, true, kCl, 4>(w_fp4, tp, tq, ty, a, u, ns, st)
+                 : launch_kind<64, 1, 1, true, kCl, 4>(w_fp4, tp, tq, ty, a, u, ns, st);
+    return b32 ? launch_kind<32, 3, 1, true, kCl, 1>(w_fp4, tp, tq, ty, a, u, ns, st)
+               : launch_kind<64, 3, 1, true, kCl, 1>(w_fp4, tp, tq, ty, a, u, ns, st);
   }
   if (pl.splits > 1)
-    return b32 ? launch_kind<32, 4, 1, true, kWs, 1>(w_fp4, tp, tq, a, u, ns, st)
-               : launch_kind<64, 4, 1, true, kWs, 1>(w_fp4, tp, tq, a, u, ns, st);
+    return b32 ? launch_kind<32, 4, 1, true, kWs, 1>(w_fp4, tp, tq, ty, a, u, ns, st)
+               : launch_kind<64, 4, 1, true, kWs, 1>(w_fp4, tp, tq, ty, a, u, ns, st);
   if (pl.kc == 4)
-    return b32 ? launch_kind<32, 2, 1, true, kNone, 4>(w_fp4, tp, tq, a, u, ns, st)
-               : launch_kind<64, 2, 1, true, kNone, 4>(w_fp4, tp, tq, a, u, ns, st);
-  return b32 ? launch_kind<32, 8, 1, true, kNone, 1>(w_fp4, tp, tq, a, u, ns, st)
-             : launch_kind<64, 8, 1, true, kNone, 1>(w_fp4, tp, tq, a, u, ns, st);
+    return b32 ? launch_kind<32, 2, 1, true, kNone, 4>(w_fp4, tp, tq, ty, a, u, ns, st)
+               : launch_kind<64, 2, 1, true, kNone, 4>(w_fp4, tp, tq, ty, a, u, ns, st);
+  return b32 ? launch_kind<32, 8, 1, true, kNone, 1>(w_fp4, tp, tq, ty, a, u, ns, st)
+             : launch_kind<64, 8, 1, true, kNone, 1>(w_fp4, tp, tq, ty, a, u, ns, st);
 }
 
 int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, const void* b_sf,
@@ -517,6 +534,11 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
   st = make_operand_map(&map_b, b, w_fp4, K, N, w_fp4 ? K / 2 : K, b_batched ? count : 1, sb,
                         b_box, pl.kc);
   if (st != BQ_OK) return st;
+  // Output y [batch][M][N] bf16 for the wide tiles' TMA-store epilogue: 128-row
+  // x 32-column boxes with the 64-byte swizzle.
+  CUtensorMap map_y;
+  st = make_y_map(&map_y, y, M, N, count, sy);
+  if (st != BQ_OK) return st;
 
   bq::GemmArgs g;
   memset(&g, 0, sizeof(g));
@@ -567,14 +589,15 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
     const int64_t u = pl.units;
     const int ns = dev->num_sms;
     if (pl.kc == 2)
-      return w_fp4 ? launch_pair<3, 2, true>(map_a, map_b, map_sfa, map_sfb, g, u, ns, s)
-                   : launch_pair<3, 2, false>(map_a, map_b, map_sfa, map_sfb, g, u, ns, s);
-    return w_fp4 ? launch_pair<6, 1, true>(map_a, map_b, map_sfa, map_sfb, g, u, ns, s)
-                 : launch_pair<6, 1, false>(map_a, map_b, map_sfa, map_sfb, g, u, ns, s);
+      return w_fp4 ? launch_pair<3, 2, true>(map_a, map_b, map_sfa, map_sfb, map_y, g, u, ns, s)
+                   : launch_pair<3, 2, false>(map_a, map_b, map_sfa, map_sfb, map_y, g, u, ns, s);
+    return w_fp4 ? launch_pair<6, 1, true>(map_a, map_b, map_sfa, map_sfb, map_y, g, u, ns, s)
+                 : launch_pair<6, 1, false>(map_a, map_b, map_sfa, map_sfb, map_y, g, u, ns, s);
   }
   const CUtensorMap& tp = pl.swap ? map_b : map_a;
   const CUtensorMap& tq = pl.swap ? map_a : map_b;
-  return run_gemm(pl, w_fp4, tp, tq, g, dev->num_sms, reinterpret_cast<cudaStream_t>(stream));
+  return run_gemm(pl, w_fp4, tp, tq, map_y, g, dev->num_sms,
+                  reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // namespace

@@ -41,6 +41,7 @@ constexpr int kBlockP = 128;  // MMA M
 constexpr int kBlockK = 128;  // inputs per stage: 128 one-byte codes = one 128B-swizzle row
 constexpr int kMmaK = 32;     // inputs per tcgen05.mma (one scale per row per MMA)
 constexpr int kSfAtom = 512;  // bytes of one 128-row x 4-column scale atom
+constexpr int kYChunkBytes = kBlockP * 32 * 2;  // a 128-row x 32-column bf16 staging tile
 // Warp roles: 0 weight-operand copies (and barrier set-up), 1 TMEM
 // allocation and MMA issue, 2-5 epilogue (one TMEM lane quadrant each),
 // 6 activation-operand copies, 7 weight-scale copies, 8 activation-scale
@@ -102,7 +103,7 @@ enum SplitMode : int { kSplitNone = 0, kSplitWorkspace = 1, kSplitCluster = 2 };
 // chunks' scale-factor atoms; more bytes behind one stage barrier means fewer
 // barrier round trips per byte, which is what bounds a CTA's copy rate.
 template <int BN, int STAGES, int ACC, bool CSPLIT = false, int KC = 1, bool OUT_STAGE = false,
-          bool LANDING = false>
+          bool LANDING = false, bool YSTAGE = false>
 struct GemmSmem {
   static constexpr int kSfqAtoms = BN > 128 ? BN / 128 : 1;
   static constexpr int kSfqCols = 4 * kSfqAtoms;
@@ -115,7 +116,11 @@ struct GemmSmem {
   static constexpr int kSfpBytes = KC * kSfAtom;              // per stage
   static constexpr int kSfqBytes = KC * kSfqAtoms * kSfAtom;  // per stage
   static constexpr int kOffQ = STAGES * kBytesP;
-  static constexpr int kOffSfp = kOffQ + STAGES * kBytesQ;
+  // wide tiles: two 128x32 bf16 staging tiles for the TMA-store epilogue
+  // (1024-byte aligned: the 64-byte swizzle follows address bits)
+  static constexpr int kOffYStage = kOffQ + STAGES * kBytesQ;
+  static constexpr int kBytesYStage = YSTAGE ? 2 * kYChunkBytes : 0;
+  static constexpr int kOffSfp = kOffYStage + kBytesYStage;
   static constexpr int kOffSfq = kOffSfp + STAGES * kSfpBytes;
   // cluster split-K: receive buffer [S slices][128/S rows][BN + 4] fp32 (the
   // +4 pad keeps float4 row accesses free of bank conflicts)
@@ -153,7 +158,8 @@ struct GemmSmem {
 // gather the slices' partial tiles in shared memory.
 template <int BN, int STAGES, int ACC, bool SWAP, int MODE, int KC>
 using KernelSmem = GemmSmem<BN, STAGES, ACC, MODE == kSplitCluster, KC,
-                            SWAP && MODE == kSplitNone, SWAP && MODE == kSplitWorkspace>;
+                            SWAP && MODE == kSplitNone, SWAP && MODE == kSplitWorkspace,
+                            !SWAP && MODE == kSplitNone>;
 
 __device__ __forceinline__ uint32_t make_idesc(uint32_t fmt_p, uint32_t fmt_q, int bn, int sf_id) {
   uint32_t d = 0;
@@ -296,6 +302,94 @@ __device__ __forceinline__ void emit32(const GemmArgs &a, int b, int prow, int q
 __device__ __forceinline__ void epi_bar_sync() {
   __syncwarp();
   asm volatile("barrier.sync 1, 128;" ::: "memory");  // the 4 epilogue warps
+}
+
+// 32 residual values of one row (4 x 16 bytes), zeros past N or without one.
+__device__ __forceinline__ void load_res32(const __nv_bfloat16 *rrow, int q0, int N,
+                                           uint4 (&r)[4]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    r[j] = (rrow && q0 + 8 * j < N) ? *reinterpret_cast<const uint4 *>(rrow + q0 + 8 * j)
+                                    : make_uint4(0u, 0u, 0u, 0u);
+}
+
+// Wide-tile epilogue (activation rows on the TMEM lanes): rows m0 .. m0+127
+// (this thread owns m0 + row) and columns n0 .. n0+NCOLS-1, in chunks of 32
+// columns: TMEM -> registers -> alpha, bias, GELU, residual in fp32 -> one
+// bf16 rounding -> a 128x32 bf16 staging tile in shared memory (the 64-byte
+// swizzle, so each warp store is conflict-free) -> one TMA store per chunk,
+// double-buffered.  Stores clip rows past M and columns past N.  The next
+// chunk's residual is loaded while the current one is computed.
+template <int NCOLS>
+__device__ __forceinline__ void epilogue_rows_tma(const GemmArgs &a, const CUtensorMap *tm_y,
+                                                  uint32_t t_row, int b, int m0, int n0, int row,
+                                                  int epi_tid, uint8_t *ystage) {
+  const int m = m0 + row;
+  const __nv_bfloat16 *rrow =
+      (a.res && m < a.M) ? a.res + b * a.res_bstride + static_cast<int64_t>(m) * a.ldres : nullptr;
+  uint4 res[4];
+  load_res32(rrow, n0, a.N, res);
+#pragma unroll 1
+  for (int c = 0; c < NCOLS / 32; ++c) {
+    const int q0 = n0 + c * 32;
+    if (q0 >= a.N) break;  // uniform
+    uint32_t v[32];
+    __syncwarp();
+    tmem_ld_32x32b_x32(t_row + c * 32, v);
+    tmem_ld_wait();
+    uint4 res_next[4];
+    load_res32(c + 1 < NCOLS / 32 ? rrow : nullptr, q0 + 32, a.N, res_next);
+    uint32_t o[16];
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      float bias8[8];
+      if (a.bias && q0 + 8 * g < a.N) {
+        const uint4 bv = __ldg(reinterpret_cast<const uint4 *>(a.bias + q0 + 8 * g));
+        const uint32_t w[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          bias8[2 * j] = bf16_bits_to_f32(w[j] & 0xFFFF);
+          bias8[2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) bias8[j] = 0.0f;
+      }
+      float t[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) t[j] = a.alpha * __uint_as_float(v[8 * g + j]) + bias8[j];
+      if (a.act == 1) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) t[j] = gelu_erf(t[j]);
+      }
+      const uint32_t rw[4] = {res[g].x, res[g].y, res[g].z, res[g].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __nv_bfloat162 p2 =
+            __floats2bfloat162_rn(t[2 * j] + bf16_bits_to_f32(rw[j] & 0xFFFF),
+                                  t[2 * j + 1] + bf16_bits_to_f32(rw[j] >> 16));
+        o[4 * g + j] = *reinterpret_cast<const uint32_t *>(&p2);
+      }
+    }
+    uint8_t *buf = ystage + (c & 1) * kYChunkBytes;
+    if (epi_tid == 0) bulk_wait_group_read<1>();  // the store two chunks back has read buf
+    epi_bar_sync();
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      *reinterpret_cast<uint4 *>(buf + row * 64 + ((j ^ ((row >> 1) & 3)) << 4)) =
+          make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+    fence_proxy_async_smem();
+    epi_bar_sync();
+    if (epi_tid == 0) {
+      if (a.batch > 1)
+        tma_store_3d(tm_y, buf, q0, m0, b);
+      else
+        tma_store_2d(tm_y, buf, q0, m0);
+      bulk_commit_group();
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) res[j] = res_next[j];
+  }
 }
 
 // Swap-AB epilogue, first half: the 32 values of output column n = prow
@@ -477,7 +571,7 @@ __device__ __forceinline__ void cluster_reduce_local(const GemmArgs &a, const Un
 template <int BN, int STAGES, int ACC, bool SWAP, bool P_FP4, bool Q_FP4, int MODE, int KC>
 __global__ void __launch_bounds__(kNumThreads, 1)
     gemm_bs_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
-                   const GemmArgs a) {
+                   const __grid_constant__ CUtensorMap tm_y, const GemmArgs a) {
   constexpr bool CSPLIT = MODE == kSplitCluster;
   static_assert(!CSPLIT || SWAP, "cluster split-K is built for the swap-AB (decode) tiles");
   static_assert(!CSPLIT || ACC == 1, "cluster split-K uses one accumulator");
@@ -780,17 +874,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         copy_out_swap<BN>(a, u, epi_tid, stage);
         if (unit + static_cast<int>(gridDim.x) < total_units) epi_bar_sync();  // staging free
       } else if constexpr (MODE == kSplitNone) {
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t v[32];
-          __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the stores
-          tmem_ld_32x32b_x32(t_row + c * 32, v);
-          tmem_ld_wait();
-          float f[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
-          emit32<SWAP>(a, u.b, prow, u.tq * BN + c * 32, f, bias_n);
-        }
+        epilogue_rows_tma<BN>(a, &tm_y, t_row, u.b, u.tp * kBlockP, u.tq * BN, row, epi_tid,
+                              smem + L::kOffYStage);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -990,6 +1075,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     }
   }
 
+  // The epilogue's last TMA stores must be done before the CTA retires.
+  if constexpr (L::kBytesYStage > 0)
+    if (threadIdx.x == 64) bulk_wait_group_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

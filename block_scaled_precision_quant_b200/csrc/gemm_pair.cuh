@@ -40,7 +40,8 @@ struct PairSmem {
   static constexpr int kSfColsChunk = 4 + 4 * kSfbAtoms;   // TMEM scale columns per chunk
   static constexpr int kSfCols = KC * kSfColsChunk;
   static constexpr int kOffB = STAGES * kBytesA;
-  static constexpr int kOffSfa = kOffB + STAGES * kBytesB;
+  static constexpr int kOffYStage = kOffB + STAGES * kBytesB;  // 1024-aligned
+  static constexpr int kOffSfa = kOffYStage + 2 * kYChunkBytes;
   static constexpr int kOffSfb = kOffSfa + STAGES * kSfaBytes;
   static constexpr int kOffBar = kOffSfb + STAGES * kSfbBytes;
   static constexpr int kNumBars = 2 * STAGES + 3;          // full, empty, tfull, tempty, drain
@@ -129,7 +130,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
                      const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_sfa,
-                     const __grid_constant__ CUtensorMap tm_sfb, const GemmArgs a) {
+                     const __grid_constant__ CUtensorMap tm_sfb,
+                     const __grid_constant__ CUtensorMap tm_y, const GemmArgs a) {
   using L = PairSmem<STAGES, KC>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -270,6 +272,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     // ---------------------------------------------------- epilogue (both CTAs) --
     const int quad = warp % 4;
     const int row = quad * 32 + lane;
+    const int epi_tid = threadIdx.x - 64;
     uint32_t acc_phase = 0;
     griddep_wait();  // the bias and residual may come from the preceding kernel
     for (int unit = pair; unit < total_units; unit += num_pairs) {
@@ -279,18 +282,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       acc_phase ^= 1;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
-      const int prow = (2 * u.tp + static_cast<int>(rank)) * kBlockP + row;
-#pragma unroll 1
-      for (int c = 0; c < kPairN / 32; ++c) {
-        uint32_t v[32];
-        __syncwarp();
-        tmem_ld_32x32b_x32(t_row + c * 32, v);
-        tmem_ld_wait();
-        float f[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
-        emit32<false>(a, u.b, prow, u.tq * kPairN + c * 32, f, 0.0f);
-      }
+      epilogue_rows_tma<kPairN>(a, &tm_y, t_row, u.b, (2 * u.tp + static_cast<int>(rank)) * kBlockP,
+                                u.tq * kPairN, row, epi_tid, smem + L::kOffYStage);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_lead);
@@ -298,7 +291,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   }
 
   // Teardown: the leader has drained its MMAs; nothing may still be arriving
-  // on either CTA's barriers or reading its TMEM when the pair frees it.
+  // on either CTA's barriers or reading its TMEM when the pair frees it, and
+  // the epilogue's last TMA stores are done.
+  if (threadIdx.x == 64) bulk_wait_group_all();
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();
