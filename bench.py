@@ -475,6 +475,9 @@ def main(argv=None):
     ap.add_argument("--profile-run", type=int, default=0, metavar="R",
                     help="no timing: build one input set and run every layer's step R "
                          "times eagerly (for ncu captures of single launches)")
+    ap.add_argument("--profile-shape", default=None, metavar="M,N,K",
+                    help="with --profile-run: run only the workload's first layer, at this "
+                         "smaller shape (a small case of the same kernel for full captures)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
@@ -502,14 +505,20 @@ def run_ours(args, spec, world, rank, local, device):
     import block_scaled_precision_quant_b200 as bq
 
     if args.profile_run:
-        layers = [Layer(sp, 1, 11 * (i + 1), device) for i, sp in enumerate(spec["layers"])]
+        specs = spec["layers"]
+        if args.profile_shape:
+            M, N, K = (int(v) for v in args.profile_shape.split(","))
+            name, wk, _, _, _, B, ex = specs[0]
+            specs = [(name, wk, M, N, K, B, ex)]
+        layers = [Layer(sp, 1, 11 * (i + 1), device) for i, sp in enumerate(specs)]
         for _ in range(args.profile_run):
             for L in layers:
                 L.launches(0)
         torch.cuda.synchronize()
         bq.device_status()
         if rank == 0:
-            print(json.dumps({"profile_run": args.profile_run, "workload": spec["desc"]}))
+            print(json.dumps({"profile_run": args.profile_run, "workload": spec["desc"],
+                              "shape": args.profile_shape}))
         return 0
 
     layers_spec = spec["layers"]
