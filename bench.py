@@ -75,14 +75,15 @@ def act_quant_bytes(layer):
     return (2.0 + 1.0 + 1.0 / 32.0) * M * K * B
 
 
-def gemm_bytes(layer):
+def gemm_bytes(layer, quant_out=False):
     """Algorithmic bytes of one GEMM launch: every operand read once, the
-    output written once (weights counted once when broadcast over a batch)."""
+    output written once (weights counted once when broadcast over a batch);
+    a quantized output is 1 + 1/32 bytes per element instead of 2."""
     _, wk, M, N, K, B, ex = layer
     w = N * K / 2.0 if wk == "mxfp4" else float(N * K)
     w += N * K / 32.0  # weight scales
     a = B * (M * K + M * K / 32.0)
-    y = B * M * N * 2.0
+    y = B * M * N * ((1.0 + 1.0 / 32.0) if quant_out else 2.0)
     if ex.get("bias"):
         a += N * 2.0
     if ex.get("residual"):
@@ -233,7 +234,7 @@ class Layer:
     """Device buffers of one linear layer, with `sets` rotating copies of the
     inputs (activations, weights, scales, bias, residual)."""
 
-    def __init__(self, spec, sets, seed, device):
+    def __init__(self, spec, sets, seed, device, quant_out=False):
         import torch
         import block_scaled_precision_quant_b200 as bq
         from block_scaled_precision_quant_b200 import synth
@@ -275,6 +276,10 @@ class Layer:
         per = bq.sf_bytes(M, K)
         self.asf = torch.empty((B, per), dtype=torch.uint8, device=device)
         self.y = torch.empty((B, M, N), dtype=torch.bfloat16, device=device)
+        self.quant_out = quant_out
+        self.qy = torch.empty((B, M, N), dtype=torch.uint8, device=device) if quant_out else None
+        self.sfy = (torch.empty((B, bq.sf_bytes(M, N)), dtype=torch.uint8, device=device)
+                    if quant_out else None)
         self.need = bq.workspace_bytes(self.wk, M, N, K, B)
         self.ws = (torch.zeros((self.need,), dtype=torch.uint8, device=device)
                    if self.need else None)
@@ -303,10 +308,13 @@ class Layer:
             if B > 1:
                 batch = dict(count=B, stride_a=M * K, stride_a_sf=self.asf.shape[1], stride_b=0,
                              stride_b_sf=0, stride_y=M * N * 2, stride_res=M * N * 2)
-            bq.gemm(self.wk, self.aq, self.asf, d["w"], d["wsf"], M, N, K, y=self.y,
-                    bias=d["bias"], residual=d["res"],
+            kw = {}
+            if self.quant_out:  # the output in MXFP8 for a next projection, no bf16 y
+                kw = dict(quantize_out=True, write_y=False, q_out=self.qy, sf_out=self.sfy)
+            bq.gemm(self.wk, self.aq, self.asf, d["w"], d["wsf"], M, N, K,
+                    y=None if self.quant_out else self.y, bias=d["bias"], residual=d["res"],
                     act=bq.BQ_ACT_GELU if self.gelu else bq.BQ_ACT_NONE, batch=batch,
-                    workspace=self.ws)
+                    workspace=self.ws, **kw)
             n += 1
         return n
 
@@ -390,16 +398,17 @@ def run_e2e(spec_layers, layers, steps, device):
     import torch
     import block_scaled_precision_quant_b200 as bq
     host_x = [L.sets[0]["x"].cpu().pin_memory() for L in layers]
-    host_y = [torch.empty(L.y.shape, dtype=torch.bfloat16).pin_memory() for L in layers]
+    outs = [L.qy if L.quant_out else L.y for L in layers]  # the step's result
+    host_y = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
     h2d = sum(h.numel() * h.element_size() for h in host_x)
     d2h = sum(h.numel() * h.element_size() for h in host_y)
     dev_x = [torch.empty_like(L.sets[0]["x"]) for L in layers]
 
     def step():
-        for L, hx, dx, hy in zip(layers, host_x, dev_x, host_y):
+        for L, hx, dx, hy, o in zip(layers, host_x, dev_x, host_y, outs):
             dx.copy_(hx, non_blocking=True)
             L.launches(0, x=dx)
-            hy.copy_(L.y, non_blocking=True)
+            hy.copy_(o, non_blocking=True)
     for _ in range(3):
         step()
     torch.cuda.synchronize()
@@ -475,6 +484,9 @@ def main(argv=None):
     ap.add_argument("--profile-run", type=int, default=0, metavar="R",
                     help="no timing: build one input set and run every layer's step R "
                          "times eagerly (for ncu captures of single launches)")
+    ap.add_argument("--quant-out", action="store_true",
+                    help="every GEMM writes its output quantized (MXFP8 codes + MMA-layout "
+                         "scales, for a next projection) instead of bf16 y")
     ap.add_argument("--profile-shape", default=None, metavar="M,N,K",
                     help="with --profile-run: run only the workload's first layer, at this "
                          "smaller shape (a small case of the same kernel for full captures)")
@@ -528,7 +540,8 @@ def run_ours(args, spec, world, rank, local, device):
     nsets = max(1, min(64, int(np.ceil(3.0 * l2 / max(set_bytes, 1)))))
     del probe
     torch.cuda.empty_cache()
-    layers = [Layer(sp, nsets, 11 * (i + 1), device) for i, sp in enumerate(layers_spec)]
+    layers = [Layer(sp, nsets, 11 * (i + 1), device, quant_out=args.quant_out)
+              for i, sp in enumerate(layers_spec)]
     graphs = build_graphs(layers, nsets, "all")
     launches_per_step = sum(
         (L.B + (1 if L.sets[0]["wx"] is not None else 0)) + 1 for L in layers)
@@ -568,7 +581,7 @@ def run_ours(args, spec, world, rank, local, device):
     bq.device_status()
 
     flops_step = sum(gemm_flops(sp) for sp in layers_spec)
-    gbytes_step = sum(gemm_bytes(sp) for sp in layers_spec)
+    gbytes_step = sum(gemm_bytes(sp, args.quant_out) for sp in layers_spec)
     qbytes_step = sum(act_quant_bytes(sp) for sp in layers_spec)
     if any(sp[1] == "mxfp8" for sp in layers_spec):
         qbytes_step += sum(act_quant_bytes((0, 0, sp[3], 0, sp[4], 1, 0))
@@ -616,7 +629,8 @@ def run_ours(args, spec, world, rank, local, device):
         "config": {"workload": spec["desc"], "parallelism": "replicas" if world > 1 else "single",
                    "l2": f"{nsets} rotating input sets of {set_bytes / 1e6:.1f} MB "
                          f"({nsets * set_bytes / 1e6:.0f} MB > L2 {l2 / 1e6:.0f} MB)",
-                   "graphs": "one CUDA graph per input set, replayed per step"},
+                   "graphs": "one CUDA graph per input set, replayed per step",
+                   "output": "mxfp8 (codes + scales, no bf16 y)" if args.quant_out else "bf16"},
         "roofline": roof,
         "act_quant": {"achieved_gbs": round(qbytes_step / (aq_ms_step * 1e-3) / 1e9, 1),
                       "frac_hbm": round(qbytes_step / (aq_ms_step * 1e-3) / 1e9 / peaks["hbm"], 4),

@@ -56,7 +56,8 @@ class BqError(RuntimeError):
 
 class Epilogue(ctypes.Structure):
     _fields_ = [("bias", ctypes.c_void_p), ("residual", ctypes.c_void_p),
-                ("ld_residual", ctypes.c_int64), ("alpha", ctypes.c_float), ("act", ctypes.c_int)]
+                ("ld_residual", ctypes.c_int64), ("alpha", ctypes.c_float), ("act", ctypes.c_int),
+                ("q_out", ctypes.c_void_p), ("sf_out", ctypes.c_void_p)]
 
 
 class Batch(ctypes.Structure):
@@ -256,20 +257,37 @@ def _workspace(device, nbytes):
 
 
 def gemm(weight_kind, a_q, a_sf, b, b_sf, M, N, K, y=None, bias=None, residual=None,
-         alpha=1.0, act=BQ_ACT_NONE, batch=None, config=None, workspace=None):
+         alpha=1.0, act=BQ_ACT_NONE, batch=None, config=None, workspace=None,
+         quantize_out=False, write_y=True, q_out=None, sf_out=None):
     """y = bf16(act(alpha * A B^T + bias) + residual) for weight_kind W_MXFP4,
     W_FP8BLK32 or W_MXFP8.  batch: None or a dict with 'count' and byte
     strides ('stride_a', 'stride_a_sf', 'stride_b', 'stride_b_sf', 'stride_y',
-    'stride_res'; 0 broadcasts).  config: GemmConfig or None (auto)."""
+    'stride_res'; 0 broadcasts).  config: GemmConfig or None (auto).
+    quantize_out: also return y quantized for the next GEMM (E4M3 codes
+    [.., M, N] u8 and MMA-layout scales, exactly act_quant of y, written to
+    q_out / sf_out when given); then returns (y or None, q, sf), with no bf16
+    y written when write_y is False."""
     torch = _torch()
     _need_cuda(a_q, a_sf, b, b_sf, bias, residual)
     count = 1 if batch is None else int(batch["count"])
-    if y is None:
-        shape = (M, N) if batch is None else (count, M, N)
+    shape = (M, N) if batch is None else (count, M, N)
+    if not write_y and not quantize_out:
+        raise ValueError("write_y=False needs quantize_out=True")
+    if y is None and write_y:
         y = torch.empty(shape, dtype=torch.bfloat16, device=a_q.device)
+    if quantize_out:
+        if q_out is None:
+            q_out = torch.empty(shape, dtype=torch.uint8, device=a_q.device)
+        if sf_out is None:
+            per = sf_bytes(M, N)
+            sf_out = torch.empty((per,) if batch is None else (count, per), dtype=torch.uint8,
+                                 device=a_q.device)
+    else:
+        q_out = sf_out = None
     need = workspace_bytes(weight_kind, M, N, K, count, config)
     plain = (bias is None and residual is None and alpha == 1.0 and act == BQ_ACT_NONE
-             and batch is None and config is None and workspace is None and need == 0)
+             and batch is None and config is None and workspace is None and need == 0
+             and not quantize_out)
     if plain:
         f = getattr(lib(), _ENTRY[weight_kind])
         _check(f(_ptr(a_q), _ptr(a_sf), _ptr(b), _ptr(b_sf), M, N, K, _ptr(y), _stream()),
@@ -277,7 +295,9 @@ def gemm(weight_kind, a_q, a_sf, b, b_sf, M, N, K, y=None, bias=None, residual=N
         return y
     epi = Epilogue(bias.data_ptr() if bias is not None else None,
                    residual.data_ptr() if residual is not None else None,
-                   residual.stride(-2) if residual is not None else 0, float(alpha), int(act))
+                   residual.stride(-2) if residual is not None else 0, float(alpha), int(act),
+                   q_out.data_ptr() if q_out is not None else None,
+                   sf_out.data_ptr() if sf_out is not None else None)
     bt = None
     if batch is not None:
         bt = Batch(count, *(int(batch.get(k, 0)) for k in (
@@ -291,6 +311,8 @@ def gemm(weight_kind, a_q, a_sf, b, b_sf, M, N, K, y=None, bias=None, residual=N
              ws.numel() if ws is not None else 0,
              ctypes.byref(config) if config is not None else None, _stream()),
            _ENTRY[weight_kind] + "_epilogue")
+    if quantize_out:
+        return (y if write_y else None), q_out, sf_out
     return y
 
 

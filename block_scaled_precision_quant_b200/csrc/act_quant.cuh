@@ -2,14 +2,8 @@
 // layout kernels (prepack / unpack) for sm_100a.
 //
 // Quantizer ("formats.py" page: act_scale, act_quant, _log2_ceil_pow2 and the
-// module docstring "act_qdq reproduces ..."), for each 32 consecutive
-// elements of a row:
-//   amax = max(max|x|, fp32(1e-4));  t = fp32(amax * fp32(1/448))
-//   e    = ceil(log2 t) from t's exponent bits;  scale byte = e + 127
-//   q    = E4M3 round-to-nearest-even of clamp(x / 2^e, -448, 448)
-// x / 2^e is computed as x * 2^-e: 2^-e is an exact binary32 power of two for
-// every e the rule can produce (-22 .. 120), so the correctly rounded product
-// equals the correctly rounded quotient.
+// module docstring "act_qdq reproduces ..."), per 32 consecutive elements of
+// a row; the arithmetic is in mx_quant.cuh.
 //
 // Work split: one warp per 512 consecutive elements of one row (16 groups);
 // a thread owns half a group (16 bf16 = two 16-byte loads), the two halves
@@ -22,22 +16,9 @@
 #include <stdint.h>
 
 #include "bq_ptx.cuh"
+#include "mx_quant.cuh"
 
 namespace bq {
-
-// Byte offset of scale (row r, column c) in an MMA-layout buffer with
-// `katoms` = ceil(G / 4) atoms per 128-row band.
-__host__ __device__ __forceinline__ int64_t sf_mma_offset(int64_t r, int64_t c, int64_t katoms) {
-  return ((r >> 7) * katoms + (c >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3);
-}
-
-__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
-  const __nv_fp8x2_storage_t lo =
-      __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
-  const __nv_fp8x2_storage_t hi =
-      __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
-  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
-}
 
 // grid: x*8 + warp = row, y = chunk of 16 groups within the row.  Rows in
 // [M, rows_pad) only write padding scale bytes (127).
@@ -69,38 +50,18 @@ __global__ void __launch_bounds__(256) act_quant_kernel(
     w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
     w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
   }
-  // amax over |x| as an integer max of the magnitude bits (order-preserving
-  // for non-negative floats); non-finite detection from the exponent bits.
-  uint32_t mx = 0, bad = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t lo = w[i] & 0x7FFFu, hi = (w[i] >> 16) & 0x7FFFu;
-    mx = max(mx, max(lo, hi));
-    bad |= ((lo & 0x7F80u) == 0x7F80u) | ((hi & 0x7F80u) == 0x7F80u);
-  }
+  // amax of the two half-groups met through one shuffle
+  uint32_t bad = 0;
+  uint32_t mx = bf16_amax_bits(w, bad);
   mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
   uint32_t sbyte = 127;
   if (active) {
     if (bad && status) atomicOr(status, 1);
-    const float amax = fmaxf(__uint_as_float(mx << 16), 1e-4f);
-    const float t = __fmul_rn(amax, __uint_as_float(0x3B124925u));  // fp32(1/448)
-    const uint32_t tb = __float_as_uint(t);
-    const int e = static_cast<int>((tb >> 23) & 0xFFu) - 127 + ((tb & 0x7FFFFFu) != 0u ? 1 : 0);
+    const int e = mx_exponent(mx);
     sbyte = static_cast<uint32_t>(e + 127);
-    const float inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e
-    float f[16];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      f[2 * i] = fminf(fmaxf(__fmul_rn(__uint_as_float(w[i] << 16), inv), -448.0f), 448.0f);
-      f[2 * i + 1] =
-          fminf(fmaxf(__fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), inv), -448.0f), 448.0f);
-    }
-    uint4 out;
-    out.x = e4m3x4(f[0], f[1], f[2], f[3]);
-    out.y = e4m3x4(f[4], f[5], f[6], f[7]);
-    out.z = e4m3x4(f[8], f[9], f[10], f[11]);
-    out.w = e4m3x4(f[12], f[13], f[14], f[15]);
-    *reinterpret_cast<uint4 *>(q + row * K + col) = out;
+    uint32_t c[4];
+    mx_encode(w, e, c);
+    *reinterpret_cast<uint4 *>(q + row * K + col) = make_uint4(c[0], c[1], c[2], c[3]);
     if (sf_row && half == 0) sf_row[row * G + g] = static_cast<uint8_t>(sbyte);
   }
   // Gather the bytes of groups 4j..4j+3 of this chunk (lanes 8j, 8j+2, 8j+4,

@@ -483,12 +483,17 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
   const int64_t count = batch ? batch->count : 1;
   if (count < 0) return BQ_ERR_SHAPE;
   if (M == 0 || N == 0 || count == 0) return BQ_OK;
-  if (!a_q || !a_sf || !b || !b_sf || !y) return BQ_ERR_NULL;
+  void* q_out = epi ? epi->q_out : nullptr;
+  void* sf_out = epi ? epi->sf_out : nullptr;
+  if ((q_out || sf_out) && N % 32 != 0) return BQ_ERR_SHAPE;
+  if ((q_out != nullptr) != (sf_out != nullptr)) return BQ_ERR_NULL;
+  if (!a_q || !a_sf || !b || !b_sf || (!y && !q_out)) return BQ_ERR_NULL;
+  if (q_out && (!aligned(q_out, 16) || !aligned(sf_out, 4))) return BQ_ERR_ALIGN;
   const bool w_fp4 = wk == kMxfp4;
   if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF || count > 65535) return BQ_ERR_SHAPE;
   if (N % 8 != 0) return BQ_ERR_SHAPE;
   if (w_fp4 && K % 128 != 0) return BQ_ERR_SHAPE;
-  if (!aligned(a_q, 16) || !aligned(a_sf, 16) || !aligned(b_sf, 16) || !aligned(y, 16) ||
+  if (!aligned(a_q, 16) || !aligned(a_sf, 16) || !aligned(b_sf, 16) || (y && !aligned(y, 16)) ||
       !aligned(b, w_fp4 ? 32 : 16))
     return BQ_ERR_ALIGN;
   const void* bias = epi ? epi->bias : nullptr;
@@ -509,6 +514,14 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
     if (sa % 16 || ssa % 16 || ssb % 16 || sy % 16 || sr % 16 || sb % (w_fp4 ? 32 : 16))
       return BQ_ERR_ALIGN;
     if (sy == 0) return BQ_ERR_SHAPE;  // problems would overwrite each other
+  }
+  // The quantized output is written by epilogues that finish a tile in one
+  // CTA: no K split (an explicit one is refused).
+  bq_gemm_config cfg_q = cfg ? *cfg : bq_gemm_config{0, 0, -1, BQ_SPLIT_AUTO, 0, 0};
+  if (q_out) {
+    if (cfg_q.split_k > 1) return BQ_ERR_INVALID;
+    cfg_q.split_k = 1;
+    cfg = &cfg_q;
   }
   Plan pl;
   st = plan_for_call(M, N, K, count, cfg, dev->num_sms, ws, ws_bytes, &pl);
@@ -536,9 +549,11 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
   if (st != BQ_OK) return st;
   // Output y [batch][M][N] bf16 for the wide tiles' TMA-store epilogue: 128-row
   // x 32-column boxes with the 64-byte swizzle.
-  CUtensorMap map_y;
-  st = make_y_map(&map_y, y, M, N, count, sy);
-  if (st != BQ_OK) return st;
+  CUtensorMap map_y = map_a;  // placeholder when no bf16 output is written
+  if (y) {
+    st = make_y_map(&map_y, y, M, N, count, sy);
+    if (st != BQ_OK) return st;
+  }
 
   bq::GemmArgs g;
   memset(&g, 0, sizeof(g));
@@ -574,6 +589,9 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
   g.res_bstride = sr / 2;
   g.alpha = epi ? epi->alpha : 1.0f;
   g.act = epi ? epi->act : BQ_ACT_NONE;
+  g.q_out = static_cast<uint8_t*>(q_out);
+  g.sf_out = static_cast<uint8_t*>(sf_out);
+  g.sf_out_bstride = static_cast<int64_t>(bq_sf_bytes(M, N));
   if (pl.splits > 1 && !pl.cluster) {
     g.ws_ticket = static_cast<int*>(ws);
     g.ws_partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kTicketRegion);

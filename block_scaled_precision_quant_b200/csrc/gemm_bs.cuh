@@ -34,6 +34,7 @@
 #include <stdint.h>
 
 #include "bq_ptx.cuh"
+#include "mx_quant.cuh"
 
 namespace bq {
 
@@ -88,6 +89,11 @@ struct GemmArgs {
   int64_t ldres, res_bstride;  // elements
   float alpha;
   int act;
+  // optional quantized output (codes [M][ldy] u8, batch stride y_bstride
+  // bytes; scales in the MMA layout, batch stride sf_out_bstride bytes)
+  uint8_t *q_out;
+  uint8_t *sf_out;
+  int64_t sf_out_bstride;
   // split-K workspace: fp32 partials [units][128][BN] and per-tile tickets
   float *ws_partial;
   int *ws_ticket;
@@ -304,6 +310,96 @@ __device__ __forceinline__ void epi_bar_sync() {
   asm volatile("barrier.sync 1, 128;" ::: "memory");  // the 4 epilogue warps
 }
 
+// Quantized output of one 32-group: row m, columns q0 .. q0+31, the bf16
+// outputs packed in o (column 2i in the low half of word i) -- the same codes
+// and scale byte bq_act_quant gives for them.  Rows in [M, rows padded to
+// 128) get the padding scale 127, and the row's last group also writes the
+// padding columns of its scale atom.
+__device__ __forceinline__ void quant_out_row32(const GemmArgs &a, int b, int m, int q0,
+                                                const uint32_t (&o)[16]) {
+  const int64_t groups = a.N >> 5;
+  const int64_t katoms = (groups + 3) >> 2;
+  const int64_t rows_pad = (static_cast<int64_t>(a.M) + 127) / 128 * 128;
+  if (m >= rows_pad) return;
+  uint8_t *sfo = a.sf_out + b * a.sf_out_bstride;
+  const int g = q0 >> 5;
+  if (m < a.M) {
+    uint32_t bad = 0;
+    const int e = mx_exponent(bf16_amax_bits(o, bad));
+    uint32_t codes[8];
+    mx_encode(o, e, codes);
+    uint4 *qd = reinterpret_cast<uint4 *>(a.q_out + b * a.y_bstride +
+                                          static_cast<int64_t>(m) * a.ldy + q0);
+    qd[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+    qd[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+    sfo[sf_mma_offset(m, g, katoms)] = static_cast<uint8_t>(e + 127);
+  } else {
+    sfo[sf_mma_offset(m, g, katoms)] = 127;
+  }
+  if (g == groups - 1)
+    for (int64_t cc = groups; cc < katoms * 4; ++cc) sfo[sf_mma_offset(m, cc, katoms)] = 127;
+}
+
+// Swap-AB tile output through the staged bf16 tile, with the quantized
+// output: rows m of the tile go out as 16-byte vectors of y (when y is
+// written) and as 8-byte vectors of codes; the 4 lanes covering one 32-group
+// of a row meet through two shuffles for its amax.  The loop is warp-uniform
+// (every lane takes part in the shuffles).  The tile of the last activation
+// rows writes the padding rows' scale bytes, the tile of the last column
+// group the padding columns.
+template <int BN>
+__device__ __forceinline__ void copy_out_swap_q(const GemmArgs &a, const UnitPos &u, int epi_tid,
+                                                const __nv_bfloat16 *stage) {
+  const int n0 = u.tp * kBlockP;
+  const int m0 = u.tq * BN;
+  const int rows = min(BN, a.M - m0);
+  const int nvec = min(kBlockP / 8, (a.N - n0) / 8);  // a multiple of 4 (N % 32 == 0)
+  const int64_t groups = a.N >> 5;
+  const int64_t katoms = (groups + 3) >> 2;
+  uint8_t *sfo = a.sf_out + u.b * a.sf_out_bstride;
+  const int lane = epi_tid & 31;
+  for (int base = epi_tid & ~31; base < rows * 16; base += 128) {
+    const int i = base + lane;
+    const int r = i >> 4, v = i & 15;
+    const bool ok = i < rows * 16 && v < nvec;
+    const uint4 val =
+        ok ? *reinterpret_cast<const uint4 *>(stage + r * kBlockP + v * 8) : make_uint4(0, 0, 0, 0);
+    const int m = m0 + r;
+    const int n = n0 + v * 8;
+    if (ok && a.y)
+      *reinterpret_cast<uint4 *>(a.y + u.b * a.y_bstride + static_cast<int64_t>(m) * a.ldy + n) =
+          val;
+    const uint32_t w[4] = {val.x, val.y, val.z, val.w};
+    uint32_t bad = 0;
+    uint32_t mx = bf16_amax_bits(w, bad);
+    mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
+    mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
+    if (ok) {
+      const int e = mx_exponent(mx);
+      uint32_t codes[2];
+      mx_encode(w, e, codes);
+      *reinterpret_cast<uint2 *>(a.q_out + u.b * a.y_bstride + static_cast<int64_t>(m) * a.ldy +
+                                 n) = make_uint2(codes[0], codes[1]);
+      if ((v & 3) == 0) sfo[sf_mma_offset(m, n >> 5, katoms)] = static_cast<uint8_t>(e + 127);
+    }
+  }
+  // padding scale bytes
+  const int64_t g0 = n0 >> 5;
+  const int64_t g1 = g0 + nvec / 4;  // this tile's groups [g0, g1)
+  const int64_t gend = g1 == groups ? katoms * 4 : g1;
+  if (u.tq == a.tiles_q - 1) {  // rows [M, 128-row padding) of this tile's columns
+    const int64_t rows_pad = (static_cast<int64_t>(a.M) + 127) / 128 * 128;
+    const int64_t nc = gend - g0;
+    for (int64_t idx = epi_tid; idx < (rows_pad - a.M) * nc; idx += 128)
+      sfo[sf_mma_offset(a.M + idx / nc, g0 + idx % nc, katoms)] = 127;
+  }
+  if (gend > g1) {  // padding columns of this tile's real rows
+    const int64_t nc = gend - g1;
+    for (int64_t idx = epi_tid; idx < rows * nc; idx += 128)
+      sfo[sf_mma_offset(m0 + idx / nc, g1 + idx % nc, katoms)] = 127;
+  }
+}
+
 // 32 residual values of one row (4 x 16 bytes), zeros past N or without one.
 __device__ __forceinline__ void load_res32(const __nv_bfloat16 *rrow, int q0, int N,
                                            uint4 (&r)[4]) {
@@ -371,21 +467,24 @@ __device__ __forceinline__ void epilogue_rows_tma(const GemmArgs &a, const CUten
         o[4 * g + j] = *reinterpret_cast<const uint32_t *>(&p2);
       }
     }
-    uint8_t *buf = ystage + (c & 1) * kYChunkBytes;
-    if (epi_tid == 0) bulk_wait_group_read<1>();  // the store two chunks back has read buf
-    epi_bar_sync();
+    if (a.q_out) quant_out_row32(a, b, m, q0, o);
+    if (a.y) {  // uniform
+      uint8_t *buf = ystage + (c & 1) * kYChunkBytes;
+      if (epi_tid == 0) bulk_wait_group_read<1>();  // the store two chunks back has read buf
+      epi_bar_sync();
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-      *reinterpret_cast<uint4 *>(buf + row * 64 + ((j ^ ((row >> 1) & 3)) << 4)) =
-          make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
-    fence_proxy_async_smem();
-    epi_bar_sync();
-    if (epi_tid == 0) {
-      if (a.batch > 1)
-        tma_store_3d(tm_y, buf, q0, m0, b);
-      else
-        tma_store_2d(tm_y, buf, q0, m0);
-      bulk_commit_group();
+      for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<uint4 *>(buf + row * 64 + ((j ^ ((row >> 1) & 3)) << 4)) =
+            make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+      fence_proxy_async_smem();
+      epi_bar_sync();
+      if (epi_tid == 0) {
+        if (a.batch > 1)
+          tma_store_3d(tm_y, buf, q0, m0, b);
+        else
+          tma_store_2d(tm_y, buf, q0, m0);
+        bulk_commit_group();
+      }
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j) res[j] = res_next[j];
@@ -871,7 +970,10 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[acc]);
         epi_bar_sync();
-        copy_out_swap<BN>(a, u, epi_tid, stage);
+        if (a.q_out)
+          copy_out_swap_q<BN>(a, u, epi_tid, stage);
+        else
+          copy_out_swap<BN>(a, u, epi_tid, stage);
         if (unit + static_cast<int>(gridDim.x) < total_units) epi_bar_sync();  // staging free
       } else if constexpr (MODE == kSplitNone) {
         epilogue_rows_tma<BN>(a, &tm_y, t_row, u.b, u.tp * kBlockP, u.tq * BN, row, epi_tid,

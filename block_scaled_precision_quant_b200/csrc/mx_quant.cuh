@@ -1,0 +1,77 @@
+// mx_quant.cuh -- the per-32 MX quantizer's arithmetic, shared by the
+// activation quantizer kernel and the GEMM epilogue that emits its output in
+// the same format.
+//
+// The quantizer ("formats.py" page: act_scale, act_quant, _log2_ceil_pow2):
+//   amax = max(max|x|, fp32(1e-4));  t = fp32(amax * fp32(1/448))
+//   e    = ceil(log2 t) from t's exponent bits;  scale byte = e + 127
+//   q    = E4M3 round-to-nearest-even of clamp(x / 2^e, -448, 448)
+// x / 2^e is computed as x * 2^-e: 2^-e is an exact binary32 power of two for
+// every e the rule can produce (-22 .. 120), so the correctly rounded product
+// equals the correctly rounded quotient.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+namespace bq {
+
+// Byte offset of scale (row r, column c) in an MMA-layout buffer with
+// `katoms` = ceil(G / 4) atoms per 128-row band.
+__host__ __device__ __forceinline__ int64_t sf_mma_offset(int64_t r, int64_t c, int64_t katoms) {
+  return ((r >> 7) * katoms + (c >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3);
+}
+
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  const __nv_fp8x2_storage_t lo =
+      __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const __nv_fp8x2_storage_t hi =
+      __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
+// Largest magnitude bits (15 bits, sign dropped) of the bf16 pairs in w: an
+// integer max is order-preserving for non-negative floats.  `bad` collects
+// non-finite inputs (all-ones exponent).
+template <int NW>
+__device__ __forceinline__ uint32_t bf16_amax_bits(const uint32_t (&w)[NW], uint32_t &bad) {
+  uint32_t mx = 0;
+#pragma unroll
+  for (int i = 0; i < NW; ++i) {
+    const uint32_t lo = w[i] & 0x7FFFu, hi = (w[i] >> 16) & 0x7FFFu;
+    mx = max(mx, max(lo, hi));
+    bad |= ((lo & 0x7F80u) == 0x7F80u) | ((hi & 0x7F80u) == 0x7F80u);
+  }
+  return mx;
+}
+
+// Scale exponent e of a group from its amax bits.
+__device__ __forceinline__ int mx_exponent(uint32_t amax_bits) {
+  const float amax = fmaxf(__uint_as_float(amax_bits << 16), 1e-4f);
+  const float t = __fmul_rn(amax, __uint_as_float(0x3B124925u));  // fp32(1/448)
+  const uint32_t tb = __float_as_uint(t);
+  return static_cast<int>((tb >> 23) & 0xFFu) - 127 + ((tb & 0x7FFFFFu) != 0u ? 1 : 0);
+}
+
+// E4M3 codes of the 2 * NW bf16 values in w (element 2i in the low half of
+// word i) scaled by 2^-e, four codes per output word.
+template <int NW>
+__device__ __forceinline__ void mx_encode(const uint32_t (&w)[NW], int e,
+                                          uint32_t (&codes)[NW / 2]) {
+  const float inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e
+#pragma unroll
+  for (int i = 0; i < NW / 2; ++i) {
+    float f[4];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const uint32_t word = w[2 * i + j];
+      f[2 * j] = fminf(fmaxf(__fmul_rn(__uint_as_float(word << 16), inv), -448.0f), 448.0f);
+      f[2 * j + 1] =
+          fminf(fmaxf(__fmul_rn(__uint_as_float(word & 0xFFFF0000u), inv), -448.0f), 448.0f);
+    }
+    codes[i] = e4m3x4(f[0], f[1], f[2], f[3]);
+  }
+}
+
+}  // namespace bq

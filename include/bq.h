@@ -164,13 +164,31 @@ enum { BQ_ACT_NONE = 0, BQ_ACT_GELU = 1 };
  *   y = bf16_RNE( act(alpha * acc + bias[n]) + residual[m, n] )
  * act: BQ_ACT_NONE or BQ_ACT_GELU (erf form 0.5 t (1 + erf(t / sqrt 2))).
  * bias: [N] bf16 or NULL.  residual: [M, ld_residual] bf16 or NULL
- * (ld_residual % 8 == 0, 16-byte aligned). */
+ * (ld_residual % 8 == 0, 16-byte aligned).
+ *
+ * Quantized output (optional, q_out and sf_out both set or both NULL): the
+ * epilogue also applies bq_act_quant to y along N -- per 32 consecutive
+ * outputs of a row, the same amax, E8M0 scale and E4M3 codes as bq_act_quant
+ * on the bf16 y -- and writes q_out [M, N] u8 (E4M3 codes, row-major) and
+ * sf_out (bq_sf_bytes(M, N) bytes, the MMA scale layout with 127 padding), so
+ * the output feeds another GEMM as its activation operand directly.  The
+ * "fp4-gemm" page (README, "Available Functions" and "Tensor Contract": the
+ * bias+GELU epilogue that emits packed FP4 plus its scale layout for the
+ * following projection) describes this epilogue for NVFP4; here it is the
+ * MXFP8 form of the activation quantizer above.  Needs N % 32 == 0,
+ * q_out 16-byte aligned, sf_out 4-byte aligned; y may then be NULL (no bf16
+ * output written).  Batched calls step q_out by stride_y / 2 bytes and sf_out
+ * by bq_sf_bytes(M, N).  Schedules that split K are not available with it
+ * (an explicit split is refused with BQ_ERR_INVALID; the automatic schedule
+ * does not split). */
 typedef struct {
   const void *bias;
   const void *residual;
   int64_t ld_residual;
   float alpha;
   int act;
+  void *q_out;
+  void *sf_out;
 } bq_epilogue;
 
 /* Batched GEMM: `count` independent problems.  Strides are in BYTES between

@@ -438,3 +438,73 @@ def test_workspace_shared_across_problems():
         ref, sabs = c.oracle_full()
         assert_close(y, ref, c.tol(ref, sabs), f"shared workspace {M}x{N}x{K}/{s}")
         assert int(ws[:65536].count_nonzero().item()) == 0
+
+
+# ------------------------------------------------- quantized GEMM output --
+
+def _quant_out_case(c, config=None, write_y=True):
+    """GEMM with the MXFP8 output: y within tolerance of the oracle, and the
+    codes and scales (padding included) byte-equal to act_quant of y."""
+    aq, asf = bq.act_quant(to_dev_bf16(c.x))
+    bd = to_dev_u8(c.b)
+    kind = bq.BQ_SF_BLK32x32 if c.wk == bq.W_FP8BLK32 else bq.BQ_SF_ROW32
+    bsf = bq.pack_weight_scales(to_dev_u8(c.bsf), kind, c.N, c.K,
+                                e4m3_codes=bd if c.wk != bq.W_MXFP4 else None)
+    kw = dict(bias=to_dev_bf16(c.bias) if c.bias is not None else None,
+              residual=to_dev_bf16(c.res) if c.res is not None else None,
+              alpha=c.alpha, act=c.act, config=config)
+    y, q, sf = bq.gemm(c.wk, aq, asf, bd, bsf, c.M, c.N, c.K, quantize_out=True, **kw)
+    bq.device_status()
+    ref, sabs = c.oracle_full()
+    yv = bf16_to_f64(y.cpu().view(torch.int16).numpy().view(np.uint16))
+    assert_close(yv, ref, c.tol(ref, sabs), "quantized-output GEMM y")
+    q_ref, sf_ref = bq.act_quant(y)
+    assert torch.equal(q, q_ref)
+    assert torch.equal(sf, sf_ref)
+    oq, osf = oracle.act_quant(y.cpu().view(torch.int16).numpy().view(np.uint16))
+    assert np.array_equal(q.cpu().numpy(), oq)
+    assert np.array_equal(bq.unpack_scales(sf, c.M, c.N).cpu().numpy(), osf)
+    if not write_y:
+        y2, q2, sf2 = bq.gemm(c.wk, aq, asf, bd, bsf, c.M, c.N, c.K, quantize_out=True,
+                              write_y=False, **kw)
+        bq.device_status()
+        assert y2 is None and torch.equal(q2, q) and torch.equal(sf2, sf)
+
+
+@pytest.mark.parametrize("M,N,K,write_y", [(300, 800, 640, True), (128, 512, 256, False)])
+def test_quant_out_wide_tiles(M, N, K, write_y):
+    _quant_out_case(Case(bq.W_MXFP4, M, N, K, seed=81, bias=True, act=bq.BQ_ACT_GELU),
+                    config=bq.config(split_k=1, swap_ab=0, block_n=128), write_y=write_y)
+
+
+def test_quant_out_pair_tiles():
+    _quant_out_case(Case(bq.W_FP8BLK32, 520, 800, 512, seed=82, residual=True),
+                    config=bq.config(split_k=1, swap_ab=0, cta_pair=2), write_y=True)
+
+
+@pytest.mark.parametrize("M,N", [(41, 1536), (17, 800), (64, 640)])
+def test_quant_out_decode(M, N):
+    _quant_out_case(Case(bq.W_MXFP4, M, N, 1536, seed=83 + M, bias=True), write_y=(M != 17))
+
+
+def test_quant_out_auto_schedule_does_not_split():
+    """A long-K decode shape the automatic schedule would split: with the
+    quantized output it runs unsplit."""
+    _quant_out_case(Case(bq.W_MXFP4, 41, 1536, 6144, seed=85, bias=True))
+
+
+def test_quant_out_refusals():
+    c = Case(bq.W_MXFP4, 41, 520, 512)
+    aq, asf = bq.act_quant(to_dev_bf16(c.x))
+    bd = to_dev_u8(c.b)
+    bsf = bq.pack_weight_scales(to_dev_u8(c.bsf), bq.BQ_SF_ROW32, 520, 512)
+    with pytest.raises(bq.BqError) as e:  # N % 32 != 0
+        bq.gemm(bq.W_MXFP4, aq, asf, bd, bsf, 41, 520, 512, quantize_out=True)
+    assert e.value.status == bq.BQ_ERR_SHAPE
+    c2 = Case(bq.W_MXFP4, 41, 512, 512)
+    aq2, asf2 = bq.act_quant(to_dev_bf16(c2.x))
+    bsf2 = bq.pack_weight_scales(to_dev_u8(c2.bsf), bq.BQ_SF_ROW32, 512, 512)
+    with pytest.raises(bq.BqError) as e:  # explicit split-K
+        bq.gemm(bq.W_MXFP4, aq2, asf2, to_dev_u8(c2.b), bsf2, 41, 512, 512, quantize_out=True,
+                config=bq.config(split_k=2, swap_ab=1))
+    assert e.value.status == bq.BQ_ERR_INVALID
