@@ -44,6 +44,7 @@ EXPORTS = (
     "bq_gemm_workspace_bytes", "bq_gemm_mxfp8_mxfp4_epilogue", "bq_gemm_mxfp8_fp8blk32_epilogue",
     "bq_gemm_mxfp8_mxfp8_epilogue", "bq_device_status", "bq_device_status_detail",
     "bq_device_report", "bq_gemm_mxfp8_mxfp4_epilogue_noalloc", "bq_noalloc_scratch_bytes",
+    "bq_gemm_bf16act_epilogue",
 )
 
 
@@ -116,6 +117,9 @@ def lib():
             ctypes.POINTER(GemmConfig), vp]
         L.bq_gemm_mxfp8_mxfp4_epilogue_noalloc.restype = i32
         L.bq_noalloc_scratch_bytes.restype = sz
+        L.bq_gemm_bf16act_epilogue.argtypes = [i32, vp, i64, vp, vp, i64, i64, i64, vp,
+                                               ctypes.POINTER(Epilogue), vp, vp, vp, vp]
+        L.bq_gemm_bf16act_epilogue.restype = i32
         L.bq_gemm_workspace_bytes.argtypes = [i32, i64, i64, i64, i64, ctypes.POINTER(GemmConfig)]
         L.bq_gemm_workspace_bytes.restype = sz
         L.bq_device_status.argtypes = [vp]
@@ -314,6 +318,48 @@ def gemm(weight_kind, a_q, a_sf, b, b_sf, M, N, K, y=None, bias=None, residual=N
     if quantize_out:
         return (y if write_y else None), q_out, sf_out
     return y
+
+
+def gemm_bf16act(weight_kind, x, b, b_sf, M, N, K, y=None, bias=None, residual=None, alpha=1.0,
+                 act=BQ_ACT_NONE, store_act=False, status=None, quantize_out=False, write_y=True,
+                 a_q=None, a_sf=None):
+    """act_quant(x) and the GEMM of weight_kind in one launch (decode shapes:
+    M <= 64, K % 128 == 0): the GEMM quantizes the bf16 activations x [M, K]
+    itself.  store_act: also return the activation codes and MMA-layout scales
+    bq_act_quant would write.  Returns y, or a tuple (y, [q, sf], [a_q, a_sf])
+    when quantize_out / store_act ask for more."""
+    torch = _torch()
+    _need_cuda(x, b, b_sf, bias, residual, status)
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a bf16 [M, K] tensor with unit column stride")
+    if not write_y and not quantize_out:
+        raise ValueError("write_y=False needs quantize_out=True")
+    dev = x.device
+    if y is None and write_y:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    q_out = sf_out = None
+    if quantize_out:
+        q_out = torch.empty((M, N), dtype=torch.uint8, device=dev)
+        sf_out = torch.empty((sf_bytes(M, N),), dtype=torch.uint8, device=dev)
+    # the library may need the activation buffers (a long-K shape runs act_quant
+    # into them and a split GEMM); they are returned only with store_act
+    a_q = torch.empty((M, K), dtype=torch.uint8, device=dev) if a_q is None else a_q
+    a_sf = torch.empty((sf_bytes(M, K),), dtype=torch.uint8, device=dev) if a_sf is None else a_sf
+    epi = Epilogue(bias.data_ptr() if bias is not None else None,
+                   residual.data_ptr() if residual is not None else None,
+                   residual.stride(-2) if residual is not None else 0, float(alpha), int(act),
+                   q_out.data_ptr() if q_out is not None else None,
+                   sf_out.data_ptr() if sf_out is not None else None)
+    _check(lib().bq_gemm_bf16act_epilogue(
+        int(weight_kind), _ptr(x), x.stride(0), _ptr(b), _ptr(b_sf), M, N, K,
+        _ptr(y) if write_y else None, ctypes.byref(epi), _ptr(a_q), _ptr(a_sf), _ptr(status),
+        _stream()), "bq_gemm_bf16act_epilogue")
+    out = [y if write_y else None]
+    if quantize_out:
+        out += [q_out, sf_out]
+    if store_act:
+        out += [a_q, a_sf]
+    return out[0] if len(out) == 1 else tuple(out)
 
 
 def gemm_mxfp8_mxfp4(a_q, a_sf, b_fp4, b_sf, M, N, K, **kw):

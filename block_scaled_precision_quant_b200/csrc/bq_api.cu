@@ -324,13 +324,14 @@ int plan_for_call(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_
 
 // --------------------------------------------------------------- launches --
 
-template <int BN, int STAGES, int ACC, bool SWAP, bool P_FP4, bool Q_FP4, int MODE, int KC>
+template <int BN, int STAGES, int ACC, bool SWAP, bool P_FP4, bool Q_FP4, int MODE, int KC,
+          bool FUSEQ = false>
 int launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap& ty,
                 const bq::GemmArgs& args,
                 int64_t units, int num_sms, cudaStream_t stream) {
   constexpr bool CSPLIT = MODE == bq::kSplitCluster;
   using L = bq::KernelSmem<BN, STAGES, ACC, SWAP, MODE, KC>;
-  auto kern = bq::gemm_bs_kernel<BN, STAGES, ACC, SWAP, P_FP4, Q_FP4, MODE, KC>;
+  auto kern = bq::gemm_bs_kernel<BN, STAGES, ACC, SWAP, P_FP4, Q_FP4, MODE, KC, FUSEQ>;
   static bool attr_set[kMaxDevices] = {};
   static int per_sm_cache[kMaxDevices] = {};
   int dev = 0;
@@ -385,15 +386,15 @@ int launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap&
   return launch_status();
 }
 
-template <int BN, int STAGES, int ACC, bool SWAP, int MODE, int KC>
+template <int BN, int STAGES, int ACC, bool SWAP, int MODE, int KC, bool FUSEQ = false>
 int launch_kind(bool w_fp4, const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap& ty,
                 const bq::GemmArgs& args, int64_t u, int num_sms, cudaStream_t st) {
   // FP4 weights sit on the P side with SWAP, on the Q side otherwise.
   if (w_fp4)
-    return launch_gemm<BN, STAGES, ACC, SWAP, SWAP, !SWAP, MODE, KC>(tp, tq, ty, args, u, num_sms,
-                                                                    st);
-  return launch_gemm<BN, STAGES, ACC, SWAP, false, false, MODE, KC>(tp, tq, ty, args, u, num_sms,
-                                                                    st);
+    return launch_gemm<BN, STAGES, ACC, SWAP, SWAP, !SWAP, MODE, KC, FUSEQ>(tp, tq, ty, args, u,
+                                                                           num_sms, st);
+  return launch_gemm<BN, STAGES, ACC, SWAP, false, false, MODE, KC, FUSEQ>(tp, tq, ty, args, u,
+                                                                           num_sms, st);
 }
 
 template <int STAGES, int KC, bool Q_FP4>
@@ -455,6 +456,10 @@ int run_gemm(const Plan& pl, bool w_fp4, const CUtensorMap& tp, const CUtensorMa
     return pl.kc == 2 ? launch_kind<128, 3, 2, false, kNone, 2>(w_fp4, tp, tq, ty, a, u, ns, st)
                       : launch_kind<128, 6, 2, false, kNone, 1>(w_fp4, tp, tq, ty, a, u, ns, st);
   }
+  if (a.x) {  // fused activation quantization: unsplit 4-chunk swap tiles
+    return b32 ? launch_kind<32, 2, 1, true, kNone, 4, true>(w_fp4, tp, tq, ty, a, u, ns, st)
+               : launch_kind<64, 2, 1, true, kNone, 4, true>(w_fp4, tp, tq, ty, a, u, ns, st);
+  }
   if (pl.cluster) {
     if (pl.kc == 4)
       return b32 ? launch_kind<32, 1, 1, true, kCl, 4>(w_fp4, tp, tq, ty, a, u, ns, st)
@@ -472,10 +477,19 @@ int run_gemm(const Plan& pl, bool w_fp4, const CUtensorMap& tp, const CUtensorMa
              : launch_kind<64, 8, 1, true, kNone, 1>(w_fp4, tp, tq, ty, a, u, ns, st);
 }
 
+// Activations given as bf16 and quantized inside the GEMM (decode tiles).
+struct FusedAct {
+  const void* x;
+  int64_t ldx;
+  void* a_q_out;   // nullable
+  void* a_sf_out;  // nullable (set together with a_q_out)
+  int* status;     // nullable
+};
+
 int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, const void* b_sf,
                int64_t M, int64_t N, int64_t K, void* y, const bq_epilogue* epi,
                const bq_batch* batch, void* ws, size_t ws_bytes, const bq_gemm_config* cfg,
-               bq_stream_t stream) {
+               bq_stream_t stream, const FusedAct* fused = nullptr) {
   DevInfo* dev = nullptr;
   int st = current_device(&dev);
   if (st != BQ_OK) return st;
@@ -487,14 +501,23 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
   void* sf_out = epi ? epi->sf_out : nullptr;
   if ((q_out || sf_out) && N % 32 != 0) return BQ_ERR_SHAPE;
   if ((q_out != nullptr) != (sf_out != nullptr)) return BQ_ERR_NULL;
-  if (!a_q || !a_sf || !b || !b_sf || (!y && !q_out)) return BQ_ERR_NULL;
+  if ((!fused && (!a_q || !a_sf)) || !b || !b_sf || (!y && !q_out)) return BQ_ERR_NULL;
+  if (fused) {
+    // one activation tile of all M rows, whole 128-K chunks, one problem
+    if (M > 64 || K % 128 != 0 || (batch && batch->count > 1)) return BQ_ERR_SHAPE;
+    if (!fused->x) return BQ_ERR_NULL;
+    if (fused->ldx < K || fused->ldx % 8 != 0 || !aligned(fused->x, 16)) return BQ_ERR_ALIGN;
+    if ((fused->a_q_out != nullptr) != (fused->a_sf_out != nullptr)) return BQ_ERR_NULL;
+    if (fused->a_q_out && (!aligned(fused->a_q_out, 16) || !aligned(fused->a_sf_out, 4)))
+      return BQ_ERR_ALIGN;
+  }
   if (q_out && (!aligned(q_out, 16) || !aligned(sf_out, 4))) return BQ_ERR_ALIGN;
   const bool w_fp4 = wk == kMxfp4;
   if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF || count > 65535) return BQ_ERR_SHAPE;
   if (N % 8 != 0) return BQ_ERR_SHAPE;
   if (w_fp4 && K % 128 != 0) return BQ_ERR_SHAPE;
-  if (!aligned(a_q, 16) || !aligned(a_sf, 16) || !aligned(b_sf, 16) || (y && !aligned(y, 16)) ||
-      !aligned(b, w_fp4 ? 32 : 16))
+  if ((!fused && (!aligned(a_q, 16) || !aligned(a_sf, 16))) || !aligned(b_sf, 16) ||
+      (y && !aligned(y, 16)) || !aligned(b, w_fp4 ? 32 : 16))
     return BQ_ERR_ALIGN;
   const void* bias = epi ? epi->bias : nullptr;
   const void* res = epi ? epi->residual : nullptr;
@@ -523,6 +546,10 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
     cfg_q.split_k = 1;
     cfg = &cfg_q;
   }
+  if (fused) {  // its one schedule: swap-AB, unsplit, 4 chunks per stage
+    cfg_q = bq_gemm_config{0, 1, 1, BQ_SPLIT_AUTO, 4, 1};
+    cfg = &cfg_q;
+  }
   Plan pl;
   st = plan_for_call(M, N, K, count, cfg, dev->num_sms, ws, ws_bytes, &pl);
   if (st != BQ_OK) return st;
@@ -542,11 +569,16 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
   const int b_box = (pl.swap || pl.pair) ? 128 : pl.bn;  // a pair CTA loads 128 of 256 rows
   const bool a_batched = count > 1 && sa != 0;
   const bool b_batched = count > 1 && sb != 0;
-  st = make_operand_map(&map_a, a_q, false, K, M, K, a_batched ? count : 1, sa, a_box, pl.kc);
-  if (st != BQ_OK) return st;
+  if (fused) {
+    st = BQ_OK;  // no activation copies: map_a is set to a placeholder below
+  } else {
+    st = make_operand_map(&map_a, a_q, false, K, M, K, a_batched ? count : 1, sa, a_box, pl.kc);
+    if (st != BQ_OK) return st;
+  }
   st = make_operand_map(&map_b, b, w_fp4, K, N, w_fp4 ? K / 2 : K, b_batched ? count : 1, sb,
                         b_box, pl.kc);
   if (st != BQ_OK) return st;
+  if (fused) map_a = map_b;
   // Output y [batch][M][N] bf16 for the wide tiles' TMA-store epilogue: 128-row
   // x 32-column boxes with the 64-byte swizzle.
   CUtensorMap map_y = map_a;  // placeholder when no bf16 output is written
@@ -569,7 +601,8 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
   g.raster_group = 8;
   g.sf_katoms = ceil_div(K, 128);
   g.sf_q_rowatoms = ceil_div(pl.swap ? M : N, 128);
-  g.q_box_rows = pl.swap ? a_box : b_box;
+  // the fused quantizer lays the activation tile out with chunks BN rows apart
+  g.q_box_rows = fused ? pl.bn : (pl.swap ? a_box : b_box);
   g.split_lg = 0;
   while ((1 << g.split_lg) < pl.splits) ++g.split_lg;
   const uint8_t* sfa = static_cast<const uint8_t*>(a_sf);
@@ -589,6 +622,13 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
   g.res_bstride = sr / 2;
   g.alpha = epi ? epi->alpha : 1.0f;
   g.act = epi ? epi->act : BQ_ACT_NONE;
+  if (fused) {
+    g.x = static_cast<const __nv_bfloat16*>(fused->x);
+    g.ldx = fused->ldx;
+    g.a_q_out = static_cast<uint8_t*>(fused->a_q_out);
+    g.a_sf_out = static_cast<uint8_t*>(fused->a_sf_out);
+    g.status = fused->status;
+  }
   g.q_out = static_cast<uint8_t*>(q_out);
   g.sf_out = static_cast<uint8_t*>(sf_out);
   g.sf_out_bstride = static_cast<int64_t>(bq_sf_bytes(M, N));
@@ -815,6 +855,33 @@ int bq_gemm_mxfp8_fp8blk32_epilogue(const void* a_q, const void* a_sf, const voi
                                     const bq_gemm_config* cfg, bq_stream_t stream) {
   return gemm_entry(kFp8Blk32, a_q, a_sf, b_e4m3, b_sf, M, N, K, y_bf16, epi, batch, workspace,
                     workspace_bytes, cfg, stream);
+}
+
+int bq_gemm_bf16act_epilogue(int weight_kind, const void* x_bf16, int64_t ldx, const void* b,
+                             const void* b_sf, int64_t M, int64_t N, int64_t K, void* y_bf16,
+                             const bq_epilogue* epi, void* a_q_out, void* a_sf_out,
+                             int* d_status, bq_stream_t stream) {
+  if (weight_kind < 0 || weight_kind > 2) return BQ_ERR_INVALID;
+  // A long K loop is faster split over a cluster than in one CTA: then the
+  // activations are quantized by bq_act_quant into the caller's buffers and
+  // the split GEMM consumes them (two launches).  The quantized output needs
+  // an unsplit tile, so it always takes the fused kernel.
+  if (M > 0 && M <= 64 && N > 0 && K > 0 && !(epi && epi->q_out)) {
+    DevInfo* dev = nullptr;
+    int st = current_device(&dev);
+    if (st != BQ_OK) return st;
+    Plan pl;
+    if (make_plan(M, N, K, 1, nullptr, dev->num_sms, &pl) == BQ_OK && pl.splits > 1) {
+      if (!a_q_out || !a_sf_out) return BQ_ERR_NULL;
+      st = bq_act_quant(x_bf16, M, K, ldx, a_q_out, a_sf_out, nullptr, d_status, stream);
+      if (st != BQ_OK) return st;
+      return gemm_entry(static_cast<WeightKind>(weight_kind), a_q_out, a_sf_out, b, b_sf, M, N,
+                        K, y_bf16, epi, nullptr, nullptr, 0, nullptr, stream);
+    }
+  }
+  const FusedAct f{x_bf16, ldx, a_q_out, a_sf_out, d_status};
+  return gemm_entry(static_cast<WeightKind>(weight_kind), nullptr, nullptr, b, b_sf, M, N, K,
+                    y_bf16, epi, nullptr, nullptr, 0, nullptr, stream, &f);
 }
 
 int bq_gemm_mxfp8_mxfp8_epilogue(const void* a_q, const void* a_sf, const void* b_e4m3,

@@ -60,32 +60,38 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// The waiting thread is suspended (issuing nothing) until the phase completes
+// or kWaitSuspendNs pass, so waiting roles leave the schedulers to the warps
+// that work.
+constexpr uint32_t kWaitSuspendNs = 20000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "n"(kWaitSuspendNs)
       : "memory");
   return ok != 0;
 }
 
 // Wait until the phase with the given parity of `bar` has completed.  Gives
 // up after BQ_WAIT_NS (or as soon as *abort is set by another role), records
-// the wait site in *err and returns false.  The timer is only read after
-// many failed polls, so ordinary waits never touch it.
+// the wait site in *err and returns false.  Each poll suspends the thread up
+// to kWaitSuspendNs (it wakes when the phase completes); the timer is read
+// only after several failed polls, so ordinary waits never touch it.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err,
                                           volatile int *abort, int site) {
   const uint32_t b = smem_u32(bar);
 #pragma unroll 1
-  for (int i = 0; i < 4096; ++i)
+  for (int i = 0; i < 16; ++i)
     if (mbar_try_wait(b, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
 #pragma unroll 1
-    for (int i = 0; i < 256; ++i)
+    for (int i = 0; i < 16; ++i)
       if (mbar_try_wait(b, parity)) return true;
     if (*abort) return false;
     if (globaltimer() - t0 > BQ_WAIT_NS) {
@@ -101,7 +107,7 @@ __device__ __forceinline__ bool mbar_wait_timed(uint64_t *bar, uint32_t parity, 
                                                 int site) {
   const uint32_t b = smem_u32(bar);
 #pragma unroll 1
-  for (int i = 0; i < 4096; ++i)
+  for (int i = 0; i < 16; ++i)
     if (mbar_try_wait(b, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (!mbar_try_wait(b, parity)) {
@@ -168,10 +174,10 @@ __device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t bar, uint32_t
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "n"(kWaitSuspendNs)
       : "memory");
   return ok != 0;
 }
@@ -181,12 +187,12 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
                                                   volatile int *abort, int site) {
   const uint32_t b = smem_u32(bar);
 #pragma unroll 1
-  for (int i = 0; i < 4096; ++i)
+  for (int i = 0; i < 16; ++i)
     if (mbar_try_wait_acq_cluster(b, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
 #pragma unroll 1
-    for (int i = 0; i < 256; ++i)
+    for (int i = 0; i < 16; ++i)
       if (mbar_try_wait_acq_cluster(b, parity)) return true;
     if (*abort) return false;
     if (globaltimer() - t0 > BQ_WAIT_NS) {

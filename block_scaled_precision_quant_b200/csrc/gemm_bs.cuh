@@ -94,6 +94,14 @@ struct GemmArgs {
   uint8_t *q_out;
   uint8_t *sf_out;
   int64_t sf_out_bstride;
+  // fused activation quantization (swap-AB decode tiles): bf16 activations x
+  // [M, ldx]; optionally their codes [M, K] and MMA-layout scales are also
+  // stored (by the CTAs of the first weight tile), non-finite input reported
+  const __nv_bfloat16 *x;
+  int64_t ldx;
+  uint8_t *a_q_out;
+  uint8_t *a_sf_out;
+  int *status;
   // split-K workspace: fp32 partials [units][128][BN] and per-tile tickets
   float *ws_partial;
   int *ws_ticket;
@@ -149,6 +157,7 @@ struct GemmSmem {
   static constexpr int kNumBars = 2 * STAGES + 2 * ACC + 1 + (CSPLIT ? 2 : 0) + (LANDING ? 1 : 0);
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 64 + 1024;  // + alignment slack
+  static constexpr int kStages = STAGES;
   static constexpr int kTmemUsed = ACC * BN + STAGES * kSfCols;
   static constexpr int kTmemCols = kTmemUsed <= 32    ? 32
                                    : kTmemUsed <= 64  ? 64
@@ -667,7 +676,102 @@ __device__ __forceinline__ void cluster_reduce_local(const GemmArgs &a, const Un
   }
 }
 
-template <int BN, int STAGES, int ACC, bool SWAP, bool P_FP4, bool Q_FP4, int MODE, int KC>
+// Fused activation quantizer (swap-AB tiles whose activation tile holds all M
+// rows): for each stage of the unit the epilogue warps read the stage's bf16
+// inputs, apply the activation quantizer per 32-group (the same arithmetic as
+// bq_act_quant) and write the E4M3 codes straight into the stage in the
+// layout a TMA copy with the 128-byte swizzle would give (row r at r * 128,
+// 16-byte unit j at j ^ (r % 8)) and the scale bytes into the stage's scale
+// atom; then each warp arrives on the stage barrier.  Up to kFusedGroups
+// groups per thread are loaded before any is quantized (a 41-row, 512-K stage
+// in one round trip).  The CTAs of the first weight tile
+// also store the codes and scales to global memory when asked.
+constexpr int kFusedGroups = 3;
+
+template <class L, int KC>
+__device__ __forceinline__ bool fused_quant_unit(const GemmArgs &a, const UnitPos &u,
+                                                 uint8_t *smem, uint64_t *full, uint64_t *empty,
+                                                 int &stage, uint32_t &phase, int epi_tid,
+                                                 int lane, volatile int *abort_flag) {
+  const int M = a.M;
+  const bool store_out = u.tp == 0 && a.a_q_out != nullptr;
+  const int64_t katoms = (static_cast<int64_t>(a.K) / 32 + 3) / 4;
+  const int q_chunk = a.q_box_rows * kBlockK;
+  for (int kt = u.kt0; kt < u.kt1; kt += KC) {
+    if (!mbar_wait(&empty[stage], phase ^ 1, a.err, abort_flag, kWaitProdEmpty)) return false;
+    const int nv = min(KC, u.kt1 - kt);
+    const int gpr = nv * 4;  // 32-groups per row in this stage
+    const int total = M * gpr;
+    uint8_t *sq = smem + L::kOffQ + stage * L::kBytesQ;
+    uint8_t *ssf = smem + L::kOffSfq + stage * L::kSfqBytes;
+#pragma unroll 1
+    for (int base = 0; base < total; base += 128 * kFusedGroups) {
+      uint32_t w[kFusedGroups][16];
+      int row[kFusedGroups], gk[kFusedGroups];
+#pragma unroll
+      for (int j = 0; j < kFusedGroups; ++j) {
+        const int idx = base + epi_tid + 128 * j;
+        row[j] = idx / gpr;
+        gk[j] = idx - row[j] * gpr;
+        if (idx < total) {
+          const uint4 *src = reinterpret_cast<const uint4 *>(
+              a.x + static_cast<int64_t>(row[j]) * a.ldx + kt * kBlockK + gk[j] * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint4 t = __ldg(src + v);
+            w[j][4 * v] = t.x;
+            w[j][4 * v + 1] = t.y;
+            w[j][4 * v + 2] = t.z;
+            w[j][4 * v + 3] = t.w;
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kFusedGroups; ++j) {
+        if (base + epi_tid + 128 * j >= total) break;
+        uint32_t bad = 0;
+        const int e = mx_exponent(bf16_amax_bits(w[j], bad));
+        uint32_t codes[8];
+        mx_encode(w[j], e, codes);
+        const int r = row[j];
+        const int c = gk[j] >> 2;  // chunk of the stage
+        const int u0 = (gk[j] & 3) * 2;
+        uint8_t *rowp = sq + c * q_chunk + r * kBlockK;
+        *reinterpret_cast<uint4 *>(rowp + ((u0 ^ (r & 7)) << 4)) =
+            make_uint4(codes[0], codes[1], codes[2], codes[3]);
+        *reinterpret_cast<uint4 *>(rowp + (((u0 + 1) ^ (r & 7)) << 4)) =
+            make_uint4(codes[4], codes[5], codes[6], codes[7]);
+        ssf[c * kSfAtom + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (gk[j] & 3)] =
+            static_cast<uint8_t>(e + 127);
+        if (store_out) {
+          const int64_t col = static_cast<int64_t>(kt) * kBlockK + gk[j] * 32;
+          uint4 *qd = reinterpret_cast<uint4 *>(a.a_q_out + static_cast<int64_t>(r) * a.K + col);
+          qd[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+          qd[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+          a.a_sf_out[sf_mma_offset(r, col >> 5, katoms)] = static_cast<uint8_t>(e + 127);
+          if (bad && a.status) atomicOr(a.status, 1);
+        }
+      }
+    }
+    fence_proxy_async_smem();  // the MMA reads the stage through the async proxy
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&full[stage]);
+    if (++stage == L::kStages) {
+      stage = 0;
+      phase ^= 1;
+    }
+  }
+  if (store_out) {  // padding rows of the stored scales (K % 128 == 0: no padding columns)
+    const int64_t rows_pad = (static_cast<int64_t>(M) + 127) / 128 * 128;
+    const int64_t c0 = static_cast<int64_t>(u.kt0) * 4, c1 = static_cast<int64_t>(u.kt1) * 4;
+    for (int64_t idx = epi_tid; idx < (rows_pad - M) * (c1 - c0); idx += 128)
+      a.a_sf_out[sf_mma_offset(M + idx / (c1 - c0), c0 + idx % (c1 - c0), katoms)] = 127;
+  }
+  return true;
+}
+
+template <int BN, int STAGES, int ACC, bool SWAP, bool P_FP4, bool Q_FP4, int MODE, int KC,
+          bool FUSEQ = false>
 __global__ void __launch_bounds__(kNumThreads, 1)
     gemm_bs_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_y, const GemmArgs a) {
@@ -718,7 +822,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   int pre_n = 0;
   if (threadIdx.x == 0) {
     for (int st = 0; st < STAGES; ++st) {
-      mbar_init(&full[st], kCopyThreads);  // one arrival per copy thread
+      // one arrival per copy thread; with fused activation quantization the
+      // two weight copiers and the four quantizing warps
+      mbar_init(&full[st], FUSEQ ? 6 : kCopyThreads);
       mbar_init(&empty[st], 1);
     }
     for (int st = 0; st < ACC; ++st) {
@@ -762,8 +868,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     // kernel; the activation copies do, and once every CTA's activation-operand
     // thread is past that wait the next kernel in the stream may launch (it,
     // in turn, waits for this grid before reading its outputs).
-    if (lane == 0) {
-      const bool weights = warp == 0 || warp == kWsfWarp;
+    const bool weights = warp == 0 || warp == kWsfWarp;
+    if (lane == 0 && (weights || !FUSEQ)) {
       const bool scales = warp == kWsfWarp || warp == kAsfWarp;
       const bool p_side = weights == SWAP;
       if (!weights) {
@@ -873,10 +979,21 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     uint32_t acc_phase = 0;
     uint32_t ready_phase = 0, free_phase = 0, land_phase = 0;
     bool free_pending = false;  // CSPLIT: owners may still be reading the previous tile
-    // The bias and residual may come from the preceding kernel.
+    // The bias and residual (and the fused path's activations) may come from
+    // the preceding kernel.
     griddep_wait();
+    int qstage = 0;
+    uint32_t qphase = 0;
+    if constexpr (FUSEQ) {
+      if (epi_tid == 0) griddep_launch_dependents();
+    }
     for (int unit = blockIdx.x; unit < total_units; unit += gridDim.x) {
       const UnitPos u = unit_pos(a, unit);
+      if constexpr (FUSEQ) {
+        if (!fused_quant_unit<L, KC>(a, u, smem, full, empty, qstage, qphase, epi_tid, lane,
+                                     abort_flag))
+          break;
+      }
       const int prow = u.tp * kBlockP + row;
       // Swap-AB: the output column (bias index) of this thread's row is known
       // before the accumulator is; fetch its bias while the mainloop runs.

@@ -256,6 +256,38 @@ int bq_gemm_mxfp8_mxfp8_epilogue(const void *a_q, const void *a_sf, const void *
                                  size_t workspace_bytes, const bq_gemm_config *cfg,
                                  bq_stream_t stream);
 
+/* ---- activation quantization fused into the decode GEMM -------------------
+ *
+ * bq_gemm_bf16act_epilogue -- bq_act_quant followed by the *_epilogue GEMM of
+ * weight_kind (0 mxfp4, 1 fp8blk32, 2 mxfp8) in one launch, for decode-shaped
+ * problems: the GEMM's CTAs quantize the bf16 activations x [M, ldx] per
+ * 32-group (the bq_act_quant arithmetic) straight into their shared-memory
+ * operand stages, so neither the separate launch nor the codes' round trip
+ * through memory is on the path.  The results equal bq_act_quant + the
+ * epilogue GEMM bit for bit.  a_q_out [M, K] u8 and a_sf_out
+ * (bq_sf_bytes(M, K) bytes, MMA layout) optionally receive the activation
+ * codes and scales as bq_act_quant writes them; d_status (nullable) gets bit 0
+ * set for a non-finite input, as with bq_act_quant.  When the problem's K
+ * loop is long enough for a split schedule to win (the 6144-deep decode
+ * projection), the call runs bq_act_quant into a_q_out / a_sf_out and the
+ * split GEMM instead (two launches; the buffers are then required,
+ * BQ_ERR_NULL without them); with a quantized output it always fuses.
+ * Scope: 1 <= M <= 64,
+ * K % 128 == 0, one problem (no batch), ldx % 8 == 0, x 16-byte aligned; the
+ * epilogue options of bq_epilogue apply (quantized output included).  The
+ * "fp4-gemm" page ("Minimal Usage") produces the packed activations and their
+ * scale layout from bf16 with a separate producer call before the GEMM; here
+ * that producer runs inside the GEMM.  Errors as the *_epilogue calls,
+ * BQ_ERR_SHAPE outside the scope.
+ * Measured on B200 it is slower than the two calls for the decode shapes
+ * (every CTA of the GEMM quantizes the whole activation block, and its
+ * ordinary loads are throttled while shared memory holds the operand ring):
+ * it is provided for callers that want one launch per layer. */
+int bq_gemm_bf16act_epilogue(int weight_kind, const void *x_bf16, int64_t ldx, const void *b,
+                             const void *b_sf, int64_t M, int64_t N, int64_t K, void *y_bf16,
+                             const bq_epilogue *epi, void *a_q_out, void *a_sf_out, int *d_status,
+                             bq_stream_t stream);
+
 /* ---- allocation-free GEMM -------------------------------------------------
  *
  * No counterpart on the pages: this is a library convenience.

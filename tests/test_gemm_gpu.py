@@ -508,3 +508,82 @@ def test_quant_out_refusals():
         bq.gemm(bq.W_MXFP4, aq2, asf2, to_dev_u8(c2.b), bsf2, 41, 512, 512, quantize_out=True,
                 config=bq.config(split_k=2, swap_ab=1))
     assert e.value.status == bq.BQ_ERR_INVALID
+
+
+# ------------------------------------- act_quant fused into the decode GEMM --
+
+def _fused_case(c, quantize_out=False, check_oracle=True,
+                ref_config=bq.config(split_k=1, swap_ab=1, k_chunks=4)):
+    """bq_gemm_bf16act_epilogue against bq_act_quant + the epilogue GEMM: y,
+    the stored activation codes / scales and the status word bit for bit;
+    y within tolerance of the oracle."""
+    xd = to_dev_bf16(c.x)
+    bd = to_dev_u8(c.b)
+    kind = bq.BQ_SF_BLK32x32 if c.wk == bq.W_FP8BLK32 else bq.BQ_SF_ROW32
+    bsf = bq.pack_weight_scales(to_dev_u8(c.bsf), kind, c.N, c.K,
+                                e4m3_codes=bd if c.wk != bq.W_MXFP4 else None)
+    kw = dict(bias=to_dev_bf16(c.bias) if c.bias is not None else None,
+              residual=to_dev_bf16(c.res) if c.res is not None else None,
+              alpha=c.alpha, act=c.act)
+    st_ref = torch.zeros(1, dtype=torch.int32, device="cuda")
+    aq, asf = bq.act_quant(xd, status=st_ref)
+    ref2 = bq.gemm(c.wk, aq, asf, bd, bsf, c.M, c.N, c.K, quantize_out=quantize_out,
+                   config=ref_config, **kw)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = bq.gemm_bf16act(c.wk, xd, bd, bsf, c.M, c.N, c.K, store_act=True, status=st,
+                          quantize_out=quantize_out, **kw)
+    bq.device_status()
+    if quantize_out:
+        y, q, sf, gq, gsf = got
+        y_ref, q_ref, sf_ref = ref2
+        assert torch.equal(q, q_ref) and torch.equal(sf, sf_ref)
+    else:
+        y, gq, gsf = got
+        y_ref = ref2
+    assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16))
+    assert torch.equal(gq, aq) and torch.equal(gsf, asf)
+    assert int(st.item()) == int(st_ref.item())
+    if not check_oracle:  # a non-finite input: y carries NaN; equality above is the check
+        return int(st.item())
+    ref, sabs = c.oracle_full()
+    yv = bf16_to_f64(y.cpu().view(torch.int16).numpy().view(np.uint16))
+    assert_close(yv, ref, c.tol(ref, sabs), "fused act_quant GEMM")
+
+
+@pytest.mark.parametrize("M", [1, 17, 41, 64])
+def test_fused_act_quant_decode(M):
+    _fused_case(Case(bq.W_MXFP4, M, 4608 if M == 41 else 520, 640 if M != 41 else 1536,
+                     seed=90 + M, bias=True))
+
+
+@pytest.mark.parametrize("wk", [bq.W_FP8BLK32, bq.W_MXFP8])
+def test_fused_act_quant_fp8_weights(wk):
+    _fused_case(Case(wk, 41, 384, 1024, seed=95, residual=True, alpha=0.5))
+
+
+def test_fused_act_quant_long_k_split():
+    """A 6144-deep decode projection: the call quantizes into the activation
+    buffers and runs the split GEMM; same results as the two calls."""
+    _fused_case(Case(bq.W_MXFP4, 41, 1536, 6144, seed=98, bias=True), ref_config=None)
+
+
+def test_fused_act_quant_gelu_quant_out():
+    _fused_case(Case(bq.W_MXFP4, 33, 1536, 6144, seed=96, bias=True, act=bq.BQ_ACT_GELU),
+                quantize_out=True)
+
+
+def test_fused_act_quant_nonfinite_and_refusals():
+    c = Case(bq.W_MXFP4, 8, 256, 256, seed=97)
+    x = c.x.copy()
+    x[3, 77] = 0x7F80  # +Inf
+    c.x = x
+    assert _fused_case(c, check_oracle=False) & 1  # status bit, codes as bq_act_quant's
+    xd = to_dev_bf16(c.x)
+    bsf = bq.pack_weight_scales(to_dev_u8(c.bsf), bq.BQ_SF_ROW32, 256, 256)
+    for M, K in ((65, 256), (8, 192)):  # M > 64, K % 128 != 0
+        xs = to_dev_bf16(synth.activations(M, K, seed=1))
+        with pytest.raises(bq.BqError) as e:
+            bq.gemm_bf16act(bq.W_MXFP8, xs, torch.zeros((256, K), dtype=torch.uint8,
+                                                         device="cuda"),
+                            bsf, M, 256, K)
+        assert e.value.status in (bq.BQ_ERR_SHAPE,)
