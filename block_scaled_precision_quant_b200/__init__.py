@@ -44,7 +44,7 @@ EXPORTS = (
     "bq_gemm_workspace_bytes", "bq_gemm_mxfp8_mxfp4_epilogue", "bq_gemm_mxfp8_fp8blk32_epilogue",
     "bq_gemm_mxfp8_mxfp8_epilogue", "bq_device_status", "bq_device_status_detail",
     "bq_device_report", "bq_gemm_mxfp8_mxfp4_epilogue_noalloc", "bq_noalloc_scratch_bytes",
-    "bq_gemm_bf16act_epilogue",
+    "bq_gemm_bf16act_epilogue", "bq_gemm_plan",
 )
 
 
@@ -122,6 +122,9 @@ def lib():
         L.bq_gemm_bf16act_epilogue.restype = i32
         L.bq_gemm_workspace_bytes.argtypes = [i32, i64, i64, i64, i64, ctypes.POINTER(GemmConfig)]
         L.bq_gemm_workspace_bytes.restype = sz
+        L.bq_gemm_plan.argtypes = [i64, i64, i64, i64, ctypes.POINTER(GemmConfig), i32,
+                                   ctypes.POINTER(GemmConfig)]
+        L.bq_gemm_plan.restype = i32
         L.bq_device_status.argtypes = [vp]
         L.bq_device_status.restype = i32
         L.bq_device_status_detail.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
@@ -246,6 +249,15 @@ def workspace_bytes(weight_kind, M, N, K, batch=1, config=None) -> int:
     cfg = config if config is not None else None
     return int(lib().bq_gemm_workspace_bytes(int(weight_kind), M, N, K, batch,
                                              ctypes.byref(cfg) if cfg is not None else None))
+
+
+def plan(M, N, K, batch=1, config=None, num_sms=148) -> GemmConfig:
+    """The schedule the built-in dispatch picks (host-only, no device): every
+    GemmConfig field resolved for a device with num_sms SMs."""
+    out = GemmConfig()
+    _check(lib().bq_gemm_plan(M, N, K, batch, ctypes.byref(config) if config is not None
+                              else None, num_sms, ctypes.byref(out)), "bq_gemm_plan")
+    return out
 
 
 def _workspace(device, nbytes):

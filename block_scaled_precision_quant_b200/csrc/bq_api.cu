@@ -155,15 +155,18 @@ int make_scale_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, in
   return r == CUDA_SUCCESS ? BQ_OK : BQ_ERR_ALIGN;
 }
 
-// The output y (bf16, row pitch N) as (N, M[, batch]); box 32 x 128 with the
-// 64-byte swizzle the epilogue's staging tile uses.
-int make_y_map(CUtensorMap* m, void* y, int64_t M, int64_t N, int64_t batch, int64_t batch_bytes) {
+// A bf16 [batch][M][ld] matrix of N used columns (the output y, or the
+// residual) as (N, M[, batch]); box 32 x 128 with the 64-byte swizzle of the
+// epilogue's staging tile.
+int make_y_map(CUtensorMap* m, const void* y, int64_t M, int64_t N, int64_t ld, int64_t batch,
+               int64_t batch_bytes) {
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M),
                         static_cast<cuuint64_t>(batch)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(N * 2), static_cast<cuuint64_t>(batch_bytes)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld * 2), static_cast<cuuint64_t>(batch_bytes)};
   cuuint32_t box[3] = {32u, 128u, 1u};
   cuuint32_t estr[3] = {1u, 1u, 1u};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, batch > 1 ? 3 : 2, y, dims, strides,
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, batch > 1 ? 3 : 2,
+                        const_cast<void*>(y), dims, strides,
                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? BQ_OK : BQ_ERR_ALIGN;
@@ -225,13 +228,15 @@ int make_plan(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_conf
       // 128x256 tile, whose single TMEM accumulator leaves its epilogue
       // unoverlapped, pays ~7 units of epilogue per tile; 128x128 tiles keep
       // two accumulators and expose only the last epilogue.  Pick the width
-      // whose waves of persistent CTAs finish first.
-      const int64_t t256 = batch * p->tiles_p * ceil_div(N, 256);
-      const int64_t t128 = batch * p->tiles_p * ceil_div(N, 128);
+      // whose tiles per SM finish first.  Tiles per SM are counted
+      // fractionally: a partial last wave runs on fewer SMs, which under the
+      // power cap clock higher, and the sweeps fit that better than whole
+      // waves.
+      const double t256 = static_cast<double>(batch * p->tiles_p * ceil_div(N, 256));
+      const double t128 = static_cast<double>(batch * p->tiles_p * ceil_div(N, 128));
       const double kt = static_cast<double>(ceil_div(K, 128));
-      const double c256 = static_cast<double>((t256 + num_sms - 1) / num_sms) * (kt + 7.0);
-      const double c128 =
-          static_cast<double>((t128 + num_sms - 1) / num_sms) * kt * 0.61 + 3.5;
+      const double c256 = t256 / num_sms * (kt + 7.0);
+      const double c128 = t128 / num_sms * kt * 0.61 + 3.5;
       p->bn = (N > 128 && c256 <= c128) ? 256 : 128;
     }
     if (p->bn != 128 && p->bn != 256) return BQ_ERR_INVALID;
@@ -257,12 +262,13 @@ int make_plan(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_conf
   const bool pow2 = (splits & (splits - 1)) == 0;
   p->cluster = p->swap && splits > 1 && pow2 && splits <= kMaxClusterSplit && !use_ws;
   if (req_mode == BQ_SPLIT_CLUSTER && splits > 1 && !p->cluster) return BQ_ERR_INVALID;
-  // 256x256 pair tiles (sweeps: +3-8 % over the best single-SM tile once a
-  // tile's K loop is >= 32 blocks and the pairs fill the SMs; shorter loops
-  // lose to 128x128 tiles, whose two accumulators hide the epilogue).
+  // 256x256 pair tiles (sweeps: ~5 % over the best single-SM tile once a
+  // tile's K loop is >= 32 blocks and each pair walks >= 4 tiles, where the
+  // steady-state mainloop dominates; with fewer tiles per pair the pair's
+  // longer prologue and its exposed epilogue cost more than it saves).
   const bool auto_pair = req_pair == 0 && req_bn == 0 && req_split <= 1 && req_kc != 4 &&
                          !p->swap && splits == 1 && p->kt_total >= 32 &&
-                         5 * batch * ceil_div(M, 256) * ceil_div(N, 256) >= 2 * num_sms;
+                         batch * ceil_div(M, 256) * ceil_div(N, 256) >= 4 * (num_sms / 2);
   if (req_pair == 2 || auto_pair) {  // 256x256 tiles on CTA pairs: wide tiles, no split
     if (p->swap || splits != 1 || (req_bn != 0 && req_bn != 256)) return BQ_ERR_INVALID;
     if (req_kc > 2 || (req_kc == 2 && K % 128 != 0)) return BQ_ERR_INVALID;
@@ -327,7 +333,7 @@ int plan_for_call(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_
 template <int BN, int STAGES, int ACC, bool SWAP, bool P_FP4, bool Q_FP4, int MODE, int KC,
           bool FUSEQ = false>
 int launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap& ty,
-                const bq::GemmArgs& args,
+                const CUtensorMap& tr, const bq::GemmArgs& args,
                 int64_t units, int num_sms, cudaStream_t stream) {
   constexpr bool CSPLIT = MODE == bq::kSplitCluster;
   using L = bq::KernelSmem<BN, STAGES, ACC, SWAP, MODE, KC>;
@@ -379,7 +385,7 @@ int launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap&
   }
   lc.attrs = attr;
   lc.numAttrs = na;
-  if (cudaLaunchKernelEx(&lc, kern, tp, tq, ty, args) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&lc, kern, tp, tq, ty, tr, args) != cudaSuccess) {
     cudaGetLastError();
     return BQ_ERR_CUDA;
   }
@@ -388,18 +394,20 @@ int launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap&
 
 template <int BN, int STAGES, int ACC, bool SWAP, int MODE, int KC, bool FUSEQ = false>
 int launch_kind(bool w_fp4, const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap& ty,
-                const bq::GemmArgs& args, int64_t u, int num_sms, cudaStream_t st) {
+                const CUtensorMap& tr, const bq::GemmArgs& args, int64_t u, int num_sms,
+                cudaStream_t st) {
   // FP4 weights sit on the P side with SWAP, on the Q side otherwise.
   if (w_fp4)
-    return launch_gemm<BN, STAGES, ACC, SWAP, SWAP, !SWAP, MODE, KC, FUSEQ>(tp, tq, ty, args, u,
+    return launch_gemm<BN, STAGES, ACC, SWAP, SWAP, !SWAP, MODE, KC, FUSEQ>(tp, tq, ty, tr, args, u,
                                                                            num_sms, st);
-  return launch_gemm<BN, STAGES, ACC, SWAP, false, false, MODE, KC, FUSEQ>(tp, tq, ty, args, u,
+  return launch_gemm<BN, STAGES, ACC, SWAP, false, false, MODE, KC, FUSEQ>(tp, tq, ty, tr, args, u,
                                                                            num_sms, st);
 }
 
 template <int STAGES, int KC, bool Q_FP4>
 int launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
-                const CUtensorMap& tsb, const CUtensorMap& ty, const bq::GemmArgs& args,
+                const CUtensorMap& tsb, const CUtensorMap& ty, const CUtensorMap& tr,
+                const bq::GemmArgs& args,
                 int64_t units, int num_sms, cudaStream_t stream) {
   using L = bq::PairSmem<STAGES, KC>;
   auto kern = bq::gemm_pair_kernel<STAGES, KC, Q_FP4>;
@@ -432,7 +440,7 @@ int launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
   attr[1].val.clusterDim.z = 1;
   lc.attrs = attr;
   lc.numAttrs = 2;
-  if (cudaLaunchKernelEx(&lc, kern, ta, tb, tsa, tsb, ty, args) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&lc, kern, ta, tb, tsa, tsb, ty, tr, args) != cudaSuccess) {
     cudaGetLastError();
     return BQ_ERR_CUDA;
   }
@@ -442,39 +450,40 @@ int launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
 // Dispatch on (swap, bn, chunks per stage, split mode, fp4 weights) to the
 // compiled instances.  Stage counts fill ~200 KB of shared memory.
 int run_gemm(const Plan& pl, bool w_fp4, const CUtensorMap& tp, const CUtensorMap& tq,
-             const CUtensorMap& ty, const bq::GemmArgs& a, int ns, cudaStream_t st) {
+             const CUtensorMap& ty, const CUtensorMap& tr, const bq::GemmArgs& a, int ns,
+             cudaStream_t st) {
   const int64_t u = pl.units;
   constexpr int kNone = bq::kSplitNone, kWs = bq::kSplitWorkspace, kCl = bq::kSplitCluster;
   const bool b32 = pl.bn == 32;
   if (!pl.swap) {
     if (pl.bn == 256) {
-      if (pl.splits > 1) return launch_kind<256, 4, 1, false, kWs, 1>(w_fp4, tp, tq, ty, a, u, ns, st);
-      return pl.kc == 2 ? launch_kind<256, 2, 1, false, kNone, 2>(w_fp4, tp, tq, ty, a, u, ns, st)
-                        : launch_kind<256, 4, 1, false, kNone, 1>(w_fp4, tp, tq, ty, a, u, ns, st);
+      if (pl.splits > 1) return launch_kind<256, 4, 1, false, kWs, 1>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
+      return pl.kc == 2 ? launch_kind<256, 2, 1, false, kNone, 2>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
+                        : launch_kind<256, 4, 1, false, kNone, 1>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
     }
-    if (pl.splits > 1) return launch_kind<128, 6, 2, false, kWs, 1>(w_fp4, tp, tq, ty, a, u, ns, st);
-    return pl.kc == 2 ? launch_kind<128, 3, 2, false, kNone, 2>(w_fp4, tp, tq, ty, a, u, ns, st)
-                      : launch_kind<128, 6, 2, false, kNone, 1>(w_fp4, tp, tq, ty, a, u, ns, st);
+    if (pl.splits > 1) return launch_kind<128, 6, 2, false, kWs, 1>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
+    return pl.kc == 2 ? launch_kind<128, 3, 2, false, kNone, 2>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
+                      : launch_kind<128, 6, 2, false, kNone, 1>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
   }
   if (a.x) {  // fused activation quantization: unsplit 4-chunk swap tiles
-    return b32 ? launch_kind<32, 2, 1, true, kNone, 4, true>(w_fp4, tp, tq, ty, a, u, ns, st)
-               : launch_kind<64, 2, 1, true, kNone, 4, true>(w_fp4, tp, tq, ty, a, u, ns, st);
+    return b32 ? launch_kind<32, 2, 1, true, kNone, 4, true>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
+               : launch_kind<64, 2, 1, true, kNone, 4, true>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
   }
   if (pl.cluster) {
     if (pl.kc == 4)
-      return b32 ? launch_kind<32, 1, 1, true, kCl, 4>(w_fp4, tp, tq, ty, a, u, ns, st)
-                 : launch_kind<64, 1, 1, true, kCl, 4>(w_fp4, tp, tq, ty, a, u, ns, st);
-    return b32 ? launch_kind<32, 3, 1, true, kCl, 1>(w_fp4, tp, tq, ty, a, u, ns, st)
-               : launch_kind<64, 3, 1, true, kCl, 1>(w_fp4, tp, tq, ty, a, u, ns, st);
+      return b32 ? launch_kind<32, 1, 1, true, kCl, 4>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
+                 : launch_kind<64, 1, 1, true, kCl, 4>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
+    return b32 ? launch_kind<32, 3, 1, true, kCl, 1>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
+               : launch_kind<64, 3, 1, true, kCl, 1>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
   }
   if (pl.splits > 1)
-    return b32 ? launch_kind<32, 4, 1, true, kWs, 1>(w_fp4, tp, tq, ty, a, u, ns, st)
-               : launch_kind<64, 4, 1, true, kWs, 1>(w_fp4, tp, tq, ty, a, u, ns, st);
+    return b32 ? launch_kind<32, 4, 1, true, kWs, 1>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
+               : launch_kind<64, 4, 1, true, kWs, 1>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
   if (pl.kc == 4)
-    return b32 ? launch_kind<32, 2, 1, true, kNone, 4>(w_fp4, tp, tq, ty, a, u, ns, st)
-               : launch_kind<64, 2, 1, true, kNone, 4>(w_fp4, tp, tq, ty, a, u, ns, st);
-  return b32 ? launch_kind<32, 8, 1, true, kNone, 1>(w_fp4, tp, tq, ty, a, u, ns, st)
-             : launch_kind<64, 8, 1, true, kNone, 1>(w_fp4, tp, tq, ty, a, u, ns, st);
+    return b32 ? launch_kind<32, 2, 1, true, kNone, 4>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
+               : launch_kind<64, 2, 1, true, kNone, 4>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
+  return b32 ? launch_kind<32, 8, 1, true, kNone, 1>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
+             : launch_kind<64, 8, 1, true, kNone, 1>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
 }
 
 // Activations given as bf16 and quantized inside the GEMM (decode tiles).
@@ -583,7 +592,14 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
   // x 32-column boxes with the 64-byte swizzle.
   CUtensorMap map_y = map_a;  // placeholder when no bf16 output is written
   if (y) {
-    st = make_y_map(&map_y, y, M, N, count, sy);
+    st = make_y_map(&map_y, y, M, N, N, count, sy);
+    if (st != BQ_OK) return st;
+  }
+  // The residual, loaded by the same tiles into the staging buffer; a zero
+  // batch stride (one residual for every problem) makes it a 2-D map.
+  CUtensorMap map_res = map_y;  // placeholder without a residual
+  if (res) {
+    st = make_y_map(&map_res, res, M, N, ldres, count > 1 && sr != 0 ? count : 1, sr);
     if (st != BQ_OK) return st;
   }
 
@@ -647,14 +663,14 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
     const int64_t u = pl.units;
     const int ns = dev->num_sms;
     if (pl.kc == 2)
-      return w_fp4 ? launch_pair<3, 2, true>(map_a, map_b, map_sfa, map_sfb, map_y, g, u, ns, s)
-                   : launch_pair<3, 2, false>(map_a, map_b, map_sfa, map_sfb, map_y, g, u, ns, s);
-    return w_fp4 ? launch_pair<6, 1, true>(map_a, map_b, map_sfa, map_sfb, map_y, g, u, ns, s)
-                 : launch_pair<6, 1, false>(map_a, map_b, map_sfa, map_sfb, map_y, g, u, ns, s);
+      return w_fp4 ? launch_pair<3, 2, true>(map_a, map_b, map_sfa, map_sfb, map_y, map_res, g, u, ns, s)
+                   : launch_pair<3, 2, false>(map_a, map_b, map_sfa, map_sfb, map_y, map_res, g, u, ns, s);
+    return w_fp4 ? launch_pair<6, 1, true>(map_a, map_b, map_sfa, map_sfb, map_y, map_res, g, u, ns, s)
+                 : launch_pair<6, 1, false>(map_a, map_b, map_sfa, map_sfb, map_y, map_res, g, u, ns, s);
   }
   const CUtensorMap& tp = pl.swap ? map_b : map_a;
   const CUtensorMap& tq = pl.swap ? map_a : map_b;
-  return run_gemm(pl, w_fp4, tp, tq, map_y, g, dev->num_sms,
+  return run_gemm(pl, w_fp4, tp, tq, map_y, map_res, g, dev->num_sms,
                   reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -806,6 +822,24 @@ size_t bq_gemm_workspace_bytes(int weight_kind, int64_t M, int64_t N, int64_t K,
   Plan pl;
   if (make_plan(M, N, K, batch, cfg, dev->num_sms, &pl) != BQ_OK) return 0;
   return plan_ws_bytes(pl);
+}
+
+int bq_gemm_plan(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_config* cfg,
+                 int num_sms, bq_gemm_config* out) {
+  if (!out) return BQ_ERR_NULL;
+  if (M <= 0 || N <= 0 || K <= 0 || K % 32 != 0 || batch <= 0 || num_sms < 1)
+    return BQ_ERR_SHAPE;
+  Plan pl;
+  const int st = make_plan(M, N, K, batch, cfg, num_sms, &pl);
+  if (st != BQ_OK) return st;
+  out->block_n = pl.bn;
+  out->split_k = pl.splits;
+  out->swap_ab = pl.swap ? 1 : 0;
+  out->split_mode =
+      pl.splits > 1 ? (pl.cluster ? BQ_SPLIT_CLUSTER : BQ_SPLIT_WORKSPACE) : BQ_SPLIT_AUTO;
+  out->k_chunks = pl.kc;
+  out->cta_pair = pl.pair ? 2 : 1;
+  return BQ_OK;
 }
 
 int bq_gemm_mxfp8_mxfp4_epilogue(const void* a_q, const void* a_sf, const void* b_fp4,

@@ -154,7 +154,9 @@ struct GemmSmem {
   static constexpr int kOffBiasS = kOffLand + kBytesLand;  // the tile's 128 biases (fp32)
   static constexpr int kBytesBiasS = LANDING ? kBlockP * 4 : 0;
   static constexpr int kOffBar = kOffBiasS + kBytesBiasS;
-  static constexpr int kNumBars = 2 * STAGES + 2 * ACC + 1 + (CSPLIT ? 2 : 0) + (LANDING ? 1 : 0);
+  static constexpr int kNumBars =
+      2 * STAGES + 2 * ACC + 1 + (CSPLIT ? 2 : 0) + (LANDING ? 1 : 0) + (YSTAGE ? 2 : 0);
+  static constexpr int kRbarIndex = kNumBars - 2;  // residual staging barriers (YSTAGE)
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 64 + 1024;  // + alignment slack
   static constexpr int kStages = STAGES;
@@ -409,41 +411,59 @@ __device__ __forceinline__ void copy_out_swap_q(const GemmArgs &a, const UnitPos
   }
 }
 
-// 32 residual values of one row (4 x 16 bytes), zeros past N or without one.
-__device__ __forceinline__ void load_res32(const __nv_bfloat16 *rrow, int q0, int N,
-                                           uint4 (&r)[4]) {
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-    r[j] = (rrow && q0 + 8 * j < N) ? *reinterpret_cast<const uint4 *>(rrow + q0 + 8 * j)
-                                    : make_uint4(0u, 0u, 0u, 0u);
-}
-
 // Wide-tile epilogue (activation rows on the TMEM lanes): rows m0 .. m0+127
 // (this thread owns m0 + row) and columns n0 .. n0+NCOLS-1, in chunks of 32
 // columns: TMEM -> registers -> alpha, bias, GELU, residual in fp32 -> one
 // bf16 rounding -> a 128x32 bf16 staging tile in shared memory (the 64-byte
 // swizzle, so each warp store is conflict-free) -> one TMA store per chunk,
-// double-buffered.  Stores clip rows past M and columns past N.  The next
-// chunk's residual is loaded while the current one is computed.
+// double-buffered.  Stores clip rows past M and columns past N.  With a
+// residual, its chunk arrives by a TMA load into the same staging slot (two
+// chunks ahead, on the slot's barrier in `rbar`); each thread reads its row
+// there and writes its outputs over it.  `rphase` carries the two slots'
+// barrier parities (bits 0 and 1) from call to call.
 template <int NCOLS>
 __device__ __forceinline__ void epilogue_rows_tma(const GemmArgs &a, const CUtensorMap *tm_y,
-                                                  uint32_t t_row, int b, int m0, int n0, int row,
-                                                  int epi_tid, uint8_t *ystage) {
+                                                  const CUtensorMap *tm_res, uint64_t *rbar,
+                                                  uint32_t &rphase, uint32_t t_row, int b, int m0,
+                                                  int n0, int row, int epi_tid, uint8_t *ystage,
+                                                  volatile int *abort_flag) {
   const int m = m0 + row;
-  const __nv_bfloat16 *rrow =
-      (a.res && m < a.M) ? a.res + b * a.res_bstride + static_cast<int64_t>(m) * a.ldres : nullptr;
-  uint4 res[4];
-  load_res32(rrow, n0, a.N, res);
+  const bool res = a.res != nullptr;
+  const int nch = min(NCOLS / 32, (a.N - n0 + 31) / 32);
+  auto load_res = [&](int c) {  // one thread: residual chunk c into slot c & 1
+    const int slot = c & 1;
+    mbar_arrive_expect_tx(&rbar[slot], static_cast<uint32_t>(kYChunkBytes));
+    if (a.batch > 1 && a.res_bstride != 0)  // else one residual serves every problem
+      tma_load_3d(ystage + slot * kYChunkBytes, tm_res, &rbar[slot], n0 + c * 32, m0, b);
+    else
+      tma_load_2d(ystage + slot * kYChunkBytes, tm_res, &rbar[slot], n0 + c * 32, m0);
+  };
+  if (res && epi_tid == 0) {
+    bulk_wait_group_read<0>();  // earlier stores have read both slots
+    load_res(0);
+    if (nch > 1) load_res(1);
+  }
 #pragma unroll 1
-  for (int c = 0; c < NCOLS / 32; ++c) {
+  for (int c = 0; c < nch; ++c) {
     const int q0 = n0 + c * 32;
-    if (q0 >= a.N) break;  // uniform
     uint32_t v[32];
     __syncwarp();
     tmem_ld_32x32b_x32(t_row + c * 32, v);
     tmem_ld_wait();
-    uint4 res_next[4];
-    load_res32(c + 1 < NCOLS / 32 ? rrow : nullptr, q0 + 32, a.N, res_next);
+    uint8_t *buf = ystage + (c & 1) * kYChunkBytes;
+    uint4 rv[4];
+    if (res) {
+      const uint32_t bit = 1u << (c & 1);
+      if (!mbar_wait(&rbar[c & 1], (rphase & bit) ? 1u : 0u, a.err, abort_flag, kWaitEpiFull))
+        return;
+      rphase ^= bit;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        rv[j] = *reinterpret_cast<const uint4 *>(buf + row * 64 + ((j ^ ((row >> 1) & 3)) << 4));
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) rv[j] = make_uint4(0u, 0u, 0u, 0u);
+    }
     uint32_t o[16];
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
@@ -467,7 +487,7 @@ __device__ __forceinline__ void epilogue_rows_tma(const GemmArgs &a, const CUten
 #pragma unroll
         for (int j = 0; j < 8; ++j) t[j] = gelu_erf(t[j]);
       }
-      const uint32_t rw[4] = {res[g].x, res[g].y, res[g].z, res[g].w};
+      const uint32_t rw[4] = {rv[g].x, rv[g].y, rv[g].z, rv[g].w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const __nv_bfloat162 p2 =
@@ -478,9 +498,10 @@ __device__ __forceinline__ void epilogue_rows_tma(const GemmArgs &a, const CUten
     }
     if (a.q_out) quant_out_row32(a, b, m, q0, o);
     if (a.y) {  // uniform
-      uint8_t *buf = ystage + (c & 1) * kYChunkBytes;
-      if (epi_tid == 0) bulk_wait_group_read<1>();  // the store two chunks back has read buf
-      epi_bar_sync();
+      if (!res) {
+        if (epi_tid == 0) bulk_wait_group_read<1>();  // the store two chunks back has read buf
+        epi_bar_sync();
+      }
 #pragma unroll
       for (int j = 0; j < 4; ++j)
         *reinterpret_cast<uint4 *>(buf + row * 64 + ((j ^ ((row >> 1) & 3)) << 4)) =
@@ -494,9 +515,13 @@ __device__ __forceinline__ void epilogue_rows_tma(const GemmArgs &a, const CUten
           tma_store_2d(tm_y, buf, q0, m0);
         bulk_commit_group();
       }
+    } else if (res) {
+      epi_bar_sync();  // every thread has read its residual from the slot
     }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) res[j] = res_next[j];
+    if (res && epi_tid == 0 && c + 2 < nch) {
+      bulk_wait_group_read<0>();  // this chunk's store has read the slot
+      load_res(c + 2);
+    }
   }
 }
 
@@ -774,7 +799,8 @@ template <int BN, int STAGES, int ACC, bool SWAP, bool P_FP4, bool Q_FP4, int MO
           bool FUSEQ = false>
 __global__ void __launch_bounds__(kNumThreads, 1)
     gemm_bs_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
-                   const __grid_constant__ CUtensorMap tm_y, const GemmArgs a) {
+                   const __grid_constant__ CUtensorMap tm_y,
+                   const __grid_constant__ CUtensorMap tm_res, const GemmArgs a) {
   constexpr bool CSPLIT = MODE == kSplitCluster;
   static_assert(!CSPLIT || SWAP, "cluster split-K is built for the swap-AB (decode) tiles");
   static_assert(!CSPLIT || ACC == 1, "cluster split-K uses one accumulator");
@@ -837,6 +863,10 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       mbar_init(peer_free, a.splits);
     }
     if constexpr (L::kBytesLand > 0) mbar_init(land_bar, 1);
+    if constexpr (L::kBytesYStage > 0) {
+      mbar_init(full + L::kRbarIndex, 1);
+      mbar_init(full + L::kRbarIndex + 1, 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_p);
@@ -984,6 +1014,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     griddep_wait();
     int qstage = 0;
     uint32_t qphase = 0;
+    uint32_t rphase = 0;  // residual staging barrier parities
     if constexpr (FUSEQ) {
       if (epi_tid == 0) griddep_launch_dependents();
     }
@@ -1093,8 +1124,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           copy_out_swap<BN>(a, u, epi_tid, stage);
         if (unit + static_cast<int>(gridDim.x) < total_units) epi_bar_sync();  // staging free
       } else if constexpr (MODE == kSplitNone) {
-        epilogue_rows_tma<BN>(a, &tm_y, t_row, u.b, u.tp * kBlockP, u.tq * BN, row, epi_tid,
-                              smem + L::kOffYStage);
+        epilogue_rows_tma<BN>(a, &tm_y, &tm_res, full + L::kRbarIndex, rphase, t_row, u.b,
+                              u.tp * kBlockP, u.tq * BN, row, epi_tid, smem + L::kOffYStage,
+                              abort_flag);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[acc]);

@@ -44,7 +44,9 @@ struct PairSmem {
   static constexpr int kOffSfa = kOffYStage + 2 * kYChunkBytes;
   static constexpr int kOffSfb = kOffSfa + STAGES * kSfaBytes;
   static constexpr int kOffBar = kOffSfb + STAGES * kSfbBytes;
-  static constexpr int kNumBars = 2 * STAGES + 3;          // full, empty, tfull, tempty, drain
+  // full, empty, tfull, tempty, drain, two residual staging barriers
+  static constexpr int kNumBars = 2 * STAGES + 5;
+  static constexpr int kRbarIndex = 2 * STAGES + 3;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 64 + 1024;      // + alignment slack
   static constexpr int kTmemUsed = kPairN + STAGES * kSfCols;
@@ -131,7 +133,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                      const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_sfa,
                      const __grid_constant__ CUtensorMap tm_sfb,
-                     const __grid_constant__ CUtensorMap tm_y, const GemmArgs a) {
+                     const __grid_constant__ CUtensorMap tm_y,
+                     const __grid_constant__ CUtensorMap tm_res, const GemmArgs a) {
   using L = PairSmem<STAGES, KC>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -164,6 +167,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     mbar_init(tfull, 1);
     mbar_init(tempty, 8);  // every epilogue warp of both CTAs
     mbar_init(drain, 1);
+    mbar_init(full + L::kRbarIndex, 1);
+    mbar_init(full + L::kRbarIndex + 1, 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_a);
@@ -274,6 +279,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     const int row = quad * 32 + lane;
     const int epi_tid = threadIdx.x - 64;
     uint32_t acc_phase = 0;
+    uint32_t rphase = 0;  // residual staging barrier parities
     griddep_wait();  // the bias and residual may come from the preceding kernel
     for (int unit = pair; unit < total_units; unit += num_pairs) {
       const UnitPos u = unit_pos(a, unit);
@@ -282,8 +288,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       acc_phase ^= 1;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
-      epilogue_rows_tma<kPairN>(a, &tm_y, t_row, u.b, (2 * u.tp + static_cast<int>(rank)) * kBlockP,
-                                u.tq * kPairN, row, epi_tid, smem + L::kOffYStage);
+      epilogue_rows_tma<kPairN>(a, &tm_y, &tm_res, full + L::kRbarIndex, rphase, t_row, u.b,
+                                (2 * u.tp + static_cast<int>(rank)) * kBlockP, u.tq * kPairN,
+                                row, epi_tid, smem + L::kOffYStage, abort_flag);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_lead);

@@ -5,9 +5,11 @@ CUDA-graph replay over rotating weight copies (more bytes than L2 holds, so
 weights stream from HBM) and prints one JSON line per candidate:
 
     python -m block_scaled_precision_quant_b200.sweep M N K [kind] [--batch B] [--gelu]
+        [--residual]
 
 kind: mxfp4 (default), fp8blk32, mxfp8.  --batch B runs B independent problems
-over one broadcast weight (batch stride 0), --gelu adds bias + GELU.  The
+over one broadcast weight (batch stride 0), --gelu adds bias + GELU,
+--residual adds a bf16 residual.  The
 built-in dispatch of bq_api.cu is derived from these measurements.
 """
 from __future__ import annotations
@@ -57,6 +59,7 @@ def main(argv=None):
     ap.add_argument("--reps", type=int, default=20)
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--gelu", action="store_true")
+    ap.add_argument("--residual", action="store_true")
     args = ap.parse_args(argv)
     import torch
     import block_scaled_precision_quant_b200 as bq
@@ -76,7 +79,8 @@ def main(argv=None):
         aq = torch.stack(aqs).reshape(B * M, K)
         asf = torch.stack(asfs)
         batch = None if B == 1 else dict(count=B, stride_a=M * K, stride_a_sf=asf.shape[1],
-                                         stride_b=0, stride_b_sf=0, stride_y=M * N * 2)
+                                         stride_b=0, stride_b_sf=0, stride_y=M * N * 2,
+                                         stride_res=M * N * 2 if args.residual else 0)
         l2 = torch.cuda.get_device_properties(dev).L2_cache_size
         wbytes = N * K // 2 if wk == bq.W_MXFP4 else N * K
         copies = max(1, min(64, int(np.ceil(2.5 * l2 / max(wbytes, 1)))))
@@ -97,6 +101,10 @@ def main(argv=None):
         bias = torch.from_numpy(synth.bias(N, seed=3).view(np.int16)).view(torch.bfloat16).to(dev)
         y = torch.empty((B, M, N) if B > 1 else (M, N), dtype=torch.bfloat16, device=dev)
         act = bq.BQ_ACT_GELU if args.gelu else bq.BQ_ACT_NONE
+        res = None
+        if args.residual:
+            res = torch.from_numpy(synth.residual(B * M, N, seed=4).view(np.int16)) \
+                .view(torch.bfloat16).to(dev).reshape(y.shape)
         for cfg in candidates(M, N, K):
             need = bq.workspace_bytes(wk, M, N, K, B, cfg)
             work = torch.zeros((max(need, 16),), dtype=torch.uint8, device=dev) if need else None
@@ -105,7 +113,7 @@ def main(argv=None):
             try:
                 def run(c):
                     bq.gemm(wk, aq, asf, ws[c][0], ws[c][1], M, N, K, y=y, bias=bias,
-                            act=act, batch=batch, config=cfg, workspace=work)
+                            act=act, residual=res, batch=batch, config=cfg, workspace=work)
                 for c in range(copies):
                     run(c)
                 torch.cuda.synchronize()
@@ -126,6 +134,7 @@ def main(argv=None):
                 us = e0.elapsed_time(e1) * 1e3 / (args.reps * copies)
                 gbytes = (wbytes + N * K / 32 + B * (M * K * 33 / 32 + 2 * M * N)) / (us * 1e-6) / 1e9
                 print(json.dumps(dict(shape=[M, N, K], batch=B, gelu=args.gelu, kind=args.kind,
+                                      residual=args.residual,
                                       cfg=desc, us=round(us, 3),
                                       tflops=round(2 * B * M * N * K / us / 1e6, 1),
                                       gbs=round(gbytes, 1))), flush=True)

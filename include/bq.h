@@ -232,6 +232,17 @@ typedef struct {
 size_t bq_gemm_workspace_bytes(int weight_kind, int64_t M, int64_t N, int64_t K, int64_t batch,
                                const bq_gemm_config *cfg);
 
+/* The schedule the built-in dispatch picks for a problem on a device with
+ * `num_sms` SMs, with `cfg` (NULL = all auto) as a *_epilogue call would get
+ * it: every field of *out resolved (block_n, split_k >= 1, swap_ab 0/1,
+ * split_mode BQ_SPLIT_WORKSPACE or BQ_SPLIT_CLUSTER when split_k > 1, else
+ * BQ_SPLIT_AUTO, k_chunks >= 1, cta_pair 1 or 2).  Host-only: touches no
+ * device.  Calls that ask for a quantized output run unsplit.  Returns
+ * BQ_ERR_NULL (out NULL), BQ_ERR_SHAPE (sizes out of range, num_sms < 1) or
+ * BQ_ERR_INVALID (cfg not schedulable, the status the GEMM call returns). */
+int bq_gemm_plan(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_config *cfg,
+                 int num_sms, bq_gemm_config *out);
+
 /* GEMM + fused epilogue (+ optional batch).  epi NULL = plain (alpha 1, no
  * bias, residual or activation).  batch NULL = one problem.  workspace: device
  * memory of at least bq_gemm_workspace_bytes(...) bytes (may be NULL when that

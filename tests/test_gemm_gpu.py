@@ -284,6 +284,46 @@ def test_pair_tiles_batched_broadcast():
         assert_close(yb[i], ref, tol, f"pair batch {i}")
 
 
+@pytest.mark.parametrize("cfg", [dict(split_k=1, swap_ab=0, block_n=256),
+                                 dict(split_k=1, swap_ab=0, block_n=128, k_chunks=2), PAIR])
+@pytest.mark.parametrize("layout", ["strided", "per_problem", "broadcast"])
+def test_residual_layouts(cfg, layout):
+    """The wide tiles load the residual tile by tile into the output staging
+    buffer: a row pitch wider than N, one residual per problem, and one
+    residual broadcast to every problem (batch stride 0)."""
+    count = 1 if layout == "strided" else 2
+    M, N, K, ld = 300, 296, 384, 296 + 40
+    xs = [synth.activations(M, K, seed=110 + i) for i in range(count)]
+    b, bsf = synth.mxfp4_weight(N, K, seed=115)
+    nres = 1 if layout == "broadcast" else count
+    res = [synth.residual(M, N, seed=120 + i) for i in range(nres)]
+    wide = np.zeros((nres, M, ld), np.uint16)
+    for i in range(nres):
+        wide[i, :, :N] = res[i]
+        wide[i, :, N:] = 0x7FC0  # NaN outside the view: must never be read
+    res_d = to_dev_bf16(wide)[:, :, :N]
+    aqs, sfs = zip(*[bq.act_quant(to_dev_bf16(x)) for x in xs])
+    aq = torch.stack(aqs).reshape(count * M, K)
+    asf = torch.stack(sfs)
+    bsf_d = bq.pack_weight_scales(to_dev_u8(bsf), bq.BQ_SF_ROW32, N, K)
+    batch = None
+    if count > 1:
+        batch = dict(count=count, stride_a=M * K, stride_a_sf=asf.shape[1], stride_b=0,
+                     stride_b_sf=0, stride_y=M * N * 2,
+                     stride_res=0 if layout == "broadcast" else M * ld * 2)
+    y = bq.gemm(bq.W_MXFP4, aq, asf if count > 1 else asf[0], to_dev_u8(b), bsf_d, M, N, K,
+                residual=res_d if count > 1 else res_d[0], batch=batch,
+                config=bq.config(**cfg))
+    bq.device_status()
+    yb = bf16_to_f64(y.cpu().view(torch.int16).numpy().view(np.uint16)).reshape(count, M, N)
+    for i, x in enumerate(xs):
+        q, s = oracle.act_quant(x)
+        r = res[0 if layout == "broadcast" else i]
+        ref, sabs = oracle.gemm(q, s, b, bsf, oracle.B_FP4, M, N, K, residual=r)
+        tol = oracle.gemm_tolerance(ref, sabs, 1.0, None, np.abs(bf16_to_f64(r)), 0)
+        assert_close(yb[i], ref, tol, f"{layout} {cfg} problem {i}")
+
+
 def test_pair_tiles_refusals():
     c = Case(bq.W_MXFP4, 300, 520, 640)
     for cfg in (bq.config(split_k=2, swap_ab=0, cta_pair=2),
