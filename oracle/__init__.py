@@ -27,6 +27,7 @@ _lib = None
 
 OK, ERR_NAN_SCALE, ERR_NAN_CODE, ERR_SHAPE, ERR_NONFINITE = 0, -1, -2, -3, -4
 B_FP4, B_FP8BLK, B_FP8ROW = 0, 1, 2
+A_E4M3, A_FP4 = 0, 1
 ACT_NONE, ACT_GELU = 0, 1
 
 CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
@@ -81,13 +82,23 @@ def _load():
     lib.oracle_act_quant_f32.restype = ctypes.c_int
     lib.oracle_act_qdq.argtypes = [u8p, u8p, i64, i64, u16p]
     lib.oracle_act_qdq.restype = ctypes.c_int
-    lib.oracle_gemm.argtypes = [u8p, u8p, u8p, u8p, ctypes.c_int, i64, i64, i64, u16p, u16p,
-                                i64, ctypes.c_double, ctypes.c_int, f64p, f64p, ctypes.c_int]
-    lib.oracle_gemm.restype = ctypes.c_int
-    lib.oracle_gemm_sampled.argtypes = [u8p, u8p, u8p, u8p, ctypes.c_int, i64, i64, i64, u16p,
-                                        u16p, i64, ctypes.c_double, ctypes.c_int, i64p, i64p,
-                                        i64, f64p, f64p, ctypes.c_int]
-    lib.oracle_gemm_sampled.restype = ctypes.c_int
+    lib.oracle_encode_fp4.argtypes = [ctypes.c_float]
+    lib.oracle_encode_fp4.restype = ctypes.c_uint8
+    lib.oracle_encode_fp4_n.argtypes = [f32p, i64, u8p]
+    lib.oracle_encode_fp4_n.restype = None
+    lib.oracle_act_quant_fp4.argtypes = [u16p, i64, i64, i64, u8p, u8p]
+    lib.oracle_act_quant_fp4.restype = ctypes.c_int
+    lib.oracle_act_quant_fp4_f32.argtypes = [f32p, i64, i64, u8p, u8p]
+    lib.oracle_act_quant_fp4_f32.restype = ctypes.c_int
+    lib.oracle_gemm_ex.argtypes = [u8p, u8p, ctypes.c_int, u8p, u8p, ctypes.c_int, i64, i64, i64,
+                                   u16p, u16p, i64, ctypes.c_double, ctypes.c_int, f64p, f64p,
+                                   ctypes.c_int]
+    lib.oracle_gemm_ex.restype = ctypes.c_int
+    lib.oracle_gemm_sampled_ex.argtypes = [u8p, u8p, ctypes.c_int, u8p, u8p, ctypes.c_int, i64,
+                                           i64, i64, u16p, u16p, i64, ctypes.c_double,
+                                           ctypes.c_int, i64p, i64p, i64, f64p, f64p,
+                                           ctypes.c_int]
+    lib.oracle_gemm_sampled_ex.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -147,6 +158,21 @@ def encode_e4m3_array(v: np.ndarray) -> np.ndarray:
     return out
 
 
+def encode_fp4(v: float) -> int:
+    """binary32 -> E2M1 code (0..15), round to nearest even, saturating at
+    +-6, sign kept (the conversion the MXFP4 activation quantizer applies
+    after its clamp)."""
+    return int(_load().oracle_encode_fp4(float(v)))
+
+
+def encode_fp4_array(v: np.ndarray) -> np.ndarray:
+    """encode_fp4 applied element-wise; one code per uint8, v's shape."""
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.empty(v.shape, dtype=np.uint8)
+    _load().oracle_encode_fp4_n(_ptr(v, ctypes.c_float), v.size, _ptr(out, ctypes.c_uint8))
+    return out
+
+
 def f32_to_bf16_bits(v: float) -> int:
     return int(_load().oracle_f32_to_bf16(float(v)))
 
@@ -183,6 +209,49 @@ def act_quant_f32(x: np.ndarray):
     return q, sf
 
 
+def act_quant_fp4(x_bf16_bits: np.ndarray):
+    """Per-32 MXFP4 activation quantization: the act_quant steps with the
+    E2M1 maximum 6 in place of 448 (the pages define the per-32 rule for
+    E4M3 activations and the E2M1 format with E8M0 scales for weights; the
+    FP4 x FP4 GEMMs of the "fp4-gemm" page need FP4 activations).
+
+    Returns (q uint8 [..., K/2] packed E2M1, low nibble = even element,
+    sf uint8 [..., K/32] E8M0 bytes)."""
+    x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
+    K = x.shape[-1]
+    M = x.size // K if K else 0
+    q = np.empty(x.shape[:-1] + (K // 2,), dtype=np.uint8)
+    sf = np.empty(x.shape[:-1] + (K // 32,), dtype=np.uint8)
+    if M:
+        _check(_load().oracle_act_quant_fp4(_ptr(x, ctypes.c_uint16), M, K, K,
+                                            _ptr(q, ctypes.c_uint8), _ptr(sf, ctypes.c_uint8)),
+               "act_quant_fp4")
+    return q, sf
+
+
+def act_quant_fp4_f32(x: np.ndarray):
+    """The MXFP4 steps on binary32 input [M, K]."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    K = x.shape[-1]
+    M = x.size // K
+    q = np.empty(x.shape[:-1] + (K // 2,), dtype=np.uint8)
+    sf = np.empty(x.shape[:-1] + (K // 32,), dtype=np.uint8)
+    _check(_load().oracle_act_quant_fp4_f32(_ptr(x, ctypes.c_float), M, K,
+                                            _ptr(q, ctypes.c_uint8), _ptr(sf, ctypes.c_uint8)),
+           "act_quant_fp4_f32")
+    return q, sf
+
+
+def unpack_fp4(q: np.ndarray) -> np.ndarray:
+    """Packed E2M1 bytes [..., K/2] -> one code per byte [..., K] (low nibble
+    first)."""
+    q = np.asarray(q, dtype=np.uint8)
+    out = np.empty(q.shape[:-1] + (2 * q.shape[-1],), dtype=np.uint8)
+    out[..., 0::2] = q & 0x0F
+    out[..., 1::2] = q >> 4
+    return out
+
+
 def act_qdq(q: np.ndarray, sf: np.ndarray) -> np.ndarray:
     """bf16 bits of fp32(q) * s (formats.py page: act_qdq)."""
     q = np.ascontiguousarray(q, dtype=np.uint8)
@@ -198,12 +267,13 @@ def act_qdq(q: np.ndarray, sf: np.ndarray) -> np.ndarray:
 # ----------------------------------------------------------------- GEMM ----
 
 def gemm(aq, asf, b, bsf, bkind, M, N, K, bias=None, residual=None, alpha=1.0,
-         act=ACT_NONE, nthreads=None):
+         act=ACT_NONE, nthreads=None, a_kind=A_E4M3):
     """Exact-decode fp64 GEMM with the fused epilogue.
 
     ref[m, n] = act(alpha * sum_k a[m,k] b[n,k] + bias[n]) + residual[m, n] and
     sumabs[m, n] = sum_k |a[m,k] b[n,k]|, where a and b are the exactly decoded
-    operands (formats.py page: decode_fp4, decode_fp8_block, e8m0_to_f32)."""
+    operands (formats.py page: decode_fp4, decode_fp8_block, e8m0_to_f32).
+    a_kind: A_E4M3 (aq [M, K]) or A_FP4 (aq [M, K/2] packed E2M1)."""
     aq = np.ascontiguousarray(aq, dtype=np.uint8)
     asf = np.ascontiguousarray(asf, dtype=np.uint8)
     b = np.ascontiguousarray(b, dtype=np.uint8)
@@ -213,9 +283,10 @@ def gemm(aq, asf, b, bsf, bkind, M, N, K, bias=None, residual=None, alpha=1.0,
     ref = np.empty((M, N), dtype=np.float64)
     sumabs = np.empty((M, N), dtype=np.float64)
     if M and N:
-        _check(_load().oracle_gemm(
-            _ptr(aq, ctypes.c_uint8), _ptr(asf, ctypes.c_uint8), _ptr(b, ctypes.c_uint8),
-            _ptr(bsf, ctypes.c_uint8), int(bkind), M, N, K, _ptr(bias, ctypes.c_uint16),
+        _check(_load().oracle_gemm_ex(
+            _ptr(aq, ctypes.c_uint8), _ptr(asf, ctypes.c_uint8), int(a_kind),
+            _ptr(b, ctypes.c_uint8), _ptr(bsf, ctypes.c_uint8), int(bkind), M, N, K,
+            _ptr(bias, ctypes.c_uint16),
             _ptr(residual, ctypes.c_uint16), N, float(alpha), int(act),
             _ptr(ref, ctypes.c_double), _ptr(sumabs, ctypes.c_double),
             int(nthreads or default_threads())), "gemm")
@@ -223,7 +294,7 @@ def gemm(aq, asf, b, bsf, bkind, M, N, K, bias=None, residual=None, alpha=1.0,
 
 
 def gemm_sampled(aq, asf, b, bsf, bkind, M, N, K, ms, ns, bias=None, residual=None,
-                 alpha=1.0, act=ACT_NONE, nthreads=None):
+                 alpha=1.0, act=ACT_NONE, nthreads=None, a_kind=A_E4M3):
     """The same per-element definition at the (ms[i], ns[i]) pairs only."""
     aq = np.ascontiguousarray(aq, dtype=np.uint8)
     asf = np.ascontiguousarray(asf, dtype=np.uint8)
@@ -236,9 +307,10 @@ def gemm_sampled(aq, asf, b, bsf, bkind, M, N, K, ms, ns, bias=None, residual=No
     ref = np.empty(ms.size, dtype=np.float64)
     sumabs = np.empty(ms.size, dtype=np.float64)
     if ms.size:
-        _check(_load().oracle_gemm_sampled(
-            _ptr(aq, ctypes.c_uint8), _ptr(asf, ctypes.c_uint8), _ptr(b, ctypes.c_uint8),
-            _ptr(bsf, ctypes.c_uint8), int(bkind), M, N, K, _ptr(bias, ctypes.c_uint16),
+        _check(_load().oracle_gemm_sampled_ex(
+            _ptr(aq, ctypes.c_uint8), _ptr(asf, ctypes.c_uint8), int(a_kind),
+            _ptr(b, ctypes.c_uint8), _ptr(bsf, ctypes.c_uint8), int(bkind), M, N, K,
+            _ptr(bias, ctypes.c_uint16),
             _ptr(residual, ctypes.c_uint16), N, float(alpha), int(act),
             _ptr(ms, ctypes.c_int64), _ptr(ns, ctypes.c_int64), ms.size,
             _ptr(ref, ctypes.c_double), _ptr(sumabs, ctypes.c_double),

@@ -15,7 +15,12 @@
  *     functions act_scale / act_quant / act_qdq / _log2_ceil_pow2;
  *   - the number formats follow the same page's module docstring
  *     ("Formats" paragraph) and its constants FP4_TABLE, FP8_MAX, BLOCK,
- *     E8M0_NAN, E4M3_NAN.
+ *     E8M0_NAN, E4M3_NAN;
+ *   - the MXFP4 activation quantizer (for FP4 x FP4 products, the A4W4 GEMMs
+ *     of the "fp4-gemm" page, README "Available Functions") is not spelled
+ *     out on the pages: it is the same per-32 rule with the E2M1 format's
+ *     largest value 6 in place of 448, and E2M1 codes packed two per byte with
+ *     the even element in the low nibble (the pages' MXFP4 weight layout).
  *
  * Floating point: compile with -ffp-contract=off and without fast-math so that
  * every float expression below is one IEEE binary32 operation, as the page's
@@ -111,6 +116,35 @@ uint8_t oracle_encode_e4m3(float v) {
 /* Element-wise oracle_encode_e4m3 over n values. */
 void oracle_encode_e4m3_n(const float *v, int64_t n, uint8_t *out) {
   for (int64_t i = 0; i < n; ++i) out[i] = oracle_encode_e4m3(v[i]);
+}
+
+/* Round a binary32 value to E2M1 (FP4) with round-to-nearest, ties to even,
+ * saturating at +-6, the sign kept (negative values that round to zero give
+ * code 8, -0).  The same method as the E4M3 encoder: the 8 non-negative
+ * magnitudes of codes 0..7 increase with the code (decoded by
+ * oracle_decode_fp4); take the nearer neighbour, on a tie the even code. */
+uint8_t oracle_encode_fp4(float v) {
+  double mag[8];
+  for (int c = 0; c < 8; ++c) mag[c] = oracle_decode_fp4((uint8_t)c);
+  uint8_t sign = signbit(v) ? 0x8 : 0x0;
+  double a = fabs((double)v);
+  uint8_t code;
+  if (a >= mag[7]) {
+    code = 7; /* 6 */
+  } else {
+    int lo = 0;
+    while (mag[lo + 1] <= a) ++lo; /* mag[lo] <= a < mag[lo + 1] */
+    int hi = lo + 1;
+    double dlo = a - mag[lo], dhi = mag[hi] - a;
+    if (dlo < dhi) code = (uint8_t)lo;
+    else if (dhi < dlo) code = (uint8_t)hi;
+    else code = (uint8_t)((lo % 2 == 0) ? lo : hi);
+  }
+  return (uint8_t)(sign | code);
+}
+
+void oracle_encode_fp4_n(const float *v, int64_t n, uint8_t *out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = oracle_encode_fp4(v[i]);
 }
 
 static float bf16_to_f32(uint16_t h) {
@@ -217,6 +251,78 @@ int oracle_act_qdq(const uint8_t *q, const uint8_t *sf, int64_t M, int64_t K, ui
   return ORACLE_OK;
 }
 
+/* MXFP4 activation quantization: the steps of act_quant_group with the
+ * E2M1 maximum 6 in place of 448:
+ *   amax = max(max_i |x_i|, 1e-4)                       (fp32)
+ *   t    = fp32(amax * fp32(1/6))
+ *   e    = ceil(log2 t) from t's exponent bits;  scale byte = e + 127
+ *   q_i  = E2M1_RNE(clamp(x_i / 2^e, -6, 6))
+ * codes[i] gets one code per byte.  Returns the scale byte, or -1 for a NaN
+ * or Inf in the group. */
+static int act_quant_fp4_group(const float *x, uint8_t *codes) {
+  float amax = 0.0f;
+  for (int i = 0; i < BLOCK; ++i) {
+    if (!isfinite(x[i])) return -1;
+    float ax = fabsf(x[i]);
+    if (ax > amax) amax = ax;
+  }
+  const float floor_ = 1e-4f;
+  if (amax < floor_) amax = floor_;
+  const float inv6 = (float)(1.0 / 6.0);
+  float t = amax * inv6;
+  uint32_t bits;
+  memcpy(&bits, &t, 4);
+  int e = (int)((bits >> 23) & 0xFF) - 127 + ((bits & 0x7FFFFF) != 0 ? 1 : 0);
+  float s = ldexpf(1.0f, e);
+  for (int i = 0; i < BLOCK; ++i) {
+    float y = x[i] / s;
+    if (y > 6.0f) y = 6.0f;
+    if (y < -6.0f) y = -6.0f;
+    codes[i] = oracle_encode_fp4(y);
+  }
+  return e + 127;
+}
+
+/* Packs 32 one-per-byte codes into 16 bytes, element 2j in the low nibble of
+ * byte j. */
+static void pack_fp4(const uint8_t *codes, uint8_t *out) {
+  for (int j = 0; j < BLOCK / 2; ++j) out[j] = (uint8_t)(codes[2 * j] | (codes[2 * j + 1] << 4));
+}
+
+/* x: bf16 bit patterns [M, ldx]; q: [M, K/2] packed E2M1 codes; sf: [M, K/32]
+ * E8M0 bytes.  Returns ORACLE_OK, ORACLE_ERR_SHAPE or ORACLE_ERR_NONFINITE. */
+int oracle_act_quant_fp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                         uint8_t *q, uint8_t *sf) {
+  if (K <= 0 || K % BLOCK) return ORACLE_ERR_SHAPE;
+  const int64_t G = K / BLOCK;
+  float buf[BLOCK];
+  uint8_t codes[BLOCK];
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t g = 0; g < G; ++g) {
+      for (int i = 0; i < BLOCK; ++i) buf[i] = bf16_to_f32(x[m * ldx + g * BLOCK + i]);
+      int b = act_quant_fp4_group(buf, codes);
+      if (b < 0) return ORACLE_ERR_NONFINITE;
+      pack_fp4(codes, q + m * (K / 2) + g * (BLOCK / 2));
+      sf[m * G + g] = (uint8_t)b;
+    }
+  return ORACLE_OK;
+}
+
+/* The same steps on binary32 input [M, K]. */
+int oracle_act_quant_fp4_f32(const float *x, int64_t M, int64_t K, uint8_t *q, uint8_t *sf) {
+  if (K <= 0 || K % BLOCK) return ORACLE_ERR_SHAPE;
+  const int64_t G = K / BLOCK;
+  uint8_t codes[BLOCK];
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t g = 0; g < G; ++g) {
+      int b = act_quant_fp4_group(x + m * K + g * BLOCK, codes);
+      if (b < 0) return ORACLE_ERR_NONFINITE;
+      pack_fp4(codes, q + m * (K / 2) + g * (BLOCK / 2));
+      sf[m * G + g] = (uint8_t)b;
+    }
+  return ORACLE_OK;
+}
+
 /* ------------------------------------------------------------------ */
 /* Exact operand decode + fp64 GEMM with the fused epilogue.            */
 /* ------------------------------------------------------------------ */
@@ -226,12 +332,17 @@ int oracle_act_qdq(const uint8_t *q, const uint8_t *sf, int64_t M, int64_t K, ui
 #define ORACLE_B_FP8BLK 1  /* E4M3 [N, K]; scales [ceil(N/32), ceil(K/32)], one per 32x32 block */
 #define ORACLE_B_FP8ROW 2  /* E4M3 [N, K]; scales [N, K/32] (MXFP8 along K) */
 
+/* Activation kinds. */
+#define ORACLE_A_E4M3 0 /* E4M3 [M, K]; scales [M, K/32] */
+#define ORACLE_A_FP4 1  /* E2M1 packed [M, K/2], low nibble = even k; scales [M, K/32] */
+
 #define ORACLE_ACT_NONE 0
 #define ORACLE_ACT_GELU 1
 
 typedef struct {
   const uint8_t *aq, *asf;
   const uint8_t *b, *bsf;
+  int akind;
   int bkind;
   int64_t M, N, K;
   const uint16_t *bias, *residual;
@@ -247,10 +358,16 @@ typedef struct {
   int status;
 } gemm_job;
 
-/* Decoded A value a[m][k] = e4m3(code) * 2^(b - 127) (exact in double). */
+/* Decoded A value a[m][k] = code * 2^(b - 127) (exact in double), the code
+ * E4M3 or packed E2M1. */
 static int dec_a(const gemm_job *J, int64_t m, int64_t k, double *v) {
   double c, s;
-  if (oracle_decode_e4m3(J->aq[m * J->K + k], &c)) return ORACLE_ERR_NAN_CODE;
+  if (J->akind == ORACLE_A_FP4) {
+    uint8_t byte = J->aq[m * (J->K / 2) + k / 2];
+    c = oracle_decode_fp4((k % 2 == 0) ? (byte & 0x0F) : (byte >> 4));
+  } else if (oracle_decode_e4m3(J->aq[m * J->K + k], &c)) {
+    return ORACLE_ERR_NAN_CODE;
+  }
   if (oracle_decode_e8m0(J->asf[m * (J->K / BLOCK) + k / BLOCK], &s)) return ORACLE_ERR_NAN_SCALE;
   *v = c * s;
   return ORACLE_OK;
@@ -353,25 +470,43 @@ static int run_jobs(gemm_job *proto, int64_t total, int nthreads) {
  * A: aq [M, K] E4M3 codes, asf [M, K/32] E8M0 (row-major).
  * B: see ORACLE_B_*.  bias: [N] bf16 or NULL.  residual: [M, ld_res] bf16 or
  * NULL.  Rows are spread over nthreads POSIX threads. */
-int oracle_gemm(const uint8_t *aq, const uint8_t *asf, const uint8_t *b, const uint8_t *bsf,
-                int bkind, int64_t M, int64_t N, int64_t K, const uint16_t *bias,
-                const uint16_t *residual, int64_t ld_res, double alpha, int act,
-                double *ref, double *sumabs, int nthreads) {
-  if (K <= 0 || K % BLOCK || bkind < 0 || bkind > 2) return ORACLE_ERR_SHAPE;
-  gemm_job J = {aq, asf, b, bsf, bkind, M, N, K, bias, residual, ld_res, alpha, act,
+int oracle_gemm_ex(const uint8_t *aq, const uint8_t *asf, int akind, const uint8_t *b,
+                   const uint8_t *bsf, int bkind, int64_t M, int64_t N, int64_t K,
+                   const uint16_t *bias, const uint16_t *residual, int64_t ld_res, double alpha,
+                   int act, double *ref, double *sumabs, int nthreads) {
+  if (K <= 0 || K % BLOCK || bkind < 0 || bkind > 2 || akind < 0 || akind > 1)
+    return ORACLE_ERR_SHAPE;
+  gemm_job J = {aq, asf, b, bsf, akind, bkind, M, N, K, bias, residual, ld_res, alpha, act,
                 ref, sumabs, NULL, NULL, 0, 0, 0, 0};
   return run_jobs(&J, M, nthreads);
 }
 
+int oracle_gemm(const uint8_t *aq, const uint8_t *asf, const uint8_t *b, const uint8_t *bsf,
+                int bkind, int64_t M, int64_t N, int64_t K, const uint16_t *bias,
+                const uint16_t *residual, int64_t ld_res, double alpha, int act,
+                double *ref, double *sumabs, int nthreads) {
+  return oracle_gemm_ex(aq, asf, ORACLE_A_E4M3, b, bsf, bkind, M, N, K, bias, residual, ld_res,
+                        alpha, act, ref, sumabs, nthreads);
+}
+
 /* Sampled GEMM: the same per-element definition at count (m, n) pairs. */
+int oracle_gemm_sampled_ex(const uint8_t *aq, const uint8_t *asf, int akind, const uint8_t *b,
+                           const uint8_t *bsf, int bkind, int64_t M, int64_t N, int64_t K,
+                           const uint16_t *bias, const uint16_t *residual, int64_t ld_res,
+                           double alpha, int act, const int64_t *ms, const int64_t *ns,
+                           int64_t count, double *ref, double *sumabs, int nthreads) {
+  if (K <= 0 || K % BLOCK || bkind < 0 || bkind > 2 || akind < 0 || akind > 1)
+    return ORACLE_ERR_SHAPE;
+  gemm_job J = {aq, asf, b, bsf, akind, bkind, M, N, K, bias, residual, ld_res, alpha, act,
+                ref, sumabs, ms, ns, count, 0, 0, 0};
+  return run_jobs(&J, count, nthreads);
+}
+
 int oracle_gemm_sampled(const uint8_t *aq, const uint8_t *asf, const uint8_t *b,
                         const uint8_t *bsf, int bkind, int64_t M, int64_t N, int64_t K,
                         const uint16_t *bias, const uint16_t *residual, int64_t ld_res,
                         double alpha, int act, const int64_t *ms, const int64_t *ns,
                         int64_t count, double *ref, double *sumabs, int nthreads) {
-  if (K <= 0 || K % BLOCK || bkind < 0 || bkind > 2) return ORACLE_ERR_SHAPE;
-  (void)M;
-  gemm_job J = {aq, asf, b, bsf, bkind, M, N, K, bias, residual, ld_res, alpha, act,
-                ref, sumabs, ms, ns, count, 0, 0, 0};
-  return run_jobs(&J, count, nthreads);
+  return oracle_gemm_sampled_ex(aq, asf, ORACLE_A_E4M3, b, bsf, bkind, M, N, K, bias, residual,
+                                ld_res, alpha, act, ms, ns, count, ref, sumabs, nthreads);
 }
