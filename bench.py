@@ -59,9 +59,24 @@ WORKLOADS = {
              "down-projection 4096x1536x6144",
         layers=[("up8", "mxfp4", 1024, 2048, 2048, 8, dict(bias=True, gelu=True)),
                 ("down", "mxfp4", 4096, 1536, 6144, 1, dict())], bound="tensor"),
+    # FP4 x FP4 (A4W4): MXFP4 activations (bq_act_quant_mxfp4) and MXFP4 weights
+    # on tcgen05.mma kind::mxf4, on the decode shapes and on a large square
+    "a4w4_decode": dict(
+        desc="decode-shaped linear, A4W4: act_quant_mxfp4 + MXFP4xMXFP4 GEMM + bias, M=41, "
+             "(N,K) in {(4608,1536),(6144,1536),(1536,6144)}",
+        layers=[("qkv", "a4w4", 41, 4608, 1536, 1, dict(bias=True)),
+                ("up", "a4w4", 41, 6144, 1536, 1, dict(bias=True)),
+                ("down", "a4w4", 41, 1536, 6144, 1, dict(bias=True))],
+        bound="hbm"),
+    "a4w4_square": dict(
+        desc="square MXFP4xMXFP4 GEMM M=N=K=8192 (activations act_quant_mxfp4'd per step, "
+             "MXFP4 weights)",
+        layers=[("square", "a4w4", 8192, 8192, 8192, 1, dict())], bound="tensor"),
 }
 
-WKIND = {"mxfp4": 0, "fp8blk32": 1, "mxfp8": 2}
+WKIND = {"mxfp4": 0, "fp8blk32": 1, "mxfp8": 2, "a4w4": 3}
+DTYPE = {"mxfp4": "mxfp8xmxfp4", "fp8blk32": "mxfp8xfp8blk32", "mxfp8": "mxfp8xmxfp8",
+         "a4w4": "mxfp4xmxfp4"}
 
 
 def gemm_flops(layer):
@@ -70,9 +85,11 @@ def gemm_flops(layer):
 
 
 def act_quant_bytes(layer):
-    """Algorithmic bytes of act_quant: read 2 B/elem, write 1 + 1/32 B/elem."""
-    _, _, M, _, K, B, _ = layer
-    return (2.0 + 1.0 + 1.0 / 32.0) * M * K * B
+    """Algorithmic bytes of act_quant: read 2 B/elem, write 1 + 1/32 B/elem
+    (E4M3 codes) or 1/2 + 1/32 B/elem (packed E2M1 codes)."""
+    _, wk, M, _, K, B, _ = layer
+    code = 0.5 if wk == "a4w4" else 1.0
+    return (2.0 + code + 1.0 / 32.0) * M * K * B
 
 
 def gemm_bytes(layer, quant_out=False):
@@ -80,9 +97,9 @@ def gemm_bytes(layer, quant_out=False):
     output written once (weights counted once when broadcast over a batch);
     a quantized output is 1 + 1/32 bytes per element instead of 2."""
     _, wk, M, N, K, B, ex = layer
-    w = N * K / 2.0 if wk == "mxfp4" else float(N * K)
+    w = N * K / 2.0 if wk in ("mxfp4", "a4w4") else float(N * K)
     w += N * K / 32.0  # weight scales
-    a = B * (M * K + M * K / 32.0)
+    a = B * (M * K * (0.5 if wk == "a4w4" else 1.0) + M * K / 32.0)
     y = B * M * N * ((1.0 + 1.0 / 32.0) if quant_out else 2.0)
     if ex.get("bias"):
         a += N * 2.0
@@ -250,7 +267,7 @@ class Layer:
                 xb = synth.activations(M, K, seed=sd + b, group_pow2=ex.get("act_gp"))
                 xs.append(torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16))
             x = torch.stack(xs).reshape(B * M, K).to(device)
-            if wk == "mxfp4":
+            if wk in ("mxfp4", "a4w4"):
                 wb, ws = synth.mxfp4_weight(N, K, seed=sd + 500)
                 w = torch.from_numpy(wb).to(device)
                 wsf = bq.pack_weight_scales(torch.from_numpy(ws).to(device), bq.BQ_SF_ROW32, N, K)
@@ -272,13 +289,15 @@ class Layer:
                    .view(torch.bfloat16).to(device) if ex.get("residual") else None)
             self.sets.append(dict(x=x, w=w, wsf=wsf, wx=wx, bias=bias, res=res))
         # outputs shared by all sets (written every step)
-        self.aq = torch.empty((B * M, K), dtype=torch.uint8, device=device)
+        self.a4 = wk == "a4w4"  # packed E2M1 activations, two codes per byte
+        self.aq = torch.empty((B * M, K // 2 if self.a4 else K), dtype=torch.uint8,
+                              device=device)
         per = bq.sf_bytes(M, K)
         self.asf = torch.empty((B, per), dtype=torch.uint8, device=device)
         self.y = torch.empty((B, M, N), dtype=torch.bfloat16, device=device)
         self.quant_out = quant_out
         # one call per layer: the GEMM quantizes its bf16 activations itself
-        self.fused_act = fused_act and M <= 64 and B == 1 and K % 128 == 0
+        self.fused_act = fused_act and M <= 64 and B == 1 and K % 128 == 0 and not self.a4
         self.qy = torch.empty((B, M, N), dtype=torch.uint8, device=device) if quant_out else None
         self.sfy = (torch.empty((B, bq.sf_bytes(M, N)), dtype=torch.uint8, device=device)
                     if quant_out else None)
@@ -310,9 +329,10 @@ class Layer:
             # rule) runs act_quant + the split GEMM instead
             return 2 if (K + 127) // 128 >= 24 and not self.quant_out else 1
         if which in ("all", "act_quant"):
+            quant = bq.act_quant_mxfp4 if self.a4 else bq.act_quant
             for b in range(B):
-                bq.act_quant(d["x"][b * M:(b + 1) * M], q=self.aq[b * M:(b + 1) * M],
-                             sf_mma=self.asf[b])
+                quant(d["x"][b * M:(b + 1) * M], q=self.aq[b * M:(b + 1) * M],
+                      sf_mma=self.asf[b])
                 n += 1
             if d["wx"] is not None:
                 bq.act_quant(d["wx"], q=d["w"], sf_mma=d["wsf"])
@@ -320,7 +340,8 @@ class Layer:
         if which in ("all", "gemm"):
             batch = None
             if B > 1:
-                batch = dict(count=B, stride_a=M * K, stride_a_sf=self.asf.shape[1], stride_b=0,
+                batch = dict(count=B, stride_a=M * self.aq.shape[1], stride_a_sf=self.asf.shape[1],
+                             stride_b=0,
                              stride_b_sf=0, stride_y=M * N * 2, stride_res=M * N * 2)
             kw = {}
             if self.quant_out:  # the output in MXFP8 for a next projection, no bf16 y
@@ -450,7 +471,7 @@ def oracle_step_sample(layers_spec, rows, seed=0, nthreads=None):
     for (name, wk, M, N, K, B, ex) in layers_spec:
         r = min(rows, M)
         x = synth.activations(r, K, seed=seed, group_pow2=ex.get("act_gp"))
-        if wk == "mxfp4":
+        if wk in ("mxfp4", "a4w4"):
             wb, ws = synth.mxfp4_weight(N, K, seed=seed + 500)
             kind = oracle.B_FP4
         elif wk == "fp8blk32":
@@ -462,10 +483,13 @@ def oracle_step_sample(layers_spec, rows, seed=0, nthreads=None):
         bias = synth.bias(N, seed=seed + 600) if ex.get("bias") else None
         res = synth.residual(r, N, seed=seed + 700) if ex.get("residual") else None
         t0 = time.perf_counter()
-        q, s = oracle.act_quant(x)
+        if wk == "a4w4":
+            q, s = oracle.act_quant_fp4(x)
+        else:
+            q, s = oracle.act_quant(x)
         oracle.gemm(q, s, wb, ws, kind, r, N, K, bias=bias, residual=res,
                     act=oracle.ACT_GELU if ex.get("gelu") else oracle.ACT_NONE,
-                    nthreads=nthreads)
+                    nthreads=nthreads, a_kind=oracle.A_FP4 if wk == "a4w4" else oracle.A_E4M3)
         t_total += time.perf_counter() - t0
         flops += 2.0 * r * N * K
     return flops, t_total, nthreads
@@ -610,7 +634,10 @@ def run_ours(args, spec, world, rank, local, device):
     capped = bool(ck) and "sw_power_cap" in (ck.get("reasons") or []) and bool(
         ck.get("sm_mhz") and ck.get("sm_max_mhz") and ck["sm_mhz"] < 0.97 * ck["sm_max_mhz"])
     tensor_kind = "bf16_sus" if capped else "bf16"
-    fp8_peak = 2.0 * peaks[tensor_kind]  # nominal dense fp8 / bf16 ratio 4.5 / 2.25
+    # nominal dense fp8 / bf16 ratio 4.5 / 2.25; FP4 x FP4 (kind::mxf4) 9 / 2.25
+    a4 = all(sp[1] == "a4w4" for sp in layers_spec)
+    tensor_ratio = 4.0 if a4 else 2.0
+    fp8_peak = tensor_ratio * peaks[tensor_kind]
     gemm_launches = len(layers_spec)
     if spec["bound"] == "hbm":
         achieved = gbytes_step / (gemm_ms_step * 1e-3) / 1e9
@@ -627,7 +654,8 @@ def run_ours(args, spec, world, rank, local, device):
                     kernel="gemm_bs_kernel", flops_per_launch=flops_step / gemm_launches,
                     avg_launch_us=round(gemm_ms_step * 1e3 / gemm_launches, 3),
                     peak_source=(f"{peaks['src']} {'bf16_tflops_sustained' if tensor_kind != 'bf16' else 'bf16_tflops'}"
-                                 " x 2 (nominal fp8/bf16 ratio)"))
+                                 f" x {tensor_ratio:g} (nominal "
+                                 f"{'fp4' if a4 else 'fp8'}/bf16 ratio)"))
     e2e_ms, h2d, d2h = run_e2e(layers_spec, layers, min(2000, max(10, args.steps // 4)), device)
     out = {
         "metric": METRIC,
@@ -640,8 +668,7 @@ def run_ours(args, spec, world, rank, local, device):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "mxfp8xmxfp4" if layers_spec[0][1] == "mxfp4" else
-                 ("mxfp8xfp8blk32" if layers_spec[0][1] == "fp8blk32" else "mxfp8xmxfp8"),
+        "dtype": DTYPE[layers_spec[0][1]],
         "data": "synthetic",
         "config": {"workload": spec["desc"], "parallelism": "replicas" if world > 1 else "single",
                    "l2": f"{nsets} rotating input sets of {set_bytes / 1e6:.1f} MB "

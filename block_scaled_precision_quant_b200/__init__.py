@@ -37,6 +37,7 @@ BQ_ACT_NONE = 0
 BQ_ACT_GELU = 1
 BQ_SPLIT_AUTO, BQ_SPLIT_WORKSPACE, BQ_SPLIT_CLUSTER = 0, 1, 2
 W_MXFP4, W_FP8BLK32, W_MXFP8 = 0, 1, 2
+W_A4W4 = 3  # MXFP4 weights with MXFP4 (packed E2M1) activations
 
 EXPORTS = (
     "bq_status_string", "bq_version", "bq_sf_bytes", "bq_act_quant", "bq_pack_weight_scales",
@@ -44,7 +45,8 @@ EXPORTS = (
     "bq_gemm_workspace_bytes", "bq_gemm_mxfp8_mxfp4_epilogue", "bq_gemm_mxfp8_fp8blk32_epilogue",
     "bq_gemm_mxfp8_mxfp8_epilogue", "bq_device_status", "bq_device_status_detail",
     "bq_device_report", "bq_gemm_mxfp8_mxfp4_epilogue_noalloc", "bq_noalloc_scratch_bytes",
-    "bq_gemm_bf16act_epilogue", "bq_gemm_plan",
+    "bq_gemm_bf16act_epilogue", "bq_gemm_plan", "bq_act_quant_mxfp4", "bq_gemm_mxfp4_mxfp4",
+    "bq_gemm_mxfp4_mxfp4_epilogue",
 )
 
 
@@ -98,16 +100,19 @@ def lib():
         L.bq_sf_bytes.restype = sz
         L.bq_act_quant.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp]
         L.bq_act_quant.restype = i32
+        L.bq_act_quant_mxfp4.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp]
+        L.bq_act_quant_mxfp4.restype = i32
         L.bq_pack_weight_scales.argtypes = [vp, i32, i64, i64, vp, vp, vp]
         L.bq_pack_weight_scales.restype = i32
         L.bq_unpack_scales.argtypes = [vp, i64, i64, vp, vp]
         L.bq_unpack_scales.restype = i32
-        for name in ("bq_gemm_mxfp8_mxfp4", "bq_gemm_mxfp8_fp8blk32", "bq_gemm_mxfp8_mxfp8"):
+        for name in ("bq_gemm_mxfp8_mxfp4", "bq_gemm_mxfp8_fp8blk32", "bq_gemm_mxfp8_mxfp8",
+                     "bq_gemm_mxfp4_mxfp4"):
             f = getattr(L, name)
             f.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp]
             f.restype = i32
         for name in ("bq_gemm_mxfp8_mxfp4_epilogue", "bq_gemm_mxfp8_fp8blk32_epilogue",
-                     "bq_gemm_mxfp8_mxfp8_epilogue"):
+                     "bq_gemm_mxfp8_mxfp8_epilogue", "bq_gemm_mxfp4_mxfp4_epilogue"):
             f = getattr(L, name)
             f.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, ctypes.POINTER(Epilogue),
                           ctypes.POINTER(Batch), vp, sz, ctypes.POINTER(GemmConfig), vp]
@@ -122,7 +127,7 @@ def lib():
         L.bq_gemm_bf16act_epilogue.restype = i32
         L.bq_gemm_workspace_bytes.argtypes = [i32, i64, i64, i64, i64, ctypes.POINTER(GemmConfig)]
         L.bq_gemm_workspace_bytes.restype = sz
-        L.bq_gemm_plan.argtypes = [i64, i64, i64, i64, ctypes.POINTER(GemmConfig), i32,
+        L.bq_gemm_plan.argtypes = [i32, i64, i64, i64, i64, ctypes.POINTER(GemmConfig), i32,
                                    ctypes.POINTER(GemmConfig)]
         L.bq_gemm_plan.restype = i32
         L.bq_device_status.argtypes = [vp]
@@ -210,6 +215,25 @@ def act_quant(x, q=None, sf_mma=None, sf_rowmajor=None, status=None):
     return q, sf_mma
 
 
+def act_quant_mxfp4(x, q=None, sf_mma=None, sf_rowmajor=None, status=None):
+    """Per-32 MXFP4 quantization of a bf16 [M, K] CUDA tensor: returns (q
+    uint8 [M, K/2] packed E2M1 codes, low nibble = even element, sf_mma uint8
+    MMA-layout scales), the operands of gemm(W_A4W4, ...)."""
+    torch = _torch()
+    _need_cuda(x)
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a bf16 [M, K] tensor with unit column stride")
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
+    if sf_mma is None:
+        sf_mma = torch.empty((max(sf_bytes(M, K), 1),), dtype=torch.uint8, device=x.device)
+    _check(lib().bq_act_quant_mxfp4(_ptr(x), M, K, x.stride(0), _ptr(q), _ptr(sf_mma),
+                                    _ptr(sf_rowmajor), _ptr(status), _stream()),
+           "bq_act_quant_mxfp4")
+    return q, sf_mma
+
+
 def pack_weight_scales(scales, kind: int, N: int, K: int, out=None, e4m3_codes=None):
     """E8M0 weight scales (ROW32 [N, K/32] or BLK32x32 [ceil(N/32), K/32]) to
     the MMA layout.  Synchronizes the stream; raises on NaN scales or codes."""
@@ -237,7 +261,7 @@ def unpack_scales(sf_mma, rows: int, K: int, out=None):
 
 _ws = {}
 _ENTRY = {W_MXFP4: "bq_gemm_mxfp8_mxfp4", W_FP8BLK32: "bq_gemm_mxfp8_fp8blk32",
-          W_MXFP8: "bq_gemm_mxfp8_mxfp8"}
+          W_MXFP8: "bq_gemm_mxfp8_mxfp8", W_A4W4: "bq_gemm_mxfp4_mxfp4"}
 
 
 def _config(block_n=0, split_k=0, swap_ab=-1, split_mode=0, k_chunks=0, cta_pair=0):
@@ -251,12 +275,13 @@ def workspace_bytes(weight_kind, M, N, K, batch=1, config=None) -> int:
                                              ctypes.byref(cfg) if cfg is not None else None))
 
 
-def plan(M, N, K, batch=1, config=None, num_sms=148) -> GemmConfig:
+def plan(M, N, K, batch=1, config=None, num_sms=148, weight_kind=0) -> GemmConfig:
     """The schedule the built-in dispatch picks (host-only, no device): every
     GemmConfig field resolved for a device with num_sms SMs."""
     out = GemmConfig()
-    _check(lib().bq_gemm_plan(M, N, K, batch, ctypes.byref(config) if config is not None
-                              else None, num_sms, ctypes.byref(out)), "bq_gemm_plan")
+    _check(lib().bq_gemm_plan(int(weight_kind), M, N, K, batch,
+                              ctypes.byref(config) if config is not None else None, num_sms,
+                              ctypes.byref(out)), "bq_gemm_plan")
     return out
 
 
@@ -276,7 +301,8 @@ def gemm(weight_kind, a_q, a_sf, b, b_sf, M, N, K, y=None, bias=None, residual=N
          alpha=1.0, act=BQ_ACT_NONE, batch=None, config=None, workspace=None,
          quantize_out=False, write_y=True, q_out=None, sf_out=None):
     """y = bf16(act(alpha * A B^T + bias) + residual) for weight_kind W_MXFP4,
-    W_FP8BLK32 or W_MXFP8.  batch: None or a dict with 'count' and byte
+    W_FP8BLK32, W_MXFP8 (E4M3 activations a_q [.., M, K]) or W_A4W4 (packed
+    E2M1 activations a_q [.., M, K/2] from act_quant_mxfp4).  batch: None or a dict with 'count' and byte
     strides ('stride_a', 'stride_a_sf', 'stride_b', 'stride_b_sf', 'stride_y',
     'stride_res'; 0 broadcasts).  config: GemmConfig or None (auto).
     quantize_out: also return y quantized for the next GEMM (E4M3 codes
@@ -384,6 +410,10 @@ def gemm_mxfp8_fp8blk32(a_q, a_sf, b_e4m3, b_sf, M, N, K, **kw):
 
 def gemm_mxfp8_mxfp8(a_q, a_sf, b_e4m3, b_sf, M, N, K, **kw):
     return gemm(W_MXFP8, a_q, a_sf, b_e4m3, b_sf, M, N, K, **kw)
+
+
+def gemm_mxfp4_mxfp4(a_fp4, a_sf, b_fp4, b_sf, M, N, K, **kw):
+    return gemm(W_A4W4, a_fp4, a_sf, b_fp4, b_sf, M, N, K, **kw)
 
 
 config = _config

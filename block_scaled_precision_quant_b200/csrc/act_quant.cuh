@@ -21,7 +21,9 @@
 namespace bq {
 
 // grid: x*8 + warp = row, y = chunk of 16 groups within the row.  Rows in
-// [M, rows_pad) only write padding scale bytes (127).
+// [M, rows_pad) only write padding scale bytes (127).  FP4: E2M1 codes
+// (packed [M, K/2], the per-32 rule with 6 in place of 448) instead of E4M3.
+template <bool FP4>
 __global__ void __launch_bounds__(256) act_quant_kernel(
     const __nv_bfloat16 *__restrict__ x, int64_t M, int64_t K, int64_t ldx, int64_t rows_pad,
     uint8_t *__restrict__ q, uint8_t *__restrict__ sf_mma, uint8_t *__restrict__ sf_row,
@@ -57,11 +59,17 @@ __global__ void __launch_bounds__(256) act_quant_kernel(
   uint32_t sbyte = 127;
   if (active) {
     if (bad && status) atomicOr(status, 1);
-    const int e = mx_exponent(mx);
+    const int e = FP4 ? mx_exponent_fp4(mx) : mx_exponent(mx);
     sbyte = static_cast<uint32_t>(e + 127);
-    uint32_t c[4];
-    mx_encode(w, e, c);
-    *reinterpret_cast<uint4 *>(q + row * K + col) = make_uint4(c[0], c[1], c[2], c[3]);
+    if constexpr (FP4) {
+      uint32_t c[2];
+      mx_encode_fp4(w, e, c);
+      *reinterpret_cast<uint2 *>(q + row * (K >> 1) + (col >> 1)) = make_uint2(c[0], c[1]);
+    } else {
+      uint32_t c[4];
+      mx_encode(w, e, c);
+      *reinterpret_cast<uint4 *>(q + row * K + col) = make_uint4(c[0], c[1], c[2], c[3]);
+    }
     if (sf_row && half == 0) sf_row[row * G + g] = static_cast<uint8_t>(sbyte);
   }
   // Gather the bytes of groups 4j..4j+3 of this chunk (lanes 8j, 8j+2, 8j+4,

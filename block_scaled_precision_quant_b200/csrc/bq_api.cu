@@ -174,7 +174,8 @@ int make_y_map(CUtensorMap* m, const void* y, int64_t M, int64_t N, int64_t ld, 
 
 // ---------------------------------------------------------------- schedule --
 
-enum WeightKind { kMxfp4 = 0, kFp8Blk32 = 1, kMxfp8 = 2 };
+// kA4W4: MXFP4 weights with MXFP4 (packed E2M1) activations, kind::mxf4.
+enum WeightKind { kMxfp4 = 0, kFp8Blk32 = 1, kMxfp8 = 2, kA4W4 = 3 };
 
 struct Plan {
   bool swap = false;
@@ -320,9 +321,24 @@ size_t plan_ws_bytes(const Plan& p) {
 }
 
 // The plan a call runs; one that needs more workspace than given is refused.
-int plan_for_call(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_config* cfg,
-                  int num_sms, const void* ws, size_t ws_bytes, Plan* p) {
-  const int st = make_plan(M, N, K, batch, cfg, num_sms, p);
+// The plan of a call of weight kind wk: packed E2M1 operands on both sides
+// (A4W4) have K/2 bytes per row, so their schedule counts chunks of 256 K;
+// they have no pair-tile kernel.
+int plan_kind(WeightKind wk, int64_t M, int64_t N, int64_t K, int64_t batch,
+              const bq_gemm_config* cfg, int num_sms, Plan* p) {
+  if (wk == kA4W4) {
+    bq_gemm_config c = cfg ? *cfg : bq_gemm_config{0, 0, -1, BQ_SPLIT_AUTO, 0, 0};
+    if (c.cta_pair == 2) return BQ_ERR_INVALID;
+    if (c.cta_pair == 0) c.cta_pair = 1;
+    return make_plan(M, N, K / 2, batch, &c, num_sms, p);
+  }
+  return make_plan(M, N, K, batch, cfg, num_sms, p);
+}
+
+int plan_for_call(WeightKind wk, int64_t M, int64_t N, int64_t K, int64_t batch,
+                  const bq_gemm_config* cfg, int num_sms, const void* ws, size_t ws_bytes,
+                  Plan* p) {
+  const int st = plan_kind(wk, M, N, K, batch, cfg, num_sms, p);
   if (st != BQ_OK) return st;
   const size_t need = plan_ws_bytes(*p);
   return (need == 0 || (ws && ws_bytes >= need)) ? BQ_OK : BQ_ERR_WORKSPACE;
@@ -331,13 +347,13 @@ int plan_for_call(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_
 // --------------------------------------------------------------- launches --
 
 template <int BN, int STAGES, int ACC, bool SWAP, bool P_FP4, bool Q_FP4, int MODE, int KC,
-          bool FUSEQ = false>
+          bool FUSEQ = false, bool A4 = false>
 int launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap& ty,
                 const CUtensorMap& tr, const bq::GemmArgs& args,
                 int64_t units, int num_sms, cudaStream_t stream) {
   constexpr bool CSPLIT = MODE == bq::kSplitCluster;
-  using L = bq::KernelSmem<BN, STAGES, ACC, SWAP, MODE, KC>;
-  auto kern = bq::gemm_bs_kernel<BN, STAGES, ACC, SWAP, P_FP4, Q_FP4, MODE, KC, FUSEQ>;
+  using L = bq::KernelSmem<BN, STAGES, ACC, SWAP, MODE, KC, A4 ? 2 : 1>;
+  auto kern = bq::gemm_bs_kernel<BN, STAGES, ACC, SWAP, P_FP4, Q_FP4, MODE, KC, FUSEQ, A4>;
   static bool attr_set[kMaxDevices] = {};
   static int per_sm_cache[kMaxDevices] = {};
   int dev = 0;
@@ -392,10 +408,14 @@ int launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap&
   return launch_status();
 }
 
-template <int BN, int STAGES, int ACC, bool SWAP, int MODE, int KC, bool FUSEQ = false>
+template <int BN, int STAGES, int ACC, bool SWAP, int MODE, int KC, bool FUSEQ = false,
+          bool A4 = false>
 int launch_kind(bool w_fp4, const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap& ty,
                 const CUtensorMap& tr, const bq::GemmArgs& args, int64_t u, int num_sms,
                 cudaStream_t st) {
+  if constexpr (A4)  // packed E2M1 on both sides: plain byte operands
+    return launch_gemm<BN, STAGES, ACC, SWAP, false, false, MODE, KC, false, true>(
+        tp, tq, ty, tr, args, u, num_sms, st);
   // FP4 weights sit on the P side with SWAP, on the Q side otherwise.
   if (w_fp4)
     return launch_gemm<BN, STAGES, ACC, SWAP, SWAP, !SWAP, MODE, KC, FUSEQ>(tp, tq, ty, tr, args, u,
@@ -447,8 +467,9 @@ int launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
   return launch_status();
 }
 
-// Dispatch on (swap, bn, chunks per stage, split mode, fp4 weights) to the
+// Dispatch on (swap, bn, chunks per stage, split mode, weight format) to the
 // compiled instances.  Stage counts fill ~200 KB of shared memory.
+template <bool A4>
 int run_gemm(const Plan& pl, bool w_fp4, const CUtensorMap& tp, const CUtensorMap& tq,
              const CUtensorMap& ty, const CUtensorMap& tr, const bq::GemmArgs& a, int ns,
              cudaStream_t st) {
@@ -457,33 +478,35 @@ int run_gemm(const Plan& pl, bool w_fp4, const CUtensorMap& tp, const CUtensorMa
   const bool b32 = pl.bn == 32;
   if (!pl.swap) {
     if (pl.bn == 256) {
-      if (pl.splits > 1) return launch_kind<256, 4, 1, false, kWs, 1>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
-      return pl.kc == 2 ? launch_kind<256, 2, 1, false, kNone, 2>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
-                        : launch_kind<256, 4, 1, false, kNone, 1>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
+      if (pl.splits > 1) return launch_kind<256, 4, 1, false, kWs, 1, false, A4>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
+      return pl.kc == 2 ? launch_kind<256, 2, 1, false, kNone, 2, false, A4>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
+                        : launch_kind<256, 4, 1, false, kNone, 1, false, A4>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
     }
-    if (pl.splits > 1) return launch_kind<128, 6, 2, false, kWs, 1>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
-    return pl.kc == 2 ? launch_kind<128, 3, 2, false, kNone, 2>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
-                      : launch_kind<128, 6, 2, false, kNone, 1>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
+    if (pl.splits > 1) return launch_kind<128, 6, 2, false, kWs, 1, false, A4>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
+    return pl.kc == 2 ? launch_kind<128, 3, 2, false, kNone, 2, false, A4>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
+                      : launch_kind<128, 6, 2, false, kNone, 1, false, A4>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
   }
-  if (a.x) {  // fused activation quantization: unsplit 4-chunk swap tiles
-    return b32 ? launch_kind<32, 2, 1, true, kNone, 4, true>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
-               : launch_kind<64, 2, 1, true, kNone, 4, true>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
+  if constexpr (!A4) {
+    if (a.x) {  // fused activation quantization: unsplit 4-chunk swap tiles
+      return b32 ? launch_kind<32, 2, 1, true, kNone, 4, true>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
+                 : launch_kind<64, 2, 1, true, kNone, 4, true>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
+    }
   }
   if (pl.cluster) {
     if (pl.kc == 4)
-      return b32 ? launch_kind<32, 1, 1, true, kCl, 4>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
-                 : launch_kind<64, 1, 1, true, kCl, 4>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
-    return b32 ? launch_kind<32, 3, 1, true, kCl, 1>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
-               : launch_kind<64, 3, 1, true, kCl, 1>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
+      return b32 ? launch_kind<32, 1, 1, true, kCl, 4, false, A4>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
+                 : launch_kind<64, 1, 1, true, kCl, 4, false, A4>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
+    return b32 ? launch_kind<32, 3, 1, true, kCl, 1, false, A4>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
+               : launch_kind<64, 3, 1, true, kCl, 1, false, A4>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
   }
   if (pl.splits > 1)
-    return b32 ? launch_kind<32, 4, 1, true, kWs, 1>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
-               : launch_kind<64, 4, 1, true, kWs, 1>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
+    return b32 ? launch_kind<32, 4, 1, true, kWs, 1, false, A4>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
+               : launch_kind<64, 4, 1, true, kWs, 1, false, A4>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
   if (pl.kc == 4)
-    return b32 ? launch_kind<32, 2, 1, true, kNone, 4>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
-               : launch_kind<64, 2, 1, true, kNone, 4>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
-  return b32 ? launch_kind<32, 8, 1, true, kNone, 1>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
-             : launch_kind<64, 8, 1, true, kNone, 1>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
+    return b32 ? launch_kind<32, 2, 1, true, kNone, 4, false, A4>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
+               : launch_kind<64, 2, 1, true, kNone, 4, false, A4>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
+  return b32 ? launch_kind<32, 8, 1, true, kNone, 1, false, A4>(w_fp4, tp, tq, ty, tr, a, u, ns, st)
+             : launch_kind<64, 8, 1, true, kNone, 1, false, A4>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
 }
 
 // Activations given as bf16 and quantized inside the GEMM (decode tiles).
@@ -522,9 +545,13 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
   }
   if (q_out && (!aligned(q_out, 16) || !aligned(sf_out, 4))) return BQ_ERR_ALIGN;
   const bool w_fp4 = wk == kMxfp4;
+  const bool a4 = wk == kA4W4;
+  if (a4 && fused) return BQ_ERR_INVALID;  // the fused quantizer emits E4M3 codes
+  // Bytes of K per operand row: packed E2M1 rows hold two codes per byte.
+  const int64_t Kb = a4 ? K / 2 : K;
   if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF || count > 65535) return BQ_ERR_SHAPE;
   if (N % 8 != 0) return BQ_ERR_SHAPE;
-  if (w_fp4 && K % 128 != 0) return BQ_ERR_SHAPE;
+  if ((w_fp4 || a4) && K % 128 != 0) return BQ_ERR_SHAPE;
   if ((!fused && (!aligned(a_q, 16) || !aligned(a_sf, 16))) || !aligned(b_sf, 16) ||
       (y && !aligned(y, 16)) || !aligned(b, w_fp4 ? 32 : 16))
     return BQ_ERR_ALIGN;
@@ -560,7 +587,7 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
     cfg = &cfg_q;
   }
   Plan pl;
-  st = plan_for_call(M, N, K, count, cfg, dev->num_sms, ws, ws_bytes, &pl);
+  st = plan_for_call(wk, M, N, K, count, cfg, dev->num_sms, ws, ws_bytes, &pl);
   if (st != BQ_OK) return st;
   const size_t need = plan_ws_bytes(pl);
   if (need > 0 && !aligned(ws, 16)) return BQ_ERR_WORKSPACE;
@@ -581,10 +608,11 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
   if (fused) {
     st = BQ_OK;  // no activation copies: map_a is set to a placeholder below
   } else {
-    st = make_operand_map(&map_a, a_q, false, K, M, K, a_batched ? count : 1, sa, a_box, pl.kc);
+    st = make_operand_map(&map_a, a_q, false, Kb, M, Kb, a_batched ? count : 1, sa, a_box,
+                          pl.kc);
     if (st != BQ_OK) return st;
   }
-  st = make_operand_map(&map_b, b, w_fp4, K, N, w_fp4 ? K / 2 : K, b_batched ? count : 1, sb,
+  st = make_operand_map(&map_b, b, w_fp4, Kb, N, w_fp4 ? K / 2 : Kb, b_batched ? count : 1, sb,
                         b_box, pl.kc);
   if (st != BQ_OK) return st;
   if (fused) map_a = map_b;
@@ -670,8 +698,11 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
   }
   const CUtensorMap& tp = pl.swap ? map_b : map_a;
   const CUtensorMap& tq = pl.swap ? map_a : map_b;
-  return run_gemm(pl, w_fp4, tp, tq, map_y, map_res, g, dev->num_sms,
-                  reinterpret_cast<cudaStream_t>(stream));
+  if (a4)
+    return run_gemm<true>(pl, false, tp, tq, map_y, map_res, g, dev->num_sms,
+                          reinterpret_cast<cudaStream_t>(stream));
+  return run_gemm<false>(pl, w_fp4, tp, tq, map_y, map_res, g, dev->num_sms,
+                         reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // namespace
@@ -705,15 +736,21 @@ size_t bq_sf_bytes(int64_t rows, int64_t K) {
   return static_cast<size_t>((rows + 127) / 128) * static_cast<size_t>((K + 127) / 128) * 512;
 }
 
-int bq_act_quant(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, void* q_e4m3,
-                 void* sf_mma, void* sf_rowmajor, int* d_status, bq_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Launch of the per-32 activation quantizer; fp4 selects E2M1 output.
+int act_quant_launch(bool fp4, const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+                     void* q_out, void* sf_mma, void* sf_rowmajor, int* d_status,
+                     bq_stream_t stream) {
   DevInfo* dev = nullptr;
   int st = current_device(&dev);
   if (st != BQ_OK) return st;
   if (M < 0 || K <= 0 || K % 32 != 0 || ldx < K) return BQ_ERR_SHAPE;
   if (M == 0) return BQ_OK;
-  if (!x_bf16 || !q_e4m3 || !sf_mma) return BQ_ERR_NULL;
-  if (!aligned(x_bf16, 16) || ldx % 8 != 0 || !aligned(q_e4m3, 16) || !aligned(sf_mma, 4))
+  if (!x_bf16 || !q_out || !sf_mma) return BQ_ERR_NULL;
+  if (!aligned(x_bf16, 16) || ldx % 8 != 0 || !aligned(q_out, 16) || !aligned(sf_mma, 4))
     return BQ_ERR_ALIGN;
   const int64_t rows_pad = (M + 127) / 128 * 128;
   const int64_t chunks = (K / 32 + 15) / 16;
@@ -727,14 +764,29 @@ int bq_act_quant(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, void* q_
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = 1;
-  if (cudaLaunchKernelEx(&lc, bq::act_quant_kernel, static_cast<const __nv_bfloat16*>(x_bf16), M,
-                         K, ldx, rows_pad, static_cast<uint8_t*>(q_e4m3),
-                         static_cast<uint8_t*>(sf_mma), static_cast<uint8_t*>(sf_rowmajor),
-                         d_status) != cudaSuccess) {
+  auto kern = fp4 ? bq::act_quant_kernel<true> : bq::act_quant_kernel<false>;
+  if (cudaLaunchKernelEx(&lc, kern, static_cast<const __nv_bfloat16*>(x_bf16), M, K, ldx,
+                         rows_pad, static_cast<uint8_t*>(q_out), static_cast<uint8_t*>(sf_mma),
+                         static_cast<uint8_t*>(sf_rowmajor), d_status) != cudaSuccess) {
     cudaGetLastError();
     return BQ_ERR_CUDA;
   }
   return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int bq_act_quant(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, void* q_e4m3,
+                 void* sf_mma, void* sf_rowmajor, int* d_status, bq_stream_t stream) {
+  return act_quant_launch(false, x_bf16, M, K, ldx, q_e4m3, sf_mma, sf_rowmajor, d_status,
+                          stream);
+}
+
+int bq_act_quant_mxfp4(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, void* q_fp4,
+                       void* sf_mma, void* sf_rowmajor, int* d_status, bq_stream_t stream) {
+  return act_quant_launch(true, x_bf16, M, K, ldx, q_fp4, sf_mma, sf_rowmajor, d_status, stream);
 }
 
 int bq_pack_weight_scales(const void* scales_u8, int kind, int64_t N, int64_t K, void* sf_mma,
@@ -814,23 +866,42 @@ int bq_gemm_mxfp8_mxfp8(const void* a_q, const void* a_sf, const void* b_e4m3, c
                     0, &kNoSplit, stream);
 }
 
+int bq_gemm_mxfp4_mxfp4(const void* a_fp4, const void* a_sf, const void* b_fp4, const void* b_sf,
+                        int64_t M, int64_t N, int64_t K, void* y_bf16, bq_stream_t stream) {
+  return gemm_entry(kA4W4, a_fp4, a_sf, b_fp4, b_sf, M, N, K, y_bf16, nullptr, nullptr, nullptr, 0,
+                    &kNoSplit, stream);
+}
+
+int bq_gemm_mxfp4_mxfp4_epilogue(const void* a_fp4, const void* a_sf, const void* b_fp4,
+                                 const void* b_sf, int64_t M, int64_t N, int64_t K, void* y_bf16,
+                                 const bq_epilogue* epi, const bq_batch* batch, void* workspace,
+                                 size_t workspace_bytes, const bq_gemm_config* cfg,
+                                 bq_stream_t stream) {
+  return gemm_entry(kA4W4, a_fp4, a_sf, b_fp4, b_sf, M, N, K, y_bf16, epi, batch, workspace,
+                    workspace_bytes, cfg, stream);
+}
+
 size_t bq_gemm_workspace_bytes(int weight_kind, int64_t M, int64_t N, int64_t K, int64_t batch,
                                const bq_gemm_config* cfg) {
-  if (weight_kind < 0 || weight_kind > 2 || M <= 0 || N <= 0 || K <= 0 || batch <= 0) return 0;
+  if (weight_kind < 0 || weight_kind > 3 || M <= 0 || N <= 0 || K <= 0 || batch <= 0) return 0;
   DevInfo* dev = nullptr;
   if (current_device(&dev) != BQ_OK) return 0;
   Plan pl;
-  if (make_plan(M, N, K, batch, cfg, dev->num_sms, &pl) != BQ_OK) return 0;
+  if (plan_kind(static_cast<WeightKind>(weight_kind), M, N, K, batch, cfg, dev->num_sms, &pl) !=
+      BQ_OK)
+    return 0;
   return plan_ws_bytes(pl);
 }
 
-int bq_gemm_plan(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_config* cfg,
-                 int num_sms, bq_gemm_config* out) {
+int bq_gemm_plan(int weight_kind, int64_t M, int64_t N, int64_t K, int64_t batch,
+                 const bq_gemm_config* cfg, int num_sms, bq_gemm_config* out) {
   if (!out) return BQ_ERR_NULL;
+  if (weight_kind < 0 || weight_kind > 3) return BQ_ERR_INVALID;
   if (M <= 0 || N <= 0 || K <= 0 || K % 32 != 0 || batch <= 0 || num_sms < 1)
     return BQ_ERR_SHAPE;
   Plan pl;
-  const int st = make_plan(M, N, K, batch, cfg, num_sms, &pl);
+  const int st = plan_kind(static_cast<WeightKind>(weight_kind), M, N, K, batch, cfg, num_sms,
+                           &pl);
   if (st != BQ_OK) return st;
   out->block_n = pl.bn;
   out->split_k = pl.splits;
@@ -944,7 +1015,8 @@ int bq_gemm_mxfp8_mxfp4_epilogue_noalloc(const void* a_q, const void* a_sf, cons
   // Same planning as the call below makes with this scratch as its workspace
   // (a schedule that needs more than the scratch is refused).
   Plan pl;
-  st = plan_for_call(M, N, K, count, cfg, dev->num_sms, scratch, kNoAllocScratchBytes, &pl);
+  st = plan_for_call(kMxfp4, M, N, K, count, cfg, dev->num_sms, scratch, kNoAllocScratchBytes,
+                     &pl);
   if (st != BQ_OK) return st;
   if (plan_ws_bytes(pl) > 0) {
     // The scratch keeps whatever the previous call left: zero this call's

@@ -429,6 +429,22 @@ __device__ __forceinline__ void tc_mma_mxf8f6f4(uint32_t d_tmem, uint64_t adesc,
       : "memory");
 }
 
+// The same with both operands packed E2M1 (two codes per byte, no padding):
+// K = 64 per instruction, two E8M0 scales per row (bytes sf_id and sf_id + 1
+// of the row's scale word, sf_id 0 or 2 in the instruction descriptor).
+__device__ __forceinline__ void tc_mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], "
+      "[%6], p;\n\t"
+      "}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
 // CTA-pair forms, issued by the pair leader: the scale copy runs in both
 // CTAs (each from its own shared memory into its own TMEM, same addresses);
 // the MMA computes the 256-row tile, rows 0-127 from the leader's operand A

@@ -55,9 +55,12 @@ constexpr int kWsfWarp = 7;
 constexpr int kAsfWarp = 8;
 constexpr int kCopyThreads = 4;
 
-// tcgen05 operand formats (instruction descriptor fields a_format / b_format).
+// tcgen05 operand formats (instruction descriptor fields a_format / b_format):
+// kind::mxf8f6f4 codes E4M3 0 and E2M1 5 (one byte slot per FP4 code in shared
+// memory); kind::mxf4 code E2M1 1 (two codes per byte).
 constexpr uint32_t kFmtE4M3 = 0;
 constexpr uint32_t kFmtE2M1 = 5;
+constexpr uint32_t kFmtMxf4E2M1 = 1;
 
 struct GemmArgs {
   int M, N, K;     // one problem: y[M, N] = A[M, K] B[N, K]^T
@@ -113,22 +116,24 @@ struct GemmArgs {
 enum SplitMode : int { kSplitNone = 0, kSplitWorkspace = 1, kSplitCluster = 2 };
 
 // Shared-memory layout of one kernel instance.  A stage holds KC chunks of
-// 128 K (each chunk a 128B-swizzled K-major tile per operand) and the
-// chunks' scale-factor atoms; more bytes behind one stage barrier means fewer
-// barrier round trips per byte, which is what bounds a CTA's copy rate.
+// 128 bytes of K per row (each chunk a 128B-swizzled K-major tile per
+// operand: 128 K of one-byte codes, or 256 K of packed E2M1 codes) and the
+// chunks' scale-factor atoms (APC atoms of 128 K per chunk and 128-row band);
+// more bytes behind one stage barrier means fewer barrier round trips per
+// byte, which is what bounds a CTA's copy rate.
 template <int BN, int STAGES, int ACC, bool CSPLIT = false, int KC = 1, bool OUT_STAGE = false,
-          bool LANDING = false, bool YSTAGE = false>
+          bool LANDING = false, bool YSTAGE = false, int APC = 1>
 struct GemmSmem {
-  static constexpr int kSfqAtoms = BN > 128 ? BN / 128 : 1;
+  static constexpr int kSfqAtoms = BN > 128 ? BN / 128 : 1;  // 128-row bands, Q side
   static constexpr int kSfqCols = 4 * kSfqAtoms;
-  static constexpr int kSfColsChunk = 4 + kSfqCols;  // TMEM scale columns per K chunk
-  static constexpr int kSfCols = KC * kSfColsChunk;  // TMEM scale columns per stage
+  static constexpr int kSfColsChunk = APC * (4 + kSfqCols);  // TMEM scale columns per chunk
+  static constexpr int kSfCols = KC * kSfColsChunk;          // TMEM scale columns per stage
   static constexpr int kChunkP = kBlockP * kBlockK;  // bytes of one 128-K chunk, P side
   static constexpr int kChunkQ = BN * kBlockK;       // Q side
   static constexpr int kBytesP = KC * kChunkP;
   static constexpr int kBytesQ = KC * kChunkQ;
-  static constexpr int kSfpBytes = KC * kSfAtom;              // per stage
-  static constexpr int kSfqBytes = KC * kSfqAtoms * kSfAtom;  // per stage
+  static constexpr int kSfpBytes = KC * APC * kSfAtom;              // per stage
+  static constexpr int kSfqBytes = KC * APC * kSfqAtoms * kSfAtom;  // per stage
   static constexpr int kOffQ = STAGES * kBytesP;
   // wide tiles: two 128x32 bf16 staging tiles for the TMA-store epilogue
   // (1024-byte aligned: the 64-byte swizzle follows address bits)
@@ -173,10 +178,10 @@ struct GemmSmem {
 // The layout a kernel instance uses: unsplit swap-AB tiles stage their bf16
 // output in shared memory for row-contiguous stores; swap-AB workspace splits
 // gather the slices' partial tiles in shared memory.
-template <int BN, int STAGES, int ACC, bool SWAP, int MODE, int KC>
+template <int BN, int STAGES, int ACC, bool SWAP, int MODE, int KC, int APC = 1>
 using KernelSmem = GemmSmem<BN, STAGES, ACC, MODE == kSplitCluster, KC,
                             SWAP && MODE == kSplitNone, SWAP && MODE == kSplitWorkspace,
-                            !SWAP && MODE == kSplitNone>;
+                            !SWAP && MODE == kSplitNone, APC>;
 
 __device__ __forceinline__ uint32_t make_idesc(uint32_t fmt_p, uint32_t fmt_q, int bn, int sf_id) {
   uint32_t d = 0;
@@ -593,13 +598,21 @@ __device__ __forceinline__ void copy_out_swap(const GemmArgs &a, const UnitPos &
   }
 }
 
-// Loads one part of one stage (KC chunks of 128 K starting at K block kt, of
-// which `nvalid` belong to the unit): the operand tile or the scale atoms of
-// the P side or the Q side.  KC == 1 uses 2-D (3-D batched) maps with the K
-// offset in elements; KC > 1 uses maps that view K as (128, K/128 chunks), so
-// one copy brings all chunks.  Scale atoms of one 128-row band are contiguous
-// along K, so one bulk copy per band brings a stage's atoms.
-template <int BN, class L, int KC>
+// Scale atoms (128 K each) of the stage chunks [kt, kt + nvalid) that exist:
+// with packed E2M1 operands a chunk spans APC = 2 atoms and the last chunk of
+// K may hold only the first.
+template <int APC>
+__device__ __forceinline__ int stage_atoms(const GemmArgs &a, int kt, int nvalid) {
+  return min(nvalid * APC, a.sf_katoms - kt * APC);
+}
+
+// Loads one part of one stage (KC chunks of 128 bytes of K starting at chunk
+// kt, of which `nvalid` belong to the unit): the operand tile or the scale
+// atoms of the P side or the Q side.  KC == 1 uses 2-D (3-D batched) maps
+// with the K offset in bytes; KC > 1 uses maps that view K as (128 bytes,
+// chunks), so one copy brings all chunks.  Scale atoms of one 128-row band
+// are contiguous along K, so one bulk copy per band brings a stage's atoms.
+template <int BN, class L, int KC, int APC = 1>
 __device__ __forceinline__ void issue_part(const GemmArgs &a, const CUtensorMap *tm_p,
                                            const CUtensorMap *tm_q, uint8_t *smem,
                                            uint64_t *full, int st, int kt, int nvalid,
@@ -607,8 +620,9 @@ __device__ __forceinline__ void issue_part(const GemmArgs &a, const CUtensorMap 
   if (p_side) {
     if (scales) {
       const uint8_t *sfp = a.sf_p + u.b * a.sf_p_bstride +
-                           (static_cast<int64_t>(u.tp) * a.sf_katoms + kt) * kSfAtom;
-      bulk_load(smem + L::kOffSfp + st * L::kSfpBytes, sfp, nvalid * kSfAtom, &full[st]);
+                           (static_cast<int64_t>(u.tp) * a.sf_katoms + kt * APC) * kSfAtom;
+      bulk_load(smem + L::kOffSfp + st * L::kSfpBytes, sfp,
+                stage_atoms<APC>(a, kt, nvalid) * kSfAtom, &full[st]);
       return;
     }
     uint8_t *dst = smem + st * L::kBytesP;
@@ -634,9 +648,9 @@ __device__ __forceinline__ void issue_part(const GemmArgs &a, const CUtensorMap 
         // serves -- reuse the last one.
         const int band = min(q_row0 / 128 + j, a.sf_q_rowatoms - 1);
         const uint8_t *sfq = a.sf_q + u.b * a.sf_q_bstride +
-                             (static_cast<int64_t>(band) * a.sf_katoms + kt) * kSfAtom;
-        bulk_load(smem + L::kOffSfq + st * L::kSfqBytes + j * KC * kSfAtom, sfq,
-                  nvalid * kSfAtom, &full[st]);
+                             (static_cast<int64_t>(band) * a.sf_katoms + kt * APC) * kSfAtom;
+        bulk_load(smem + L::kOffSfq + st * L::kSfqBytes + j * KC * APC * kSfAtom, sfq,
+                  stage_atoms<APC>(a, kt, nvalid) * kSfAtom, &full[st]);
       }
       return;
     }
@@ -796,7 +810,7 @@ __device__ __forceinline__ bool fused_quant_unit(const GemmArgs &a, const UnitPo
 }
 
 template <int BN, int STAGES, int ACC, bool SWAP, bool P_FP4, bool Q_FP4, int MODE, int KC,
-          bool FUSEQ = false>
+          bool FUSEQ = false, bool A4 = false>
 __global__ void __launch_bounds__(kNumThreads, 1)
     gemm_bs_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_y,
@@ -804,7 +818,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   constexpr bool CSPLIT = MODE == kSplitCluster;
   static_assert(!CSPLIT || SWAP, "cluster split-K is built for the swap-AB (decode) tiles");
   static_assert(!CSPLIT || ACC == 1, "cluster split-K uses one accumulator");
-  using L = KernelSmem<BN, STAGES, ACC, SWAP, MODE, KC>;
+  // A4: both operands packed E2M1 with E8M0 scales (kind::mxf4, K = 64 per
+  // MMA); a 128-byte chunk is 256 K and spans two scale atoms.
+  static_assert(!A4 || (!P_FP4 && !Q_FP4 && !FUSEQ), "A4 operands are plain packed bytes");
+  constexpr int APC = A4 ? 2 : 1;
+  using L = KernelSmem<BN, STAGES, ACC, SWAP, MODE, KC, APC>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -834,8 +852,10 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   // memory with one byte-slot per code but counts its packed size (half the
   // footprint).  Scale atoms are copied for the unit's chunks only.
   const int q_box_bytes = KC * a.q_box_rows * kBlockK;
-  auto tx_part = [q_box_bytes](int nv, bool p_side, bool scales) -> uint32_t {
-    if (scales) return static_cast<uint32_t>(nv * (p_side ? 1 : L::kSfqAtoms) * kSfAtom);
+  auto tx_part = [q_box_bytes, &a](int kt, int nv, bool p_side, bool scales) -> uint32_t {
+    if (scales)
+      return static_cast<uint32_t>(stage_atoms<APC>(a, kt, nv) * (p_side ? 1 : L::kSfqAtoms) *
+                                   kSfAtom);
     return p_side ? static_cast<uint32_t>(P_FP4 ? L::kBytesP / 2 : L::kBytesP)
                   : static_cast<uint32_t>(Q_FP4 ? q_box_bytes / 2 : q_box_bytes);
   };
@@ -877,8 +897,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       for (int j = 0; j < pre_n; ++j) {
         const int kt = u.kt0 + j * KC;
         const int nv = min(KC, u.kt1 - kt);
-        mbar_arrive_expect_tx(&full[j], tx_part(nv, SWAP, false));
-        issue_part<BN, L, KC>(a, &tm_p, &tm_q, smem, full, j, kt, nv, u, SWAP, false);
+        mbar_arrive_expect_tx(&full[j], tx_part(kt, nv, SWAP, false));
+        issue_part<BN, L, KC, APC>(a, &tm_p, &tm_q, smem, full, j, kt, nv, u, SWAP, false);
       }
     }
   }
@@ -925,8 +945,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             break;
           }
           const int nv = min(KC, u.kt1 - kt);
-          mbar_arrive_expect_tx(&full[stage], tx_part(nv, p_side, scales));
-          issue_part<BN, L, KC>(a, &tm_p, &tm_q, smem, full, stage, kt, nv, u, p_side, scales);
+          mbar_arrive_expect_tx(&full[stage], tx_part(kt, nv, p_side, scales));
+          issue_part<BN, L, KC, APC>(a, &tm_p, &tm_q, smem, full, stage, kt, nv, u, p_side,
+                                     scales);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
@@ -966,20 +987,40 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           const uint32_t sfq0 = smem_u32(s_sfq + stage * L::kSfqBytes);
 #pragma unroll 1
           for (int c = 0; c < nv; ++c) {
+            // TMEM scale columns of a chunk: the P side's APC atoms (4 columns
+            // each), then per atom the Q side's kSfqAtoms bands.
             const uint32_t sf_t = sf_stage + c * L::kSfColsChunk;
-            tc_cp_sf(sf_t, desc_sf_32x128b(sfp0 + c * kSfAtom));
+            const uint32_t sfq_t = sf_t + 4 * APC;
+            const int na = stage_atoms<APC>(a, kt + c, 1);
+            for (int t = 0; t < na; ++t) {
+              tc_cp_sf(sf_t + 4 * t, desc_sf_32x128b(sfp0 + (c * APC + t) * kSfAtom));
 #pragma unroll
-            for (int j = 0; j < L::kSfqAtoms; ++j)
-              tc_cp_sf(sf_t + 4 + 4 * j, desc_sf_32x128b(sfq0 + (j * KC + c) * kSfAtom));
+              for (int j = 0; j < L::kSfqAtoms; ++j)
+                tc_cp_sf(sfq_t + 4 * (t * L::kSfqAtoms + j),
+                         desc_sf_32x128b(sfq0 + (j * KC * APC + c * APC + t) * kSfAtom));
+            }
             const uint32_t pa = pa0 + c * L::kChunkP;
             const uint32_t qa = qa0 + c * q_chunk;
 #pragma unroll
             for (int ks = 0; ks < kBlockK / kMmaK; ++ks) {
-              const uint32_t idesc = make_idesc(P_FP4 ? kFmtE2M1 : kFmtE4M3,
-                                                Q_FP4 ? kFmtE2M1 : kFmtE4M3, BN, ks);
-              tc_mma_mxf8f6f4(d_tmem, desc_kmajor_sw128(pa + ks * kMmaK),
-                              desc_kmajor_sw128(qa + ks * kMmaK), idesc, sf_t,
-                              sf_t + 4 + sfq_row_off, (kt > u.kt0 || c > 0 || ks > 0) ? 1u : 0u);
+              const uint32_t acc_in = (kt > u.kt0 || c > 0 || ks > 0) ? 1u : 0u;
+              if constexpr (A4) {
+                // 64 K per MMA: atom ks / 2, scale bytes 2 (ks % 2) and 2 (ks % 2) + 1
+                const int t = ks >> 1;
+                if (t < na) {
+                  const uint32_t idesc =
+                      make_idesc(kFmtMxf4E2M1, kFmtMxf4E2M1, BN, (ks & 1) * 2);
+                  tc_mma_mxf4(d_tmem, desc_kmajor_sw128(pa + ks * kMmaK),
+                              desc_kmajor_sw128(qa + ks * kMmaK), idesc, sf_t + 4 * t,
+                              sfq_t + 4 * t * L::kSfqAtoms + sfq_row_off, acc_in);
+                }
+              } else {
+                const uint32_t idesc = make_idesc(P_FP4 ? kFmtE2M1 : kFmtE4M3,
+                                                  Q_FP4 ? kFmtE2M1 : kFmtE4M3, BN, ks);
+                tc_mma_mxf8f6f4(d_tmem, desc_kmajor_sw128(pa + ks * kMmaK),
+                                desc_kmajor_sw128(qa + ks * kMmaK), idesc, sf_t, sfq_t + sfq_row_off,
+                                acc_in);
+              }
             }
           }
           tc_commit(&empty[stage]);

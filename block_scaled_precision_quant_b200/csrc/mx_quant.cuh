@@ -12,6 +12,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <stdint.h>
 
@@ -72,6 +73,40 @@ __device__ __forceinline__ void mx_encode(const uint32_t (&w)[NW], int e,
     }
     codes[i] = e4m3x4(f[0], f[1], f[2], f[3]);
   }
+}
+
+// MXFP4 form of the quantizer (E2M1 codes): the same rule with the E2M1
+// maximum 6 in place of 448,
+//   t = fp32(amax * fp32(1/6)),  e = ceil(log2 t),  q = E2M1_RNE(clamp(x / 2^e, -6, 6)),
+// codes packed two per byte with the even element in the low nibble.
+__device__ __forceinline__ int mx_exponent_fp4(uint32_t amax_bits) {
+  const float amax = fmaxf(__uint_as_float(amax_bits << 16), 1e-4f);
+  const float t = __fmul_rn(amax, __uint_as_float(0x3E2AAAABu));  // fp32(1/6)
+  const uint32_t tb = __float_as_uint(t);
+  return static_cast<int>((tb >> 23) & 0xFFu) - 127 + ((tb & 0x7FFFFFu) != 0u ? 1 : 0);
+}
+
+// One byte of two E2M1 codes for the bf16 pair in `word` (element 2i in the
+// low half) scaled by inv = 2^-e: round to nearest even with saturation at
+// +-6 (the clamp), then each code's sign bit set from its input, so that
+// negative values that round to zero keep their sign (-0, code 8).
+__device__ __forceinline__ uint32_t e2m1x2_byte(uint32_t word, float inv) {
+  const float lo = __fmul_rn(__uint_as_float(word << 16), inv);
+  const float hi = __fmul_rn(__uint_as_float(word & 0xFFFF0000u), inv);
+  const uint32_t b = static_cast<uint32_t>(
+      __nv_cvt_float2_to_fp4x2(make_float2(lo, hi), __NV_E2M1, cudaRoundNearest));
+  return (b & 0xFFu) | ((word >> 12) & 0x8u) | ((word >> 24) & 0x80u);
+}
+
+// Packed E2M1 bytes of the 2 * NW bf16 values in w, four bytes per word.
+template <int NW>
+__device__ __forceinline__ void mx_encode_fp4(const uint32_t (&w)[NW], int e,
+                                              uint32_t (&packed)[NW / 4]) {
+  const float inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e
+#pragma unroll
+  for (int i = 0; i < NW / 4; ++i)
+    packed[i] = e2m1x2_byte(w[4 * i], inv) | (e2m1x2_byte(w[4 * i + 1], inv) << 8) |
+                (e2m1x2_byte(w[4 * i + 2], inv) << 16) | (e2m1x2_byte(w[4 * i + 3], inv) << 24);
 }
 
 }  // namespace bq

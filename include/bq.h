@@ -100,6 +100,20 @@ size_t bq_sf_bytes(int64_t rows, int64_t K);
 int bq_act_quant(const void *x_bf16, int64_t M, int64_t K, int64_t ldx, void *q_e4m3,
                  void *sf_mma, void *sf_rowmajor, int *d_status, bq_stream_t stream);
 
+/* bq_act_quant_mxfp4 -- per-32 MXFP4 quantization of bf16 activations, for the
+ * FP4 x FP4 GEMM (the A4W4 kernels of the "fp4-gemm" page, README "Available
+ * Functions" and "Tensor Contract": packed E2M1 activations with block
+ * scales).  The pages define the per-32 rule for E4M3 codes (bq_act_quant);
+ * for E2M1 codes the same rule takes the format's largest value 6 in place of
+ * 448: t = fp32(amax * fp32(1/6)), e = ceil(log2 t), scale byte = e + 127,
+ * q = E2M1 round-to-nearest-even of clamp(x / 2^e, -6, 6), the sign kept
+ * (negative values that round to zero give code 8, -0).  Two codes per byte,
+ * the even element in the low nibble (the pages' MXFP4 weight layout).
+ *   q_fp4  out [M, K/2] packed E2M1 codes, row stride K/2 bytes, 16-byte aligned
+ *   all other arguments and errors as bq_act_quant. */
+int bq_act_quant_mxfp4(const void *x_bf16, int64_t M, int64_t K, int64_t ldx, void *q_fp4,
+                       void *sf_mma, void *sf_rowmajor, int *d_status, bq_stream_t stream);
+
 /* ---- weight scale prepack (off the hot path) --------------------------- */
 
 enum {
@@ -156,6 +170,21 @@ int bq_gemm_mxfp8_fp8blk32(const void *a_q, const void *a_sf, const void *b_e4m3
                            const void *b_sf, int64_t M, int64_t N, int64_t K, void *y_bf16,
                            bq_stream_t stream);
 int bq_gemm_mxfp8_mxfp8(const void *a_q, const void *a_sf, const void *b_e4m3, const void *b_sf,
+                        int64_t M, int64_t N, int64_t K, void *y_bf16, bq_stream_t stream);
+
+/* bq_gemm_mxfp4_mxfp4 -- the FP4 x FP4 (A4W4) product ("fp4-gemm" page,
+ * README "Available Functions": the bf16-output A4W4 GEMM; "Tensor
+ * Contract": a_packed [M, K/2], b_packed [N, K/2], scale buffers in the MMA
+ * layout, bf16 [M, N] out) with E8M0 scales per 32 inputs on both sides
+ * (MXFP4), on tcgen05.mma kind::mxf4:
+ *   a_fp4  [M, K/2] packed E2M1 activation codes (bq_act_quant_mxfp4), 16-byte aligned
+ *   a_sf   MMA-layout scales of A (bq_act_quant_mxfp4), bq_sf_bytes(M, K)
+ *   b_fp4  [N, K/2] packed E2M1 weight codes, low nibble = even input, 16-byte aligned
+ *   b_sf   bq_pack_weight_scales(BQ_SF_ROW32) of the [N, K/32] weight scales
+ * K % 128 == 0; everything else (y, errors, stream order) as the GEMMs above.
+ * The pages' A4W4 kernels use NVFP4 (E4M3 scales per 16 inputs); that scale
+ * format is not implemented here. */
+int bq_gemm_mxfp4_mxfp4(const void *a_fp4, const void *a_sf, const void *b_fp4, const void *b_sf,
                         int64_t M, int64_t N, int64_t K, void *y_bf16, bq_stream_t stream);
 
 enum { BQ_ACT_NONE = 0, BQ_ACT_GELU = 1 };
@@ -228,20 +257,23 @@ typedef struct {
 } bq_gemm_config;
 
 /* Workspace bytes the *_epilogue calls need for a problem (0 when the chosen
- * schedule needs none).  weight_kind: 0 mxfp4, 1 fp8blk32, 2 mxfp8. */
+ * schedule needs none).  weight_kind: 0 mxfp4, 1 fp8blk32, 2 mxfp8, 3 mxfp4 weights
+ * with MXFP4 activations (bq_gemm_mxfp4_mxfp4*). */
 size_t bq_gemm_workspace_bytes(int weight_kind, int64_t M, int64_t N, int64_t K, int64_t batch,
                                const bq_gemm_config *cfg);
 
-/* The schedule the built-in dispatch picks for a problem on a device with
- * `num_sms` SMs, with `cfg` (NULL = all auto) as a *_epilogue call would get
- * it: every field of *out resolved (block_n, split_k >= 1, swap_ab 0/1,
+/* The schedule the built-in dispatch picks for a problem of weight_kind (as
+ * for bq_gemm_workspace_bytes) on a device with `num_sms` SMs, with `cfg`
+ * (NULL = all auto) as a *_epilogue call would get it: every field of *out
+ * resolved (block_n, split_k >= 1, swap_ab 0/1,
  * split_mode BQ_SPLIT_WORKSPACE or BQ_SPLIT_CLUSTER when split_k > 1, else
  * BQ_SPLIT_AUTO, k_chunks >= 1, cta_pair 1 or 2).  Host-only: touches no
  * device.  Calls that ask for a quantized output run unsplit.  Returns
  * BQ_ERR_NULL (out NULL), BQ_ERR_SHAPE (sizes out of range, num_sms < 1) or
- * BQ_ERR_INVALID (cfg not schedulable, the status the GEMM call returns). */
-int bq_gemm_plan(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_config *cfg,
-                 int num_sms, bq_gemm_config *out);
+ * BQ_ERR_INVALID (weight_kind or cfg not schedulable, the status the GEMM call
+ * returns).  MXFP4 activations (weight_kind 3) have no pair tiles. */
+int bq_gemm_plan(int weight_kind, int64_t M, int64_t N, int64_t K, int64_t batch,
+                 const bq_gemm_config *cfg, int num_sms, bq_gemm_config *out);
 
 /* GEMM + fused epilogue (+ optional batch).  epi NULL = plain (alpha 1, no
  * bias, residual or activation).  batch NULL = one problem.  workspace: device
@@ -262,6 +294,13 @@ int bq_gemm_mxfp8_fp8blk32_epilogue(const void *a_q, const void *a_sf, const voi
                                     void *workspace, size_t workspace_bytes,
                                     const bq_gemm_config *cfg, bq_stream_t stream);
 int bq_gemm_mxfp8_mxfp8_epilogue(const void *a_q, const void *a_sf, const void *b_e4m3,
+                                 const void *b_sf, int64_t M, int64_t N, int64_t K, void *y_bf16,
+                                 const bq_epilogue *epi, const bq_batch *batch, void *workspace,
+                                 size_t workspace_bytes, const bq_gemm_config *cfg,
+                                 bq_stream_t stream);
+/* A4W4 (bq_gemm_mxfp4_mxfp4) with the same epilogue, batch, workspace and
+ * schedule options; cta_pair 2 is refused (BQ_ERR_INVALID). */
+int bq_gemm_mxfp4_mxfp4_epilogue(const void *a_fp4, const void *a_sf, const void *b_fp4,
                                  const void *b_sf, int64_t M, int64_t N, int64_t K, void *y_bf16,
                                  const bq_epilogue *epi, const bq_batch *batch, void *workspace,
                                  size_t workspace_bytes, const bq_gemm_config *cfg,
