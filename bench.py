@@ -639,11 +639,17 @@ def run_ours(args, spec, world, rank, local, device):
     tensor_ratio = 4.0 if a4 else 2.0
     fp8_peak = tensor_ratio * peaks[tensor_kind]
     gemm_launches = len(layers_spec)
+    # the GEMM kernel(s) the built-in dispatch runs for these layers
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    kernels = sorted({("gemm_pair_kernel" if bq.plan(sp[2], sp[3], sp[4], sp[5], num_sms=sms,
+                                                     weight_kind=WKIND[sp[1]]).cta_pair == 2
+                       else "gemm_bs_kernel") for sp in layers_spec})
+    kernel_name = "+".join(kernels)
     if spec["bound"] == "hbm":
         achieved = gbytes_step / (gemm_ms_step * 1e-3) / 1e9
         roof = dict(bound="hbm", achieved=round(achieved, 1), peak=peaks["hbm"], unit="GB/s",
                     frac=round(achieved / peaks["hbm"], 4), traffic=stored_traffic(args.workload),
-                    kernel="gemm_bs_kernel", algorithmic_bytes_per_launch=gbytes_step / gemm_launches,
+                    kernel=kernel_name, algorithmic_bytes_per_launch=gbytes_step / gemm_launches,
                     avg_launch_us=round(gemm_ms_step * 1e3 / gemm_launches, 3),
                     peak_source=f"{peaks['src']} hbm_gbs (burst)")
     else:
@@ -651,7 +657,7 @@ def run_ours(args, spec, world, rank, local, device):
         roof = dict(bound="tensor", achieved=round(achieved, 1), peak=round(fp8_peak, 1),
                     unit="TFLOP/s", frac=round(achieved / fp8_peak, 4),
                     traffic=stored_traffic(args.workload),
-                    kernel="gemm_bs_kernel", flops_per_launch=flops_step / gemm_launches,
+                    kernel=kernel_name, flops_per_launch=flops_step / gemm_launches,
                     avg_launch_us=round(gemm_ms_step * 1e3 / gemm_launches, 3),
                     peak_source=(f"{peaks['src']} {'bf16_tflops_sustained' if tensor_kind != 'bf16' else 'bf16_tflops'}"
                                  f" x {tensor_ratio:g} (nominal "
