@@ -27,7 +27,8 @@ _lib = None
 
 OK, ERR_NAN_SCALE, ERR_NAN_CODE, ERR_SHAPE, ERR_NONFINITE = 0, -1, -2, -3, -4
 B_FP4, B_FP8BLK, B_FP8ROW = 0, 1, 2
-A_E4M3, A_FP4 = 0, 1
+A_E4M3, A_FP4, A_E5M2 = 0, 1, 2
+Q_E4M3, Q_E5M2 = 0, 1  # code formats of the transposed quantizer
 ACT_NONE, ACT_GELU = 0, 1
 
 CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
@@ -90,6 +91,25 @@ def _load():
     lib.oracle_act_quant_fp4.restype = ctypes.c_int
     lib.oracle_act_quant_fp4_f32.argtypes = [f32p, i64, i64, u8p, u8p]
     lib.oracle_act_quant_fp4_f32.restype = ctypes.c_int
+    u64 = ctypes.c_uint64
+    u64p = ctypes.POINTER(ctypes.c_uint64)
+    lib.oracle_decode_e5m2.argtypes = [ctypes.c_uint8, f64p]
+    lib.oracle_decode_e5m2.restype = ctypes.c_int
+    lib.oracle_encode_e5m2.argtypes = [ctypes.c_float]
+    lib.oracle_encode_e5m2.restype = ctypes.c_uint8
+    lib.oracle_encode_e5m2_n.argtypes = [f32p, i64, u8p]
+    lib.oracle_encode_e5m2_n.restype = None
+    lib.oracle_encode_e5m2_sr.argtypes = [ctypes.c_float, ctypes.c_double]
+    lib.oracle_encode_e5m2_sr.restype = ctypes.c_uint8
+    lib.oracle_philox4x64_10.argtypes = [u64p, u64p, u64p]
+    lib.oracle_philox4x64_10.restype = None
+    lib.oracle_uniform.argtypes = [u64, u64]
+    lib.oracle_uniform.restype = ctypes.c_double
+    lib.oracle_grad_quant.argtypes = [u16p, i64, i64, i64, ctypes.c_int, u64, u8p, u8p]
+    lib.oracle_grad_quant.restype = ctypes.c_int
+    lib.oracle_quant_transposed.argtypes = [u16p, i64, i64, i64, ctypes.c_int, ctypes.c_int, u64,
+                                            u8p, u8p]
+    lib.oracle_quant_transposed.restype = ctypes.c_int
     lib.oracle_gemm_ex.argtypes = [u8p, u8p, ctypes.c_int, u8p, u8p, ctypes.c_int, i64, i64, i64,
                                    u16p, u16p, i64, ctypes.c_double, ctypes.c_int, f64p, f64p,
                                    ctypes.c_int]
@@ -171,6 +191,79 @@ def encode_fp4_array(v: np.ndarray) -> np.ndarray:
     out = np.empty(v.shape, dtype=np.uint8)
     _load().oracle_encode_fp4_n(_ptr(v, ctypes.c_float), v.size, _ptr(out, ctypes.c_uint8))
     return out
+
+
+def decode_e5m2(b: int) -> float:
+    """E5M2 byte -> value (bias 15, 2 mantissa bits); Inf / NaN codes refused."""
+    out = ctypes.c_double()
+    _check(_load().oracle_decode_e5m2(int(b), ctypes.byref(out)), "decode_e5m2")
+    return out.value
+
+
+def encode_e5m2(v: float) -> int:
+    """binary32 -> E5M2 byte, round to nearest even, saturating at +-57344."""
+    return int(_load().oracle_encode_e5m2(float(v)))
+
+
+def encode_e5m2_array(v: np.ndarray) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.empty(v.shape, dtype=np.uint8)
+    _load().oracle_encode_e5m2_n(_ptr(v, ctypes.c_float), v.size, _ptr(out, ctypes.c_uint8))
+    return out
+
+
+def encode_e5m2_sr(v: float, u: float) -> int:
+    """Stochastic E5M2 rounding of v with the uniform draw u in [0, 1): the
+    upper neighbour when u < (|v| - lo) / (hi - lo)."""
+    return int(_load().oracle_encode_e5m2_sr(float(v), float(u)))
+
+
+def philox4x64_10(ctr, key):
+    """Philox4x64-10 of a 4-word counter under a 2-word key (4 uint64 words)."""
+    c = np.ascontiguousarray(ctr, dtype=np.uint64)
+    k = np.ascontiguousarray(key, dtype=np.uint64)
+    out = np.empty(4, dtype=np.uint64)
+    _load().oracle_philox4x64_10(_ptr(c, ctypes.c_uint64), _ptr(k, ctypes.c_uint64),
+                                 _ptr(out, ctypes.c_uint64))
+    return out
+
+
+def uniform(seed: int, index: int) -> float:
+    """The stochastic-rounding draw of element `index` under `seed`."""
+    return _load().oracle_uniform(int(seed), int(index))
+
+
+def grad_quant(x_bf16_bits: np.ndarray, stochastic=False, seed=0):
+    """Per-32 E5M2 gradient quantization along the last dimension ("hip_quant"
+    README: "Stochastic E5M2 Backward Gradients", "Block-wise FP8 Scaling"; the
+    scale rule of the formats.py page with 57344 in place of 448).
+    Returns (q uint8 [M, K] E5M2 codes, sf uint8 [M, K/32] E8M0 bytes)."""
+    x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
+    M, K = x.shape
+    q = np.empty((M, K), dtype=np.uint8)
+    sf = np.empty((M, K // 32), dtype=np.uint8)
+    if M:
+        _check(_load().oracle_grad_quant(_ptr(x, ctypes.c_uint16), M, K, K, int(bool(stochastic)),
+                                         int(seed), _ptr(q, ctypes.c_uint8),
+                                         _ptr(sf, ctypes.c_uint8)), "grad_quant")
+    return q, sf
+
+
+def quant_transposed(x_bf16_bits: np.ndarray, fmt=Q_E4M3, stochastic=False, seed=0):
+    """Quantization along the FIRST dimension of x [R, C] (per 32 rows of a
+    column), written transposed: (q uint8 [C, R], sf uint8 [C, R/32]).  fmt
+    Q_E4M3 (the act_quant rule) or Q_E5M2 (the gradient rule; its stochastic
+    draws use the element's index r * C + c in x)."""
+    x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
+    R, C = x.shape
+    q = np.empty((C, R), dtype=np.uint8)
+    sf = np.empty((C, R // 32), dtype=np.uint8)
+    if C:
+        _check(_load().oracle_quant_transposed(_ptr(x, ctypes.c_uint16), R, C, C, int(fmt),
+                                               int(bool(stochastic)), int(seed),
+                                               _ptr(q, ctypes.c_uint8), _ptr(sf, ctypes.c_uint8)),
+               "quant_transposed")
+    return q, sf
 
 
 def f32_to_bf16_bits(v: float) -> int:
@@ -273,7 +366,8 @@ def gemm(aq, asf, b, bsf, bkind, M, N, K, bias=None, residual=None, alpha=1.0,
     ref[m, n] = act(alpha * sum_k a[m,k] b[n,k] + bias[n]) + residual[m, n] and
     sumabs[m, n] = sum_k |a[m,k] b[n,k]|, where a and b are the exactly decoded
     operands (formats.py page: decode_fp4, decode_fp8_block, e8m0_to_f32).
-    a_kind: A_E4M3 (aq [M, K]) or A_FP4 (aq [M, K/2] packed E2M1)."""
+    a_kind: A_E4M3 (aq [M, K]), A_FP4 (aq [M, K/2] packed E2M1) or A_E5M2
+    (aq [M, K] E5M2 gradient codes)."""
     aq = np.ascontiguousarray(aq, dtype=np.uint8)
     asf = np.ascontiguousarray(asf, dtype=np.uint8)
     b = np.ascontiguousarray(b, dtype=np.uint8)

@@ -20,7 +20,15 @@
  *     of the "fp4-gemm" page, README "Available Functions") is not spelled
  *     out on the pages: it is the same per-32 rule with the E2M1 format's
  *     largest value 6 in place of 448, and E2M1 codes packed two per byte with
- *     the even element in the low nibble (the pages' MXFP4 weight layout).
+ *     the even element in the low nibble (the pages' MXFP4 weight layout);
+ *   - the gradient quantizer of the backward pass (E5M2 codes, the pages'
+ *     "hip_quant" README, "Stochastic E5M2 Backward Gradients" and "Block-wise
+ *     FP8 Scaling") takes the same per-32 rule with E5M2's largest finite
+ *     value 57344, rounding to nearest even or stochastically between the two
+ *     neighbouring E5M2 values; the stochastic draw comes from a counter-based
+ *     generator (Philox4x64-10) keyed by the seed and counted by the element's
+ *     index, the "stateless per-element hash of (seed, element_index)" the page
+ *     describes.
  *
  * Floating point: compile with -ffp-contract=off and without fast-math so that
  * every float expression below is one IEEE binary32 operation, as the page's
@@ -145,6 +153,111 @@ uint8_t oracle_encode_fp4(float v) {
 
 void oracle_encode_fp4_n(const float *v, int64_t n, uint8_t *out) {
   for (int64_t i = 0; i < n; ++i) out[i] = oracle_encode_fp4(v[i]);
+}
+
+/* E5M2: bias 15, two mantissa bits, exponent field 31 is Inf / NaN (refused
+ * here: the quantizer never produces them).  Normal: (-1)^s 2^(E-15) (1 + m/4);
+ * subnormal (E = 0): (-1)^s 2^-14 (m/4).  Largest finite 0x7B = 57344. */
+int oracle_decode_e5m2(uint8_t b, double *out) {
+  int s = b >> 7;
+  int E = (b >> 2) & 0x1F;
+  int m = b & 3;
+  if (E == 31) return ORACLE_ERR_NAN_CODE;
+  double mag = (E == 0) ? ldexp(m / 4.0, -14) : ldexp(1.0 + m / 4.0, E - 15);
+  *out = s ? -mag : mag;
+  return ORACLE_OK;
+}
+
+/* The 124 non-negative finite E5M2 magnitudes, codes 0x00..0x7B, increasing. */
+static double e5m2_mag[124];
+static int e5m2_mag_ready = 0;
+static void e5m2_table_init(void) {
+  if (e5m2_mag_ready) return;
+  for (int c = 0; c < 124; ++c) oracle_decode_e5m2((uint8_t)c, &e5m2_mag[c]);
+  e5m2_mag_ready = 1;
+}
+
+/* Index of the largest finite E5M2 magnitude <= a (a >= 0, below the top). */
+static int e5m2_floor_code(double a) {
+  int lo = 0, hi = 123; /* mag[lo] <= a < mag[hi] */
+  while (hi - lo > 1) {
+    int mid = (lo + hi) / 2;
+    if (e5m2_mag[mid] <= a) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+/* binary32 -> E5M2, round to nearest even, saturating at +-57344, sign kept. */
+uint8_t oracle_encode_e5m2(float v) {
+  e5m2_table_init();
+  uint8_t sign = signbit(v) ? 0x80 : 0x00;
+  double a = fabs((double)v);
+  uint8_t code;
+  if (a >= e5m2_mag[123]) {
+    code = 123;
+  } else {
+    int lo = e5m2_floor_code(a), hi = lo + 1;
+    double dlo = a - e5m2_mag[lo], dhi = e5m2_mag[hi] - a;
+    if (dlo < dhi) code = (uint8_t)lo;
+    else if (dhi < dlo) code = (uint8_t)hi;
+    else code = (uint8_t)((lo % 2 == 0) ? lo : hi);
+  }
+  return (uint8_t)(sign | code);
+}
+
+void oracle_encode_e5m2_n(const float *v, int64_t n, uint8_t *out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = oracle_encode_e5m2(v[i]);
+}
+
+/* Philox4x64-10 (Salmon, Moraes, Dror and Shaw, "Parallel random numbers: as
+ * easy as 1, 2, 3", SC 2011): ten rounds of two 64 x 64 -> 128-bit
+ * multiplications on a 4-word counter, the 2-word key bumped by the Weyl
+ * constants between rounds. */
+static void mulhilo64(uint64_t a, uint64_t b, uint64_t *hi, uint64_t *lo) {
+  unsigned __int128 p = (unsigned __int128)a * (unsigned __int128)b;
+  *hi = (uint64_t)(p >> 64);
+  *lo = (uint64_t)p;
+}
+
+void oracle_philox4x64_10(const uint64_t ctr[4], const uint64_t key[2], uint64_t out[4]) {
+  const uint64_t M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
+  const uint64_t W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
+  uint64_t x0 = ctr[0], x1 = ctr[1], x2 = ctr[2], x3 = ctr[3];
+  uint64_t k0 = key[0], k1 = key[1];
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k0 += W0;
+      k1 += W1;
+    }
+    uint64_t hi0, lo0, hi1, lo1;
+    mulhilo64(M0, x0, &hi0, &lo0);
+    mulhilo64(M1, x2, &hi1, &lo1);
+    uint64_t y0 = hi1 ^ x1 ^ k0, y1 = lo1, y2 = hi0 ^ x3 ^ k1, y3 = lo0;
+    x0 = y0; x1 = y1; x2 = y2; x3 = y3;
+  }
+  out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
+}
+
+/* The uniform draw of element `index` under `seed`: word (index % 4) of
+ * Philox4x64-10 at counter (index / 4, 0, 0, 0) with key (seed, 0), its top
+ * 53 bits as a double in [0, 1). */
+double oracle_uniform(uint64_t seed, uint64_t index) {
+  uint64_t ctr[4] = {index >> 2, 0, 0, 0}, key[2] = {seed, 0}, out[4];
+  oracle_philox4x64_10(ctr, key, out);
+  return ldexp((double)(out[index & 3] >> 11), -53);
+}
+
+/* Stochastic E5M2 rounding of binary32 v (|v| <= 57344 after the clamp):
+ * lo and hi are the neighbouring E5M2 magnitudes around |v|; the result is hi
+ * when u < (|v| - lo) / (hi - lo) (exact in double), else lo; sign kept. */
+uint8_t oracle_encode_e5m2_sr(float v, double u) {
+  e5m2_table_init();
+  uint8_t sign = signbit(v) ? 0x80 : 0x00;
+  double a = fabs((double)v);
+  if (a >= e5m2_mag[123]) return (uint8_t)(sign | 123);
+  int lo = e5m2_floor_code(a);
+  double d = (a - e5m2_mag[lo]) / (e5m2_mag[lo + 1] - e5m2_mag[lo]);
+  return (uint8_t)(sign | (u < d ? lo + 1 : lo));
 }
 
 static float bf16_to_f32(uint16_t h) {
@@ -323,6 +436,94 @@ int oracle_act_quant_fp4_f32(const float *x, int64_t M, int64_t K, uint8_t *q, u
   return ORACLE_OK;
 }
 
+/* Gradient quantization, E5M2 codes: the per-32 rule with E5M2's largest
+ * finite value 57344 in place of 448,
+ *   t = fp32(max(amax, 1e-4) * fp32(1/57344)),  e = ceil(log2 t),
+ *   q = E5M2(clamp(x / 2^e, -57344, 57344)), round to nearest even, or
+ *       stochastic with the uniform draw of the element's index (sr != 0),
+ * for the 32 values x[i * stride] whose source indices are idx0 + i * istride.
+ * Writes one code per element to q[i * qstride]; returns the scale byte or -1
+ * for a NaN / Inf. */
+static int grad_quant_group(const float *x, int64_t stride, uint8_t *q, int64_t qstride,
+                            int sr, uint64_t seed, uint64_t idx0, uint64_t istride) {
+  float amax = 0.0f;
+  for (int i = 0; i < BLOCK; ++i) {
+    float v = x[i * stride];
+    if (!isfinite(v)) return -1;
+    float av = fabsf(v);
+    if (av > amax) amax = av;
+  }
+  const float floor_ = 1e-4f;
+  if (amax < floor_) amax = floor_;
+  const float inv = (float)(1.0 / 57344.0);
+  float t = amax * inv;
+  uint32_t bits;
+  memcpy(&bits, &t, 4);
+  int e = (int)((bits >> 23) & 0xFF) - 127 + ((bits & 0x7FFFFF) != 0 ? 1 : 0);
+  float s = ldexpf(1.0f, e);
+  for (int i = 0; i < BLOCK; ++i) {
+    float y = x[i * stride] / s;
+    if (y > 57344.0f) y = 57344.0f;
+    if (y < -57344.0f) y = -57344.0f;
+    q[i * qstride] = sr ? oracle_encode_e5m2_sr(y, oracle_uniform(seed, idx0 + i * istride))
+                        : oracle_encode_e5m2(y);
+  }
+  return e + 127;
+}
+
+/* The E4M3 rule of act_quant_group on a strided group (for the transposed
+ * activation operand of the weight gradient). */
+static int e4m3_quant_group_strided(const float *x, int64_t stride, uint8_t *q, int64_t qstride) {
+  float buf[BLOCK];
+  uint8_t codes[BLOCK];
+  for (int i = 0; i < BLOCK; ++i) buf[i] = x[i * stride];
+  int b = act_quant_group(buf, codes);
+  if (b < 0) return -1;
+  for (int i = 0; i < BLOCK; ++i) q[i * qstride] = codes[i];
+  return b;
+}
+
+/* Row-wise gradient quantization: x bf16 [M, ldx] -> q [M, K] E5M2, sf
+ * [M, K/32].  Element (m, k) has index m * K + k. */
+int oracle_grad_quant(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, int sr,
+                      uint64_t seed, uint8_t *q, uint8_t *sf) {
+  if (K <= 0 || K % BLOCK) return ORACLE_ERR_SHAPE;
+  const int64_t G = K / BLOCK;
+  float buf[BLOCK];
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t g = 0; g < G; ++g) {
+      for (int i = 0; i < BLOCK; ++i) buf[i] = bf16_to_f32(x[m * ldx + g * BLOCK + i]);
+      int b = grad_quant_group(buf, 1, q + m * K + g * BLOCK, 1, sr, seed,
+                               (uint64_t)(m * K + g * BLOCK), 1);
+      if (b < 0) return ORACLE_ERR_NONFINITE;
+      sf[m * G + g] = (uint8_t)b;
+    }
+  return ORACLE_OK;
+}
+
+/* Transposed quantization: x bf16 [R, ldx] (C columns used) quantized along
+ * R, per 32 consecutive rows of one column, written transposed: q [C, R],
+ * sf [C, R/32].  fmt 0: E4M3 (the act_quant rule), 1: E5M2 (the gradient
+ * rule; element (r, c) has index r * C + c).  This is the quantization of the
+ * transposed matrix by the row-wise rule. */
+int oracle_quant_transposed(const uint16_t *x, int64_t R, int64_t C, int64_t ldx, int fmt,
+                            int sr, uint64_t seed, uint8_t *q, uint8_t *sf) {
+  if (R <= 0 || R % BLOCK || C < 0 || fmt < 0 || fmt > 1 || (sr && fmt != 1))
+    return ORACLE_ERR_SHAPE;
+  const int64_t G = R / BLOCK;
+  float col[BLOCK];
+  for (int64_t c = 0; c < C; ++c)
+    for (int64_t g = 0; g < G; ++g) {
+      for (int i = 0; i < BLOCK; ++i) col[i] = bf16_to_f32(x[(g * BLOCK + i) * ldx + c]);
+      int b = fmt == 1 ? grad_quant_group(col, 1, q + c * R + g * BLOCK, 1, sr, seed,
+                                          (uint64_t)(g * BLOCK * C + c), (uint64_t)C)
+                       : e4m3_quant_group_strided(col, 1, q + c * R + g * BLOCK, 1);
+      if (b < 0) return ORACLE_ERR_NONFINITE;
+      sf[c * G + g] = (uint8_t)b;
+    }
+  return ORACLE_OK;
+}
+
 /* ------------------------------------------------------------------ */
 /* Exact operand decode + fp64 GEMM with the fused epilogue.            */
 /* ------------------------------------------------------------------ */
@@ -335,6 +536,7 @@ int oracle_act_quant_fp4_f32(const float *x, int64_t M, int64_t K, uint8_t *q, u
 /* Activation kinds. */
 #define ORACLE_A_E4M3 0 /* E4M3 [M, K]; scales [M, K/32] */
 #define ORACLE_A_FP4 1  /* E2M1 packed [M, K/2], low nibble = even k; scales [M, K/32] */
+#define ORACLE_A_E5M2 2 /* E5M2 [M, K] (gradients); scales [M, K/32] */
 
 #define ORACLE_ACT_NONE 0
 #define ORACLE_ACT_GELU 1
@@ -365,6 +567,8 @@ static int dec_a(const gemm_job *J, int64_t m, int64_t k, double *v) {
   if (J->akind == ORACLE_A_FP4) {
     uint8_t byte = J->aq[m * (J->K / 2) + k / 2];
     c = oracle_decode_fp4((k % 2 == 0) ? (byte & 0x0F) : (byte >> 4));
+  } else if (J->akind == ORACLE_A_E5M2) {
+    if (oracle_decode_e5m2(J->aq[m * J->K + k], &c)) return ORACLE_ERR_NAN_CODE;
   } else if (oracle_decode_e4m3(J->aq[m * J->K + k], &c)) {
     return ORACLE_ERR_NAN_CODE;
   }
@@ -474,7 +678,7 @@ int oracle_gemm_ex(const uint8_t *aq, const uint8_t *asf, int akind, const uint8
                    const uint8_t *bsf, int bkind, int64_t M, int64_t N, int64_t K,
                    const uint16_t *bias, const uint16_t *residual, int64_t ld_res, double alpha,
                    int act, double *ref, double *sumabs, int nthreads) {
-  if (K <= 0 || K % BLOCK || bkind < 0 || bkind > 2 || akind < 0 || akind > 1)
+  if (K <= 0 || K % BLOCK || bkind < 0 || bkind > 2 || akind < 0 || akind > 2)
     return ORACLE_ERR_SHAPE;
   gemm_job J = {aq, asf, b, bsf, akind, bkind, M, N, K, bias, residual, ld_res, alpha, act,
                 ref, sumabs, NULL, NULL, 0, 0, 0, 0};
@@ -495,7 +699,7 @@ int oracle_gemm_sampled_ex(const uint8_t *aq, const uint8_t *asf, int akind, con
                            const uint16_t *bias, const uint16_t *residual, int64_t ld_res,
                            double alpha, int act, const int64_t *ms, const int64_t *ns,
                            int64_t count, double *ref, double *sumabs, int nthreads) {
-  if (K <= 0 || K % BLOCK || bkind < 0 || bkind > 2 || akind < 0 || akind > 1)
+  if (K <= 0 || K % BLOCK || bkind < 0 || bkind > 2 || akind < 0 || akind > 2)
     return ORACLE_ERR_SHAPE;
   gemm_job J = {aq, asf, b, bsf, akind, bkind, M, N, K, bias, residual, ld_res, alpha, act,
                 ref, sumabs, ms, ns, count, 0, 0, 0};
