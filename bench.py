@@ -72,22 +72,44 @@ WORKLOADS = {
         desc="square MXFP4xMXFP4 GEMM M=N=K=8192 (activations act_quant_mxfp4'd per step, "
              "MXFP4 weights)",
         layers=[("square", "a4w4", 8192, 8192, 8192, 1, dict())], bound="tensor"),
+    # Backward of one linear layer y = x W^T (x [T, K], W [N, K]): the output
+    # gradient dY [T, N] quantized to E5M2 with stochastic rounding along N
+    # (for dX) and along T (for dW), x and the bf16 master weight W quantized
+    # along T and along N (transposed quantizers), then dX = dY W [T, K] and
+    # dW = dY^T x [N, K] on E5M2 x MXFP8 GEMMs.  Shape: the MLP workload's
+    # down-projection, T = 4096 tokens, N = 1536, K = 6144.
+    "backward": dict(
+        desc="backward of a 4096x1536x6144 linear layer: E5M2 stochastic gradient quantization "
+             "(row-wise and transposed), transposed E4M3 quantization of x and W, "
+             "dX = dY W and dW = dY^T x on E5M2 x MXFP8 GEMMs",
+        layers=[("bwd", "grad", 4096, 1536, 6144, 1, dict())], bound="tensor"),
 }
 
-WKIND = {"mxfp4": 0, "fp8blk32": 1, "mxfp8": 2, "a4w4": 3}
+WKIND = {"mxfp4": 0, "fp8blk32": 1, "mxfp8": 2, "a4w4": 3, "grad": 4}
 DTYPE = {"mxfp4": "mxfp8xmxfp4", "fp8blk32": "mxfp8xfp8blk32", "mxfp8": "mxfp8xmxfp8",
-         "a4w4": "mxfp4xmxfp4"}
+         "a4w4": "mxfp4xmxfp4", "grad": "e5m2xmxfp8"}
+
+
+def gemm_shapes(layer):
+    """(M, N, K, batch) of each GEMM launch of a layer: the backward layer
+    runs dX = dY W ([T, K], contraction N) and dW = dY^T x ([N, K], over T)."""
+    _, wk, M, N, K, B, _ = layer
+    if wk == "grad":
+        return [(M, K, N, 1), (N, K, M, 1)]
+    return [(M, N, K, B)]
 
 
 def gemm_flops(layer):
-    _, _, M, N, K, B, _ = layer
-    return 2.0 * M * N * K * B
+    _, wk, M, N, K, B, _ = layer
+    return (4.0 if wk == "grad" else 2.0) * M * N * K * B  # backward: dX and dW
 
 
 def act_quant_bytes(layer):
     """Algorithmic bytes of act_quant: read 2 B/elem, write 1 + 1/32 B/elem
     (E4M3 codes) or 1/2 + 1/32 B/elem (packed E2M1 codes)."""
-    _, wk, M, _, K, B, _ = layer
+    _, wk, M, N, K, B, _ = layer
+    if wk == "grad":  # dY twice (row-wise, transposed), x^T and W^T
+        return (2.0 + 1.0 + 1.0 / 32.0) * (2 * M * N + M * K + N * K)
     code = 0.5 if wk == "a4w4" else 1.0
     return (2.0 + code + 1.0 / 32.0) * M * K * B
 
@@ -97,6 +119,9 @@ def gemm_bytes(layer, quant_out=False):
     output written once (weights counted once when broadcast over a batch);
     a quantized output is 1 + 1/32 bytes per element instead of 2."""
     _, wk, M, N, K, B, ex = layer
+    if wk == "grad":  # dX: dY codes [M, N] x W^T codes [K, N]; dW: dY^T [N, M] x x^T [K, M]
+        code = 1.0 + 1.0 / 32.0
+        return code * (M * N + K * N) + 2.0 * M * K + code * (N * M + K * M) + 2.0 * N * K
     w = N * K / 2.0 if wk in ("mxfp4", "a4w4") else float(N * K)
     w += N * K / 32.0  # weight scales
     a = B * (M * K * (0.5 if wk == "a4w4" else 1.0) + M * K / 32.0)
@@ -354,6 +379,75 @@ class Layer:
         return n
 
 
+class BackwardLayer:
+    """Device buffers of the backward of one linear layer (T tokens, N
+    outputs, K inputs), with `sets` rotating copies of x, W and dY.  Same
+    interface as Layer: launches(s, which) issues the quantizers ("act_quant")
+    and the two GEMMs ("gemm"); y is dX (the step's result passed on)."""
+
+    def __init__(self, spec, sets, seed, device, **_):
+        import torch
+        import block_scaled_precision_quant_b200 as bq
+        from block_scaled_precision_quant_b200 import synth
+        self.spec = spec
+        name, wk, T, N, K, B, ex = spec
+        self.T, self.N, self.K = T, N, K
+        self.wk = WKIND[wk]
+        self.quant_out = False
+        self.qy = None
+
+        def bf16(bits):
+            return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(device)
+        self.sets = []
+        for s in range(sets):
+            sd = seed + 1000 * s
+            self.sets.append(dict(
+                x=bf16(synth.activations(T, N, seed=sd + 2, group_pow2=(-20, 4))),  # dY
+                xin=bf16(synth.activations(T, K, seed=sd)),
+                w=bf16(synth.activations(N, K, seed=sd + 1, std=0.05))))
+        u8 = dict(dtype=torch.uint8, device=device)
+        self.gq, self.gsf = torch.empty((T, N), **u8), torch.empty((bq.sf_bytes(T, N),), **u8)
+        self.wtq, self.wtsf = torch.empty((K, N), **u8), torch.empty((bq.sf_bytes(K, N),), **u8)
+        self.gtq, self.gtsf = torch.empty((N, T), **u8), torch.empty((bq.sf_bytes(N, T),), **u8)
+        self.xtq, self.xtsf = torch.empty((K, T), **u8), torch.empty((bq.sf_bytes(K, T),), **u8)
+        self.y = torch.empty((T, K), dtype=torch.bfloat16, device=device)   # dX
+        self.dw = torch.empty((N, K), dtype=torch.bfloat16, device=device)
+        self.need = max(bq.workspace_bytes(self.wk, T, K, N, 1),
+                        bq.workspace_bytes(self.wk, N, K, T, 1))
+        self.ws = torch.zeros((self.need,), **u8) if self.need else None
+        self.set_bytes = sum(t.numel() * t.element_size() for t in self.sets[0].values())
+        self.step = 0
+
+    def launches(self, s, which="all", x=None):
+        import block_scaled_precision_quant_b200 as bq
+        d = dict(self.sets[s])
+        if x is not None:
+            d["x"] = x
+        T, N, K = self.T, self.N, self.K
+        n = 0
+        if which in ("all", "act_quant"):
+            seed = 1000 + s  # a fresh stochastic-rounding seed per input set
+            bq.grad_quant(d["x"], stochastic=True, seed=seed, q=self.gq, sf_mma=self.gsf)
+            bq.quant_transposed(d["w"], fmt=bq.BQ_FMT_E4M3, q=self.wtq, sf_mma=self.wtsf)
+            bq.quant_transposed(d["x"], fmt=bq.BQ_FMT_E5M2, stochastic=True, seed=seed + 1,
+                                q=self.gtq, sf_mma=self.gtsf)
+            bq.quant_transposed(d["xin"], fmt=bq.BQ_FMT_E4M3, q=self.xtq, sf_mma=self.xtsf)
+            n += 4
+        if which in ("all", "gemm"):
+            bq.gemm(bq.W_GRAD, self.gq, self.gsf, self.wtq, self.wtsf, T, K, N, y=self.y,
+                    workspace=self.ws)
+            bq.gemm(bq.W_GRAD, self.gtq, self.gtsf, self.xtq, self.xtsf, N, K, T, y=self.dw,
+                    workspace=self.ws)
+            n += 2
+        return n
+
+
+def make_layer(spec, sets, seed, device, **kw):
+    if spec[1] == "grad":
+        return BackwardLayer(spec, sets, seed, device, **kw)
+    return Layer(spec, sets, seed, device, **kw)
+
+
 def build_graphs(layers, nsets, which):
     """One CUDA graph per input set (one step each) and one rotation graph
     holding the steps of all sets back to back."""
@@ -470,6 +564,24 @@ def oracle_step_sample(layers_spec, rows, seed=0, nthreads=None):
     t_total = 0.0
     for (name, wk, M, N, K, B, ex) in layers_spec:
         r = min(rows, M)
+        if wk == "grad":
+            # backward: `r` rows of dX (over all N) and `r` rows of dW (over all T tokens)
+            dy = synth.activations(M, N, seed=seed + 2, group_pow2=(-20, 4))
+            w = synth.activations(N, K, seed=seed + 1, std=0.05)
+            xin = synth.activations(M, K, seed=seed)
+            t0 = time.perf_counter()
+            gq, gs = oracle.grad_quant(dy[:r], stochastic=True, seed=seed)
+            wq, ws = oracle.quant_transposed(w, oracle.Q_E4M3)
+            oracle.gemm(gq, gs, wq, ws, oracle.B_FP8ROW, r, K, N, a_kind=oracle.A_E5M2,
+                        nthreads=nthreads)
+            gtq, gts = oracle.quant_transposed(dy[:, :max(8, r)], oracle.Q_E5M2, stochastic=True,
+                                               seed=seed)
+            xq, xs = oracle.quant_transposed(xin, oracle.Q_E4M3)
+            oracle.gemm(gtq[:r], gts[:r], xq, xs, oracle.B_FP8ROW, r, K, M,
+                        a_kind=oracle.A_E5M2, nthreads=nthreads)
+            t_total += time.perf_counter() - t0
+            flops += 2.0 * r * K * N + 2.0 * r * K * M
+            continue
         x = synth.activations(r, K, seed=seed, group_pow2=ex.get("act_gp"))
         if wk in ("mxfp4", "a4w4"):
             wb, ws = synth.mxfp4_weight(N, K, seed=seed + 500)
@@ -563,7 +675,7 @@ def run_ours(args, spec, world, rank, local, device):
             M, N, K = (int(v) for v in args.profile_shape.split(","))
             name, wk, _, _, _, B, ex = specs[0]
             specs = [(name, wk, M, N, K, B, ex)]
-        layers = [Layer(sp, 1, 11 * (i + 1), device) for i, sp in enumerate(specs)]
+        layers = [make_layer(sp, 1, 11 * (i + 1), device) for i, sp in enumerate(specs)]
         for _ in range(args.profile_run):
             for L in layers:
                 L.launches(0)
@@ -576,13 +688,13 @@ def run_ours(args, spec, world, rank, local, device):
 
     layers_spec = spec["layers"]
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    probe = [Layer(sp, 1, 11 * (i + 1), device) for i, sp in enumerate(layers_spec)]
+    probe = [make_layer(sp, 1, 11 * (i + 1), device) for i, sp in enumerate(layers_spec)]
     set_bytes = sum(L.set_bytes for L in probe)
     nsets = max(1, min(64, int(np.ceil(3.0 * l2 / max(set_bytes, 1)))))
     del probe
     torch.cuda.empty_cache()
-    layers = [Layer(sp, nsets, 11 * (i + 1), device, quant_out=args.quant_out,
-                    fused_act=args.fused_act)
+    layers = [make_layer(sp, nsets, 11 * (i + 1), device, quant_out=args.quant_out,
+                         fused_act=args.fused_act)
               for i, sp in enumerate(layers_spec)]
     graphs = build_graphs(layers, nsets, "all")
     launches_per_step = sum(L.launches_per_step for L in layers)
@@ -638,12 +750,13 @@ def run_ours(args, spec, world, rank, local, device):
     a4 = all(sp[1] == "a4w4" for sp in layers_spec)
     tensor_ratio = 4.0 if a4 else 2.0
     fp8_peak = tensor_ratio * peaks[tensor_kind]
-    gemm_launches = len(layers_spec)
+    shapes = [(WKIND[sp[1]],) + g for sp in layers_spec for g in gemm_shapes(sp)]
+    gemm_launches = len(shapes)
     # the GEMM kernel(s) the built-in dispatch runs for these layers
     sms = torch.cuda.get_device_properties(device).multi_processor_count
-    kernels = sorted({("gemm_pair_kernel" if bq.plan(sp[2], sp[3], sp[4], sp[5], num_sms=sms,
-                                                     weight_kind=WKIND[sp[1]]).cta_pair == 2
-                       else "gemm_bs_kernel") for sp in layers_spec})
+    kernels = sorted({("gemm_pair_kernel" if bq.plan(M, N, K, B, num_sms=sms,
+                                                     weight_kind=wk).cta_pair == 2
+                       else "gemm_bs_kernel") for (wk, M, N, K, B) in shapes})
     kernel_name = "+".join(kernels)
     if spec["bound"] == "hbm":
         achieved = gbytes_step / (gemm_ms_step * 1e-3) / 1e9

@@ -38,6 +38,9 @@ BQ_ACT_GELU = 1
 BQ_SPLIT_AUTO, BQ_SPLIT_WORKSPACE, BQ_SPLIT_CLUSTER = 0, 1, 2
 W_MXFP4, W_FP8BLK32, W_MXFP8 = 0, 1, 2
 W_A4W4 = 3  # MXFP4 weights with MXFP4 (packed E2M1) activations
+W_GRAD = 4  # E5M2 gradient codes x MXFP8 (E4M3) operand: the backward products
+BQ_ROUND_NEAREST, BQ_ROUND_STOCHASTIC = 0, 1
+BQ_FMT_E4M3, BQ_FMT_E5M2 = 0, 1
 
 EXPORTS = (
     "bq_status_string", "bq_version", "bq_sf_bytes", "bq_act_quant", "bq_pack_weight_scales",
@@ -46,7 +49,8 @@ EXPORTS = (
     "bq_gemm_mxfp8_mxfp8_epilogue", "bq_device_status", "bq_device_status_detail",
     "bq_device_report", "bq_gemm_mxfp8_mxfp4_epilogue_noalloc", "bq_noalloc_scratch_bytes",
     "bq_gemm_bf16act_epilogue", "bq_gemm_plan", "bq_act_quant_mxfp4", "bq_gemm_mxfp4_mxfp4",
-    "bq_gemm_mxfp4_mxfp4_epilogue",
+    "bq_gemm_mxfp4_mxfp4_epilogue", "bq_grad_quant", "bq_quant_transposed", "bq_gemm_e5m2_mxfp8",
+    "bq_gemm_e5m2_mxfp8_epilogue",
 )
 
 
@@ -102,17 +106,23 @@ def lib():
         L.bq_act_quant.restype = i32
         L.bq_act_quant_mxfp4.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp]
         L.bq_act_quant_mxfp4.restype = i32
+        L.bq_grad_quant.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, i32, ctypes.c_uint64, vp]
+        L.bq_grad_quant.restype = i32
+        L.bq_quant_transposed.argtypes = [vp, i64, i64, i64, i32, i32, ctypes.c_uint64, vp, vp,
+                                          vp, vp]
+        L.bq_quant_transposed.restype = i32
         L.bq_pack_weight_scales.argtypes = [vp, i32, i64, i64, vp, vp, vp]
         L.bq_pack_weight_scales.restype = i32
         L.bq_unpack_scales.argtypes = [vp, i64, i64, vp, vp]
         L.bq_unpack_scales.restype = i32
         for name in ("bq_gemm_mxfp8_mxfp4", "bq_gemm_mxfp8_fp8blk32", "bq_gemm_mxfp8_mxfp8",
-                     "bq_gemm_mxfp4_mxfp4"):
+                     "bq_gemm_mxfp4_mxfp4", "bq_gemm_e5m2_mxfp8"):
             f = getattr(L, name)
             f.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp]
             f.restype = i32
         for name in ("bq_gemm_mxfp8_mxfp4_epilogue", "bq_gemm_mxfp8_fp8blk32_epilogue",
-                     "bq_gemm_mxfp8_mxfp8_epilogue", "bq_gemm_mxfp4_mxfp4_epilogue"):
+                     "bq_gemm_mxfp8_mxfp8_epilogue", "bq_gemm_mxfp4_mxfp4_epilogue",
+                     "bq_gemm_e5m2_mxfp8_epilogue"):
             f = getattr(L, name)
             f.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, ctypes.POINTER(Epilogue),
                           ctypes.POINTER(Batch), vp, sz, ctypes.POINTER(GemmConfig), vp]
@@ -234,6 +244,49 @@ def act_quant_mxfp4(x, q=None, sf_mma=None, sf_rowmajor=None, status=None):
     return q, sf_mma
 
 
+def grad_quant(g, stochastic=False, seed=0, q=None, sf_mma=None, sf_rowmajor=None,
+               status=None):
+    """Per-32 E5M2 quantization of a bf16 [M, K] gradient along K (round to
+    nearest even, or stochastic with Philox draws keyed by seed): returns (q
+    uint8 [M, K] E5M2 codes, sf_mma MMA-layout scales)."""
+    torch = _torch()
+    _need_cuda(g)
+    if g.dtype != torch.bfloat16 or g.dim() != 2 or g.stride(1) != 1:
+        raise ValueError("g must be a bf16 [M, K] tensor with unit column stride")
+    M, K = g.shape
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.uint8, device=g.device)
+    if sf_mma is None:
+        sf_mma = torch.empty((max(sf_bytes(M, K), 1),), dtype=torch.uint8, device=g.device)
+    _check(lib().bq_grad_quant(_ptr(g), M, K, g.stride(0), _ptr(q), _ptr(sf_mma),
+                               _ptr(sf_rowmajor), _ptr(status),
+                               BQ_ROUND_STOCHASTIC if stochastic else BQ_ROUND_NEAREST,
+                               int(seed) & (2 ** 64 - 1), _stream()), "bq_grad_quant")
+    return q, sf_mma
+
+
+def quant_transposed(x, fmt=BQ_FMT_E4M3, stochastic=False, seed=0, q=None, sf_mma=None,
+                     status=None):
+    """Quantize a bf16 [R, C] tensor along R (per 32 rows of each column) and
+    write it transposed: returns (q uint8 [C, R] codes, sf_mma MMA-layout
+    scales of a [C, R] operand).  fmt BQ_FMT_E4M3 or BQ_FMT_E5M2 (stochastic
+    rounding for E5M2 only)."""
+    torch = _torch()
+    _need_cuda(x)
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a bf16 [R, C] tensor with unit column stride")
+    R, C = x.shape
+    if q is None:
+        q = torch.empty((C, R), dtype=torch.uint8, device=x.device)
+    if sf_mma is None:
+        sf_mma = torch.empty((max(sf_bytes(C, R), 1),), dtype=torch.uint8, device=x.device)
+    _check(lib().bq_quant_transposed(_ptr(x), R, C, x.stride(0), int(fmt),
+                                     BQ_ROUND_STOCHASTIC if stochastic else BQ_ROUND_NEAREST,
+                                     int(seed) & (2 ** 64 - 1), _ptr(q), _ptr(sf_mma),
+                                     _ptr(status), _stream()), "bq_quant_transposed")
+    return q, sf_mma
+
+
 def pack_weight_scales(scales, kind: int, N: int, K: int, out=None, e4m3_codes=None):
     """E8M0 weight scales (ROW32 [N, K/32] or BLK32x32 [ceil(N/32), K/32]) to
     the MMA layout.  Synchronizes the stream; raises on NaN scales or codes."""
@@ -261,7 +314,8 @@ def unpack_scales(sf_mma, rows: int, K: int, out=None):
 
 _ws = {}
 _ENTRY = {W_MXFP4: "bq_gemm_mxfp8_mxfp4", W_FP8BLK32: "bq_gemm_mxfp8_fp8blk32",
-          W_MXFP8: "bq_gemm_mxfp8_mxfp8", W_A4W4: "bq_gemm_mxfp4_mxfp4"}
+          W_MXFP8: "bq_gemm_mxfp8_mxfp8", W_A4W4: "bq_gemm_mxfp4_mxfp4",
+          W_GRAD: "bq_gemm_e5m2_mxfp8"}
 
 
 def _config(block_n=0, split_k=0, swap_ab=-1, split_mode=0, k_chunks=0, cta_pair=0):
@@ -301,8 +355,9 @@ def gemm(weight_kind, a_q, a_sf, b, b_sf, M, N, K, y=None, bias=None, residual=N
          alpha=1.0, act=BQ_ACT_NONE, batch=None, config=None, workspace=None,
          quantize_out=False, write_y=True, q_out=None, sf_out=None):
     """y = bf16(act(alpha * A B^T + bias) + residual) for weight_kind W_MXFP4,
-    W_FP8BLK32, W_MXFP8 (E4M3 activations a_q [.., M, K]) or W_A4W4 (packed
-    E2M1 activations a_q [.., M, K/2] from act_quant_mxfp4).  batch: None or a dict with 'count' and byte
+    W_FP8BLK32, W_MXFP8 (E4M3 activations a_q [.., M, K]), W_A4W4 (packed
+    E2M1 activations a_q [.., M, K/2] from act_quant_mxfp4) or W_GRAD (E5M2
+    gradient codes a_q [.., M, K], MXFP8 b).  batch: None or a dict with 'count' and byte
     strides ('stride_a', 'stride_a_sf', 'stride_b', 'stride_b_sf', 'stride_y',
     'stride_res'; 0 broadcasts).  config: GemmConfig or None (auto).
     quantize_out: also return y quantized for the next GEMM (E4M3 codes
@@ -414,6 +469,10 @@ def gemm_mxfp8_mxfp8(a_q, a_sf, b_e4m3, b_sf, M, N, K, **kw):
 
 def gemm_mxfp4_mxfp4(a_fp4, a_sf, b_fp4, b_sf, M, N, K, **kw):
     return gemm(W_A4W4, a_fp4, a_sf, b_fp4, b_sf, M, N, K, **kw)
+
+
+def gemm_e5m2_mxfp8(a_e5m2, a_sf, b_e4m3, b_sf, M, N, K, **kw):
+    return gemm(W_GRAD, a_e5m2, a_sf, b_e4m3, b_sf, M, N, K, **kw)
 
 
 config = _config

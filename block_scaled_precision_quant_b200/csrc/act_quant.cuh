@@ -20,14 +20,49 @@
 
 namespace bq {
 
+// Code formats of the quantizers.
+enum QuantFmt : int { kQE4M3 = 0, kQFP4 = 1, kQE5M2 = 2 };
+
+// E5M2 codes of 16 bf16 values (8 words, element 2i in the low half of word
+// i) scaled by 2^-e; SR: stochastic rounding with the draws of elements
+// idx0 .. idx0 + 15 (idx0 a multiple of 4) under `seed`.
+template <bool SR>
+__device__ __forceinline__ void e5m2_encode16(const uint32_t (&w)[8], int e, uint64_t seed,
+                                              uint64_t idx0, uint32_t (&codes)[4]) {
+  const float inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float f[4];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const uint32_t word = w[2 * i + j];
+      f[2 * j] = fminf(fmaxf(__fmul_rn(__uint_as_float(word << 16), inv), -57344.0f), 57344.0f);
+      f[2 * j + 1] =
+          fminf(fmaxf(__fmul_rn(__uint_as_float(word & 0xFFFF0000u), inv), -57344.0f), 57344.0f);
+    }
+    if constexpr (SR) {
+      const Philox4 r = philox4x64_10((idx0 >> 2) + i, seed);
+      codes[i] = e5m2_sr(f[0], philox_uniform(r.w[0])) |
+                 (e5m2_sr(f[1], philox_uniform(r.w[1])) << 8) |
+                 (e5m2_sr(f[2], philox_uniform(r.w[2])) << 16) |
+                 (e5m2_sr(f[3], philox_uniform(r.w[3])) << 24);
+    } else {
+      codes[i] = e5m2x2(f[0], f[1]) | (e5m2x2(f[2], f[3]) << 16);
+    }
+  }
+}
+
 // grid: x*8 + warp = row, y = chunk of 16 groups within the row.  Rows in
-// [M, rows_pad) only write padding scale bytes (127).  FP4: E2M1 codes
-// (packed [M, K/2], the per-32 rule with 6 in place of 448) instead of E4M3.
-template <bool FP4>
+// [M, rows_pad) only write padding scale bytes (127).  FMT: E4M3 codes; FP4:
+// E2M1 codes (packed [M, K/2], the per-32 rule with 6 in place of 448); E5M2:
+// gradient codes (the rule with 57344), SR with stochastic rounding (the
+// draw of element (row, col) is index row * K + col under `seed`).
+template <int FMT, bool SR = false>
 __global__ void __launch_bounds__(256) act_quant_kernel(
     const __nv_bfloat16 *__restrict__ x, int64_t M, int64_t K, int64_t ldx, int64_t rows_pad,
     uint8_t *__restrict__ q, uint8_t *__restrict__ sf_mma, uint8_t *__restrict__ sf_row,
-    int *__restrict__ status) {
+    int *__restrict__ status, uint64_t seed) {
+  static_assert(!SR || FMT == kQE5M2, "stochastic rounding is for E5M2 gradients");
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (row >= rows_pad) return;
@@ -59,9 +94,15 @@ __global__ void __launch_bounds__(256) act_quant_kernel(
   uint32_t sbyte = 127;
   if (active) {
     if (bad && status) atomicOr(status, 1);
-    const int e = FP4 ? mx_exponent_fp4(mx) : mx_exponent(mx);
+    const int e = FMT == kQFP4    ? mx_exponent_fp4(mx)
+                  : FMT == kQE5M2 ? mx_exponent_e5m2(mx)
+                                  : mx_exponent(mx);
     sbyte = static_cast<uint32_t>(e + 127);
-    if constexpr (FP4) {
+    if constexpr (FMT == kQE5M2) {
+      uint32_t c[4];
+      e5m2_encode16<SR>(w, e, seed, static_cast<uint64_t>(row * K + col), c);
+      *reinterpret_cast<uint4 *>(q + row * K + col) = make_uint4(c[0], c[1], c[2], c[3]);
+    } else if constexpr (FMT == kQFP4) {
       uint32_t c[2];
       mx_encode_fp4(w, e, c);
       *reinterpret_cast<uint2 *>(q + row * (K >> 1) + (col >> 1)) = make_uint2(c[0], c[1]);
@@ -84,6 +125,129 @@ __global__ void __launch_bounds__(256) act_quant_kernel(
       const uint32_t word = sbyte | (b1 << 8) | (b2 << 16) | (b3 << 24);
       *reinterpret_cast<uint32_t *>(sf_mma + sf_mma_offset(row, g4, katoms)) = word;
     }
+  }
+}
+
+// Transposed quantization (the operands of the weight gradient, and the
+// weight operand of the input gradient): x bf16 [R, ldx] with C columns used,
+// quantized along R -- per 32 consecutive rows of one column -- and written
+// transposed: codes [C, R] (row pitch R) and scales in the MMA layout of a
+// [C, R] operand.  FMT kQE4M3 (the act_quant rule) or kQE5M2 (the gradient
+// rule; SR: the draw of element (r, c) is index r * C + c under `seed`).
+//
+// A warp owns 32 rows x 64 columns: lane l loads row r0 + l (64 values, 8 x
+// 16 B); the amax of every column over the 32 rows is a 5-step butterfly on
+// two columns per word (packed 16-bit maxima); each lane encodes its 64 values
+// with their columns' scales; the codes turn around through 2 KB of shared
+// memory per warp and leave as 32-byte pieces of the output rows.
+// grid.x = row group (32 rows), grid.y * 8 + warp = column tile (64 columns).
+// Tiles past C or past R/32 write padding scales (127) only.
+template <int FMT, bool SR>
+__global__ void __launch_bounds__(256) quant_t_kernel(
+    const __nv_bfloat16 *__restrict__ x, int64_t R, int64_t C, int64_t ldx, int64_t col_tiles,
+    uint8_t *__restrict__ q, uint8_t *__restrict__ sf_mma, int *__restrict__ status,
+    uint64_t seed) {
+  static_assert(FMT == kQE4M3 || FMT == kQE5M2, "E4M3 or E5M2 codes");
+  static_assert(!SR || FMT == kQE5M2, "stochastic rounding is for E5M2 gradients");
+  __shared__ __align__(16) uint8_t stage[8][64 * 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t ct = static_cast<int64_t>(blockIdx.y) * 8 + warp;
+  if (ct >= col_tiles) return;  // whole warps leave; only warp-level sync below
+  const int64_t c0 = ct * 64;
+  const int64_t g = blockIdx.x;
+  const int64_t r0 = g * 32;
+  const int64_t G = R >> 5;
+  const int64_t katoms = (G + 3) >> 2;
+  const bool rows_ok = g < G;
+  griddep_wait();
+  griddep_launch_dependents();
+
+  uint32_t w[32];  // columns 2i (low half) and 2i + 1 (high half) of row r0 + lane
+#pragma unroll
+  for (int v = 0; v < 8; ++v) {
+    uint4 t = make_uint4(0u, 0u, 0u, 0u);
+    const int64_t c = c0 + v * 8;
+    if (rows_ok && c < C)
+      t = __ldg(reinterpret_cast<const uint4 *>(x + (r0 + lane) * ldx + c));
+    w[4 * v] = t.x;
+    w[4 * v + 1] = t.y;
+    w[4 * v + 2] = t.z;
+    w[4 * v + 3] = t.w;
+  }
+  uint32_t m[32];
+  uint32_t bad = 0;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    m[i] = w[i] & 0x7FFF7FFFu;
+    bad |= ((m[i] & 0x7F80u) == 0x7F80u) | ((m[i] & 0x7F800000u) == 0x7F800000u);
+  }
+#pragma unroll
+  for (int k = 16; k >= 1; k >>= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) m[i] = __vmaxu2(m[i], __shfl_xor_sync(0xFFFFFFFFu, m[i], k));
+  }
+  if (bad && status && rows_ok) atomicOr(status, 1);
+
+  uint8_t *st = stage[warp];
+  const int64_t row = r0 + lane;
+  int e_lo = 0, e_hi = 0;  // the exponents of columns c0 + lane and c0 + lane + 32
+  Philox4 rnd;             // SR: the draws of the current 4 columns
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const uint32_t a0 = m[i] & 0xFFFFu, a1 = m[i] >> 16;
+    const int e0 = FMT == kQE5M2 ? mx_exponent_e5m2(a0) : mx_exponent(a0);
+    const int e1 = FMT == kQE5M2 ? mx_exponent_e5m2(a1) : mx_exponent(a1);
+    if (2 * i == lane) e_lo = e0;
+    if (2 * i + 1 == lane) e_lo = e1;
+    if (2 * i == lane + 32) e_hi = e0;
+    if (2 * i + 1 == lane + 32) e_hi = e1;
+    const float inv0 = __uint_as_float(static_cast<uint32_t>(127 - e0) << 23);
+    const float inv1 = __uint_as_float(static_cast<uint32_t>(127 - e1) << 23);
+    const float lim = FMT == kQE5M2 ? 57344.0f : 448.0f;
+    const float f0 =
+        fminf(fmaxf(__fmul_rn(__uint_as_float(w[i] << 16), inv0), -lim), lim);
+    const float f1 =
+        fminf(fmaxf(__fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), inv1), -lim), lim);
+    uint32_t b0, b1;
+    if constexpr (SR) {
+      // draws of columns c0 + 2i, c0 + 2i + 1: one Philox block serves 4
+      // columns (row * C + c0 is a multiple of 4: C % 8 == 0, c0 % 64 == 0)
+      if (i % 2 == 0)
+        rnd = philox4x64_10(static_cast<uint64_t>(row * C + c0 + 2 * i) >> 2, seed);
+      b0 = e5m2_sr(f0, philox_uniform(rnd.w[(2 * i) & 3]));
+      b1 = e5m2_sr(f1, philox_uniform(rnd.w[((2 * i) & 3) + 1]));
+    } else if constexpr (FMT == kQE5M2) {
+      const uint32_t p = e5m2x2(f0, f1);
+      b0 = p & 0xFFu;
+      b1 = p >> 8;
+    } else {
+      const uint32_t p = e4m3x4(f0, f1, 0.0f, 0.0f);
+      b0 = p & 0xFFu;
+      b1 = (p >> 8) & 0xFFu;
+    }
+    st[(2 * i) * 32 + lane] = static_cast<uint8_t>(b0);
+    st[(2 * i + 1) * 32 + lane] = static_cast<uint8_t>(b1);
+  }
+  __syncwarp();
+  if (rows_ok) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int j = 2 * lane + h;
+      if (c0 + j < C) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(st + j * 32);
+        uint4 *dst = reinterpret_cast<uint4 *>(q + (c0 + j) * R + r0);
+        dst[0] = src[0];
+        dst[1] = src[1];
+      }
+    }
+  }
+  // scales of columns c0 + lane and c0 + lane + 32 (padding: 127)
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int j = lane + 32 * h;
+    const uint32_t b = (rows_ok && c0 + j < C) ? static_cast<uint32_t>((h ? e_hi : e_lo) + 127)
+                                              : 127u;
+    sf_mma[sf_mma_offset(c0 + j, g, katoms)] = static_cast<uint8_t>(b);
   }
 }
 

@@ -175,7 +175,9 @@ int make_y_map(CUtensorMap* m, const void* y, int64_t M, int64_t N, int64_t ld, 
 // ---------------------------------------------------------------- schedule --
 
 // kA4W4: MXFP4 weights with MXFP4 (packed E2M1) activations, kind::mxf4.
-enum WeightKind { kMxfp4 = 0, kFp8Blk32 = 1, kMxfp8 = 2, kA4W4 = 3 };
+// kGrad: E5M2 gradient codes on the activation side, an E4M3 operand with
+// per-32 scales (MXFP8) on the weight side (the backward GEMMs).
+enum WeightKind { kMxfp4 = 0, kFp8Blk32 = 1, kMxfp8 = 2, kA4W4 = 3, kGrad = 4 };
 
 struct Plan {
   bool swap = false;
@@ -634,6 +636,12 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
   bq::GemmArgs g;
   memset(&g, 0, sizeof(g));
   g.M = static_cast<int>(M);
+  {
+    const uint32_t f_act = wk == kGrad ? bq::kFmtE5M2 : bq::kFmtE4M3;
+    const uint32_t f_w = w_fp4 ? bq::kFmtE2M1 : bq::kFmtE4M3;
+    g.fmt_p = pl.swap ? f_w : f_act;
+    g.fmt_q = pl.swap ? f_act : f_w;
+  }
   g.N = static_cast<int>(N);
   g.K = static_cast<int>(K);
   g.batch = static_cast<int>(count);
@@ -740,9 +748,10 @@ size_t bq_sf_bytes(int64_t rows, int64_t K) {
 
 namespace {
 
-// Launch of the per-32 activation quantizer; fp4 selects E2M1 output.
-int act_quant_launch(bool fp4, const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
-                     void* q_out, void* sf_mma, void* sf_rowmajor, int* d_status,
+// Launch of the per-32 quantizer along rows: fmt bq::kQE4M3 / kQFP4 /
+// kQE5M2, sr stochastic rounding (E5M2 only) under `seed`.
+int act_quant_launch(int fmt, bool sr, uint64_t seed, const void* x_bf16, int64_t M, int64_t K,
+                     int64_t ldx, void* q_out, void* sf_mma, void* sf_rowmajor, int* d_status,
                      bq_stream_t stream) {
   DevInfo* dev = nullptr;
   int st = current_device(&dev);
@@ -764,10 +773,49 @@ int act_quant_launch(bool fp4, const void* x_bf16, int64_t M, int64_t K, int64_t
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = 1;
-  auto kern = fp4 ? bq::act_quant_kernel<true> : bq::act_quant_kernel<false>;
+  auto kern = fmt == bq::kQFP4    ? bq::act_quant_kernel<bq::kQFP4>
+              : fmt == bq::kQE5M2 ? (sr ? bq::act_quant_kernel<bq::kQE5M2, true>
+                                        : bq::act_quant_kernel<bq::kQE5M2>)
+                                  : bq::act_quant_kernel<bq::kQE4M3>;
   if (cudaLaunchKernelEx(&lc, kern, static_cast<const __nv_bfloat16*>(x_bf16), M, K, ldx,
                          rows_pad, static_cast<uint8_t*>(q_out), static_cast<uint8_t*>(sf_mma),
-                         static_cast<uint8_t*>(sf_rowmajor), d_status) != cudaSuccess) {
+                         static_cast<uint8_t*>(sf_rowmajor), d_status, seed) != cudaSuccess) {
+    cudaGetLastError();
+    return BQ_ERR_CUDA;
+  }
+  return launch_status();
+}
+
+// Launch of the transposed quantizer: x [R, ldx] (C columns) along R into
+// codes [C, R] and the MMA-layout scales of a [C, R] operand.
+int quant_t_launch(int fmt, bool sr, uint64_t seed, const void* x_bf16, int64_t R, int64_t C,
+                   int64_t ldx, void* q_t, void* sf_mma, int* d_status, bq_stream_t stream) {
+  DevInfo* dev = nullptr;
+  int st = current_device(&dev);
+  if (st != BQ_OK) return st;
+  if (R <= 0 || R % 32 != 0 || C < 0 || C % 8 != 0 || ldx < C) return BQ_ERR_SHAPE;
+  if (C == 0) return BQ_OK;
+  if (!x_bf16 || !q_t || !sf_mma) return BQ_ERR_NULL;
+  if (!aligned(x_bf16, 16) || ldx % 8 != 0 || !aligned(q_t, 16)) return BQ_ERR_ALIGN;
+  const int64_t rows_pad = (C + 127) / 128 * 128;  // rows of the transposed operand
+  const int64_t col_tiles = rows_pad / 64;
+  const int64_t groups_pad = (R / 32 + 3) / 4 * 4;
+  if (groups_pad > 0x7FFFFFFF || (col_tiles + 7) / 8 > 65535) return BQ_ERR_SHAPE;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(static_cast<unsigned>(groups_pad), static_cast<unsigned>((col_tiles + 7) / 8));
+  lc.blockDim = dim3(256);
+  lc.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  auto kern = fmt == bq::kQE5M2 ? (sr ? bq::quant_t_kernel<bq::kQE5M2, true>
+                                      : bq::quant_t_kernel<bq::kQE5M2, false>)
+                                : bq::quant_t_kernel<bq::kQE4M3, false>;
+  if (cudaLaunchKernelEx(&lc, kern, static_cast<const __nv_bfloat16*>(x_bf16), R, C, ldx,
+                         col_tiles, static_cast<uint8_t*>(q_t), static_cast<uint8_t*>(sf_mma),
+                         d_status, seed) != cudaSuccess) {
     cudaGetLastError();
     return BQ_ERR_CUDA;
   }
@@ -780,13 +828,33 @@ extern "C" {
 
 int bq_act_quant(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, void* q_e4m3,
                  void* sf_mma, void* sf_rowmajor, int* d_status, bq_stream_t stream) {
-  return act_quant_launch(false, x_bf16, M, K, ldx, q_e4m3, sf_mma, sf_rowmajor, d_status,
-                          stream);
+  return act_quant_launch(bq::kQE4M3, false, 0, x_bf16, M, K, ldx, q_e4m3, sf_mma, sf_rowmajor,
+                          d_status, stream);
 }
 
 int bq_act_quant_mxfp4(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, void* q_fp4,
                        void* sf_mma, void* sf_rowmajor, int* d_status, bq_stream_t stream) {
-  return act_quant_launch(true, x_bf16, M, K, ldx, q_fp4, sf_mma, sf_rowmajor, d_status, stream);
+  return act_quant_launch(bq::kQFP4, false, 0, x_bf16, M, K, ldx, q_fp4, sf_mma, sf_rowmajor,
+                          d_status, stream);
+}
+
+int bq_grad_quant(const void* g_bf16, int64_t M, int64_t K, int64_t ldg, void* q_e5m2,
+                  void* sf_mma, void* sf_rowmajor, int* d_status, int rounding, uint64_t seed,
+                  bq_stream_t stream) {
+  if (rounding != BQ_ROUND_NEAREST && rounding != BQ_ROUND_STOCHASTIC) return BQ_ERR_INVALID;
+  return act_quant_launch(bq::kQE5M2, rounding == BQ_ROUND_STOCHASTIC, seed, g_bf16, M, K, ldg,
+                          q_e5m2, sf_mma, sf_rowmajor, d_status, stream);
+}
+
+int bq_quant_transposed(const void* x_bf16, int64_t R, int64_t C, int64_t ldx, int fmt,
+                        int rounding, uint64_t seed, void* q_t, void* sf_mma, int* d_status,
+                        bq_stream_t stream) {
+  if (fmt != BQ_FMT_E4M3 && fmt != BQ_FMT_E5M2) return BQ_ERR_INVALID;
+  if (rounding != BQ_ROUND_NEAREST && rounding != BQ_ROUND_STOCHASTIC) return BQ_ERR_INVALID;
+  if (rounding == BQ_ROUND_STOCHASTIC && fmt != BQ_FMT_E5M2) return BQ_ERR_INVALID;
+  return quant_t_launch(fmt == BQ_FMT_E5M2 ? bq::kQE5M2 : bq::kQE4M3,
+                        rounding == BQ_ROUND_STOCHASTIC, seed, x_bf16, R, C, ldx, q_t, sf_mma,
+                        d_status, stream);
 }
 
 int bq_pack_weight_scales(const void* scales_u8, int kind, int64_t N, int64_t K, void* sf_mma,
@@ -866,6 +934,22 @@ int bq_gemm_mxfp8_mxfp8(const void* a_q, const void* a_sf, const void* b_e4m3, c
                     0, &kNoSplit, stream);
 }
 
+int bq_gemm_e5m2_mxfp8(const void* a_e5m2, const void* a_sf, const void* b_e4m3,
+                       const void* b_sf, int64_t M, int64_t N, int64_t K, void* y_bf16,
+                       bq_stream_t stream) {
+  return gemm_entry(kGrad, a_e5m2, a_sf, b_e4m3, b_sf, M, N, K, y_bf16, nullptr, nullptr, nullptr,
+                    0, &kNoSplit, stream);
+}
+
+int bq_gemm_e5m2_mxfp8_epilogue(const void* a_e5m2, const void* a_sf, const void* b_e4m3,
+                                const void* b_sf, int64_t M, int64_t N, int64_t K, void* y_bf16,
+                                const bq_epilogue* epi, const bq_batch* batch, void* workspace,
+                                size_t workspace_bytes, const bq_gemm_config* cfg,
+                                bq_stream_t stream) {
+  return gemm_entry(kGrad, a_e5m2, a_sf, b_e4m3, b_sf, M, N, K, y_bf16, epi, batch, workspace,
+                    workspace_bytes, cfg, stream);
+}
+
 int bq_gemm_mxfp4_mxfp4(const void* a_fp4, const void* a_sf, const void* b_fp4, const void* b_sf,
                         int64_t M, int64_t N, int64_t K, void* y_bf16, bq_stream_t stream) {
   return gemm_entry(kA4W4, a_fp4, a_sf, b_fp4, b_sf, M, N, K, y_bf16, nullptr, nullptr, nullptr, 0,
@@ -883,7 +967,7 @@ int bq_gemm_mxfp4_mxfp4_epilogue(const void* a_fp4, const void* a_sf, const void
 
 size_t bq_gemm_workspace_bytes(int weight_kind, int64_t M, int64_t N, int64_t K, int64_t batch,
                                const bq_gemm_config* cfg) {
-  if (weight_kind < 0 || weight_kind > 3 || M <= 0 || N <= 0 || K <= 0 || batch <= 0) return 0;
+  if (weight_kind < 0 || weight_kind > 4 || M <= 0 || N <= 0 || K <= 0 || batch <= 0) return 0;
   DevInfo* dev = nullptr;
   if (current_device(&dev) != BQ_OK) return 0;
   Plan pl;
@@ -896,7 +980,7 @@ size_t bq_gemm_workspace_bytes(int weight_kind, int64_t M, int64_t N, int64_t K,
 int bq_gemm_plan(int weight_kind, int64_t M, int64_t N, int64_t K, int64_t batch,
                  const bq_gemm_config* cfg, int num_sms, bq_gemm_config* out) {
   if (!out) return BQ_ERR_NULL;
-  if (weight_kind < 0 || weight_kind > 3) return BQ_ERR_INVALID;
+  if (weight_kind < 0 || weight_kind > 4) return BQ_ERR_INVALID;
   if (M <= 0 || N <= 0 || K <= 0 || K % 32 != 0 || batch <= 0 || num_sms < 1)
     return BQ_ERR_SHAPE;
   Plan pl;

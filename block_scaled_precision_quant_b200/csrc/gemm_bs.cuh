@@ -56,14 +56,16 @@ constexpr int kAsfWarp = 8;
 constexpr int kCopyThreads = 4;
 
 // tcgen05 operand formats (instruction descriptor fields a_format / b_format):
-// kind::mxf8f6f4 codes E4M3 0 and E2M1 5 (one byte slot per FP4 code in shared
-// memory); kind::mxf4 code E2M1 1 (two codes per byte).
+// kind::mxf8f6f4 codes E4M3 0, E5M2 1 and E2M1 5 (one byte slot per FP4 code in
+// shared memory); kind::mxf4 code E2M1 1 (two codes per byte).
 constexpr uint32_t kFmtE4M3 = 0;
+constexpr uint32_t kFmtE5M2 = 1;
 constexpr uint32_t kFmtE2M1 = 5;
 constexpr uint32_t kFmtMxf4E2M1 = 1;
 
 struct GemmArgs {
   int M, N, K;     // one problem: y[M, N] = A[M, K] B[N, K]^T
+  uint32_t fmt_p, fmt_q;  // kind::mxf8f6f4 operand formats of the P and Q sides
   int batch;       // number of problems
   int kt_total;    // ceil(K / 128)
   int splits;      // K slices per output tile (1 = no split)
@@ -1015,8 +1017,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                               sfq_t + 4 * t * L::kSfqAtoms + sfq_row_off, acc_in);
                 }
               } else {
-                const uint32_t idesc = make_idesc(P_FP4 ? kFmtE2M1 : kFmtE4M3,
-                                                  Q_FP4 ? kFmtE2M1 : kFmtE4M3, BN, ks);
+                const uint32_t idesc = make_idesc(a.fmt_p, a.fmt_q, BN, ks);
                 tc_mma_mxf8f6f4(d_tmem, desc_kmajor_sw128(pa + ks * kMmaK),
                                 desc_kmajor_sw128(qa + ks * kMmaK), idesc, sf_t, sfq_t + sfq_row_off,
                                 acc_in);

@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       const uint32_t b0 = smem_u32(smem + L::kOffB);
       const uint32_t sfa0 = smem_u32(smem + L::kOffSfa);
       const uint32_t sfb0 = smem_u32(smem + L::kOffSfb);
-      const uint32_t fmt_b = Q_FP4 ? kFmtE2M1 : kFmtE4M3;
+      const uint32_t fmt_a = a.fmt_p, fmt_b = a.fmt_q;
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             for (int ks = 0; ks < kBlockK / kMmaK; ++ks)
               tc_mma2_mxf8f6f4(tmem_base, desc_kmajor_sw128(pa + ks * kMmaK),
                                desc_kmajor_sw128(pb + ks * kMmaK),
-                               make_idesc_m(kFmtE4M3, fmt_b, 2 * kBlockP, kPairN, ks), sf_t,
+                               make_idesc_m(fmt_a, fmt_b, 2 * kBlockP, kPairN, ks), sf_t,
                                sf_t + 4, (kt > 0 || c > 0 || ks > 0) ? 1u : 0u);
           }
           tc_commit2(mapa_shared(smem_u32(&empty[stage]), 0));

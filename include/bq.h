@@ -114,6 +114,48 @@ int bq_act_quant(const void *x_bf16, int64_t M, int64_t K, int64_t ldx, void *q_
 int bq_act_quant_mxfp4(const void *x_bf16, int64_t M, int64_t K, int64_t ldx, void *q_fp4,
                        void *sf_mma, void *sf_rowmajor, int *d_status, bq_stream_t stream);
 
+/* ---- backward-pass quantizers ------------------------------------------- */
+
+enum { BQ_ROUND_NEAREST = 0, BQ_ROUND_STOCHASTIC = 1 };
+enum { BQ_FMT_E4M3 = 0, BQ_FMT_E5M2 = 1 };
+
+/* bq_grad_quant -- per-32 E5M2 quantization of bf16 gradients along the last
+ * dimension (the "hip_quant" README on the pages: E5M2 for backward gradients,
+ * "Stochastic E5M2 Backward Gradients", "Block-wise FP8 Scaling"), with the
+ * scale rule of bq_act_quant taking E5M2's largest finite value 57344 in place
+ * of 448: t = fp32(max(amax, 1e-4) * fp32(1/57344)), e = ceil(log2 t), scale
+ * byte e + 127, q = E5M2 of clamp(g / 2^e, -57344, 57344).
+ *   rounding BQ_ROUND_NEAREST: round to nearest even (saturating), sign kept.
+ *   rounding BQ_ROUND_STOCHASTIC: between the two neighbouring E5M2 values of
+ *            |g / 2^e| (lo, hi; the 2^-16 grid below 2^-14), hi when
+ *            u < (|v| - lo) / (hi - lo), u the element's draw: the top 53 bits
+ *            (times 2^-53) of word (i mod 4) of Philox4x64-10 at counter
+ *            (i / 4, 0, 0, 0) under key (seed, 0), i = row * K + column, so the
+ *            draws are a stateless function of (seed, element index).
+ *   g_bf16 [M, K] (row stride ldg), q_e5m2 out [M, K], sf_mma out
+ *   bq_sf_bytes(M, K) (MMA layout), sf_rowmajor / d_status as bq_act_quant.
+ * Errors: as bq_act_quant, BQ_ERR_INVALID for a bad rounding mode. */
+int bq_grad_quant(const void *g_bf16, int64_t M, int64_t K, int64_t ldg, void *q_e5m2,
+                  void *sf_mma, void *sf_rowmajor, int *d_status, int rounding, uint64_t seed,
+                  bq_stream_t stream);
+
+/* bq_quant_transposed -- quantization along the FIRST dimension, written
+ * transposed (the operands of the weight gradient dW = dY^T X contract over
+ * the token dimension, and the input gradient dX = dY W over the output
+ * dimension: "quantize_e5m2_transpose" on the "hip_quant" README page).
+ * x [R, C] bf16 (row stride ldx >= C, ldx % 8 == 0, C % 8 == 0, R % 32 == 0) is
+ * quantized per 32 consecutive rows of each column by the bq_act_quant rule
+ * (fmt BQ_FMT_E4M3) or the bq_grad_quant rule (fmt BQ_FMT_E5M2; stochastic
+ * rounding draws with i = r * C + c, the element's index in x), and stored as
+ *   q_t     out [C, R] codes (row pitch R), 16-byte aligned
+ *   sf_mma  out bq_sf_bytes(C, R): the MMA-layout scales of the [C, R] operand
+ * so that (q_t, sf_mma) is an operand of the GEMMs with C rows and K = R.
+ * Errors: BQ_ERR_NULL, BQ_ERR_SHAPE, BQ_ERR_ALIGN, BQ_ERR_INVALID (fmt,
+ * rounding, or stochastic E4M3), BQ_ERR_ARCH, BQ_ERR_CUDA. */
+int bq_quant_transposed(const void *x_bf16, int64_t R, int64_t C, int64_t ldx, int fmt,
+                        int rounding, uint64_t seed, void *q_t, void *sf_mma, int *d_status,
+                        bq_stream_t stream);
+
 /* ---- weight scale prepack (off the hot path) --------------------------- */
 
 enum {
@@ -187,6 +229,17 @@ int bq_gemm_mxfp8_mxfp8(const void *a_q, const void *a_sf, const void *b_e4m3, c
 int bq_gemm_mxfp4_mxfp4(const void *a_fp4, const void *a_sf, const void *b_fp4, const void *b_sf,
                         int64_t M, int64_t N, int64_t K, void *y_bf16, bq_stream_t stream);
 
+/* bq_gemm_e5m2_mxfp8 -- the backward products: A holds E5M2 gradient codes
+ * with E8M0 scales per 32 along K (bq_grad_quant, or bq_quant_transposed with
+ * BQ_FMT_E5M2), B E4M3 codes with per-32 scales along K (bq_act_quant /
+ * bq_quant_transposed with BQ_FMT_E4M3), y = A B^T in bf16 (fp32 accumulate,
+ * kind::mxf8f6f4 with an E5M2 A operand).  dX = bq_gemm_e5m2_mxfp8(dY_q,
+ * W^T_q) with W^T quantized along the output dimension; dW =
+ * bq_gemm_e5m2_mxfp8(dY^T_q, X^T_q), both transposed along the token
+ * dimension.  Operand layouts, alignment and errors as the other GEMMs. */
+int bq_gemm_e5m2_mxfp8(const void *a_e5m2, const void *a_sf, const void *b_e4m3, const void *b_sf,
+                       int64_t M, int64_t N, int64_t K, void *y_bf16, bq_stream_t stream);
+
 enum { BQ_ACT_NONE = 0, BQ_ACT_GELU = 1 };
 
 /* Fused epilogue, applied in fp32 with one bf16 rounding at the end:
@@ -258,7 +311,7 @@ typedef struct {
 
 /* Workspace bytes the *_epilogue calls need for a problem (0 when the chosen
  * schedule needs none).  weight_kind: 0 mxfp4, 1 fp8blk32, 2 mxfp8, 3 mxfp4 weights
- * with MXFP4 activations (bq_gemm_mxfp4_mxfp4*). */
+ * with MXFP4 activations (bq_gemm_mxfp4_mxfp4*), 4 E5M2 x MXFP8 (bq_gemm_e5m2_mxfp8*). */
 size_t bq_gemm_workspace_bytes(int weight_kind, int64_t M, int64_t N, int64_t K, int64_t batch,
                                const bq_gemm_config *cfg);
 
@@ -298,6 +351,12 @@ int bq_gemm_mxfp8_mxfp8_epilogue(const void *a_q, const void *a_sf, const void *
                                  const bq_epilogue *epi, const bq_batch *batch, void *workspace,
                                  size_t workspace_bytes, const bq_gemm_config *cfg,
                                  bq_stream_t stream);
+/* E5M2 x MXFP8 (bq_gemm_e5m2_mxfp8) with the same options. */
+int bq_gemm_e5m2_mxfp8_epilogue(const void *a_e5m2, const void *a_sf, const void *b_e4m3,
+                                const void *b_sf, int64_t M, int64_t N, int64_t K, void *y_bf16,
+                                const bq_epilogue *epi, const bq_batch *batch, void *workspace,
+                                size_t workspace_bytes, const bq_gemm_config *cfg,
+                                bq_stream_t stream);
 /* A4W4 (bq_gemm_mxfp4_mxfp4) with the same epilogue, batch, workspace and
  * schedule options; cta_pair 2 is refused (BQ_ERR_INVALID). */
 int bq_gemm_mxfp4_mxfp4_epilogue(const void *a_fp4, const void *a_sf, const void *b_fp4,
