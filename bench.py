@@ -137,13 +137,18 @@ def gemm_bytes(layer, quant_out=False):
 
 # ------------------------------------------------------- profile evidence --
 
+# The sources a GEMM launch is built and configured from (kernels, PTX
+# wrappers, the epilogue's quantizer arithmetic, the host dispatch).
+GEMM_SOURCES = ("gemm_bs.cuh", "gemm_pair.cuh", "bq_ptx.cuh", "mx_quant.cuh", "bq_api.cu")
+
+
 def kernel_source_sha():
-    """Hash of the CUDA sources and the header: a stored DRAM-traffic figure
-    is used only while the kernels it was measured on are unchanged."""
-    import glob
+    """Hash of the GEMM's sources and the header: a stored DRAM-traffic
+    figure is used only while the kernel it was measured on is unchanged."""
     import hashlib
     h = hashlib.sha256()
-    files = sorted(glob.glob(os.path.join(ROOT, "block_scaled_precision_quant_b200", "csrc", "*")))
+    files = [os.path.join(ROOT, "block_scaled_precision_quant_b200", "csrc", f)
+             for f in GEMM_SOURCES]
     files.append(os.path.join(ROOT, "include", "bq.h"))
     for f in files:
         with open(f, "rb") as fh:

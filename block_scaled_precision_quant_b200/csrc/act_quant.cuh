@@ -16,6 +16,7 @@
 #include <stdint.h>
 
 #include "bq_ptx.cuh"
+#include "grad_quant.cuh"
 #include "mx_quant.cuh"
 
 namespace bq {
@@ -42,10 +43,8 @@ __device__ __forceinline__ void e5m2_encode16(const uint32_t (&w)[8], int e, uin
     }
     if constexpr (SR) {
       const Philox4 r = philox4x64_10((idx0 >> 2) + i, seed);
-      codes[i] = e5m2_sr(f[0], philox_uniform(r.w[0])) |
-                 (e5m2_sr(f[1], philox_uniform(r.w[1])) << 8) |
-                 (e5m2_sr(f[2], philox_uniform(r.w[2])) << 16) |
-                 (e5m2_sr(f[3], philox_uniform(r.w[3])) << 24);
+      codes[i] = e5m2_sr(f[0], r.w[0]) | (e5m2_sr(f[1], r.w[1]) << 8) |
+                 (e5m2_sr(f[2], r.w[2]) << 16) | (e5m2_sr(f[3], r.w[3]) << 24);
     } else {
       codes[i] = e5m2x2(f[0], f[1]) | (e5m2x2(f[2], f[3]) << 16);
     }
@@ -136,10 +135,13 @@ __global__ void __launch_bounds__(256) act_quant_kernel(
 // rule; SR: the draw of element (r, c) is index r * C + c under `seed`).
 //
 // A warp owns 32 rows x 64 columns: lane l loads row r0 + l (64 values, 8 x
-// 16 B); the amax of every column over the 32 rows is a 5-step butterfly on
-// two columns per word (packed 16-bit maxima); each lane encodes its 64 values
-// with their columns' scales; the codes turn around through 2 KB of shared
-// memory per warp and leave as 32-byte pieces of the output rows.
+// 16 B).  The column maxima over the 32 rows come from a reduce-scatter of
+// the packed 16-bit magnitudes (two columns per word, recursive halving: 31
+// shuffles) that leaves lane l with columns 2l and 2l + 1; that lane forms
+// their scale exponents and stores their scale bytes, and 32 shuffles hand
+// every lane all 64 exponents.  Each lane encodes its 64 values, the codes
+// turn around through 2 KB of shared memory per warp and leave as 32-byte
+// pieces of the output rows.
 // grid.x = row group (32 rows), grid.y * 8 + warp = column tile (64 columns).
 // Tiles past C or past R/32 write padding scales (127) only.
 template <int FMT, bool SR>
@@ -174,6 +176,8 @@ __global__ void __launch_bounds__(256) quant_t_kernel(
     w[4 * v + 2] = t.z;
     w[4 * v + 3] = t.w;
   }
+  // reduce-scatter of the column maxima: after the step of distance k the
+  // lane keeps k words (the upper half when lane bit k is set)
   uint32_t m[32];
   uint32_t bad = 0;
 #pragma unroll
@@ -183,47 +187,58 @@ __global__ void __launch_bounds__(256) quant_t_kernel(
   }
 #pragma unroll
   for (int k = 16; k >= 1; k >>= 1) {
+    const bool up = (lane & k) != 0;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) m[i] = __vmaxu2(m[i], __shfl_xor_sync(0xFFFFFFFFu, m[i], k));
+    for (int i = 0; i < k; ++i) {
+      const uint32_t send = up ? m[i] : m[i + k];
+      const uint32_t keep = up ? m[i + k] : m[i];
+      m[i] = __vmaxu2(keep, __shfl_xor_sync(0xFFFFFFFFu, send, k));
+    }
   }
   if (bad && status && rows_ok) atomicOr(status, 1);
+  // lane l: columns 2l, 2l + 1 -> scale bytes (padding 127), packed pair
+  uint32_t pe;
+  {
+    const uint32_t a0 = m[0] & 0xFFFFu, a1 = m[0] >> 16;
+    const int e0 = FMT == kQE5M2 ? mx_exponent_e5m2(a0) : mx_exponent(a0);
+    const int e1 = FMT == kQE5M2 ? mx_exponent_e5m2(a1) : mx_exponent(a1);
+    pe = static_cast<uint32_t>(e0 + 127) | (static_cast<uint32_t>(e1 + 127) << 8);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int64_t c = c0 + 2 * lane + h;
+      const uint32_t b = (rows_ok && c < C) ? ((pe >> (8 * h)) & 0xFFu) : 127u;
+      sf_mma[sf_mma_offset(c, g, katoms)] = static_cast<uint8_t>(b);
+    }
+  }
 
   uint8_t *st = stage[warp];
   const int64_t row = r0 + lane;
-  int e_lo = 0, e_hi = 0;  // the exponents of columns c0 + lane and c0 + lane + 32
-  Philox4 rnd;             // SR: the draws of the current 4 columns
+  Philox4 rnd;  // SR: the draws of the current 4 columns
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
-    const uint32_t a0 = m[i] & 0xFFFFu, a1 = m[i] >> 16;
-    const int e0 = FMT == kQE5M2 ? mx_exponent_e5m2(a0) : mx_exponent(a0);
-    const int e1 = FMT == kQE5M2 ? mx_exponent_e5m2(a1) : mx_exponent(a1);
-    if (2 * i == lane) e_lo = e0;
-    if (2 * i + 1 == lane) e_lo = e1;
-    if (2 * i == lane + 32) e_hi = e0;
-    if (2 * i + 1 == lane + 32) e_hi = e1;
-    const float inv0 = __uint_as_float(static_cast<uint32_t>(127 - e0) << 23);
-    const float inv1 = __uint_as_float(static_cast<uint32_t>(127 - e1) << 23);
-    const float lim = FMT == kQE5M2 ? 57344.0f : 448.0f;
-    const float f0 =
-        fminf(fmaxf(__fmul_rn(__uint_as_float(w[i] << 16), inv0), -lim), lim);
-    const float f1 =
-        fminf(fmaxf(__fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), inv1), -lim), lim);
+    const uint32_t p = __shfl_sync(0xFFFFFFFFu, pe, i);  // scale bytes of columns 2i, 2i + 1
+    const float inv0 = __uint_as_float((254u - (p & 0xFFu)) << 23);  // 2^-e
+    const float inv1 = __uint_as_float((254u - (p >> 8)) << 23);
+    // |x| / 2^e never exceeds the format's largest value for bf16 input; the
+    // satfinite conversions would clamp it anyway
+    const float f0 = __fmul_rn(__uint_as_float(w[i] << 16), inv0);
+    const float f1 = __fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), inv1);
     uint32_t b0, b1;
     if constexpr (SR) {
       // draws of columns c0 + 2i, c0 + 2i + 1: one Philox block serves 4
       // columns (row * C + c0 is a multiple of 4: C % 8 == 0, c0 % 64 == 0)
       if (i % 2 == 0)
         rnd = philox4x64_10(static_cast<uint64_t>(row * C + c0 + 2 * i) >> 2, seed);
-      b0 = e5m2_sr(f0, philox_uniform(rnd.w[(2 * i) & 3]));
-      b1 = e5m2_sr(f1, philox_uniform(rnd.w[((2 * i) & 3) + 1]));
+      b0 = e5m2_sr(fminf(fmaxf(f0, -57344.0f), 57344.0f), rnd.w[(2 * i) & 3]);
+      b1 = e5m2_sr(fminf(fmaxf(f1, -57344.0f), 57344.0f), rnd.w[((2 * i) & 3) + 1]);
     } else if constexpr (FMT == kQE5M2) {
-      const uint32_t p = e5m2x2(f0, f1);
-      b0 = p & 0xFFu;
-      b1 = p >> 8;
+      const uint32_t pk = e5m2x2(f0, f1);
+      b0 = pk & 0xFFu;
+      b1 = pk >> 8;
     } else {
-      const uint32_t p = e4m3x4(f0, f1, 0.0f, 0.0f);
-      b0 = p & 0xFFu;
-      b1 = (p >> 8) & 0xFFu;
+      const uint32_t pk = e4m3x4(f0, f1, 0.0f, 0.0f);
+      b0 = pk & 0xFFu;
+      b1 = (pk >> 8) & 0xFFu;
     }
     st[(2 * i) * 32 + lane] = static_cast<uint8_t>(b0);
     st[(2 * i + 1) * 32 + lane] = static_cast<uint8_t>(b1);
@@ -240,14 +255,6 @@ __global__ void __launch_bounds__(256) quant_t_kernel(
         dst[1] = src[1];
       }
     }
-  }
-  // scales of columns c0 + lane and c0 + lane + 32 (padding: 127)
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int j = lane + 32 * h;
-    const uint32_t b = (rows_ok && c0 + j < C) ? static_cast<uint32_t>((h ? e_hi : e_lo) + 127)
-                                              : 127u;
-    sf_mma[sf_mma_offset(c0 + j, g, katoms)] = static_cast<uint8_t>(b);
   }
 }
 
