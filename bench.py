@@ -80,7 +80,7 @@ WORKLOADS = {
     # down-projection, T = 4096 tokens, N = 1536, K = 6144.
     "backward": dict(
         desc="backward of a 4096x1536x6144 linear layer: E5M2 stochastic gradient quantization "
-             "(row-wise and transposed), transposed E4M3 quantization of x and W, "
+             "(row-wise and transposed in one pass), transposed E4M3 quantization of x and W, "
              "dX = dY W and dW = dY^T x on E5M2 x MXFP8 GEMMs",
         layers=[("bwd", "grad", 4096, 1536, 6144, 1, dict())], bound="tensor"),
 }
@@ -432,12 +432,12 @@ class BackwardLayer:
         n = 0
         if which in ("all", "act_quant"):
             seed = 1000 + s  # a fresh stochastic-rounding seed per input set
-            bq.grad_quant(d["x"], stochastic=True, seed=seed, q=self.gq, sf_mma=self.gsf)
+            # dY along N (for dX) and along T (for dW) in one pass, shared draws
+            bq.grad_quant_dual(d["x"], stochastic=True, seed=seed,
+                               out=(self.gq, self.gsf, self.gtq, self.gtsf))
             bq.quant_transposed(d["w"], fmt=bq.BQ_FMT_E4M3, q=self.wtq, sf_mma=self.wtsf)
-            bq.quant_transposed(d["x"], fmt=bq.BQ_FMT_E5M2, stochastic=True, seed=seed + 1,
-                                q=self.gtq, sf_mma=self.gtsf)
             bq.quant_transposed(d["xin"], fmt=bq.BQ_FMT_E4M3, q=self.xtq, sf_mma=self.xtsf)
-            n += 4
+            n += 3
         if which in ("all", "gemm"):
             bq.gemm(bq.W_GRAD, self.gq, self.gsf, self.wtq, self.wtsf, T, K, N, y=self.y,
                     workspace=self.ws)

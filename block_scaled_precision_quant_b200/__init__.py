@@ -50,7 +50,7 @@ EXPORTS = (
     "bq_device_report", "bq_gemm_mxfp8_mxfp4_epilogue_noalloc", "bq_noalloc_scratch_bytes",
     "bq_gemm_bf16act_epilogue", "bq_gemm_plan", "bq_act_quant_mxfp4", "bq_gemm_mxfp4_mxfp4",
     "bq_gemm_mxfp4_mxfp4_epilogue", "bq_grad_quant", "bq_quant_transposed", "bq_gemm_e5m2_mxfp8",
-    "bq_gemm_e5m2_mxfp8_epilogue",
+    "bq_gemm_e5m2_mxfp8_epilogue", "bq_grad_quant_dual",
 )
 
 
@@ -111,6 +111,9 @@ def lib():
         L.bq_quant_transposed.argtypes = [vp, i64, i64, i64, i32, i32, ctypes.c_uint64, vp, vp,
                                           vp, vp]
         L.bq_quant_transposed.restype = i32
+        L.bq_grad_quant_dual.argtypes = [vp, i64, i64, i64, i32, ctypes.c_uint64, vp, vp, vp, vp,
+                                         vp, vp]
+        L.bq_grad_quant_dual.restype = i32
         L.bq_pack_weight_scales.argtypes = [vp, i32, i64, i64, vp, vp, vp]
         L.bq_pack_weight_scales.restype = i32
         L.bq_unpack_scales.argtypes = [vp, i64, i64, vp, vp]
@@ -263,6 +266,28 @@ def grad_quant(g, stochastic=False, seed=0, q=None, sf_mma=None, sf_rowmajor=Non
                                BQ_ROUND_STOCHASTIC if stochastic else BQ_ROUND_NEAREST,
                                int(seed) & (2 ** 64 - 1), _stream()), "bq_grad_quant")
     return q, sf_mma
+
+
+def grad_quant_dual(g, stochastic=False, seed=0, out=None, status=None):
+    """Both E5M2 quantizations of a bf16 [R, C] gradient in one pass: returns
+    (q_row [R, C], sf_row, q_t [C, R], sf_t), equal to grad_quant(g) and
+    quant_transposed(g, BQ_FMT_E5M2) with the same seed."""
+    torch = _torch()
+    _need_cuda(g)
+    if g.dtype != torch.bfloat16 or g.dim() != 2 or g.stride(1) != 1:
+        raise ValueError("g must be a bf16 [R, C] tensor with unit column stride")
+    R, C = g.shape
+    if out is None:
+        u8 = dict(dtype=torch.uint8, device=g.device)
+        out = (torch.empty((R, C), **u8), torch.empty((max(sf_bytes(R, C), 1),), **u8),
+               torch.empty((C, R), **u8), torch.empty((max(sf_bytes(C, R), 1),), **u8))
+    q_row, sf_row, q_t, sf_t = out
+    _check(lib().bq_grad_quant_dual(_ptr(g), R, C, g.stride(0),
+                                    BQ_ROUND_STOCHASTIC if stochastic else BQ_ROUND_NEAREST,
+                                    int(seed) & (2 ** 64 - 1), _ptr(q_row), _ptr(sf_row),
+                                    _ptr(q_t), _ptr(sf_t), _ptr(status), _stream()),
+           "bq_grad_quant_dual")
+    return q_row, sf_row, q_t, sf_t
 
 
 def quant_transposed(x, fmt=BQ_FMT_E4M3, stochastic=False, seed=0, q=None, sf_mma=None,

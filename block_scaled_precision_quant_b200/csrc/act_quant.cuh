@@ -26,11 +26,12 @@ enum QuantFmt : int { kQE4M3 = 0, kQFP4 = 1, kQE5M2 = 2 };
 
 // E5M2 codes of 16 bf16 values (8 words, element 2i in the low half of word
 // i) scaled by 2^-e; SR: stochastic rounding with the draws of elements
-// idx0 .. idx0 + 15 (idx0 a multiple of 4) under `seed`.
+// idx0 .. idx0 + 15 (idx0 a multiple of 8: two Philox blocks) under `seed`.
 template <bool SR>
 __device__ __forceinline__ void e5m2_encode16(const uint32_t (&w)[8], int e, uint64_t seed,
                                               uint64_t idx0, uint32_t (&codes)[4]) {
   const float inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e
+  Philox4 r;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     float f[4];
@@ -42,9 +43,11 @@ __device__ __forceinline__ void e5m2_encode16(const uint32_t (&w)[8], int e, uin
           fminf(fmaxf(__fmul_rn(__uint_as_float(word & 0xFFFF0000u), inv), -57344.0f), 57344.0f);
     }
     if constexpr (SR) {
-      const Philox4 r = philox4x64_10((idx0 >> 2) + i, seed);
-      codes[i] = e5m2_sr(f[0], r.w[0]) | (e5m2_sr(f[1], r.w[1]) << 8) |
-                 (e5m2_sr(f[2], r.w[2]) << 16) | (e5m2_sr(f[3], r.w[3]) << 24);
+      if (i % 2 == 0) r = philox4x64_10((idx0 >> 3) + (i >> 1), seed);
+      const int j0 = (4 * i) & 7;
+      codes[i] = e5m2_sr(f[0], philox_draw(r, j0)) | (e5m2_sr(f[1], philox_draw(r, j0 + 1)) << 8) |
+                 (e5m2_sr(f[2], philox_draw(r, j0 + 2)) << 16) |
+                 (e5m2_sr(f[3], philox_draw(r, j0 + 3)) << 24);
     } else {
       codes[i] = e5m2x2(f[0], f[1]) | (e5m2x2(f[2], f[3]) << 16);
     }
@@ -213,7 +216,7 @@ __global__ void __launch_bounds__(256) quant_t_kernel(
 
   uint8_t *st = stage[warp];
   const int64_t row = r0 + lane;
-  Philox4 rnd;  // SR: the draws of the current 4 columns
+  Philox4 rnd;  // SR: the draws of the current 8 columns
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
     const uint32_t p = __shfl_sync(0xFFFFFFFFu, pe, i);  // scale bytes of columns 2i, 2i + 1
@@ -225,12 +228,12 @@ __global__ void __launch_bounds__(256) quant_t_kernel(
     const float f1 = __fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), inv1);
     uint32_t b0, b1;
     if constexpr (SR) {
-      // draws of columns c0 + 2i, c0 + 2i + 1: one Philox block serves 4
-      // columns (row * C + c0 is a multiple of 4: C % 8 == 0, c0 % 64 == 0)
-      if (i % 2 == 0)
-        rnd = philox4x64_10(static_cast<uint64_t>(row * C + c0 + 2 * i) >> 2, seed);
-      b0 = e5m2_sr(fminf(fmaxf(f0, -57344.0f), 57344.0f), rnd.w[(2 * i) & 3]);
-      b1 = e5m2_sr(fminf(fmaxf(f1, -57344.0f), 57344.0f), rnd.w[((2 * i) & 3) + 1]);
+      // draws of columns c0 + 2i, c0 + 2i + 1: one Philox block serves 8
+      // columns (row * C + c0 is a multiple of 8: C % 8 == 0, c0 % 64 == 0)
+      if (i % 4 == 0)
+        rnd = philox4x64_10(static_cast<uint64_t>(row * C + c0 + 2 * i) >> 3, seed);
+      b0 = e5m2_sr(fminf(fmaxf(f0, -57344.0f), 57344.0f), philox_draw(rnd, (2 * i) & 7));
+      b1 = e5m2_sr(fminf(fmaxf(f1, -57344.0f), 57344.0f), philox_draw(rnd, ((2 * i) & 7) + 1));
     } else if constexpr (FMT == kQE5M2) {
       const uint32_t pk = e5m2x2(f0, f1);
       b0 = pk & 0xFFu;
@@ -256,6 +259,218 @@ __global__ void __launch_bounds__(256) quant_t_kernel(
       }
     }
   }
+}
+
+// Transposed quantization with round to nearest even (E4M3, or E5M2 without
+// stochastic rounding): a warp owns 32 rows x 64 columns and lane l the two
+// columns c0 + 2l, c0 + 2l + 1 -- one 4-byte load per row, so every warp load
+// is one 128-byte row segment.  A lane's two columns are whole groups: their
+// maxima, scales and codes need no other lane, and each output row (one
+// column, 32 codes) leaves from its lane as two 16-byte stores.
+// grid.x = row group (32 rows), grid.y * 8 + warp = column tile (64 columns).
+template <int FMT>
+__global__ void __launch_bounds__(256) quant_t_rne_kernel(
+    const __nv_bfloat16 *__restrict__ x, int64_t R, int64_t C, int64_t ldx, int64_t col_tiles,
+    uint8_t *__restrict__ q, uint8_t *__restrict__ sf_mma, int *__restrict__ status) {
+  static_assert(FMT == kQE4M3 || FMT == kQE5M2, "E4M3 or E5M2 codes");
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t ct = static_cast<int64_t>(blockIdx.y) * 8 + warp;
+  if (ct >= col_tiles) return;
+  const int64_t c = ct * 64 + 2 * lane;  // this lane's first column
+  const int64_t g = blockIdx.x;
+  const int64_t r0 = g * 32;
+  const int64_t G = R >> 5;
+  const int64_t katoms = (G + 3) >> 2;
+  const bool ok = g < G && c < C;  // C % 8 == 0: both columns or neither
+  griddep_wait();
+  griddep_launch_dependents();
+
+  uint32_t w[32];  // row r0 + r: column c (low half), c + 1 (high half)
+#pragma unroll
+  for (int r = 0; r < 32; ++r)
+    w[r] = ok ? __ldg(reinterpret_cast<const unsigned int *>(x + (r0 + r) * ldx + c)) : 0u;
+  uint32_t m = 0;
+#pragma unroll
+  for (int r = 0; r < 32; ++r) m = __vmaxu2(m, w[r] & 0x7FFF7FFFu);
+  const uint32_t a0 = m & 0xFFFFu, a1 = m >> 16;
+  if (ok && (a0 >= 0x7F80u || a1 >= 0x7F80u) && status) atomicOr(status, 1);
+  const int e0 = FMT == kQE5M2 ? mx_exponent_e5m2(a0) : mx_exponent(a0);
+  const int e1 = FMT == kQE5M2 ? mx_exponent_e5m2(a1) : mx_exponent(a1);
+  sf_mma[sf_mma_offset(c, g, katoms)] = static_cast<uint8_t>(ok ? e0 + 127 : 127);
+  sf_mma[sf_mma_offset(c + 1, g, katoms)] = static_cast<uint8_t>(ok ? e1 + 127 : 127);
+  if (!ok) return;
+  const float inv0 = __uint_as_float(static_cast<uint32_t>(127 - e0) << 23);  // 2^-e
+  const float inv1 = __uint_as_float(static_cast<uint32_t>(127 - e1) << 23);
+  uint32_t out0[8], out1[8];  // the codes of columns c and c + 1, rows r0 .. r0 + 31
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    uint32_t p[4];  // rows 4j .. 4j + 3: byte 0 column c, byte 1 column c + 1
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const uint32_t v = w[4 * j + t];
+      const float f0 = __fmul_rn(__uint_as_float(v << 16), inv0);
+      const float f1 = __fmul_rn(__uint_as_float(v & 0xFFFF0000u), inv1);
+      p[t] = FMT == kQE5M2 ? e5m2x2(f0, f1) : e4m3x2(f0, f1);
+    }
+    const uint32_t lo = __byte_perm(p[0], p[1], 0x5140), hi = __byte_perm(p[2], p[3], 0x5140);
+    out0[j] = __byte_perm(lo, hi, 0x5410);
+    out1[j] = __byte_perm(lo, hi, 0x7632);
+  }
+  uint4 *d0 = reinterpret_cast<uint4 *>(q + c * R + r0);
+  uint4 *d1 = reinterpret_cast<uint4 *>(q + (c + 1) * R + r0);
+  d0[0] = make_uint4(out0[0], out0[1], out0[2], out0[3]);
+  d0[1] = make_uint4(out0[4], out0[5], out0[6], out0[7]);
+  d1[0] = make_uint4(out1[0], out1[1], out1[2], out1[3]);
+  d1[1] = make_uint4(out1[4], out1[5], out1[6], out1[7]);
+}
+
+// Both quantizations of a gradient in one pass (the output gradient dY feeds
+// dX = dY W, contracting over its columns, and dW = dY^T x, contracting over
+// its rows): g bf16 [R, ldg] (C columns) -> E5M2 codes q_row [R, C] with
+// scales along C (bq_grad_quant) and q_t [C, R] with scales along R
+// (bq_quant_transposed), each element's stochastic draw (index r * C + c
+// under `seed`) drawn once and used by both.  R % 32 == 0, C % 32 == 0.
+// The warp tile, the column reduce-scatter and the transposed store are those
+// of quant_t_kernel; a lane's 64 values of one row are two row groups whose
+// maxima need no shuffles, and its 64 row codes leave as four 16-byte stores.
+template <bool SR>
+__global__ void __launch_bounds__(256, 3) grad_quant_dual_kernel(
+    const __nv_bfloat16 *__restrict__ x, int64_t R, int64_t C, int64_t ldx, int64_t col_tiles,
+    int64_t row_tiles, uint8_t *__restrict__ q_row, uint8_t *__restrict__ sf_row,
+    uint8_t *__restrict__ q_t, uint8_t *__restrict__ sf_t, int *__restrict__ status,
+    uint64_t seed) {
+  __shared__ __align__(16) uint8_t stage[8][64 * 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t ct = static_cast<int64_t>(blockIdx.y) * 8 + warp;
+  if (ct >= col_tiles) return;  // whole warps leave; only warp-level sync below
+  const int64_t c0 = ct * 64;
+  const int64_t g = blockIdx.x;  // 32-row group
+  const int64_t r0 = g * 32;
+  const int64_t G_t = R >> 5, G_r = C >> 5;  // groups per row of q_t, of q_row
+  const int64_t katoms_t = (G_t + 3) >> 2, katoms_r = (G_r + 3) >> 2;
+  const bool rows_ok = g < G_t;
+  griddep_wait();
+  griddep_launch_dependents();
+
+  uint32_t w[32];
+#pragma unroll
+  for (int v = 0; v < 8; ++v) {
+    uint4 t = make_uint4(0u, 0u, 0u, 0u);
+    const int64_t c = c0 + v * 8;
+    if (rows_ok && c < C)
+      t = __ldg(reinterpret_cast<const uint4 *>(x + (r0 + lane) * ldx + c));
+    w[4 * v] = t.x;
+    w[4 * v + 1] = t.y;
+    w[4 * v + 2] = t.z;
+    w[4 * v + 3] = t.w;
+  }
+  uint32_t m[32];
+  uint32_t rmax[2] = {0u, 0u};  // this row's two 32-column groups
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    m[i] = w[i] & 0x7FFF7FFFu;
+    rmax[i / 16] = max(rmax[i / 16], max(m[i] & 0xFFFFu, m[i] >> 16));
+  }
+#pragma unroll
+  for (int k = 16; k >= 1; k >>= 1) {
+    const bool up = (lane & k) != 0;
+#pragma unroll
+    for (int i = 0; i < k; ++i) {
+      const uint32_t send = up ? m[i] : m[i + k];
+      const uint32_t keep = up ? m[i + k] : m[i];
+      m[i] = __vmaxu2(keep, __shfl_xor_sync(0xFFFFFFFFu, send, k));
+    }
+  }
+  // lane l: transposed scales of columns 2l, 2l + 1
+  uint32_t pe;
+  {
+    const uint32_t a0 = m[0] & 0xFFFFu, a1 = m[0] >> 16;
+    if ((a0 >= 0x7F80u || a1 >= 0x7F80u) && status && rows_ok) atomicOr(status, 1);
+    pe = static_cast<uint32_t>(mx_exponent_e5m2(a0) + 127) |
+         (static_cast<uint32_t>(mx_exponent_e5m2(a1) + 127) << 8);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int64_t c = c0 + 2 * lane + h;
+      const uint32_t b = (rows_ok && c < C) ? ((pe >> (8 * h)) & 0xFFu) : 127u;
+      sf_t[sf_mma_offset(c, g, katoms_t)] = static_cast<uint8_t>(b);
+    }
+  }
+  // this row's scales; the row-wise buffer's padding rows and groups are
+  // written by the tiles that cover them
+  const int64_t row = r0 + lane;
+  const int er0 = mx_exponent_e5m2(rmax[0]), er1 = mx_exponent_e5m2(rmax[1]);
+  {
+    const int64_t rows_pad_r = (R + 127) / 128 * 128;
+    const int64_t gc = c0 >> 5;  // first row group of this tile's columns
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const bool valid = rows_ok && c0 + 32 * h < C;
+      if (row < rows_pad_r && gc + h < katoms_r * 4)
+        sf_row[sf_mma_offset(row, gc + h, katoms_r)] =
+            static_cast<uint8_t>(valid ? (h ? er1 : er0) + 127 : 127);
+    }
+  }
+  const float rinv0 = __uint_as_float(static_cast<uint32_t>(127 - er0) << 23);
+  const float rinv1 = __uint_as_float(static_cast<uint32_t>(127 - er1) << 23);
+
+  uint8_t *st = stage[warp];
+  Philox4 rnd;
+  uint32_t rowc[16];  // this row's 64 codes, four per word
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const uint32_t p = __shfl_sync(0xFFFFFFFFu, pe, i);
+    const float inv0 = __uint_as_float((254u - (p & 0xFFu)) << 23);
+    const float inv1 = __uint_as_float((254u - (p >> 8)) << 23);
+    const float rinv = i < 16 ? rinv0 : rinv1;
+    const float x0 = __uint_as_float(w[i] << 16), x1 = __uint_as_float(w[i] & 0xFFFF0000u);
+    const float t0 = __fmul_rn(x0, inv0), t1 = __fmul_rn(x1, inv1);  // transposed scaling
+    const float r0f = __fmul_rn(x0, rinv), r1f = __fmul_rn(x1, rinv);  // row-wise scaling
+    uint32_t bt0, bt1, br0, br1;
+    if constexpr (SR) {
+      if (i % 4 == 0)
+        rnd = philox4x64_10(static_cast<uint64_t>(row * C + c0 + 2 * i) >> 3, seed);
+      const uint32_t u0 = philox_draw(rnd, (2 * i) & 7), u1 = philox_draw(rnd, ((2 * i) & 7) + 1);
+      bt0 = e5m2_sr(fminf(fmaxf(t0, -57344.0f), 57344.0f), u0);
+      bt1 = e5m2_sr(fminf(fmaxf(t1, -57344.0f), 57344.0f), u1);
+      br0 = e5m2_sr(fminf(fmaxf(r0f, -57344.0f), 57344.0f), u0);
+      br1 = e5m2_sr(fminf(fmaxf(r1f, -57344.0f), 57344.0f), u1);
+    } else {
+      const uint32_t pt = e5m2x2(t0, t1), pr = e5m2x2(r0f, r1f);
+      bt0 = pt & 0xFFu;
+      bt1 = pt >> 8;
+      br0 = pr & 0xFFu;
+      br1 = pr >> 8;
+    }
+    st[(2 * i) * 32 + lane] = static_cast<uint8_t>(bt0);
+    st[(2 * i + 1) * 32 + lane] = static_cast<uint8_t>(bt1);
+    const uint32_t pair = br0 | (br1 << 8);
+    if (i % 2 == 0)
+      rowc[i / 2] = pair;
+    else
+      rowc[i / 2] |= pair << 16;
+  }
+  if (rows_ok) {
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      if (c0 + 16 * v < C)
+        *reinterpret_cast<uint4 *>(q_row + row * C + c0 + 16 * v) =
+            make_uint4(rowc[4 * v], rowc[4 * v + 1], rowc[4 * v + 2], rowc[4 * v + 3]);
+    }
+  }
+  __syncwarp();
+  if (rows_ok) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int j = 2 * lane + h;
+      if (c0 + j < C) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(st + j * 32);
+        uint4 *dst = reinterpret_cast<uint4 *>(q_t + (c0 + j) * R + r0);
+        dst[0] = src[0];
+        dst[1] = src[1];
+      }
+    }
+  }
+  (void)row_tiles;
 }
 
 // Row-major scales (ROW32: [N, G]; BLK32x32: [ceil(N/32), G] repeated over

@@ -810,12 +810,55 @@ int quant_t_launch(int fmt, bool sr, uint64_t seed, const void* x_bf16, int64_t 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = 1;
-  auto kern = fmt == bq::kQE5M2 ? (sr ? bq::quant_t_kernel<bq::kQE5M2, true>
-                                      : bq::quant_t_kernel<bq::kQE5M2, false>)
-                                : bq::quant_t_kernel<bq::kQE4M3, false>;
-  if (cudaLaunchKernelEx(&lc, kern, static_cast<const __nv_bfloat16*>(x_bf16), R, C, ldx,
-                         col_tiles, static_cast<uint8_t*>(q_t), static_cast<uint8_t*>(sf_mma),
-                         d_status, seed) != cudaSuccess) {
+  cudaError_t e;
+  if (sr) {  // stochastic: the row-per-lane kernel, one Philox block per 4 columns
+    e = cudaLaunchKernelEx(&lc, bq::quant_t_kernel<bq::kQE5M2, true>,
+                           static_cast<const __nv_bfloat16*>(x_bf16), R, C, ldx, col_tiles,
+                           static_cast<uint8_t*>(q_t), static_cast<uint8_t*>(sf_mma), d_status,
+                           seed);
+  } else {
+    auto kern = fmt == bq::kQE5M2 ? bq::quant_t_rne_kernel<bq::kQE5M2>
+                                  : bq::quant_t_rne_kernel<bq::kQE4M3>;
+    e = cudaLaunchKernelEx(&lc, kern, static_cast<const __nv_bfloat16*>(x_bf16), R, C, ldx,
+                           col_tiles, static_cast<uint8_t*>(q_t), static_cast<uint8_t*>(sf_mma),
+                           d_status);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return BQ_ERR_CUDA;
+  }
+  return launch_status();
+}
+
+// Launch of the fused row-wise + transposed gradient quantizer.
+int grad_dual_launch(bool sr, uint64_t seed, const void* g_bf16, int64_t R, int64_t C,
+                     int64_t ldg, void* q_row, void* sf_row, void* q_t, void* sf_t,
+                     int* d_status, bq_stream_t stream) {
+  DevInfo* dev = nullptr;
+  int st = current_device(&dev);
+  if (st != BQ_OK) return st;
+  if (R < 0 || R % 32 != 0 || C <= 0 || C % 32 != 0 || ldg < C) return BQ_ERR_SHAPE;
+  if (R == 0) return BQ_OK;
+  if (!g_bf16 || !q_row || !sf_row || !q_t || !sf_t) return BQ_ERR_NULL;
+  if (!aligned(g_bf16, 16) || ldg % 8 != 0 || !aligned(q_row, 16) || !aligned(q_t, 16))
+    return BQ_ERR_ALIGN;
+  const int64_t col_tiles = (C + 127) / 128 * 128 / 64;
+  const int64_t groups_pad = (R / 32 + 3) / 4 * 4;
+  if (groups_pad > 0x7FFFFFFF || (col_tiles + 7) / 8 > 65535) return BQ_ERR_SHAPE;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(static_cast<unsigned>(groups_pad), static_cast<unsigned>((col_tiles + 7) / 8));
+  lc.blockDim = dim3(256);
+  lc.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  auto kern = sr ? bq::grad_quant_dual_kernel<true> : bq::grad_quant_dual_kernel<false>;
+  if (cudaLaunchKernelEx(&lc, kern, static_cast<const __nv_bfloat16*>(g_bf16), R, C, ldg,
+                         col_tiles, groups_pad, static_cast<uint8_t*>(q_row),
+                         static_cast<uint8_t*>(sf_row), static_cast<uint8_t*>(q_t),
+                         static_cast<uint8_t*>(sf_t), d_status, seed) != cudaSuccess) {
     cudaGetLastError();
     return BQ_ERR_CUDA;
   }
@@ -844,6 +887,14 @@ int bq_grad_quant(const void* g_bf16, int64_t M, int64_t K, int64_t ldg, void* q
   if (rounding != BQ_ROUND_NEAREST && rounding != BQ_ROUND_STOCHASTIC) return BQ_ERR_INVALID;
   return act_quant_launch(bq::kQE5M2, rounding == BQ_ROUND_STOCHASTIC, seed, g_bf16, M, K, ldg,
                           q_e5m2, sf_mma, sf_rowmajor, d_status, stream);
+}
+
+int bq_grad_quant_dual(const void* g_bf16, int64_t R, int64_t C, int64_t ldg, int rounding,
+                       uint64_t seed, void* q_row, void* sf_row, void* q_t, void* sf_t,
+                       int* d_status, bq_stream_t stream) {
+  if (rounding != BQ_ROUND_NEAREST && rounding != BQ_ROUND_STOCHASTIC) return BQ_ERR_INVALID;
+  return grad_dual_launch(rounding == BQ_ROUND_STOCHASTIC, seed, g_bf16, R, C, ldg, q_row, sf_row,
+                          q_t, sf_t, d_status, stream);
 }
 
 int bq_quant_transposed(const void* x_bf16, int64_t R, int64_t C, int64_t ldx, int fmt,

@@ -51,30 +51,41 @@ __device__ __forceinline__ Philox4 philox4x64_10(uint64_t c0, uint64_t k0) {
   return Philox4{{x0, x1, x2, x3}};
 }
 
-// Stochastic E5M2 rounding of y (|y| <= 57344) with the element's Philox
-// word: lo and hi are the E5M2 magnitudes around |y| -- truncation to two
-// mantissa bits for |y| >= 2^-14, the 2^-16 grid below -- and the result is
-// hi when u < (|y| - lo) / (hi - lo), u = (word >> 11) * 2^-53 the draw, with
-// y's sign; returns the code byte.  |y| - lo is exact (lo truncates |y| on its
-// own grid) and hi - lo is a power of two, so the fraction d is exact in fp32;
-// u < d is decided exactly in integers as (word >> 11) < ceil(d * 2^53).
-__device__ __forceinline__ uint32_t e5m2_sr(float y, uint64_t word) {
-  const float a = fabsf(y);
-  float lo, step, inv_step;
-  if (a >= 0x1.0p-14f) {
-    const uint32_t eb = __float_as_uint(a) & 0x7F800000u;  // 2^exp of |y|
-    lo = __uint_as_float(__float_as_uint(a) & ~((1u << 21) - 1u));
-    step = __uint_as_float(eb - (2u << 23));                     // 2^(exp - 2)
-    inv_step = __uint_as_float((254u << 23) - eb + (2u << 23));  // 2^(2 - exp)
+// The draw of element j (0..7) of a Philox block: the 32-bit half (j % 2, low
+// half first) of word j / 2.  A block at counter i / 8 serves elements i with
+// the same i / 8.
+__device__ __forceinline__ uint32_t philox_draw(const Philox4 &r, int j) {
+  const uint64_t w = r.w[(j >> 1) & 3];
+  return (j & 1) ? static_cast<uint32_t>(w >> 32) : static_cast<uint32_t>(w);
+}
+
+// Stochastic E5M2 rounding of y (|y| <= 57344) with the element's 32-bit
+// draw: lo and hi are the E5M2 magnitudes around |y| and the result is hi when
+// u < (|y| - lo) / (hi - lo), u = draw * 2^-32, with y's sign; returns the code
+// byte.
+//   |y| >= 2^-14 (E5M2 normal): lo is |y| truncated to two mantissa bits, its
+//     code (exponent rebiased from 127 to 15, two mantissa bits) is read off
+//     the fp32 bits, and the fraction is k / 2^21 with k the 21 dropped
+//     mantissa bits, so u < d exactly when (draw >> 11) < k.
+//   |y| < 2^-14 (E5M2 subnormal, step 2^-16): t = |y| 2^16 is exact, lo = floor
+//     t, the fraction t - lo is exact in fp32 and compared with the draw
+//     exactly as draw < ceil(frac 2^32).
+__device__ __forceinline__ uint32_t e5m2_sr(float y, uint32_t draw) {
+  const uint32_t bits = __float_as_uint(y);
+  const uint32_t sign = (bits >> 24) & 0x80u;
+  const uint32_t mag = bits & 0x7FFFFFFFu;
+  uint32_t code;
+  if (mag >= 0x38800000u) {  // 2^-14
+    const uint32_t k = mag & 0x1FFFFFu;
+    code = (mag >> 21) - (112u << 2) + ((draw >> 11) < k ? 1u : 0u);
   } else {
-    lo = floorf(a * 65536.0f) * 0x1.0p-16f;
-    step = 0x1.0p-16f;
-    inv_step = 65536.0f;
+    const float t = __fmul_rn(__uint_as_float(mag), 65536.0f);
+    const float lo = floorf(t);
+    const float frac = t - lo;
+    const uint64_t thr = __float2ull_rz(ceilf(__fmul_rn(frac, 0x1.0p32f)));
+    code = static_cast<uint32_t>(lo) + (static_cast<uint64_t>(draw) < thr ? 1u : 0u);
   }
-  const float d = __fmul_rn(a - lo, inv_step);                     // in [0, 1), exact
-  const uint64_t thr = __float2ull_rz(ceilf(__fmul_rn(d, 0x1.0p53f)));  // exact integer
-  const float m = ((word >> 11) < thr) ? lo + step : lo;               // an E5M2 value
-  return e5m2x2(copysignf(m, y), 0.0f) & 0xFFu;
+  return sign | code;
 }
 
 }  // namespace bq

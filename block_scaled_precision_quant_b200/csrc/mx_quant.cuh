@@ -32,6 +32,11 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+  return static_cast<uint32_t>(
+      __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
+}
+
 // Largest magnitude bits (15 bits, sign dropped) of the bf16 pairs in w: an
 // integer max is order-preserving for non-negative floats.  `bad` collects
 // non-finite inputs (all-ones exponent).

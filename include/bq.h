@@ -128,10 +128,11 @@ enum { BQ_FMT_E4M3 = 0, BQ_FMT_E5M2 = 1 };
  *   rounding BQ_ROUND_NEAREST: round to nearest even (saturating), sign kept.
  *   rounding BQ_ROUND_STOCHASTIC: between the two neighbouring E5M2 values of
  *            |g / 2^e| (lo, hi; the 2^-16 grid below 2^-14), hi when
- *            u < (|v| - lo) / (hi - lo), u the element's draw: the top 53 bits
- *            (times 2^-53) of word (i mod 4) of Philox4x64-10 at counter
- *            (i / 4, 0, 0, 0) under key (seed, 0), i = row * K + column, so the
- *            draws are a stateless function of (seed, element index).
+ *            u < (|v| - lo) / (hi - lo), u the element's draw times 2^-32: the
+ *            32-bit half (i mod 2, low half first) of word (i / 2) mod 4 of
+ *            Philox4x64-10 at counter (i / 8, 0, 0, 0) under key (seed, 0),
+ *            i = row * K + column, so the draws are a stateless function of
+ *            (seed, element index).
  *   g_bf16 [M, K] (row stride ldg), q_e5m2 out [M, K], sf_mma out
  *   bq_sf_bytes(M, K) (MMA layout), sf_rowmajor / d_status as bq_act_quant.
  * Errors: as bq_act_quant, BQ_ERR_INVALID for a bad rounding mode. */
@@ -155,6 +156,17 @@ int bq_grad_quant(const void *g_bf16, int64_t M, int64_t K, int64_t ldg, void *q
 int bq_quant_transposed(const void *x_bf16, int64_t R, int64_t C, int64_t ldx, int fmt,
                         int rounding, uint64_t seed, void *q_t, void *sf_mma, int *d_status,
                         bq_stream_t stream);
+
+/* bq_grad_quant_dual -- both quantizations of an output gradient g [R, C] in
+ * one pass: q_row [R, C] with scales along C (exactly bq_grad_quant) and q_t
+ * [C, R] with scales along R (exactly bq_quant_transposed with BQ_FMT_E5M2),
+ * reading g once and drawing each element's stochastic draw (index r * C + c
+ * under `seed`) once for both.  R % 32 == 0, C % 32 == 0, ldg >= C,
+ * ldg % 8 == 0; sf_row: bq_sf_bytes(R, C), sf_t: bq_sf_bytes(C, R); q_row and
+ * q_t 16-byte aligned.  Errors as bq_grad_quant. */
+int bq_grad_quant_dual(const void *g_bf16, int64_t R, int64_t C, int64_t ldg, int rounding,
+                       uint64_t seed, void *q_row, void *sf_row, void *q_t, void *sf_t,
+                       int *d_status, bq_stream_t stream);
 
 /* ---- weight scale prepack (off the hot path) --------------------------- */
 

@@ -238,13 +238,16 @@ void oracle_philox4x64_10(const uint64_t ctr[4], const uint64_t key[2], uint64_t
   out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
 }
 
-/* The uniform draw of element `index` under `seed`: word (index % 4) of
- * Philox4x64-10 at counter (index / 4, 0, 0, 0) with key (seed, 0), its top
- * 53 bits as a double in [0, 1). */
+/* The uniform draw of element `index` under `seed`: one Philox4x64-10 block
+ * (counter (index / 8, 0, 0, 0), key (seed, 0)) serves 8 elements, element
+ * index takes the 32-bit half (index % 2, low half first) of word
+ * (index / 2) % 4, as a double in [0, 1) with 2^-32 resolution. */
 double oracle_uniform(uint64_t seed, uint64_t index) {
-  uint64_t ctr[4] = {index >> 2, 0, 0, 0}, key[2] = {seed, 0}, out[4];
+  uint64_t ctr[4] = {index >> 3, 0, 0, 0}, key[2] = {seed, 0}, out[4];
   oracle_philox4x64_10(ctr, key, out);
-  return ldexp((double)(out[index & 3] >> 11), -53);
+  uint64_t word = out[(index >> 1) & 3];
+  uint32_t half = (uint32_t)((index & 1) ? (word >> 32) : (word & 0xFFFFFFFFu));
+  return ldexp((double)half, -32);
 }
 
 /* Stochastic E5M2 rounding of binary32 v (|v| <= 57344 after the clamp):

@@ -158,6 +158,25 @@ def test_quant_transposed_refusals():
     assert e.value.status == bq.BQ_ERR_SHAPE
 
 
+@pytest.mark.parametrize("R,C", [(32, 32), (96, 160), (160, 96), (4096, 1536)])
+@pytest.mark.parametrize("stochastic", [False, True])
+def test_grad_quant_dual_equals_both_quantizers(R, C, stochastic):
+    g = grads(R, C, seed=R * 3 + C)
+    q_row, sf_row, q_t, sf_t = bq.grad_quant_dual(dev_bf16(g), stochastic=stochastic, seed=21)
+    bq.device_status()
+    o_row, o_rs = oracle.grad_quant(g, stochastic=stochastic, seed=21)
+    o_t, o_ts = oracle.quant_transposed(g, oracle.Q_E5M2, stochastic=stochastic, seed=21)
+    assert np.array_equal(q_row.cpu().numpy(), o_row)
+    assert np.array_equal(q_t.cpu().numpy(), o_t)
+    rp, cp = (R + 127) // 128 * 128, (C + 127) // 128 * 128
+    full_r = bq.unpack_scales(sf_row, rp, cp).cpu().numpy()
+    full_t = bq.unpack_scales(sf_t, cp, rp).cpu().numpy()
+    assert np.array_equal(full_r[:R, :C // 32], o_rs)
+    assert np.array_equal(full_t[:C, :R // 32], o_ts)
+    assert np.all(full_r[R:, :] == 127) and np.all(full_r[:, C // 32:] == 127)
+    assert np.all(full_t[C:, :] == 127) and np.all(full_t[:, R // 32:] == 127)
+
+
 # ------------------------------------------------------- backward GEMMs ----
 
 def check_grad_gemm(aq, asf, b, bsf, M, N, K, config=None, workspace=None, what=""):
@@ -200,17 +219,16 @@ def backward_case(T, N, K, seed):
     dy = grads(T, N, seed=seed + 2)
     xd, wd, dyd = dev_bf16(x), dev_bf16(w), dev_bf16(dy)
     # dX [T, K] = dY W: contraction over N
-    gq, gsf = bq.grad_quant(dyd, stochastic=True, seed=11)
+    gq, gsf, gtq, gtsf = bq.grad_quant_dual(dyd, stochastic=True, seed=11)  # dY, dY^T [N, T]
     wtq, wtsf = bq.quant_transposed(wd, fmt=bq.BQ_FMT_E4M3)              # W^T [K, N]
     dx = bq.gemm(bq.W_GRAD, gq, gsf, wtq, wtsf, T, K, N)
     # dW [N, K] = dY^T X: contraction over T
-    gtq, gtsf = bq.quant_transposed(dyd, fmt=bq.BQ_FMT_E5M2, stochastic=True, seed=12)  # [N, T]
     xtq, xtsf = bq.quant_transposed(xd, fmt=bq.BQ_FMT_E4M3)              # X^T [K, T]
     dw = bq.gemm(bq.W_GRAD, gtq, gtsf, xtq, xtsf, N, K, T)
     bq.device_status()
     og, ogs = oracle.grad_quant(dy, stochastic=True, seed=11)
     owt, owts = oracle.quant_transposed(w, oracle.Q_E4M3)
-    ogt, ogts = oracle.quant_transposed(dy, oracle.Q_E5M2, stochastic=True, seed=12)
+    ogt, ogts = oracle.quant_transposed(dy, oracle.Q_E5M2, stochastic=True, seed=11)
     oxt, oxts = oracle.quant_transposed(x, oracle.Q_E4M3)
     assert np.array_equal(gq.cpu().numpy(), og)
     assert np.array_equal(wtq.cpu().numpy(), owt)

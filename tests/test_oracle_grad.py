@@ -83,15 +83,16 @@ def test_philox_matches_numpy(key, ctr):
 
 
 def test_uniform_draw_is_philox_word():
-    for seed, idx in ((0, 0), (5, 3), (99, 4), (2 ** 63, 12345)):
+    """Element i's draw: 32-bit half (i % 2) of word (i / 2) % 4 of the Philox
+    block at counter i / 8 (numpy's block j comes from counter j + 1)."""
+    for seed, idx in ((0, 0), (5, 3), (99, 12), (2 ** 63, 12345), (7, 8)):
+        blk = idx >> 3
+        ctr = [blk - 1, 0, 0, 0] if blk else [2 ** 64 - 1] * 4
         bg = np.random.Philox(key=np.array([seed, 0], dtype=np.uint64),
-                              counter=np.array([(idx >> 2) - 1 if idx >> 2 else 2 ** 64 - 1,
-                                                0 if idx >> 2 else 2 ** 64 - 1,
-                                                0 if idx >> 2 else 2 ** 64 - 1,
-                                                0 if idx >> 2 else 2 ** 64 - 1],
-                                               dtype=np.uint64))
-        word = int(bg.random_raw(4)[idx & 3])
-        assert oracle.uniform(seed, idx) == (word >> 11) * 2.0 ** -53
+                              counter=np.array(ctr, dtype=np.uint64))
+        word = int(bg.random_raw(4)[(idx >> 1) & 3])
+        half = (word >> 32) if idx & 1 else (word & 0xFFFFFFFF)
+        assert oracle.uniform(seed, idx) == half * 2.0 ** -32
     u = np.array([oracle.uniform(7, i) for i in range(20000)])
     assert u.min() >= 0.0 and u.max() < 1.0 and abs(u.mean() - 0.5) < 0.01
 
