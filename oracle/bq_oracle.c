@@ -25,10 +25,10 @@
  *     "hip_quant" README, "Stochastic E5M2 Backward Gradients" and "Block-wise
  *     FP8 Scaling") takes the same per-32 rule with E5M2's largest finite
  *     value 57344, rounding to nearest even or stochastically between the two
- *     neighbouring E5M2 values; the stochastic draw comes from a counter-based
- *     generator (Philox4x64-10) keyed by the seed and counted by the element's
- *     index, the "stateless per-element hash of (seed, element_index)" the page
- *     describes.
+ *     neighbouring E5M2 values; the page draws each element's random number
+ *     from its seed and its index with no state, which here is a
+ *     counter-based generator (Philox4x64-10) keyed by the seed and counted by
+ *     the element's index.
  *
  * Floating point: compile with -ffp-contract=off and without fast-math so that
  * every float expression below is one IEEE binary32 operation, as the page's

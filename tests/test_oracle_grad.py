@@ -4,11 +4,11 @@ to nearest even and stochastic), the transposed quantizer and the GEMM over
 E5M2 gradient codes.
 
 The "hip_quant" README on the pages describes E5M2 backward gradients with
-optional stochastic rounding ("rounds between adjacent E5M2 bins with
-probability proportional to the input value's distance between those bins,
-using a stateless per-element hash of (seed, element_index)") and block-wise
-scaling along the last dimension; the scale rule is the formats.py page's
-with 57344 in place of 448.  Pins: torch's float8_e5m2 for the format,
+optional stochastic rounding (the upper neighbour is taken with a probability
+that grows linearly with the value's position between the two E5M2 values,
+the random number a function of the seed and the element's index alone) and
+block-wise scaling along the last dimension; the scale rule is the formats.py
+page's with 57344 in place of 448.  Pins: torch's float8_e5m2 for the format,
 numpy's Philox bit generator for the draws, hand-worked scales, a numpy
 restatement, the stochastic rule's bracket and frequency, the plain
 definition of the transposed quantization, rational brute force for the GEMM.
