@@ -323,18 +323,24 @@ size_t plan_ws_bytes(const Plan& p) {
 }
 
 // The plan a call runs; one that needs more workspace than given is refused.
-// The plan of a call of weight kind wk: packed E2M1 operands on both sides
+// The plan of a call of weight kind wk.  Packed E2M1 operands on both sides
 // (A4W4) have K/2 bytes per row, so their schedule counts chunks of 256 K;
-// they have no pair-tile kernel.
+// they move half the shared-memory bytes per MMA, so pair tiles do not pay
+// (sweep, 8192^3: 367 us against 347 us for 128x256 tiles) and are used only
+// on request, and wide tiles take 2 chunks per stage (347 vs 354 us).
 int plan_kind(WeightKind wk, int64_t M, int64_t N, int64_t K, int64_t batch,
               const bq_gemm_config* cfg, int num_sms, Plan* p) {
-  if (wk == kA4W4) {
-    bq_gemm_config c = cfg ? *cfg : bq_gemm_config{0, 0, -1, BQ_SPLIT_AUTO, 0, 0};
-    if (c.cta_pair == 2) return BQ_ERR_INVALID;
-    if (c.cta_pair == 0) c.cta_pair = 1;
-    return make_plan(M, N, K / 2, batch, &c, num_sms, p);
+  if (wk != kA4W4) return make_plan(M, N, K, batch, cfg, num_sms, p);
+  const int64_t Kb = K / 2;
+  bq_gemm_config c = cfg ? *cfg : bq_gemm_config{0, 0, -1, BQ_SPLIT_AUTO, 0, 0};
+  if (c.cta_pair == 0) c.cta_pair = 1;
+  int st = make_plan(M, N, Kb, batch, &c, num_sms, p);
+  if (st == BQ_OK && c.k_chunks == 0 && !p->swap && !p->pair && p->splits == 1 && p->kc == 1 &&
+      Kb % 128 == 0) {
+    c.k_chunks = 2;
+    st = make_plan(M, N, Kb, batch, &c, num_sms, p);
   }
-  return make_plan(M, N, K, batch, cfg, num_sms, p);
+  return st;
 }
 
 int plan_for_call(WeightKind wk, int64_t M, int64_t N, int64_t K, int64_t batch,
@@ -426,13 +432,13 @@ int launch_kind(bool w_fp4, const CUtensorMap& tp, const CUtensorMap& tq, const 
                                                                            num_sms, st);
 }
 
-template <int STAGES, int KC, bool Q_FP4>
+template <int STAGES, int KC, bool Q_FP4, bool A4 = false>
 int launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
                 const CUtensorMap& tsb, const CUtensorMap& ty, const CUtensorMap& tr,
                 const bq::GemmArgs& args,
                 int64_t units, int num_sms, cudaStream_t stream) {
-  using L = bq::PairSmem<STAGES, KC>;
-  auto kern = bq::gemm_pair_kernel<STAGES, KC, Q_FP4>;
+  using L = bq::PairSmem<STAGES, KC, A4 ? 2 : 1>;
+  auto kern = bq::gemm_pair_kernel<STAGES, KC, Q_FP4, A4>;
   static bool attr_set[kMaxDevices] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -691,13 +697,21 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
   g.err = dev->err_ptr;
   if (pl.pair) {
     CUtensorMap map_sfa, map_sfb;
-    st = make_scale_map(&map_sfa, a_sf, M, K, a_batched ? count : 1, ssa, pl.kc, 1);
+    // a stage's scale box: its chunks' atoms (two per chunk for packed E2M1)
+    const int sf_box = pl.kc * (a4 ? 2 : 1);
+    st = make_scale_map(&map_sfa, a_sf, M, K, a_batched ? count : 1, ssa, sf_box, 1);
     if (st != BQ_OK) return st;
-    st = make_scale_map(&map_sfb, b_sf, N, K, b_batched ? count : 1, ssb, pl.kc, 2);
+    st = make_scale_map(&map_sfb, b_sf, N, K, b_batched ? count : 1, ssb, sf_box, 2);
     if (st != BQ_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int64_t u = pl.units;
     const int ns = dev->num_sms;
+    if (a4)  // the packed stages hold the scale atoms of 256 K per chunk: fewer fit
+      return pl.kc == 2
+                 ? launch_pair<2, 2, false, true>(map_a, map_b, map_sfa, map_sfb, map_y, map_res,
+                                                  g, u, ns, s)
+                 : launch_pair<5, 1, false, true>(map_a, map_b, map_sfa, map_sfb, map_y, map_res,
+                                                  g, u, ns, s);
     if (pl.kc == 2)
       return w_fp4 ? launch_pair<3, 2, true>(map_a, map_b, map_sfa, map_sfb, map_y, map_res, g, u, ns, s)
                    : launch_pair<3, 2, false>(map_a, map_b, map_sfa, map_sfb, map_y, map_res, g, u, ns, s);

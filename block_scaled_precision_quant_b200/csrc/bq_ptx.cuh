@@ -466,6 +466,19 @@ __device__ __forceinline__ void tc_mma2_mxf8f6f4(uint32_t d_tmem, uint64_t adesc
       : "memory");
 }
 
+__device__ __forceinline__ void tc_mma2_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], "
+      "[%6], p;\n\t"
+      "}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
 // Arrive on the mbarrier at `bar_cluster` (shared::cluster address, in either
 // CTA of the pair) once every pair MMA / copy this thread issued has completed.
 __device__ __forceinline__ void tc_commit2(uint32_t bar_cluster) {

@@ -27,17 +27,19 @@ namespace bq {
 
 constexpr int kPairN = 256;  // B rows (output columns) of a pair tile
 
-// Shared-memory layout of one CTA of a pair: STAGES stages of KC chunks.
-template <int STAGES, int KC>
+// Shared-memory layout of one CTA of a pair: STAGES stages of KC chunks,
+// each chunk with APC scale atoms per 128-row band (2 for packed E2M1
+// operands, whose 128-byte chunk is 256 K).
+template <int STAGES, int KC, int APC = 1>
 struct PairSmem {
   static constexpr int kChunkA = kBlockP * kBlockK;        // own 128 rows
   static constexpr int kChunkB = (kPairN / 2) * kBlockK;   // own 128 of the 256 B rows
   static constexpr int kBytesA = KC * kChunkA;
   static constexpr int kBytesB = KC * kChunkB;
   static constexpr int kSfbAtoms = kPairN / 128;           // scale bands of all 256 B rows
-  static constexpr int kSfaBytes = KC * kSfAtom;
-  static constexpr int kSfbBytes = KC * kSfbAtoms * kSfAtom;
-  static constexpr int kSfColsChunk = 4 + 4 * kSfbAtoms;   // TMEM scale columns per chunk
+  static constexpr int kSfaBytes = KC * APC * kSfAtom;
+  static constexpr int kSfbBytes = KC * APC * kSfbAtoms * kSfAtom;
+  static constexpr int kSfColsChunk = APC * (4 + 4 * kSfbAtoms);  // TMEM scale columns per chunk
   static constexpr int kSfCols = KC * kSfColsChunk;
   static constexpr int kOffB = STAGES * kBytesA;
   static constexpr int kOffYStage = kOffB + STAGES * kBytesB;  // 1024-aligned
@@ -71,9 +73,10 @@ __device__ __forceinline__ uint32_t make_idesc_m(uint32_t fmt_a, uint32_t fmt_b,
 // Loads one part of a stage into this CTA's shared memory, completing on the
 // leader's stage barrier `bar`: the A tile (own 128 activation rows), the B
 // tile (own 128 weight rows), the A scale atoms (own band) or the B scale
-// atoms (both bands).  Operand maps view K as (128, K/128 chunks) when KC > 1;
-// scale maps view a scale buffer as (128 words, K blocks, 128-row bands).
-template <class L, int KC>
+// atoms (both bands).  Operand maps view K as (128 bytes, chunks) when KC > 1;
+// scale maps view a scale buffer as (128 words, K atoms, 128-row bands), a
+// box KC * APC atoms long.
+template <class L, int KC, int APC = 1>
 __device__ __forceinline__ void pair_issue(const GemmArgs &a, const CUtensorMap *tm_a,
                                            const CUtensorMap *tm_b, const CUtensorMap *tm_sfa,
                                            const CUtensorMap *tm_sfb, uint8_t *smem, int st,
@@ -84,9 +87,9 @@ __device__ __forceinline__ void pair_issue(const GemmArgs &a, const CUtensorMap 
     if (scales) {
       uint8_t *dst = smem + L::kOffSfa + st * L::kSfaBytes;
       if (a.p_batched)
-        tma2_load_4d(dst, tm_sfa, bar, 0, kt, band_a, u.b);
+        tma2_load_4d(dst, tm_sfa, bar, 0, kt * APC, band_a, u.b);
       else
-        tma2_load_3d(dst, tm_sfa, bar, 0, kt, band_a);
+        tma2_load_3d(dst, tm_sfa, bar, 0, kt * APC, band_a);
       return;
     }
     uint8_t *dst = smem + st * L::kBytesA;
@@ -107,9 +110,9 @@ __device__ __forceinline__ void pair_issue(const GemmArgs &a, const CUtensorMap 
   if (scales) {
     uint8_t *dst = smem + L::kOffSfb + st * L::kSfbBytes;
     if (a.q_batched)
-      tma2_load_4d(dst, tm_sfb, bar, 0, kt, 2 * u.tq, u.b);
+      tma2_load_4d(dst, tm_sfb, bar, 0, kt * APC, 2 * u.tq, u.b);
     else
-      tma2_load_3d(dst, tm_sfb, bar, 0, kt, 2 * u.tq);
+      tma2_load_3d(dst, tm_sfb, bar, 0, kt * APC, 2 * u.tq);
     return;
   }
   uint8_t *dst = smem + L::kOffB + st * L::kBytesB;
@@ -127,7 +130,7 @@ __device__ __forceinline__ void pair_issue(const GemmArgs &a, const CUtensorMap 
   }
 }
 
-template <int STAGES, int KC, bool Q_FP4>
+template <int STAGES, int KC, bool Q_FP4, bool A4 = false>
 __global__ void __launch_bounds__(kNumThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
                      const __grid_constant__ CUtensorMap tm_b,
@@ -135,7 +138,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                      const __grid_constant__ CUtensorMap tm_sfb,
                      const __grid_constant__ CUtensorMap tm_y,
                      const __grid_constant__ CUtensorMap tm_res, const GemmArgs a) {
-  using L = PairSmem<STAGES, KC>;
+  // A4: both operands packed E2M1 (kind::mxf4, K = 64 per MMA, two scale
+  // atoms per 128-byte chunk), as in gemm_bs_kernel.
+  static_assert(!A4 || !Q_FP4, "A4 operands are plain packed bytes");
+  constexpr int APC = A4 ? 2 : 1;
+  using L = PairSmem<STAGES, KC, APC>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -209,7 +216,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             break;
           }
           if (rank == 0) mbar_arrive_expect_tx(&full[stage], tx);
-          pair_issue<L, KC>(a, &tm_a, &tm_b, &tm_sfa, &tm_sfb, smem, stage,
+          pair_issue<L, KC, APC>(a, &tm_a, &tm_b, &tm_sfa, &tm_sfb, smem, stage,
                             mapa_shared(smem_u32(&full[stage]), 0), kt, u, rank, weights, scales);
           if (++stage == STAGES) {
             stage = 0;
@@ -243,20 +250,39 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           const uint32_t sf_stage = tmem_base + kPairN + stage * L::kSfCols;
 #pragma unroll 1
           for (int c = 0; c < nv; ++c) {
+            // scale columns of a chunk: A's APC atoms, then per atom B's two bands
             const uint32_t sf_t = sf_stage + c * L::kSfColsChunk;
-            tc_cp_sf2(sf_t, desc_sf_32x128b(sfa0 + stage * L::kSfaBytes + c * kSfAtom));
+            const uint32_t sfb_t = sf_t + 4 * APC;
+            const int na = min(APC, a.sf_katoms - (kt + c) * APC);
+            for (int t = 0; t < na; ++t) {
+              tc_cp_sf2(sf_t + 4 * t,
+                        desc_sf_32x128b(sfa0 + stage * L::kSfaBytes + (c * APC + t) * kSfAtom));
 #pragma unroll
-            for (int j = 0; j < L::kSfbAtoms; ++j)
-              tc_cp_sf2(sf_t + 4 + 4 * j,
-                        desc_sf_32x128b(sfb0 + stage * L::kSfbBytes + (j * KC + c) * kSfAtom));
+              for (int j = 0; j < L::kSfbAtoms; ++j)
+                tc_cp_sf2(sfb_t + 4 * (t * L::kSfbAtoms + j),
+                          desc_sf_32x128b(sfb0 + stage * L::kSfbBytes +
+                                          (j * KC * APC + c * APC + t) * kSfAtom));
+            }
             const uint32_t pa = a0 + stage * L::kBytesA + c * L::kChunkA;
             const uint32_t pb = b0 + stage * L::kBytesB + c * L::kChunkB;
 #pragma unroll
-            for (int ks = 0; ks < kBlockK / kMmaK; ++ks)
-              tc_mma2_mxf8f6f4(tmem_base, desc_kmajor_sw128(pa + ks * kMmaK),
+            for (int ks = 0; ks < kBlockK / kMmaK; ++ks) {
+              const uint32_t acc_in = (kt > 0 || c > 0 || ks > 0) ? 1u : 0u;
+              if constexpr (A4) {
+                const int t = ks >> 1;  // atom of this K = 64 step
+                if (t < na)
+                  tc_mma2_mxf4(tmem_base, desc_kmajor_sw128(pa + ks * kMmaK),
                                desc_kmajor_sw128(pb + ks * kMmaK),
-                               make_idesc_m(fmt_a, fmt_b, 2 * kBlockP, kPairN, ks), sf_t,
-                               sf_t + 4, (kt > 0 || c > 0 || ks > 0) ? 1u : 0u);
+                               make_idesc_m(kFmtMxf4E2M1, kFmtMxf4E2M1, 2 * kBlockP, kPairN,
+                                            (ks & 1) * 2),
+                               sf_t + 4 * t, sfb_t + 4 * t * L::kSfbAtoms, acc_in);
+              } else {
+                tc_mma2_mxf8f6f4(tmem_base, desc_kmajor_sw128(pa + ks * kMmaK),
+                                 desc_kmajor_sw128(pb + ks * kMmaK),
+                                 make_idesc_m(fmt_a, fmt_b, 2 * kBlockP, kPairN, ks), sf_t,
+                                 sfb_t, acc_in);
+              }
+            }
           }
           tc_commit2(mapa_shared(smem_u32(&empty[stage]), 0));
           tc_commit2(mapa_shared(smem_u32(&empty[stage]), 1));

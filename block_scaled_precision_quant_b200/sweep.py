@@ -7,7 +7,7 @@ weights stream from HBM) and prints one JSON line per candidate:
     python -m block_scaled_precision_quant_b200.sweep M N K [kind] [--batch B] [--gelu]
         [--residual]
 
-kind: mxfp4 (default), fp8blk32, mxfp8.  --batch B runs B independent problems
+kind: mxfp4 (default), fp8blk32, mxfp8, a4w4 (MXFP4 activations and weights).  --batch B runs B independent problems
 over one broadcast weight (batch stride 0), --gelu adds bias + GELU,
 --residual adds a bf16 residual.  The
 built-in dispatch of bq_api.cu is derived from these measurements.
@@ -65,7 +65,10 @@ def main(argv=None):
     import block_scaled_precision_quant_b200 as bq
     from block_scaled_precision_quant_b200 import synth
     M, N, K, B = args.M, args.N, args.K, args.batch
-    wk = {"mxfp4": bq.W_MXFP4, "fp8blk32": bq.W_FP8BLK32, "mxfp8": bq.W_MXFP8}[args.kind]
+    wk = {"mxfp4": bq.W_MXFP4, "fp8blk32": bq.W_FP8BLK32, "mxfp8": bq.W_MXFP8,
+          "a4w4": bq.W_A4W4}[args.kind]
+    quant = bq.act_quant_mxfp4 if wk == bq.W_A4W4 else bq.act_quant
+    kb = K // 2 if wk == bq.W_A4W4 else K  # activation bytes per row
     dev = torch.device("cuda")
     stream = torch.cuda.Stream()
     with torch.cuda.stream(stream):
@@ -73,20 +76,20 @@ def main(argv=None):
         for b in range(B):
             x = torch.from_numpy(synth.activations(M, K, seed=1 + b).view(np.int16)) \
                 .view(torch.bfloat16).to(dev)
-            q, f = bq.act_quant(x)
+            q, f = quant(x)
             aqs.append(q)
             asfs.append(f)
-        aq = torch.stack(aqs).reshape(B * M, K)
+        aq = torch.stack(aqs).reshape(B * M, kb)
         asf = torch.stack(asfs)
-        batch = None if B == 1 else dict(count=B, stride_a=M * K, stride_a_sf=asf.shape[1],
+        batch = None if B == 1 else dict(count=B, stride_a=M * kb, stride_a_sf=asf.shape[1],
                                          stride_b=0, stride_b_sf=0, stride_y=M * N * 2,
                                          stride_res=M * N * 2 if args.residual else 0)
         l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-        wbytes = N * K // 2 if wk == bq.W_MXFP4 else N * K
+        wbytes = N * K // 2 if wk in (bq.W_MXFP4, bq.W_A4W4) else N * K
         copies = max(1, min(64, int(np.ceil(2.5 * l2 / max(wbytes, 1)))))
         ws = []
         for c in range(copies):
-            if wk == bq.W_MXFP4:
+            if wk in (bq.W_MXFP4, bq.W_A4W4):
                 b, s = synth.mxfp4_weight(N, K, seed=10 + c)
                 kind = bq.BQ_SF_ROW32
             elif wk == bq.W_FP8BLK32:
@@ -132,7 +135,7 @@ def main(argv=None):
                 torch.cuda.synchronize()
                 bq.device_status()
                 us = e0.elapsed_time(e1) * 1e3 / (args.reps * copies)
-                gbytes = (wbytes + N * K / 32 + B * (M * K * 33 / 32 + 2 * M * N)) / (us * 1e-6) / 1e9
+                gbytes = (wbytes + N * K / 32 + B * (M * (kb + K / 32) + 2 * M * N)) / (us * 1e-6) / 1e9
                 print(json.dumps(dict(shape=[M, N, K], batch=B, gelu=args.gelu, kind=args.kind,
                                       residual=args.residual,
                                       cfg=desc, us=round(us, 3),

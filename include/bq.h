@@ -336,7 +336,7 @@ size_t bq_gemm_workspace_bytes(int weight_kind, int64_t M, int64_t N, int64_t K,
  * device.  Calls that ask for a quantized output run unsplit.  Returns
  * BQ_ERR_NULL (out NULL), BQ_ERR_SHAPE (sizes out of range, num_sms < 1) or
  * BQ_ERR_INVALID (weight_kind or cfg not schedulable, the status the GEMM call
- * returns).  MXFP4 activations (weight_kind 3) have no pair tiles. */
+ * returns). */
 int bq_gemm_plan(int weight_kind, int64_t M, int64_t N, int64_t K, int64_t batch,
                  const bq_gemm_config *cfg, int num_sms, bq_gemm_config *out);
 
@@ -370,7 +370,7 @@ int bq_gemm_e5m2_mxfp8_epilogue(const void *a_e5m2, const void *a_sf, const void
                                 size_t workspace_bytes, const bq_gemm_config *cfg,
                                 bq_stream_t stream);
 /* A4W4 (bq_gemm_mxfp4_mxfp4) with the same epilogue, batch, workspace and
- * schedule options; cta_pair 2 is refused (BQ_ERR_INVALID). */
+ * schedule options. */
 int bq_gemm_mxfp4_mxfp4_epilogue(const void *a_fp4, const void *a_sf, const void *b_fp4,
                                  const void *b_sf, int64_t M, int64_t N, int64_t K, void *y_bf16,
                                  const bq_epilogue *epi, const bq_batch *batch, void *workspace,

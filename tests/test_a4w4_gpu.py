@@ -160,6 +160,43 @@ def test_a4w4_wide_tiles(block_n, k_chunks):
         bq.config(block_n=block_n, split_k=1, swap_ab=0, k_chunks=k_chunks))
 
 
+@pytest.mark.parametrize("k_chunks,K", [(1, 1408), (2, 1536)])
+def test_a4w4_pair_tiles(k_chunks, K):
+    """256x256 tiles on CTA pairs with kind::mxf4 (cta_group::2): ragged M and
+    N; with one chunk per stage K ends in a half chunk (128 of 256 K)."""
+    A4Case(600, 776, K, seed=12 + k_chunks, bias=True, residual=True).check_full(
+        bq.config(split_k=1, swap_ab=0, cta_pair=2, k_chunks=k_chunks))
+
+
+def test_a4w4_pair_tiles_persistent():
+    """More pair tiles than SM pairs: every pair walks several tiles."""
+    A4Case(2304, 2560, 512, seed=17).check_full(bq.config(split_k=1, swap_ab=0, cta_pair=2))
+
+
+def test_a4w4_pair_tiles_batched_gelu():
+    count, M, N, K = 2, 300, 520, 1024
+    xs = [synth.activations(M, K, seed=80 + i) for i in range(count)]
+    b, bsf = synth.mxfp4_weight(N, K, seed=85)
+    bias = synth.bias(N, seed=86)
+    qs, sfs = zip(*[bq.act_quant_mxfp4(dev_bf16(x)) for x in xs])
+    aq = torch.stack(qs).reshape(count * M, K // 2)
+    asf = torch.stack(sfs)
+    bsf_d = bq.pack_weight_scales(dev_u8(bsf), bq.BQ_SF_ROW32, N, K)
+    y = bq.gemm(bq.W_A4W4, aq, asf, dev_u8(b), bsf_d, M, N, K, bias=dev_bf16(bias),
+                act=bq.BQ_ACT_GELU, config=bq.config(split_k=1, swap_ab=0, cta_pair=2),
+                batch=dict(count=count, stride_a=M * K // 2, stride_a_sf=asf.shape[1],
+                           stride_b=0, stride_b_sf=0, stride_y=M * N * 2))
+    bq.device_status()
+    yv = f64(y.cpu().view(torch.int16).numpy().view(np.uint16))
+    for i, x in enumerate(xs):
+        q, s = oracle.act_quant_fp4(x)
+        ref, sabs = oracle.gemm(q, s, b, bsf, oracle.B_FP4, M, N, K, bias=bias,
+                                act=oracle.ACT_GELU, a_kind=oracle.A_FP4)
+        tol = oracle.gemm_tolerance(ref, sabs, 1.0, np.abs(f64(bias))[None, :], None,
+                                    oracle.ACT_GELU)
+        assert_close(yv[i], ref, tol, f"pair batch {i}")
+
+
 @pytest.mark.parametrize("M", [1, 17, 41, 64])
 @pytest.mark.parametrize("k_chunks", [1, 4])
 def test_a4w4_decode_swap(M, k_chunks):
@@ -253,10 +290,6 @@ def test_a4w4_refusals():
     aq, asf = bq.act_quant_mxfp4(dev_bf16(c.x))
     bd = dev_u8(c.b)
     bsf = bq.pack_weight_scales(dev_u8(c.bsf), bq.BQ_SF_ROW32, c.N, c.K)
-    with pytest.raises(bq.BqError) as e:  # no pair tiles for packed E2M1 activations
-        bq.gemm(bq.W_A4W4, aq, asf, bd, bsf, c.M, c.N, c.K,
-                config=bq.config(split_k=1, swap_ab=0, cta_pair=2))
-    assert e.value.status == bq.BQ_ERR_INVALID
     with pytest.raises(bq.BqError) as e:  # K % 128
         bq.gemm(bq.W_A4W4, aq, asf, bd, bsf, c.M, c.N, 608)
     assert e.value.status == bq.BQ_ERR_SHAPE

@@ -92,3 +92,16 @@ def test_bad_sizes():
         assert e.value.status == bq.BQ_ERR_SHAPE
     with pytest.raises(bq.BqError):
         bq.plan(64, 512, 1024, num_sms=0)
+
+
+def test_a4w4_plans():
+    """Packed E2M1 operands: chunks of 256 K, wide tiles with 2 chunks per
+    stage, no pair tiles unless asked for."""
+    c = bq.plan(8192, 8192, 8192, num_sms=SMS, weight_kind=bq.W_A4W4)
+    assert (c.block_n, c.cta_pair, c.k_chunks, c.swap_ab) == (256, 1, 2, 0)
+    c = bq.plan(8192, 8192, 8192, num_sms=SMS, weight_kind=bq.W_A4W4,
+                config=bq.config(split_k=1, swap_ab=0, cta_pair=2))
+    assert (c.cta_pair, c.k_chunks) == (2, 2)
+    c = bq.plan(41, 4608, 1536, num_sms=SMS, weight_kind=bq.W_A4W4)
+    assert c.swap_ab == 1 and c.split_k == 1
+    assert bq.plan(41, 1536, 6144, num_sms=SMS, weight_kind=bq.W_A4W4).split_k > 1
