@@ -26,8 +26,8 @@ _lock = threading.Lock()
 _lib = None
 
 OK, ERR_NAN_SCALE, ERR_NAN_CODE, ERR_SHAPE, ERR_NONFINITE = 0, -1, -2, -3, -4
-B_FP4, B_FP8BLK, B_FP8ROW = 0, 1, 2
-A_E4M3, A_FP4, A_E5M2 = 0, 1, 2
+B_FP4, B_FP8BLK, B_FP8ROW, B_NVFP4 = 0, 1, 2, 3
+A_E4M3, A_FP4, A_E5M2, A_NVFP4 = 0, 1, 2, 3
 Q_E4M3, Q_E5M2 = 0, 1  # code formats of the transposed quantizer
 ACT_NONE, ACT_GELU = 0, 1
 
@@ -110,6 +110,10 @@ def _load():
     lib.oracle_quant_transposed.argtypes = [u16p, i64, i64, i64, ctypes.c_int, ctypes.c_int, u64,
                                             u8p, u8p]
     lib.oracle_quant_transposed.restype = ctypes.c_int
+    lib.oracle_e4m3_ceil.argtypes = [ctypes.c_float]
+    lib.oracle_e4m3_ceil.restype = ctypes.c_uint8
+    lib.oracle_act_quant_nvfp4.argtypes = [u16p, i64, i64, i64, ctypes.c_float, u8p, u8p]
+    lib.oracle_act_quant_nvfp4.restype = ctypes.c_int
     lib.oracle_gemm_ex.argtypes = [u8p, u8p, ctypes.c_int, u8p, u8p, ctypes.c_int, i64, i64, i64,
                                    u16p, u16p, i64, ctypes.c_double, ctypes.c_int, f64p, f64p,
                                    ctypes.c_int]
@@ -335,6 +339,29 @@ def act_quant_fp4_f32(x: np.ndarray):
     return q, sf
 
 
+def e4m3_ceil(t: float) -> int:
+    """The smallest positive E4M3 value >= t, as its byte (the NVFP4 block
+    scale): 0x01 (2^-9) at or below it, 0x7E (448) above 448."""
+    return int(_load().oracle_e4m3_ceil(float(t)))
+
+
+def act_quant_nvfp4(x_bf16_bits: np.ndarray, g: float = 1.0):
+    """NVFP4 quantization: every value first fp32(x * g) (g the per-tensor
+    scale), then per 16 consecutive values an E4M3 scale s = the smallest E4M3
+    value >= fp32(amax * fp32(1/6)) and E2M1 codes of fp32(x / s) (round to
+    nearest even, sign kept).  Returns (q uint8 [M, K/2] packed, low nibble
+    first, sf uint8 [M, K/16] E4M3 bytes)."""
+    x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
+    M, K = x.shape
+    q = np.empty((M, K // 2), dtype=np.uint8)
+    sf = np.empty((M, K // 16), dtype=np.uint8)
+    if M:
+        _check(_load().oracle_act_quant_nvfp4(_ptr(x, ctypes.c_uint16), M, K, K, float(g),
+                                              _ptr(q, ctypes.c_uint8), _ptr(sf, ctypes.c_uint8)),
+               "act_quant_nvfp4")
+    return q, sf
+
+
 def unpack_fp4(q: np.ndarray) -> np.ndarray:
     """Packed E2M1 bytes [..., K/2] -> one code per byte [..., K] (low nibble
     first)."""
@@ -366,8 +393,9 @@ def gemm(aq, asf, b, bsf, bkind, M, N, K, bias=None, residual=None, alpha=1.0,
     ref[m, n] = act(alpha * sum_k a[m,k] b[n,k] + bias[n]) + residual[m, n] and
     sumabs[m, n] = sum_k |a[m,k] b[n,k]|, where a and b are the exactly decoded
     operands (formats.py page: decode_fp4, decode_fp8_block, e8m0_to_f32).
-    a_kind: A_E4M3 (aq [M, K]), A_FP4 (aq [M, K/2] packed E2M1) or A_E5M2
-    (aq [M, K] E5M2 gradient codes)."""
+    a_kind: A_E4M3 (aq [M, K]), A_FP4 (aq [M, K/2] packed E2M1), A_E5M2
+    (aq [M, K] E5M2 gradient codes) or A_NVFP4 (aq [M, K/2] packed E2M1 with
+    E4M3 scales asf [M, K/16]); bkind B_NVFP4 likewise for b."""
     aq = np.ascontiguousarray(aq, dtype=np.uint8)
     asf = np.ascontiguousarray(asf, dtype=np.uint8)
     b = np.ascontiguousarray(b, dtype=np.uint8)

@@ -21,6 +21,13 @@
  *     out on the pages: it is the same per-32 rule with the E2M1 format's
  *     largest value 6 in place of 448, and E2M1 codes packed two per byte with
  *     the even element in the low nibble (the pages' MXFP4 weight layout);
+ *   - NVFP4 (the A4W4 kernels of the "fp4-gemm" page name it: E2M1 codes
+ *     with one E4M3 scale per 16 values and a per-tensor fp32 scale) is not
+ *     spelled out either: the tensor is first multiplied by the caller's
+ *     per-tensor scale, each block of 16 takes the smallest E4M3 scale that
+ *     holds its largest value (the round-up counterpart of the MX rule, so no
+ *     value clips below the top of the E4M3 range), codes are E2M1 of
+ *     x / scale; the GEMM undoes the per-tensor scales through alpha;
  *   - the gradient quantizer of the backward pass (E5M2 codes, the pages'
  *     "hip_quant" README, "Stochastic E5M2 Backward Gradients" and "Block-wise
  *     FP8 Scaling") takes the same per-32 rule with E5M2's largest finite
@@ -439,6 +446,65 @@ int oracle_act_quant_fp4_f32(const float *x, int64_t M, int64_t K, uint8_t *q, u
   return ORACLE_OK;
 }
 
+/* NVFP4 block scale: the smallest positive E4M3 value >= t (t >= 0 finite):
+ * 2^-9 (the smallest subnormal) for t <= 2^-9, 448 for t > 448. */
+uint8_t oracle_e4m3_ceil(float t) {
+  e4m3_table_init();
+  double a = (double)t;
+  if (a <= e4m3_mag[1]) return 1;
+  if (a >= e4m3_mag[126]) return 126;
+  int c = 1;
+  while (e4m3_mag[c] < a) ++c; /* mag[c - 1] < a <= mag[c] */
+  return (uint8_t)c;
+}
+
+/* NVFP4 quantization of one group of 16 values already multiplied by the
+ * per-tensor scale (binary32): amax = max |x|, t = fp32(amax * fp32(1/6)),
+ * s = oracle_e4m3_ceil(t), q = E2M1_RNE(clamp(fp32(x / s), -6, 6)) with the
+ * sign kept.  Returns the scale byte, -1 for a NaN / Inf. */
+static int nvfp4_group(const float *x, uint8_t *codes) {
+  float amax = 0.0f;
+  for (int i = 0; i < 16; ++i) {
+    if (!isfinite(x[i])) return -1;
+    float ax = fabsf(x[i]);
+    if (ax > amax) amax = ax;
+  }
+  const float inv6 = (float)(1.0 / 6.0);
+  float t = amax * inv6;
+  uint8_t sb = oracle_e4m3_ceil(t);
+  double sd;
+  oracle_decode_e4m3(sb, &sd);
+  float s = (float)sd;
+  for (int i = 0; i < 16; ++i) {
+    float y = x[i] / s;
+    if (y > 6.0f) y = 6.0f;
+    if (y < -6.0f) y = -6.0f;
+    codes[i] = oracle_encode_fp4(y);
+  }
+  return sb;
+}
+
+/* x bf16 [M, ldx]; g the per-tensor scale; q [M, K/2] packed E2M1 codes,
+ * sf [M, K/16] E4M3 scale bytes.  Each value is first fp32(x * g).
+ * K % 16 == 0. */
+int oracle_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, float g,
+                           uint8_t *q, uint8_t *sf) {
+  if (K <= 0 || K % 16) return ORACLE_ERR_SHAPE;
+  const int64_t G = K / 16;
+  float buf[16];
+  uint8_t codes[16];
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t gi = 0; gi < G; ++gi) {
+      for (int i = 0; i < 16; ++i) buf[i] = bf16_to_f32(x[m * ldx + gi * 16 + i]) * g;
+      int b = nvfp4_group(buf, codes);
+      if (b < 0) return ORACLE_ERR_NONFINITE;
+      for (int j = 0; j < 8; ++j)
+        q[m * (K / 2) + gi * 8 + j] = (uint8_t)(codes[2 * j] | (codes[2 * j + 1] << 4));
+      sf[m * G + gi] = (uint8_t)b;
+    }
+  return ORACLE_OK;
+}
+
 /* Gradient quantization, E5M2 codes: the per-32 rule with E5M2's largest
  * finite value 57344 in place of 448,
  *   t = fp32(max(amax, 1e-4) * fp32(1/57344)),  e = ceil(log2 t),
@@ -535,11 +601,13 @@ int oracle_quant_transposed(const uint16_t *x, int64_t R, int64_t C, int64_t ldx
 #define ORACLE_B_FP4 0     /* E2M1 packed [N, K/2], low nibble = even k; scales [N, K/32] */
 #define ORACLE_B_FP8BLK 1  /* E4M3 [N, K]; scales [ceil(N/32), ceil(K/32)], one per 32x32 block */
 #define ORACLE_B_FP8ROW 2  /* E4M3 [N, K]; scales [N, K/32] (MXFP8 along K) */
+#define ORACLE_B_NVFP4 3   /* E2M1 packed [N, K/2]; E4M3 scales [N, K/16] */
 
 /* Activation kinds. */
 #define ORACLE_A_E4M3 0 /* E4M3 [M, K]; scales [M, K/32] */
 #define ORACLE_A_FP4 1  /* E2M1 packed [M, K/2], low nibble = even k; scales [M, K/32] */
 #define ORACLE_A_E5M2 2 /* E5M2 [M, K] (gradients); scales [M, K/32] */
+#define ORACLE_A_NVFP4 3 /* E2M1 packed [M, K/2]; E4M3 scales [M, K/16] */
 
 #define ORACLE_ACT_NONE 0
 #define ORACLE_ACT_GELU 1
@@ -567,6 +635,13 @@ typedef struct {
  * E4M3 or packed E2M1. */
 static int dec_a(const gemm_job *J, int64_t m, int64_t k, double *v) {
   double c, s;
+  if (J->akind == ORACLE_A_NVFP4) {
+    uint8_t byte = J->aq[m * (J->K / 2) + k / 2];
+    c = oracle_decode_fp4((k % 2 == 0) ? (byte & 0x0F) : (byte >> 4));
+    if (oracle_decode_e4m3(J->asf[m * (J->K / 16) + k / 16], &s)) return ORACLE_ERR_NAN_SCALE;
+    *v = c * s;
+    return ORACLE_OK;
+  }
   if (J->akind == ORACLE_A_FP4) {
     uint8_t byte = J->aq[m * (J->K / 2) + k / 2];
     c = oracle_decode_fp4((k % 2 == 0) ? (byte & 0x0F) : (byte >> 4));
@@ -586,6 +661,13 @@ static int dec_b(const gemm_job *J, int64_t n, int64_t k, double *v) {
   const int64_t K = J->K;
   double c, s;
   uint8_t sb;
+  if (J->bkind == ORACLE_B_NVFP4) {
+    uint8_t byte = J->b[n * (K / 2) + k / 2];
+    c = oracle_decode_fp4((k % 2 == 0) ? (byte & 0x0F) : (byte >> 4));
+    if (oracle_decode_e4m3(J->bsf[n * (K / 16) + k / 16], &s)) return ORACLE_ERR_NAN_SCALE;
+    *v = c * s;
+    return ORACLE_OK;
+  }
   if (J->bkind == ORACLE_B_FP4) {
     uint8_t byte = J->b[n * (K / 2) + k / 2];
     uint8_t code = (k % 2 == 0) ? (byte & 0x0F) : (byte >> 4);
@@ -681,7 +763,7 @@ int oracle_gemm_ex(const uint8_t *aq, const uint8_t *asf, int akind, const uint8
                    const uint8_t *bsf, int bkind, int64_t M, int64_t N, int64_t K,
                    const uint16_t *bias, const uint16_t *residual, int64_t ld_res, double alpha,
                    int act, double *ref, double *sumabs, int nthreads) {
-  if (K <= 0 || K % BLOCK || bkind < 0 || bkind > 2 || akind < 0 || akind > 2)
+  if (K <= 0 || K % BLOCK || bkind < 0 || bkind > 3 || akind < 0 || akind > 3)
     return ORACLE_ERR_SHAPE;
   gemm_job J = {aq, asf, b, bsf, akind, bkind, M, N, K, bias, residual, ld_res, alpha, act,
                 ref, sumabs, NULL, NULL, 0, 0, 0, 0};
@@ -702,7 +784,7 @@ int oracle_gemm_sampled_ex(const uint8_t *aq, const uint8_t *asf, int akind, con
                            const uint16_t *bias, const uint16_t *residual, int64_t ld_res,
                            double alpha, int act, const int64_t *ms, const int64_t *ns,
                            int64_t count, double *ref, double *sumabs, int nthreads) {
-  if (K <= 0 || K % BLOCK || bkind < 0 || bkind > 2 || akind < 0 || akind > 2)
+  if (K <= 0 || K % BLOCK || bkind < 0 || bkind > 3 || akind < 0 || akind > 3)
     return ORACLE_ERR_SHAPE;
   gemm_job J = {aq, asf, b, bsf, akind, bkind, M, N, K, bias, residual, ld_res, alpha, act,
                 ref, sumabs, ms, ns, count, 0, 0, 0};
