@@ -72,6 +72,10 @@ WORKLOADS = {
         desc="square MXFP4xMXFP4 GEMM M=N=K=8192 (activations act_quant_mxfp4'd per step, "
              "MXFP4 weights)",
         layers=[("square", "a4w4", 8192, 8192, 8192, 1, dict())], bound="tensor"),
+    "nvfp4_square": dict(
+        desc="square NVFP4xNVFP4 GEMM M=N=K=8192 (activations act_quant_nvfp4'd per step, "
+             "NVFP4 weights)",
+        layers=[("square", "nvfp4", 8192, 8192, 8192, 1, dict())], bound="tensor"),
     # Backward of one linear layer y = x W^T (x [T, K], W [N, K]): the output
     # gradient dY [T, N] quantized to E5M2 with stochastic rounding along N
     # (for dX) and along T (for dW), x and the bf16 master weight W quantized
@@ -85,9 +89,10 @@ WORKLOADS = {
         layers=[("bwd", "grad", 4096, 1536, 6144, 1, dict())], bound="tensor"),
 }
 
-WKIND = {"mxfp4": 0, "fp8blk32": 1, "mxfp8": 2, "a4w4": 3, "grad": 4}
+WKIND = {"mxfp4": 0, "fp8blk32": 1, "mxfp8": 2, "a4w4": 3, "grad": 4, "nvfp4": 5}
 DTYPE = {"mxfp4": "mxfp8xmxfp4", "fp8blk32": "mxfp8xfp8blk32", "mxfp8": "mxfp8xmxfp8",
-         "a4w4": "mxfp4xmxfp4", "grad": "e5m2xmxfp8"}
+         "a4w4": "mxfp4xmxfp4", "grad": "e5m2xmxfp8", "nvfp4": "nvfp4xnvfp4"}
+FP4_ACT = ("a4w4", "nvfp4")  # packed E2M1 activations
 
 
 def gemm_shapes(layer):
@@ -110,6 +115,8 @@ def act_quant_bytes(layer):
     _, wk, M, N, K, B, _ = layer
     if wk == "grad":  # dY twice (row-wise, transposed), x^T and W^T
         return (2.0 + 1.0 + 1.0 / 32.0) * (2 * M * N + M * K + N * K)
+    if wk == "nvfp4":
+        return (2.0 + 0.5 + 1.0 / 16.0) * M * K * B
     code = 0.5 if wk == "a4w4" else 1.0
     return (2.0 + code + 1.0 / 32.0) * M * K * B
 
@@ -122,9 +129,10 @@ def gemm_bytes(layer, quant_out=False):
     if wk == "grad":  # dX: dY codes [M, N] x W^T codes [K, N]; dW: dY^T [N, M] x x^T [K, M]
         code = 1.0 + 1.0 / 32.0
         return code * (M * N + K * N) + 2.0 * M * K + code * (N * M + K * M) + 2.0 * N * K
-    w = N * K / 2.0 if wk in ("mxfp4", "a4w4") else float(N * K)
-    w += N * K / 32.0  # weight scales
-    a = B * (M * K * (0.5 if wk == "a4w4" else 1.0) + M * K / 32.0)
+    w = N * K / 2.0 if wk in ("mxfp4",) + FP4_ACT else float(N * K)
+    sfb = 16.0 if wk == "nvfp4" else 32.0  # inputs per scale byte
+    w += N * K / sfb  # weight scales
+    a = B * (M * K * (0.5 if wk in FP4_ACT else 1.0) + M * K / sfb)
     y = B * M * N * ((1.0 + 1.0 / 32.0) if quant_out else 2.0)
     if ex.get("bias"):
         a += N * 2.0
@@ -297,7 +305,12 @@ class Layer:
                 xb = synth.activations(M, K, seed=sd + b, group_pow2=ex.get("act_gp"))
                 xs.append(torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16))
             x = torch.stack(xs).reshape(B * M, K).to(device)
-            if wk in ("mxfp4", "a4w4"):
+            if wk == "nvfp4":  # weights quantized once here, on the device
+                wxb = synth.activations(N, K, seed=sd + 500, std=0.05)
+                wx = torch.from_numpy(wxb.view(np.int16)).view(torch.bfloat16).to(device)
+                w, wsf = bq.act_quant_nvfp4(wx)
+                wx = None
+            elif wk in ("mxfp4", "a4w4"):
                 wb, ws = synth.mxfp4_weight(N, K, seed=sd + 500)
                 w = torch.from_numpy(wb).to(device)
                 wsf = bq.pack_weight_scales(torch.from_numpy(ws).to(device), bq.BQ_SF_ROW32, N, K)
@@ -319,10 +332,11 @@ class Layer:
                    .view(torch.bfloat16).to(device) if ex.get("residual") else None)
             self.sets.append(dict(x=x, w=w, wsf=wsf, wx=wx, bias=bias, res=res))
         # outputs shared by all sets (written every step)
-        self.a4 = wk == "a4w4"  # packed E2M1 activations, two codes per byte
+        self.a4 = wk in FP4_ACT  # packed E2M1 activations, two codes per byte
+        self.nv = wk == "nvfp4"
         self.aq = torch.empty((B * M, K // 2 if self.a4 else K), dtype=torch.uint8,
                               device=device)
-        per = bq.sf_bytes(M, K)
+        per = bq.sf_bytes_nvfp4(M, K) if self.nv else bq.sf_bytes(M, K)
         self.asf = torch.empty((B, per), dtype=torch.uint8, device=device)
         self.y = torch.empty((B, M, N), dtype=torch.bfloat16, device=device)
         self.quant_out = quant_out
@@ -359,7 +373,8 @@ class Layer:
             # rule) runs act_quant + the split GEMM instead
             return 2 if (K + 127) // 128 >= 24 and not self.quant_out else 1
         if which in ("all", "act_quant"):
-            quant = bq.act_quant_mxfp4 if self.a4 else bq.act_quant
+            quant = (bq.act_quant_nvfp4 if self.nv else
+                     bq.act_quant_mxfp4 if self.a4 else bq.act_quant)
             for b in range(B):
                 quant(d["x"][b * M:(b + 1) * M], q=self.aq[b * M:(b + 1) * M],
                       sf_mma=self.asf[b])
@@ -588,7 +603,10 @@ def oracle_step_sample(layers_spec, rows, seed=0, nthreads=None):
             flops += 2.0 * r * K * N + 2.0 * r * K * M
             continue
         x = synth.activations(r, K, seed=seed, group_pow2=ex.get("act_gp"))
-        if wk in ("mxfp4", "a4w4"):
+        if wk == "nvfp4":
+            wb, ws = oracle.act_quant_nvfp4(synth.activations(N, K, seed=seed + 500, std=0.05))
+            kind = oracle.B_NVFP4
+        elif wk in ("mxfp4", "a4w4"):
             wb, ws = synth.mxfp4_weight(N, K, seed=seed + 500)
             kind = oracle.B_FP4
         elif wk == "fp8blk32":
@@ -600,13 +618,16 @@ def oracle_step_sample(layers_spec, rows, seed=0, nthreads=None):
         bias = synth.bias(N, seed=seed + 600) if ex.get("bias") else None
         res = synth.residual(r, N, seed=seed + 700) if ex.get("residual") else None
         t0 = time.perf_counter()
-        if wk == "a4w4":
+        if wk == "nvfp4":
+            q, s = oracle.act_quant_nvfp4(x)
+        elif wk == "a4w4":
             q, s = oracle.act_quant_fp4(x)
         else:
             q, s = oracle.act_quant(x)
+        a_kind = {"a4w4": oracle.A_FP4, "nvfp4": oracle.A_NVFP4}.get(wk, oracle.A_E4M3)
         oracle.gemm(q, s, wb, ws, kind, r, N, K, bias=bias, residual=res,
                     act=oracle.ACT_GELU if ex.get("gelu") else oracle.ACT_NONE,
-                    nthreads=nthreads, a_kind=oracle.A_FP4 if wk == "a4w4" else oracle.A_E4M3)
+                    nthreads=nthreads, a_kind=a_kind)
         t_total += time.perf_counter() - t0
         flops += 2.0 * r * N * K
     return flops, t_total, nthreads
@@ -752,7 +773,7 @@ def run_ours(args, spec, world, rank, local, device):
         ck.get("sm_mhz") and ck.get("sm_max_mhz") and ck["sm_mhz"] < 0.97 * ck["sm_max_mhz"])
     tensor_kind = "bf16_sus" if capped else "bf16"
     # nominal dense fp8 / bf16 ratio 4.5 / 2.25; FP4 x FP4 (kind::mxf4) 9 / 2.25
-    a4 = all(sp[1] == "a4w4" for sp in layers_spec)
+    a4 = all(sp[1] in FP4_ACT for sp in layers_spec)  # FP4 x FP4: the FP4 tensor rate
     tensor_ratio = 4.0 if a4 else 2.0
     fp8_peak = tensor_ratio * peaks[tensor_kind]
     shapes = [(WKIND[sp[1]],) + g for sp in layers_spec for g in gemm_shapes(sp)]

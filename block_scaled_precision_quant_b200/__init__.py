@@ -33,12 +33,14 @@ BQ_ERR_INVALID = 11
 
 BQ_SF_ROW32 = 0
 BQ_SF_BLK32x32 = 1
+BQ_SF_ROW16_E4M3 = 2
 BQ_ACT_NONE = 0
 BQ_ACT_GELU = 1
 BQ_SPLIT_AUTO, BQ_SPLIT_WORKSPACE, BQ_SPLIT_CLUSTER = 0, 1, 2
 W_MXFP4, W_FP8BLK32, W_MXFP8 = 0, 1, 2
 W_A4W4 = 3  # MXFP4 weights with MXFP4 (packed E2M1) activations
 W_GRAD = 4  # E5M2 gradient codes x MXFP8 (E4M3) operand: the backward products
+W_NVFP4 = 5  # NVFP4 x NVFP4 (E2M1 with E4M3 scales per 16)
 BQ_ROUND_NEAREST, BQ_ROUND_STOCHASTIC = 0, 1
 BQ_FMT_E4M3, BQ_FMT_E5M2 = 0, 1
 
@@ -50,7 +52,8 @@ EXPORTS = (
     "bq_device_report", "bq_gemm_mxfp8_mxfp4_epilogue_noalloc", "bq_noalloc_scratch_bytes",
     "bq_gemm_bf16act_epilogue", "bq_gemm_plan", "bq_act_quant_mxfp4", "bq_gemm_mxfp4_mxfp4",
     "bq_gemm_mxfp4_mxfp4_epilogue", "bq_grad_quant", "bq_quant_transposed", "bq_gemm_e5m2_mxfp8",
-    "bq_gemm_e5m2_mxfp8_epilogue", "bq_grad_quant_dual",
+    "bq_gemm_e5m2_mxfp8_epilogue", "bq_grad_quant_dual", "bq_sf_bytes_nvfp4", "bq_act_quant_nvfp4",
+    "bq_gemm_nvfp4_nvfp4", "bq_gemm_nvfp4_nvfp4_epilogue",
 )
 
 
@@ -106,6 +109,10 @@ def lib():
         L.bq_act_quant.restype = i32
         L.bq_act_quant_mxfp4.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp]
         L.bq_act_quant_mxfp4.restype = i32
+        L.bq_act_quant_nvfp4.argtypes = [vp, i64, i64, i64, ctypes.c_float, vp, vp, vp, vp, vp]
+        L.bq_act_quant_nvfp4.restype = i32
+        L.bq_sf_bytes_nvfp4.argtypes = [i64, i64]
+        L.bq_sf_bytes_nvfp4.restype = sz
         L.bq_grad_quant.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, i32, ctypes.c_uint64, vp]
         L.bq_grad_quant.restype = i32
         L.bq_quant_transposed.argtypes = [vp, i64, i64, i64, i32, i32, ctypes.c_uint64, vp, vp,
@@ -119,13 +126,13 @@ def lib():
         L.bq_unpack_scales.argtypes = [vp, i64, i64, vp, vp]
         L.bq_unpack_scales.restype = i32
         for name in ("bq_gemm_mxfp8_mxfp4", "bq_gemm_mxfp8_fp8blk32", "bq_gemm_mxfp8_mxfp8",
-                     "bq_gemm_mxfp4_mxfp4", "bq_gemm_e5m2_mxfp8"):
+                     "bq_gemm_mxfp4_mxfp4", "bq_gemm_e5m2_mxfp8", "bq_gemm_nvfp4_nvfp4"):
             f = getattr(L, name)
             f.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp]
             f.restype = i32
         for name in ("bq_gemm_mxfp8_mxfp4_epilogue", "bq_gemm_mxfp8_fp8blk32_epilogue",
                      "bq_gemm_mxfp8_mxfp8_epilogue", "bq_gemm_mxfp4_mxfp4_epilogue",
-                     "bq_gemm_e5m2_mxfp8_epilogue"):
+                     "bq_gemm_e5m2_mxfp8_epilogue", "bq_gemm_nvfp4_nvfp4_epilogue"):
             f = getattr(L, name)
             f.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, ctypes.POINTER(Epilogue),
                           ctypes.POINTER(Batch), vp, sz, ctypes.POINTER(GemmConfig), vp]
@@ -247,6 +254,29 @@ def act_quant_mxfp4(x, q=None, sf_mma=None, sf_rowmajor=None, status=None):
     return q, sf_mma
 
 
+def sf_bytes_nvfp4(rows: int, K: int) -> int:
+    return int(lib().bq_sf_bytes_nvfp4(rows, K))
+
+
+def act_quant_nvfp4(x, g=1.0, q=None, sf_mma=None, sf_rowmajor=None, status=None):
+    """NVFP4 quantization of a bf16 [M, K] CUDA tensor scaled by the per-tensor
+    g: returns (q uint8 [M, K/2] packed E2M1, sf_mma MMA-layout E4M3 scales per
+    16), the operands of gemm(W_NVFP4, ...) (with alpha = 1 / (g_a g_b))."""
+    torch = _torch()
+    _need_cuda(x)
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a bf16 [M, K] tensor with unit column stride")
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
+    if sf_mma is None:
+        sf_mma = torch.empty((max(sf_bytes_nvfp4(M, K), 1),), dtype=torch.uint8, device=x.device)
+    _check(lib().bq_act_quant_nvfp4(_ptr(x), M, K, x.stride(0), float(g), _ptr(q), _ptr(sf_mma),
+                                    _ptr(sf_rowmajor), _ptr(status), _stream()),
+           "bq_act_quant_nvfp4")
+    return q, sf_mma
+
+
 def grad_quant(g, stochastic=False, seed=0, q=None, sf_mma=None, sf_rowmajor=None,
                status=None):
     """Per-32 E5M2 quantization of a bf16 [M, K] gradient along K (round to
@@ -313,12 +343,13 @@ def quant_transposed(x, fmt=BQ_FMT_E4M3, stochastic=False, seed=0, q=None, sf_mm
 
 
 def pack_weight_scales(scales, kind: int, N: int, K: int, out=None, e4m3_codes=None):
-    """E8M0 weight scales (ROW32 [N, K/32] or BLK32x32 [ceil(N/32), K/32]) to
-    the MMA layout.  Synchronizes the stream; raises on NaN scales or codes."""
+    """Weight scales (E8M0 ROW32 [N, K/32] or BLK32x32 [ceil(N/32), K/32], or
+    E4M3 ROW16_E4M3 [N, K/16] for NVFP4) to the MMA layout.  Synchronizes the stream; raises on NaN scales or codes."""
     torch = _torch()
     _need_cuda(scales, e4m3_codes)
     if out is None:
-        out = torch.empty((max(sf_bytes(N, K), 1),), dtype=torch.uint8, device=scales.device)
+        n = sf_bytes_nvfp4(N, K) if kind == BQ_SF_ROW16_E4M3 else sf_bytes(N, K)
+        out = torch.empty((max(n, 1),), dtype=torch.uint8, device=scales.device)
     _check(lib().bq_pack_weight_scales(_ptr(scales), int(kind), N, K, _ptr(out),
                                        _ptr(e4m3_codes), _stream()), "bq_pack_weight_scales")
     return out
@@ -340,7 +371,7 @@ def unpack_scales(sf_mma, rows: int, K: int, out=None):
 _ws = {}
 _ENTRY = {W_MXFP4: "bq_gemm_mxfp8_mxfp4", W_FP8BLK32: "bq_gemm_mxfp8_fp8blk32",
           W_MXFP8: "bq_gemm_mxfp8_mxfp8", W_A4W4: "bq_gemm_mxfp4_mxfp4",
-          W_GRAD: "bq_gemm_e5m2_mxfp8"}
+          W_GRAD: "bq_gemm_e5m2_mxfp8", W_NVFP4: "bq_gemm_nvfp4_nvfp4"}
 
 
 def _config(block_n=0, split_k=0, swap_ab=-1, split_mode=0, k_chunks=0, cta_pair=0):
@@ -494,6 +525,10 @@ def gemm_mxfp8_mxfp8(a_q, a_sf, b_e4m3, b_sf, M, N, K, **kw):
 
 def gemm_mxfp4_mxfp4(a_fp4, a_sf, b_fp4, b_sf, M, N, K, **kw):
     return gemm(W_A4W4, a_fp4, a_sf, b_fp4, b_sf, M, N, K, **kw)
+
+
+def gemm_nvfp4_nvfp4(a_fp4, a_sf, b_fp4, b_sf, M, N, K, **kw):
+    return gemm(W_NVFP4, a_fp4, a_sf, b_fp4, b_sf, M, N, K, **kw)
 
 
 def gemm_e5m2_mxfp8(a_e5m2, a_sf, b_e4m3, b_sf, M, N, K, **kw):

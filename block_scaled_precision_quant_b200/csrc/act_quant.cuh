@@ -130,6 +130,75 @@ __global__ void __launch_bounds__(256) act_quant_kernel(
   }
 }
 
+// NVFP4 quantization: every value first fp32(x * g) (g the per-tensor scale),
+// then per 16 consecutive values of a row an E4M3 scale s = the smallest E4M3
+// value >= fp32(amax * fp32(1/6)) (2^-9 at least, 448 at most) and E2M1 codes
+// of fp32(x / s), round to nearest even with the sign kept, packed two per
+// byte (even element low).  Scales go to the MMA layout of 16-input groups
+// (an atom covers 64 inputs); padding bytes are 0x38 (1.0: 127 would be an
+// E4M3 NaN).  Work split as act_quant_kernel: a lane owns one group of 16.
+// grid: x*8 + warp = row, y = chunk of 32 groups within the row.
+__global__ void __launch_bounds__(256) nvfp4_quant_kernel(
+    const __nv_bfloat16 *__restrict__ x, int64_t M, int64_t K, int64_t ldx, int64_t rows_pad,
+    float gs, uint8_t *__restrict__ q, uint8_t *__restrict__ sf_mma,
+    uint8_t *__restrict__ sf_row, int *__restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (row >= rows_pad) return;
+  const int64_t G = K >> 4;  // 16-input groups per row
+  const int64_t katoms = (G + 3) >> 2;
+  const int64_t grp = static_cast<int64_t>(blockIdx.y) * 32 + lane;
+  const bool active = row < M && grp < G;
+  const int64_t col = grp * 16;
+  uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+  griddep_wait();
+  griddep_launch_dependents();
+  if (active) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + row * ldx + col);
+    const uint4 v0 = __ldg(src);
+    const uint4 v1 = __ldg(src + 1);
+    w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+    w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+  }
+  uint32_t bad = 0;
+  const uint32_t mx = bf16_amax_bits(w, bad);
+  uint32_t sbyte = 0x38u;
+  if (active) {
+    if (bad && status) atomicOr(status, 1);
+    // max |x g| = fp32(max|x| g): rounding is monotonic
+    const float amax = __fmul_rn(__uint_as_float(mx << 16), gs);
+    const float t = __fmul_rn(amax, __uint_as_float(0x3E2AAAABu));  // fp32(1/6)
+    sbyte = e4m3_ceil(t);
+    const float s = e4m3_value(sbyte);
+    uint32_t packed[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t v = w[4 * h + j];
+        const float lo = __fdiv_rn(__fmul_rn(__uint_as_float(v << 16), gs), s);
+        const float hi = __fdiv_rn(__fmul_rn(__uint_as_float(v & 0xFFFF0000u), gs), s);
+        const uint32_t b = static_cast<uint32_t>(
+            __nv_cvt_float2_to_fp4x2(make_float2(lo, hi), __NV_E2M1, cudaRoundNearest));
+        // each code's sign from its input (and g > 0), so -0 keeps its sign
+        word |= ((b & 0xFFu) | ((v >> 12) & 0x8u) | ((v >> 24) & 0x80u)) << (8 * j);
+      }
+      packed[h] = word;
+    }
+    *reinterpret_cast<uint2 *>(q + row * (K >> 1) + (col >> 1)) = make_uint2(packed[0], packed[1]);
+    if (sf_row) sf_row[row * G + grp] = static_cast<uint8_t>(sbyte);
+  }
+  // groups 4j..4j+3 are lanes 4j..4j+3: one word per four lanes
+  const uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, sbyte, 1);
+  const uint32_t b2 = __shfl_down_sync(0xFFFFFFFFu, sbyte, 2);
+  const uint32_t b3 = __shfl_down_sync(0xFFFFFFFFu, sbyte, 3);
+  if ((lane & 3) == 0 && grp < katoms * 4) {
+    const uint32_t word = sbyte | (b1 << 8) | (b2 << 16) | (b3 << 24);
+    *reinterpret_cast<uint32_t *>(sf_mma + sf_mma_offset(row, grp, katoms)) = word;
+  }
+}
+
 // Transposed quantization (the operands of the weight gradient, and the
 // weight operand of the input gradient): x bf16 [R, ldx] with C columns used,
 // quantized along R -- per 32 consecutive rows of one column -- and written
@@ -474,9 +543,10 @@ __global__ void __launch_bounds__(256, 3) grad_quant_dual_kernel(
 }
 
 // Row-major scales (ROW32: [N, G]; BLK32x32: [ceil(N/32), G] repeated over
-// the 32 rows of each block) -> MMA layout with 127 padding.  One thread per
-// output 32-bit word (4 scale columns of one row).  Flags 255 bytes in
-// flags bit 0.
+// the 32 rows of each block; ROW16_E4M3: [N, G] E4M3 bytes of 16-input
+// groups) -> MMA layout with 127 padding (0x38 for E4M3).  One thread per
+// output 32-bit word (4 scale columns of one row).  Flags NaN scale bytes
+// (E8M0 255, E4M3 0x7F / 0xFF) in flags bit 0.
 __global__ void pack_scales_kernel(const uint8_t *__restrict__ src, int kind, int64_t N, int64_t G,
                                    int64_t rows_pad, uint8_t *__restrict__ dst,
                                    int *__restrict__ flags) {
@@ -490,11 +560,12 @@ __global__ void pack_scales_kernel(const uint8_t *__restrict__ src, int kind, in
     bool nan = false;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      uint32_t b = 127;
+      // kind 2 (ROW16_E4M3): E4M3 bytes, NaN 0x7F / 0xFF, padding 1.0 (0x38)
+      uint32_t b = kind == 2 ? 0x38u : 127u;
       const int64_t c = c0 + j;
       if (r < N && c < G) {
-        b = (kind == 0) ? src[r * G + c] : src[(r >> 5) * G + c];
-        nan |= (b == 255u);
+        b = (kind == 1) ? src[(r >> 5) * G + c] : src[r * G + c];
+        nan |= kind == 2 ? ((b & 0x7Fu) == 0x7Fu) : (b == 255u);
       }
       word |= b << (8 * j);
     }

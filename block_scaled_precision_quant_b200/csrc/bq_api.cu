@@ -6,6 +6,7 @@
 
 #include <algorithm>
 #include <cstdio>
+#include <cmath>
 #include <cstring>
 #include <mutex>
 
@@ -177,7 +178,8 @@ int make_y_map(CUtensorMap* m, const void* y, int64_t M, int64_t N, int64_t ld, 
 // kA4W4: MXFP4 weights with MXFP4 (packed E2M1) activations, kind::mxf4.
 // kGrad: E5M2 gradient codes on the activation side, an E4M3 operand with
 // per-32 scales (MXFP8) on the weight side (the backward GEMMs).
-enum WeightKind { kMxfp4 = 0, kFp8Blk32 = 1, kMxfp8 = 2, kA4W4 = 3, kGrad = 4 };
+// kNv4: NVFP4 x NVFP4 (E4M3 scales per 16), kind::mxf4nvf4.
+enum WeightKind { kMxfp4 = 0, kFp8Blk32 = 1, kMxfp8 = 2, kA4W4 = 3, kGrad = 4, kNv4 = 5 };
 
 struct Plan {
   bool swap = false;
@@ -330,6 +332,16 @@ size_t plan_ws_bytes(const Plan& p) {
 // on request, and wide tiles take 2 chunks per stage (347 vs 354 us).
 int plan_kind(WeightKind wk, int64_t M, int64_t N, int64_t K, int64_t batch,
               const bq_gemm_config* cfg, int num_sms, Plan* p) {
+  if (wk == kNv4) {
+    // NVFP4 stages carry four scale atoms per chunk: one chunk per stage,
+    // unsplit, single-SM tiles
+    bq_gemm_config c = cfg ? *cfg : bq_gemm_config{0, 0, -1, BQ_SPLIT_AUTO, 0, 0};
+    if (c.cta_pair == 2 || c.split_k > 1 || c.k_chunks > 1) return BQ_ERR_INVALID;
+    c.cta_pair = 1;
+    c.split_k = 1;
+    c.k_chunks = 1;
+    return make_plan(M, N, K / 2, batch, &c, num_sms, p);
+  }
   if (wk != kA4W4) return make_plan(M, N, K, batch, cfg, num_sms, p);
   const int64_t Kb = K / 2;
   bq_gemm_config c = cfg ? *cfg : bq_gemm_config{0, 0, -1, BQ_SPLIT_AUTO, 0, 0};
@@ -355,12 +367,12 @@ int plan_for_call(WeightKind wk, int64_t M, int64_t N, int64_t K, int64_t batch,
 // --------------------------------------------------------------- launches --
 
 template <int BN, int STAGES, int ACC, bool SWAP, bool P_FP4, bool Q_FP4, int MODE, int KC,
-          bool FUSEQ = false, bool A4 = false>
+          bool FUSEQ = false, int A4 = 0>
 int launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap& ty,
                 const CUtensorMap& tr, const bq::GemmArgs& args,
                 int64_t units, int num_sms, cudaStream_t stream) {
   constexpr bool CSPLIT = MODE == bq::kSplitCluster;
-  using L = bq::KernelSmem<BN, STAGES, ACC, SWAP, MODE, KC, A4 ? 2 : 1>;
+  using L = bq::KernelSmem<BN, STAGES, ACC, SWAP, MODE, KC, A4 == 2 ? 4 : (A4 ? 2 : 1)>;
   auto kern = bq::gemm_bs_kernel<BN, STAGES, ACC, SWAP, P_FP4, Q_FP4, MODE, KC, FUSEQ, A4>;
   static bool attr_set[kMaxDevices] = {};
   static int per_sm_cache[kMaxDevices] = {};
@@ -417,12 +429,12 @@ int launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap&
 }
 
 template <int BN, int STAGES, int ACC, bool SWAP, int MODE, int KC, bool FUSEQ = false,
-          bool A4 = false>
+          int A4 = 0>
 int launch_kind(bool w_fp4, const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap& ty,
                 const CUtensorMap& tr, const bq::GemmArgs& args, int64_t u, int num_sms,
                 cudaStream_t st) {
-  if constexpr (A4)  // packed E2M1 on both sides: plain byte operands
-    return launch_gemm<BN, STAGES, ACC, SWAP, false, false, MODE, KC, false, true>(
+  if constexpr (A4 != 0)  // packed E2M1 on both sides: plain byte operands
+    return launch_gemm<BN, STAGES, ACC, SWAP, false, false, MODE, KC, false, A4>(
         tp, tq, ty, tr, args, u, num_sms, st);
   // FP4 weights sit on the P side with SWAP, on the Q side otherwise.
   if (w_fp4)
@@ -477,7 +489,7 @@ int launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
 
 // Dispatch on (swap, bn, chunks per stage, split mode, weight format) to the
 // compiled instances.  Stage counts fill ~200 KB of shared memory.
-template <bool A4>
+template <int A4>
 int run_gemm(const Plan& pl, bool w_fp4, const CUtensorMap& tp, const CUtensorMap& tq,
              const CUtensorMap& ty, const CUtensorMap& tr, const bq::GemmArgs& a, int ns,
              cudaStream_t st) {
@@ -517,6 +529,23 @@ int run_gemm(const Plan& pl, bool w_fp4, const CUtensorMap& tp, const CUtensorMa
              : launch_kind<64, 8, 1, true, kNone, 1, false, A4>(w_fp4, tp, tq, ty, tr, a, u, ns, st);
 }
 
+// NVFP4 x NVFP4: one chunk per stage (four scale atoms each), unsplit.
+int run_gemm_nv(const Plan& pl, const CUtensorMap& tp, const CUtensorMap& tq,
+                const CUtensorMap& ty, const CUtensorMap& tr, const bq::GemmArgs& a, int ns,
+                cudaStream_t st) {
+  const int64_t u = pl.units;
+  constexpr int kNone = bq::kSplitNone;
+  if (!pl.swap)
+    return pl.bn == 256
+               ? launch_kind<256, 3, 1, false, kNone, 1, false, 2>(false, tp, tq, ty, tr, a, u,
+                                                                   ns, st)
+               : launch_kind<128, 5, 2, false, kNone, 1, false, 2>(false, tp, tq, ty, tr, a, u,
+                                                                   ns, st);
+  return pl.bn == 32
+             ? launch_kind<32, 6, 1, true, kNone, 1, false, 2>(false, tp, tq, ty, tr, a, u, ns, st)
+             : launch_kind<64, 6, 1, true, kNone, 1, false, 2>(false, tp, tq, ty, tr, a, u, ns, st);
+}
+
 // Activations given as bf16 and quantized inside the GEMM (decode tiles).
 struct FusedAct {
   const void* x;
@@ -553,7 +582,7 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
   }
   if (q_out && (!aligned(q_out, 16) || !aligned(sf_out, 4))) return BQ_ERR_ALIGN;
   const bool w_fp4 = wk == kMxfp4;
-  const bool a4 = wk == kA4W4;
+  const bool a4 = wk == kA4W4 || wk == kNv4;  // packed E2M1 activations and weights
   if (a4 && fused) return BQ_ERR_INVALID;  // the fused quantizer emits E4M3 codes
   // Bytes of K per operand row: packed E2M1 rows hold two codes per byte.
   const int64_t Kb = a4 ? K / 2 : K;
@@ -657,7 +686,7 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
   g.tiles_p = pl.tiles_p;
   g.tiles_q = pl.tiles_q;
   g.raster_group = 8;
-  g.sf_katoms = ceil_div(K, 128);
+  g.sf_katoms = ceil_div(K, wk == kNv4 ? 64 : 128);  // scale atoms: 4 groups of 16 or 32
   g.sf_q_rowatoms = ceil_div(pl.swap ? M : N, 128);
   // the fused quantizer lays the activation tile out with chunks BN rows apart
   g.q_box_rows = fused ? pl.bn : (pl.swap ? a_box : b_box);
@@ -720,11 +749,14 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
   }
   const CUtensorMap& tp = pl.swap ? map_b : map_a;
   const CUtensorMap& tq = pl.swap ? map_a : map_b;
+  if (wk == kNv4)
+    return run_gemm_nv(pl, tp, tq, map_y, map_res, g, dev->num_sms,
+                       reinterpret_cast<cudaStream_t>(stream));
   if (a4)
-    return run_gemm<true>(pl, false, tp, tq, map_y, map_res, g, dev->num_sms,
-                          reinterpret_cast<cudaStream_t>(stream));
-  return run_gemm<false>(pl, w_fp4, tp, tq, map_y, map_res, g, dev->num_sms,
-                         reinterpret_cast<cudaStream_t>(stream));
+    return run_gemm<1>(pl, false, tp, tq, map_y, map_res, g, dev->num_sms,
+                       reinterpret_cast<cudaStream_t>(stream));
+  return run_gemm<0>(pl, w_fp4, tp, tq, map_y, map_res, g, dev->num_sms,
+                     reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // namespace
@@ -756,6 +788,11 @@ int bq_version(void) { return 100; }
 size_t bq_sf_bytes(int64_t rows, int64_t K) {
   if (rows < 0 || K <= 0 || K % 32 != 0) return 0;
   return static_cast<size_t>((rows + 127) / 128) * static_cast<size_t>((K + 127) / 128) * 512;
+}
+
+size_t bq_sf_bytes_nvfp4(int64_t rows, int64_t K) {
+  if (rows < 0 || K <= 0 || K % 16 != 0) return 0;
+  return static_cast<size_t>((rows + 127) / 128) * static_cast<size_t>((K + 63) / 64) * 512;
 }
 
 }  // extern "C"
@@ -895,6 +932,40 @@ int bq_act_quant_mxfp4(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, vo
                           d_status, stream);
 }
 
+int bq_act_quant_nvfp4(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, float g,
+                       void* q_fp4, void* sf_mma, void* sf_rowmajor, int* d_status,
+                       bq_stream_t stream) {
+  DevInfo* dev = nullptr;
+  int st = current_device(&dev);
+  if (st != BQ_OK) return st;
+  if (M < 0 || K <= 0 || K % 32 != 0 || ldx < K) return BQ_ERR_SHAPE;
+  if (!(g > 0.0f) || !std::isfinite(g)) return BQ_ERR_INVALID;
+  if (M == 0) return BQ_OK;
+  if (!x_bf16 || !q_fp4 || !sf_mma) return BQ_ERR_NULL;
+  if (!aligned(x_bf16, 16) || ldx % 8 != 0 || !aligned(q_fp4, 16) || !aligned(sf_mma, 4))
+    return BQ_ERR_ALIGN;
+  const int64_t rows_pad = (M + 127) / 128 * 128;
+  const int64_t chunks = (K / 16 + 31) / 32;
+  if (rows_pad / 8 > 0x7FFFFFFF || chunks > 65535) return BQ_ERR_SHAPE;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(static_cast<unsigned>(rows_pad / 8), static_cast<unsigned>(chunks));
+  lc.blockDim = dim3(256);
+  lc.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  if (cudaLaunchKernelEx(&lc, bq::nvfp4_quant_kernel, static_cast<const __nv_bfloat16*>(x_bf16),
+                         M, K, ldx, rows_pad, g, static_cast<uint8_t*>(q_fp4),
+                         static_cast<uint8_t*>(sf_mma), static_cast<uint8_t*>(sf_rowmajor),
+                         d_status) != cudaSuccess) {
+    cudaGetLastError();
+    return BQ_ERR_CUDA;
+  }
+  return launch_status();
+}
+
 int bq_grad_quant(const void* g_bf16, int64_t M, int64_t K, int64_t ldg, void* q_e5m2,
                   void* sf_mma, void* sf_rowmajor, int* d_status, int rounding, uint64_t seed,
                   bq_stream_t stream) {
@@ -927,14 +998,15 @@ int bq_pack_weight_scales(const void* scales_u8, int kind, int64_t N, int64_t K,
   DevInfo* dev = nullptr;
   int st = current_device(&dev);
   if (st != BQ_OK) return st;
-  if (kind != BQ_SF_ROW32 && kind != BQ_SF_BLK32x32) return BQ_ERR_INVALID;
-  if (N < 0 || K <= 0 || K % 32 != 0) return BQ_ERR_SHAPE;
+  if (kind != BQ_SF_ROW32 && kind != BQ_SF_BLK32x32 && kind != BQ_SF_ROW16_E4M3)
+    return BQ_ERR_INVALID;
+  if (N < 0 || K <= 0 || K % (kind == BQ_SF_ROW16_E4M3 ? 16 : 32) != 0) return BQ_ERR_SHAPE;
   if (N == 0) return BQ_OK;
   if (!scales_u8 || !sf_mma) return BQ_ERR_NULL;
   if (!aligned(sf_mma, 4) || (e4m3_codes && !aligned(e4m3_codes, 16))) return BQ_ERR_ALIGN;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(dev->flags_ptr, 0, sizeof(int), s) != cudaSuccess) return BQ_ERR_CUDA;
-  const int64_t G = K / 32;
+  const int64_t G = K / (kind == BQ_SF_ROW16_E4M3 ? 16 : 32);
   const int64_t rows_pad = (N + 127) / 128 * 128;
   const int64_t words = rows_pad * ((G + 3) / 4);
   const int64_t blocks = (words + 255) / 256 < 4096 ? (words + 255) / 256 : 4096;
@@ -1015,6 +1087,21 @@ int bq_gemm_e5m2_mxfp8_epilogue(const void* a_e5m2, const void* a_sf, const void
                     workspace_bytes, cfg, stream);
 }
 
+int bq_gemm_nvfp4_nvfp4(const void* a_fp4, const void* a_sf, const void* b_fp4, const void* b_sf,
+                        int64_t M, int64_t N, int64_t K, void* y_bf16, bq_stream_t stream) {
+  return gemm_entry(kNv4, a_fp4, a_sf, b_fp4, b_sf, M, N, K, y_bf16, nullptr, nullptr, nullptr, 0,
+                    nullptr, stream);
+}
+
+int bq_gemm_nvfp4_nvfp4_epilogue(const void* a_fp4, const void* a_sf, const void* b_fp4,
+                                 const void* b_sf, int64_t M, int64_t N, int64_t K, void* y_bf16,
+                                 const bq_epilogue* epi, const bq_batch* batch, void* workspace,
+                                 size_t workspace_bytes, const bq_gemm_config* cfg,
+                                 bq_stream_t stream) {
+  return gemm_entry(kNv4, a_fp4, a_sf, b_fp4, b_sf, M, N, K, y_bf16, epi, batch, workspace,
+                    workspace_bytes, cfg, stream);
+}
+
 int bq_gemm_mxfp4_mxfp4(const void* a_fp4, const void* a_sf, const void* b_fp4, const void* b_sf,
                         int64_t M, int64_t N, int64_t K, void* y_bf16, bq_stream_t stream) {
   return gemm_entry(kA4W4, a_fp4, a_sf, b_fp4, b_sf, M, N, K, y_bf16, nullptr, nullptr, nullptr, 0,
@@ -1032,7 +1119,7 @@ int bq_gemm_mxfp4_mxfp4_epilogue(const void* a_fp4, const void* a_sf, const void
 
 size_t bq_gemm_workspace_bytes(int weight_kind, int64_t M, int64_t N, int64_t K, int64_t batch,
                                const bq_gemm_config* cfg) {
-  if (weight_kind < 0 || weight_kind > 4 || M <= 0 || N <= 0 || K <= 0 || batch <= 0) return 0;
+  if (weight_kind < 0 || weight_kind > 5 || M <= 0 || N <= 0 || K <= 0 || batch <= 0) return 0;
   DevInfo* dev = nullptr;
   if (current_device(&dev) != BQ_OK) return 0;
   Plan pl;
@@ -1045,7 +1132,7 @@ size_t bq_gemm_workspace_bytes(int weight_kind, int64_t M, int64_t N, int64_t K,
 int bq_gemm_plan(int weight_kind, int64_t M, int64_t N, int64_t K, int64_t batch,
                  const bq_gemm_config* cfg, int num_sms, bq_gemm_config* out) {
   if (!out) return BQ_ERR_NULL;
-  if (weight_kind < 0 || weight_kind > 4) return BQ_ERR_INVALID;
+  if (weight_kind < 0 || weight_kind > 5) return BQ_ERR_INVALID;
   if (M <= 0 || N <= 0 || K <= 0 || K % 32 != 0 || batch <= 0 || num_sms < 1)
     return BQ_ERR_SHAPE;
   Plan pl;

@@ -812,7 +812,7 @@ __device__ __forceinline__ bool fused_quant_unit(const GemmArgs &a, const UnitPo
 }
 
 template <int BN, int STAGES, int ACC, bool SWAP, bool P_FP4, bool Q_FP4, int MODE, int KC,
-          bool FUSEQ = false, bool A4 = false>
+          bool FUSEQ = false, int A4 = 0>
 __global__ void __launch_bounds__(kNumThreads, 1)
     gemm_bs_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_y,
@@ -820,10 +820,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   constexpr bool CSPLIT = MODE == kSplitCluster;
   static_assert(!CSPLIT || SWAP, "cluster split-K is built for the swap-AB (decode) tiles");
   static_assert(!CSPLIT || ACC == 1, "cluster split-K uses one accumulator");
-  // A4: both operands packed E2M1 with E8M0 scales (kind::mxf4, K = 64 per
-  // MMA); a 128-byte chunk is 256 K and spans two scale atoms.
+  // A4: both operands packed E2M1 (K = 64 per MMA); a 128-byte chunk is 256 K.
+  //   A4 == 1: MXFP4, E8M0 scales per 32 (kind::mxf4): two scale atoms a chunk;
+  //   A4 == 2: NVFP4, E4M3 scales per 16 (kind::mxf4nvf4): four atoms a chunk.
   static_assert(!A4 || (!P_FP4 && !Q_FP4 && !FUSEQ), "A4 operands are plain packed bytes");
-  constexpr int APC = A4 ? 2 : 1;
+  constexpr int APC = A4 == 2 ? 4 : (A4 ? 2 : 1);
   using L = KernelSmem<BN, STAGES, ACC, SWAP, MODE, KC, APC>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -1006,7 +1007,16 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 #pragma unroll
             for (int ks = 0; ks < kBlockK / kMmaK; ++ks) {
               const uint32_t acc_in = (kt > u.kt0 || c > 0 || ks > 0) ? 1u : 0u;
-              if constexpr (A4) {
+              if constexpr (A4 == 2) {
+                // 64 K per MMA: atom ks, its four scale bytes (16 K each, E4M3)
+                if (ks < na) {
+                  const uint32_t idesc =
+                      make_idesc(kFmtMxf4E2M1, kFmtMxf4E2M1, BN, 0) & ~(1u << 23);  // UE4M3
+                  tc_mma_nvf4(d_tmem, desc_kmajor_sw128(pa + ks * kMmaK),
+                              desc_kmajor_sw128(qa + ks * kMmaK), idesc, sf_t + 4 * ks,
+                              sfq_t + 4 * ks * L::kSfqAtoms + sfq_row_off, acc_in);
+                }
+              } else if constexpr (A4) {
                 // 64 K per MMA: atom ks / 2, scale bytes 2 (ks % 2) and 2 (ks % 2) + 1
                 const int t = ks >> 1;
                 if (t < na) {

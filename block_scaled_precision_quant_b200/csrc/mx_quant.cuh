@@ -12,6 +12,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <stdint.h>
@@ -35,6 +36,20 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
 __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
   return static_cast<uint32_t>(
       __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
+}
+
+// The value of a non-negative finite E4M3 byte.
+__device__ __forceinline__ float e4m3_value(uint32_t byte) {
+  const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(byte), __NV_E4M3);
+  return __half2float(__half(h));
+}
+
+// The smallest positive E4M3 value >= t (t >= 0): the nearest one, moved up
+// one code when below t; at least 2^-9 (byte 1), at most 448 (byte 0x7E).
+__device__ __forceinline__ uint32_t e4m3_ceil(float t) {
+  uint32_t b = e4m3x2(t, 0.0f) & 0xFFu;  // nearest, saturating at 448
+  if (b < 0x7Eu && e4m3_value(b) < t) ++b;
+  return b < 1u ? 1u : b;
 }
 
 // Largest magnitude bits (15 bits, sign dropped) of the bf16 pairs in w: an

@@ -77,6 +77,11 @@ int bq_version(void);
  * (K % 32 == 0): ceil(rows / 128) * ceil(K / 128) * 512.  0 for bad sizes. */
 size_t bq_sf_bytes(int64_t rows, int64_t K);
 
+/* Bytes of an MMA-layout buffer of NVFP4 scales (one E4M3 byte per 16 inputs,
+ * K % 16 == 0): ceil(rows / 128) * ceil(K / 64) * 512 (an atom holds 4 groups
+ * of 16).  0 for bad sizes. */
+size_t bq_sf_bytes_nvfp4(int64_t rows, int64_t K);
+
 /* ---- activation quantization ------------------------------------------ */
 
 /* bq_act_quant -- per-32 MX quantization of bf16 activations
@@ -113,6 +118,26 @@ int bq_act_quant(const void *x_bf16, int64_t M, int64_t K, int64_t ldx, void *q_
  *   all other arguments and errors as bq_act_quant. */
 int bq_act_quant_mxfp4(const void *x_bf16, int64_t M, int64_t K, int64_t ldx, void *q_fp4,
                        void *sf_mma, void *sf_rowmajor, int *d_status, bq_stream_t stream);
+
+/* bq_act_quant_nvfp4 -- NVFP4 quantization of bf16 activations for the NVFP4
+ * A4W4 GEMM (the "fp4-gemm" page, README: NVFP4 A4W4 kernels, E2M1 codes with
+ * CUTLASS-layout scale buffers).  The pages give no quantization rule; this
+ * one: every value is first fp32(x * g), g > 0 the caller's per-tensor scale;
+ * per 16 consecutive values of a row the scale is s = the smallest E4M3 value
+ * >= fp32(amax * fp32(1/6)) (2^-9 at least, 448 at most: the round-up
+ * counterpart of bq_act_quant's rule, so no value clips unless amax g > 2688)
+ * and q = E2M1 round-to-nearest-even of fp32(x g / s), sign kept.  A GEMM of
+ * two such operands returns alpha * sum(q_a s_a q_b s_b); alpha = 1 / (g_a g_b)
+ * in the epilogue gives the product of the unscaled tensors.
+ *   q_fp4   out [M, K/2] packed E2M1 (even element low), 16-byte aligned
+ *   sf_mma  out bq_sf_bytes_nvfp4(M, K): MMA layout of 16-input groups,
+ *           padding bytes 0x38 (1.0)
+ *   sf_rowmajor optional out [M, K/16]; K % 32 == 0; other arguments as
+ *   bq_act_quant.  Errors: as bq_act_quant, BQ_ERR_INVALID for g <= 0 or not
+ *   finite. */
+int bq_act_quant_nvfp4(const void *x_bf16, int64_t M, int64_t K, int64_t ldx, float g,
+                       void *q_fp4, void *sf_mma, void *sf_rowmajor, int *d_status,
+                       bq_stream_t stream);
 
 /* ---- backward-pass quantizers ------------------------------------------- */
 
@@ -172,7 +197,9 @@ int bq_grad_quant_dual(const void *g_bf16, int64_t R, int64_t C, int64_t ldg, in
 
 enum {
   BQ_SF_ROW32 = 0,    /* scales [N, K/32]: one per 32 inputs of a row (MXFP4, MXFP8) */
-  BQ_SF_BLK32x32 = 1  /* scales [ceil(N/32), ceil(K/32)]: one per 32x32 block (FP8 weights) */
+  BQ_SF_BLK32x32 = 1, /* scales [ceil(N/32), ceil(K/32)]: one per 32x32 block (FP8 weights) */
+  BQ_SF_ROW16_E4M3 = 2 /* NVFP4: E4M3 scales [N, K/16], one per 16 inputs of a row; output
+                          bq_sf_bytes_nvfp4(N, K) bytes, padding 0x38; 0x7F/0xFF refused */
 };
 
 /* bq_pack_weight_scales -- E8M0 weight scales to MMA layout
@@ -239,6 +266,17 @@ int bq_gemm_mxfp8_mxfp8(const void *a_q, const void *a_sf, const void *b_e4m3, c
  * The pages' A4W4 kernels use NVFP4 (E4M3 scales per 16 inputs); that scale
  * format is not implemented here. */
 int bq_gemm_mxfp4_mxfp4(const void *a_fp4, const void *a_sf, const void *b_fp4, const void *b_sf,
+                        int64_t M, int64_t N, int64_t K, void *y_bf16, bq_stream_t stream);
+
+/* bq_gemm_nvfp4_nvfp4 -- the NVFP4 A4W4 product ("fp4-gemm" page, README
+ * "Available Functions": the bf16-output NVFP4 GEMM with alpha) on
+ * tcgen05.mma kind::mxf4nvf4 (scale_vec::4X, UE4M3 scales): a_fp4 / b_fp4
+ * packed E2M1 [M, K/2] / [N, K/2], a_sf from bq_act_quant_nvfp4, b_sf from
+ * bq_pack_weight_scales(BQ_SF_ROW16_E4M3).  K % 128 == 0.  Schedules: wide
+ * tiles (128 x 128, 128 x 256) and unsplit swap-AB decode tiles, one 256-K
+ * chunk per stage; a K split, pair tiles or more chunks per stage are
+ * refused (BQ_ERR_INVALID).  Everything else as the other GEMMs. */
+int bq_gemm_nvfp4_nvfp4(const void *a_fp4, const void *a_sf, const void *b_fp4, const void *b_sf,
                         int64_t M, int64_t N, int64_t K, void *y_bf16, bq_stream_t stream);
 
 /* bq_gemm_e5m2_mxfp8 -- the backward products: A holds E5M2 gradient codes
@@ -323,7 +361,8 @@ typedef struct {
 
 /* Workspace bytes the *_epilogue calls need for a problem (0 when the chosen
  * schedule needs none).  weight_kind: 0 mxfp4, 1 fp8blk32, 2 mxfp8, 3 mxfp4 weights
- * with MXFP4 activations (bq_gemm_mxfp4_mxfp4*), 4 E5M2 x MXFP8 (bq_gemm_e5m2_mxfp8*). */
+ * with MXFP4 activations (bq_gemm_mxfp4_mxfp4*), 4 E5M2 x MXFP8 (bq_gemm_e5m2_mxfp8*),
+ * 5 NVFP4 x NVFP4 (bq_gemm_nvfp4_nvfp4*). */
 size_t bq_gemm_workspace_bytes(int weight_kind, int64_t M, int64_t N, int64_t K, int64_t batch,
                                const bq_gemm_config *cfg);
 
@@ -359,6 +398,13 @@ int bq_gemm_mxfp8_fp8blk32_epilogue(const void *a_q, const void *a_sf, const voi
                                     void *workspace, size_t workspace_bytes,
                                     const bq_gemm_config *cfg, bq_stream_t stream);
 int bq_gemm_mxfp8_mxfp8_epilogue(const void *a_q, const void *a_sf, const void *b_e4m3,
+                                 const void *b_sf, int64_t M, int64_t N, int64_t K, void *y_bf16,
+                                 const bq_epilogue *epi, const bq_batch *batch, void *workspace,
+                                 size_t workspace_bytes, const bq_gemm_config *cfg,
+                                 bq_stream_t stream);
+/* NVFP4 x NVFP4 with the same epilogue (alpha = 1 / (g_a g_b) undoes the
+ * per-tensor scales), batch and schedule options within the limits above. */
+int bq_gemm_nvfp4_nvfp4_epilogue(const void *a_fp4, const void *a_sf, const void *b_fp4,
                                  const void *b_sf, int64_t M, int64_t N, int64_t K, void *y_bf16,
                                  const bq_epilogue *epi, const bq_batch *batch, void *workspace,
                                  size_t workspace_bytes, const bq_gemm_config *cfg,
