@@ -223,12 +223,30 @@ __device__ __forceinline__ UnitPos unit_pos(const GemmArgs &a, int unit) {
   return u;
 }
 
-// erf-form GELU, inline: an out-of-line call per element costs the unrolled
-// epilogue its registers at every call and dominated GELU layers.  Callers
-// branch on the activation once per group of values, so code without GELU
-// never runs through it.
+// erf-form GELU, 0.5 t (1 + erf(t / sqrt 2)), inline: an out-of-line call
+// per element costs the unrolled epilogue its registers at every call.
+// erf is the rational-exponential approximation of Abramowitz and Stegun,
+// Handbook of Mathematical Functions, formula 7.1.26 (after Hastings):
+//   erf(x) = 1 - (a1 u + a2 u^2 + a3 u^3 + a4 u^4 + a5 u^5) exp(-x^2),
+//   u = 1 / (1 + p x), x >= 0, odd in x, absolute error <= 1.5e-7,
+// evaluated with the fast division and exponential (relative errors near
+// 2^-22): one branch-free formula, so the epilogue's values interleave.  The
+// GELU's error is then below 1e-7 |t|, far inside the GEMM's tolerance
+// (2^-20 |alpha| sum |a b| + |bias| >= 1e-6 |t|) and half a bf16 ulp of large
+// outputs.  Callers branch on the activation once per group of values, so
+// code without GELU never runs through it.
 __device__ __forceinline__ float gelu_erf(float t) {
-  return 0.5f * t * (1.0f + erff(t * 0.70710678118654752f));
+  const float x = fabsf(t) * 0.70710678118654752f;
+  const float u = __fdividef(1.0f, fmaf(0.3275911f, x, 1.0f));
+  float poly = fmaf(u, 1.061405429f, -1.453152027f);
+  poly = fmaf(u, poly, 1.421413741f);
+  poly = fmaf(u, poly, -0.284496736f);
+  poly = fmaf(u, poly, 0.254829592f);
+  poly *= u;
+  const float erfc_x = poly * __expf(-x * x);  // 1 - erf(x)
+  // 1 + erf(t / sqrt 2): 2 - erfc for t >= 0, erfc for t < 0 (odd erf)
+  const float one_plus = t >= 0.0f ? 2.0f - erfc_x : erfc_x;
+  return 0.5f * t * one_plus;
 }
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) {
