@@ -373,6 +373,8 @@ int launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap&
                 int64_t units, int num_sms, cudaStream_t stream) {
   constexpr bool CSPLIT = MODE == bq::kSplitCluster;
   using L = bq::KernelSmem<BN, STAGES, ACC, SWAP, MODE, KC, A4 == 2 ? 4 : (A4 ? 2 : 1)>;
+  // unsplit wide tiles run a second group of epilogue warps
+  constexpr int kThreads = (!SWAP && MODE == bq::kSplitNone) ? bq::kWideThreads : bq::kNumThreads;
   auto kern = bq::gemm_bs_kernel<BN, STAGES, ACC, SWAP, P_FP4, Q_FP4, MODE, KC, FUSEQ, A4>;
   static bool attr_set[kMaxDevices] = {};
   static int per_sm_cache[kMaxDevices] = {};
@@ -385,7 +387,7 @@ int launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap&
                              cudaSharedmemCarveoutMaxShared) != cudaSuccess)
       return BQ_ERR_CUDA;
     int per_sm = 1;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, bq::kNumThreads, L::kBytes);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, L::kBytes);
     if (per_sm < 1) per_sm = 1;
     // Co-resident CTAs share the SM's 512 TMEM columns.
     const int tmem_fit = 512 / L::kTmemCols;
@@ -400,7 +402,7 @@ int launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap&
   if (grid > units) grid = units;  // units is a multiple of S
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3(static_cast<unsigned>(grid));
-  lc.blockDim = dim3(bq::kNumThreads);
+  lc.blockDim = dim3(kThreads);
   lc.dynamicSmemBytes = L::kBytes;
   lc.stream = stream;
   cudaLaunchAttribute attr[2];

@@ -54,6 +54,13 @@ constexpr int kActWarp = 6;
 constexpr int kWsfWarp = 7;
 constexpr int kAsfWarp = 8;
 constexpr int kCopyThreads = 4;
+// Unsplit wide tiles (activation rows on the TMEM lanes) add a second group
+// of four epilogue warps (9-12, one per TMEM lane quadrant): the two groups
+// take alternate 32-column chunks of the accumulator, so an epilogue with a
+// heavy activation (erf-GELU) or one accumulator (128 x 256 tiles) takes
+// half the time next to the mainloop.
+constexpr int kWideThreads = kNumThreads + 128;
+constexpr int kEpi2FirstThread = (kAsfWarp + 1) * 32;  // first thread of the second group
 
 // tcgen05 operand formats (instruction descriptor fields a_format / b_format):
 // kind::mxf8f6f4 codes E4M3 0, E5M2 1 and E2M1 5 (one byte slot per FP4 code in
@@ -341,9 +348,10 @@ __device__ __forceinline__ void emit32(const GemmArgs &a, int b, int prow, int q
   }
 }
 
-__device__ __forceinline__ void epi_bar_sync() {
+__device__ __forceinline__ void epi_bar_sync(int group = 0) {
   __syncwarp();
-  asm volatile("barrier.sync 1, 128;" ::: "memory");  // the 4 epilogue warps
+  // the 4 warps of epilogue group `group` (named barriers 1 and 2)
+  asm volatile("barrier.sync %0, 128;" ::"r"(1 + group) : "memory");
 }
 
 // Quantized output of one 32-group: row m, columns q0 .. q0+31, the bf16
@@ -546,6 +554,107 @@ __device__ __forceinline__ void epilogue_rows_tma(const GemmArgs &a, const CUten
     if (res && epi_tid == 0 && c + 2 < nch) {
       bulk_wait_group_read<0>();  // this chunk's store has read the slot
       load_res(c + 2);
+    }
+  }
+}
+
+// The same with two epilogue groups (unsplit wide tiles of gemm_bs_kernel):
+// group g takes chunks g, g + 2, ... of the accumulator row and staging slot
+// g; its first thread waits for the group's previous TMA store to have read
+// the slot before the slot is refilled (with the next chunk's residual, by a
+// TMA load on rbar[g], or with outputs).  `rphase` bit g carries the slot
+// barrier's parity.
+template <int NCOLS>
+__device__ __forceinline__ void epilogue_rows_tma_g2(const GemmArgs &a, const CUtensorMap *tm_y,
+                                                     const CUtensorMap *tm_res, uint64_t *rbar,
+                                                     uint32_t &rphase, uint32_t t_row, int b,
+                                                     int m0, int n0, int row, int epi_tid,
+                                                     int group, uint8_t *ystage,
+                                                     volatile int *abort_flag) {
+  const int m = m0 + row;
+  const bool res = a.res != nullptr;
+  const int nch = min(NCOLS / 32, (a.N - n0 + 31) / 32);
+  uint8_t *buf = ystage + group * kYChunkBytes;
+  const bool batched_res = a.batch > 1 && a.res_bstride != 0;
+#pragma unroll 1
+  for (int c = group; c < nch; c += 2) {
+    const int q0 = n0 + c * 32;
+    if (epi_tid == 0) {
+      bulk_wait_group_read<0>();  // the group's previous store has read the slot
+      if (res) {
+        mbar_arrive_expect_tx(&rbar[group], static_cast<uint32_t>(kYChunkBytes));
+        if (batched_res)
+          tma_load_3d(buf, tm_res, &rbar[group], q0, m0, b);
+        else
+          tma_load_2d(buf, tm_res, &rbar[group], q0, m0);
+      }
+    }
+    uint32_t v[32];
+    __syncwarp();
+    tmem_ld_32x32b_x32(t_row + c * 32, v);
+    tmem_ld_wait();
+    uint4 rv[4];
+    if (res) {
+      if (!mbar_wait(&rbar[group], (rphase >> group) & 1u, a.err, abort_flag, kWaitEpiFull))
+        return;
+      rphase ^= 1u << group;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        rv[j] = *reinterpret_cast<const uint4 *>(buf + row * 64 + ((j ^ ((row >> 1) & 3)) << 4));
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) rv[j] = make_uint4(0u, 0u, 0u, 0u);
+      if (a.y) epi_bar_sync(group);  // the slot is free
+    }
+    uint32_t o[16];
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      float bias8[8];
+      if (a.bias && q0 + 8 * g < a.N) {
+        const uint4 bv = __ldg(reinterpret_cast<const uint4 *>(a.bias + q0 + 8 * g));
+        const uint32_t w[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          bias8[2 * j] = bf16_bits_to_f32(w[j] & 0xFFFF);
+          bias8[2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) bias8[j] = 0.0f;
+      }
+      float t[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) t[j] = a.alpha * __uint_as_float(v[8 * g + j]) + bias8[j];
+      if (a.act == 1) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) t[j] = gelu_erf(t[j]);
+      }
+      const uint32_t rw[4] = {rv[g].x, rv[g].y, rv[g].z, rv[g].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __nv_bfloat162 p2 =
+            __floats2bfloat162_rn(t[2 * j] + bf16_bits_to_f32(rw[j] & 0xFFFF),
+                                  t[2 * j + 1] + bf16_bits_to_f32(rw[j] >> 16));
+        o[4 * g + j] = *reinterpret_cast<const uint32_t *>(&p2);
+      }
+    }
+    if (a.q_out) quant_out_row32(a, b, m, q0, o);
+    if (a.y) {  // uniform
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<uint4 *>(buf + row * 64 + ((j ^ ((row >> 1) & 3)) << 4)) =
+            make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+      fence_proxy_async_smem();
+      epi_bar_sync(group);
+      if (epi_tid == 0) {
+        if (a.batch > 1)
+          tma_store_3d(tm_y, buf, q0, m0, b);
+        else
+          tma_store_2d(tm_y, buf, q0, m0);
+        bulk_commit_group();
+      }
+    } else if (res) {
+      epi_bar_sync(group);  // every row has read its residual before the next load
     }
   }
 }
@@ -831,7 +940,7 @@ __device__ __forceinline__ bool fused_quant_unit(const GemmArgs &a, const UnitPo
 
 template <int BN, int STAGES, int ACC, bool SWAP, bool P_FP4, bool Q_FP4, int MODE, int KC,
           bool FUSEQ = false, int A4 = 0>
-__global__ void __launch_bounds__(kNumThreads, 1)
+__global__ void __launch_bounds__((!SWAP && MODE == kSplitNone) ? kWideThreads : kNumThreads, 1)
     gemm_bs_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_y,
                    const __grid_constant__ CUtensorMap tm_res, const GemmArgs a) {
@@ -896,7 +1005,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     }
     for (int st = 0; st < ACC; ++st) {
       mbar_init(&tfull[st], 1);
-      mbar_init(&tempty[st], 4);  // one arrival per epilogue warp
+      // one arrival per epilogue warp (two groups on unsplit wide tiles)
+      mbar_init(&tempty[st], (!SWAP && MODE == kSplitNone) ? 8 : 4);
     }
     mbar_init(drain, 1);
     if constexpr (CSPLIT) {
@@ -932,7 +1042,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0 || warp >= kActWarp) {
+  if (warp == 0 || (warp >= kActWarp && warp <= kAsfWarp)) {
     // ----------------------------------------------------------- producers --
     // All four walk the same stage ring; each arrives once per stage with the
     // bytes of its own part.  The weight copies never wait for the preceding
@@ -1074,7 +1184,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     // ------------------------------------------------------------ epilogue --
     const int quad = warp % 4;  // TMEM lane quadrant this warp may access
     const int row = quad * 32 + lane;
-    const int epi_tid = threadIdx.x - 64;  // 0..127
+    // epilogue group 0: warps 2-5; group 1 (unsplit wide tiles): warps 9-12
+    const int egroup = warp > kAsfWarp ? 1 : 0;
+    const int epi_tid = threadIdx.x - (egroup ? kEpi2FirstThread : 64);  // 0..127
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t ready_phase = 0, free_phase = 0, land_phase = 0;
@@ -1194,9 +1306,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           copy_out_swap<BN>(a, u, epi_tid, stage);
         if (unit + static_cast<int>(gridDim.x) < total_units) epi_bar_sync();  // staging free
       } else if constexpr (MODE == kSplitNone) {
-        epilogue_rows_tma<BN>(a, &tm_y, &tm_res, full + L::kRbarIndex, rphase, t_row, u.b,
-                              u.tp * kBlockP, u.tq * BN, row, epi_tid, smem + L::kOffYStage,
-                              abort_flag);
+        epilogue_rows_tma_g2<BN>(a, &tm_y, &tm_res, full + L::kRbarIndex, rphase, t_row, u.b,
+                                 u.tp * kBlockP, u.tq * BN, row, epi_tid, egroup,
+                                 smem + L::kOffYStage, abort_flag);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -1398,7 +1510,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 
   // The epilogue's last TMA stores must be done before the CTA retires.
   if constexpr (L::kBytesYStage > 0)
-    if (threadIdx.x == 64) bulk_wait_group_all();
+    if (threadIdx.x == 64 || threadIdx.x == kEpi2FirstThread) bulk_wait_group_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
