@@ -267,13 +267,11 @@ int make_plan(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_conf
   const bool pow2 = (splits & (splits - 1)) == 0;
   p->cluster = p->swap && splits > 1 && pow2 && splits <= kMaxClusterSplit && !use_ws;
   if (req_mode == BQ_SPLIT_CLUSTER && splits > 1 && !p->cluster) return BQ_ERR_INVALID;
-  // 256x256 pair tiles (sweeps: ~5 % over the best single-SM tile once a
-  // tile's K loop is >= 32 blocks and each pair walks >= 4 tiles, where the
-  // steady-state mainloop dominates; with fewer tiles per pair the pair's
-  // longer prologue and its exposed epilogue cost more than it saves).
-  const bool auto_pair = req_pair == 0 && req_bn == 0 && req_split <= 1 && req_kc != 4 &&
-                         !p->swap && splits == 1 && p->kt_total >= 32 &&
-                         batch * ceil_div(M, 256) * ceil_div(N, 256) >= 4 * (num_sms / 2);
+  // 256x256 pair tiles run on request only: since the single-SM 128x256 tile
+  // has two epilogue groups its epilogue no longer stalls the next tile, and
+  // it matches or beats the pair tile in every sweep (8192^3 MXFP8: 494 us
+  // against 536 us in one run; 4096x1536x6144: 50.7 against 55.6 us).
+  const bool auto_pair = false;
   if (req_pair == 2 || auto_pair) {  // 256x256 tiles on CTA pairs: wide tiles, no split
     if (p->swap || splits != 1 || (req_bn != 0 && req_bn != 256)) return BQ_ERR_INVALID;
     if (req_kc > 2 || (req_kc == 2 && K % 128 != 0)) return BQ_ERR_INVALID;

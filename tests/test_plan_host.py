@@ -44,7 +44,7 @@ def test_small_m_tiles():
     (1024, 4096, 4096, 1, dict(block_n=256, cta_pair=1, k_chunks=1)),   # fp8blk + residual
     (1024, 2048, 2048, 8, dict(block_n=128, cta_pair=1, k_chunks=2)),   # batched MLP up
     (4096, 1536, 6144, 1, dict(block_n=256, cta_pair=1, k_chunks=1)),   # down-projection
-    (8192, 8192, 8192, 1, dict(block_n=256, cta_pair=2, k_chunks=2)),   # square
+    (8192, 8192, 8192, 1, dict(block_n=256, cta_pair=1, k_chunks=1)),   # square
 ])
 def test_wide_tile_workloads(M, N, K, batch, want):
     d = desc(bq.plan(M, N, K, batch=batch, num_sms=SMS))
@@ -53,13 +53,11 @@ def test_wide_tile_workloads(M, N, K, batch, want):
         assert d[k] == v, (k, d)
 
 
-def test_pair_needs_long_k_and_many_tiles():
-    # 4 pair tiles per pair of SMs and >= 32 K blocks
-    assert bq.plan(4096, 8192, 4096, num_sms=SMS).cta_pair == 2
-    assert bq.plan(4096, 8192, 2048, num_sms=SMS).cta_pair == 1   # short K loop
-    assert bq.plan(2048, 2048, 8192, num_sms=SMS).cta_pair == 1   # 64 pair tiles
-    # a smaller device is filled sooner
-    assert bq.plan(2048, 2048, 8192, num_sms=32).cta_pair == 2
+def test_pair_tiles_only_on_request():
+    for shape in ((4096, 8192, 4096), (8192, 8192, 8192), (2048, 2048, 8192)):
+        assert bq.plan(*shape, num_sms=SMS).cta_pair == 1
+    c = bq.plan(8192, 8192, 8192, num_sms=SMS, config=bq.config(split_k=1, swap_ab=0, cta_pair=2))
+    assert (c.cta_pair, c.block_n) == (2, 256)
 
 
 def test_explicit_requests_kept():
