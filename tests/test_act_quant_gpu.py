@@ -80,6 +80,15 @@ def test_row_stride_larger_than_k():
     check(synth.activations(33, 320, seed=5), ldx=512)
 
 
+@pytest.mark.parametrize("M,K,ldx", [(1000, 4128, None), (4113, 1120, None), (2050, 2048, 2304),
+                                     (256, 16384, None)])
+def test_large_inputs_tma_path(M, K, ldx):
+    """Inputs of >= 4 Mi elements go through the TMA-staged quantizer: rows
+    past the last 32-row tile boundary, a last 256-column tile holding only a
+    few groups, a row stride wider than K, long rows."""
+    check(synth.activations(M, K, seed=M + K, group_pow2=(-12, 12)), ldx=ldx)
+
+
 def test_every_bf16_pattern():
     """All finite bf16 patterns, shuffled into groups so that each value meets
     many different group maxima (and so many scales)."""
