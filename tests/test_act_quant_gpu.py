@@ -82,10 +82,10 @@ def test_row_stride_larger_than_k():
 
 @pytest.mark.parametrize("M,K,ldx", [(1000, 4128, None), (4113, 1120, None), (2050, 2048, 2304),
                                      (256, 16384, None)])
-def test_large_inputs_tma_path(M, K, ldx):
-    """Inputs of >= 4 Mi elements go through the TMA-staged quantizer: rows
-    past the last 32-row tile boundary, a last 256-column tile holding only a
-    few groups, a row stride wider than K, long rows."""
+def test_large_inputs(M, K, ldx):
+    """Inputs of >= 4 Mi elements: rows past a 128-row band boundary, a last
+    512-column chunk holding only a few groups, a row stride wider than K,
+    long rows."""
     check(synth.activations(M, K, seed=M + K, group_pow2=(-12, 12)), ldx=ldx)
 
 
