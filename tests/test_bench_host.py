@@ -18,6 +18,30 @@ def test_decode_algorithmic_bytes():
 
 def test_act_quant_bytes_per_element():
     assert bench.act_quant_bytes(("x", "mxfp4", 1, 0, 32, 1, {})) == 32 * 3.03125
+    # packed E2M1 activations: half a byte per code; NVFP4 one scale per 16
+    assert bench.act_quant_bytes(("x", "a4w4", 1, 0, 32, 1, {})) == 32 * (2 + 0.5 + 1 / 32)
+    assert bench.act_quant_bytes(("x", "nvfp4", 1, 0, 32, 1, {})) == 32 * (2 + 0.5 + 1 / 16)
+
+
+def test_every_workload_is_accounted():
+    """Each workload names a dtype, a bound and positive flop / byte counts."""
+    for name, spec in bench.WORKLOADS.items():
+        assert spec["bound"] in ("hbm", "tensor"), name
+        for layer in spec["layers"]:
+            assert layer[1] in bench.WKIND and layer[1] in bench.DTYPE, name
+            assert bench.gemm_flops(layer) > 0 and bench.gemm_bytes(layer) > 0, name
+            assert bench.act_quant_bytes(layer) > 0, name
+            assert bench.gemm_shapes(layer), name
+
+
+def test_backward_accounting():
+    """dX and dW: two GEMMs of 2 T N K flops each; the quantizers read dY twice
+    (row-wise and transposed), x and W once."""
+    layer = bench.WORKLOADS["backward"]["layers"][0]
+    _, _, T, N, K, _, _ = layer
+    assert bench.gemm_flops(layer) == 4.0 * T * N * K
+    assert bench.gemm_shapes(layer) == [(T, K, N, 1), (N, K, T, 1)]
+    assert bench.act_quant_bytes(layer) == 3.03125 * (2 * T * N + T * K + N * K)
 
 
 def _free_port():
