@@ -819,6 +819,7 @@ __device__ __forceinline__ void cluster_reduce_local(const GemmArgs &a, const Un
 #pragma unroll
   for (int i = 0; i < kIters; ++i) {
     const int c4 = (epi_tid + 128 * i) / R;
+    if (u.tq * BN + c4 * 4 >= a.M) continue;  // columns past M were not pushed
     float4 acc = *reinterpret_cast<const float4 *>(recv + rl * kStride + c4 * 4);
 #pragma unroll
     for (int s = 1; s < S; ++s) {
@@ -1241,16 +1242,20 @@ __global__ void __launch_bounds__((!SWAP && MODE == kSplitNone) ? kWideThreads :
         const uint32_t dst =
             mapa_shared(smem_u32(recv), owner) +
             static_cast<uint32_t>((u.split * R + (row & (R - 1))) * L::kRecvStride * 4);
+        // only the tile's activation columns that exist are pushed (a 41-row
+        // operand fills 41 of 64): the owners read no others
+        const int mvalid = min(BN, a.M - u.tq * BN);
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < BN / 32 && c * 32 < mvalid; ++c) {  // warp-uniform
           uint32_t v[32];
           __syncwarp();
           tmem_ld_32x32b_x32(t_row + c * 32, v);
           tmem_ld_wait();
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            st_dsmem_u4(dst + static_cast<uint32_t>((c * 32 + 4 * q) * 4), v[4 * q], v[4 * q + 1],
-                        v[4 * q + 2], v[4 * q + 3]);
+            if (c * 32 + 4 * q < mvalid)
+              st_dsmem_u4(dst + static_cast<uint32_t>((c * 32 + 4 * q) * 4), v[4 * q],
+                          v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
         }
         tc_fence_before();
         __syncwarp();
