@@ -150,18 +150,45 @@ def gemm_bytes(layer, quant_out=False):
 GEMM_SOURCES = ("gemm_bs.cuh", "gemm_pair.cuh", "bq_ptx.cuh", "mx_quant.cuh", "bq_api.cu")
 
 
+def strip_c_comments(text):
+    """C/C++ source without its comments and blank lines (string and character
+    literals kept as written), so that editing a comment leaves the code's
+    hash unchanged."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (ln.rstrip() for ln in "".join(out).splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def kernel_source_sha():
-    """Hash of the GEMM's sources and the header: a stored DRAM-traffic
-    figure is used only while the kernel it was measured on is unchanged."""
+    """Hash of the GEMM's sources and the header, comments left out: a stored
+    DRAM-traffic figure is used only while the code it was measured on is
+    unchanged."""
     import hashlib
     h = hashlib.sha256()
     files = [os.path.join(ROOT, "block_scaled_precision_quant_b200", "csrc", f)
              for f in GEMM_SOURCES]
     files.append(os.path.join(ROOT, "include", "bq.h"))
     for f in files:
-        with open(f, "rb") as fh:
+        with open(f) as fh:
             h.update(os.path.basename(f).encode())
-            h.update(fh.read())
+            h.update(strip_c_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -8,21 +8,32 @@
 // prepack).  The decoded operands are code * 2^(scale - 127) ("formats.py"
 // page, docstring "Formats"; decode_fp4, decode_fp8_block), multiplied exactly
 // and accumulated in fp32 by tcgen05.mma kind::mxf8f6f4 with block scaling.
+// The same kernel also runs E5M2 gradient operands (kind::mxf8f6f4 format 1),
+// packed E2M1 x E2M1 (kind::mxf4, A4 == 1) and NVFP4 with E4M3 scales per 16
+// inputs (kind::mxf4nvf4, A4 == 2).  The epilogue can emit MXFP8 codes and
+// scales of y instead of bf16 (GemmArgs::q_out), and decode tiles can quantize
+// their bf16 activation rows in the producer themselves (FUSEQ).
 //
-// Structure (one persistent CTA per SM, warp-specialized, 6 warps):
-//   warp 0   TMA producer: operand tiles (128B swizzle) and the 512-byte
-//            scale-factor atoms into a STAGES-deep shared-memory ring, each
-//            stage signalled on an mbarrier with a transaction count;
+// Structure (one persistent CTA per SM, warp-specialized; 9 warps, 13 for
+// unsplit wide tiles):
+//   warps 0, 6, 7, 8   TMA copy threads: the weight tile, the activation tile,
+//            the weight scales and the activation scales of each stage
+//            (operands 128B-swizzled, scales as 512-byte atoms) into a
+//            STAGES-deep shared-memory ring; every thread arrives on the
+//            stage's mbarrier with its own transaction bytes;
 //   warp 1   TMEM allocator and MMA issuer: per stage, tcgen05.cp copies the
-//            scale atoms into TMEM, then 4 MMAs of K = 32 each consume the
-//            stage; tcgen05.commit releases the stage and, after the last
-//            k-block of a tile, signals the accumulator as full;
-//   warps 2-5 epilogue: tcgen05.ld of the fp32 accumulator (one TMEM lane
-//            quadrant per warp), alpha / bias / GELU / residual in fp32, one
-//            bf16 rounding, vector stores.  With split-K every slice writes
-//            fp32 partials to the workspace and the last slice to arrive
-//            (atomic ticket) sums all slices in slice order -- the result does
-//            not depend on which slice arrives last -- and runs the epilogue.
+//            scale atoms into TMEM, then the stage's MMAs consume it;
+//            tcgen05.commit releases the stage and, after the last k-block of
+//            a tile, signals the accumulator (ACC buffers) as full;
+//   warps 2-5 (and 9-12) epilogue: tcgen05.ld of the fp32 accumulator (one
+//            TMEM lane quadrant per warp), alpha / bias / GELU / residual in
+//            fp32, one bf16 rounding, a swizzled shared-memory staging tile
+//            written out by TMA stores (residual tiles arrive by TMA into the
+//            same slots).  Split-K runs either through an fp32 workspace (the
+//            last slice to arrive, by atomic ticket, sums all slices in slice
+//            order, so the result does not depend on arrival order) or across
+//            a thread-block cluster whose CTAs reduce their slices through
+//            distributed shared memory in a fixed order.
 //
 // "P" is the operand on the MMA's 128-row side and "Q" the one on its BN-row
 // side.  Normally P = activations and Q = weights (y[p][q]); with SWAP the

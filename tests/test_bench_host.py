@@ -50,6 +50,18 @@ def _free_port():
     p = s.getsockname()[1]
     s.close()
     return p
+def test_source_hash_ignores_comments_only():
+    """The stored-traffic key changes with the code, not with its comments."""
+    a = 'int f(int x) {  // twice\n  return 2 * x;  /* no\n overflow */\n}\n'
+    b = '// header\nint f(int x) {\n\n  return 2 * x;\n}\n'
+    assert bench.strip_c_comments(a) == bench.strip_c_comments(b)
+    assert bench.strip_c_comments('s = "a//b /* c */";') == 's = "a//b /* c */";'
+    assert bench.strip_c_comments("c = '/'; // x") == "c = '/';"
+    assert bench.strip_c_comments("return 3 * x;") != bench.strip_c_comments("return 2 * x;")
+    sha = bench.kernel_source_sha()
+    assert len(sha) == 16 and sha == bench.kernel_source_sha()
+
+
 
 
 def _worker(rank, world, port, q):
