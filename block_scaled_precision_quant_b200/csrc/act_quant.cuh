@@ -54,41 +54,19 @@ __device__ __forceinline__ void e5m2_encode16(const uint32_t (&w)[8], int e, uin
   }
 }
 
-// grid: x*8 + warp = row, y = chunk of 16 groups within the row.  Rows in
-// [M, rows_pad) only write padding scale bytes (127).  FMT: E4M3 codes; FP4:
-// E2M1 codes (packed [M, K/2], the per-32 rule with 6 in place of 448); E5M2:
-// gradient codes (the rule with 57344), SR with stochastic rounding (the
-// draw of element (row, col) is index row * K + col under `seed`).
-template <int FMT, bool SR = false>
-__global__ void __launch_bounds__(256) act_quant_kernel(
-    const __nv_bfloat16 *__restrict__ x, int64_t M, int64_t K, int64_t ldx, int64_t rows_pad,
-    uint8_t *__restrict__ q, uint8_t *__restrict__ sf_mma, uint8_t *__restrict__ sf_row,
-    int *__restrict__ status, uint64_t seed) {
-  static_assert(!SR || FMT == kQE5M2, "stochastic rounding is for E5M2 gradients");
-  const int lane = threadIdx.x & 31;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  if (row >= rows_pad) return;
-  const int64_t G = K >> 5;            // groups per row
-  const int64_t katoms = (G + 3) >> 2;
-  const int64_t g = static_cast<int64_t>(blockIdx.y) * 16 + (lane >> 1);  // this lane's group
+// One warp's share of one row in act_quant_kernel: lane 2i + h holds half h
+// (16 bf16 values, 8 words) of group g = chunk * 16 + i; `active` is false for
+// padding rows and for groups past the row's end, whose lanes carry zeros
+// through the full-warp shuffles.
+template <int FMT, bool SR>
+__device__ __forceinline__ void act_quant_row_part(const uint32_t (&w)[8], int64_t row, bool active,
+                                                   int lane, int64_t g, int64_t col, int64_t K,
+                                                   int64_t G, int64_t katoms,
+                                                   uint8_t *__restrict__ q,
+                                                   uint8_t *__restrict__ sf_mma,
+                                                   uint8_t *__restrict__ sf_row,
+                                                   int *__restrict__ status, uint64_t seed) {
   const int half = lane & 1;
-
-  // Every lane runs the shuffles below (full-warp masks); lanes without data
-  // (past the row's last group, or padding rows) carry zeros through them.
-  const bool active = row < M && g < G;
-  const int64_t col = g * 32 + half * 16;
-  uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-  // Programmatic dependent launch: x may come from the kernel before this one;
-  // the kernel after this one (the GEMM) may begin its prologue now.
-  griddep_wait();
-  griddep_launch_dependents();
-  if (active) {
-    const uint4 *src = reinterpret_cast<const uint4 *>(x + row * ldx + col);
-    const uint4 v0 = __ldg(src);
-    const uint4 v1 = __ldg(src + 1);
-    w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
-    w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
-  }
   // amax of the two half-groups met through one shuffle
   uint32_t bad = 0;
   uint32_t mx = bf16_amax_bits(w, bad);
@@ -127,6 +105,54 @@ __global__ void __launch_bounds__(256) act_quant_kernel(
       const uint32_t word = sbyte | (b1 << 8) | (b2 << 16) | (b3 << 24);
       *reinterpret_cast<uint32_t *>(sf_mma + sf_mma_offset(row, g4, katoms)) = word;
     }
+  }
+}
+
+// grid: x = band of 8 * R rows (warp w takes rows band * 8R + w + 8r, r < R),
+// y = chunk of 16 groups within the row; rows_pad is a multiple of 8 * R.
+// Each warp loads all R rows' data before quantizing any of them, so a thread
+// has R x 32 bytes in flight.  Rows in [M, rows_pad) only write padding scale
+// bytes (127).  FMT: E4M3 codes; FP4: E2M1 codes (packed [M, K/2], the per-32
+// rule with 6 in place of 448); E5M2: gradient codes (the rule with 57344), SR
+// with stochastic rounding (the draw of element (row, col) is index
+// row * K + col under `seed`).
+template <int FMT, bool SR = false, int R = 1>
+__global__ void __launch_bounds__(256) act_quant_kernel(
+    const __nv_bfloat16 *__restrict__ x, int64_t M, int64_t K, int64_t ldx, int64_t rows_pad,
+    uint8_t *__restrict__ q, uint8_t *__restrict__ sf_mma, uint8_t *__restrict__ sf_row,
+    int *__restrict__ status, uint64_t seed) {
+  static_assert(!SR || FMT == kQE5M2, "stochastic rounding is for E5M2 gradients");
+  const int lane = threadIdx.x & 31;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * (8 * R) + (threadIdx.x >> 5);
+  const int64_t G = K >> 5;            // groups per row
+  const int64_t katoms = (G + 3) >> 2;
+  const int64_t g = static_cast<int64_t>(blockIdx.y) * 16 + (lane >> 1);  // this lane's group
+  const int64_t col = g * 32 + (lane & 1) * 16;
+
+  uint32_t w[R][8];
+  // Programmatic dependent launch: x may come from the kernel before this one;
+  // the kernel after this one (the GEMM) may begin its prologue now.
+  griddep_wait();
+  griddep_launch_dependents();
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int64_t row = row0 + 8 * r;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[r][i] = 0u;
+    if (row < M && g < G) {
+      const uint4 *src = reinterpret_cast<const uint4 *>(x + row * ldx + col);
+      const uint4 v0 = __ldg(src);
+      const uint4 v1 = __ldg(src + 1);
+      w[r][0] = v0.x; w[r][1] = v0.y; w[r][2] = v0.z; w[r][3] = v0.w;
+      w[r][4] = v1.x; w[r][5] = v1.y; w[r][6] = v1.z; w[r][7] = v1.w;
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int64_t row = row0 + 8 * r;  // warp-uniform
+    if (row >= rows_pad) break;
+    act_quant_row_part<FMT, SR>(w[r], row, row < M && g < G, lane, g, col, K, G, katoms, q,
+                                sf_mma, sf_row, status, seed);
   }
 }
 

@@ -801,6 +801,10 @@ namespace {
 
 // Launch of the per-32 quantizer along rows: fmt bq::kQE4M3 / kQFP4 /
 // kQE5M2, sr stochastic rounding (E5M2 only) under `seed`.
+// Rows per warp of act_quant_kernel on large operands (rows_pad is a multiple
+// of 128, so of 8 * kAqRows).
+constexpr int kAqRows = 2;
+
 int act_quant_launch(int fmt, bool sr, uint64_t seed, const void* x_bf16, int64_t M, int64_t K,
                      int64_t ldx, void* q_out, void* sf_mma, void* sf_rowmajor, int* d_status,
                      bq_stream_t stream) {
@@ -815,8 +819,16 @@ int act_quant_launch(int fmt, bool sr, uint64_t seed, const void* x_bf16, int64_
   const int64_t rows_pad = (M + 127) / 128 * 128;
   const int64_t chunks = (K / 32 + 15) / 16;
   if (rows_pad / 8 > 0x7FFFFFFF || chunks > 65535) return BQ_ERR_SHAPE;
+  // Grids of >= 6144 one-row blocks (about five waves of resident blocks):
+  // each warp takes kAqRows rows, their loads all in flight before any is
+  // quantized, and half as many blocks come and go (8192 x 8192: 47.9 ->
+  // 45.1 us).  Smaller grids keep one row per warp: there the longer per-warp
+  // path costs more than it saves (1024 x 4096: 4.6 -> 6.1 us).  Stochastic
+  // rounding is bound by its Philox arithmetic and keeps one row.
+  const int rows_per_warp = (!sr && (rows_pad / 8) * chunks >= 6144) ? kAqRows : 1;
   cudaLaunchConfig_t lc = {};
-  lc.gridDim = dim3(static_cast<unsigned>(rows_pad / 8), static_cast<unsigned>(chunks));
+  lc.gridDim = dim3(static_cast<unsigned>(rows_pad / (8 * rows_per_warp)),
+                    static_cast<unsigned>(chunks));
   lc.blockDim = dim3(256);
   lc.stream = reinterpret_cast<cudaStream_t>(stream);
   cudaLaunchAttribute attr[1];
@@ -824,10 +836,16 @@ int act_quant_launch(int fmt, bool sr, uint64_t seed, const void* x_bf16, int64_
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = 1;
-  auto kern = fmt == bq::kQFP4    ? bq::act_quant_kernel<bq::kQFP4>
-              : fmt == bq::kQE5M2 ? (sr ? bq::act_quant_kernel<bq::kQE5M2, true>
-                                        : bq::act_quant_kernel<bq::kQE5M2>)
-                                  : bq::act_quant_kernel<bq::kQE4M3>;
+  const bool multi = rows_per_warp > 1;
+  auto kern = fmt == bq::kQFP4
+                  ? (multi ? bq::act_quant_kernel<bq::kQFP4, false, kAqRows>
+                           : bq::act_quant_kernel<bq::kQFP4>)
+              : fmt == bq::kQE5M2
+                  ? (sr ? bq::act_quant_kernel<bq::kQE5M2, true>
+                        : multi ? bq::act_quant_kernel<bq::kQE5M2, false, kAqRows>
+                                : bq::act_quant_kernel<bq::kQE5M2>)
+                  : (multi ? bq::act_quant_kernel<bq::kQE4M3, false, kAqRows>
+                           : bq::act_quant_kernel<bq::kQE4M3>);
   if (cudaLaunchKernelEx(&lc, kern, static_cast<const __nv_bfloat16*>(x_bf16), M, K, ldx,
                          rows_pad, static_cast<uint8_t*>(q_out), static_cast<uint8_t*>(sf_mma),
                          static_cast<uint8_t*>(sf_rowmajor), d_status, seed) != cudaSuccess) {

@@ -35,7 +35,10 @@ def assert_close(y, ref, tol, what=""):
 
 # ------------------------------------------------------------ act_quant ----
 
-@pytest.mark.parametrize("M,K", [(1, 32), (7, 96), (64, 1024), (130, 544), (300, 4096)])
+# (6100, 4128): a grid of >= 6144 one-row blocks, so two rows per warp, with
+# ragged rows and a last chunk of one group
+@pytest.mark.parametrize("M,K", [(1, 32), (7, 96), (64, 1024), (130, 544), (300, 4096),
+                                 (6100, 4128)])
 def test_act_quant_mxfp4_bit_exact(M, K):
     x = synth.activations(M, K, seed=M + K, group_pow2=(-10, 10))
     q, sf = bq.act_quant_mxfp4(dev_bf16(x))

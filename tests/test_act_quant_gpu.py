@@ -81,11 +81,12 @@ def test_row_stride_larger_than_k():
 
 
 @pytest.mark.parametrize("M,K,ldx", [(1000, 4128, None), (4113, 1120, None), (2050, 2048, 2304),
-                                     (256, 16384, None)])
+                                     (256, 16384, None), (6100, 4128, 4160)])
 def test_large_inputs(M, K, ldx):
     """Inputs of >= 4 Mi elements: rows past a 128-row band boundary, a last
     512-column chunk holding only a few groups, a row stride wider than K,
-    long rows."""
+    long rows; the last case launches >= 6144 one-row blocks' worth of work,
+    so its warps take two rows each."""
     check(synth.activations(M, K, seed=M + K, group_pow2=(-12, 12)), ldx=ldx)
 
 

@@ -39,7 +39,9 @@ def grads(M, K, seed, spread=(-20, 4)):
 
 # ------------------------------------------------------- gradient quant ----
 
-@pytest.mark.parametrize("M,K", [(1, 32), (7, 96), (130, 544), (512, 4096)])
+# (5000, 5056): a grid of >= 6144 one-row blocks (two rows per warp when rounding
+# to nearest), ragged rows and chunks
+@pytest.mark.parametrize("M,K", [(1, 32), (7, 96), (130, 544), (512, 4096), (5000, 5056)])
 @pytest.mark.parametrize("stochastic", [False, True])
 def test_grad_quant_bit_exact(M, K, stochastic):
     g = grads(M, K, seed=M + K)
