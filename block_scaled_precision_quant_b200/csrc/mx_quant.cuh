@@ -52,18 +52,25 @@ __device__ __forceinline__ uint32_t e4m3_ceil(float t) {
   return b < 1u ? 1u : b;
 }
 
+// Per-halfword unsigned maximum of two words of 16-bit pairs.
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 // Largest magnitude bits (15 bits, sign dropped) of the bf16 pairs in w: an
-// integer max is order-preserving for non-negative floats.  `bad` collects
-// non-finite inputs (all-ones exponent).
+// integer max is order-preserving for non-negative floats, taken on both
+// halves of each word at once.  `bad` collects non-finite inputs: a value has
+// an all-ones exponent exactly when its magnitude bits are >= 0x7F80, so the
+// largest magnitude tells whether any of them has.
 template <int NW>
 __device__ __forceinline__ uint32_t bf16_amax_bits(const uint32_t (&w)[NW], uint32_t &bad) {
-  uint32_t mx = 0;
+  uint32_t m = w[0] & 0x7FFF7FFFu;
 #pragma unroll
-  for (int i = 0; i < NW; ++i) {
-    const uint32_t lo = w[i] & 0x7FFFu, hi = (w[i] >> 16) & 0x7FFFu;
-    mx = max(mx, max(lo, hi));
-    bad |= ((lo & 0x7F80u) == 0x7F80u) | ((hi & 0x7F80u) == 0x7F80u);
-  }
+  for (int i = 1; i < NW; ++i) m = max_u16x2(m, w[i] & 0x7FFF7FFFu);
+  const uint32_t mx = max(m & 0xFFFFu, m >> 16);
+  bad |= mx >= 0x7F80u ? 1u : 0u;
   return mx;
 }
 
@@ -76,7 +83,10 @@ __device__ __forceinline__ int mx_exponent(uint32_t amax_bits) {
 }
 
 // E4M3 codes of the 2 * NW bf16 values in w (element 2i in the low half of
-// word i) scaled by 2^-e, four codes per output word.
+// word i) scaled by 2^-e, four codes per output word.  The clamp to +-448 is
+// the conversion's saturation: a finite value above 448 (below 464 it rounds
+// to 448 anyway) becomes 448 with its sign, which is what clamping first and
+// rounding gives.
 template <int NW>
 __device__ __forceinline__ void mx_encode(const uint32_t (&w)[NW], int e,
                                           uint32_t (&codes)[NW / 2]) {
@@ -87,9 +97,8 @@ __device__ __forceinline__ void mx_encode(const uint32_t (&w)[NW], int e,
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       const uint32_t word = w[2 * i + j];
-      f[2 * j] = fminf(fmaxf(__fmul_rn(__uint_as_float(word << 16), inv), -448.0f), 448.0f);
-      f[2 * j + 1] =
-          fminf(fmaxf(__fmul_rn(__uint_as_float(word & 0xFFFF0000u), inv), -448.0f), 448.0f);
+      f[2 * j] = __fmul_rn(__uint_as_float(word << 16), inv);
+      f[2 * j + 1] = __fmul_rn(__uint_as_float(word & 0xFFFF0000u), inv);
     }
     codes[i] = e4m3x4(f[0], f[1], f[2], f[3]);
   }
