@@ -412,7 +412,9 @@ def gemm(weight_kind, a_q, a_sf, b, b_sf, M, N, K, y=None, bias=None, residual=N
          quantize_out=False, write_y=True, q_out=None, sf_out=None):
     """y = bf16(act(alpha * A B^T + bias) + residual) for weight_kind W_MXFP4,
     W_FP8BLK32, W_MXFP8 (E4M3 activations a_q [.., M, K]), W_A4W4 (packed
-    E2M1 activations a_q [.., M, K/2] from act_quant_mxfp4) or W_GRAD (E5M2
+    E2M1 activations a_q [.., M, K/2] from act_quant_mxfp4), W_NVFP4 (packed
+    E2M1 activations and weights with E4M3 scales per 16, from act_quant_nvfp4;
+    alpha = 1 / (g_a g_b) undoes the per-tensor scales) or W_GRAD (E5M2
     gradient codes a_q [.., M, K], MXFP8 b).  batch: None or a dict with 'count' and byte
     strides ('stride_a', 'stride_a_sf', 'stride_b', 'stride_b_sf', 'stride_y',
     'stride_res'; 0 broadcasts).  config: GemmConfig or None (auto).
