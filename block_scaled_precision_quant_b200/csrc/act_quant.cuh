@@ -2,7 +2,7 @@
 // layout kernels (prepack / unpack) for sm_100a.
 //
 // Quantizer ("formats.py" page: act_scale, act_quant, _log2_ceil_pow2 and the
-// module docstring "act_qdq reproduces ..."), per 32 consecutive elements of
+// module docstring's description of act_qdq), per 32 consecutive elements of
 // a row; the arithmetic is in mx_quant.cuh.
 //
 // Work split: one warp per 512 consecutive elements of one row (16 groups);

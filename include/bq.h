@@ -4,8 +4,8 @@
  *
  * What the calls compute is defined on the "formats.py" page
  * (dsv41-sampled-drafting, code/offload/dspark/native/formats.py): the
- * activation quantizer (act_scale / act_quant, module docstring "act_qdq
- * reproduces ...") and the exact decoders of the weight formats (module
+ * activation quantizer (act_scale / act_quant and the module docstring's
+ * description of act_qdq) and the exact decoders of the weight formats (module
  * docstring "Formats", decode_fp4, decode_fp8_block).  The fused bias /
  * residual / GELU epilogue follows the FlashRT "fp4-gemm" page ("Available
  * Functions": nvfp4_gemm_bias_bf16, ..._bias_residual_bf16, ..._bias_gelu_bf16)
@@ -85,7 +85,7 @@ size_t bq_sf_bytes_nvfp4(int64_t rows, int64_t K);
 /* ---- activation quantization ------------------------------------------ */
 
 /* bq_act_quant -- per-32 MX quantization of bf16 activations
- * ("formats.py" page: act_scale, act_quant; docstring "act_qdq reproduces").
+ * ("formats.py" page: act_scale, act_quant; the module docstring on act_qdq).
  *
  * For every 32 consecutive elements of a row: amax = max(max|x|, 1e-4) in
  * fp32; t = fp32(amax * fp32(1/448)); e = ceil(log2 t) from t's exponent bits;

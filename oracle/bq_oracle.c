@@ -11,8 +11,9 @@
  *   - every operand is decoded exactly and products are summed in fp64;
  *   - the activation quantizer follows the step order of the
  *     "formats.py" page (dsv41-sampled-drafting, code/offload/dspark/native):
- *     module docstring "act_qdq reproduces kernel.act_quant ..." and the
- *     functions act_scale / act_quant / act_qdq / _log2_ceil_pow2;
+ *     module docstring's description of act_qdq (the kernel quantizer it
+ *     mirrors) and the functions act_scale / act_quant / act_qdq /
+ *     _log2_ceil_pow2;
  *   - the number formats follow the same page's module docstring
  *     ("Formats" paragraph) and its constants FP4_TABLE, FP8_MAX, BLOCK,
  *     E8M0_NAN, E4M3_NAN;
@@ -290,7 +291,7 @@ uint16_t oracle_f32_to_bf16(float f) {
 
 /* ------------------------------------------------------------------ */
 /* Activation quantization (formats.py page: act_scale, act_quant,      */
-/* act_qdq, _log2_ceil_pow2; docstring "act_qdq reproduces ...").       */
+/* act_qdq, _log2_ceil_pow2; the module docstring on act_qdq).          */
 /* ------------------------------------------------------------------ */
 
 /* The per-group steps, for one group of 32 binary32 values:
