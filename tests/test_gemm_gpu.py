@@ -400,6 +400,36 @@ def test_square_mxfp8_full_size():
     run_sampled(Case(bq.W_MXFP8, 8192, 8192, 8192, seed=3), n=600)
 
 
+def test_batched_mlp_up_full_size():
+    """The MLP workload's up-projection at full size: 8 problems of 1024 x 2048 x 2048 over
+    one broadcast MXFP4 weight (stride 0), bias + GELU, in the dispatch's own schedule;
+    sampled outputs of every problem against the oracle."""
+    count, M, N, K = 8, 1024, 2048, 2048
+    xs = [synth.activations(M, K, seed=60 + i) for i in range(count)]
+    b, bsf = synth.mxfp4_weight(N, K, seed=70)
+    bias = synth.bias(N, seed=71)
+    aqs, sfs = zip(*[bq.act_quant(to_dev_bf16(x)) for x in xs])
+    aq = torch.stack(aqs)
+    asf = torch.stack(sfs)
+    bsf_d = bq.pack_weight_scales(to_dev_u8(bsf), bq.BQ_SF_ROW32, N, K)
+    y = bq.gemm(bq.W_MXFP4, aq, asf, to_dev_u8(b), bsf_d, M, N, K, bias=to_dev_bf16(bias),
+                act=bq.BQ_ACT_GELU,
+                batch=dict(count=count, stride_a=M * K, stride_a_sf=asf.shape[1], stride_b=0,
+                           stride_b_sf=0, stride_y=M * N * 2))
+    bq.device_status()
+    yv = bf16_to_f64(y.cpu().view(torch.int16).numpy().view(np.uint16))
+    babs = np.abs(bf16_to_f64(bias))
+    rng = np.random.default_rng(6)
+    for i in range(count):
+        ms = np.concatenate([rng.integers(0, M, 400), [0, M - 1, 0, M - 1]])
+        ns = np.concatenate([rng.integers(0, N, 400), [0, 0, N - 1, N - 1]])
+        q, sc = oracle.act_quant(xs[i])
+        ref, sabs = oracle.gemm_sampled(q, sc, b, bsf, oracle.B_FP4, M, N, K, ms, ns,
+                                        bias=bias, act=oracle.ACT_GELU)
+        tol = oracle.gemm_tolerance(ref, sabs, 1.0, babs[ns], None, oracle.ACT_GELU)
+        assert_close(yv[i][ms, ns], ref, tol, f"batched MLP up, problem {i}")
+
+
 def test_down_projection_full_size():
     """Down-projection 4096 x 1536 x 6144, MXFP4 weights."""
     run_sampled(Case(bq.W_MXFP4, 4096, 1536, 6144, seed=4), n=3000)
