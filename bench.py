@@ -1,25 +1,36 @@
 """Benchmark of the block-scaled linear-layer hot path on B200.
 
 One step = the whole hot path over one batch: for each linear layer of the
-workload, bq_act_quant (bf16 -> E4M3 + E8M0 in the MMA scale layout) and the
-block-scaled GEMM with its fused epilogue.  The default workload is the
-decode-shaped linear (M = 41 rows, MXFP8 activations x MXFP4 weights + bias,
-(N, K) in {(4608, 1536), (6144, 1536), (1536, 6144)}).
+workload, the activation quantizer (bf16 -> E4M3 + E8M0 in the MMA scale
+layout) and the block-scaled GEMM with its fused epilogue.
+
+The default run reports the square MXFP8 x MXFP8 GEMM at M = N = K = 8192
+(both bf16 operands quantized by act_quant inside every step) as the headline
+line, and carries every other workload of the suite as a sub-record of that
+line ("suite"): the 64x512x1024 MXFP8 x MXFP4 reference case, the three
+decode-shaped (M = 41) layers with bias, the FP8 32x32-block weights at
+1024x4096x4096 with a residual, the batched MLP up-projection 8 x
+(1024x2048x2048) with bias + GELU and its 4096x1536x6144 down-projection.
+Every record has its own roofline, act_quant bandwidth, end-to-end number and
+CPU-oracle baseline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode|pr1|fp8blk|square|mlp]
+                    [--workload suite|square|decode|pr1|fp8blk|mlp|mlp_up|...]
 
-Prints one JSON line (rank 0).  Timing: W untimed warm-up steps, then K steps
-between a barrier + device synchronize on both sides, timed with CUDA events on
-the launching stream, max over ranks.  Each step's launches are replayed from
-a CUDA graph (one graph per rotating input set); inputs rotate over enough
-copies that every step reads its weights from HBM, not L2.  `--impl reference`
-times the CPU oracle on a bounded sample of the same workload instead.
+Timing: W untimed warm-up steps, then windows of exactly K steps, each window
+one CUDA-graph replay between two CUDA events on the launching stream; the
+windows run back to back between a barrier + device synchronize on both
+sides, at least 100 of them, and the median window gives ms_per_step (max
+over ranks).  Consecutive windows continue one rotation over enough copies of
+the inputs (more than 3x the L2 size) that every step reads its weights and
+activations from HBM.  `--impl reference` times the CPU oracle on a bounded
+sample of the same workload instead.
 """
 from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -59,6 +70,14 @@ WORKLOADS = {
              "down-projection 4096x1536x6144",
         layers=[("up8", "mxfp4", 1024, 2048, 2048, 8, dict(bias=True, gelu=True)),
                 ("down", "mxfp4", 4096, 1536, 6144, 1, dict())], bound="tensor"),
+    "mlp_up": dict(
+        desc="batched MLP up-projection: 8x(1024x2048x2048) MXFP8xMXFP4, broadcast weight, "
+             "bias+GELU",
+        layers=[("up8", "mxfp4", 1024, 2048, 2048, 8, dict(bias=True, gelu=True))],
+        bound="tensor"),
+    "mlp_down": dict(
+        desc="MLP down-projection: MXFP8xMXFP4 GEMM M=4096 N=1536 K=6144",
+        layers=[("down", "mxfp4", 4096, 1536, 6144, 1, dict())], bound="tensor"),
     # FP4 x FP4 (A4W4): MXFP4 activations (bq_act_quant_mxfp4) and MXFP4 weights
     # on tcgen05.mma kind::mxf4, on the decode shapes and on a large square
     "a4w4_decode": dict(
@@ -88,6 +107,10 @@ WORKLOADS = {
              "dX = dY W and dW = dY^T x on E5M2 x MXFP8 GEMMs",
         layers=[("bwd", "grad", 4096, 1536, 6144, 1, dict())], bound="tensor"),
 }
+
+# The default run: the headline workload, then the suite's sub-records.
+HEADLINE = "square"
+SUITE = ("pr1", "decode", "fp8blk", "mlp_up", "mlp_down")
 
 WKIND = {"mxfp4": 0, "fp8blk32": 1, "mxfp8": 2, "a4w4": 3, "grad": 4, "nvfp4": 5}
 DTYPE = {"mxfp4": "mxfp8xmxfp4", "fp8blk32": "mxfp8xfp8blk32", "mxfp8": "mxfp8xmxfp8",
@@ -208,6 +231,12 @@ def stored_traffic(workload):
 
 # ------------------------------------------------------------------- peaks --
 
+# Nominal dense figures of one B200, for the fractions stated against them
+# next to the measured-peak fractions: HBM3e ~8 TB/s, FP8 4.5 PFLOP/s, FP4
+# 9 PFLOP/s (NVIDIA's doubled figures assume 2:4 sparsity).
+NOMINAL = dict(hbm=8000.0, fp8=4500.0, fp4=9000.0)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -218,6 +247,19 @@ def load_peaks():
                     src="measured")
     except Exception:
         return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), or the platform's."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine()
 
 
 # ---------------------------------------------------------------- distributed --
@@ -312,11 +354,19 @@ class ClockSampler:
 
 # -------------------------------------------------------------- GPU workload --
 
+def _bf16_dev(bits, device):
+    import torch
+    return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(device)
+
+
 class Layer:
     """Device buffers of one linear layer, with `sets` rotating copies of the
-    inputs (activations, weights, scales, bias, residual)."""
+    inputs (activations, weights, scales, bias, residual).  The first
+    `distinct` sets are drawn from their own seeds; the others are device
+    copies of them (distinct memory, so the rotation still streams every
+    step's operands from HBM)."""
 
-    def __init__(self, spec, sets, seed, device, quant_out=False, fused_act=False):
+    def __init__(self, spec, sets, seed, device, quant_out=False, fused_act=False, distinct=2):
         import torch
         import block_scaled_precision_quant_b200 as bq
         from block_scaled_precision_quant_b200 import synth
@@ -326,15 +376,19 @@ class Layer:
         self.gelu = bool(ex.get("gelu"))
         self.sets = []
         for s in range(sets):
+            if s >= distinct:
+                src = self.sets[s % distinct]
+                self.sets.append({k: (v.clone() if v is not None else None)
+                                  for k, v in src.items()})
+                continue
             sd = seed + 1000 * s
             xs = []
             for b in range(B):
-                xb = synth.activations(M, K, seed=sd + b, group_pow2=ex.get("act_gp"))
-                xs.append(torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16))
+                xs.append(_bf16_dev(synth.activations(M, K, seed=sd + b,
+                                                      group_pow2=ex.get("act_gp")), "cpu"))
             x = torch.stack(xs).reshape(B * M, K).to(device)
             if wk == "nvfp4":  # weights quantized once here, on the device
-                wxb = synth.activations(N, K, seed=sd + 500, std=0.05)
-                wx = torch.from_numpy(wxb.view(np.int16)).view(torch.bfloat16).to(device)
+                wx = _bf16_dev(synth.activations(N, K, seed=sd + 500, std=0.05), device)
                 w, wsf = bq.act_quant_nvfp4(wx)
                 wx = None
             elif wk in ("mxfp4", "a4w4"):
@@ -349,14 +403,12 @@ class Layer:
                                             N, K)
                 wx = None
             else:  # MXFP8 weight operand, quantized by act_quant inside the step
-                wxb = synth.activations(N, K, seed=sd + 500)
-                wx = torch.from_numpy(wxb.view(np.int16)).view(torch.bfloat16).to(device)
+                wx = _bf16_dev(synth.activations(N, K, seed=sd + 500), device)
                 w = torch.empty((N, K), dtype=torch.uint8, device=device)
                 wsf = torch.empty((bq.sf_bytes(N, K),), dtype=torch.uint8, device=device)
-            bias = (torch.from_numpy(synth.bias(N, seed=sd + 600).view(np.int16))
-                    .view(torch.bfloat16).to(device) if ex.get("bias") else None)
-            res = (torch.from_numpy(synth.residual(B * M, N, seed=sd + 700).view(np.int16))
-                   .view(torch.bfloat16).to(device) if ex.get("residual") else None)
+            bias = _bf16_dev(synth.bias(N, seed=sd + 600), device) if ex.get("bias") else None
+            res = (_bf16_dev(synth.residual(B * M, N, seed=sd + 700), device)
+                   if ex.get("residual") else None)
             self.sets.append(dict(x=x, w=w, wsf=wsf, wx=wx, bias=bias, res=res))
         # outputs shared by all sets (written every step)
         self.a4 = wk in FP4_ACT  # packed E2M1 activations, two codes per byte
@@ -378,13 +430,25 @@ class Layer:
         self.set_bytes = sum(t.numel() * t.element_size() for t in self.sets[0].values()
                              if t is not None)
 
-    def launches(self, s, which="all", x=None):
+    def step_inputs(self, s):
+        """The bf16 tensors a step copies in from the host (end-to-end path):
+        the activations, and for the square workload the bf16 weight operand
+        that every step quantizes."""
+        d = self.sets[s]
+        return dict(x=d["x"]) if d["wx"] is None else dict(x=d["x"], wx=d["wx"])
+
+    def output(self):
+        return self.qy if self.quant_out else self.y
+
+    def launches(self, s, which="all", x=None, wx=None):
         """Issue this layer's kernels for input set s on the current stream
-        (x: optional activations replacing the set's own)."""
+        (x, wx: optional bf16 operands replacing the set's own)."""
         import block_scaled_precision_quant_b200 as bq
         d = dict(self.sets[s])
         if x is not None:
             d["x"] = x
+        if wx is not None:
+            d["wx"] = wx
         M, N, K, B = self.M, self.N, self.K, self.B
         n = 0
         if self.fused_act and which == "all":
@@ -432,7 +496,7 @@ class BackwardLayer:
     interface as Layer: launches(s, which) issues the quantizers ("act_quant")
     and the two GEMMs ("gemm"); y is dX (the step's result passed on)."""
 
-    def __init__(self, spec, sets, seed, device, **_):
+    def __init__(self, spec, sets, seed, device, distinct=2, **_):
         import torch
         import block_scaled_precision_quant_b200 as bq
         from block_scaled_precision_quant_b200 import synth
@@ -442,16 +506,16 @@ class BackwardLayer:
         self.wk = WKIND[wk]
         self.quant_out = False
         self.qy = None
-
-        def bf16(bits):
-            return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(device)
         self.sets = []
         for s in range(sets):
+            if s >= distinct:
+                self.sets.append({k: v.clone() for k, v in self.sets[s % distinct].items()})
+                continue
             sd = seed + 1000 * s
             self.sets.append(dict(
-                x=bf16(synth.activations(T, N, seed=sd + 2, group_pow2=(-20, 4))),  # dY
-                xin=bf16(synth.activations(T, K, seed=sd)),
-                w=bf16(synth.activations(N, K, seed=sd + 1, std=0.05))))
+                x=_bf16_dev(synth.activations(T, N, seed=sd + 2, group_pow2=(-20, 4)), device),
+                xin=_bf16_dev(synth.activations(T, K, seed=sd), device),
+                w=_bf16_dev(synth.activations(N, K, seed=sd + 1, std=0.05), device)))
         u8 = dict(dtype=torch.uint8, device=device)
         self.gq, self.gsf = torch.empty((T, N), **u8), torch.empty((bq.sf_bytes(T, N),), **u8)
         self.wtq, self.wtsf = torch.empty((K, N), **u8), torch.empty((bq.sf_bytes(K, N),), **u8)
@@ -463,9 +527,14 @@ class BackwardLayer:
                         bq.workspace_bytes(self.wk, N, K, T, 1))
         self.ws = torch.zeros((self.need,), **u8) if self.need else None
         self.set_bytes = sum(t.numel() * t.element_size() for t in self.sets[0].values())
-        self.step = 0
 
-    def launches(self, s, which="all", x=None):
+    def step_inputs(self, s):
+        return dict(x=self.sets[s]["x"])  # the output gradient dY
+
+    def output(self):
+        return self.y
+
+    def launches(self, s, which="all", x=None, wx=None):
         import block_scaled_precision_quant_b200 as bq
         d = dict(self.sets[s])
         if x is not None:
@@ -495,182 +564,381 @@ def make_layer(spec, sets, seed, device, **kw):
     return Layer(spec, sets, seed, device, **kw)
 
 
-def build_graphs(layers, nsets, which):
-    """One CUDA graph per input set (one step each) and one rotation graph
-    holding the steps of all sets back to back."""
+# ------------------------------------------------------------------ timing --
+
+def _sf_bytes(rows, K, per=32):
+    """Bytes of an MMA-layout scale buffer (512-byte atoms of 128 rows x 4
+    scale columns)."""
+    return -(-rows // 128) * -(-K // (4 * per)) * 512
+
+
+def input_set_bytes(layer):
+    """Device bytes of one rotating copy of a layer's step inputs: bf16
+    activations, weight codes and scales (the square workload's bf16 weight
+    operand, its codes and scales), bias and residual."""
+    _, wk, M, N, K, B, ex = layer
+    if wk == "grad":  # dY [T, N], x [T, K], W [N, K], all bf16
+        return 2 * (M * N + M * K + N * K)
+    x = 2 * B * M * K
+    if wk in ("mxfp4", "a4w4"):
+        w = N * K // 2 + _sf_bytes(N, K)
+    elif wk == "nvfp4":
+        w = N * K // 2 + _sf_bytes(N, K, per=16)
+    elif wk == "fp8blk32":
+        w = N * K + _sf_bytes(N, K)
+    else:  # mxfp8: bf16 operand + its codes + scales
+        w = 2 * N * K + N * K + _sf_bytes(N, K)
+    return x + w + (2 * N if ex.get("bias") else 0) + (2 * B * M * N if ex.get("residual") else 0)
+
+
+def rotation_sets(set_bytes, l2_bytes, cap=64):
+    """Rotating input copies so that consecutive steps read more than 3x the
+    L2 size before an input comes round again (at least 2, at most cap)."""
+    return max(2, min(cap, int(math.ceil(3.0 * l2_bytes / max(set_bytes, 1)))))
+
+
+def window_starts(steps, nsets, cap=64):
+    """Input sets at which consecutive windows of `steps` steps begin when the
+    windows continue one rotation over nsets sets: window j starts at set
+    (j * steps) mod nsets, and the pattern repeats after nsets / gcd(steps,
+    nsets) windows (capped)."""
+    n = nsets // math.gcd(steps, nsets)
+    return [(j * steps) % nsets for j in range(min(n, cap))]
+
+
+def capture_windows(layers, nsets, which, steps):
+    """One CUDA graph per window start, each holding exactly `steps` steps
+    (input sets start, start+1, ... mod nsets) of the layers' launches.
+    Returns (graphs, launches per step)."""
     import torch
-    graphs = []
     stream = torch.cuda.current_stream()
-    for s in range(nsets):
-        # warm once outside capture (sets function attributes, caches)
-        for L in layers:
-            L.launches_per_step = L.launches(s, which)
-        torch.cuda.synchronize()
+    per_step = 0
+    for L in layers:  # warm once outside capture (function attributes, caches)
+        per_step += L.launches(0, which)
+    torch.cuda.synchronize()
+    graphs = []
+    for start in window_starts(steps, nsets):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            for L in layers:
-                L.launches(s, which)
+            for i in range(steps):
+                for L in layers:
+                    L.launches((start + i) % nsets, which)
         graphs.append(g)
-    rot = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(rot, stream=stream):
-        for s in range(nsets):
-            for L in layers:
-                L.launches(s, which)
     torch.cuda.synchronize()
-    return graphs, rot
+    return graphs, per_step
 
 
-def replay_steps(graphs, rot, start, count):
-    """Replay `count` steps beginning at input set `start` (mod the number of
-    sets); whole rotations go through the rotation graph."""
-    n = len(graphs)
-    i, left = start, count
-    while left > 0 and i % n != 0:
-        graphs[i % n].replay()
-        i, left = i + 1, left - 1
-    while left >= n:
-        rot.replay()
-        i, left = i + n, left - n
-    while left > 0:
-        graphs[i % n].replay()
-        i, left = i + 1, left - 1
-    return i
-
-
-def time_graphs(graph_pair, steps, warmup, world, device, min_warm_s=1.0, nvtx=None):
-    """Warm-up (at least `warmup` steps and `min_warm_s` seconds), then time
-    exactly `steps` steps between barrier + synchronize, CUDA events on the
-    launching stream, max over ranks.  Returns (ms, warm-up steps run)."""
+def time_windows(graphs, steps, warmup, world, device, min_windows=100, budget_s=1.0,
+                 max_windows=20000):
+    """Warm-up (at least `warmup` steps), then windows of exactly `steps`
+    steps replayed back to back, each between two CUDA events on the
+    launching stream, with a barrier + synchronize before the first and after
+    the last.  The window count is sized to about budget_s of GPU time, at
+    least min_windows.  Returns (median ms per window, max over ranks;
+    windows; per-window ms of this rank)."""
     import torch
-    graphs, rot = graph_pair
-    i = replay_steps(graphs, rot, 0, warmup)
-    t0 = time.perf_counter()
-    while time.perf_counter() - t0 < min_warm_s and i < 2_000_000:
-        i = replay_steps(graphs, rot, i, len(graphs))
-        torch.cuda.synchronize()
-    torch.cuda.synchronize()
-    barrier(world, device)
-    torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
+    n = len(graphs)
+    done = 0
+    j = 0
+    while done < warmup or j < n:
+        graphs[j % n].replay()
+        j += 1
+        done += steps
+    torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    if nvtx:
-        torch.cuda.nvtx.range_push(nvtx)
     e0.record(stream)
-    replay_steps(graphs, rot, i, steps)
+    for i in range(n):
+        graphs[(j + i) % n].replay()
     e1.record(stream)
-    if nvtx:
-        torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+    j += n
+    per = max(e0.elapsed_time(e1) / n, 1e-4)
+    windows = int(min(max_windows, max(min_windows, budget_s * 1e3 / per)))
+    windows = reduce_max(float(windows), world, device)  # same count on every rank
+    windows = int(windows)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(windows + 1)]
     torch.cuda.synchronize()
     barrier(world, device)
-    ms = e0.elapsed_time(e1)
-    return reduce_max(ms, world, device), i
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for i in range(windows):
+        graphs[(j + i) % n].replay()
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world, device)
+    ts = [ev[i].elapsed_time(ev[i + 1]) for i in range(windows)]
+    return reduce_max(statistics.median(ts), world, device), windows, ts
 
 
-def run_e2e(spec_layers, layers, steps, device):
-    """The same step through the public API with host buffers: pinned host
-    activations copied in, act_quant + GEMM launched eagerly, outputs read
-    back, every step."""
+def run_e2e(layers, nsets, device, budget_s=0.3, max_steps=2000):
+    """The same step through the public API with host buffers, every step:
+    the step's bf16 inputs copied in from pinned host memory, act_quant + GEMM
+    launched eagerly on the input set's weights (rotating like the timed
+    windows), the result copied back to pinned host memory.  Runs about
+    budget_s of steps (at least 5).  Returns (ms per step, steps, H2D bytes
+    per step, D2H bytes per step)."""
     import torch
-    import block_scaled_precision_quant_b200 as bq
-    host_x = [L.sets[0]["x"].cpu().pin_memory() for L in layers]
-    outs = [L.qy if L.quant_out else L.y for L in layers]  # the step's result
+    host = [{k: v.cpu().pin_memory() for k, v in L.step_inputs(0).items()} for L in layers]
+    dev = [{k: torch.empty_like(v, device=device) for k, v in h.items()} for h in host]
+    outs = [L.output() for L in layers]
     host_y = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
-    h2d = sum(h.numel() * h.element_size() for h in host_x)
+    h2d = sum(v.numel() * v.element_size() for h in host for v in h.values())
     d2h = sum(h.numel() * h.element_size() for h in host_y)
-    dev_x = [torch.empty_like(L.sets[0]["x"]) for L in layers]
 
-    def step():
-        for L, hx, dx, hy, o in zip(layers, host_x, dev_x, host_y, outs):
-            dx.copy_(hx, non_blocking=True)
-            L.launches(0, x=dx)
+    def step(s):
+        for L, h, d, hy, o in zip(layers, host, dev, host_y, outs):
+            for k in h:
+                d[k].copy_(h[k], non_blocking=True)
+            L.launches(s % nsets, **d)
             hy.copy_(o, non_blocking=True)
-    for _ in range(3):
-        step()
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
-        step()
-    e1.record()
-    torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / steps, h2d, d2h
+
+    def timed(first, count):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for s in range(first, first + count):
+            step(s)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / count
+    one = timed(0, 3)  # warm-up, and the size of the timed run
+    steps = int(min(max_steps, max(5, budget_s * 1e3 / max(one, 1e-3))))
+    return timed(3, steps), steps, h2d, d2h
 
 
 # ------------------------------------------------------------- CPU oracle --
 
-def oracle_step_sample(layers_spec, rows, seed=0, nthreads=None):
-    """One bounded sample of the workload on the CPU oracle: for each layer,
-    act_quant of `rows` activation rows and the GEMM of those rows against the
-    full weight.  Returns (flops done, seconds, threads)."""
-    import oracle
-    from block_scaled_precision_quant_b200 import synth
-    nthreads = nthreads or oracle.default_threads()
-    flops = 0.0
-    t_total = 0.0
-    for (name, wk, M, N, K, B, ex) in layers_spec:
-        r = min(rows, M)
-        if wk == "grad":
-            # backward: `r` rows of dX (over all N) and `r` rows of dW (over all T tokens)
-            dy = synth.activations(M, N, seed=seed + 2, group_pow2=(-20, 4))
-            w = synth.activations(N, K, seed=seed + 1, std=0.05)
-            xin = synth.activations(M, K, seed=seed)
+class OracleSample:
+    """A workload's step on the CPU oracle, on a bounded sample: for each
+    layer, the activation quantizer on `rows` activation rows and the GEMM of
+    those rows against the full weight (flops 2 rows N K).  The square
+    workload quantizes its bf16 weight operand every step; the sample charges
+    that share too, the quantizer on rows * N / M of its rows.  Weights are
+    prepared once (outside the timed sample), as the GPU path prepacks them.
+    The backward workload times the gradient quantizers on `rows` rows and
+    columns of dY and the dX and dW GEMMs on `rows` output rows."""
+
+    def __init__(self, layers_spec, seed=0):
+        import oracle
+        from block_scaled_precision_quant_b200 import synth
+        self.o, self.synth = oracle, synth
+        self.layers = []
+        for (name, wk, M, N, K, B, ex) in layers_spec:
+            d = dict(spec=(name, wk, M, N, K, B, ex))
+            if wk == "grad":
+                d["dy"] = synth.activations(M, N, seed=seed + 2, group_pow2=(-20, 4))
+                d["xin"] = synth.activations(M, K, seed=seed)
+                d["wq"] = oracle.quant_transposed(synth.activations(N, K, seed=seed + 1, std=0.05),
+                                                  oracle.Q_E4M3)
+            elif wk == "nvfp4":
+                d["w"] = oracle.act_quant_nvfp4(synth.activations(N, K, seed=seed + 500, std=0.05))
+                d["kind"] = oracle.B_NVFP4
+            elif wk in ("mxfp4", "a4w4"):
+                d["w"] = synth.mxfp4_weight(N, K, seed=seed + 500)
+                d["kind"] = oracle.B_FP4
+            elif wk == "fp8blk32":
+                d["w"] = synth.fp8_weight_blk32(N, K, seed=seed + 500)
+                d["kind"] = oracle.B_FP8BLK
+            else:  # mxfp8: the bf16 weight operand, quantized once for the GEMM
+                d["wx"] = synth.activations(N, K, seed=seed + 500)
+                d["w"] = oracle.act_quant(d["wx"])
+                d["kind"] = oracle.B_FP8ROW
+            if wk != "grad":
+                d["bias"] = synth.bias(N, seed=seed + 600) if ex.get("bias") else None
+            self.layers.append(d)
+
+    def run(self, rows, seed=0, nthreads=None):
+        """Returns (flops done, seconds, threads)."""
+        o, synth = self.o, self.synth
+        nthreads = nthreads or o.default_threads()
+        flops, t_total = 0.0, 0.0
+        for d in self.layers:
+            name, wk, M, N, K, B, ex = d["spec"]
+            r = min(rows, M)
+            if wk == "grad":
+                dy, xin = d["dy"], d["xin"]
+                wq, ws = d["wq"]
+                cols = max(32, r)
+                t0 = time.perf_counter()
+                gq, gs = o.grad_quant(dy[:r], stochastic=True, seed=seed)
+                o.gemm(gq, gs, wq, ws, o.B_FP8ROW, r, K, N, a_kind=o.A_E5M2, nthreads=nthreads)
+                gtq, gts = o.quant_transposed(dy[:, :cols], o.Q_E5M2, stochastic=True, seed=seed)
+                xq, xs = o.quant_transposed(xin, o.Q_E4M3)
+                o.gemm(gtq[:r], gts[:r], xq, xs, o.B_FP8ROW, r, K, M, a_kind=o.A_E5M2,
+                       nthreads=nthreads)
+                t_total += time.perf_counter() - t0
+                flops += 2.0 * r * K * N + 2.0 * r * K * M
+                continue
+            x = synth.activations(r, K, seed=seed, group_pow2=ex.get("act_gp"))
+            res = synth.residual(r, N, seed=seed + 700) if ex.get("residual") else None
+            wb, ws = d["w"]
+            wrows = max(1, (r * N) // M) if wk == "mxfp8" else 0
             t0 = time.perf_counter()
-            gq, gs = oracle.grad_quant(dy[:r], stochastic=True, seed=seed)
-            wq, ws = oracle.quant_transposed(w, oracle.Q_E4M3)
-            oracle.gemm(gq, gs, wq, ws, oracle.B_FP8ROW, r, K, N, a_kind=oracle.A_E5M2,
-                        nthreads=nthreads)
-            gtq, gts = oracle.quant_transposed(dy[:, :max(8, r)], oracle.Q_E5M2, stochastic=True,
-                                               seed=seed)
-            xq, xs = oracle.quant_transposed(xin, oracle.Q_E4M3)
-            oracle.gemm(gtq[:r], gts[:r], xq, xs, oracle.B_FP8ROW, r, K, M,
-                        a_kind=oracle.A_E5M2, nthreads=nthreads)
+            if wk == "nvfp4":
+                q, s = o.act_quant_nvfp4(x)
+            elif wk == "a4w4":
+                q, s = o.act_quant_fp4(x)
+            else:
+                q, s = o.act_quant(x)
+            if wrows:
+                o.act_quant(d["wx"][:wrows])
+            a_kind = {"a4w4": o.A_FP4, "nvfp4": o.A_NVFP4}.get(wk, o.A_E4M3)
+            o.gemm(q, s, wb, ws, d["kind"], r, N, K, bias=d["bias"], residual=res,
+                   act=o.ACT_GELU if ex.get("gelu") else o.ACT_NONE,
+                   nthreads=nthreads, a_kind=a_kind)
             t_total += time.perf_counter() - t0
-            flops += 2.0 * r * K * N + 2.0 * r * K * M
-            continue
-        x = synth.activations(r, K, seed=seed, group_pow2=ex.get("act_gp"))
-        if wk == "nvfp4":
-            wb, ws = oracle.act_quant_nvfp4(synth.activations(N, K, seed=seed + 500, std=0.05))
-            kind = oracle.B_NVFP4
-        elif wk in ("mxfp4", "a4w4"):
-            wb, ws = synth.mxfp4_weight(N, K, seed=seed + 500)
-            kind = oracle.B_FP4
-        elif wk == "fp8blk32":
-            wb, ws = synth.fp8_weight_blk32(N, K, seed=seed + 500)
-            kind = oracle.B_FP8BLK
-        else:
-            wb, ws = oracle.act_quant(synth.activations(N, K, seed=seed + 500))
-            kind = oracle.B_FP8ROW
-        bias = synth.bias(N, seed=seed + 600) if ex.get("bias") else None
-        res = synth.residual(r, N, seed=seed + 700) if ex.get("residual") else None
-        t0 = time.perf_counter()
-        if wk == "nvfp4":
-            q, s = oracle.act_quant_nvfp4(x)
-        elif wk == "a4w4":
-            q, s = oracle.act_quant_fp4(x)
-        else:
-            q, s = oracle.act_quant(x)
-        a_kind = {"a4w4": oracle.A_FP4, "nvfp4": oracle.A_NVFP4}.get(wk, oracle.A_E4M3)
-        oracle.gemm(q, s, wb, ws, kind, r, N, K, bias=bias, residual=res,
-                    act=oracle.ACT_GELU if ex.get("gelu") else oracle.ACT_NONE,
-                    nthreads=nthreads, a_kind=a_kind)
-        t_total += time.perf_counter() - t0
-        flops += 2.0 * r * N * K
-    return flops, t_total, nthreads
+            flops += 2.0 * r * N * K
+        return flops, t_total, nthreads
 
 
-def cpu_baseline(spec, budget_s=15.0):
-    """The oracle as it stands on this host's cores, on a bounded sample."""
-    rows = 4
-    flops, secs, th = oracle_step_sample(spec["layers"], rows)
-    # grow the sample toward the time budget (bounded)
-    while secs < budget_s / 4 and rows < 64:
+def cpu_baseline(spec, budget_s=15.0, sample=None):
+    """The oracle as it stands on this host's cores, on a bounded sample of
+    the workload grown toward budget_s of CPU time."""
+    import oracle
+    sample = sample or OracleSample(spec["layers"])
+    rows = oracle.default_threads()  # the oracle's GEMM spreads rows over its threads
+    flops, secs, th = sample.run(rows)
+    while secs < budget_s / 3 and rows < 1024:
         rows *= 2
-        flops, secs, th = oracle_step_sample(spec["layers"], rows)
+        flops, secs, th = sample.run(rows)
+    rows = min(rows, max(sp[2] for sp in spec["layers"]))  # at most the layers' own rows
     return dict(value=flops / secs / 1e12, unit="TFLOP/s", cores=th, kind="oracle",
+                cpu_model=cpu_model(),
                 sample=f"{rows} activation rows per layer (act_quant + exact-decode fp64 GEMM "
-                       f"against the full weight), {flops / 1e9:.2f} GFLOP in {secs:.1f} s")
+                       f"against the full weight), {flops / 1e9:.2f} GFLOP in {secs:.1f} s "
+                       f"on {th} threads")
+
+
+# ----------------------------------------------------------------- records --
+
+def roofline(spec, layers_spec, gemm_ms_step, ck, peaks, kernels, workload, quant_out=False):
+    """The dominant kernel's roofline object: algorithmic bytes (HBM-bound
+    workloads) or flops (tensor-bound) per GEMM launch over the measured
+    average launch time, against the measured peak and the nominal one."""
+    flops_step = sum(gemm_flops(sp) for sp in layers_spec)
+    bytes_step = sum(gemm_bytes(sp, quant_out) for sp in layers_spec)
+    launches = sum(len(gemm_shapes(sp)) for sp in layers_spec)
+    avg_us = gemm_ms_step * 1e3 / launches
+    common = dict(kernel=kernels, avg_launch_us=round(avg_us, 3),
+                  traffic=stored_traffic(workload), launches_per_step=launches)
+    if spec["bound"] == "hbm":
+        achieved = bytes_step / (gemm_ms_step * 1e-3) / 1e9
+        return dict(bound="hbm", achieved=round(achieved, 1), peak=peaks["hbm"], unit="GB/s",
+                    frac=round(achieved / peaks["hbm"], 4),
+                    frac_nominal=round(achieved / NOMINAL["hbm"], 4),
+                    peak_nominal=NOMINAL["hbm"],
+                    algorithmic_bytes_per_launch=bytes_step / launches,
+                    peak_source=f"{peaks['src']} hbm_gbs (burst)", **common)
+    # A kernel whose median SM clock over the timed region sat under the power
+    # cap is held to the sustained tensor figure, otherwise to the burst one.
+    capped = bool(ck) and "sw_power_cap" in (ck.get("reasons") or []) and bool(
+        ck.get("sm_mhz") and ck.get("sm_max_mhz") and ck["sm_mhz"] < 0.97 * ck["sm_max_mhz"])
+    kind = "bf16_sus" if capped else "bf16"
+    fp4 = all(sp[1] in FP4_ACT for sp in layers_spec)  # FP4 x FP4: the FP4 tensor rate
+    ratio = 4.0 if fp4 else 2.0  # nominal dense fp8 (fp4) / bf16 ratio: 4.5 (9) / 2.25
+    peak = ratio * peaks[kind]
+    nominal = NOMINAL["fp4" if fp4 else "fp8"]
+    achieved = flops_step / (gemm_ms_step * 1e-3) / 1e12
+    out = dict(bound="tensor", achieved=round(achieved, 1), peak=round(peak, 1), unit="TFLOP/s",
+               frac=round(achieved / peak, 4), frac_nominal=round(achieved / nominal, 4),
+               peak_nominal=nominal, flops_per_launch=flops_step / launches,
+               peak_source=(f"{peaks['src']} "
+                            f"{'bf16_tflops_sustained' if capped else 'bf16_tflops'} x {ratio:g} "
+                            f"(nominal {'fp4' if fp4 else 'fp8'}/bf16 ratio)"), **common)
+    if ck and ck.get("sm_mhz"):  # clock-normalised: time x median SM clock
+        out["us_x_ghz_per_launch"] = round(avg_us * ck["sm_mhz"] / 1e3, 3)
+    return out
+
+
+def measure(name, args, world, rank, local, device, cpu_budget_s, time_budget_s=1.0):
+    """Every number of one workload's record (see the module docstring)."""
+    import torch
+    import block_scaled_precision_quant_b200 as bq
+    spec = WORKLOADS[name]
+    layers_spec = spec["layers"]
+    props = torch.cuda.get_device_properties(device)
+    l2 = props.L2_cache_size
+    sms = props.multi_processor_count
+    set_bytes = sum(input_set_bytes(sp) for sp in layers_spec)
+    nsets = rotation_sets(set_bytes, l2)
+    layers = [make_layer(sp, nsets, 11 * (i + 1), device, quant_out=args.quant_out,
+                         fused_act=args.fused_act)
+              for i, sp in enumerate(layers_spec)]
+    K = args.steps
+    graphs, per_step = capture_windows(layers, nsets, "all", K)
+    clocks = ClockSampler(local)
+    clocks.start()
+    ms_win, windows, _ = time_windows(graphs, K, args.warmup, world, device,
+                                      budget_s=time_budget_s)
+    del graphs
+    # the dominant kernel: the GEMM alone, same windows and rotation
+    ggraphs, _ = capture_windows(layers, nsets, "gemm", K)
+    gms_win, _, _ = time_windows(ggraphs, K, args.warmup, world, device,
+                                 budget_s=time_budget_s / 2)
+    del ggraphs
+    ck = clocks.stop()
+    qgraphs, _ = capture_windows(layers, nsets, "act_quant", K)
+    qms_win, _, _ = time_windows(qgraphs, K, args.warmup, world, device,
+                                 budget_s=time_budget_s / 4)
+    del qgraphs
+    per_layer_us = None
+    if len(layers) > 1:  # each layer's GEMM alone, same rotation
+        per_layer_us = []
+        for L in layers:
+            lg, _ = capture_windows([L], nsets, "gemm", K)
+            lms, _, _ = time_windows(lg, K, args.warmup, world, device,
+                                     budget_s=time_budget_s / 4)
+            per_layer_us.append(round(lms / K * 1e3, 3))
+            del lg
+    ms_step, gemm_ms_step, aq_ms_step = ms_win / K, gms_win / K, qms_win / K
+    e2e_ms, e2e_steps, h2d, d2h = run_e2e(layers, nsets, device)
+    bq.device_status()  # raises if a kernel gave up on one of its waits
+
+    flops_step = sum(gemm_flops(sp) for sp in layers_spec)
+    qbytes_step = sum(act_quant_bytes(sp) for sp in layers_spec)
+    qbytes_step += sum(act_quant_bytes((0, 0, sp[3], 0, sp[4], 1, 0))
+                       for sp in layers_spec if sp[1] == "mxfp8")  # the quantized weight operand
+    peaks = load_peaks()
+    shapes = [(WKIND[sp[1]],) + g for sp in layers_spec for g in gemm_shapes(sp)]
+    kernels = "+".join(sorted({("gemm_pair_kernel" if bq.plan(
+        M, N, Kd, B, num_sms=sms, weight_kind=wk).cta_pair == 2 else "gemm_bs_kernel")
+        for (wk, M, N, Kd, B) in shapes}))
+    qgbs = qbytes_step / (aq_ms_step * 1e-3) / 1e9
+    rec = {
+        "workload": spec["desc"],
+        "value": round(world * flops_step / (ms_step * 1e-3) / 1e12, 3),
+        "unit": "TFLOP/s",
+        "ms_per_step": round(ms_step, 6),
+        "steps": K,
+        "windows": windows,
+        "dtype": DTYPE[layers_spec[0][1]],
+        "roofline": roofline(spec, layers_spec, gemm_ms_step, ck, peaks, kernels, name,
+                             args.quant_out),
+        "act_quant": {"achieved_gbs": round(qgbs, 1), "frac_hbm": round(qgbs / peaks["hbm"], 4),
+                      "frac_hbm_nominal": round(qgbs / NOMINAL["hbm"], 4),
+                      "us_per_step": round(aq_ms_step * 1e3, 3),
+                      "algorithmic_bytes_per_step": qbytes_step},
+        "gemm_us_per_step": round(gemm_ms_step * 1e3, 3),
+        "gemm_us_per_layer": per_layer_us,
+        "e2e": {"value": round(world * flops_step / (e2e_ms * 1e-3) / 1e12, 3),
+                "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 4), "steps": e2e_steps},
+        "clocks": ck,
+        "l2": (f"{nsets} rotating input sets of {set_bytes / 1e6:.1f} MB "
+               f"({nsets * set_bytes / 1e6:.0f} MB > 3 x L2 {l2 / 1e6:.0f} MB or 64 sets; "
+               f"2 drawn from seeds, the rest device copies)"),
+        "gpu_launches": per_step * K * windows,
+        "launches_per_step": per_step,
+    }
+    del layers
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    if world == 1 and rank == 0 and cpu_budget_s > 0:
+        rec["cpu_baseline"] = cpu_baseline(spec, cpu_budget_s)
+    return rec
 
 
 # ------------------------------------------------------------------- main --
@@ -678,11 +946,12 @@ def cpu_baseline(spec, budget_s=15.0):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=None,
-                    help="timed steps (default: about 2 s of timed work)")
-    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20, help="steps per timed window")
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
+    ap.add_argument("--workload", choices=["suite"] + sorted(WORKLOADS), default="suite",
+                    help="suite (default): the square 8192^3 headline with every other "
+                         "workload of the suite as a sub-record")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-run", type=int, default=0, metavar="R",
                     help="no timing: build one input set and run every layer's step R "
@@ -697,16 +966,16 @@ def main(argv=None):
                     help="with --profile-run: run only the workload's first layer, at this "
                          "smaller shape (a small case of the same kernel for full captures)")
     args = ap.parse_args(argv)
-    if args.warmup < 3:
-        args.warmup = 3
-    spec = WORKLOADS[args.workload]
+    args.warmup = max(3, args.warmup)
+    args.steps = max(1, args.steps)
     world, rank, local = dist_env()
+    suite = args.workload == "suite"
+    name = HEADLINE if suite else args.workload
 
     if args.impl == "reference":
-        return run_reference(args, spec, world, rank)
+        return run_reference(args, name, world, rank)
 
     import torch
-    import block_scaled_precision_quant_b200 as bq
     from block_scaled_precision_quant_b200 import build as bq_build
     bq_build.build()
     torch.cuda.set_device(local)
@@ -715,176 +984,97 @@ def main(argv=None):
     # All work on one non-default stream: graphs are captured and replayed on
     # it, and the CUDA events are recorded on it.
     with torch.cuda.stream(torch.cuda.Stream(device)):
-        return run_ours(args, spec, world, rank, local, device)
+        rc = run_ours(args, name, suite, world, rank, local, device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return rc
 
 
-def run_ours(args, spec, world, rank, local, device):
+def run_profile(args, name, rank, device):
     import torch
     import block_scaled_precision_quant_b200 as bq
-
-    if args.profile_run:
-        specs = spec["layers"]
-        if args.profile_shape:
-            M, N, K = (int(v) for v in args.profile_shape.split(","))
-            name, wk, _, _, _, B, ex = specs[0]
-            specs = [(name, wk, M, N, K, B, ex)]
-        layers = [make_layer(sp, 1, 11 * (i + 1), device) for i, sp in enumerate(specs)]
-        for _ in range(args.profile_run):
-            for L in layers:
-                L.launches(0)
-        torch.cuda.synchronize()
-        bq.device_status()
-        if rank == 0:
-            print(json.dumps({"profile_run": args.profile_run, "workload": spec["desc"],
-                              "shape": args.profile_shape}))
-        return 0
-
-    layers_spec = spec["layers"]
-    l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    probe = [make_layer(sp, 1, 11 * (i + 1), device) for i, sp in enumerate(layers_spec)]
-    set_bytes = sum(L.set_bytes for L in probe)
-    nsets = max(1, min(64, int(np.ceil(3.0 * l2 / max(set_bytes, 1)))))
-    del probe
-    torch.cuda.empty_cache()
-    layers = [make_layer(sp, nsets, 11 * (i + 1), device, quant_out=args.quant_out,
-                         fused_act=args.fused_act)
-              for i, sp in enumerate(layers_spec)]
-    graphs = build_graphs(layers, nsets, "all")
-    launches_per_step = sum(L.launches_per_step for L in layers)
-
-    if args.steps is None:  # calibrate: about 2 s of timed work
-        rot = graphs[1]
-        rot.replay()
-        torch.cuda.synchronize()
-        c0 = time.perf_counter()
-        rot.replay()
-        torch.cuda.synchronize()
-        per = (time.perf_counter() - c0) / nsets
-        args.steps = int(min(200000, max(50, 2.0 / max(per, 1e-7))))
-    clocks = ClockSampler(local)
-    clocks.start()
-    ms, warm_steps = time_graphs(graphs, args.steps, args.warmup, world, device,
-                                 nvtx="bq_timed")
-    ck = clocks.stop()
-    ms_step = ms / args.steps
-
-    # dominant kernel: the GEMM.  Time GEMM-only graphs over the same rotation,
-    # and act_quant-only graphs likewise.
-    ggraphs = build_graphs(layers, nsets, "gemm")
-    gms, _ = time_graphs(ggraphs, args.steps, args.warmup, world, device, min_warm_s=0.2)
-    gemm_ms_step = gms / args.steps
-    qgraphs = build_graphs(layers, nsets, "act_quant")
-    qms, _ = time_graphs(qgraphs, args.steps, args.warmup, world, device, min_warm_s=0.2)
-    aq_ms_step = qms / args.steps
-    per_layer_us = None
-    if len(layers) > 1:  # each layer's GEMM alone, same rotation
-        per_layer_us = []
+    specs = WORKLOADS[name]["layers"]
+    if args.profile_shape:
+        M, N, K = (int(v) for v in args.profile_shape.split(","))
+        lname, wk, _, _, _, B, ex = specs[0]
+        specs = [(lname, wk, M, N, K, B, ex)]
+    layers = [make_layer(sp, 1, 11 * (i + 1), device) for i, sp in enumerate(specs)]
+    for _ in range(args.profile_run):
         for L in layers:
-            lg = build_graphs([L], nsets, "gemm")
-            lms, _ = time_graphs(lg, args.steps, args.warmup, world, device, min_warm_s=0.1)
-            per_layer_us.append(round(lms / args.steps * 1e3, 3))
-            del lg
+            L.launches(0)
+    torch.cuda.synchronize()
     bq.device_status()
+    if rank == 0:
+        print(json.dumps({"profile_run": args.profile_run, "workload": WORKLOADS[name]["desc"],
+                          "shape": args.profile_shape}))
+    return 0
 
-    flops_step = sum(gemm_flops(sp) for sp in layers_spec)
-    gbytes_step = sum(gemm_bytes(sp, args.quant_out) for sp in layers_spec)
-    qbytes_step = sum(act_quant_bytes(sp) for sp in layers_spec)
-    if any(sp[1] == "mxfp8" for sp in layers_spec):
-        qbytes_step += sum(act_quant_bytes((0, 0, sp[3], 0, sp[4], 1, 0))
-                           for sp in layers_spec if sp[1] == "mxfp8")
-    value = world * flops_step / (ms_step * 1e-3) / 1e12
-    peaks = load_peaks()
-    # A kernel whose median SM clock over the timed region sat under the power
-    # cap is held to the sustained tensor figure, otherwise to the burst one.
-    capped = bool(ck) and "sw_power_cap" in (ck.get("reasons") or []) and bool(
-        ck.get("sm_mhz") and ck.get("sm_max_mhz") and ck["sm_mhz"] < 0.97 * ck["sm_max_mhz"])
-    tensor_kind = "bf16_sus" if capped else "bf16"
-    # nominal dense fp8 / bf16 ratio 4.5 / 2.25; FP4 x FP4 (kind::mxf4) 9 / 2.25
-    a4 = all(sp[1] in FP4_ACT for sp in layers_spec)  # FP4 x FP4: the FP4 tensor rate
-    tensor_ratio = 4.0 if a4 else 2.0
-    fp8_peak = tensor_ratio * peaks[tensor_kind]
-    shapes = [(WKIND[sp[1]],) + g for sp in layers_spec for g in gemm_shapes(sp)]
-    gemm_launches = len(shapes)
-    # the GEMM kernel(s) the built-in dispatch runs for these layers
-    sms = torch.cuda.get_device_properties(device).multi_processor_count
-    kernels = sorted({("gemm_pair_kernel" if bq.plan(M, N, K, B, num_sms=sms,
-                                                     weight_kind=wk).cta_pair == 2
-                       else "gemm_bs_kernel") for (wk, M, N, K, B) in shapes})
-    kernel_name = "+".join(kernels)
-    if spec["bound"] == "hbm":
-        achieved = gbytes_step / (gemm_ms_step * 1e-3) / 1e9
-        roof = dict(bound="hbm", achieved=round(achieved, 1), peak=peaks["hbm"], unit="GB/s",
-                    frac=round(achieved / peaks["hbm"], 4), traffic=stored_traffic(args.workload),
-                    kernel=kernel_name, algorithmic_bytes_per_launch=gbytes_step / gemm_launches,
-                    avg_launch_us=round(gemm_ms_step * 1e3 / gemm_launches, 3),
-                    peak_source=f"{peaks['src']} hbm_gbs (burst)")
-    else:
-        achieved = flops_step / (gemm_ms_step * 1e-3) / 1e12
-        roof = dict(bound="tensor", achieved=round(achieved, 1), peak=round(fp8_peak, 1),
-                    unit="TFLOP/s", frac=round(achieved / fp8_peak, 4),
-                    traffic=stored_traffic(args.workload),
-                    kernel=kernel_name, flops_per_launch=flops_step / gemm_launches,
-                    avg_launch_us=round(gemm_ms_step * 1e3 / gemm_launches, 3),
-                    peak_source=(f"{peaks['src']} {'bf16_tflops_sustained' if tensor_kind != 'bf16' else 'bf16_tflops'}"
-                                 f" x {tensor_ratio:g} (nominal "
-                                 f"{'fp4' if a4 else 'fp8'}/bf16 ratio)"))
-    e2e_ms, h2d, d2h = run_e2e(layers_spec, layers, min(2000, max(10, args.steps // 4)), device)
+
+def run_ours(args, name, suite, world, rank, local, device):
+    if args.profile_run:
+        return run_profile(args, name, rank, device)
+    cpu = not args.no_cpu_baseline
+    head = measure(name, args, world, rank, local, device, cpu_budget_s=15.0 if cpu else 0,
+                   time_budget_s=1.5)
+    subs = {}
+    if suite:
+        for sub in SUITE:
+            subs[sub] = measure(sub, args, world, rank, local, device,
+                                cpu_budget_s=4.0 if cpu else 0, time_budget_s=0.6)
     out = {
         "metric": METRIC,
-        "value": round(value, 3),
+        "value": head["value"],
         "unit": "TFLOP/s",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(ms_step, 6),
+        "ms_per_step": head["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": DTYPE[layers_spec[0][1]],
+        "dtype": head["dtype"],
         "data": "synthetic",
-        "config": {"workload": spec["desc"], "parallelism": "replicas" if world > 1 else "single",
-                   "l2": f"{nsets} rotating input sets of {set_bytes / 1e6:.1f} MB "
-                         f"({nsets * set_bytes / 1e6:.0f} MB > L2 {l2 / 1e6:.0f} MB)",
-                   "graphs": "one CUDA graph per input set, replayed per step",
+        "config": {"workload": head["workload"],
+                   "parallelism": "replicas" if world > 1 else "single",
+                   "timing": (f"median of {head['windows']} windows of exactly {args.steps} "
+                              f"steps, each window one CUDA-graph replay between CUDA events"),
+                   "l2": head["l2"],
                    "output": "mxfp8 (codes + scales, no bf16 y)" if args.quant_out else "bf16",
                    "act_quant": "fused into the GEMM (one call per decode layer)"
                                 if args.fused_act else "separate launch"},
-        "roofline": roof,
-        "act_quant": {"achieved_gbs": round(qbytes_step / (aq_ms_step * 1e-3) / 1e9, 1),
-                      "frac_hbm": round(qbytes_step / (aq_ms_step * 1e-3) / 1e9 / peaks["hbm"], 4),
-                      "us_per_step": round(aq_ms_step * 1e3, 3),
-                      "algorithmic_bytes_per_step": qbytes_step},
-        "gemm_us_per_step": round(gemm_ms_step * 1e3, 3),
-        "gemm_us_per_layer": per_layer_us,
-        "e2e": {"value": round(world * flops_step / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": round(e2e_ms, 4)},
-        "gpu_launches": launches_per_step * args.steps,
-        "warmup_steps_run": warm_steps,
-        "clocks": ck,
+        "roofline": head["roofline"],
+        "act_quant": head["act_quant"],
+        "gemm_us_per_step": head["gemm_us_per_step"],
+        "gemm_us_per_layer": head["gemm_us_per_layer"],
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
+        "clocks": head["clocks"],
     }
-    if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(spec)
+    if "cpu_baseline" in head:
+        out["cpu_baseline"] = head["cpu_baseline"]
+    if subs:
+        out["suite"] = subs
     if rank == 0:
         print(json.dumps(out), flush=True)
-    del graphs, ggraphs, qgraphs
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
     return 0
 
 
-def run_reference(args, spec, world, rank):
+def run_reference(args, name, world, rank):
     """Reference arm: the CPU oracle on the host cores, on a bounded sample of
-    the same workload per step.  Under torchrun only rank 0 works."""
+    the same workload per step (one activation row per oracle thread and
+    layer).  Under torchrun only rank 0 works."""
     if rank != 0:
         return 0
-    rows = 2
+    import oracle
+    spec = WORKLOADS[name]
+    rows = oracle.default_threads()
+    sample = OracleSample(spec["layers"])
     times = []
     flops = 0.0
     th = 1
     for i in range(args.warmup + args.steps):
-        f, s, th = oracle_step_sample(spec["layers"], rows, seed=i)
+        f, s, th = sample.run(rows, seed=i)
         if i >= args.warmup:
             times.append(s)
             flops += f
@@ -897,9 +1087,10 @@ def run_reference(args, spec, world, rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": spec["desc"], "parallelism": "cpu oracle"},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": th,
-                         "kind": "oracle",
+                         "kind": "oracle", "cpu_model": cpu_model(),
                          "sample": f"{rows} activation rows per layer per step (act_quant + "
-                                   "exact-decode fp64 GEMM against the full weight)"},
+                                   "exact-decode fp64 GEMM against the full weight; the square "
+                                   "workload also quantizes rows*N/M of its weight operand)"},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

@@ -9,7 +9,7 @@ one JSON line of {"<fmt> <M>x<K>": [us per launch, algorithmic GB/s]}, the
 algorithmic bytes being 2 (bf16 read) + 1 or 1/2 (code) + 1/32 (scale) per
 element.
 
-    python -m block_scaled_precision_quant_b200.quant_timing [--fmt e4m3,fp4] [MxK ...]
+    python quant_timing.py [--fmt e4m3,fp4] [MxK ...]
 """
 from __future__ import annotations
 

@@ -4,7 +4,7 @@ For one problem shape, times every candidate schedule (bq_gemm_config) with
 CUDA-graph replay over rotating weight copies (more bytes than L2 holds, so
 weights stream from HBM) and prints one JSON line per candidate:
 
-    python -m block_scaled_precision_quant_b200.sweep M N K [kind] [--batch B] [--gelu]
+    python sweep.py M N K [kind] [--batch B] [--gelu]
         [--residual]
 
 kind: mxfp4 (default), fp8blk32, mxfp8, a4w4 (MXFP4 activations and weights).  --batch B runs B independent problems

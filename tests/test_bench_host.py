@@ -95,3 +95,45 @@ def test_reference_arm_other_ranks_do_nothing(capsys, monkeypatch):
     monkeypatch.setenv("WORLD_SIZE", "2")
     assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"]) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_windows_continue_one_rotation():
+    """Back-to-back windows of exactly `steps` steps walk the input sets in
+    rotation order whether steps is below, equal to or above the set count,
+    so a timed result does not depend on --steps through L2 reuse."""
+    for steps, nsets in ((20, 28), (1, 7), (28, 28), (45, 28), (3, 2), (20, 2)):
+        starts = bench.window_starts(steps, nsets)
+        seq = [(s + i) % nsets for s in starts for i in range(steps)]
+        assert seq == [i % nsets for i in range(len(seq))], (steps, nsets)
+        # the next window after the last one starts where the first one did
+        assert (starts[-1] + steps) % nsets == starts[0]
+    assert bench.window_starts(20, 28) == [0, 20, 12, 4, 24, 16, 8]
+
+
+def test_rotation_exceeds_three_l2():
+    l2 = 126 * 2 ** 20
+    for name, spec in bench.WORKLOADS.items():
+        b = sum(bench.input_set_bytes(sp) for sp in spec["layers"])
+        n = bench.rotation_sets(b, l2)
+        assert 2 <= n <= 64
+        assert n * b > 3 * l2 or n == 64, name
+
+
+def test_input_set_bytes_by_hand():
+    # decode layer 1: bf16 x 41x1536, FP4 weights 4608x768 bytes, scales
+    # 36 x 12 atoms of 512 bytes, bias 4608 bf16
+    qkv = bench.WORKLOADS["decode"]["layers"][0]
+    assert bench.input_set_bytes(qkv) == 41 * 1536 * 2 + 4608 * 768 + 36 * 12 * 512 + 4608 * 2
+    # square: bf16 x and bf16 weight operand, its E4M3 codes and scales
+    sq = bench.WORKLOADS["square"]["layers"][0]
+    n = 8192 * 8192
+    assert bench.input_set_bytes(sq) == 2 * n + 2 * n + n + 64 * 64 * 512
+
+
+def test_suite_names_every_workload_once():
+    assert bench.HEADLINE not in bench.SUITE
+    assert len(set(bench.SUITE)) == len(bench.SUITE)
+    assert all(s in bench.WORKLOADS for s in (bench.HEADLINE,) + bench.SUITE)
+    # the batched up-projection and the down-projection are separate records
+    assert bench.WORKLOADS["mlp_up"]["layers"] + bench.WORKLOADS["mlp_down"]["layers"] == \
+        bench.WORKLOADS["mlp"]["layers"]

@@ -1,7 +1,7 @@
 """Host-side accounting of the standalone act_quant timing module (no device)."""
 import pytest
 
-from block_scaled_precision_quant_b200 import quant_timing as qt
+import quant_timing as qt
 
 
 def test_algorithmic_bytes():
