@@ -53,7 +53,8 @@ EXPORTS = (
     "bq_gemm_bf16act_epilogue", "bq_gemm_plan", "bq_act_quant_mxfp4", "bq_gemm_mxfp4_mxfp4",
     "bq_gemm_mxfp4_mxfp4_epilogue", "bq_grad_quant", "bq_quant_transposed", "bq_gemm_e5m2_mxfp8",
     "bq_gemm_e5m2_mxfp8_epilogue", "bq_grad_quant_dual", "bq_sf_bytes_nvfp4", "bq_act_quant_nvfp4",
-    "bq_gemm_nvfp4_nvfp4", "bq_gemm_nvfp4_nvfp4_epilogue",
+    "bq_gemm_nvfp4_nvfp4", "bq_gemm_nvfp4_nvfp4_epilogue", "bq_selftest_wait_timeout",
+    "bq_debug_override_compute_capability",
 )
 
 
@@ -156,6 +157,10 @@ def lib():
         L.bq_device_status_detail.restype = i32
         L.bq_device_report.argtypes = [ctypes.c_char_p, sz]
         L.bq_device_report.restype = i32
+        L.bq_selftest_wait_timeout.argtypes = [i64, vp]
+        L.bq_selftest_wait_timeout.restype = i32
+        L.bq_debug_override_compute_capability.argtypes = [i32, i32]
+        L.bq_debug_override_compute_capability.restype = i32
         _lib = L
         return L
 
@@ -208,7 +213,8 @@ def device_report() -> str:
 def device_status():
     """Synchronizes the current stream; raises BqError(BQ_ERR_TIMEOUT) if a
     kernel gave up on a barrier wait since the last check (the message carries
-    the raw error word naming the wait site)."""
+    the raw error word naming the wait site), BqError(BQ_ERR_NONFINITE) if a
+    quantized-output GEMM epilogue met a NaN or Inf output."""
     detail = ctypes.c_int(0)
     st = lib().bq_device_status_detail(_stream(), ctypes.byref(detail))
     _check(st, f"device status (detail 0x{detail.value:x})")

@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdio>
 #include <cmath>
 #include <cstring>
@@ -37,6 +38,10 @@ struct DevInfo {
 std::mutex g_mu;
 DevInfo g_dev[kMaxDevices];
 
+// Compute capability the arch check compares instead of the probed one
+// (major * 10 + minor; -1 = the probe's): set by bq_debug_override_compute_capability.
+std::atomic<int> g_cc_override{-1};
+
 // Returns BQ_OK and fills `info` for the current device, BQ_ERR_ARCH if it is
 // not compute capability 10.0.
 int current_device(DevInfo** info) {
@@ -60,7 +65,23 @@ int current_device(DevInfo** info) {
     d.ready = true;
   }
   *info = &d;
-  return d.arch_ok ? BQ_OK : BQ_ERR_ARCH;
+  const int ov = g_cc_override.load();
+  return (d.arch_ok && (ov < 0 || ov == 100)) ? BQ_OK : BQ_ERR_ARCH;
+}
+
+// Watchdog self-test: one thread waits, with the bounded wait every kernel of
+// the library uses, on a shared-memory barrier that nothing ever arrives on,
+// so the wait runs out after limit_ns, records the timeout (site
+// kWaitSelftest) in the error word and returns.
+__global__ void wait_selftest_kernel(int* err, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    bq::mbar_init(&bar, 1);
+    abort_flag = 0;
+    bq::fence_mbar_init();
+    bq::mbar_wait(&bar, 0, err, &abort_flag, bq::kWaitSelftest, limit_ns);
+  }
 }
 
 inline bool aligned(const void* p, uintptr_t a) {
@@ -558,7 +579,7 @@ struct FusedAct {
 int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, const void* b_sf,
                int64_t M, int64_t N, int64_t K, void* y, const bq_epilogue* epi,
                const bq_batch* batch, void* ws, size_t ws_bytes, const bq_gemm_config* cfg,
-               bq_stream_t stream, const FusedAct* fused = nullptr) {
+               bq_stream_t stream, const FusedAct* fused = nullptr, bool clear_tickets = false) {
   DevInfo* dev = nullptr;
   int st = current_device(&dev);
   if (st != BQ_OK) return st;
@@ -724,6 +745,12 @@ int gemm_entry(WeightKind wk, const void* a_q, const void* a_sf, const void* b, 
     g.ws_partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kTicketRegion);
   }
   g.err = dev->err_ptr;
+  // A workspace that may hold another call's leftovers (the allocation-free
+  // entry's scratch): its ticket counters are zeroed on the stream only now,
+  // after every argument check, right before the kernel that reads them.
+  if (clear_tickets && pl.splits > 1 && !pl.cluster &&
+      cudaMemsetAsync(ws, 0, pl.ws_ticket, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return BQ_ERR_CUDA;
   if (pl.pair) {
     CUtensorMap map_sfa, map_sfb;
     // a stage's scale box: its chunks' atoms (two per chunk for packed E2M1)
@@ -1266,21 +1293,11 @@ int bq_gemm_mxfp8_mxfp4_epilogue_noalloc(const void* a_q, const void* a_sf, cons
   void* scratch = nullptr;
   st = noalloc_scratch(&scratch);
   if (st != BQ_OK) return st;
-  // Same planning as the call below makes with this scratch as its workspace
-  // (a schedule that needs more than the scratch is refused).
-  Plan pl;
-  st = plan_for_call(kMxfp4, M, N, K, count, cfg, dev->num_sms, scratch, kNoAllocScratchBytes,
-                     &pl);
-  if (st != BQ_OK) return st;
-  if (plan_ws_bytes(pl) > 0) {
-    // The scratch keeps whatever the previous call left: zero this call's
-    // ticket counters before the kernel reads them.
-    if (cudaMemsetAsync(scratch, 0, pl.ws_ticket, reinterpret_cast<cudaStream_t>(stream)) !=
-        cudaSuccess)
-      return BQ_ERR_CUDA;
-  }
+  // The scratch keeps whatever the previous call left: the call zeroes this
+  // problem's ticket counters itself, after its argument checks, just before
+  // the kernel.
   return gemm_entry(kMxfp4, a_q, a_sf, b_fp4, b_sf, M, N, K, y_bf16, epi, batch, scratch,
-                    kNoAllocScratchBytes, cfg, stream);
+                    kNoAllocScratchBytes, cfg, stream, nullptr, /*clear_tickets=*/true);
 }
 
 size_t bq_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
@@ -1297,7 +1314,28 @@ int bq_device_status_detail(bq_stream_t stream, int* detail) {
       cudaStreamSynchronize(s) != cudaSuccess)
     return BQ_ERR_CUDA;
   if (detail) *detail = err;
-  return err ? BQ_ERR_TIMEOUT : BQ_OK;
+  if (err & BQ_DEV_ERR_TIMEOUT) return BQ_ERR_TIMEOUT;
+  return (err & BQ_DEV_ERR_NONFINITE) ? BQ_ERR_NONFINITE : BQ_OK;
+}
+
+int bq_selftest_wait_timeout(int64_t limit_us, bq_stream_t stream) {
+  DevInfo* dev = nullptr;
+  int st = current_device(&dev);
+  if (st != BQ_OK) return st;
+  if (limit_us < 1 || limit_us > 1000000) return BQ_ERR_SHAPE;
+  wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      dev->err_ptr, static_cast<uint64_t>(limit_us) * 1000u);
+  return launch_status();
+}
+
+int bq_debug_override_compute_capability(int major, int minor) {
+  if (major < 0 || minor < 0) {
+    g_cc_override.store(-1);
+    return BQ_OK;
+  }
+  if (major > 99 || minor > 9) return BQ_ERR_INVALID;
+  g_cc_override.store(major * 10 + minor);
+  return BQ_OK;
 }
 
 int bq_device_status(bq_stream_t stream) { return bq_device_status_detail(stream, nullptr); }

@@ -8,9 +8,11 @@
 #include <cuda.h>
 #include <stdint.h>
 
-// Device error word: 0 = fine; otherwise BQ_DEV_ERR_TIMEOUT | (site << 8) of
-// the first wait that gave up.
+// Device error word: 0 = fine.  Bit BQ_DEV_ERR_TIMEOUT: a wait gave up (bits
+// 8..15 then name the site of the first one); bit BQ_DEV_ERR_NONFINITE: a
+// quantizing GEMM epilogue met a NaN or Inf output.
 #define BQ_DEV_ERR_TIMEOUT 1
+#define BQ_DEV_ERR_NONFINITE 2
 
 #ifndef BQ_WAIT_NS
 #define BQ_WAIT_NS 1000000000ull  // 1 s
@@ -28,6 +30,7 @@ enum WaitSite : int {
   kWaitPeerReady = 6,      // epilogue waiting for the cluster's partial tiles
   kWaitPeerDone = 7,       // epilogue waiting for the owners to free their receive buffers
   kWaitLanding = 8,        // last K slice waiting for the other slices' partial tiles
+  kWaitSelftest = 9,       // the watchdog self-test's wait on a barrier nothing completes
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -77,13 +80,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Records a wait that gave up in the error word: the timeout bit, and the
+// site of the first such wait.
+__device__ __forceinline__ void record_timeout(int *err, int site) {
+  if (!err) return;
+  const int old = atomicOr(err, BQ_DEV_ERR_TIMEOUT);
+  if (!(old & BQ_DEV_ERR_TIMEOUT)) atomicOr(err, (site & 0xFF) << 8);
+}
+
 // Wait until the phase with the given parity of `bar` has completed.  Gives
-// up after BQ_WAIT_NS (or as soon as *abort is set by another role), records
+// up after limit_ns (or as soon as *abort is set by another role), records
 // the wait site in *err and returns false.  Each poll suspends the thread up
 // to kWaitSuspendNs (it wakes when the phase completes); the timer is read
 // only after several failed polls, so ordinary waits never touch it.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err,
-                                          volatile int *abort, int site) {
+                                          volatile int *abort, int site,
+                                          uint64_t limit_ns = BQ_WAIT_NS) {
   const uint32_t b = smem_u32(bar);
 #pragma unroll 1
   for (int i = 0; i < 16; ++i)
@@ -94,9 +106,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *e
     for (int i = 0; i < 16; ++i)
       if (mbar_try_wait(b, parity)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > BQ_WAIT_NS) {
+    if (globaltimer() - t0 > limit_ns) {
       *abort = 1;
-      if (err) atomicCAS(err, 0, BQ_DEV_ERR_TIMEOUT | (site << 8));
+      record_timeout(err, site);
       return false;
     }
   }
@@ -112,7 +124,7 @@ __device__ __forceinline__ bool mbar_wait_timed(uint64_t *bar, uint32_t parity, 
   const uint64_t t0 = globaltimer();
   while (!mbar_try_wait(b, parity)) {
     if (globaltimer() - t0 > BQ_WAIT_NS) {
-      if (err) atomicCAS(err, 0, BQ_DEV_ERR_TIMEOUT | (site << 8));
+      record_timeout(err, site);
       return false;
     }
   }
@@ -184,7 +196,8 @@ __device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t bar, uint32_t
 
 // Bounded wait with cluster-scope acquire (the arrivals come from other CTAs).
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, int *err,
-                                                  volatile int *abort, int site) {
+                                                  volatile int *abort, int site,
+                                                  uint64_t limit_ns = BQ_WAIT_NS) {
   const uint32_t b = smem_u32(bar);
 #pragma unroll 1
   for (int i = 0; i < 16; ++i)
@@ -195,9 +208,9 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
     for (int i = 0; i < 16; ++i)
       if (mbar_try_wait_acq_cluster(b, parity)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > BQ_WAIT_NS) {
+    if (globaltimer() - t0 > limit_ns) {
       *abort = 1;
-      if (err) atomicCAS(err, 0, BQ_DEV_ERR_TIMEOUT | (site << 8));
+      record_timeout(err, site);
       return false;
     }
   }
@@ -320,6 +333,14 @@ __device__ __forceinline__ void bulk_wait_group_all() {
 // proxy (a TMA store that reads them after a barrier).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Order this thread's generic-proxy global-memory accesses against its
+// async-proxy ones (bulk copies): a writer issues it after storing data that a
+// bulk copy will read, and the thread that issues that copy issues it again
+// after it has observed the writer's release (the split-K partial tiles).
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // Contiguous global -> shared copy; src and dst 16-byte aligned, bytes % 16 == 0.

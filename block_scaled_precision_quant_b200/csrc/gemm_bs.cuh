@@ -388,6 +388,7 @@ __device__ __forceinline__ void quant_out_row32(const GemmArgs &a, int b, int m,
     qd[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
     qd[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
     sfo[sf_mma_offset(m, g, katoms)] = static_cast<uint8_t>(e + 127);
+    if (bad) atomicOr(a.err, BQ_DEV_ERR_NONFINITE);  // NaN or Inf among the outputs
   } else {
     sfo[sf_mma_offset(m, g, katoms)] = 127;
   }
@@ -436,6 +437,7 @@ __device__ __forceinline__ void copy_out_swap_q(const GemmArgs &a, const UnitPos
       *reinterpret_cast<uint2 *>(a.q_out + u.b * a.y_bstride + static_cast<int64_t>(m) * a.ldy +
                                  n) = make_uint2(codes[0], codes[1]);
       if ((v & 3) == 0) sfo[sf_mma_offset(m, n >> 5, katoms)] = static_cast<uint8_t>(e + 127);
+      if (bad) atomicOr(a.err, BQ_DEV_ERR_NONFINITE);  // NaN or Inf among the outputs
     }
   }
   // padding scale bytes
@@ -952,7 +954,8 @@ __device__ __forceinline__ bool fused_quant_unit(const GemmArgs &a, const UnitPo
 
 template <int BN, int STAGES, int ACC, bool SWAP, bool P_FP4, bool Q_FP4, int MODE, int KC,
           bool FUSEQ = false, int A4 = 0>
-__global__ void __launch_bounds__((!SWAP && MODE == kSplitNone) ? kWideThreads : kNumThreads, 1)
+__global__ void __launch_bounds__((!SWAP && MODE == kSplitNone) ? kWideThreads : kNumThreads,
+                                  (MODE == kSplitCluster && KC == 1) ? 2 : 1)
     gemm_bs_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_y,
                    const __grid_constant__ CUtensorMap tm_res, const GemmArgs a) {
@@ -1350,6 +1353,8 @@ __global__ void __launch_bounds__((!SWAP && MODE == kSplitNone) ? kWideThreads :
           for (int j = 0; j < 32; ++j)
             if (q0 + j < mt) __stcg(mine + (q0 + j) * kBlockP, __uint_as_float(v[j]));
         }
+        // the last slice's bulk copies (async proxy) read these partials
+        fence_proxy_async_global();
         epi_bar_sync();  // every partial store of this CTA is issued
         if (epi_tid == 0) {
           __threadfence();  // ... and visible device-wide before the ticket
@@ -1387,6 +1392,9 @@ __global__ void __launch_bounds__((!SWAP && MODE == kSplitNone) ? kWideThreads :
               ++s1;
             }
             if (n > 0 && epi_tid == 0) {
+              // the other slices' generic stores, acquired through the
+              // ticket, are read next by bulk copies (async proxy)
+              fence_proxy_async_global();
               mbar_arrive_expect_tx(land_bar, static_cast<uint32_t>(n * tile_floats * 4));
               int slot = 0;
               for (int sl = s0; sl < s1; ++sl)

@@ -13,11 +13,13 @@ namespace bq {
 // Gradient form (E5M2 codes): the same rule with E5M2's largest finite value
 // 57344 in place of 448 (fp32(1/57344) = fp32(1/448) * 2^-7), rounding to
 // nearest even or stochastically between the two neighbouring E5M2 values.
+// Capped at 113 (the largest bf16 gives 113, byte 240) as mx_exponent is.
 __device__ __forceinline__ int mx_exponent_e5m2(uint32_t amax_bits) {
   const float amax = fmaxf(__uint_as_float(amax_bits << 16), 1e-4f);
   const float t = __fmul_rn(amax, __uint_as_float(0x37924925u));  // fp32(1/57344)
   const uint32_t tb = __float_as_uint(t);
-  return static_cast<int>((tb >> 23) & 0xFFu) - 127 + ((tb & 0x7FFFFFu) != 0u ? 1 : 0);
+  const int e = static_cast<int>((tb >> 23) & 0xFFu) - 127 + ((tb & 0x7FFFFFu) != 0u ? 1 : 0);
+  return min(e, 113);
 }
 
 __device__ __forceinline__ uint32_t e5m2x2(float a, float b) {

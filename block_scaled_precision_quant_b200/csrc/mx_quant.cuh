@@ -74,12 +74,18 @@ __device__ __forceinline__ uint32_t bf16_amax_bits(const uint32_t (&w)[NW], uint
   return mx;
 }
 
-// Scale exponent e of a group from its amax bits.
+// Scale exponent e of a group from its amax bits.  Finite bf16 input gives
+// e <= 120 (amax = the largest bf16, byte 247); a group holding an Inf would
+// give 128 (byte 255, the NaN scale), so e is capped at 120: such a group,
+// which every caller reports as non-finite, still gets a valid scale byte
+// (its Inf codes saturate to +-448, a NaN input stays a NaN code), and a GEMM
+// that consumes it never meets the NaN scale.
 __device__ __forceinline__ int mx_exponent(uint32_t amax_bits) {
   const float amax = fmaxf(__uint_as_float(amax_bits << 16), 1e-4f);
   const float t = __fmul_rn(amax, __uint_as_float(0x3B124925u));  // fp32(1/448)
   const uint32_t tb = __float_as_uint(t);
-  return static_cast<int>((tb >> 23) & 0xFFu) - 127 + ((tb & 0x7FFFFFu) != 0u ? 1 : 0);
+  const int e = static_cast<int>((tb >> 23) & 0xFFu) - 127 + ((tb & 0x7FFFFFu) != 0u ? 1 : 0);
+  return min(e, 120);
 }
 
 // E4M3 codes of the 2 * NW bf16 values in w (element 2i in the low half of
@@ -108,11 +114,14 @@ __device__ __forceinline__ void mx_encode(const uint32_t (&w)[NW], int e,
 // maximum 6 in place of 448,
 //   t = fp32(amax * fp32(1/6)),  e = ceil(log2 t),  q = E2M1_RNE(clamp(x / 2^e, -6, 6)),
 // codes packed two per byte with the even element in the low nibble.
+// Capped at 126 (the largest bf16 gives 126, byte 253) for the same reason
+// as mx_exponent.
 __device__ __forceinline__ int mx_exponent_fp4(uint32_t amax_bits) {
   const float amax = fmaxf(__uint_as_float(amax_bits << 16), 1e-4f);
   const float t = __fmul_rn(amax, __uint_as_float(0x3E2AAAABu));  // fp32(1/6)
   const uint32_t tb = __float_as_uint(t);
-  return static_cast<int>((tb >> 23) & 0xFFu) - 127 + ((tb & 0x7FFFFFu) != 0u ? 1 : 0);
+  const int e = static_cast<int>((tb >> 23) & 0xFFu) - 127 + ((tb & 0x7FFFFFu) != 0u ? 1 : 0);
+  return min(e, 126);
 }
 
 // One byte of two E2M1 codes for the bf16 pair in `word` (element 2i in the

@@ -63,7 +63,7 @@ enum {
   BQ_ERR_WORKSPACE = 7,   /* workspace NULL or smaller than bq_gemm_workspace_bytes() */
   BQ_ERR_CUDA = 8,        /* a CUDA runtime call or kernel launch failed */
   BQ_ERR_TIMEOUT = 9,     /* a kernel gave up waiting on one of its own barriers */
-  BQ_ERR_NONFINITE = 10,  /* act_quant saw a NaN or Inf input */
+  BQ_ERR_NONFINITE = 10,  /* a NaN or Inf input (act_quant) or quantized output (GEMM) */
   BQ_ERR_INVALID = 11     /* an enum argument is out of range */
 };
 
@@ -225,7 +225,15 @@ int bq_unpack_scales(const void *sf_mma, int64_t rows, int64_t K, void *rowmajor
  *   a_q   [M, K] E4M3 activation codes (from bq_act_quant), 16-byte aligned
  *   a_sf  MMA-layout scales of A (from bq_act_quant), bq_sf_bytes(M, K)
  *   b     weights, 16-byte aligned (MXFP4: 32-byte aligned):
- *           mxfp4:    [N, K/2] packed E2M1, requires K % 128 == 0
+ *           mxfp4:    [N, K/2] packed E2M1, requires K % 128 == 0 (BQ_ERR_SHAPE
+ *                     otherwise).  The "formats.py" page ("Formats") only asks
+ *                     for K % 32 == 0; the narrower rule is this library's: the
+ *                     tensor-memory-access type that spreads 4-bit codes to the
+ *                     byte slots the MMA reads moves whole 128-code rows, and a
+ *                     tail shorter than 128 codes would need a read past the end
+ *                     of the weight buffer.  Pad K of both operands to a multiple
+ *                     of 128 with zero codes (and any finite scale) to use other
+ *                     sizes.
  *           fp8blk32: [N, K] E4M3 (32x32 block scales, packed by
  *                     bq_pack_weight_scales(BQ_SF_BLK32x32))
  *           mxfp8:    [N, K] E4M3 (per-32 row scales, from bq_act_quant or
@@ -488,15 +496,38 @@ size_t bq_noalloc_scratch_bytes(void);
 /* ---- diagnostics -------------------------------------------------------- */
 
 /* Reads and clears the library's device error word on the current device.
- * SYNCHRONIZES `stream`.  Returns BQ_OK, or BQ_ERR_TIMEOUT when a kernel gave
- * up on a barrier wait since the last call (its outputs are then invalid). */
+ * SYNCHRONIZES `stream`.  Returns BQ_OK; BQ_ERR_TIMEOUT when a kernel gave up
+ * on a barrier wait since the last call (its outputs are then invalid); else
+ * BQ_ERR_NONFINITE when a GEMM's quantized-output epilogue met a NaN or Inf
+ * output (those groups' scale bytes stay valid, their codes are unspecified). */
 int bq_device_status(bq_stream_t stream);
 
 /* bq_device_status, also returning the raw error word in *detail (may be
- * NULL): 0, or 1 | (site << 8) where site names the first wait that gave up
- * (1 producer/free stage, 2 MMA/free accumulator, 3 MMA/loaded stage,
- * 4 epilogue/finished accumulator, 5 teardown drain).  SYNCHRONIZES. */
+ * NULL): 0, or bit 0 (a wait gave up) with bits 8..15 naming the site of the
+ * first wait that gave up (1 producer/free stage, 2 MMA/free accumulator,
+ * 3 MMA/loaded stage, 4 epilogue/finished accumulator, 5 teardown drain,
+ * 6/7 cluster split exchange, 8 workspace split landing, 9 the self-test
+ * below), and bit 1 (non-finite quantized output).  SYNCHRONIZES. */
 int bq_device_status_detail(bq_stream_t stream, int *detail);
+
+/* Watchdog self-test (the hip_quant README's memory-safety guards on the
+ * pages, restated for this library's waits): launches one thread that waits,
+ * with the bounded wait every kernel here uses, on a barrier nothing ever
+ * completes.  The wait gives up after limit_us microseconds (1 .. 1000000),
+ * records the timeout in the device error word and the kernel returns: the
+ * next bq_device_status call reports BQ_ERR_TIMEOUT (site 9) and clears it,
+ * and the context stays usable.  Errors: BQ_ERR_SHAPE (limit out of range),
+ * BQ_ERR_ARCH, BQ_ERR_CUDA. */
+int bq_selftest_wait_timeout(int64_t limit_us, bq_stream_t stream);
+
+/* Test hook for the architecture check (the hip_quant README's guards on the
+ * pages): every entry point that checks the device compares (major, minor)
+ * instead of the probed compute capability, so a value other than 10.0 makes
+ * them return BQ_ERR_ARCH before launching anything.  It can only refuse: a
+ * device that is not 10.0 is refused whatever the override.  Negative values
+ * restore the probe.  Host-only; not thread-safe against concurrent calls.
+ * Errors: BQ_ERR_INVALID (major > 99 or minor > 9). */
+int bq_debug_override_compute_capability(int major, int minor);
 
 /* Writes a one-line report of the current device (name, compute capability,
  * SM count, L2 size, clocks) into buf (always NUL-terminated). */

@@ -125,9 +125,18 @@ def test_nonfinite_input_sets_status():
     x[1, 40] = 0x7F80  # +Inf
     xd = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    bq.act_quant(xd, status=status)
+    q, sf = bq.act_quant(xd, status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 1
+    # the group holding the Inf gets a valid scale byte (the exponent's cap,
+    # 247), never the NaN scale 255; the other groups are exact
+    sf_row = bq.unpack_scales(sf, 2, 64).cpu().numpy()
+    assert sf_row[1, 1] == 247
+    q_ref, s_ref = oracle.act_quant(x[:, :32])
+    assert np.array_equal(sf_row[:, 0], s_ref[:, 0])
+    assert np.array_equal(q.cpu().numpy()[:, :32], q_ref)
+    q_ref0, s_ref0 = oracle.act_quant(x[:1, 32:])
+    assert sf_row[0, 1] == s_ref0[0, 0]
 
 
 def test_empty_m_launches_nothing():

@@ -4,9 +4,11 @@ Some callers cannot allocate device memory (a plugin given only its inputs and
 outputs, a serving loop with a fixed memory budget); this entry point runs the
 K-split MXFP4 GEMM on a scratch array the library owns.  The test calls it
 through the C ABI twice in a row (the second call finds the first call's
-leftovers in the shared scratch) and compares each result with the existing
-workspace entry point, within the tolerance the parity tests use.  The file is
-named to be collected last; it passes on its own in a fresh process too.
+leftovers in the shared scratch) and checks each result against the oracle's
+fp64 reference, within the tolerance the parity tests use, and bit for bit
+against the existing workspace entry point (both reduce the K slices in the
+same fixed order).  The file is named to be collected last; it passes on its
+own in a fresh process too.
 """
 import ctypes
 
@@ -63,13 +65,15 @@ def test_noalloc_matches_workspace_entry_twice():
         bq.device_status()
 
         q, s = oracle.act_quant(x)
-        _, sabs = oracle.gemm(q, s, w, ws, oracle.B_FP4, M, N, K, bias=bias)
-        old = _f64(y_old)
+        assert np.array_equal(aq.cpu().numpy(), q)
+        ref, sabs = oracle.gemm(q, s, w, ws, oracle.B_FP4, M, N, K, bias=bias)
         babs = np.abs((bias.astype(np.uint32) << 16).view(np.float32).astype(np.float64))
-        tol = oracle.gemm_tolerance(old, sabs, 1.0, babs[None, :])
+        tol = oracle.gemm_tolerance(ref, sabs, 1.0, babs[None, :])
         new = _f64(y_new)
         assert np.all(np.isfinite(new))
-        assert np.all(np.abs(new - old) <= tol), f"call {call}"
+        assert np.all(np.abs(new - ref) <= tol), f"call {call}: outside the oracle tolerance"
+        assert torch.equal(y_new.view(torch.int16), y_old.view(torch.int16)), \
+            f"call {call}: differs from the workspace entry point"
 
 
 def test_noalloc_rejects_problems_beyond_the_scratch():
@@ -83,3 +87,21 @@ def test_noalloc_rejects_problems_beyond_the_scratch():
         dummy.data_ptr(), None, None, ctypes.byref(cfg),
         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == bq.BQ_ERR_WORKSPACE
+
+
+def test_noalloc_checks_arguments_like_the_workspace_entry():
+    """Argument errors come first and in the same order as the workspace entry
+    point's: a NULL output is BQ_ERR_NULL even for a problem too large for the
+    scratch, and a misaligned one BQ_ERR_ALIGN, before anything is enqueued."""
+    L = bq.lib()
+    M, N, K = 64, 16384, 4096
+    cfg = bq.config(split_k=16, swap_ab=1, split_mode=bq.BQ_SPLIT_WORKSPACE)
+    dummy = torch.zeros((1 << 20,), dtype=torch.uint8, device="cuda")
+    p = dummy.data_ptr()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for y, want in ((None, bq.BQ_ERR_NULL), (p + 2, bq.BQ_ERR_ALIGN)):
+        st_new = L.bq_gemm_mxfp8_mxfp4_epilogue_noalloc(p, p, p, p, M, N, K, y, None, None,
+                                                        ctypes.byref(cfg), stream)
+        st_old = L.bq_gemm_mxfp8_mxfp4_epilogue(p, p, p, p, M, N, K, y, None, None, None, 0,
+                                                ctypes.byref(cfg), stream)
+        assert st_new == st_old == want
