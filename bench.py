@@ -460,9 +460,10 @@ class Layer:
                             residual=d["res"],
                             act=bq.BQ_ACT_GELU if self.gelu else bq.BQ_ACT_NONE,
                             a_q=self.aq, a_sf=self.asf[0], **kw)
-            # one fused launch; a K loop of >= 24 blocks (the library's split
-            # rule) runs act_quant + the split GEMM instead
-            return 2 if (K + 127) // 128 >= 24 and not self.quant_out else 1
+            # one fused launch; a shape the library splits runs act_quant +
+            # the split GEMM instead
+            split = bq.plan(M, N, K, weight_kind=self.wk).split_k > 1
+            return 2 if split and not self.quant_out else 1
         if which in ("all", "act_quant"):
             quant = (bq.act_quant_nvfp4 if self.nv else
                      bq.act_quant_mxfp4 if self.a4 else bq.act_quant)

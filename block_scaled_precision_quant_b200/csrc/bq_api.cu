@@ -273,15 +273,23 @@ int make_plan(int64_t M, int64_t N, int64_t K, int64_t batch, const bq_gemm_conf
   const bool use_ws = req_mode == BQ_SPLIT_WORKSPACE;
   if (splits == 0) {
     splits = 1;
-    // Decode tiles (sweeps): up to ~12 K blocks an unsplit tile with 4-chunk
-    // stages is fastest -- a split pays ~3 us of exchange (fence, ticket and
-    // a gather through L2, or a DSMEM exchange), more than it saves.  With a
-    // long K loop (>= 24 K blocks) a power-of-two cluster split wins: spread
-    // it while the grid stays within one CTA per SM.
+    // Decode tiles (sweeps): a cluster split pays ~2 us of exchange (the
+    // slices' fp32 rows through DSMEM, ~1 us for the last of them to land,
+    // the owners' reduce), so it wins only where it cuts a long per-tile
+    // mainloop.  With a long K loop (>= 24 K blocks) a power-of-two cluster
+    // split wins: spread it while the grid stays within one CTA per SM.
+    // With 12..23 K blocks it wins only when the slices fill nearly every
+    // SM (41x4608x1536: 36 tiles x 4 slices on 148 SMs, 6.8 against 7.0 us
+    // unsplit; 48 tiles x 2 slices lose, 7.7 against 7.1 us).
     if (p->swap && req_mode != BQ_SPLIT_WORKSPACE && p->kt_total >= 24) {
       while (splits * 2 <= kMaxClusterSplit && tiles * splits * 2 <= num_sms &&
              p->kt_total / (splits * 2) >= 4)
         splits *= 2;
+    } else if (p->swap && req_mode != BQ_SPLIT_WORKSPACE && p->kt_total >= 12) {
+      int s = 1;
+      while (s * 2 <= kMaxClusterSplit && tiles * s * 2 <= num_sms && p->kt_total / (s * 2) >= 3)
+        s *= 2;
+      if (s > 1 && tiles * s * 10 >= num_sms * 9) splits = s;
     }
   }
   if (splits > p->kt_total) splits = p->kt_total;

@@ -223,6 +223,19 @@ __device__ __forceinline__ void st_dsmem_u4(uint32_t cluster_addr, uint32_t x, u
                : "memory");
 }
 
+// Asynchronous 16-byte store into another CTA of the cluster that, once it
+// has landed, completes 16 bytes of transaction count on the mbarrier at
+// cluster_bar (an mbarrier of that same CTA): the receiver learns of the data
+// by waiting on its barrier, with no release fence and arrive by the sender.
+__device__ __forceinline__ void st_async_u4(uint32_t cluster_addr, uint32_t x, uint32_t y,
+                                            uint32_t z, uint32_t w, uint32_t cluster_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::
+          "r"(cluster_addr),
+      "r"(x), "r"(y), "r"(z), "r"(w), "r"(cluster_bar)
+      : "memory");
+}
+
 __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t cluster_addr) {
   float4 v;
   asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"

@@ -1025,7 +1025,8 @@ __global__ void __launch_bounds__((!SWAP && MODE == kSplitNone) ? kWideThreads :
     }
     mbar_init(drain, 1);
     if constexpr (CSPLIT) {
-      mbar_init(peer_ready, a.splits);
+      // one arrival: this CTA's own expect_tx for the rows its peers send
+      mbar_init(peer_ready, 1);
       mbar_init(peer_free, a.splits);
     }
     if constexpr (L::kBytesLand > 0) mbar_init(land_bar, 1);
@@ -1240,10 +1241,13 @@ __global__ void __launch_bounds__((!SWAP && MODE == kSplitNone) ? kWideThreads :
       const uint32_t t_row = tmem_base + acc * BN + (static_cast<uint32_t>(quad * 32) << 16);
       if constexpr (MODE == kSplitCluster) {
         // Cluster split-K: the S CTAs of this cluster hold the S K-slices of
-        // one output tile.  Every CTA pushes each row of its fp32 partial
-        // straight from TMEM registers into the receive buffer of the CTA that
-        // owns that row (DSMEM stores), signals the owners, then finishes its
-        // own 128/S rows from local shared memory.
+        // one output tile.  Every CTA sends each row of its fp32 partial
+        // straight from TMEM registers to the CTA that owns that row: rows it
+        // owns itself go to its own receive buffer by plain stores, the others
+        // by asynchronous DSMEM stores that complete transaction bytes on the
+        // owner's peer_ready barrier (armed by the owner with the bytes its
+        // S - 1 peers send), so no release fence or remote arrive is needed.
+        // Then each CTA finishes its own 128/S rows from local shared memory.
         const int lg = a.split_lg;
         const int S = 1 << lg;
         if (free_pending) {  // the owners' receive buffers are free again
@@ -1252,13 +1256,19 @@ __global__ void __launch_bounds__((!SWAP && MODE == kSplitNone) ? kWideThreads :
           free_pending = false;
         }
         const int R = kBlockP >> lg;
-        const uint32_t owner = static_cast<uint32_t>(row >> (7 - lg));
-        const uint32_t dst =
-            mapa_shared(smem_u32(recv), owner) +
-            static_cast<uint32_t>((u.split * R + (row & (R - 1))) * L::kRecvStride * 4);
-        // only the tile's activation columns that exist are pushed (a 41-row
-        // operand fills 41 of 64): the owners read no others
+        // only the tile's activation columns that exist are sent (a 41-row
+        // operand fills 41 of 64), in 16-byte pieces: ceil(mvalid / 4) per row
         const int mvalid = min(BN, a.M - u.tq * BN);
+        const int pieces = (mvalid + 3) >> 2;
+        if (epi_tid == 0)
+          mbar_arrive_expect_tx(peer_ready, static_cast<uint32_t>((S - 1) * R * pieces * 16));
+        const uint32_t owner = static_cast<uint32_t>(row >> (7 - lg));
+        const bool mine = owner == static_cast<uint32_t>(u.split);  // cluster rank == slice
+        const uint32_t slot =
+            static_cast<uint32_t>((u.split * R + (row & (R - 1))) * L::kRecvStride * 4);
+        const uint32_t dst = mapa_shared(smem_u32(recv), owner) + slot;
+        const uint32_t dbar = mapa_shared(smem_u32(peer_ready), owner);
+        float *local = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(recv) + slot);
 #pragma unroll 1
         for (int c = 0; c < BN / 32 && c * 32 < mvalid; ++c) {  // warp-uniform
           uint32_t v[32];
@@ -1266,20 +1276,21 @@ __global__ void __launch_bounds__((!SWAP && MODE == kSplitNone) ? kWideThreads :
           tmem_ld_32x32b_x32(t_row + c * 32, v);
           tmem_ld_wait();
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            if (c * 32 + 4 * q < mvalid)
-              st_dsmem_u4(dst + static_cast<uint32_t>((c * 32 + 4 * q) * 4), v[4 * q],
-                          v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          for (int q = 0; q < 8; ++q) {
+            if (c * 32 + 4 * q < mvalid) {
+              if (mine)
+                *reinterpret_cast<uint4 *>(local + c * 32 + 4 * q) =
+                    make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+              else
+                st_async_u4(dst + static_cast<uint32_t>((c * 32 + 4 * q) * 4), v[4 * q],
+                            v[4 * q + 1], v[4 * q + 2], v[4 * q + 3], dbar);
+            }
+          }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[acc]);
-        epi_bar_sync();
-        if (epi_tid == 0) {
-          fence_acq_rel_cluster();
-          const uint32_t rb = smem_u32(peer_ready);
-          for (int r = 0; r < S; ++r) mbar_arrive_cluster(mapa_shared(rb, static_cast<uint32_t>(r)));
-        }
+        epi_bar_sync();  // this CTA's own rows are in its receive buffer
         if (!mbar_wait_cluster(peer_ready, ready_phase, a.err, abort_flag, kWaitPeerReady)) break;
         ready_phase ^= 1;
         switch (lg) {

@@ -20,10 +20,12 @@ def desc(c):
                 split_mode=c.split_mode, k_chunks=c.k_chunks, cta_pair=c.cta_pair)
 
 
-@pytest.mark.parametrize("N,K,split", [(4608, 1536, 1), (6144, 1536, 1), (1536, 6144, 8)])
+@pytest.mark.parametrize("N,K,split", [(4608, 1536, 4), (6144, 1536, 1), (1536, 6144, 8)])
 def test_decode_layers(N, K, split):
-    """M = 41: swap-AB tiles of 64 activation rows; the short-K layers unsplit
-    with 4 chunks per stage, the long-K layer on 8-CTA cluster slices."""
+    """M = 41: swap-AB tiles of 64 activation rows; the 6144-wide short-K
+    layer unsplit with 4 chunks per stage, the 4608-wide one on 4-CTA
+    cluster slices (36 x 4 CTAs fill 144 of 148 SMs), the long-K layer on
+    8-CTA cluster slices."""
     d = desc(bq.plan(41, N, K, num_sms=SMS))
     assert d["swap_ab"] == 1 and d["block_n"] == 64 and d["cta_pair"] == 1
     assert d["split_k"] == split
@@ -32,6 +34,14 @@ def test_decode_layers(N, K, split):
     else:
         assert d["split_mode"] == bq.BQ_SPLIT_CLUSTER
     assert (N // 128) * split <= SMS  # one CTA per SM
+
+
+def test_short_k_split_needs_nearly_every_sm():
+    # 36 tiles: 4 slices fill 144 of 148 SMs; on 160 SMs 144 is below 90 %
+    assert bq.plan(41, 4608, 1536, num_sms=148).split_k == 4
+    assert bq.plan(41, 4608, 1536, num_sms=170).split_k == 1
+    # 12 K blocks at most; fewer stay unsplit
+    assert bq.plan(41, 4608, 1280, num_sms=148).split_k == 1
 
 
 def test_small_m_tiles():

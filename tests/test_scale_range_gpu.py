@@ -15,9 +15,7 @@ at the top (234..254), the top of the weights' range (230..246) against the
 bottom of the activations', and both sides spread over 94..160 (products
 spanning 2^+-60 inside one output).  The exponent sums stay where fp32 holds
 the result.  Products that fall into fp32's subnormal range (a separate
-case) are compared with an allowance for the tensor core flushing them:
-(K/32 + 1) * 2^-126, one flushed block partial per 32-input block and the
-accumulator.
+case) are held to the same bound.
 
 The cancellation cases pair every term of the first half of K with its
 negation in the second half (same magnitudes, same scales), so sum a b = 0
@@ -46,7 +44,6 @@ FINITE_E4M3 = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.u
 # E4M3 codes of magnitude >= 2^-2 (exponent field >= 5), for the cancellation
 # cases: with them every partial sum of a row fits fp64 exactly
 WIDE_E4M3 = np.array([c for c in FINITE_E4M3 if (c >> 3) & 0xF >= 5], dtype=np.uint8)
-FTZ_ALLOWANCE = 2.0 ** -126
 
 
 def dev_u8(a):
@@ -83,12 +80,12 @@ def gemm_gpu(wk, aq, asf, b, bsf, M, N, K, config=None):
     return f64(y.cpu().view(torch.int16).numpy().view(np.uint16))
 
 
-def check(wk, aq, asf, b, bsf, M, N, K, config=None, allowance=0.0, what=""):
+def check(wk, aq, asf, b, bsf, M, N, K, config=None, what=""):
     _, _, okind, akind = KINDS[wk]
     y = gemm_gpu(wk, aq, asf, b, bsf, M, N, K, config)
     ref, sabs = oracle.gemm(aq, asf, b, bsf, okind, M, N, K, a_kind=akind)
     assert np.all(np.isfinite(y)), f"{what}: non-finite output"
-    tol = oracle.gemm_tolerance(ref, sabs) + allowance
+    tol = oracle.gemm_tolerance(ref, sabs)
     err = np.abs(y - ref)
     bad = np.argwhere(~(err <= tol))
     assert bad.size == 0, (f"{what}: {bad.shape[0]} of {err.size} outside tolerance; first "
@@ -146,11 +143,12 @@ def test_scale_bands_decode_tiles(wk, band, split):
 @pytest.mark.parametrize("wk", [bq.W_MXFP4, bq.W_MXFP8, bq.W_A4W4])
 def test_scale_band_subnormal_products(wk):
     """Exponent sums a + b - 254 in [-154, -107]: products and block partials
-    in or below fp32's subnormal range.  The tensor core may flush them; the
-    bound then widens by one 2^-126 per 32-input block and the accumulator."""
+    in or below fp32's subnormal range, outputs down to ~1e-40.  The pages
+    leave the treatment of such values open; the plain bound holds (the
+    tensor core does not flush them on B200), so no allowance is given."""
     M, N, K = 130, 136, 256
     ops = operands(wk, M, N, K, (100, 127), (0, 20), seed=31, b_force=0)
-    check(wk, *ops, M, N, K, allowance=(K // 32 + 1) * FTZ_ALLOWANCE, what=f"subnormal {wk}")
+    check(wk, *ops, M, N, K, what=f"subnormal {wk}")
 
 
 # ------------------------------------------------------------- cancellation --
