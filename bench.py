@@ -10,9 +10,10 @@ line, and carries every other workload of the suite as a sub-record of that
 line ("suite"): the 64x512x1024 MXFP8 x MXFP4 reference case, the three
 decode-shaped (M = 41) layers with bias, the FP8 32x32-block weights at
 1024x4096x4096 with a residual, the batched MLP up-projection 8 x
-(1024x2048x2048) with bias + GELU and its 4096x1536x6144 down-projection.
-Every record has its own roofline, act_quant bandwidth, end-to-end number and
-CPU-oracle baseline.
+(1024x2048x2048) with bias + GELU and its 4096x1536x6144 down-projection,
+then the FP4 x FP4 rows (MXFP4 decode layers and 8192^3, NVFP4 8192^3) and
+the backward of a 4096x1536x6144 layer.  Every record has its own roofline,
+act_quant bandwidth, end-to-end number and CPU-oracle baseline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload suite|square|decode|pr1|fp8blk|mlp|mlp_up|...]
@@ -108,9 +109,11 @@ WORKLOADS = {
         layers=[("bwd", "grad", 4096, 1536, 6144, 1, dict())], bound="tensor"),
 }
 
-# The default run: the headline workload, then the suite's sub-records.
+# The default run: the headline workload, then the suite's sub-records (the
+# reference configurations, then the FP4 x FP4 and backward rows).
 HEADLINE = "square"
-SUITE = ("pr1", "decode", "fp8blk", "mlp_up", "mlp_down")
+SUITE = ("pr1", "decode", "fp8blk", "mlp_up", "mlp_down", "a4w4_decode", "a4w4_square",
+         "nvfp4_square", "backward")
 
 WKIND = {"mxfp4": 0, "fp8blk32": 1, "mxfp8": 2, "a4w4": 3, "grad": 4, "nvfp4": 5}
 DTYPE = {"mxfp4": "mxfp8xmxfp4", "fp8blk32": "mxfp8xfp8blk32", "mxfp8": "mxfp8xmxfp8",

@@ -137,3 +137,26 @@ def test_suite_names_every_workload_once():
     # the batched up-projection and the down-projection are separate records
     assert bench.WORKLOADS["mlp_up"]["layers"] + bench.WORKLOADS["mlp_down"]["layers"] == \
         bench.WORKLOADS["mlp"]["layers"]
+
+
+def test_reference_arm_line(capsys):
+    """The reference arm on the smallest workload: one JSON line with the
+    oracle timed on this host, its thread count and CPU model."""
+    import json
+    assert bench.main(["--impl", "reference", "--workload", "pr1", "--steps", "1",
+                       "--warmup", "3"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["value"] > 0 and line["unit"] == "TFLOP/s" and line["steps"] == 1
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["cpu_model"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_oracle_sample_counts_the_weight_quantization():
+    """The square workload's sample quantizes rows*N/M rows of its weight
+    operand on top of the activation rows (a smaller square stands in)."""
+    spec = [("sq", "mxfp8", 256, 256, 256, 1, {})]
+    sample = bench.OracleSample(spec)
+    flops, secs, threads = sample.run(4)
+    assert flops == 2.0 * 4 * 256 * 256 and secs > 0 and threads >= 1
