@@ -672,6 +672,92 @@ __device__ __forceinline__ void epilogue_rows_tma_g2(const GemmArgs &a, const CU
   }
 }
 
+// The two-group epilogue without a residual, accumulator released first: each
+// thread reads its row's chunks of the group (NCOLS / 64 of them) from TMEM and
+// turns them into final bf16 values in registers, then the group's warps
+// release the accumulator (`tempty`) and only afterwards stage and store the
+// chunks.  The accumulator is then busy only for the TMEM reads, so with one
+// accumulator per CTA the next tile's MMAs start while this tile's output is
+// still being written.  (With a residual the final value needs the residual
+// tile, which is brought in chunk by chunk through the staging slot:
+// epilogue_rows_tma_g2 keeps the accumulator until the last chunk.)
+template <int NCOLS>
+__device__ __forceinline__ void epilogue_rows_drain_g2(const GemmArgs &a, const CUtensorMap *tm_y,
+                                                       uint32_t t_row, int b, int m0, int n0,
+                                                       int row, int epi_tid, int group,
+                                                       uint8_t *ystage, uint64_t *tempty_bar) {
+  constexpr int kPer = NCOLS / 64;  // chunks of 32 columns per group
+  const int m = m0 + row;
+  const int nch = min(NCOLS / 32, (a.N - n0 + 31) / 32);
+  uint8_t *buf = ystage + group * kYChunkBytes;
+  uint32_t o[kPer][16];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int c = group + 2 * i;
+    if (c >= nch) break;  // uniform
+    const int q0 = n0 + c * 32;
+    uint32_t v[32];
+    __syncwarp();
+    tmem_ld_32x32b_x32(t_row + c * 32, v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      float bias8[8];
+      if (a.bias && q0 + 8 * g < a.N) {
+        const uint4 bv = __ldg(reinterpret_cast<const uint4 *>(a.bias + q0 + 8 * g));
+        const uint32_t w[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          bias8[2 * j] = bf16_bits_to_f32(w[j] & 0xFFFF);
+          bias8[2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) bias8[j] = 0.0f;
+      }
+      float t[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) t[j] = a.alpha * __uint_as_float(v[8 * g + j]) + bias8[j];
+      if (a.act == 1) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) t[j] = gelu_erf(t[j]);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __nv_bfloat162 p2 = __floats2bfloat162_rn(t[2 * j], t[2 * j + 1]);
+        o[i][4 * g + j] = *reinterpret_cast<const uint32_t *>(&p2);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(tempty_bar);
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int c = group + 2 * i;
+    if (c >= nch) break;  // uniform
+    const int q0 = n0 + c * 32;
+    if (a.q_out) quant_out_row32(a, b, m, q0, o[i]);
+    if (a.y) {  // uniform
+      if (epi_tid == 0) bulk_wait_group_read<0>();  // the group's previous store has read the slot
+      epi_bar_sync(group);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<uint4 *>(buf + row * 64 + ((j ^ ((row >> 1) & 3)) << 4)) =
+            make_uint4(o[i][4 * j], o[i][4 * j + 1], o[i][4 * j + 2], o[i][4 * j + 3]);
+      fence_proxy_async_smem();
+      epi_bar_sync(group);
+      if (epi_tid == 0) {
+        if (a.batch > 1)
+          tma_store_3d(tm_y, buf, q0, m0, b);
+        else
+          tma_store_2d(tm_y, buf, q0, m0);
+        bulk_commit_group();
+      }
+    }
+  }
+}
+
 // Swap-AB epilogue, first half: the 32 values of output column n = prow
 // (rows m = q0 .. q0+31, tile columns c0 .. c0+31) become final bf16 values
 // in the staging tile stage[c][n - n0].  Across a warp each row is written as
@@ -1336,12 +1422,17 @@ __global__ void __launch_bounds__((!SWAP && MODE == kSplitNone) ? kWideThreads :
           copy_out_swap<BN>(a, u, epi_tid, stage);
         if (unit + static_cast<int>(gridDim.x) < total_units) epi_bar_sync();  // staging free
       } else if constexpr (MODE == kSplitNone) {
-        epilogue_rows_tma_g2<BN>(a, &tm_y, &tm_res, full + L::kRbarIndex, rphase, t_row, u.b,
-                                 u.tp * kBlockP, u.tq * BN, row, epi_tid, egroup,
-                                 smem + L::kOffYStage, abort_flag);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[acc]);
+        if (a.res == nullptr) {
+          epilogue_rows_drain_g2<BN>(a, &tm_y, t_row, u.b, u.tp * kBlockP, u.tq * BN, row,
+                                     epi_tid, egroup, smem + L::kOffYStage, &tempty[acc]);
+        } else {
+          epilogue_rows_tma_g2<BN>(a, &tm_y, &tm_res, full + L::kRbarIndex, rphase, t_row, u.b,
+                                   u.tp * kBlockP, u.tq * BN, row, epi_tid, egroup,
+                                   smem + L::kOffYStage, abort_flag);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[acc]);
+        }
       } else if constexpr (MODE == kSplitWorkspace && SWAP) {
         // Split-K, swap-AB: publish this slice's fp32 partial (valid rows m
         // only, stored [m][n] so a warp writes 128 contiguous bytes per m) and
