@@ -16,9 +16,12 @@
 //     report back to the leader before it reuses the accumulator.
 // Per 128-K block an SM then moves 32 KB into shared memory and its tensor
 // core reads 32 KB (own A + own half of B, shared with the peer), where a
-// single-SM 128x256 tile moves 48 KB and reads 48 KB for the same MMA work:
-// that single-SM tile is bound by shared-memory bandwidth, the pair tile by
-// the tensor pipe.
+// single-SM 128x256 tile moves 48 KB and reads 48 KB for the same MMA work.
+// Measured on the 8192^3 MXFP8 problem the copies are not what limits either
+// kernel, and this one is the slower: it holds one accumulator per CTA whose
+// four epilogue warps drain it chunk by chunk while the next tile's MMAs
+// wait, and even with no copies at all its mainloop runs well below the MMA
+// rate.  The built-in dispatch therefore runs it only on request.
 #pragma once
 
 #include "gemm_bs.cuh"
