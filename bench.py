@@ -470,12 +470,15 @@ class Layer:
         if which in ("all", "act_quant"):
             quant = (bq.act_quant_nvfp4 if self.nv else
                      bq.act_quant_mxfp4 if self.a4 else bq.act_quant)
+            # The weight operand first: a GEMM may read its weights while the
+            # kernel just before it is still running (programmatic launch), so
+            # that kernel must be the activations' quantizer, not the weights'.
+            if d["wx"] is not None:
+                bq.act_quant(d["wx"], q=d["w"], sf_mma=d["wsf"])
+                n += 1
             for b in range(B):
                 quant(d["x"][b * M:(b + 1) * M], q=self.aq[b * M:(b + 1) * M],
                       sf_mma=self.asf[b])
-                n += 1
-            if d["wx"] is not None:
-                bq.act_quant(d["wx"], q=d["w"], sf_mma=d["wsf"])
                 n += 1
         if which in ("all", "gemm"):
             batch = None

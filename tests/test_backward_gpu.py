@@ -220,12 +220,15 @@ def backward_case(T, N, K, seed):
     w = synth.activations(N, K, seed=seed + 1, std=0.05)
     dy = grads(T, N, seed=seed + 2)
     xd, wd, dyd = dev_bf16(x), dev_bf16(w), dev_bf16(dy)
-    # dX [T, K] = dY W: contraction over N
-    gq, gsf, gtq, gtsf = bq.grad_quant_dual(dyd, stochastic=True, seed=11)  # dY, dY^T [N, T]
+    # The B operands (W^T, X^T) are quantized before dY: a GEMM may read its
+    # B operand while the kernel just before it is still running, so that
+    # kernel is the quantizer of its A operand.
     wtq, wtsf = bq.quant_transposed(wd, fmt=bq.BQ_FMT_E4M3)              # W^T [K, N]
+    xtq, xtsf = bq.quant_transposed(xd, fmt=bq.BQ_FMT_E4M3)              # X^T [K, T]
+    gq, gsf, gtq, gtsf = bq.grad_quant_dual(dyd, stochastic=True, seed=11)  # dY, dY^T [N, T]
+    # dX [T, K] = dY W: contraction over N
     dx = bq.gemm(bq.W_GRAD, gq, gsf, wtq, wtsf, T, K, N)
     # dW [N, K] = dY^T X: contraction over T
-    xtq, xtsf = bq.quant_transposed(xd, fmt=bq.BQ_FMT_E4M3)              # X^T [K, T]
     dw = bq.gemm(bq.W_GRAD, gtq, gtsf, xtq, xtsf, N, K, T)
     bq.device_status()
     og, ogs = oracle.grad_quant(dy, stochastic=True, seed=11)
