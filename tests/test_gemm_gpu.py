@@ -363,8 +363,11 @@ def test_decode_workload_full(N, K):
 
 # ----------------------------------------------------------------- batch --
 
-def test_batched_broadcast_weight_bias_gelu():
-    """Independent problems over one broadcast weight (stride 0), bias+GELU."""
+@pytest.mark.parametrize("cfg", [None, dict(split_k=1, swap_ab=0, block_n=256),
+                                 dict(split_k=1, swap_ab=0, block_n=128)])
+def test_batched_broadcast_weight_bias_gelu(cfg):
+    """Independent problems over one broadcast weight (stride 0), bias+GELU, in
+    the built-in schedule and on both wide tile widths (3-D output stores)."""
     count, M, N, K = 3, 200, 264, 256
     xs = [synth.activations(M, K, seed=40 + i) for i in range(count)]
     b, bsf = synth.mxfp4_weight(N, K, seed=50)
@@ -374,7 +377,7 @@ def test_batched_broadcast_weight_bias_gelu():
     asf = torch.stack(sfs)
     bsf_d = bq.pack_weight_scales(to_dev_u8(bsf), bq.BQ_SF_ROW32, N, K)
     y = bq.gemm(bq.W_MXFP4, aq, asf, to_dev_u8(b), bsf_d, M, N, K, bias=to_dev_bf16(bias),
-                act=bq.BQ_ACT_GELU,
+                act=bq.BQ_ACT_GELU, config=bq.config(**cfg) if cfg else None,
                 batch=dict(count=count, stride_a=M * K, stride_a_sf=asf.shape[1], stride_b=0,
                            stride_b_sf=0, stride_y=M * N * 2))
     bq.device_status()
@@ -541,10 +544,15 @@ def _quant_out_case(c, config=None, write_y=True):
         assert y2 is None and torch.equal(q2, q) and torch.equal(sf2, sf)
 
 
-@pytest.mark.parametrize("M,N,K,write_y", [(300, 800, 640, True), (128, 512, 256, False)])
-def test_quant_out_wide_tiles(M, N, K, write_y):
+@pytest.mark.parametrize("M,N,K,write_y,bn", [(300, 800, 640, True, 128), (128, 512, 256, False, 128),
+                                               (300, 800, 640, True, 256),
+                                               (136, 544, 384, False, 256)])
+def test_quant_out_wide_tiles(M, N, K, write_y, bn):
+    # 128 x 256 tiles keep one accumulator and read all of a row's chunks into
+    # registers before the stores; N = 800 and 544 end in a tile of one
+    # 32-column chunk, where the second epilogue group has no chunk at all.
     _quant_out_case(Case(bq.W_MXFP4, M, N, K, seed=81, bias=True, act=bq.BQ_ACT_GELU),
-                    config=bq.config(split_k=1, swap_ab=0, block_n=128), write_y=write_y)
+                    config=bq.config(split_k=1, swap_ab=0, block_n=bn), write_y=write_y)
 
 
 def test_quant_out_pair_tiles():
