@@ -171,7 +171,7 @@ struct GemmSmem {
   static constexpr int kBytesOut = OUT_STAGE ? BN * kBlockP * 2 : 0;
   // swap-AB workspace split: this slice's fp32 partial tile [BN m][128 n],
   // then the landing area for the other slices' partial tiles ([slice][m][128
-  // n], as many slices per round as fit)
+  // n], as many slices per pass as fit)
   static constexpr int kOffAcc = kOffOut + kBytesOut;
   static constexpr int kBytesAcc = LANDING ? BN * kBlockP * 4 : 0;
   static constexpr int kOffLand = kOffAcc + kBytesAcc;
@@ -1068,7 +1068,7 @@ __global__ void __launch_bounds__((!SWAP && MODE == kSplitNone) ? kWideThreads :
   uint64_t *drain = tempty + ACC;
   uint64_t *peer_ready = drain + 1;  // CSPLIT: every slice's rows for this CTA have arrived
   uint64_t *peer_free = drain + 2;   // CSPLIT: every owner has consumed the previous tile
-  uint64_t *land_bar = drain + 1;    // workspace split: a round of partial tiles has landed
+  uint64_t *land_bar = drain + 1;    // workspace split: a pass of partial tiles has landed
   float *recv = reinterpret_cast<float *>(smem + L::kOffPart);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
@@ -1471,7 +1471,7 @@ __global__ void __launch_bounds__((!SWAP && MODE == kSplitNone) ? kWideThreads :
         epi_bar_sync();
         if (*last_flag) {
           // The other slices' partial tiles arrive by bulk copies (one per
-          // slice, as many per round as the landing area holds) while this
+          // slice, as many per pass as the landing area holds) while this
           // slice's own partial goes from TMEM into shared memory in the same
           // [m][n] layout.  Then every thread sums float4 groups of the tile
           // (up to BN/4 of them, all loads independent) in slice order and
@@ -1487,7 +1487,7 @@ __global__ void __launch_bounds__((!SWAP && MODE == kSplitNone) ? kWideThreads :
           bool ok = true, dumped = false;
 #pragma unroll 1
           for (int s0 = 0; s0 < a.splits && ok;) {
-            // slices [s0, s1) of this round hold `n` landed (other) slices
+            // slices [s0, s1) of this pass hold `n` landed (other) slices
             int s1 = s0, n = 0;
             while (s1 < a.splits && (n < cap || s1 == u.split)) {
               if (s1 != u.split) ++n;
