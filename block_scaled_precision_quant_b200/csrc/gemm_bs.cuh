@@ -1540,7 +1540,7 @@ __global__ void __launch_bounds__((!SWAP && MODE == kSplitNone) ? kWideThreads :
                 }
               }
             }
-            epi_bar_sync();  // the landing area is free for the next round
+            epi_bar_sync();  // the landing area is free for the next pass
             s0 = s1;
           }
           const float *bias_s = reinterpret_cast<const float *>(smem + L::kOffBiasS);
