@@ -294,7 +294,8 @@ int bq_gemm_nvfp4_nvfp4(const void *a_fp4, const void *a_sf, const void *b_fp4, 
  * kind::mxf8f6f4 with an E5M2 A operand).  dX = bq_gemm_e5m2_mxfp8(dY_q,
  * W^T_q) with W^T quantized along the output dimension; dW =
  * bq_gemm_e5m2_mxfp8(dY^T_q, X^T_q), both transposed along the token
- * dimension.  Operand layouts, alignment and errors as the other GEMMs. */
+ * dimension.  Operand layouts, alignment, errors and stream order as the other
+ * GEMMs: B is read early, so quantize both B operands (W^T, X^T) before dY. */
 int bq_gemm_e5m2_mxfp8(const void *a_e5m2, const void *a_sf, const void *b_e4m3, const void *b_sf,
                        int64_t M, int64_t N, int64_t K, void *y_bf16, bq_stream_t stream);
 
